@@ -1,0 +1,232 @@
+"""ctypes binding of liblstm.so (C ABI declared in include/liblstm.h).
+
+Argument marshalling only: every step of the LSTM forward pass and BPTT runs
+inside the library's CUDA kernels.  torch tensors are used for device memory
+and for the current CUDA stream; nothing here computes on them.  When the
+shared library is missing, every entry point raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblstm.so")
+
+LSTM_OK = 0
+LSTM_ERR_INVALID_ARG = 1
+LSTM_ERR_UNSUPPORTED = 2
+LSTM_ERR_WORKSPACE = 3
+LSTM_ERR_CUDA = 4
+LSTM_ERR_TIMEOUT = 5
+LSTM_ERR_NOT_CORESIDENT = 6
+
+LSTM_F32 = 0
+LSTM_BF16 = 1
+
+EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd", "lstm_bwd",
+           "lstm_status", "lstm_profile_begin", "lstm_profile_end", "lstm_launch_count",
+           "lstm_strerror", "lstm_abi_version")
+
+PHASES = ("input_proj", "fwd_recur", "bwd_recur", "dW", "db", "dx", "other")
+
+
+class LstmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: liblstm status {code} ({strerror(code)})")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("B", ctypes.c_int), ("I", ctypes.c_int),
+                ("H", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load liblstm.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"liblstm.so not found at {path}: build it with "
+                           "`python -m backward_lstm_fwd_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, ip = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    dp = ctypes.POINTER(Dims)
+    lib.lstm_fwd_workspace_size.argtypes = [dp]
+    lib.lstm_fwd_workspace_size.restype = sz
+    lib.lstm_bwd_workspace_size.argtypes = [dp]
+    lib.lstm_bwd_workspace_size.restype = sz
+    lib.lstm_fwd.argtypes = [dp] + [vp] * 10 + [vp, sz, vp]
+    lib.lstm_fwd.restype = ip
+    lib.lstm_bwd.argtypes = [dp] + [vp] * 15 + [vp, sz, vp]
+    lib.lstm_bwd.restype = ip
+    lib.lstm_status.argtypes = [vp, sz, vp]
+    lib.lstm_status.restype = ip
+    lib.lstm_strerror.argtypes = [ip]
+    lib.lstm_strerror.restype = ctypes.c_char_p
+    lib.lstm_abi_version.argtypes = []
+    lib.lstm_abi_version.restype = ip
+    lib.lstm_profile_begin.argtypes = []
+    lib.lstm_profile_begin.restype = ip
+    lib.lstm_profile_end.argtypes = [ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(ctypes.c_longlong)]
+    lib.lstm_profile_end.restype = ip
+    lib.lstm_launch_count.argtypes = []
+    lib.lstm_launch_count.restype = ctypes.c_longlong
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    try:
+        return load().lstm_strerror(int(code)).decode()
+    except RuntimeError:
+        return "liblstm not loaded"
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return LSTM_F32
+    if dt == torch.bfloat16:
+        return LSTM_BF16
+    raise ValueError(f"unsupported compute dtype {dt}")
+
+
+def dims(T: int, B: int, I: int, H: int, dtype) -> Dims:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return Dims(int(T), int(B), int(I), int(H), code)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def fwd_workspace_size(d: Dims) -> int:
+    return int(load().lstm_fwd_workspace_size(ctypes.byref(d)))
+
+
+def bwd_workspace_size(d: Dims) -> int:
+    return int(load().lstm_bwd_workspace_size(ctypes.byref(d)))
+
+
+def lstm_fwd(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes=None,
+             stream=None, check: bool = True) -> int:
+    """Direct call of the C entry point lstm_fwd (device tensors or raw pointers)."""
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    rc = load().lstm_fwd(ctypes.byref(d), _p(x), _p(W), _p(b), _p(h0), _p(c0), _p(y), _p(hT),
+                         _p(cT), _p(gates), _p(cells), _p(ws), ws_bytes, _stream(stream))
+    if check and rc != LSTM_OK:
+        raise LstmError(rc, "lstm_fwd")
+    return rc
+
+
+def lstm_bwd(d: Dims, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0, ws,
+             ws_bytes=None, stream=None, check: bool = True) -> int:
+    """Direct call of the C entry point lstm_bwd (device tensors or raw pointers)."""
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    rc = load().lstm_bwd(ctypes.byref(d), _p(dy), _p(dhT), _p(dcT), _p(x), _p(W), _p(h0), _p(c0),
+                         _p(y), _p(gates), _p(cells), _p(dx), _p(dW), _p(db), _p(dh0), _p(dc0),
+                         _p(ws), ws_bytes, _stream(stream))
+    if check and rc != LSTM_OK:
+        raise LstmError(rc, "lstm_bwd")
+    return rc
+
+
+def lstm_status(ws, ws_bytes=None, stream=None) -> int:
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    return int(load().lstm_status(_p(ws), ws_bytes, _stream(stream)))
+
+
+def profile_begin() -> None:
+    load().lstm_profile_begin()
+
+
+def profile_end():
+    """Per-phase (device ms, kernel launches) since profile_begin()."""
+    n = len(PHASES)
+    ms = (ctypes.c_double * n)()
+    la = (ctypes.c_longlong * n)()
+    rc = load().lstm_profile_end(ms, la)
+    if rc != LSTM_OK:
+        raise LstmError(rc, "lstm_profile_end")
+    return {p: (ms[i], la[i]) for i, p in enumerate(PHASES)}
+
+
+def launch_count() -> int:
+    return int(load().lstm_launch_count())
+
+
+# ------------------------------------------------------------------ helpers
+def empty_workspace(nbytes: int, device) -> torch.Tensor:
+    """A byte tensor usable as workspace (torch's allocator returns 256-byte
+    aligned blocks)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class State:
+    """Outputs of one forward call (device tensors), kept for the backward."""
+
+    def __init__(self, T, B, I, H, cd, device):
+        self.dims = dims(T, B, I, H, cd)
+        self.y = torch.empty((T, B, H), dtype=cd, device=device)
+        self.hT = torch.empty((B, H), dtype=cd, device=device)
+        self.cT = torch.empty((B, H), dtype=torch.float32, device=device)
+        self.gates = torch.empty((T, B, 4 * H), dtype=cd, device=device)
+        self.cells = torch.empty((T, B, H), dtype=torch.float32, device=device)
+
+
+class Grads:
+    def __init__(self, T, B, I, H, device):
+        f = torch.float32
+        self.dx = torch.empty((T, B, I), dtype=f, device=device)
+        self.dW = torch.empty((4 * H, H + I), dtype=f, device=device)
+        self.db = torch.empty((4 * H,), dtype=f, device=device)
+        self.dh0 = torch.empty((B, H), dtype=f, device=device)
+        self.dc0 = torch.empty((B, H), dtype=f, device=device)
+
+
+def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None) -> State:
+    """Allocate outputs and run lstm_fwd.  x [T,B,I] and W [4H,H+I] share the
+    compute dtype (float32 or bfloat16); c0 is float32."""
+    T, B, I = x.shape
+    H = W.shape[0] // 4
+    st = State(T, B, I, H, x.dtype, x.device)
+    if ws is None:
+        ws = empty_workspace(fwd_workspace_size(st.dims), x.device)
+    lstm_fwd(st.dims, x, W, b, h0, c0, st.y, st.hT, st.cT, st.gates, st.cells, ws, stream=stream)
+    return st
+
+
+def backward(st: State, x, W, h0=None, c0=None, dy=None, dhT=None, dcT=None, ws=None,
+             stream=None) -> Grads:
+    """Allocate gradients and run lstm_bwd on the saved state of forward()."""
+    T, B, I = x.shape
+    H = W.shape[0] // 4
+    g = Grads(T, B, I, H, x.device)
+    if ws is None:
+        ws = empty_workspace(bwd_workspace_size(st.dims), x.device)
+    lstm_bwd(st.dims, dy, dhT, dcT, x, W, h0, c0, st.y, st.gates, st.cells, g.dx, g.dW, g.db,
+             g.dh0, g.dc0, ws, stream=stream)
+    return g

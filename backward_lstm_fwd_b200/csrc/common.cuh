@@ -1,0 +1,55 @@
+// common.cuh -- element conversions, activations and the workspace control
+// block shared by every liblstm kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+namespace lstm {
+
+// Host-side count of kernel launches issued by the library (diagnostics).
+inline std::atomic<long long> &launch_counter() {
+    static std::atomic<long long> n{0};
+    return n;
+}
+inline void note_launch(long long k = 1) { launch_counter().fetch_add(k); }
+
+// ---------------------------------------------------------------- elements
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <class T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// ------------------------------------------------------------- activations
+// Gate nonlinearities of the forward-formula table ("SingleLayerLstmGrad"):
+// sigma for the input, forget and output gates, tanh for the candidate state
+// and for the cell state feeding h_t.  expf / tanhf are CUDA's own functions.
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + expf(-a)); }
+__device__ __forceinline__ float tanhf_(float a) { return tanhf(a); }
+
+// ------------------------------------------------------- workspace control
+// The first 256 bytes of every workspace.  `status` is sticky: kernels only
+// ever set it, and lstm_status() reads and clears it.  Barrier counters are
+// zeroed at the start of every call.
+struct Ctrl {
+    unsigned int status;     // 0 or an LSTM_ERR_* code
+    unsigned int fail_site;  // which wait gave up (for diagnostics)
+    unsigned int pad[14];
+    unsigned int bar[48];    // grid-barrier counters
+};
+static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
+
+constexpr size_t kCtrlBytes = 256;
+
+__host__ __device__ __forceinline__ size_t align_up(size_t v, size_t a) {
+    return (v + a - 1) / a * a;
+}
+
+}  // namespace lstm

@@ -1,0 +1,399 @@
+// liblstm.cu -- C ABI of liblstm (declared in include/liblstm.h): argument
+// checks, workspace layout and the stream-ordered kernel sequence of the LSTM
+// forward pass and its backpropagation through time ("SingleLayerLstmGrad").
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <climits>
+#include <vector>
+
+#include "../../include/liblstm.h"
+#include "common.cuh"
+#include "simt.cuh"
+
+using namespace lstm;
+
+namespace {
+
+// ---------------------------------------------------------------- profiling
+// Optional per-phase event pairs (lstm_profile_begin / lstm_profile_end).
+namespace prof {
+bool g_on = false;
+struct Rec {
+    int phase;
+    cudaEvent_t a, b;
+    long long launches;
+};
+std::vector<Rec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// RAII scope: records an event before and after the phase's launches.
+struct Phase {
+    int phase;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr;
+    long long l0;
+    Phase(int p, cudaStream_t st) : phase(p), s(st), l0(launch_counter().load()) {
+        if (g_on && (a = take_event()) != nullptr) cudaEventRecord(a, s);
+    }
+    ~Phase() {
+        if (!g_on || !a) return;
+        cudaEvent_t b = take_event();
+        if (!b) return;
+        cudaEventRecord(b, s);
+        g_recs.push_back({phase, a, b, launch_counter().load() - l0});
+    }
+};
+}  // namespace prof
+
+// ------------------------------------------------------------ validation
+bool dims_ok(const lstm_dims *d) {
+    if (!d) return false;
+    if (d->T < 0 || d->B < 0 || d->I < 0 || d->H < 0) return false;
+    if (d->dtype != LSTM_F32 && d->dtype != LSTM_BF16) return false;
+    const long long TB = (long long)d->T * d->B;
+    const long long G4 = 4LL * d->H;
+    const long long K = (long long)d->H + d->I;
+    // every row / column index used by the kernels fits in an int
+    if (TB > INT_MAX || G4 > INT_MAX || K > INT_MAX) return false;
+    return true;
+}
+
+// Column extents beyond the 65535 x 64 columns one grid dimension covers.
+bool dims_supported(const lstm_dims *d) {
+    const long long maxcols = 65535LL * 64;
+    return 4LL * d->H <= maxcols && (long long)d->H + d->I <= maxcols;
+}
+
+size_t esize(const lstm_dims *d) { return d->dtype == LSTM_BF16 ? 2 : 4; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// A pointer argument: must be non-NULL when `needed`, and 16-byte aligned.
+bool ptr_ok(const void *p, bool needed) {
+    if (!p) return !needed;
+    return aligned16(p);
+}
+
+struct FwdLayout {
+    size_t gx, total;
+};
+FwdLayout fwd_layout(const lstm_dims *d) {
+    FwdLayout L;
+    const size_t TB = (size_t)d->T * d->B, G4 = 4 * (size_t)d->H;
+    L.gx = kCtrlBytes;
+    L.total = align_up(L.gx + TB * G4 * sizeof(float), 256);
+    return L;
+}
+
+// db partial sums: at most kDbMaxChunks row chunks of >= 256 rows each.
+constexpr long long kDbMaxChunks = 2048;
+
+struct BwdLayout {
+    size_t dG, dc, dbpart, total;
+    int db_chunks, db_rows_per_chunk;
+};
+BwdLayout bwd_layout(const lstm_dims *d) {
+    BwdLayout L;
+    const size_t TB = (size_t)d->T * d->B, G4 = 4 * (size_t)d->H;
+    const size_t BH = (size_t)d->B * d->H;
+    long long rows = 256;
+    if ((long long)TB > rows * kDbMaxChunks) rows = ((long long)TB + kDbMaxChunks - 1) / kDbMaxChunks;
+    L.db_rows_per_chunk = (int)rows;
+    L.db_chunks = (int)(((long long)TB + rows - 1) / rows);
+    L.dG = kCtrlBytes;
+    L.dc = align_up(L.dG + TB * G4 * esize(d), 256);
+    L.dbpart = align_up(L.dc + 2 * BH * sizeof(float), 256);
+    L.total = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
+    return L;
+}
+
+int ws_ok(void *ws, size_t ws_bytes, size_t need) {
+    if (!ws || ws_bytes < need || ((uintptr_t)ws & 255u) != 0) return LSTM_ERR_WORKSPACE;
+    return LSTM_OK;
+}
+
+#define LSTM_TRY(expr)                                    \
+    do {                                                  \
+        cudaError_t e_ = (expr);                          \
+        if (e_ != cudaSuccess) return LSTM_ERR_CUDA;      \
+    } while (0)
+
+cudaError_t reset_barriers(void *ws, cudaStream_t s) {
+    return cudaMemsetAsync((char *)ws + offsetof(Ctrl, bar), 0, sizeof(((Ctrl *)0)->bar), s);
+}
+
+template <class T>
+cudaError_t launch_copy_or_zero(const T *in, T *out, long long n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    simt::copy_or_zero<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(in, out, n);
+    note_launch();
+    return cudaGetLastError();
+}
+
+template <class T>
+cudaError_t launch_to_float(const T *in, float *out, long long n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    simt::to_float_copy<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(in, out, n);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ forward pass
+template <class T>
+int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
+             const float *c0, T *y, T *hT, float *cT, T *gates, float *cells, char *ws,
+             cudaStream_t s) {
+    const int T_ = d->T, B = d->B, I = d->I, H = d->H;
+    const long long BH = (long long)B * H;
+    const FwdLayout L = fwd_layout(d);
+    float *Gx = (float *)(ws + L.gx);
+    if ((long long)T_ * B > 0 && H > 0) {
+        {   // a1: Gx = X W_x^T + b over all T*B rows (input concat, x-part)
+            prof::Phase ph(LSTM_PHASE_INPUT_PROJ, s);
+            LSTM_TRY((simt::gemm<true, true>(T_ * B, 4 * H, I, simt::RowMajor<T>{x, I},
+                                              simt::WxT<T>{W, H, I},
+                                              simt::EpGx<T>{Gx, b, 4 * H}, s)));
+        }
+        // a2: the recurrence, one fused GEMM + gate/cell/hidden epilogue per step
+        prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
+        for (int t = 0; t < T_; ++t) {
+            const T *hp = t > 0 ? y + (long long)(t - 1) * BH : h0;
+            const float *cp = t > 0 ? cells + (long long)(t - 1) * BH : c0;
+            simt::EpFwdStep<T> ep{Gx + (long long)t * B * 4 * H, cp, y + (long long)t * BH,
+                                  gates + (long long)t * B * 4 * H, cells + (long long)t * BH, H};
+            LSTM_TRY((simt::gemm<true, true>(B, 4 * H, H, simt::Hprev<T>{hp, H},
+                                              simt::WhT4<T>{W, H, I}, ep, s)));
+        }
+    }
+    if (BH > 0) {
+        prof::Phase ph(LSTM_PHASE_OTHER, s);
+        if (T_ > 0) {
+            LSTM_TRY(cudaMemcpyAsync(hT, y + (long long)(T_ - 1) * BH, BH * sizeof(T),
+                                     cudaMemcpyDeviceToDevice, s));
+            LSTM_TRY(cudaMemcpyAsync(cT, cells + (long long)(T_ - 1) * BH, BH * sizeof(float),
+                                     cudaMemcpyDeviceToDevice, s));
+        } else {
+            LSTM_TRY(launch_copy_or_zero<T>(h0, hT, BH, s));
+            LSTM_TRY(launch_copy_or_zero<float>(c0, cT, BH, s));
+        }
+    }
+    return LSTM_OK;
+}
+
+// ----------------------------------------------------------- backward pass
+template <class T>
+int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, const T *x,
+             const T *W, const T *h0, const float *c0, const T *y, const T *gates,
+             const float *cells, float *dx, float *dW, float *db, float *dh0, float *dc0,
+             char *ws, cudaStream_t s) {
+    const int T_ = d->T, B = d->B, I = d->I, H = d->H;
+    const long long BH = (long long)B * H, TB = (long long)T_ * B;
+    const int G4 = 4 * H, K = H + I;
+    const BwdLayout L = bwd_layout(d);
+    T *dG = (T *)(ws + L.dG);
+    float *dcbuf[2] = {(float *)(ws + L.dc), (float *)(ws + L.dc) + BH};
+
+    if (TB == 0 || H == 0) {
+        // no step runs: the incoming gradients pass straight through
+        prof::Phase ph(LSTM_PHASE_OTHER, s);
+        LSTM_TRY(launch_to_float<T>(T_ == 0 ? dhT : nullptr, dh0, BH, s));
+        LSTM_TRY(launch_copy_or_zero<float>(T_ == 0 ? dcT : nullptr, dc0, BH, s));
+        if ((long long)G4 * K > 0) LSTM_TRY(cudaMemsetAsync(dW, 0, (size_t)G4 * K * sizeof(float), s));
+        if (G4 > 0) LSTM_TRY(cudaMemsetAsync(db, 0, (size_t)G4 * sizeof(float), s));
+        if (TB * I > 0) LSTM_TRY(cudaMemsetAsync(dx, 0, (size_t)(TB * I) * sizeof(float), s));
+        return LSTM_OK;
+    }
+
+    // a3: reverse-time recursion, steps 1-3 and 5 fused with delta h = W_h^T dG_{t+1}
+    {
+    prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
+    for (int t = T_ - 1; t >= 0; --t) {
+        const bool last = (t == T_ - 1);
+        simt::EpBwdStep<T> ep;
+        ep.dy = dy ? dy + (long long)t * BH : nullptr;
+        ep.dh_in = last ? dhT : nullptr;
+        ep.dc_in = last ? dcT : dcbuf[(t + 1) & 1];
+        ep.gates = gates + (long long)t * B * G4;
+        ep.cells = cells + (long long)t * BH;
+        ep.cprev = t > 0 ? cells + (long long)(t - 1) * BH : c0;
+        ep.dG = dG + (long long)t * B * G4;
+        ep.dc_out = (t == 0) ? dc0 : dcbuf[t & 1];
+        ep.H = H;
+        ep.use_acc = !last;
+        const T *dGn = last ? dG : dG + (long long)(t + 1) * B * G4;
+        LSTM_TRY((simt::gemm<true, false>(B, H, last ? 0 : G4, simt::RowMajor<T>{dGn, G4},
+                                           simt::RowMajor<T>{W, K}, ep, s)));
+    }
+    // dinitH = W_h^T dG_0 (delta h_prev at t = 0, step 5)
+    LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG, G4},
+                                       simt::RowMajor<T>{W, K}, simt::EpStore{dh0, H}, s)));
+    }
+    {   // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
+        prof::Phase ph(LSTM_PHASE_DW, s);
+        LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
+                                            simt::Zrows<T>{x, y, h0, B, I, H},
+                                            simt::EpStore{dW, K}, s)));
+    }
+    // a5: db = column sums of dG (step 4)
+    {
+        prof::Phase ph(LSTM_PHASE_DB, s);
+        float *part = (float *)(ws + L.dbpart);
+        dim3 g1((G4 + 255) / 256, L.db_chunks);
+        simt::colsum_partial<T><<<g1, 256, 0, s>>>(dG, (int)TB, G4, L.db_rows_per_chunk, part);
+        note_launch();
+        LSTM_TRY(cudaGetLastError());
+        simt::colsum_final<<<(G4 + 255) / 256, 256, 0, s>>>(part, L.db_chunks, G4, db);
+        note_launch();
+        LSTM_TRY(cudaGetLastError());
+    }
+    // a6: dx = dG W_x (x-part of delta z, step 5)
+    prof::Phase ph(LSTM_PHASE_DX, s);
+    if (I > 0)
+        LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
+                                           simt::RowMajor<T>{W + H, K},
+                                           simt::EpStore{dx, I}, s)));
+    return LSTM_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+int lstm_abi_version(void) { return 100; }
+
+const char *lstm_strerror(int code) {
+    switch (code) {
+        case LSTM_OK: return "ok";
+        case LSTM_ERR_INVALID_ARG: return "invalid argument (dims, dtype, NULL or misaligned pointer)";
+        case LSTM_ERR_UNSUPPORTED: return "unsupported configuration";
+        case LSTM_ERR_WORKSPACE: return "workspace NULL, too small or not 256-byte aligned";
+        case LSTM_ERR_CUDA: return "CUDA runtime error";
+        case LSTM_ERR_TIMEOUT: return "device-side wait timed out";
+        case LSTM_ERR_NOT_CORESIDENT: return "persistent grid cannot be co-resident";
+        default: return "unknown status";
+    }
+}
+
+size_t lstm_fwd_workspace_size(const lstm_dims *d) {
+    if (!dims_ok(d)) return 0;
+    return fwd_layout(d).total;
+}
+
+size_t lstm_bwd_workspace_size(const lstm_dims *d) {
+    if (!dims_ok(d)) return 0;
+    return bwd_layout(d).total;
+}
+
+int lstm_fwd(const lstm_dims *d, const void *x, const void *W, const void *b, const void *h0,
+             const float *c0, void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
+             size_t ws_bytes, void *stream) {
+    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
+    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
+    if (!ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(b, false) ||
+        !ptr_ok(h0, false) || !ptr_ok(c0, false) || !ptr_ok(y, TB * d->H > 0) ||
+        !ptr_ok(hT, BH > 0) || !ptr_ok(cT, BH > 0) || !ptr_ok(gates, TB * d->H > 0) ||
+        !ptr_ok(cells, TB * d->H > 0))
+        return LSTM_ERR_INVALID_ARG;
+    const int wsrc = ws_ok(ws, ws_bytes, fwd_layout(d).total);
+    if (wsrc != LSTM_OK) return wsrc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (d->dtype == LSTM_F32)
+        return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
+                               (const float *)h0, c0, (float *)y, (float *)hT, cT,
+                               (float *)gates, cells, (char *)ws, s);
+    return fwd_simt<__nv_bfloat16>(d, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)W,
+                                   (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)h0, c0,
+                                   (__nv_bfloat16 *)y, (__nv_bfloat16 *)hT, cT,
+                                   (__nv_bfloat16 *)gates, cells, (char *)ws, s);
+}
+
+int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *dcT,
+             const void *x, const void *W, const void *h0, const float *c0, const void *y,
+             const void *gates, const float *cells, float *dx, float *dW, float *db,
+             float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream) {
+    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
+    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
+    const long long G4 = 4LL * d->H, K = (long long)d->H + d->I;
+    if (!ptr_ok(dy, false) || !ptr_ok(dhT, false) || !ptr_ok(dcT, false) ||
+        !ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(h0, false) ||
+        !ptr_ok(c0, false) || !ptr_ok(y, TB * d->H > 0) || !ptr_ok(gates, TB * d->H > 0) ||
+        !ptr_ok(cells, TB * d->H > 0) || !ptr_ok(dx, TB * d->I > 0) ||
+        !ptr_ok(dW, G4 * K > 0) || !ptr_ok(db, G4 > 0) || !ptr_ok(dh0, BH > 0) ||
+        !ptr_ok(dc0, BH > 0))
+        return LSTM_ERR_INVALID_ARG;
+    const int wsrc = ws_ok(ws, ws_bytes, bwd_layout(d).total);
+    if (wsrc != LSTM_OK) return wsrc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (d->dtype == LSTM_F32)
+        return bwd_simt<float>(d, (const float *)dy, (const float *)dhT, dcT, (const float *)x,
+                               (const float *)W, (const float *)h0, c0, (const float *)y,
+                               (const float *)gates, cells, dx, dW, db, dh0, dc0, (char *)ws, s);
+    typedef __nv_bfloat16 bf;
+    return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
+                        (const bf *)h0, c0, (const bf *)y, (const bf *)gates, cells, dx, dW, db,
+                        dh0, dc0, (char *)ws, s);
+}
+
+int lstm_profile_begin(void) {
+    for (auto &r : prof::g_recs) {
+        prof::g_pool.push_back(r.a);
+        prof::g_pool.push_back(r.b);
+    }
+    prof::g_recs.clear();
+    prof::g_on = true;
+    return LSTM_OK;
+}
+
+int lstm_profile_end(double *ms, long long *launches) {
+    prof::g_on = false;
+    if (ms)
+        for (int i = 0; i < LSTM_NUM_PHASES; ++i) ms[i] = 0.0;
+    if (launches)
+        for (int i = 0; i < LSTM_NUM_PHASES; ++i) launches[i] = 0;
+    int rc = LSTM_OK;
+    for (auto &r : prof::g_recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess ||
+            cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = LSTM_ERR_CUDA;
+        if (ms) ms[r.phase] += t;
+        if (launches) launches[r.phase] += r.launches;
+        prof::g_pool.push_back(r.a);
+        prof::g_pool.push_back(r.b);
+    }
+    prof::g_recs.clear();
+    return rc;
+}
+
+long long lstm_launch_count(void) { return launch_counter().load(); }
+
+int lstm_status(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < kCtrlBytes || ((uintptr_t)ws & 255u) != 0) return LSTM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LSTM_ERR_CUDA;
+    unsigned int st = 0;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (st != 0 && cudaMemset(ws, 0, 2 * sizeof(unsigned int)) != cudaSuccess) return LSTM_ERR_CUDA;
+    return (int)st;
+}
+
+}  // extern "C"

@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Throughput of the LSTM forward pass + BPTT (lstm_fwd + lstm_bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = lstm_fwd + lstm_bwd over the whole workload (every row of the
+method: input projection, forward recurrence, backward recurrence, dW, db,
+dx), on synthetic seeded inputs already resident in HBM.  The default workload
+is T=256, B=128, I=1024, H=1024 in bf16 (fp32 accumulate and cell state).
+Rank 0 prints one JSON line.  Under torchrun (N > 1) every rank runs an
+independent replica of the workload ("replicas only": the path needs no
+exchange between GPUs), timed as the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (whole sequences).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from backward_lstm_fwd_b200 import synth  # noqa: E402
+
+METRIC = "LSTM fwd+bwd (T·B) timesteps/sec and % of bf16 tensor peak, 1×B200"
+UNIT = "timesteps/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def phase_work(w: synth.Workload):
+    """Algorithmic work per phase: FLOPs for the contractions (2 * M * N * K of
+    the products the method defines), bytes for the db column reduction."""
+    TB, H, I = w.rows, w.H, w.I
+    es = 2 if w.dtype == "bf16" else 4
+    return {
+        "input_proj": ("flop", 2.0 * TB * 4 * H * I),
+        "fwd_recur": ("flop", 2.0 * TB * 4 * H * H),
+        "bwd_recur": ("flop", 2.0 * TB * 4 * H * H),
+        "dW": ("flop", 2.0 * TB * 4 * H * (H + I)),
+        "db": ("byte", float(TB * 4 * H * es + 4 * H * 4)),
+        "dx": ("flop", 2.0 * TB * 4 * H * I),
+        "other": ("byte", 0.0),
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(w: synth.Workload, inputs, max_seconds=30.0):
+    """The fp64 oracle, as it stands, on a bounded sample of whole sequences."""
+    import oracle
+    threads = oracle.max_threads()
+    nseq = max(1, min(w.B, threads))
+    # calibrate on one sequence, then size the sample to stay well inside budget
+    t0 = time.perf_counter()
+    oracle.lstm_fwd_bwd(**synth.as_float64(synth.select_sequences(inputs, [0])))
+    one = time.perf_counter() - t0
+    waves = max(1, int(max_seconds / max(one, 1e-3)))
+    nseq = max(1, min(w.B, nseq * waves, threads * waves))
+    sub = synth.as_float64(synth.select_sequences(inputs, list(range(nseq))))
+    t0 = time.perf_counter()
+    oracle.lstm_fwd_bwd(**sub)
+    dt = time.perf_counter() - t0
+    return {"value": w.T * nseq / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{nseq} of {w.B} sequences x T={w.T} steps, fwd+bwd, fp64, "
+                      f"{dt:.1f} s wall on {threads} OpenMP threads"}
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    inputs = synth.make_inputs(w)
+    threads = oracle.max_threads()
+    nseq = max(1, min(w.B, threads))
+    sub = synth.as_float64(synth.select_sequences(inputs, list(range(nseq))))
+    for _ in range(args.warmup):
+        oracle.lstm_fwd_bwd(**sub)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.lstm_fwd_bwd(**sub)
+    dt = time.perf_counter() - t0
+    value = w.T * nseq * args.steps / dt
+    sample = (f"{nseq} of {w.B} sequences x T={w.T} steps per step, fwd+bwd, fp64, "
+              f"{threads} OpenMP threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "B": w.B, "I": w.I, "H": w.H,
+                   "inputs": w.dtype, "sample_sequences": nseq},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w, rank, world, local_rank):
+    from backward_lstm_fwd_b200 import binding as L
+    from backward_lstm_fwd_b200 import build as lbuild
+    lbuild.build()
+    L.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    inputs = synth.make_inputs(w)
+    d = {k: v.to(dev) for k, v in inputs.items()}
+    cd = synth.torch_dtype(w.dtype)
+    T, B, I, H = w.T, w.B, w.I, w.H
+    st = L.State(T, B, I, H, cd, dev)
+    gr = L.Grads(T, B, I, H, dev)
+    dims = st.dims
+    ws_f = L.empty_workspace(L.fwd_workspace_size(dims), dev)
+    ws_b = L.empty_workspace(L.bwd_workspace_size(dims), dev)
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+
+    def step(src):
+        L.lstm_fwd(dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT, st.cT,
+                   st.gates, st.cells, ws_f, stream=stream)
+        L.lstm_bwd(dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
+                   src["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0,
+                   ws_b, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(d)
+    torch.cuda.synchronize(dev)
+    for ws in (ws_f, ws_b):
+        if L.lstm_status(ws, stream=stream) != L.LSTM_OK:
+            raise RuntimeError("device-side status set during warm-up")
+
+    # ---------------------------------------------------------- timed region
+    clocks = ClockSampler(dev) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = L.launch_count()
+    L.profile_begin()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step(d)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    phases = L.profile_end()
+    launches = L.launch_count() - n0
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    for ws in (ws_f, ws_b):
+        if L.lstm_status(ws, stream=stream) != L.LSTM_OK:
+            raise RuntimeError("device-side status set during the timed region")
+
+    # -------------------------------------------------- end to end (host I/O)
+    pin_in = {k: v.pin_memory() for k, v in inputs.items()}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in inputs.items()}
+    outs = (gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0)
+    pin_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    def e2e_step():
+        for k in pin_in:
+            dev_in[k].copy_(pin_in[k], non_blocking=True)
+        step(dev_in)
+        for o, p in zip(outs, pin_out):
+            p.copy_(o, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1))
+
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    work = phase_work(w)
+    dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
+    dom_ms, dom_launches = phases[dom]
+    kind, amount = work[dom]
+    amount *= args.steps  # work of the timed region
+    if kind == "flop":
+        achieved = amount / (dom_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None}
+    else:
+        achieved = amount / (dom_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None}
+    roof.update({"kernel": dom, "launches_per_step": dom_launches / args.steps,
+                 "ms_per_step": dom_ms / args.steps,
+                 "peak_source": f"{peak_src} ({'sustained bf16' if kind == 'flop' else 'HBM copy'})"})
+    step_s = ms / args.steps * 1e-3
+    value = world * w.rows / step_s
+    tflops = w.flops / step_s / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded, distributions of the workload definition)",
+        "config": {"workload": w.name, "T": T, "B": B, "I": I, "H": H,
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+                   "l2": "working set > 126 MB L2 per step (no flush needed)"},
+        "tflops": tflops,
+        "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
+        "roofline": roof,
+        "phases_ms_per_step": {p: v[0] / args.steps for p, v in phases.items()},
+        "gpu_launches": launches,
+        "e2e": {"value": world * w.rows * args.steps / (ms_e2e * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inputs)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * liblstm.h -- C ABI of liblstm: single-layer, unidirectional LSTM forward pass
+ * and backpropagation through time on one NVIDIA B200 (sm_100a).
+ *
+ * The operation is the one defined on the "SingleLayerLstmGrad" operator page
+ * (CANN ops-nn):
+ *   forward-formula table      z_t = [h_{t-1}; x_t]
+ *                              i,f,o = sigmoid(W_* z_t + b_*), g = tanh(W_g z_t + b_g)
+ *                              c_t = f (.) c_{t-1} + i (.) g,  h_t = o (.) tanh(c_t)
+ *   backward algorithm         steps 1-6 (time step t -> t-1), which return the
+ *                              gradients of x, W, b, initH and initC.
+ *
+ * Conventions (all entry points):
+ *   - W is the packed weight [4H][H+I], row-major.  Rows are grouped by gate in
+ *     the order [i | f | g | o] (gate_order "ifjo", j = g); columns are [h | x],
+ *     i.e. W = [W_h | W_x] applied to z_t = [h_{t-1}; x_t].
+ *   - One bias b[4H] (same gate grouping); the page's db shape [4, H] is the
+ *     same memory.
+ *   - Sequences are time-major and row-major: x[T][B][I], y[T][B][H], ...
+ *     Row r = t*B + n of a [T*B][.] view is time step t of sequence n.
+ *   - "compute type" (lstm_dims.dtype) is the element type of x, W, b, h0, y,
+ *     hT, gates, dy and dhT: LSTM_F32 (float) or LSTM_BF16 (bfloat16).  The cell
+ *     state (c0, cT, cells, dcT) and every gradient output (dx, dW, db, dh0,
+ *     dc0) are float.  Products accumulate in float.
+ *   - Every pointer is a DEVICE pointer into memory the caller allocated and
+ *     owns; it must be 16-byte aligned.  The library allocates no device memory
+ *     and keeps no device state between calls; all scratch lives in the
+ *     caller's workspace.  (Its only process state is the optional profiling
+ *     record and a launch counter, see lstm_profile_begin.)
+ *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream).  Argument errors are returned synchronously before anything is
+ *     enqueued.  Device-side waits that give up record LSTM_ERR_TIMEOUT in the
+ *     workspace's status word, which lstm_status() reports.
+ *   - Two calls that share a workspace must not run concurrently.
+ */
+#ifndef LIBLSTM_H
+#define LIBLSTM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define LSTM_OK 0
+#define LSTM_ERR_INVALID_ARG 1    /* bad dims, dtype, NULL or misaligned pointer */
+#define LSTM_ERR_UNSUPPORTED 2    /* valid arguments this build cannot run */
+#define LSTM_ERR_WORKSPACE 3      /* workspace NULL, too small or misaligned */
+#define LSTM_ERR_CUDA 4           /* a CUDA runtime call or launch failed */
+#define LSTM_ERR_TIMEOUT 5        /* a device-side wait gave up (see lstm_status) */
+#define LSTM_ERR_NOT_CORESIDENT 6 /* a persistent grid cannot be fully resident */
+
+/* Compute types. */
+#define LSTM_F32 0
+#define LSTM_BF16 1
+
+/* Problem sizes: T time steps, B sequences, I input features, H hidden units
+ * (parameter table: x [T, batch, input_size], w [4*hidden, input+hidden]).
+ * All must be >= 0; T, B or I may be 0 (empty problems are valid). */
+typedef struct lstm_dims {
+    int T;
+    int B;
+    int I;
+    int H;
+    int dtype; /* LSTM_F32 or LSTM_BF16 */
+} lstm_dims;
+
+/* Workspace bytes lstm_fwd / lstm_bwd need for these dims (0 on invalid dims).
+ * The workspace must be 256-byte aligned. */
+size_t lstm_fwd_workspace_size(const lstm_dims *d);
+size_t lstm_bwd_workspace_size(const lstm_dims *d);
+
+/*
+ * lstm_fwd -- forward pass ("SingleLayerLstmGrad", forward-formula table).
+ *
+ *   x     [T][B][I]   compute type  input sequence
+ *   W     [4H][H+I]   compute type  packed weights [W_h | W_x], gate rows i,f,g,o
+ *   b     [4H]        compute type  bias, or NULL for zero
+ *   h0    [B][H]      compute type  initH (h_{-1}), or NULL for zero
+ *   c0    [B][H]      float         initC (c_{-1}), or NULL for zero
+ * outputs (overwritten):
+ *   y     [T][B][H]   compute type  h_t for every step
+ *   hT    [B][H]      compute type  h_{T-1} (h0 when T == 0)
+ *   cT    [B][H]      float         c_{T-1} (c0 when T == 0)
+ *   gates [T][B][4H]  compute type  post-activation i,f,g,o of every step, kept
+ *                                    for lstm_bwd (the page's i, j, f, o inputs)
+ *   cells [T][B][H]   float         c_t of every step, kept for lstm_bwd
+ *   ws / ws_bytes                   scratch, >= lstm_fwd_workspace_size(d)
+ *
+ * y, gates and cells must stay unchanged until the matching lstm_bwd has run.
+ * Returns LSTM_OK or an LSTM_ERR_* code.
+ */
+int lstm_fwd(const lstm_dims *d, const void *x, const void *W, const void *b,
+             const void *h0, const float *c0, void *y, void *hT, float *cT,
+             void *gates, float *cells, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lstm_bwd -- backpropagation through time ("SingleLayerLstmGrad", backward
+ * algorithm steps 1-6 and gradient derivation).  It returns the gradients of
+ * the loss L whose partial derivatives the page's dy, dh and dc inputs give:
+ *   L = sum_t <dy_t, h_t> + <dhT, h_{T-1}> + <dcT, c_{T-1}>.
+ *
+ *   dy    [T][B][H]   compute type  dL/dh_t of every step, or NULL for zero
+ *   dhT   [B][H]      compute type  gradient at h_{T-1} (page input dh), or NULL
+ *   dcT   [B][H]      float         gradient at c_{T-1} (page input dc), or NULL
+ *   x, W, h0, c0                    the forward's inputs (h0, c0 may be NULL)
+ *   y, gates, cells                 the forward's saved outputs
+ * outputs (overwritten, never accumulated):
+ *   dx    [T][B][I]   float         dL/dx
+ *   dW    [4H][H+I]   float         dL/dW, same layout as W
+ *   db    [4H]        float         dL/db (the page's db [4, H])
+ *   dh0   [B][H]      float         dL/dinitH (the page's dh_prev at t = 0)
+ *   dc0   [B][H]      float         dL/dinitC (the page's dc_prev at t = 0)
+ *   ws / ws_bytes                   scratch, >= lstm_bwd_workspace_size(d)
+ *
+ * Returns LSTM_OK or an LSTM_ERR_* code.
+ */
+int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *dcT,
+             const void *x, const void *W, const void *h0, const float *c0,
+             const void *y, const void *gates, const float *cells, float *dx,
+             float *dW, float *db, float *dh0, float *dc0, void *ws, size_t ws_bytes,
+             void *stream);
+
+/*
+ * lstm_status -- synchronise `stream`, then read and clear the device status
+ * word kept in the first bytes of a workspace used by lstm_fwd / lstm_bwd.
+ * Returns LSTM_OK, LSTM_ERR_TIMEOUT (a device-side wait gave up; the results of
+ * that call are invalid), LSTM_ERR_CUDA, or LSTM_ERR_INVALID_ARG.
+ */
+int lstm_status(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Per-phase device timing (diagnostics, not thread-safe).  Between
+ * lstm_profile_begin() and lstm_profile_end(), every lstm_fwd / lstm_bwd call
+ * records a CUDA event pair around each phase of the path on its stream and
+ * counts the kernels it launches.  lstm_profile_end() waits for those events
+ * and writes, per phase, the summed device milliseconds and kernel launches
+ * (arrays of LSTM_NUM_PHASES entries; either may be NULL).  Phases:
+ */
+#define LSTM_PHASE_INPUT_PROJ 0 /* Gx = X W_x^T + b over all T*B rows          */
+#define LSTM_PHASE_FWD_RECUR 1  /* the forward recurrence over t = 0..T-1      */
+#define LSTM_PHASE_BWD_RECUR 2  /* the backward recurrence over t = T-1..0     */
+#define LSTM_PHASE_DW 3         /* dW = dG^T [h_prev | x]                       */
+#define LSTM_PHASE_DB 4         /* db = column sums of dG                       */
+#define LSTM_PHASE_DX 5         /* dx = dG W_x                                  */
+#define LSTM_PHASE_OTHER 6      /* copies, pass-through and set-up launches     */
+#define LSTM_NUM_PHASES 7
+int lstm_profile_begin(void);
+int lstm_profile_end(double *ms, long long *launches);
+
+/* Kernel launches issued by this process's liblstm calls so far. */
+long long lstm_launch_count(void);
+
+/* Static description of a status code. */
+const char *lstm_strerror(int code);
+
+/* ABI version: 100 * major + minor. */
+int lstm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBLSTM_H */

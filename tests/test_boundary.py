@@ -1,0 +1,155 @@
+"""The C ABI boundary, checked without a GPU: the library loads, exports every
+function include/liblstm.h declares, sizes its workspaces, and rejects bad
+arguments with a status code before it enqueues anything.  (Every rejected call
+below returns before its first CUDA runtime call, so none needs a device.)"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from backward_lstm_fwd_b200 import build as lbuild
+from backward_lstm_fwd_b200 import binding as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "liblstm.h")
+
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lbuild.build()
+    return L.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lstm_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) >= set(L.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in liblstm.h but not exported"
+    assert lib.lstm_abi_version() == 100
+
+
+def test_strerror(lib):
+    for code in range(7):
+        assert L.strerror(code)
+    assert L.strerror(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    d = L.dims(256, 128, 1024, 1024, L.LSTM_BF16)
+    fw, bw = L.fwd_workspace_size(d), L.bwd_workspace_size(d)
+    TB, G4 = 256 * 128, 4 * 1024
+    assert fw >= 256 + TB * G4 * 4 and fw % 256 == 0
+    assert bw >= 256 + TB * G4 * 2 and bw % 256 == 0
+    assert L.fwd_workspace_size(L.dims(-1, 2, 3, 4, 0)) == 0
+    assert L.bwd_workspace_size(L.dims(1, 2, 3, 4, 7)) == 0
+    assert L.fwd_workspace_size(L.dims(0, 0, 0, 0, 0)) >= 256
+
+
+def fwd_args(d, **over):
+    a = dict(x=FAKE, W=FAKE, b=None, h0=None, c0=None, y=FAKE, hT=FAKE, cT=FAKE, gates=FAKE,
+             cells=FAKE, ws=FAKE, ws_bytes=L.fwd_workspace_size(d))
+    a.update(over)
+    return a
+
+
+def call_fwd(d, **over):
+    a = fwd_args(d, **over)
+    return L.lstm_fwd(d, a["x"], a["W"], a["b"], a["h0"], a["c0"], a["y"], a["hT"], a["cT"],
+                      a["gates"], a["cells"], a["ws"], ws_bytes=a["ws_bytes"], stream=0,
+                      check=False)
+
+
+def call_bwd(d, **over):
+    a = dict(dy=None, dhT=None, dcT=None, x=FAKE, W=FAKE, h0=None, c0=None, y=FAKE, gates=FAKE,
+             cells=FAKE, dx=FAKE, dW=FAKE, db=FAKE, dh0=FAKE, dc0=FAKE, ws=FAKE,
+             ws_bytes=L.bwd_workspace_size(d))
+    a.update(over)
+    return L.lstm_bwd(d, a["dy"], a["dhT"], a["dcT"], a["x"], a["W"], a["h0"], a["c0"], a["y"],
+                      a["gates"], a["cells"], a["dx"], a["dW"], a["db"], a["dh0"], a["dc0"],
+                      a["ws"], ws_bytes=a["ws_bytes"], stream=0, check=False)
+
+
+D = L.dims(4, 3, 5, 8, L.LSTM_F32)
+
+
+@pytest.mark.parametrize("bad", [
+    L.dims(-1, 3, 5, 8, 0), L.dims(4, -3, 5, 8, 0), L.dims(4, 3, -5, 8, 0),
+    L.dims(4, 3, 5, -8, 0), L.dims(4, 3, 5, 8, 2), L.dims(1 << 20, 1 << 12, 5, 8, 0),
+    L.dims(1, 1, 5, 1 << 29, 0),
+])
+def test_bad_dims(lib, bad):
+    assert call_fwd(bad, ws_bytes=1 << 30) == L.LSTM_ERR_INVALID_ARG
+    assert call_bwd(bad, ws_bytes=1 << 30) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_unsupported_extent(lib):
+    d = L.dims(1, 1, 5, 1 << 21, 0)
+    assert call_fwd(d, ws_bytes=1 << 40) == L.LSTM_ERR_UNSUPPORTED
+    assert call_bwd(d, ws_bytes=1 << 40) == L.LSTM_ERR_UNSUPPORTED
+
+
+def test_null_dims_pointer(lib):
+    rc = lib.lstm_fwd(None, *([None] * 10), None, 0, None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["x", "W", "y", "hT", "cT", "gates", "cells"])
+def test_fwd_required_pointer_null(lib, name):
+    assert call_fwd(D, **{name: None}) == L.LSTM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["x", "W", "b", "h0", "c0", "y", "hT", "cT", "gates", "cells"])
+def test_fwd_misaligned_pointer(lib, name):
+    assert call_fwd(D, **{name: FAKE + 4}) == L.LSTM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["x", "W", "y", "gates", "cells", "dx", "dW", "db", "dh0", "dc0"])
+def test_bwd_required_pointer_null(lib, name):
+    assert call_bwd(D, **{name: None}) == L.LSTM_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["dy", "dhT", "dcT", "x", "W", "h0", "c0", "y", "gates",
+                                  "cells", "dx", "dW", "db", "dh0", "dc0"])
+def test_bwd_misaligned_pointer(lib, name):
+    assert call_bwd(D, **{name: FAKE + 8}) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_workspace_errors(lib):
+    need = L.fwd_workspace_size(D)
+    assert call_fwd(D, ws=None) == L.LSTM_ERR_WORKSPACE
+    assert call_fwd(D, ws_bytes=need - 1) == L.LSTM_ERR_WORKSPACE
+    assert call_fwd(D, ws=FAKE + 16) == L.LSTM_ERR_WORKSPACE
+    need = L.bwd_workspace_size(D)
+    assert call_bwd(D, ws=None) == L.LSTM_ERR_WORKSPACE
+    assert call_bwd(D, ws_bytes=need - 1) == L.LSTM_ERR_WORKSPACE
+    assert call_bwd(D, ws=FAKE + 128) == L.LSTM_ERR_WORKSPACE
+
+
+def test_empty_problem_needs_no_data_pointers(lib):
+    # With T*B == 0 only the workspace is touched; the outputs hT/cT are
+    # still required when B*H > 0.
+    d = L.dims(0, 0, 5, 8, L.LSTM_F32)
+    assert call_fwd(d, x=None, y=None, gates=None, cells=None, hT=None, cT=None,
+                    ws=None) == L.LSTM_ERR_WORKSPACE
+    d = L.dims(0, 3, 5, 8, L.LSTM_F32)
+    assert call_fwd(d, x=None, y=None, gates=None, cells=None, hT=None) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_status_argument_checks(lib):
+    assert lib.lstm_status(None, 256, None) == L.LSTM_ERR_INVALID_ARG
+    assert lib.lstm_status(FAKE, 16, None) == L.LSTM_ERR_INVALID_ARG
+    assert lib.lstm_status(FAKE + 16, 4096, None) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError):
+        L.load(str(tmp_path / "nope.so"))

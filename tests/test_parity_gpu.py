@@ -1,0 +1,115 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Full-size runs of the five workloads (the launch configuration bench.py times),
+odd shapes that leave ragged tiles, and the degenerate cases (empty sequence or
+batch, no input features, absent optional inputs).  Tolerance per output
+tensor: max|gpu - ref| / max|ref| <= 1e-4 (fp32) or 2e-2 (bf16)."""
+import numpy as np
+import pytest
+import torch
+
+from backward_lstm_fwd_b200 import synth
+from tests.parity_util import (OUTS, TOL, assert_within, compare, mask_upstream, rel_err,
+                               run_gpu, run_oracle)
+
+pytestmark = pytest.mark.gpu
+
+# Workloads small enough for the full oracle; the other two are checked on
+# sampled sequences (all per-sequence outputs) plus a masked-gradient run that
+# makes dW and db checkable on the same sample.
+FULL = ["lstm_T8_B2_I16_H32_fp32", "lstm_T64_B32_I256_H256_fp32", "lstm_T128_B64_I512_H512_bf16"]
+SAMPLED = {"lstm_T256_B128_I1024_H1024_bf16": [0, 37, 101, 127],
+           "lstm_T1024_B16_I256_H1024_bf16": [0, 11]}
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_workload_full(name, cuda_device):
+    w = synth.WORKLOADS[name]
+    inp = synth.make_inputs(w)
+    gpu = run_gpu(inp, cuda_device)
+    ref = run_oracle(inp)
+    errs = compare(gpu, ref, w.dtype, OUTS + ("gates", "cells"))
+    assert_within(errs, w.dtype, name)
+
+
+@pytest.mark.parametrize("name", sorted(SAMPLED))
+def test_workload_sampled(name, cuda_device):
+    w = synth.WORKLOADS[name]
+    idx = SAMPLED[name]
+    inp = synth.make_inputs(w)
+    gpu = run_gpu(inp, cuda_device)
+    ref = run_oracle(synth.select_sequences(inp, idx))
+    errs = compare(gpu, ref, w.dtype, ("y", "hT", "cT", "dx", "dh0", "dc0"), idx=idx)
+    assert_within(errs, w.dtype, name + " per-sequence")
+    # dW, db: only the sampled sequences carry upstream gradient
+    masked = mask_upstream(inp, idx)
+    gpu_m = run_gpu(masked, cuda_device)
+    ref_m = run_oracle(synth.select_sequences(masked, idx))
+    errs = compare(gpu_m, ref_m, w.dtype, ("dW", "db"))
+    assert_within(errs, w.dtype, name + " dW/db")
+
+
+ODD = [
+    (5, 3, 37, 45, "fp32"), (1, 1, 1, 1, "fp32"), (3, 67, 100, 72, "fp32"),
+    (2, 130, 64, 128, "fp32"), (7, 5, 16, 33, "fp32"),
+    (5, 3, 37, 45, "bf16"), (1, 1, 1, 1, "bf16"), (3, 67, 100, 72, "bf16"),
+    (4, 130, 128, 128, "bf16"), (9, 16, 64, 64, "bf16"), (3, 200, 192, 256, "bf16"),
+]
+
+
+@pytest.mark.parametrize("T,B,I,H,dt", ODD)
+def test_odd_shapes(T, B, I, H, dt, cuda_device):
+    w = synth.custom(T, B, I, H, dt, seed=T * 1000 + B + I + H)
+    inp = synth.make_inputs(w)
+    gpu = run_gpu(inp, cuda_device)
+    ref = run_oracle(inp)
+    assert_within(compare(gpu, ref, dt), dt, w.name)
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_optional_inputs_absent(dt, cuda_device):
+    w = synth.custom(6, 4, 24, 40, dt, seed=5)
+    inp = synth.make_inputs(w)
+    drop = ("b", "h0", "c0", "dhT", "dcT")
+    gpu = run_gpu(inp, cuda_device, drop=drop)
+    ref = run_oracle(inp, drop=drop)
+    assert_within(compare(gpu, ref, dt), dt, "optional inputs NULL")
+    drop = ("dy",)
+    gpu = run_gpu(inp, cuda_device, drop=drop)
+    ref = run_oracle(inp, drop=drop)
+    assert_within(compare(gpu, ref, dt), dt, "dy NULL")
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_empty_sequence(dt, cuda_device):
+    w = synth.custom(0, 3, 8, 16, dt, seed=2)
+    inp = synth.make_inputs(w)
+    gpu = run_gpu(inp, cuda_device)
+    np.testing.assert_array_equal(gpu["hT"], inp["h0"].double().numpy())
+    np.testing.assert_array_equal(gpu["cT"], inp["c0"].double().numpy())
+    np.testing.assert_array_equal(gpu["dh0"], inp["dhT"].double().numpy())
+    np.testing.assert_array_equal(gpu["dc0"], inp["dcT"].double().numpy())
+    assert not gpu["dW"].any() and not gpu["db"].any()
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_empty_batch_and_no_inputs(dt, cuda_device):
+    gpu = run_gpu(synth.make_inputs(synth.custom(4, 0, 8, 16, dt)), cuda_device)
+    assert gpu["y"].shape == (4, 0, 16)
+    assert not gpu["dW"].any() and not gpu["db"].any()
+    w = synth.custom(4, 3, 0, 16, dt, seed=9)
+    inp = synth.make_inputs(w)
+    assert_within(compare(run_gpu(inp, cuda_device), run_oracle(inp), dt), dt, "I = 0")
+
+
+def test_side_stream_and_repeat(cuda_device):
+    """Calls are ordered on the stream they are given, and a second call with
+    the same workspace gives the same bits."""
+    w = synth.custom(12, 8, 64, 64, "bf16", seed=3)
+    inp = synth.make_inputs(w)
+    s = torch.cuda.Stream()
+    a = run_gpu(inp, cuda_device, stream=s)
+    b = run_gpu(inp, cuda_device, stream=s)
+    for k in OUTS:
+        np.testing.assert_array_equal(a[k], b[k])
+    assert_within(compare(a, run_oracle(inp), "bf16"), "bf16", "side stream")
