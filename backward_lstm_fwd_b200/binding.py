@@ -79,6 +79,9 @@ def load(path: str = LIB_PATH):
     lib.lstm_profile_end.restype = ip
     lib.lstm_launch_count.argtypes = []
     lib.lstm_launch_count.restype = ctypes.c_longlong
+    ll = ctypes.c_longlong
+    lib.lstm_test_tc_gemm.argtypes = [ip, ip, ip, vp, ll, ip, vp, ll, ip, vp, vp, ll, vp, sz, vp]
+    lib.lstm_test_tc_gemm.restype = ip
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -176,6 +179,14 @@ def profile_end():
 
 def launch_count() -> int:
     return int(load().lstm_launch_count())
+
+
+def test_tc_gemm(M, N, K, A, lda, a_mn_major, Bm, ldb, b_mn_major, bias, C, ldc, ws,
+                 stream=None) -> int:
+    """Test hook (include/liblstm_testing.h): C = A B^T (+ bias) on the tcgen05 core."""
+    return int(load().lstm_test_tc_gemm(M, N, K, _p(A), lda, a_mn_major, _p(Bm), ldb, b_mn_major,
+                                         _p(bias), _p(C), ldc, _p(ws),
+                                         ws.numel() * ws.element_size(), _stream(stream)))
 
 
 # ------------------------------------------------------------------ helpers

@@ -7,11 +7,14 @@
 #include <stdint.h>
 
 #include <climits>
+#include <cstdlib>
 #include <vector>
 
 #include "../../include/liblstm.h"
+#include "../../include/liblstm_testing.h"
 #include "common.cuh"
 #include "simt.cuh"
+#include "tc_host.cuh"
 
 using namespace lstm;
 
@@ -121,6 +124,18 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     return L;
 }
 
+// The tcgen05 GEMM core serves bf16 problems whose rows are whole 16-byte
+// groups (TMA strides and the W_x base offset are then 16-byte aligned).
+bool tc_gemm_ok(const lstm_dims *d) {
+    static int force_simt = -1;
+    if (force_simt < 0) {
+        const char *e = getenv("LSTM_FORCE_SIMT");
+        force_simt = (e && e[0] == '1') ? 1 : 0;
+    }
+    return !force_simt && d->dtype == LSTM_BF16 && d->H >= 8 && d->I >= 8 && d->H % 8 == 0 &&
+           d->I % 8 == 0 && tcg::encode_fn() != nullptr;
+}
+
 int ws_ok(void *ws, size_t ws_bytes, size_t need) {
     if (!ws || ws_bytes < need || ((uintptr_t)ws & 255u) != 0) return LSTM_ERR_WORKSPACE;
     return LSTM_OK;
@@ -152,6 +167,53 @@ cudaError_t launch_to_float(const T *in, float *out, long long n, cudaStream_t s
     return cudaGetLastError();
 }
 
+// ------------------------------------------- tensor-core GEMM problems
+typedef __nv_bfloat16 bf16;
+
+// a1 on tcgen05: Gx[TB][4H] = X[TB][I] W_x^T + b, both operands K-major.
+cudaError_t tc_input_projection(const lstm_dims *d, const bf16 *x, const bf16 *W, const bf16 *b,
+                                float *Gx, Ctrl *ctrl, cudaStream_t s) {
+    const long long TB = (long long)d->T * d->B, H = d->H, I = d->I;
+    tcg::Builder bld(ctrl);
+    const int mx = bld.add_map({x, TB, I, I}, 0, tcg::BM);
+    const int mw = bld.add_map({W + H, 4 * H, I, H + I}, 0, tcg::BN);
+    tcg::Problem &q = bld.add_problem((int)TB, (int)(4 * H), 0, 0, Gx, 4 * H, 0, b);
+    tcg::Builder::add_seg(q, mx, 0, mw, 0, I);
+    if (!bld.ok) return cudaErrorInvalidValue;
+    return tcg::launch(bld, s);
+}
+
+// a4 + a6 on tcgen05 in one persistent launch:
+//   dW[:, 0:H]  = dG[B:]^T y[:-B] + dG[:B]^T h0   (h_prev = [h0; y[0:T-1]])
+//   dW[:, H:]   = dG^T X
+//   dx          = dG W_x
+// dG^T and the z-rows are MN-major operands read straight from their
+// row-major storage; the time shift of h_prev is a TMA row offset.
+cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf16 *W,
+                     const bf16 *h0, const bf16 *y, float *dW, float *dx, Ctrl *ctrl,
+                     cudaStream_t s) {
+    const long long T = d->T, B = d->B, TB = T * B, H = d->H, I = d->I, G4 = 4 * H;
+    tcg::Builder bld(ctrl);
+    const int m_dg_mn = bld.add_map({dG, TB, G4, G4}, 1, 0);
+    const int m_x_mn = bld.add_map({x, TB, I, I}, 1, 0);
+    const int m_dg_k = bld.add_map({dG, TB, G4, G4}, 0, tcg::BM);
+    const int m_wx_mn = bld.add_map({W + H, G4, I, H + I}, 1, 0);
+    const int m_y_mn = (T > 1) ? bld.add_map({y, (T - 1) * B, H, H}, 1, 0) : -1;
+    const int m_h0_mn = h0 ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
+    // dW, h-part (zero when T == 1 and h0 is absent: no K segment)
+    tcg::Problem &p0 = bld.add_problem((int)G4, (int)H, 1, 1, dW, H + I, 0, nullptr);
+    if (m_y_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, (int)B, m_y_mn, 0, (T - 1) * B);
+    if (m_h0_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, 0, m_h0_mn, 0, B);
+    // dW, x-part
+    tcg::Problem &p1 = bld.add_problem((int)G4, (int)I, 1, 1, dW, H + I, (int)H, nullptr);
+    tcg::Builder::add_seg(p1, m_dg_mn, 0, m_x_mn, 0, TB);
+    // dx
+    tcg::Problem &p2 = bld.add_problem((int)TB, (int)I, 0, 1, dx, I, 0, nullptr);
+    tcg::Builder::add_seg(p2, m_dg_k, 0, m_wx_mn, 0, G4);
+    if (!bld.ok) return cudaErrorInvalidValue;
+    return tcg::launch(bld, s);
+}
+
 // ------------------------------------------------------------ forward pass
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
@@ -164,9 +226,15 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
     if ((long long)T_ * B > 0 && H > 0) {
         {   // a1: Gx = X W_x^T + b over all T*B rows (input concat, x-part)
             prof::Phase ph(LSTM_PHASE_INPUT_PROJ, s);
-            LSTM_TRY((simt::gemm<true, true>(T_ * B, 4 * H, I, simt::RowMajor<T>{x, I},
-                                              simt::WxT<T>{W, H, I},
-                                              simt::EpGx<T>{Gx, b, 4 * H}, s)));
+            if (tc_gemm_ok(d)) {
+                LSTM_TRY(tc_input_projection(d, (const __nv_bfloat16 *)x,
+                                             (const __nv_bfloat16 *)W,
+                                             (const __nv_bfloat16 *)b, Gx, (Ctrl *)ws, s));
+            } else {
+                LSTM_TRY((simt::gemm<true, true>(T_ * B, 4 * H, I, simt::RowMajor<T>{x, I},
+                                                  simt::WxT<T>{W, H, I},
+                                                  simt::EpGx<T>{Gx, b, 4 * H}, s)));
+            }
         }
         // a2: the recurrence, one fused GEMM + gate/cell/hidden epilogue per step
         prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
@@ -242,7 +310,14 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG, G4},
                                        simt::RowMajor<T>{W, K}, simt::EpStore{dh0, H}, s)));
     }
-    {   // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
+    const bool tc = tc_gemm_ok(d);
+    if (tc) {
+        // a4 + a6 together on the tensor cores (one launch, timed as dW)
+        prof::Phase ph(LSTM_PHASE_DW, s);
+        LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
+                          (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s));
+    } else {
+        // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
         prof::Phase ph(LSTM_PHASE_DW, s);
         LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
                                             simt::Zrows<T>{x, y, h0, B, I, H},
@@ -262,7 +337,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     }
     // a6: dx = dG W_x (x-part of delta z, step 5)
     prof::Phase ph(LSTM_PHASE_DX, s);
-    if (I > 0)
+    if (I > 0 && !tc)
         LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
                                            simt::RowMajor<T>{W + H, K},
                                            simt::EpStore{dx, I}, s)));
@@ -385,6 +460,26 @@ int lstm_profile_end(double *ms, long long *launches) {
 }
 
 long long lstm_launch_count(void) { return launch_counter().load(); }
+
+int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_mn_major,
+                      const void *Bm, long long ldb, int b_mn_major, const void *bias, float *C,
+                      long long ldc, void *ws, size_t ws_bytes, void *stream) {
+    if (M < 0 || N < 0 || K < 0 || !A || !Bm || !C || !aligned16(A) || !aligned16(Bm) ||
+        !ptr_ok(bias, false) || (lda % 8) || (ldb % 8))
+        return LSTM_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < kCtrlBytes) return LSTM_ERR_WORKSPACE;
+    if (!tcg::encode_fn()) return LSTM_ERR_UNSUPPORTED;
+    tcg::Builder bld((Ctrl *)ws);
+    // A: K-major = [M][K] (lda), MN-major = [K][M] (lda); B likewise with N.
+    const int ma = a_mn_major ? bld.add_map({(const bf16 *)A, K, M, lda}, 1, 0)
+                              : bld.add_map({(const bf16 *)A, M, K, lda}, 0, tcg::BM);
+    const int mb = b_mn_major ? bld.add_map({(const bf16 *)Bm, K, N, ldb}, 1, 0)
+                              : bld.add_map({(const bf16 *)Bm, N, K, ldb}, 0, tcg::BN);
+    tcg::Problem &q = bld.add_problem(M, N, a_mn_major, b_mn_major, C, ldc, 0, (const bf16 *)bias);
+    tcg::Builder::add_seg(q, ma, 0, mb, 0, K);
+    if (!bld.ok) return LSTM_ERR_UNSUPPORTED;
+    return tcg::launch(bld, (cudaStream_t)stream) == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
 
 int lstm_status(void *ws, size_t ws_bytes, void *stream) {
     if (!ws || ws_bytes < kCtrlBytes || ((uintptr_t)ws & 255u) != 0) return LSTM_ERR_INVALID_ARG;

@@ -1,0 +1,265 @@
+// tc_gemm.cuh -- persistent tcgen05 / TMA GEMM core for bf16 operands with fp32
+// accumulation in TMEM, used for the time-parallel contractions of the path:
+//   input projection   Gx = X W_x^T + b        (A = X K-major, B = W_x K-major)
+//   dW                 dG^T [h_prev | x]        (A = dG MN-major, B = y / x MN-major)
+//   dx                 dG W_x                  (A = dG K-major, B = W_x MN-major)
+//
+// One launch walks a table of up to four problems (each with up to two K
+// segments drawn from different tensor maps), one 128 x 256 output tile per
+// step of a static persistent schedule.  Warp roles:
+//   warp 0      one thread issues TMA loads into a 4-stage shared-memory ring;
+//   warp 1      allocates TMEM and one thread issues tcgen05.mma (M=128,
+//               N=256, K=16 per instruction) into one of two accumulators;
+//   warps 2-5   epilogue: TMEM -> registers -> (+ bias) -> fp32 global stores,
+//               overlapping the next tile's MMAs through the second accumulator.
+#pragma once
+
+#include <cuda.h>
+
+#include "tc_ptx.cuh"
+
+namespace lstm {
+namespace tcg {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_BYTES = BN * BK * 2;          // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;             // two fp32 accumulators of BN columns
+constexpr int MAX_MAPS = 6, MAX_PROB = 4;
+constexpr int MN_BOX_BYTES = 64 * BK * 2;     // one 64 (MN) x 64 (K) box: 8 KB
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct Seg {
+    int a_map, b_map;  // indices into Params::maps
+    int a_k0, b_k0;    // K coordinate of the segment's first block in each map
+    int nkb;           // number of BK-deep K blocks
+};
+
+struct Problem {
+    int M, N;                  // output extent
+    int a_mn_major, b_mn_major;
+    int a_mn0, b_mn0;          // MN coordinate of output row / column 0 in the maps
+    int nseg;
+    Seg seg[2];
+    float *out;                // out[m * ldo + out_col0 + n]
+    long long ldo;
+    int out_col0;
+    const __nv_bfloat16 *bias; // added per column n, or NULL
+    int tiles_n, tile_begin, tile_end;
+};
+
+struct Params {
+    CUtensorMap maps[MAX_MAPS];
+    Problem prob[MAX_PROB];
+    int nprob, total_tiles;
+    Ctrl *ctrl;
+};
+
+__device__ __forceinline__ int locate(const Params &p, int tile, int &mt, int &nt) {
+    int pi = 0;
+    while (pi + 1 < p.nprob && tile >= p.prob[pi].tile_end) ++pi;
+    const int local = tile - p.prob[pi].tile_begin;
+    mt = local / p.prob[pi].tiles_n;
+    nt = local % p.prob[pi].tiles_n;
+    return pi;
+}
+
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int k16) {
+    // K-major: rows of 128 B (64 bf16 of K), 8-row groups 1024 B apart; a
+    //          K=16 step moves 32 B inside the 128-byte swizzle row.
+    // MN-major: 64-element MN chunks one 8 KB box apart (leading offset),
+    //          8-row K groups 1024 B apart; a K=16 step moves two groups.
+    return mn_major ? tc::smem_desc_sw128(base + k16 * 2048, MN_BOX_BYTES, 1024)
+                    : tc::smem_desc_sw128(base + k16 * 32, 16, 1024);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * A_BYTES;
+    uint64_t *full = (uint64_t *)(sB + STAGES * B_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *tfull = empty + STAGES;
+    uint64_t *tempty = tfull + 2;
+    uint32_t *tmem_slot = (uint32_t *)(tempty + 2);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(&tfull[a], 1);
+            tc::mbar_init(&tempty[a], 4);
+        }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0)
+        for (int i = 0; i < MAX_MAPS; ++i) tc::tma_prefetch_desc(&p.maps[i]);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            uint32_t issued_parity[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                int mt, nt;
+                const Problem &P = p.prob[locate(p, tile, mt, nt)];
+                const int m0 = P.a_mn0 + mt * BM, n0 = P.b_mn0 + nt * BN;
+                for (int sg = 0; ok && sg < P.nseg; ++sg) {
+                    const Seg &S = P.seg[sg];
+                    for (int kb = 0; kb < S.nkb; ++kb) {
+                        if (!tc::mbar_wait(&empty[stage], phase ^ 1, p.ctrl, abort_flag, 0x101)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                        uint8_t *a = sA + stage * A_BYTES;
+                        uint8_t *b = sB + stage * B_BYTES;
+                        const CUtensorMap *am = &p.maps[S.a_map];
+                        const CUtensorMap *bm = &p.maps[S.b_map];
+                        const int ka = S.a_k0 + kb * BK, kbb = S.b_k0 + kb * BK;
+                        if (!P.a_mn_major) {
+                            tc::tma_load_2d(a, am, &full[stage], ka, m0);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < BM / 64; ++c)
+                                tc::tma_load_2d(a + c * MN_BOX_BYTES, am, &full[stage], m0 + 64 * c, ka);
+                        }
+                        if (!P.b_mn_major) {
+                            tc::tma_load_2d(b, bm, &full[stage], kbb, n0);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < BN / 64; ++c)
+                                tc::tma_load_2d(b + c * MN_BOX_BYTES, bm, &full[stage], n0 + 64 * c, kbb);
+                        }
+                        issued[stage] = true;
+                        issued_parity[stage] = phase;
+                        if (++stage == STAGES) stage = 0, phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: let every copy this thread issued land before exiting
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s])
+                        tc::mbar_wait(&full[s], issued_parity[s], nullptr, nullptr, 0, 200000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0, acc = 0, aphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+                int mt, nt;
+                const Problem &P = p.prob[locate(p, tile, mt, nt)];
+                if (!tc::mbar_wait(&tempty[acc], aphase ^ 1, p.ctrl, abort_flag, 0x102)) break;
+                tc::tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, P.a_mn_major, P.b_mn_major);
+                uint32_t accumulate = 0;
+                for (int sg = 0; ok && sg < P.nseg; ++sg) {
+                    const Seg &S = P.seg[sg];
+                    for (int kb = 0; kb < S.nkb; ++kb) {
+                        if (!tc::mbar_wait(&full[stage], phase, p.ctrl, abort_flag, 0x103)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                        const uint32_t a_addr = tc::smem_u32(sA + stage * A_BYTES);
+                        const uint32_t b_addr = tc::smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            tc::mma_bf16(d, operand_desc(a_addr, P.a_mn_major, k),
+                                         operand_desc(b_addr, P.b_mn_major, k), idesc, accumulate);
+                            accumulate = 1;
+                        }
+                        tc::mma_commit(&empty[stage]);
+                        if (++stage == STAGES) stage = 0, phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                if (accumulate) tc::mma_commit(&tfull[acc]);
+                else tc::mbar_arrive(&tfull[acc]);  // empty K: nothing to wait for
+                acc ^= 1;
+                if (acc == 0) aphase ^= 1;
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quarter this warp may read
+        uint32_t acc = 0, aphase = 0;
+        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+            int mt, nt;
+            const Problem &P = p.prob[locate(p, tile, mt, nt)];
+            if (!tc::mbar_wait(&tfull[acc], aphase, p.ctrl, abort_flag, 0x104)) break;
+            tc::tc_fence_after();
+            int nk = 0;
+            for (int sg = 0; sg < P.nseg; ++sg) nk += P.seg[sg].nkb;
+            const int m = mt * BM + q * 32 + lane;
+            const int nbase = nt * BN;
+            const bool vec = ((P.ldo & 3) == 0) && ((P.out_col0 & 3) == 0) &&
+                             ((((uintptr_t)P.out) & 15) == 0);
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                if (nbase + c0 >= P.N) break;  // warp-uniform
+                uint32_t r[32];
+                tc::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c0, r);
+                tc::tmem_ld_wait();
+                if (m < P.M) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = nbase + c0 + j;
+                        float x = nk ? __uint_as_float(r[j]) : 0.f;
+                        if (P.bias && n < P.N) x += __bfloat162float(P.bias[n]);
+                        v[j] = x;
+                    }
+                    float *orow = P.out + (long long)m * P.ldo + P.out_col0 + nbase + c0;
+                    if (vec && nbase + c0 + 32 <= P.N) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(orow + j) =
+                                make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (nbase + c0 + j < P.N) orow[j] = v[j];
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+            acc ^= 1;
+            if (acc == 0) aphase ^= 1;
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace tcg
+}  // namespace lstm

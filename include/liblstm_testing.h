@@ -1,0 +1,34 @@
+/*
+ * liblstm_testing.h -- test hooks of liblstm.  Not part of the LSTM API: they
+ * expose the library's internal kernels so that tests can check each one in
+ * isolation against a library routine.
+ */
+#ifndef LIBLSTM_TESTING_H
+#define LIBLSTM_TESTING_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * C[M][N] (float, row stride ldc) = A B^T (+ bias[n]) through the tcgen05 / TMA
+ * GEMM core that the input projection, dW and dx use, with bf16 operands.
+ *   a_mn_major = 0: A is [M][K] row-major with row stride lda (K-major)
+ *   a_mn_major = 1: A is [K][M] row-major with row stride lda (MN-major)
+ *   b_mn_major = 0: B is [N][K] row-major with row stride ldb (K-major)
+ *   b_mn_major = 1: B is [K][N] row-major with row stride ldb (MN-major)
+ * bias is bf16 [N] or NULL.  Device pointers, 16-byte aligned; lda and ldb
+ * multiples of 8.  ws holds at least 256 bytes (the status word).
+ * Returns an LSTM_* status code (see liblstm.h).
+ */
+int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_mn_major,
+                      const void *B, long long ldb, int b_mn_major, const void *bias, float *C,
+                      long long ldc, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBLSTM_TESTING_H */
