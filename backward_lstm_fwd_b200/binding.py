@@ -79,6 +79,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_profile_end.restype = ip
     lib.lstm_launch_count.argtypes = []
     lib.lstm_launch_count.restype = ctypes.c_longlong
+    lib.lstm_fwd_noalloc.argtypes = [dp] + [vp] * 10 + [vp]
+    lib.lstm_fwd_noalloc.restype = ip
     ll = ctypes.c_longlong
     lib.lstm_test_tc_gemm.argtypes = [ip, ip, ip, vp, ll, ip, vp, ll, ip, vp, vp, ll, vp, sz, vp]
     lib.lstm_test_tc_gemm.restype = ip
@@ -153,6 +155,21 @@ def lstm_bwd(d: Dims, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, d
                          _p(ws), ws_bytes, _stream(stream))
     if check and rc != LSTM_OK:
         raise LstmError(rc, "lstm_bwd")
+    return rc
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def lstm_fwd_noalloc(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, stream=None,
+                     check: bool = True) -> int:
+    """Direct call of lstm_fwd_noalloc: lstm_fwd with the library's static
+    device scratch instead of a caller workspace (for callers that may not
+    allocate device memory)."""
+    rc = load().lstm_fwd_noalloc(ctypes.byref(d), _p(x), _p(W), _p(b), _p(h0), _p(c0), _p(y),
+                                 _p(hT), _p(cT), _p(gates), _p(cells), _stream(stream))
+    if check and rc != LSTM_OK:
+        raise LstmError(rc, "lstm_fwd_noalloc")
     return rc
 
 

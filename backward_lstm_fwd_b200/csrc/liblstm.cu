@@ -8,6 +8,7 @@
 
 #include <climits>
 #include <cstdlib>
+#include <mutex>
 #include <vector>
 
 #include "../../include/liblstm.h"
@@ -346,6 +347,35 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
 
 }  // namespace
 
+// ------------------------------------------ scratch for lstm_fwd_noalloc
+// A file-scope device array: every GPU that loads this library holds
+// LSTM_NOALLOC_SCRATCH_BYTES of it until the process exits.  In host code the
+// name g_noalloc_scratch is only a host-side stand-in for the symbol, never a
+// device address; the address is looked up per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LSTM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+int noalloc_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return LSTM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LSTM_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LSTM_OK;
+}
+}  // namespace
+
 // =================================================================== C ABI
 extern "C" {
 
@@ -460,6 +490,24 @@ int lstm_profile_end(double *ms, long long *launches) {
 }
 
 long long lstm_launch_count(void) { return launch_counter().load(); }
+
+int lstm_fwd_noalloc(const lstm_dims *d, const void *x, const void *W, const void *b,
+                     const void *h0, const float *c0, void *y, void *hT, float *cT,
+                     void *gates, float *cells, void *stream) {
+    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
+    const size_t need = fwd_layout(d).total;
+    if (need > (size_t)LSTM_NOALLOC_SCRATCH_BYTES) return LSTM_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    const int rc = noalloc_scratch(&ws);
+    if (rc != LSTM_OK) return rc;
+    // the shared buffer keeps the last call's bytes: zero the control block
+    // (status word and barrier counters) that the kernels expect at zero
+    if (cudaMemsetAsync(ws, 0, kCtrlBytes, (cudaStream_t)stream) != cudaSuccess)
+        return LSTM_ERR_CUDA;
+    return lstm_fwd(d, x, W, b, h0, c0, y, hT, cT, gates, cells, ws,
+                    (size_t)LSTM_NOALLOC_SCRATCH_BYTES, stream);
+}
 
 int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_mn_major,
                       const void *Bm, long long ldb, int b_mn_major, const void *bias, float *C,

@@ -152,6 +152,39 @@ int lstm_profile_end(double *ms, long long *launches);
 /* Kernel launches issued by this process's liblstm calls so far. */
 long long lstm_launch_count(void);
 
+/*
+ * lstm_fwd_noalloc -- the forward pass for callers that may not allocate
+ * device memory.  (The paper has no counterpart; this is a deployment aid.)
+ *
+ * Some callers cannot call cudaMalloc: a plugin inside a host program that owns
+ * the whole device-memory budget and forbids allocations it does not make
+ * itself, or a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device synchronisation.  This entry point takes the same inputs and outputs
+ * as lstm_fwd, but instead of a caller workspace it uses a scratch buffer of
+ * LSTM_NOALLOC_SCRATCH_BYTES that is a static device array inside the library:
+ * every GPU on which the library is loaded holds that buffer until the
+ * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Problems whose lstm_fwd_workspace_size() exceeds
+ *     LSTM_NOALLOC_SCRATCH_BYTES are rejected with LSTM_ERR_UNSUPPORTED
+ *     before anything is enqueued.
+ *   - The first call on a device (the current device) looks up that device's
+ *     address of the buffer; make that first call before any stream capture.
+ *   - All calls share the one buffer per device, which keeps the previous
+ *     call's contents; each call clears the parts that must start at zero (the
+ *     status word and barrier counters).  Calls whose executions overlap on the
+ *     GPU (different streams, or different host threads) race on the buffer:
+ *     serialise them.
+ *   - The status word lives in the shared buffer, so lstm_status cannot be
+ *     used with this entry point; callers that need device-side status use
+ *     lstm_fwd with their own workspace.
+ * Returns LSTM_OK or an LSTM_ERR_* code, like lstm_fwd.
+ */
+#define LSTM_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int lstm_fwd_noalloc(const lstm_dims *d, const void *x, const void *W, const void *b,
+                     const void *h0, const float *c0, void *y, void *hT, float *cT,
+                     void *gates, float *cells, void *stream);
+
 /* Static description of a status code. */
 const char *lstm_strerror(int code);
 
