@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH):
     ll = ctypes.c_longlong
     lib.lstm_test_tc_gemm.argtypes = [ip, ip, ip, vp, ll, ip, vp, ll, ip, vp, vp, ll, vp, sz, vp]
     lib.lstm_test_tc_gemm.restype = ip
+    lib.lstm_test_set_wait_fault.argtypes = [ip, ll]
+    lib.lstm_test_set_wait_fault.restype = ip
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -204,6 +206,12 @@ def test_tc_gemm(M, N, K, A, lda, a_mn_major, Bm, ldb, b_mn_major, bias, C, ldc,
     return int(load().lstm_test_tc_gemm(M, N, K, _p(A), lda, a_mn_major, _p(Bm), ldb, b_mn_major,
                                          _p(bias), _p(C), ldc, _p(ws),
                                          ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def test_set_wait_fault(skip_cta: int, wait_ns: int) -> None:
+    """Test hook: CTA `skip_cta` of persistent launches never arrives (-1: off);
+    device-side waits give up after wait_ns (<= 0: default 2 s)."""
+    load().lstm_test_set_wait_fault(int(skip_cta), int(wait_ns))
 
 
 # ------------------------------------------------------------------ helpers

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "simt.cuh"
 #include "tc_host.cuh"
+#include "tc_recur.cuh"
 
 using namespace lstm;
 
@@ -215,6 +216,106 @@ cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf
     return tcg::launch(bld, s);
 }
 
+// ------------------------------------------- persistent recurrence (bf16)
+// Test hooks (include/liblstm_testing.h): one CTA that never arrives, and the
+// bound of every device-side wait.
+int g_fault_skip_cta = -1;
+unsigned long long g_wait_ns = 2000000000ull;
+
+struct RecPlan {
+    int S, G, NB, kch, stages;
+    size_t smem;
+};
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// Grid of the persistent forward recurrence: S = H/16 unit slices times G
+// batch groups of NB rows (NB a power of two in 16..128), S*G <= SM count.
+bool plan_fwd_recur(const lstm_dims *d, RecPlan &P) {
+    if (d->dtype != LSTM_BF16 || d->H % rec::UNITS != 0 || d->H > 1024 || d->B < 1 ||
+        tcg::encode_fn() == nullptr)
+        return false;
+    const char *e = getenv("LSTM_FORCE_SIMT");
+    if (e && e[0] == '1') return false;
+    P.S = d->H / rec::UNITS;
+    const int gmax = tcg::sm_count() / P.S;
+    if (gmax < 1) return false;
+    int G = std::min(gmax, (d->B + 15) / 16);
+    int NB = 16;
+    while (NB < (d->B + G - 1) / G) NB *= 2;
+    if (NB > 128) return false;
+    P.G = (d->B + NB - 1) / NB;
+    if (P.G > gmax || P.G > 48) return false;
+    P.NB = NB;
+    P.kch = (d->H + 63) / 64;
+    const size_t fixed = rec::FwdSmem(P.kch, 0, NB).total + 1024;
+    const size_t per_stage = (size_t)NB * 128;
+    if (fixed + 2 * per_stage > kMaxSmem) return false;
+    P.stages = (int)std::min<size_t>(8, (kMaxSmem - fixed) / per_stage);
+    P.smem = rec::FwdSmem(P.kch, P.stages, NB).total + 1024;
+    return true;
+}
+
+template <int NB>
+cudaError_t launch_fwd_recur(const rec::FwdParams &prm, int grid, size_t smem, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(rec::fwd_kernel<NB>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    } else {
+        cudaFuncSetAttribute(rec::fwd_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(rec::NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;  // all CTAs co-resident, or the launch fails
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, rec::fwd_kernel<NB>, prm);
+    note_launch();
+    return e;
+}
+
+// a2 as one persistent cooperative launch (see tc_recur.cuh).
+int tc_fwd_recurrence(const lstm_dims *d, const RecPlan &P, const bf16 *W, const bf16 *h0,
+                      const float *c0, const float *Gx, bf16 *y, bf16 *hT, float *cT, bf16 *gates,
+                      float *cells, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I;
+    rec::FwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    bool ok = tcg::make_map(&prm.map_w, W, H + I, 4 * H, (H + I) * 2, 64, rec::UNITS) &&
+              tcg::make_map(&prm.map_y, y, H, T * B, H * 2, 64, P.NB);
+    if (h0) ok = ok && tcg::make_map(&prm.map_h0, h0, H, B, H * 2, 64, P.NB);
+    else prm.map_h0 = prm.map_y;
+    if (!ok) return LSTM_ERR_UNSUPPORTED;
+    prm.Gx = Gx; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
+    prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.S = P.S; prm.G = P.G;
+    prm.kch = P.kch; prm.stages = P.stages; prm.has_h0 = h0 != nullptr;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const int grid = P.S * P.G;
+    cudaError_t e;
+    switch (P.NB) {
+        case 16: e = launch_fwd_recur<16>(prm, grid, P.smem, s); break;
+        case 32: e = launch_fwd_recur<32>(prm, grid, P.smem, s); break;
+        case 64: e = launch_fwd_recur<64>(prm, grid, P.smem, s); break;
+        default: e = launch_fwd_recur<128>(prm, grid, P.smem, s); break;
+    }
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ forward pass
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
@@ -237,8 +338,16 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
                                                   simt::EpGx<T>{Gx, b, 4 * H}, s)));
             }
         }
-        // a2: the recurrence, one fused GEMM + gate/cell/hidden epilogue per step
+        // a2: the recurrence
         prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
+        RecPlan plan;
+        if (plan_fwd_recur(d, plan)) {
+            // persistent tcgen05 kernel: all T steps in one launch; it writes hT and cT
+            return tc_fwd_recurrence(d, plan, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
+                                     (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells, (Ctrl *)ws,
+                                     s);
+        }
+        // otherwise one fused GEMM + gate/cell/hidden epilogue launch per step
         for (int t = 0; t < T_; ++t) {
             const T *hp = t > 0 ? y + (long long)(t - 1) * BH : h0;
             const float *cp = t > 0 ? cells + (long long)(t - 1) * BH : c0;
@@ -527,6 +636,12 @@ int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_m
     tcg::Builder::add_seg(q, ma, 0, mb, 0, K);
     if (!bld.ok) return LSTM_ERR_UNSUPPORTED;
     return tcg::launch(bld, (cudaStream_t)stream) == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+int lstm_test_set_wait_fault(int skip_cta, long long wait_ns) {
+    g_fault_skip_cta = skip_cta;
+    g_wait_ns = wait_ns > 0 ? (unsigned long long)wait_ns : 2000000000ull;
+    return LSTM_OK;
 }
 
 int lstm_status(void *ws, size_t ws_bytes, void *stream) {

@@ -27,6 +27,16 @@ int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_m
                       const void *B, long long ldb, int b_mn_major, const void *bias, float *C,
                       long long ldc, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Failure-detection hook for the persistent recurrent kernels: from now on,
+ * CTA `skip_cta` of every persistent launch never signals its step barrier
+ * (-1 turns that off), and every device-side wait gives up after `wait_ns`
+ * nanoseconds (<= 0 restores the default of 2 s).  A wait that gives up records
+ * LSTM_ERR_TIMEOUT in the workspace status word and the kernel returns; nothing
+ * faults.  Process-wide, not thread-safe.
+ */
+int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
+
 #ifdef __cplusplus
 }
 #endif
