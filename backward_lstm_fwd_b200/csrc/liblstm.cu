@@ -108,9 +108,10 @@ FwdLayout fwd_layout(const lstm_dims *d) {
 constexpr long long kDbMaxChunks = 2048;
 
 struct BwdLayout {
-    size_t dG, dc, dbpart, total;
+    size_t dG, dc, dbpart, wt, dbgroup, total;
     int db_chunks, db_rows_per_chunk;
 };
+constexpr int kMaxGroups = 48;
 BwdLayout bwd_layout(const lstm_dims *d) {
     BwdLayout L;
     const size_t TB = (size_t)d->T * d->B, G4 = 4 * (size_t)d->H;
@@ -122,7 +123,14 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     L.dG = kCtrlBytes;
     L.dc = align_up(L.dG + TB * G4 * esize(d), 256);
     L.dbpart = align_up(L.dc + 2 * BH * sizeof(float), 256);
-    L.total = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
+    L.wt = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
+    L.dbgroup = L.wt;
+    L.total = L.wt;
+    if (d->dtype == LSTM_BF16) {
+        // W_h^T [H][4H] and per-batch-group db partials of the persistent kernel
+        L.dbgroup = align_up(L.wt + (size_t)d->H * G4 * 2, 256);
+        L.total = align_up(L.dbgroup + (size_t)kMaxGroups * G4 * sizeof(float), 256);
+    }
     return L;
 }
 
@@ -258,15 +266,12 @@ bool plan_fwd_recur(const lstm_dims *d, RecPlan &P) {
 
 template <int NB>
 cudaError_t launch_fwd_recur(const rec::FwdParams &prm, int grid, size_t smem, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
+    static size_t attr_smem = 0;
+    if (attr_smem < smem) {
         cudaError_t e = cudaFuncSetAttribute(rec::fwd_kernel<NB>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr = true;
-    } else {
-        cudaFuncSetAttribute(rec::fwd_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+        attr_smem = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -314,6 +319,88 @@ int tc_fwd_recurrence(const lstm_dims *d, const RecPlan &P, const bf16 *W, const
         return LSTM_ERR_NOT_CORESIDENT;
     }
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+// Grid of the persistent backward recurrence: S = H/16 unit slices times G
+// batch groups of NB <= 64 rows (the MMA's M is 64), S*G <= SM count.
+bool plan_bwd_recur(const lstm_dims *d, RecPlan &P) {
+    if (d->dtype != LSTM_BF16 || d->H % rec::UNITS != 0 || d->H > 1024 || d->B < 1 ||
+        tcg::encode_fn() == nullptr)
+        return false;
+    const char *e = getenv("LSTM_FORCE_SIMT");
+    if (e && e[0] == '1') return false;
+    P.S = d->H / rec::UNITS;
+    const int gmax = std::min(tcg::sm_count() / P.S, kMaxGroups);
+    if (gmax < 1) return false;
+    int G = std::min(gmax, (d->B + 15) / 16);
+    int NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    if (NB > 64) {
+        G = (d->B + 63) / 64;
+        NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    }
+    P.G = (d->B + NB - 1) / NB;
+    if (P.G > gmax) return false;
+    P.NB = NB;
+    P.kch = 4 * d->H / 64;
+    const size_t fixed = rec::BwdSmem(P.kch, 0).total + 1024;
+    if (fixed + 2 * rec::BWD_STAGE_BYTES > kMaxSmem) return false;
+    P.stages = (int)std::min<size_t>(8, (kMaxSmem - fixed) / rec::BWD_STAGE_BYTES);
+    P.smem = rec::BwdSmem(P.kch, P.stages).total + 1024;
+    return true;
+}
+
+// a3 (+ a5) as one persistent cooperative launch (see tc_recur.cuh); W_h^T is
+// written to the workspace first, and db is the sum of the groups' partials.
+int tc_bwd_recurrence(const lstm_dims *d, const RecPlan &P, const bf16 *dy, const bf16 *dhT,
+                      const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
+                      const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
+                      float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I, G4 = 4 * H;
+    {
+        dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
+        rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)I);
+        note_launch();
+        if (cudaGetLastError() != cudaSuccess) return LSTM_ERR_CUDA;
+    }
+    rec::BwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!tcg::make_map(&prm.map_wt, WT, G4, H, G4 * 2, 64, rec::UNITS) ||
+        !tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB))
+        return LSTM_ERR_UNSUPPORTED;
+    prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
+    prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
+    prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.S = P.S; prm.G = P.G; prm.NB = P.NB;
+    prm.kch4 = P.kch; prm.stages = P.stages;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    static size_t attr_smem = 0;
+    if (attr_smem < P.smem) {
+        if (cudaFuncSetAttribute(rec::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)P.smem) != cudaSuccess)
+            return LSTM_ERR_CUDA;
+        attr_smem = P.smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(P.S * P.G);
+    cfg.blockDim = dim3(rec::NUM_THREADS);
+    cfg.dynamicSmemBytes = P.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, rec::bwd_kernel, prm);
+    note_launch();
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    if (e != cudaSuccess) return LSTM_ERR_CUDA;
+    simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ forward pass
@@ -393,6 +480,37 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         if ((long long)G4 * K > 0) LSTM_TRY(cudaMemsetAsync(dW, 0, (size_t)G4 * K * sizeof(float), s));
         if (G4 > 0) LSTM_TRY(cudaMemsetAsync(db, 0, (size_t)G4 * sizeof(float), s));
         if (TB * I > 0) LSTM_TRY(cudaMemsetAsync(dx, 0, (size_t)(TB * I) * sizeof(float), s));
+        return LSTM_OK;
+    }
+
+    RecPlan plan;
+    if (plan_bwd_recur(d, plan)) {
+        {   // a3 + a5: persistent tcgen05 recurrence with db fused
+            prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
+            const int rc = tc_bwd_recurrence(
+                d, plan, (const bf16 *)dy, (const bf16 *)dhT, dcT, (const bf16 *)W, c0,
+                (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
+                (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
+            if (rc != LSTM_OK) return rc;
+        }
+        if (tc_gemm_ok(d)) {
+            prof::Phase ph(LSTM_PHASE_DW, s);
+            LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
+                              (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s));
+            return LSTM_OK;
+        }
+        // dW / dx on CUDA cores (shapes off the TMA grid)
+        {
+            prof::Phase ph(LSTM_PHASE_DW, s);
+            LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
+                                                simt::Zrows<T>{x, y, h0, B, I, H},
+                                                simt::EpStore{dW, K}, s)));
+        }
+        prof::Phase ph(LSTM_PHASE_DX, s);
+        if (I > 0)
+            LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
+                                               simt::RowMajor<T>{W + H, K},
+                                               simt::EpStore{dx, I}, s)));
         return LSTM_OK;
     }
 

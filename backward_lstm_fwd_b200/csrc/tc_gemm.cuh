@@ -210,7 +210,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
         for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
             int mt, nt;
             const Problem &P = p.prob[locate(p, tile, mt, nt)];
-            if (!tc::mbar_wait(&tfull[acc], aphase, p.ctrl, abort_flag, 0x104)) break;
+            const bool w = tc::mbar_wait(&tfull[acc], aphase, p.ctrl, abort_flag, 0x104);
+            if (!__all_sync(0xffffffffu, w)) break;  // the whole warp leaves together
             tc::tc_fence_after();
             int nk = 0;
             for (int sg = 0; sg < P.nseg; ++sg) nk += P.seg[sg].nkb;

@@ -64,6 +64,22 @@ __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// AND of `v` over the 128 epilogue threads (named barrier 2), so that every
+// epilogue thread takes the same branch after a bounded wait -- no thread is
+// left alone at a later barrier or warp-synchronous TMEM load.
+__device__ __forceinline__ bool epi_vote_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
 // Wait until *ctr >= target (acquire).  Bounded by limit_ns of %globaltimer;
 // on time-out record LSTM_ERR_TIMEOUT with `site` and raise the abort flag.
 __device__ __forceinline__ bool wait_counter(const unsigned int *ctr, unsigned int target,
@@ -245,8 +261,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
         load_gx(0);
         for (int t = 0; t < p.T; ++t) {
             const int acc = t & 1;
-            if (!tc::mbar_wait(&mma_done[acc], (t >> 1) & 1, p.ctrl, abort_flag, 0x205, p.wait_ns))
-                break;
+            const bool w = tc::mbar_wait(&mma_done[acc], (t >> 1) & 1, p.ctrl, abort_flag, 0x205,
+                                         p.wait_ns);
+            if (!epi_vote_all(w)) break;
             tc::tc_fence_after();
             const bool zero = (t == 0 && !p.has_h0);
             // TMEM rows of this warp: gate q, unit = lane (lanes 0..15)
@@ -305,6 +322,366 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
     if (warp == 1) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+
+// ===========================================================================
+// Persistent tcgen05 kernel of the backward recurrence (bf16), "SingleLayerLstmGrad"
+// backward algorithm steps 1-3, 5 and 6, with db (step 4) accumulated on the way:
+// for t = T-1 .. 0
+//   delta h_t  = dy_t + (t == T-1 ? dhT : dG_{t+1} W_h)          (steps 1, 5, 6)
+//   delta c_t  = delta h_t o (1 - tanh^2 c_t) + delta c_next      (step 2)
+//   do, dg, di, df                                                (step 3)
+//   delta c_next = delta c_t f_t                                  (steps 5, 6)
+// and finally dh0 = dG_0 W_h, dc0 = delta c_next.
+//
+// Decomposition: CTA (s, gi) owns hidden units j0 = 16 s .. j0 + 15 and batch
+// rows b0 = gi * NB .. b0 + NB - 1 (NB <= 64).  Its product is
+// D[64 batch rows, 16 units] = dG_{t+1}[rows, 0:4H] . W_h[0:4H, units]: A = the
+// dG rows, TMA-streamed in 64-wide K chunks after the group barrier; B = the
+// CTA's 16 rows of W_h^T (a transposed copy in the workspace), resident in
+// shared memory (K-major, 128-byte swizzle).  Only the first NB rows of each A
+// chunk are loaded; the rest of the 64-row tile is stale and its output rows
+// are never read.  dG_t of all units is exchanged through global memory with
+// one release/acquire counter per batch group, exactly as in the forward kernel.
+//
+// Epilogue thread (q, lane): batch row m = 16 q + lane % 16 (the TMEM lane of
+// that row in an M = 64 accumulator), units j0 + 8 * (lane / 16) .. + 7; lanes
+// 16..31 receive their eight values from lane - 16 by shuffle.
+// ===========================================================================
+
+constexpr int BWD_STAGE_BYTES = 64 * 128;  // one 64-row x 64-wide A chunk
+constexpr int WT_CHUNK_BYTES = UNITS * 128;
+
+struct BwdParams {
+    CUtensorMap map_wt;   // W_h^T [H][4H], box {64, 16}
+    CUtensorMap map_dg;   // dG [T*B][4H], box {64, NB}
+    const __nv_bfloat16 *dy, *dhT, *gates;
+    const float *dcT, *cells, *c0;
+    __nv_bfloat16 *dG;
+    float *dh0, *dc0, *db_part;  // db_part [G][4H]
+    Ctrl *ctrl;
+    int T, B, H, S, G, NB, kch4, stages;
+    int fault_skip_cta;
+    unsigned long long wait_ns;
+};
+
+struct BwdSmem {
+    int wt, ring, bars, total;
+    __host__ __device__ BwdSmem(int kch4, int stages) {
+        wt = 0;
+        ring = kch4 * WT_CHUNK_BYTES;
+        bars = ring + stages * BWD_STAGE_BYTES;
+        total = bars + 256;
+    }
+};
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&f)[8]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&f)[8]) {
+    uint4 v;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    return v;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const BwdSmem L(p.kch4, p.stages);
+    uint8_t *sWT = smem + L.wt;
+    uint8_t *ring = smem + L.ring;
+    uint64_t *bars = (uint64_t *)(smem + L.bars);
+    uint64_t *full = bars;
+    uint64_t *empty = bars + 8;
+    uint64_t *w_full = bars + 16;
+    uint64_t *mma_done = bars + 17;
+    uint32_t *tmem_slot = (uint32_t *)(bars + 20);
+    volatile int *abort_flag = (volatile int *)(bars + 21);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int s = blockIdx.x % p.S, gi = blockIdx.x / p.S;
+    const int j0 = s * UNITS, b0 = gi * p.NB;
+    const int H = p.H, B = p.B, T = p.T, NB = p.NB;
+    unsigned int *ctr = &p.ctrl->bar[gi];
+    constexpr uint32_t TMEM_COLS = 32;  // two 16-column accumulators
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.stages; ++i) {
+            tc::mbar_init(&full[i], 1);
+            tc::mbar_init(&empty[i], 1);
+        }
+        tc::mbar_init(w_full, 1);
+        tc::mbar_init(&mma_done[0], 1);
+        tc::mbar_init(&mma_done[1], 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(w_full, (uint32_t)(p.kch4 * WT_CHUNK_BYTES));
+            for (int kc = 0; kc < p.kch4; ++kc)
+                tc::tma_load_2d(sWT + kc * WT_CHUNK_BYTES, &p.map_wt, w_full, 64 * kc, j0);
+            uint32_t stage = 0, phase = 0;
+            bool aborted = false;
+            // MMA iteration i = 1..T consumes dG_{T-i}, written in iteration i-1
+            for (int i = 1; i <= T && !aborted; ++i) {
+                if (!wait_counter(ctr, (unsigned)(p.S * i), p.ctrl, abort_flag, 0x301, p.wait_ns)) {
+                    aborted = true;
+                    break;
+                }
+                tc::fence_proxy_async_global();
+                const int row0 = (T - i) * B + b0;
+                for (int kc = 0; kc < p.kch4; ++kc) {
+                    if (!tc::mbar_wait(&empty[stage], phase ^ 1, p.ctrl, abort_flag, 0x302,
+                                       p.wait_ns)) {
+                        aborted = true;
+                        break;
+                    }
+                    tc::mbar_arrive_expect_tx(&full[stage], NB * 128);
+                    tc::tma_load_2d(ring + stage * BWD_STAGE_BYTES, &p.map_dg, &full[stage], 64 * kc,
+                                    row0);
+                    if (++stage == (uint32_t)p.stages) stage = 0, phase ^= 1;
+                }
+            }
+            if (aborted) {
+                tc::mbar_wait(w_full, 0, nullptr, nullptr, 0, 200000000ull);
+                for (int i = 0; i < p.stages; ++i) {
+                    if (stage == 0) stage = p.stages, phase ^= 1;
+                    --stage;
+                    tc::mbar_wait(&full[stage], phase, nullptr, nullptr, 0, 200000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t stage = 0, phase = 0;
+            const uint32_t idesc = tc::idesc_bf16_f32(64, UNITS, 0, 0);
+            bool ok = tc::mbar_wait(w_full, 0, p.ctrl, abort_flag, 0x303, p.wait_ns);
+            for (int i = 1; ok && i <= T; ++i) {
+                const uint32_t d = tmem_base + (i & 1) * UNITS;
+                for (int kc = 0; kc < p.kch4; ++kc) {
+                    if (!tc::mbar_wait(&full[stage], phase, p.ctrl, abort_flag, 0x304, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint32_t a = tc::smem_u32(ring + stage * BWD_STAGE_BYTES);
+                    const uint32_t b = tc::smem_u32(sWT + kc * WT_CHUNK_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        tc::mma_bf16(d, tc::smem_desc_sw128(a + 32 * k, 16, 1024),
+                                     tc::smem_desc_sw128(b + 32 * k, 16, 1024), idesc,
+                                     (kc | k) != 0);
+                    tc::mma_commit(&empty[stage]);
+                    if (++stage == (uint32_t)p.stages) stage = 0, phase ^= 1;
+                }
+                if (ok) tc::mma_commit(&mma_done[i & 1]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;
+        const int q = warp & 3;
+        const int m = 16 * q + (lane & 15);
+        const int half = lane >> 4;
+        const int b = b0 + m;
+        const int jb = j0 + 8 * half;
+        const bool valid = (m < NB) && (b < B);
+        const long long G4 = 4LL * H;
+        float dc[8], dbacc[4][8];
+        float gv[4][8], ct[8], cp[8], dyv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            dc[u] = (valid && p.dcT) ? p.dcT[(long long)b * H + jb + u] : 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) dbacc[g][u] = 0.f;
+        }
+        // saved forward state of step t for this thread's 8 (row, unit) pairs
+        auto load_step = [&](int t) {
+            if (!valid) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    ct[u] = cp[u] = dyv[u] = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) gv[g][u] = 0.f;
+                }
+                return;
+            }
+            const long long row = (long long)t * B + b;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + g * H + jb)),
+                              gv[g]);
+            const float4 *c4 = reinterpret_cast<const float4 *>(p.cells + row * H + jb);
+            const float4 x0 = __ldg(c4), x1 = __ldg(c4 + 1);
+            ct[0] = x0.x; ct[1] = x0.y; ct[2] = x0.z; ct[3] = x0.w;
+            ct[4] = x1.x; ct[5] = x1.y; ct[6] = x1.z; ct[7] = x1.w;
+            const float *cpp = t > 0 ? p.cells + (row - B) * H + jb
+                                     : (p.c0 ? p.c0 + (long long)b * H + jb : nullptr);
+            if (cpp) {
+                const float4 y0 = __ldg(reinterpret_cast<const float4 *>(cpp));
+                const float4 y1 = __ldg(reinterpret_cast<const float4 *>(cpp) + 1);
+                cp[0] = y0.x; cp[1] = y0.y; cp[2] = y0.z; cp[3] = y0.w;
+                cp[4] = y1.x; cp[5] = y1.y; cp[6] = y1.z; cp[7] = y1.w;
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) cp[u] = 0.f;
+            }
+            if (p.dy) {
+                bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.dy + row * H + jb)), dyv);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) dyv[u] = 0.f;
+            }
+        };
+        // delta h from the MMA of iteration i (accumulator i & 1), 8 units per thread
+        uint32_t dphase[2] = {0, 0};
+        auto read_dh = [&](int i, float (&dh)[8]) -> bool {
+            const int acc = i & 1;
+            const bool w =
+                tc::mbar_wait(&mma_done[acc], dphase[acc], p.ctrl, abort_flag, 0x305, p.wait_ns);
+            if (!epi_vote_all(w)) return false;
+            dphase[acc] ^= 1;
+            tc::tc_fence_after();
+            uint32_t r[16];
+            tc::tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + acc * UNITS, r);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float hi = __shfl_sync(0xffffffffu, __uint_as_float(r[8 + u]), lane & 15);
+                dh[u] = half ? hi : __uint_as_float(r[u]);
+            }
+            tc::tc_fence_before();
+            return true;
+        };
+
+        load_step(T - 1);
+        bool ok = true;
+        for (int i = 0; i < T; ++i) {
+            const int t = T - 1 - i;
+            float dhr[8];
+            if (i == 0) {
+                if (valid && p.dhT) {
+                    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.dhT + (long long)b * H + jb)),
+                                  dhr);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dhr[u] = 0.f;
+                }
+            } else if (!read_dh(i, dhr)) {
+                ok = false;
+                break;
+            }
+            float dI[8], dF[8], dGg[8], dO[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float ig = gv[0][u], fg = gv[1][u], gg = gv[2][u], og = gv[3][u];
+                const float dh = dyv[u] + dhr[u];                       // step 1
+                const float tc_ = tanhf_(ct[u]);
+                const float dcv = dh * og * (1.f - tc_ * tc_) + dc[u];  // step 2
+                dO[u] = dh * tc_ * og * (1.f - og);                     // step 3
+                dGg[u] = dcv * ig * (1.f - gg * gg);
+                dI[u] = dcv * gg * ig * (1.f - ig);
+                dF[u] = dcv * cp[u] * fg * (1.f - fg);
+                dc[u] = dcv * fg;                                       // step 5
+            }
+            if (valid) {
+                __nv_bfloat16 *o = p.dG + ((long long)t * B + b) * G4 + jb;
+                const uint4 vi = f32x8_to_bf16(dI), vf = f32x8_to_bf16(dF);
+                const uint4 vg = f32x8_to_bf16(dGg), vo = f32x8_to_bf16(dO);
+                *reinterpret_cast<uint4 *>(o) = vi;
+                *reinterpret_cast<uint4 *>(o + H) = vf;
+                *reinterpret_cast<uint4 *>(o + 2 * H) = vg;
+                *reinterpret_cast<uint4 *>(o + 3 * H) = vo;
+                // db (step 4) sums the stored (rounded) values, as dW does
+                float ri[8], rf[8], rg[8], ro[8];
+                bf16x8_to_f32(vi, ri); bf16x8_to_f32(vf, rf);
+                bf16x8_to_f32(vg, rg); bf16x8_to_f32(vo, ro);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    dbacc[0][u] += ri[u];
+                    dbacc[1][u] += rf[u];
+                    dbacc[2][u] += rg[u];
+                    dbacc[3][u] += ro[u];
+                }
+            }
+            tc::fence_proxy_async_global();  // dG_t is read next by TMA
+            named_bar(1, EPI_THREADS);
+            if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) {
+                __threadfence();
+                red_release_add(ctr, 1u);
+            }
+            if (t > 0) load_step(t - 1);
+        }
+        float dh0v[8];
+        ok = ok && read_dh(T, dh0v);  // uniform over the epilogue threads
+        if (ok && valid) {
+            float4 *o = reinterpret_cast<float4 *>(p.dh0 + (long long)b * H + jb);
+            o[0] = make_float4(dh0v[0], dh0v[1], dh0v[2], dh0v[3]);
+            o[1] = make_float4(dh0v[4], dh0v[5], dh0v[6], dh0v[7]);
+            float4 *oc = reinterpret_cast<float4 *>(p.dc0 + (long long)b * H + jb);
+            oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
+            oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
+        }
+        // db partial of this CTA: sum over its rows, in a fixed order
+        if (ok) {
+            float *red = reinterpret_cast<float *>(ring);  // [64 rows][64 = 4 gates x 16 units]
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    red[m * 64 + g * 16 + 8 * half + u] = valid ? dbacc[g][u] : 0.f;
+            named_bar(1, EPI_THREADS);
+            if (et < 64) {
+                float sum = 0.f;
+                for (int r = 0; r < 64; ++r) sum += red[r * 64 + et];
+                const int g = et / 16, u = et % 16;
+                p.db_part[(long long)gi * G4 + (long long)g * H + j0 + u] = sum;
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// W_h^T [H][4H] from W [4H][H+I] (the K-major B operand of the backward kernel).
+__global__ void transpose_wh(const __nv_bfloat16 *__restrict__ W, __nv_bfloat16 *__restrict__ WT,
+                             int H, int I) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;  // rows of W (4H), columns (H)
+    const int tx = threadIdx.x, ty = threadIdx.y;          // 32 x 8
+    for (int k = ty; k < 32; k += 8) {
+        const int r = r0 + k, c = c0 + tx;
+        if (r < 4 * H && c < H) tile[k][tx] = W[(long long)r * (H + I) + c];
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+        const int c = c0 + k, r = r0 + tx;
+        if (r < 4 * H && c < H) WT[(long long)c * 4 * H + r] = tile[tx][k];
     }
 }
 
