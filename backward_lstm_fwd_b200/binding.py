@@ -86,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_tc_gemm.restype = ip
     lib.lstm_test_set_wait_fault.argtypes = [ip, ll]
     lib.lstm_test_set_wait_fault.restype = ip
+    lib.lstm_test_last_paths.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
+    lib.lstm_test_last_paths.restype = ip
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -212,6 +214,14 @@ def test_set_wait_fault(skip_cta: int, wait_ns: int) -> None:
     """Test hook: CTA `skip_cta` of persistent launches never arrives (-1: off);
     device-side waits give up after wait_ns (<= 0: default 2 s)."""
     load().lstm_test_set_wait_fault(int(skip_cta), int(wait_ns))
+
+
+def test_last_paths():
+    """Test hook: (forward, backward) recurrent kernel of the last calls:
+    0 per-step CUDA cores, 1 persistent K-resident, 2 persistent cluster."""
+    f, b = ctypes.c_int(), ctypes.c_int()
+    load().lstm_test_last_paths(ctypes.byref(f), ctypes.byref(b))
+    return f.value, b.value
 
 
 # ------------------------------------------------------------------ helpers

@@ -17,6 +17,7 @@
 #include "simt.cuh"
 #include "tc_host.cuh"
 #include "tc_recur.cuh"
+#include "tc_recur2.cuh"
 
 using namespace lstm;
 
@@ -228,6 +229,9 @@ cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf
 // Test hooks (include/liblstm_testing.h): one CTA that never arrives, and the
 // bound of every device-side wait.
 int g_fault_skip_cta = -1;
+// Which recurrent kernel the last lstm_fwd / lstm_bwd used (test hook):
+// 0 per-step CUDA-core kernels, 1 persistent K-resident kernel, 2 cluster kernel.
+int g_last_fwd_path = -1, g_last_bwd_path = -1;
 unsigned long long g_wait_ns = 2000000000ull;
 
 struct RecPlan {
@@ -259,7 +263,7 @@ bool plan_fwd_recur(const lstm_dims *d, RecPlan &P) {
     const size_t fixed = rec::FwdSmem(P.kch, 0, NB).total + 1024;
     const size_t per_stage = (size_t)NB * 128;
     if (fixed + 2 * per_stage > kMaxSmem) return false;
-    P.stages = (int)std::min<size_t>(8, (kMaxSmem - fixed) / per_stage);
+    P.stages = (int)std::min<size_t>(rec::MAX_STAGES, (kMaxSmem - fixed) / per_stage);
     P.smem = rec::FwdSmem(P.kch, P.stages, NB).total + 1024;
     return true;
 }
@@ -344,7 +348,7 @@ bool plan_bwd_recur(const lstm_dims *d, RecPlan &P) {
     P.kch = 4 * d->H / 64;
     const size_t fixed = rec::BwdSmem(P.kch, 0).total + 1024;
     if (fixed + 2 * rec::BWD_STAGE_BYTES > kMaxSmem) return false;
-    P.stages = (int)std::min<size_t>(8, (kMaxSmem - fixed) / rec::BWD_STAGE_BYTES);
+    P.stages = (int)std::min<size_t>(rec::MAX_STAGES, (kMaxSmem - fixed) / rec::BWD_STAGE_BYTES);
     P.smem = rec::BwdSmem(P.kch, P.stages).total + 1024;
     return true;
 }
@@ -403,6 +407,237 @@ int tc_bwd_recurrence(const lstm_dims *d, const RecPlan &P, const bf16 *dy, cons
     return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
+// --------------------------------------- cluster recurrence kernels (bf16)
+struct Rec2Plan {
+    int KS, G, NB, kcc, R, stages;
+    size_t smem;
+};
+
+bool force_simt() {
+    const char *e = getenv("LSTM_FORCE_SIMT");
+    return e && e[0] == '1';
+}
+
+int max_active_clusters(const void *kern, int threads, size_t smem, int KS) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(KS);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = KS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+const void *fwd2_kernel_ptr(int NB, int KS) {
+#define LSTM_F2(nb, ks) \
+    if (NB == nb && KS == ks) return (const void *)rec2::fwd2_kernel<nb, ks>;
+    LSTM_F2(16, 1) LSTM_F2(16, 2) LSTM_F2(16, 4)
+    LSTM_F2(32, 1) LSTM_F2(32, 2) LSTM_F2(32, 4) LSTM_F2(32, 8)
+    LSTM_F2(64, 2) LSTM_F2(64, 4) LSTM_F2(64, 8)
+    LSTM_F2(128, 4) LSTM_F2(128, 8)
+#undef LSTM_F2
+    return nullptr;
+}
+
+// Forward: R = H/32 row slices x KS K-parts x G batch groups of NB rows;
+// R * G clusters of KS must be co-resident.
+bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
+    if (d->dtype != LSTM_BF16 || d->H % rec2::F_UNITS != 0 || d->B < 1 ||
+        tcg::encode_fn() == nullptr || force_simt())
+        return false;
+    const int nsm = tcg::sm_count();
+    P.R = d->H / rec2::F_UNITS;
+    for (int KS : {4, 2, 8, 1}) {
+        if ((d->H / KS) % 64 != 0 || d->H % KS != 0) continue;
+        const int kcc = d->H / KS / 64;
+        if (kcc < 1 || kcc > rec2::MAX_KCC) continue;
+        const int gsm = std::min(nsm / (P.R * KS), kMaxGroups);  // SM bound first
+        if (gsm < 1) continue;
+        const int G0 = std::min(gsm, (d->B + 15) / 16);
+        int NB = 16;
+        while (NB < (d->B + G0 - 1) / G0) NB *= 2;
+        NB = std::max(NB, 4 * KS);
+        if (NB > 128 || NB / KS > 32) continue;
+        const int G = (d->B + NB - 1) / NB;
+        const size_t smem = rec2::Fwd2Smem(kcc, NB, KS).total + 1024;
+        if (smem > kMaxSmem) continue;
+        const void *kern = fwd2_kernel_ptr(NB, KS);
+        if (!kern) continue;
+        const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
+        if (G * P.R > maxc) continue;
+        P.KS = KS; P.G = G; P.NB = NB; P.kcc = kcc; P.smem = smem;
+        return true;
+    }
+    return false;
+}
+
+// Backward: U = H/128 unit slices x 8 K-parts of 4H x G batch groups of NB rows;
+// U * G clusters of 8 must be co-resident (cudaOccupancyMaxActiveClusters).
+bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
+    if (d->dtype != LSTM_BF16 || d->H % rec2::B_UNITS != 0 || d->B < 1 ||
+        tcg::encode_fn() == nullptr || force_simt())
+        return false;
+    P.KS = rec2::B_KS;
+    P.R = d->H / rec2::B_UNITS;
+    P.kcc = 4 * d->H / rec2::B_KS / 64;
+    if (P.kcc < 1 || P.kcc > rec2::MAX_KCC) return false;
+    const size_t fixed = rec2::Bwd2Smem(P.kcc, 0).total + 1024;
+    if (fixed + 2 * rec2::B_ACHUNK > kMaxSmem) return false;
+    const int stages = (int)std::min<size_t>(std::min(P.kcc, rec2::MAX_KCC),
+                                             (kMaxSmem - fixed) / rec2::B_ACHUNK);
+    if (stages < 2 && P.kcc > 1) return false;
+    P.NB = stages;  // (ring stages; NB is reassigned to the batch rows below)
+    P.smem = rec2::Bwd2Smem(P.kcc, stages).total + 1024;
+    const int maxc = max_active_clusters((const void *)rec2::bwd2_kernel, rec2::B_THREADS, P.smem,
+                                         P.KS);
+    const int gmax = std::min(maxc / P.R, kMaxGroups);
+    if (gmax < 1) return false;
+    int G = std::min(gmax, (d->B + 15) / 16);
+    int NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    if (NB > rec2::B_MROWS) {
+        G = (d->B + rec2::B_MROWS - 1) / rec2::B_MROWS;
+        NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    }
+    P.G = (d->B + NB - 1) / NB;
+    if (P.G > gmax) return false;
+    P.stages = stages;
+    P.NB = NB;
+    return true;
+}
+
+// One cooperative launch of `grid` CTAs in clusters of KS (all CTAs co-resident
+// or the launch fails).  If this runtime refuses cooperative cluster launches,
+// the cluster launch goes ahead when the occupancy calculator says every
+// cluster fits at once (the kernels' waits are bounded either way).
+template <class Kern, class Prm>
+cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t smem,
+                           cudaStream_t s, int threads = rec::NUM_THREADS) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = KS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeCooperative;
+    at[1].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    note_launch();
+    if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) return e;
+    cudaGetLastError();
+    cfg.numAttrs = 1;  // cluster launch without the cooperative attribute
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess ||
+        nclusters * KS < grid) {
+        cudaGetLastError();
+        return cudaErrorCooperativeLaunchTooLarge;
+    }
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+template <int NB, int KS>
+cudaError_t launch_fwd2_t(const rec2::Fwd2Params &prm, const Rec2Plan &P, cudaStream_t s) {
+    return launch_cluster(rec2::fwd2_kernel<NB, KS>, prm, P.R * KS * P.G, KS, P.smem, s,
+                          rec2::F_THREADS);
+}
+
+cudaError_t launch_fwd2(const rec2::Fwd2Params &prm, const Rec2Plan &P, cudaStream_t s) {
+#define LSTM_F2(nb, ks) \
+    if (P.NB == nb && P.KS == ks) return launch_fwd2_t<nb, ks>(prm, P, s);
+    LSTM_F2(16, 1) LSTM_F2(16, 2) LSTM_F2(16, 4)
+    LSTM_F2(32, 1) LSTM_F2(32, 2) LSTM_F2(32, 4) LSTM_F2(32, 8)
+    LSTM_F2(64, 2) LSTM_F2(64, 4) LSTM_F2(64, 8)
+    LSTM_F2(128, 4) LSTM_F2(128, 8)
+#undef LSTM_F2
+    return cudaErrorInvalidConfiguration;
+}
+
+// a2 on the cluster kernel; returns LSTM_ERR_UNSUPPORTED (nothing launched)
+// when the plan has no instantiation, so that the caller can fall back.
+int tc_fwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *W, const bf16 *h0,
+                       const float *c0, const float *Gx, bf16 *y, bf16 *hT, float *cT,
+                       bf16 *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I;
+    rec2::Fwd2Params prm;
+    memset(&prm, 0, sizeof(prm));
+    bool ok = tcg::make_map(&prm.map_w, W, H + I, 4 * H, (H + I) * 2, 64, rec2::F_UNITS) &&
+              tcg::make_map(&prm.map_y, y, H, T * B, H * 2, 64, P.NB);
+    if (h0) ok = ok && tcg::make_map(&prm.map_h0, h0, H, B, H * 2, 64, P.NB);
+    else prm.map_h0 = prm.map_y;
+    if (!ok) return LSTM_ERR_UNSUPPORTED;
+    prm.Gx = Gx; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
+    prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.R = P.R; prm.G = P.G; prm.kcc = P.kcc;
+    prm.has_h0 = h0 != nullptr;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_fwd2(prm, P, s);
+    if (e == cudaErrorInvalidConfiguration || e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+// a3 (+ a5) on the cluster kernel.  W_h^T is written to the workspace first;
+// db is the sum of the batch groups' partials.
+int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
+                       const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
+                       const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
+                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I, G4 = 4 * H;
+    {
+        dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
+        rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)I);
+        note_launch();
+        if (cudaGetLastError() != cudaSuccess) return LSTM_ERR_CUDA;
+    }
+    rec2::Bwd2Params prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!tcg::make_map(&prm.map_wt, WT, G4, H, G4 * 2, 64, rec2::B_UNITS) ||
+        !tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB))
+        return LSTM_ERR_UNSUPPORTED;
+    prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
+    prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
+    prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
+    prm.kcc = P.kcc; prm.stages = P.stages;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_cluster(rec2::bwd2_kernel, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
+                                         rec2::B_THREADS);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    if (e != cudaSuccess) return LSTM_ERR_CUDA;
+    simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ forward pass
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
@@ -427,14 +662,24 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         }
         // a2: the recurrence
         prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
+        Rec2Plan plan2;
+        if (plan_fwd2(d, plan2)) {
+            const int rc = tc_fwd_recurrence2(d, plan2, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
+                                              (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells,
+                                              (Ctrl *)ws, s);
+            g_last_fwd_path = 2;
+            if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
+        }
         RecPlan plan;
         if (plan_fwd_recur(d, plan)) {
+            g_last_fwd_path = 1;
             // persistent tcgen05 kernel: all T steps in one launch; it writes hT and cT
             return tc_fwd_recurrence(d, plan, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
                                      (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells, (Ctrl *)ws,
                                      s);
         }
         // otherwise one fused GEMM + gate/cell/hidden epilogue launch per step
+        g_last_fwd_path = 0;
         for (int t = 0; t < T_; ++t) {
             const T *hp = t > 0 ? y + (long long)(t - 1) * BH : h0;
             const float *cp = t > 0 ? cells + (long long)(t - 1) * BH : c0;
@@ -484,13 +729,25 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     }
 
     RecPlan plan;
-    if (plan_bwd_recur(d, plan)) {
+    Rec2Plan plan2;
+    const bool v2 = plan_bwd2(d, plan2);
+    if (v2 || plan_bwd_recur(d, plan)) {
         {   // a3 + a5: persistent tcgen05 recurrence with db fused
             prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
-            const int rc = tc_bwd_recurrence(
+            int rc = LSTM_ERR_NOT_CORESIDENT;
+            g_last_bwd_path = 2;
+            if (v2)
+                rc = tc_bwd_recurrence2(d, plan2, (const bf16 *)dy, (const bf16 *)dhT, dcT,
+                                        (const bf16 *)W, c0, (const bf16 *)gates, cells,
+                                        (bf16 *)dG, (bf16 *)(ws + L.wt),
+                                        (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
+            if (rc == LSTM_ERR_NOT_CORESIDENT && plan_bwd_recur(d, plan)) {
+                g_last_bwd_path = 1;
+                rc = tc_bwd_recurrence(
                 d, plan, (const bf16 *)dy, (const bf16 *)dhT, dcT, (const bf16 *)W, c0,
                 (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
                 (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
+            }
             if (rc != LSTM_OK) return rc;
         }
         if (tc_gemm_ok(d)) {
@@ -515,6 +772,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     }
 
     // a3: reverse-time recursion, steps 1-3 and 5 fused with delta h = W_h^T dG_{t+1}
+    g_last_bwd_path = 0;
     {
     prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
     for (int t = T_ - 1; t >= 0; --t) {
@@ -759,6 +1017,12 @@ int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_m
 int lstm_test_set_wait_fault(int skip_cta, long long wait_ns) {
     g_fault_skip_cta = skip_cta;
     g_wait_ns = wait_ns > 0 ? (unsigned long long)wait_ns : 2000000000ull;
+    return LSTM_OK;
+}
+
+int lstm_test_last_paths(int *fwd_path, int *bwd_path) {
+    if (fwd_path) *fwd_path = g_last_fwd_path;
+    if (bwd_path) *bwd_path = g_last_bwd_path;
     return LSTM_OK;
 }
 

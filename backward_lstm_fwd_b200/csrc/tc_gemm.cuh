@@ -22,6 +22,7 @@ namespace lstm {
 namespace tcg {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+static_assert(BK == 64, "the MMA issuer unrolls four K=16 steps per stage");
 constexpr int A_BYTES = BM * BK * 2;          // 16 KB
 constexpr int B_BYTES = BN * BK * 2;          // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -165,9 +166,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
+        // The issuing thread is the critical path, so every descriptor is a
+        // base plus integer offsets: the start-address field is (addr >> 4) in
+        // the low 14 bits, and no offset here carries out of it (smem < 256 KB).
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, acc = 0, aphase = 0;
             bool ok = true;
+            const uint64_t a_lo0 = tc::smem_u32(sA) >> 4, b_lo0 = tc::smem_u32(sB) >> 4;
             for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
                 int mt, nt;
                 const Problem &P = p.prob[locate(p, tile, mt, nt)];
@@ -175,23 +180,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
                 tc::tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, P.a_mn_major, P.b_mn_major);
+                const uint64_t a_hi = operand_desc(0, P.a_mn_major, 0);  // address field 0
+                const uint64_t b_hi = operand_desc(0, P.b_mn_major, 0);
+                const uint32_t a_k = P.a_mn_major ? 2048 >> 4 : 32 >> 4;  // per K=16 step
+                const uint32_t b_k = P.b_mn_major ? 2048 >> 4 : 32 >> 4;
                 uint32_t accumulate = 0;
                 for (int sg = 0; ok && sg < P.nseg; ++sg) {
-                    const Seg &S = P.seg[sg];
-                    for (int kb = 0; kb < S.nkb; ++kb) {
+                    const int nkb = P.seg[sg].nkb;
+                    for (int kb = 0; kb < nkb; ++kb) {
                         if (!tc::mbar_wait(&full[stage], phase, p.ctrl, abort_flag, 0x103)) {
                             ok = false;
                             break;
                         }
                         tc::tc_fence_after();
-                        const uint32_t a_addr = tc::smem_u32(sA + stage * A_BYTES);
-                        const uint32_t b_addr = tc::smem_u32(sB + stage * B_BYTES);
-#pragma unroll
-                        for (int k = 0; k < BK / 16; ++k) {
-                            tc::mma_bf16(d, operand_desc(a_addr, P.a_mn_major, k),
-                                         operand_desc(b_addr, P.b_mn_major, k), idesc, accumulate);
-                            accumulate = 1;
-                        }
+                        const uint64_t ad = a_hi | (a_lo0 + stage * (A_BYTES >> 4));
+                        const uint64_t bd = b_hi | (b_lo0 + stage * (B_BYTES >> 4));
+                        tc::mma_bf16(d, ad, bd, idesc, accumulate);
+                        tc::mma_bf16(d, ad + a_k, bd + b_k, idesc, 1);
+                        tc::mma_bf16(d, ad + 2 * a_k, bd + 2 * b_k, idesc, 1);
+                        tc::mma_bf16(d, ad + 3 * a_k, bd + 3 * b_k, idesc, 1);
+                        accumulate = 1;
                         tc::mma_commit(&empty[stage]);
                         if (++stage == STAGES) stage = 0, phase ^= 1;
                     }

@@ -64,6 +64,22 @@ __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// AND of `v` over the N epilogue threads (named barrier 2), so that every
+// epilogue thread takes the same branch after a bounded wait.
+template <int N>
+__device__ __forceinline__ bool epi_vote_all_n(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 2, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(N)
+        : "memory");
+    return r != 0;
+}
+
 // AND of `v` over the 128 epilogue threads (named barrier 2), so that every
 // epilogue thread takes the same branch after a bounded wait -- no thread is
 // left alone at a later barrier or warp-synchronous TMEM load.
@@ -79,6 +95,16 @@ __device__ __forceinline__ bool epi_vote_all(bool v) {
         : "memory");
     return r != 0;
 }
+
+// Activations of the bf16 recurrent kernels: the hardware tanh approximation
+// (MUFU, about 2^-11 relative error, well below bf16's 2^-8 storage step) and
+// the logistic function through the identity sigma(x) = (1 + tanh(x / 2)) / 2.
+__device__ __forceinline__ float tanh_fast(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sigmoid_fast(float x) { return fmaf(0.5f, tanh_fast(0.5f * x), 0.5f); }
 
 // Wait until *ctr >= target (acquire).  Bounded by limit_ns of %globaltimer;
 // on time-out record LSTM_ERR_TIMEOUT with `site` and raise the abort flag.
@@ -100,14 +126,20 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *ctr, unsigned i
 }
 
 // Shared-memory plan (bytes from the 1024-aligned base).
+// The gate-exchange buffer (4 x NB x 16 fp32) aliases the ring: the ring is
+// idle between the last MMA of a step and the group barrier of the next one,
+// which is exactly when the epilogue uses the buffer.
+constexpr int MAX_STAGES = 16;
+constexpr int BAR_BYTES = 512;
 struct FwdSmem {
     int w, ring, xbuf, bars, total;
     __host__ __device__ FwdSmem(int kch, int stages, int NB) {
         w = 0;
         ring = kch * KCH_BYTES;
-        xbuf = ring + stages * NB * 128;
-        bars = xbuf + 4 * NB * UNITS * 4;
-        total = bars + 256;
+        xbuf = ring;
+        const int ring_bytes = stages * NB * 128, x_bytes = 4 * NB * UNITS * 4;
+        bars = ring + (ring_bytes > x_bytes ? ring_bytes : x_bytes);
+        total = bars + BAR_BYTES;
     }
 };
 
@@ -122,11 +154,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
     float *xbuf = (float *)(smem + L.xbuf);
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *full = bars;                  // [stages]
-    uint64_t *empty = bars + 8;             // [stages]
-    uint64_t *w_full = bars + 16;
-    uint64_t *mma_done = bars + 17;         // [2]
-    uint32_t *tmem_slot = (uint32_t *)(bars + 20);
-    volatile int *abort_flag = (volatile int *)(bars + 21);
+    uint64_t *empty = bars + MAX_STAGES;    // [stages]
+    uint64_t *w_full = bars + 2 * MAX_STAGES;
+    uint64_t *mma_done = w_full + 1;        // [2]
+    uint32_t *tmem_slot = (uint32_t *)(mma_done + 3);
+    volatile int *abort_flag = (volatile int *)(mma_done + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int s = blockIdx.x % p.S, gi = blockIdx.x / p.S;
@@ -134,6 +166,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
     const int H = p.H, B = p.B;
     unsigned int *ctr = &p.ctrl->bar[gi];
     constexpr uint32_t TMEM_COLS = (2 * NB < 32) ? 32 : 2 * NB;
+    // every CTA of a group walks the K chunks from a different start, so that
+    // concurrent TMA requests spread over the L2 slices
+    const int rot = (s * 5 + gi * 3) % p.kch;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) {
@@ -180,7 +215,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
                 const CUtensorMap *m = t > 0 ? &p.map_y : &p.map_h0;
                 const int row0 = t > 0 ? (t - 1) * B + b0 : b0;
                 bool ok = true;
-                for (int kc = 0; kc < p.kch; ++kc) {
+                int kc = rot;
+                for (int ic = 0; ic < p.kch; ++ic, kc = (kc + 1 == p.kch) ? 0 : kc + 1) {
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, p.ctrl, abort_flag, 0x202,
                                        p.wait_ns)) {
                         ok = false;
@@ -207,8 +243,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // descriptors = base + integer offsets (see tc_gemm.cuh); the issuing
+            // thread is on every step's critical path
             uint32_t stage = 0, phase = 0;
             const uint32_t idesc = tc::idesc_bf16_f32(MROWS, NB, 0, 0);
+            const uint64_t hi = tc::smem_desc_sw128(0, 16, 1024);
+            const uint64_t w_lo0 = tc::smem_u32(sW) >> 4, r_lo0 = tc::smem_u32(ring) >> 4;
+            constexpr uint32_t WSTEP = KCH_BYTES >> 4, RSTEP = (NB * 128) >> 4;
             bool ok = tc::mbar_wait(w_full, 0, p.ctrl, abort_flag, 0x203, p.wait_ns);
             for (int t = 0; ok && t < p.T; ++t) {
                 const int acc = t & 1;
@@ -217,19 +258,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
                     continue;
                 }
                 const uint32_t d = tmem_base + acc * NB;
-                for (int kc = 0; kc < p.kch; ++kc) {
+                int kc = rot;
+                for (int ic = 0; ic < p.kch; ++ic, kc = (kc + 1 == p.kch) ? 0 : kc + 1) {
                     if (!tc::mbar_wait(&full[stage], phase, p.ctrl, abort_flag, 0x204, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
-                    const uint32_t a = tc::smem_u32(sW + kc * KCH_BYTES);
-                    const uint32_t b = tc::smem_u32(ring + stage * NB * 128);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(d, tc::smem_desc_sw128(a + 32 * k, 16, 1024),
-                                     tc::smem_desc_sw128(b + 32 * k, 16, 1024), idesc,
-                                     (kc | k) != 0);
+                    const uint64_t ad = hi | (w_lo0 + kc * WSTEP);
+                    const uint64_t bd = hi | (r_lo0 + stage * RSTEP);
+                    tc::mma_bf16(d, ad, bd, idesc, ic != 0);
+                    tc::mma_bf16(d, ad + 2, bd + 2, idesc, 1);
+                    tc::mma_bf16(d, ad + 4, bd + 4, idesc, 1);
+                    tc::mma_bf16(d, ad + 6, bd + 6, idesc, 1);
                     tc::mma_commit(&empty[stage]);
                     if (++stage == (uint32_t)p.stages) stage = 0, phase ^= 1;
                 }
@@ -266,16 +307,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
             if (!epi_vote_all(w)) break;
             tc::tc_fence_after();
             const bool zero = (t == 0 && !p.has_h0);
-            // TMEM rows of this warp: gate q, unit = lane (lanes 0..15)
+            // TMEM rows of this warp: gate q, unit = lane (lanes 0..15); all
+            // loads in flight before one wait
+            constexpr int CB = NB < 64 ? NB : (NB >= 128 ? 32 : 64);  // columns per wait
 #pragma unroll
-            for (int c0 = 0; c0 < NB; c0 += 16) {
-                uint32_t r[16];
-                tc::tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + c0, r);
+            for (int cb = 0; cb < NB; cb += CB) {
+                uint32_t r[CB / 16][16];
+#pragma unroll
+                for (int c = 0; c < CB / 16; ++c)
+                    tc::tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + cb + 16 * c,
+                                  r[c]);
                 tc::tmem_ld_wait();
                 if (lane < UNITS) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        xbuf[(q * NB + c0 + i) * UNITS + lane] = zero ? 0.f : __uint_as_float(r[i]);
+                    for (int c = 0; c < CB / 16; ++c)
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            xbuf[(q * NB + cb + 16 * c + i) * UNITS + lane] =
+                                zero ? 0.f : __uint_as_float(r[c][i]);
                 }
             }
             tc::tc_fence_before();
@@ -286,12 +335,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
 #pragma unroll
             for (int k = 0; k < NK; ++k) {
                 const int n = nq + 8 * k, b = b0 + n;
-                const float ig = sigmoidf_(xbuf[(0 * NB + n) * UNITS + u] + gx[0][k]);
-                const float fg = sigmoidf_(xbuf[(1 * NB + n) * UNITS + u] + gx[1][k]);
-                const float gg = tanhf_(xbuf[(2 * NB + n) * UNITS + u] + gx[2][k]);
-                const float og = sigmoidf_(xbuf[(3 * NB + n) * UNITS + u] + gx[3][k]);
+                const float ig = sigmoid_fast(xbuf[(0 * NB + n) * UNITS + u] + gx[0][k]);
+                const float fg = sigmoid_fast(xbuf[(1 * NB + n) * UNITS + u] + gx[1][k]);
+                const float gg = tanh_fast(xbuf[(2 * NB + n) * UNITS + u] + gx[2][k]);
+                const float og = sigmoid_fast(xbuf[(3 * NB + n) * UNITS + u] + gx[3][k]);
                 c[k] = fg * c[k] + ig * gg;
-                const float h = og * tanhf_(c[k]);
+                const float h = og * tanh_fast(c[k]);
                 if (b < B) {
                     const long long o = (long long)b * H + j;
                     yt[o] = __float2bfloat16_rn(h);
@@ -311,8 +360,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
             tc::fence_proxy_async_global();  // y[t] is read next by TMA (async proxy)
             named_bar(1, EPI_THREADS);       // all of y[t] stored; xbuf free again
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) {
-                __threadfence();
-                red_release_add(ctr, 1u);
+                red_release_add(ctr, 1u);  // release: the step's stores, ordered by bar.sync
             }
         }
     }
@@ -373,7 +421,7 @@ struct BwdSmem {
         wt = 0;
         ring = kch4 * WT_CHUNK_BYTES;
         bars = ring + stages * BWD_STAGE_BYTES;
-        total = bars + 256;
+        total = bars + BAR_BYTES;
     }
 };
 
@@ -402,11 +450,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
     uint8_t *ring = smem + L.ring;
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *full = bars;
-    uint64_t *empty = bars + 8;
-    uint64_t *w_full = bars + 16;
-    uint64_t *mma_done = bars + 17;
-    uint32_t *tmem_slot = (uint32_t *)(bars + 20);
-    volatile int *abort_flag = (volatile int *)(bars + 21);
+    uint64_t *empty = bars + MAX_STAGES;
+    uint64_t *w_full = bars + 2 * MAX_STAGES;
+    uint64_t *mma_done = w_full + 1;
+    uint32_t *tmem_slot = (uint32_t *)(mma_done + 3);
+    volatile int *abort_flag = (volatile int *)(mma_done + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int s = blockIdx.x % p.S, gi = blockIdx.x / p.S;
@@ -414,6 +462,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
     const int H = p.H, B = p.B, T = p.T, NB = p.NB;
     unsigned int *ctr = &p.ctrl->bar[gi];
     constexpr uint32_t TMEM_COLS = 32;  // two 16-column accumulators
+    const int rot = (s * 5 + gi * 3) % p.kch4;  // spread concurrent TMA requests over L2
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) {
@@ -450,7 +499,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
                 }
                 tc::fence_proxy_async_global();
                 const int row0 = (T - i) * B + b0;
-                for (int kc = 0; kc < p.kch4; ++kc) {
+                int kc = rot;
+                for (int ic = 0; ic < p.kch4; ++ic, kc = (kc + 1 == p.kch4) ? 0 : kc + 1) {
                     if (!tc::mbar_wait(&empty[stage], phase ^ 1, p.ctrl, abort_flag, 0x302,
                                        p.wait_ns)) {
                         aborted = true;
@@ -475,22 +525,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             const uint32_t idesc = tc::idesc_bf16_f32(64, UNITS, 0, 0);
+            const uint64_t hi = tc::smem_desc_sw128(0, 16, 1024);
+            const uint64_t r_lo0 = tc::smem_u32(ring) >> 4, w_lo0 = tc::smem_u32(sWT) >> 4;
+            constexpr uint32_t RSTEP = BWD_STAGE_BYTES >> 4, WSTEP = WT_CHUNK_BYTES >> 4;
             bool ok = tc::mbar_wait(w_full, 0, p.ctrl, abort_flag, 0x303, p.wait_ns);
             for (int i = 1; ok && i <= T; ++i) {
                 const uint32_t d = tmem_base + (i & 1) * UNITS;
-                for (int kc = 0; kc < p.kch4; ++kc) {
+                int kc = rot;
+                for (int ic = 0; ic < p.kch4; ++ic, kc = (kc + 1 == p.kch4) ? 0 : kc + 1) {
                     if (!tc::mbar_wait(&full[stage], phase, p.ctrl, abort_flag, 0x304, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
-                    const uint32_t a = tc::smem_u32(ring + stage * BWD_STAGE_BYTES);
-                    const uint32_t b = tc::smem_u32(sWT + kc * WT_CHUNK_BYTES);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        tc::mma_bf16(d, tc::smem_desc_sw128(a + 32 * k, 16, 1024),
-                                     tc::smem_desc_sw128(b + 32 * k, 16, 1024), idesc,
-                                     (kc | k) != 0);
+                    const uint64_t ad = hi | (r_lo0 + stage * RSTEP);
+                    const uint64_t bd = hi | (w_lo0 + kc * WSTEP);
+                    tc::mma_bf16(d, ad, bd, idesc, ic != 0);
+                    tc::mma_bf16(d, ad + 2, bd + 2, idesc, 1);
+                    tc::mma_bf16(d, ad + 4, bd + 4, idesc, 1);
+                    tc::mma_bf16(d, ad + 6, bd + 6, idesc, 1);
                     tc::mma_commit(&empty[stage]);
                     if (++stage == (uint32_t)p.stages) stage = 0, phase ^= 1;
                 }
@@ -596,7 +649,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
             for (int u = 0; u < 8; ++u) {
                 const float ig = gv[0][u], fg = gv[1][u], gg = gv[2][u], og = gv[3][u];
                 const float dh = dyv[u] + dhr[u];                       // step 1
-                const float tc_ = tanhf_(ct[u]);
+                const float tc_ = tanh_fast(ct[u]);
                 const float dcv = dh * og * (1.f - tc_ * tc_) + dc[u];  // step 2
                 dO[u] = dh * tc_ * og * (1.f - og);                     // step 3
                 dGg[u] = dcv * ig * (1.f - gg * gg);
@@ -627,8 +680,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
             tc::fence_proxy_async_global();  // dG_t is read next by TMA
             named_bar(1, EPI_THREADS);
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) {
-                __threadfence();
-                red_release_add(ctr, 1u);
+                red_release_add(ctr, 1u);  // release: the step's stores, ordered by bar.sync
             }
             if (t > 0) load_step(t - 1);
         }

@@ -2,7 +2,8 @@
 CTA 0 never signals its step barrier must give up after its bounded wait,
 record LSTM_ERR_TIMEOUT in the workspace status word (read by lstm_status), and
 leave the context usable -- the next normal call succeeds and matches the
-oracle."""
+oracle.  Covered for the K-resident kernels (H = 64) and the cluster kernels
+(H = 256: forward clusters of 4, backward clusters of 8)."""
 import pytest
 import torch
 
@@ -14,19 +15,25 @@ from tests.parity_util import assert_within, compare, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 
-def test_missing_arrival_times_out_and_recovers(cuda_device):
+@pytest.mark.parametrize("H", [64, 256])
+def test_missing_arrival_times_out_and_recovers(H, cuda_device):
     lbuild.build()
-    w = synth.custom(6, 32, 64, 64, "bf16", seed=11)
+    w = synth.custom(6, 32, 64, H, "bf16", seed=11)
     inp = {k: v.to(cuda_device) for k, v in synth.make_inputs(w).items()}
-    T, B, I, H = w.T, w.B, w.I, w.H
+    T, B, I = w.T, w.B, w.I
     st = L.State(T, B, I, H, torch.bfloat16, cuda_device)
-    ws = L.empty_workspace(L.fwd_workspace_size(st.dims), cuda_device)
+    gr = L.Grads(T, B, I, H, cuda_device)
+    wsf = L.empty_workspace(L.fwd_workspace_size(st.dims), cuda_device)
+    wsb = L.empty_workspace(L.bwd_workspace_size(st.dims), cuda_device)
     try:
-        L.test_set_wait_fault(0, 50_000_000)  # 50 ms
+        L.test_set_wait_fault(0, 50_000_000)  # CTA 0 never arrives; waits give up after 50 ms
         L.lstm_fwd(st.dims, inp["x"], inp["W"], inp["b"], inp["h0"], inp["c0"], st.y, st.hT,
-                   st.cT, st.gates, st.cells, ws)
-        assert L.lstm_status(ws) == L.LSTM_ERR_TIMEOUT
-        assert L.lstm_status(ws) == L.LSTM_OK  # reading clears the word
+                   st.cT, st.gates, st.cells, wsf)
+        assert L.lstm_status(wsf) == L.LSTM_ERR_TIMEOUT
+        assert L.lstm_status(wsf) == L.LSTM_OK  # reading clears the word
+        L.lstm_bwd(st.dims, inp["dy"], inp["dhT"], inp["dcT"], inp["x"], inp["W"], inp["h0"],
+                   inp["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0, wsb)
+        assert L.lstm_status(wsb) == L.LSTM_ERR_TIMEOUT
     finally:
         L.test_set_wait_fault(-1, 0)
     # the context is still usable and the next call is correct

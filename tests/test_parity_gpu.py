@@ -8,6 +8,7 @@ import numpy as np
 import pytest
 import torch
 
+from backward_lstm_fwd_b200 import binding as L
 from backward_lstm_fwd_b200 import synth
 from tests.parity_util import (OUTS, TOL, assert_within, compare, mask_upstream, rel_err,
                                run_gpu, run_oracle)
@@ -22,11 +23,19 @@ SAMPLED = {"lstm_T256_B128_I1024_H1024_bf16": [0, 37, 101, 127],
            "lstm_T1024_B16_I256_H1024_bf16": [0, 11]}
 
 
+# recurrent kernel each workload must run on (see lstm_test_last_paths)
+EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (0, 0), "lstm_T64_B32_I256_H256_fp32": (0, 0),
+                  "lstm_T128_B64_I512_H512_bf16": (2, 2),
+                  "lstm_T256_B128_I1024_H1024_bf16": (2, 2),
+                  "lstm_T1024_B16_I256_H1024_bf16": (2, 2)}
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_workload_full(name, cuda_device):
     w = synth.WORKLOADS[name]
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
+    assert L.test_last_paths() == EXPECTED_PATHS[name]
     ref = run_oracle(inp)
     errs = compare(gpu, ref, w.dtype, OUTS + ("gates", "cells"))
     assert_within(errs, w.dtype, name)
@@ -38,6 +47,7 @@ def test_workload_sampled(name, cuda_device):
     idx = SAMPLED[name]
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
+    assert L.test_last_paths() == EXPECTED_PATHS[name]
     ref = run_oracle(synth.select_sequences(inp, idx))
     errs = compare(gpu, ref, w.dtype, ("y", "hT", "cT", "dx", "dh0", "dc0"), idx=idx)
     assert_within(errs, w.dtype, name + " per-sequence")
