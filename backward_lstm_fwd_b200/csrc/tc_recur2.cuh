@@ -59,6 +59,11 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
     }
 }
 
+// Receive buffers are chunk-major: [source][chunk of VW columns][row][VW].
+// Consecutive rows (= consecutive lanes) are consecutive VW-float vectors, so
+// one warp-wide vector store moves a contiguous 32 * VW * 4 bytes and the
+// matching vector reads are bank-conflict free.
+
 // =========================================================================
 // forward
 // =========================================================================
@@ -100,13 +105,14 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
     constexpr int NBc = NB / KS;       // batch columns finalised by this CTA
     constexpr int NBh = NBc / 2;       // columns each of the two warps of a quarter moves
     constexpr int NP = (NBc + 7) / 8;  // (unit, batch) pairs per epilogue thread
+    constexpr int VW = NBh >= 4 ? 4 : 2;  // floats per DSMEM store / receive chunk
     static_assert(NBc >= 4 && NBc % 4 == 0 && NBc <= 32, "columns per CTA");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Fwd2Smem L(p.kcc, NB, KS);
     uint8_t *sW = smem + L.w;
     uint8_t *ring = smem + L.ring;
-    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][NBc][128 rows]
+    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][NBc/VW chunks][128 rows][VW]
     float *xbuf = (float *)(smem + L.xbuf);  // [4 gates][NBc][32 units]
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *full = bars;
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
 #pragma unroll
         for (int d = 0; d < KS; ++d) {
             const int slot = ((int)kpart < d) ? (int)kpart : (int)kpart - 1;
-            peer_recv[d] = tc::map_rank(tc::smem_u32(recv + slot * NBc * F_ROWS), d);
+            peer_recv[d] = tc::map_rank(tc::smem_u32(recv + slot * F_ROWS * NBc), d);
             peer_bar[d] = tc::map_rank(tc::smem_u32(recv_full), d);
         }
         // pointwise pairs of this thread: pair index et + 256 k -> unit, column
@@ -280,10 +286,18 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                         for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(v[n]);
                     } else {
 #pragma unroll
-                        for (int n = 0; n < NBh; ++n)
-                            tc::st_cluster_f32(
-                                peer_recv[d] + (uint32_t)(((hh * NBh + n) * F_ROWS + mrow) * 4),
-                                __uint_as_float(v[n]));
+                        for (int k = 0; k < NBh / VW; ++k) {
+                            const int ch = hh * (NBh / VW) + k;
+                            const uint32_t a = peer_recv[d] + (uint32_t)(((ch * F_ROWS + mrow) * VW) * 4);
+                            if constexpr (VW == 4)
+                                tc::st_cluster_v4(a, __uint_as_float(v[4 * k]),
+                                                  __uint_as_float(v[4 * k + 1]),
+                                                  __uint_as_float(v[4 * k + 2]),
+                                                  __uint_as_float(v[4 * k + 3]));
+                            else
+                                tc::st_cluster_v2(a, __uint_as_float(v[2 * k]),
+                                                  __uint_as_float(v[2 * k + 1]));
+                        }
                     }
                 }
                 tc::tc_fence_before();
@@ -299,13 +313,26 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                     rph ^= 1;
                 }
 #pragma unroll
-                for (int n = 0; n < NBh; ++n) {
-                    const int col = hh * NBh + n;
-                    float sum = own[n];
+                for (int sl = 0; sl < KS - 1; ++sl) {
+                    const float *src = recv + sl * F_ROWS * NBc;
 #pragma unroll
-                    for (int sl = 0; sl < KS - 1; ++sl) sum += recv[(sl * NBc + col) * F_ROWS + mrow];
-                    xbuf[(q * NBc + col) * F_UNITS + lane] = sum;
+                    for (int k = 0; k < NBh / VW; ++k) {
+                        const int ch = hh * (NBh / VW) + k;
+                        if constexpr (VW == 4) {
+                            const float4 x = *reinterpret_cast<const float4 *>(src + (ch * F_ROWS + mrow) * 4);
+                            own[4 * k] += x.x;
+                            own[4 * k + 1] += x.y;
+                            own[4 * k + 2] += x.z;
+                            own[4 * k + 3] += x.w;
+                        } else {
+                            const float2 x = *reinterpret_cast<const float2 *>(src + (ch * F_ROWS + mrow) * 2);
+                            own[2 * k] += x.x;
+                            own[2 * k + 1] += x.y;
+                        }
+                    }
                 }
+#pragma unroll
+                for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
             }
             rec::named_bar(1, F_EPI_THREADS);
             __nv_bfloat16 *yt = p.y + (long long)t * B * H;
@@ -397,7 +424,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
     const Bwd2Smem L(p.kcc, p.stages);
     uint8_t *sWT = smem + L.wt;
     uint8_t *ring = smem + L.ring;
-    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][UPC units][128 rows]
+    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][4 chunks][128 rows][4 units]
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *full = bars;
     uint64_t *empty = bars + MAX_KCC;
@@ -516,13 +543,13 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
         const int uo = 8 * hh;               // offset of this thread's units within the 16
         const int jb = j0 + (int)kpart * UPC + uo;
         const long long G4 = 4LL * H;
-        uint32_t peer_recv[KS], peer_bar[KS];
-#pragma unroll
-        for (int d = 0; d < KS; ++d) {
+        // DSMEM addresses in partner d: this CTA's slot of its receive buffer,
+        // and its receive barrier (mapa is cheap; not kept in registers)
+        const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
+        auto peer_recv = [&](int d) {
             const int slot = ((int)kpart < d) ? (int)kpart : (int)kpart - 1;
-            peer_recv[d] = tc::map_rank(tc::smem_u32(recv + slot * UPC * B_MROWS), d);
-            peer_bar[d] = tc::map_rank(tc::smem_u32(recv_full), d);
-        }
+            return tc::map_rank(recv_lo + (uint32_t)(slot * B_MROWS * UPC * 4), (uint32_t)d);
+        };
         float dc[UPT], dbacc[4][UPT];
         float gv[4][UPT], ct[UPT], cp[UPT], dyv[UPT];
 #pragma unroll
@@ -588,9 +615,13 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                     for (int u = 0; u < UPT; ++u) dh[u] = __uint_as_float(v[u]);
                 } else {
 #pragma unroll
-                    for (int u = 0; u < UPT; ++u)
-                        tc::st_cluster_f32(peer_recv[d] + (uint32_t)(((uo + u) * B_MROWS + m) * 4),
-                                           __uint_as_float(v[u]));
+                    for (int k = 0; k < 2; ++k) {  // units uo + 4k .. +3: chunk uo/4 + k
+                        const int ch = uo / 4 + k;
+                        tc::st_cluster_v4(peer_recv(d) + (uint32_t)(((ch * B_MROWS + m) * 4) * 4),
+                                          __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                          __uint_as_float(v[4 * k + 2]),
+                                          __uint_as_float(v[4 * k + 3]));
+                    }
                 }
             }
             tc::tc_fence_before();
@@ -598,15 +629,23 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
             if (lane == 0)
 #pragma unroll
                 for (int d = 0; d < KS; ++d)
-                    if (d != (int)kpart) tc::mbar_arrive_remote(peer_bar[d]);
+                    if (d != (int)kpart) tc::mbar_arrive_remote(tc::map_rank(recvbar_lo, (uint32_t)d));
             const bool w2 =
                 tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x506, p.wait_ns);
             if (!rec::epi_vote_all_n<B_EPI_THREADS>(w2)) return false;
             rph ^= 1;
 #pragma unroll
-            for (int sl = 0; sl < KS - 1; ++sl)
+            for (int sl = 0; sl < KS - 1; ++sl) {
+                const float *src = recv + sl * B_MROWS * UPC;
 #pragma unroll
-                for (int u = 0; u < UPT; ++u) dh[u] += recv[(sl * UPC + uo + u) * B_MROWS + m];
+                for (int k = 0; k < 2; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(src + ((uo / 4 + k) * B_MROWS + m) * 4);
+                    dh[4 * k] += x.x;
+                    dh[4 * k + 1] += x.y;
+                    dh[4 * k + 2] += x.z;
+                    dh[4 * k + 3] += x.w;
+                }
+            }
             // partners refill recv only after the next group barrier, which
             // needs this CTA's next arrival: these reads are safe
             return true;
