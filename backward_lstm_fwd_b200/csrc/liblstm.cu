@@ -543,10 +543,18 @@ cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t s
     at[1].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, kern, prm);
-    note_launch();
-    if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) return e;
-    cudaGetLastError();
+    // LSTM_LAUNCH_NONCOOP=1 (profiling aid: some profilers cannot replay a
+    // cooperative cluster launch) skips straight to the occupancy-checked
+    // cluster launch below.
+    const char *nc = getenv("LSTM_LAUNCH_NONCOOP");
+    if (!(nc && nc[0] == '1')) {
+        e = cudaLaunchKernelEx(&cfg, kern, prm);
+        if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) {
+            note_launch();
+            return e;
+        }
+        cudaGetLastError();
+    }
     cfg.numAttrs = 1;  // cluster launch without the cooperative attribute
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess ||
@@ -554,6 +562,7 @@ cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t s
         cudaGetLastError();
         return cudaErrorCooperativeLaunchTooLarge;
     }
+    note_launch();
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 

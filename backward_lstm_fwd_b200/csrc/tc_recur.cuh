@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
                         aborted = true;
                         break;
                     }
+                    // the group's generic-proxy stores were released to this
+                    // thread's acquire; order the TMA (async-proxy) reads after it
                     tc::fence_proxy_async_global();
                 } else if (!p.has_h0) {
                     continue;  // h_{-1} = 0: no MMA at t = 0
@@ -357,7 +359,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fwd_kernel(const __grid_consta
                 }
             }
             if (t + 1 < p.T) load_gx(t + 1);
-            tc::fence_proxy_async_global();  // y[t] is read next by TMA (async proxy)
             named_bar(1, EPI_THREADS);       // all of y[t] stored; xbuf free again
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) {
                 red_release_add(ctr, 1u);  // release: the step's stores, ordered by bar.sync
@@ -497,6 +498,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
                     aborted = true;
                     break;
                 }
+                // acquire above, then the proxy fence: the TMA reads below see
+                // every dG store the group released
                 tc::fence_proxy_async_global();
                 const int row0 = (T - i) * B + b0;
                 int kc = rot;
@@ -677,7 +680,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_kernel(const __grid_consta
                     dbacc[3][u] += ro[u];
                 }
             }
-            tc::fence_proxy_async_global();  // dG_t is read next by TMA
             named_bar(1, EPI_THREADS);
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) {
                 red_release_add(ctr, 1u);  // release: the step's stores, ordered by bar.sync

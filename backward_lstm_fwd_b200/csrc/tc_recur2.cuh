@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                         aborted = true;
                         break;
                     }
+                    // the group's generic-proxy stores were released to this
+                    // thread's acquire; order the TMA (async-proxy) reads after it
                     tc::fence_proxy_async_global();
                 } else if (!p.has_h0) {
                     continue;
@@ -365,7 +367,6 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                 }
             }
             if (t + 1 < p.T) load_gx(t + 1);
-            tc::fence_proxy_async_global();    // y[t] is read next by TMA
             rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
         }
@@ -482,6 +483,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                     aborted = true;
                     break;
                 }
+                // acquire above, then the proxy fence: the TMA reads below see
+                // every dG store the group released
                 tc::fence_proxy_async_global();
                 const int row0 = (T - i) * B + b0;
                 for (int c = 0; c < kcc; ++c) {
@@ -702,7 +705,6 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                     dbacc[3][u] += ro[u];
                 }
             }
-            tc::fence_proxy_async_global();  // dG_t is read next by TMA
             rec::named_bar(1, B_EPI_THREADS);
             if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
             if (t > 0) load_step(t - 1);

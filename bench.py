@@ -49,6 +49,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def measured_traffic(phase: str, workload: str):
+    """DRAM bytes per launch of a phase's kernel from the committed ncu record
+    (profiles/traffic.json), or None when there is none for this workload or
+    the kernel source changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(phase)
+        if not rec or rec.get("workload") != workload or not rec.get("source_sha256"):
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return float(rec["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 def phase_work(w: synth.Workload):
     """Algorithmic work per phase: FLOPs for the contractions (2 * M * N * K of
     the products the method defines), bytes for the db column reduction."""
@@ -284,7 +302,7 @@ def run_ours(args, w, rank, world, local_rank):
         achieved = amount / (dom_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None}
+                "frac": achieved / peak, "traffic": measured_traffic(dom, w.name)}
     else:
         achieved = amount / (dom_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
@@ -328,8 +346,14 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override T (profiling aid: same per-step shape, fewer steps)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.seq_len is not None:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_T{args.seq_len}", T=args.seq_len,
+                                dy_last=None if w.dy_last is None else min(w.dy_last, args.seq_len))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
