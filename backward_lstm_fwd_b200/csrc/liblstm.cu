@@ -498,9 +498,12 @@ bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
     if (P.kcc < 1 || P.kcc > rec2::MAX_KCC) return false;
     const size_t fixed = rec2::Bwd2Smem(P.kcc, 0).total + 1024;
     if (fixed + 2 * rec2::B_ACHUNK > kMaxSmem) return false;
-    const int stages = (int)std::min<size_t>(std::min(P.kcc, rec2::MAX_KCC),
+    // At least two stages: the ring also stages the first exchange round
+    // (B_ROUND0 partners x 8 KB = 32 KB) between an iteration's last MMA and the
+    // next iteration's loads.
+    const int stages = (int)std::min<size_t>(std::max(2, std::min(P.kcc, rec2::MAX_KCC)),
                                              (kMaxSmem - fixed) / rec2::B_ACHUNK);
-    if (stages < 2 && P.kcc > 1) return false;
+    if (stages < 2 || (size_t)stages * rec2::B_ACHUNK < rec2::B_STAGE_BYTES) return false;
     P.NB = stages;  // (ring stages; NB is reassigned to the batch rows below)
     P.smem = rec2::Bwd2Smem(P.kcc, stages).total + 1024;
     const int maxc = max_active_clusters((const void *)rec2::bwd2_kernel, rec2::B_THREADS, P.smem,

@@ -214,6 +214,24 @@ __device__ __forceinline__ void st_cluster_v2(uint32_t caddr, float a, float b) 
     asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(caddr), "f"(a), "f"(b)
                  : "memory");
 }
+// Bulk copy (TMA engine) of `bytes` from this CTA's shared memory to shared
+// memory of another CTA of the cluster; completes `bytes` transactions on the
+// destination CTA's mbarrier.  Addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_caddr, const void *src,
+                                                  uint32_t bytes, uint32_t peer_bar_caddr) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst_caddr), "r"(smem_u32(src)), "r"(bytes), "r"(peer_bar_caddr)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk copy of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Arrive on an mbarrier of another CTA of the cluster, releasing this
 // thread's earlier writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {

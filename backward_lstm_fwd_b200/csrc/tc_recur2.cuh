@@ -87,15 +87,21 @@ struct Fwd2Params {
     unsigned long long wait_ns;
 };
 
+// Partials for the other CTAs of the cluster are staged in `send` ([KS-1
+// destinations][chunks][128 rows][VW], the layout of the receive buffers) and
+// moved by bulk copies; `send` aliases the ring (idle between the step's last
+// MMA and the next step's loads) when the ring is large enough.
 struct Fwd2Smem {
-    int w, ring, recv, xbuf, bars, total;
+    int w, ring, recv, xbuf, send, bars, total;
     __host__ __device__ Fwd2Smem(int kcc, int NB, int KS) {
         const int NBc = NB / KS;
+        const int ring_bytes = kcc * NB * 128, part_bytes = (KS - 1) * NBc * F_ROWS * 4;
         w = 0;
         ring = kcc * F_WCHUNK;
-        recv = ring + kcc * NB * 128;
-        xbuf = recv + (KS - 1) * NBc * F_ROWS * 4;
-        bars = xbuf + 4 * NBc * F_UNITS * 4;
+        recv = ring + ring_bytes;
+        xbuf = recv + part_bytes;
+        send = ring_bytes >= part_bytes ? ring : xbuf + 4 * NBc * F_UNITS * 4;
+        bars = (send == ring ? xbuf + 4 * NBc * F_UNITS * 4 : send + part_bytes);
         total = bars + BAR_BYTES;
     }
 };
@@ -114,6 +120,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
     uint8_t *ring = smem + L.ring;
     float *recv = (float *)(smem + L.recv);  // [KS-1 sources][NBc/VW chunks][128 rows][VW]
     float *xbuf = (float *)(smem + L.xbuf);  // [4 gates][NBc][32 units]
+    float *send = (float *)(smem + L.send);  // [KS-1 destinations][NBc/VW][128 rows][VW]
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *full = bars;
     uint64_t *empty = bars + MAX_KCC;
@@ -142,7 +149,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
         tc::mbar_init(w_full, 1);
         tc::mbar_init(&mma_done[0], 1);
         tc::mbar_init(&mma_done[1], 1);
-        tc::mbar_init(recv_full, KS > 1 ? F_EPI_WARPS * (KS - 1) : 1);
+        tc::mbar_init(recv_full, 1);  // one local arrival (with the expected bytes) per step
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -236,14 +243,11 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
         const int hh = (warp - 2) >> 2;   // which half of each column block it moves
         const int mrow = 32 * q + lane;   // row of the partial tile: gate q, unit lane
         const int bc0 = b0 + (int)kpart * NBc;  // first batch row finalised here
-        // DSMEM addresses of this CTA's slot in each partner's receive buffer
-        uint32_t peer_recv[KS], peer_bar[KS];
-#pragma unroll
-        for (int d = 0; d < KS; ++d) {
-            const int slot = ((int)kpart < d) ? (int)kpart : (int)kpart - 1;
-            peer_recv[d] = tc::map_rank(tc::smem_u32(recv + slot * F_ROWS * NBc), d);
-            peer_bar[d] = tc::map_rank(tc::smem_u32(recv_full), d);
-        }
+        constexpr uint32_t PART_BYTES = NBc * F_ROWS * 4;  // one partner's partial tile
+        // position of destination d among this CTA's partners (its send block),
+        // and of this CTA among d's sources (its receive slot at d)
+        auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
+        auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
         // pointwise pairs of this thread: pair index et + 256 k -> unit, column
         float c[NP], gx[4][NP];
         auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
@@ -287,28 +291,40 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
 #pragma unroll
                         for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(v[n]);
                     } else {
+                        float *blk = send + dst_pos(d) * (PART_BYTES / 4);
 #pragma unroll
                         for (int k = 0; k < NBh / VW; ++k) {
                             const int ch = hh * (NBh / VW) + k;
-                            const uint32_t a = peer_recv[d] + (uint32_t)(((ch * F_ROWS + mrow) * VW) * 4);
+                            float *a = blk + (ch * F_ROWS + mrow) * VW;
                             if constexpr (VW == 4)
-                                tc::st_cluster_v4(a, __uint_as_float(v[4 * k]),
-                                                  __uint_as_float(v[4 * k + 1]),
-                                                  __uint_as_float(v[4 * k + 2]),
-                                                  __uint_as_float(v[4 * k + 3]));
+                                *reinterpret_cast<float4 *>(a) =
+                                    make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                __uint_as_float(v[4 * k + 2]),
+                                                __uint_as_float(v[4 * k + 3]));
                             else
-                                tc::st_cluster_v2(a, __uint_as_float(v[2 * k]),
-                                                  __uint_as_float(v[2 * k + 1]));
+                                *reinterpret_cast<float2 *>(a) =
+                                    make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
                         }
                     }
                 }
                 tc::tc_fence_before();
                 if (KS > 1) {
-                    __syncwarp();
-                    if (lane == 0)
+                    // staged partials -> async proxy -> one bulk copy per partner,
+                    // completing on the partner's receive barrier
+                    tc::fence_proxy_async_smem();
+                    rec::named_bar(1, F_EPI_THREADS);
+                    if (et == 0) {
+                        tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
+                        const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(recv_full);
 #pragma unroll
                         for (int d = 0; d < KS; ++d)
-                            if (d != (int)kpart) tc::mbar_arrive_remote(peer_bar[d]);
+                            if (d != (int)kpart)
+                                tc::bulk_copy_to_peer(
+                                    tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                                    send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                                    tc::map_rank(bar_lo, (uint32_t)d));
+                        tc::bulk_commit();
+                    }
                     const bool w2 = tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x406,
                                                           p.wait_ns);
                     if (!rec::epi_vote_all_n<F_EPI_THREADS>(w2)) break;
@@ -368,8 +384,14 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
             }
             if (t + 1 < p.T) load_gx(t + 1);
             rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
-            if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+            if (et == 0) {
+                // the staging block (the ring) must be read out before this
+                // CTA's arrival lets the next step's TMA refill the ring
+                if (KS > 1) tc::bulk_wait_read_all();
+                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+            }
         }
+        if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
     }
 
     tc::tc_fence_before();
@@ -393,6 +415,9 @@ constexpr int B_ACHUNK = B_MROWS * 128;    // 16 KB: 128 rows x 64 K of dG
 constexpr int B_EPI_WARPS = 8;             // two warps per TMEM lane quarter
 constexpr int B_EPI_THREADS = 32 * B_EPI_WARPS;
 constexpr int B_THREADS = 64 + B_EPI_THREADS;
+constexpr int B_ROUND0 = 4;                                   // partners in the first exchange round
+constexpr int B_PART_BYTES = B_UPC * B_MROWS * 4;             // one partner's partial: 8 KB
+constexpr int B_STAGE_BYTES = B_ROUND0 * B_PART_BYTES;        // ring bytes the exchange stages
 
 struct Bwd2Params {
     CUtensorMap map_wt;  // W_h^T [H][4H], box {64, 128}
@@ -454,7 +479,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
         tc::mbar_init(w_full, 1);
         tc::mbar_init(&mma_done[0], 1);
         tc::mbar_init(&mma_done[1], 1);
-        tc::mbar_init(recv_full, B_EPI_WARPS * (KS - 1));
+        tc::mbar_init(recv_full, 1);  // one local arrival (with the expected bytes) per step
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -546,13 +571,16 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
         const int uo = 8 * hh;               // offset of this thread's units within the 16
         const int jb = j0 + (int)kpart * UPC + uo;
         const long long G4 = 4LL * H;
-        // DSMEM addresses in partner d: this CTA's slot of its receive buffer,
-        // and its receive barrier (mapa is cheap; not kept in registers)
+        // Partials for the seven partners are staged in the ring (idle between
+        // the last MMA of an iteration and the next iteration's loads) and sent
+        // by bulk copies in two rounds (4 + 3 partners, 8 KB each): the ring
+        // holds 32 KB.  Receive slots are per source, so sums are deterministic.
+        constexpr uint32_t PART_BYTES = B_PART_BYTES;  // one partner's 16 units
+        constexpr int ROUND0 = B_ROUND0;
+        float *stage = reinterpret_cast<float *>(ring);
+        auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
+        auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
         const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
-        auto peer_recv = [&](int d) {
-            const int slot = ((int)kpart < d) ? (int)kpart : (int)kpart - 1;
-            return tc::map_rank(recv_lo + (uint32_t)(slot * B_MROWS * UPC * 4), (uint32_t)d);
-        };
         float dc[UPT], dbacc[4][UPT];
         float gv[4][UPT], ct[UPT], cp[UPT], dyv[UPT];
 #pragma unroll
@@ -608,31 +636,51 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
             if (!rec::epi_vote_all_n<B_EPI_THREADS>(w)) return false;
             dph[acc] ^= 1;
             tc::tc_fence_after();
-#pragma unroll
-            for (int d = 0; d < KS; ++d) {
+            const uint32_t col0 = tmem_base + ((uint32_t)(32 * q) << 16) + acc * B_UNITS + uo;
+            {   // own 8 units
                 uint32_t v[UPT];
-                tc::tmem_ld8(tmem_base + ((uint32_t)(32 * q) << 16) + acc * B_UNITS + d * UPC + uo, v);
+                tc::tmem_ld8(col0 + kpart * UPC, v);
                 tc::tmem_ld_wait();
-                if (d == (int)kpart) {
 #pragma unroll
-                    for (int u = 0; u < UPT; ++u) dh[u] = __uint_as_float(v[u]);
-                } else {
+                for (int u = 0; u < UPT; ++u) dh[u] = __uint_as_float(v[u]);
+            }
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {  // units uo + 4k .. +3: chunk uo/4 + k
-                        const int ch = uo / 4 + k;
-                        tc::st_cluster_v4(peer_recv(d) + (uint32_t)(((ch * B_MROWS + m) * 4) * 4),
-                                          __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                          __uint_as_float(v[4 * k + 2]),
-                                          __uint_as_float(v[4 * k + 3]));
+            for (int round = 0; round < 2; ++round) {
+                const int p0 = round ? ROUND0 : 0, p1 = round ? KS - 1 : ROUND0;
+                if (round) {
+                    // the first round's copies must have read the ring
+                    if (et == 0) tc::bulk_wait_read_all();
+                    rec::named_bar(1, B_EPI_THREADS);
+                }
+#pragma unroll
+                for (int d = 0; d < KS; ++d) {
+                    if (d == (int)kpart || dst_pos(d) < p0 || dst_pos(d) >= p1) continue;
+                    uint32_t v[UPT];
+                    tc::tmem_ld8(col0 + d * UPC, v);
+                    tc::tmem_ld_wait();
+                    float *blk = stage + (dst_pos(d) - p0) * (PART_BYTES / 4);
+#pragma unroll
+                    for (int k = 0; k < 2; ++k)  // units uo + 4k .. +3: chunk uo/4 + k
+                        *reinterpret_cast<float4 *>(blk + ((uo / 4 + k) * B_MROWS + m) * 4) =
+                            make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                        __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
+                }
+                tc::fence_proxy_async_smem();
+                rec::named_bar(1, B_EPI_THREADS);
+                if (et == 0) {
+                    if (round == 0) tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
+#pragma unroll
+                    for (int d = 0; d < KS; ++d) {
+                        if (d == (int)kpart || dst_pos(d) < p0 || dst_pos(d) >= p1) continue;
+                        tc::bulk_copy_to_peer(
+                            tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                            stage + (dst_pos(d) - p0) * (PART_BYTES / 4), PART_BYTES,
+                            tc::map_rank(recvbar_lo, (uint32_t)d));
                     }
+                    tc::bulk_commit();
                 }
             }
             tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-#pragma unroll
-                for (int d = 0; d < KS; ++d)
-                    if (d != (int)kpart) tc::mbar_arrive_remote(tc::map_rank(recvbar_lo, (uint32_t)d));
             const bool w2 =
                 tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x506, p.wait_ns);
             if (!rec::epi_vote_all_n<B_EPI_THREADS>(w2)) return false;
@@ -706,7 +754,10 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                 }
             }
             rec::named_bar(1, B_EPI_THREADS);
-            if (et == 0 && (int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+            if (et == 0) {
+                tc::bulk_wait_read_all();  // the ring is refilled after this arrival
+                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+            }
             if (t > 0) load_step(t - 1);
         }
         float dh0v[UPT];
@@ -719,10 +770,11 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
             oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
             oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
         }
+        if (et == 0) tc::bulk_wait_all();  // no copy of this CTA in flight from here on
         if (ok) {
             // db partial of this CTA: its 128 rows x (4 gates x 16 units), in a
-            // fixed order.  recv is free: every partner's last write preceded
-            // the arrival this CTA just waited for.
+            // fixed order.  recv is free: every partner's last copy completed on
+            // the receive barrier this CTA just waited for.
             rec::named_bar(1, B_EPI_THREADS);
             float *red = recv;  // [128 rows][64]
 #pragma unroll
