@@ -356,6 +356,7 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
             __nv_bfloat16 *yt = p.y + (long long)t * B * H;
             __nv_bfloat16 *gt = p.gates + (long long)t * B * 4 * H;
             float *ct = p.cells + (long long)t * B * H;
+            float gsave[4][NP];
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const int n = pair_col(k), uu = pair_unit(k);
@@ -367,22 +368,16 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                 const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + gx[3][k]);
                 c[k] = fg * c[k] + ig * gg;
                 const float h = og * rec::tanh_fast(c[k]);
+                gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
                 if (b < B) {
                     const long long o = (long long)b * H + j;
-                    yt[o] = __float2bfloat16_rn(h);
-                    ct[o] = c[k];
-                    __nv_bfloat16 *g4 = gt + (long long)b * 4 * H + j;
-                    g4[0] = __float2bfloat16_rn(ig);
-                    g4[H] = __float2bfloat16_rn(fg);
-                    g4[2 * H] = __float2bfloat16_rn(gg);
-                    g4[3 * H] = __float2bfloat16_rn(og);
+                    yt[o] = __float2bfloat16_rn(h);  // h_t: what the other CTAs wait for
                     if (t == p.T - 1) {
                         p.hT[o] = __float2bfloat16_rn(h);
                         p.cT[o] = c[k];
                     }
                 }
             }
-            if (t + 1 < p.T) load_gx(t + 1);
             rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
             if (et == 0) {
                 // the staging block (the ring) must be read out before this
@@ -390,6 +385,22 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                 if (KS > 1) tc::bulk_wait_read_all();
                 if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
             }
+            // saved state for the backward pass: not needed by the other CTAs
+            // during the recurrence, so stored after the arrival (outside the
+            // writes its release has to cover)
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = pair_col(k), uu = pair_unit(k);
+                const int b = bc0 + n, j = u0 + uu;
+                if (n >= NBc || b >= B) continue;
+                ct[(long long)b * H + j] = c[k];
+                __nv_bfloat16 *g4 = gt + (long long)b * 4 * H + j;
+                g4[0] = __float2bfloat16_rn(gsave[0][k]);
+                g4[H] = __float2bfloat16_rn(gsave[1][k]);
+                g4[2 * H] = __float2bfloat16_rn(gsave[2][k]);
+                g4[3 * H] = __float2bfloat16_rn(gsave[3][k]);
+            }
+            if (t + 1 < p.T) load_gx(t + 1);
         }
         if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
     }
