@@ -316,13 +316,16 @@ __global__ void __launch_bounds__(F_THREADS, 1) fwd2_kernel(const __grid_constan
                     if (et == 0) {
                         tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
                         const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(recv_full);
+                        // rank kpart + s first: each CTA receives from one
+                        // sender at a time instead of all sending to rank 0
 #pragma unroll
-                        for (int d = 0; d < KS; ++d)
-                            if (d != (int)kpart)
-                                tc::bulk_copy_to_peer(
-                                    tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
-                                    send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
-                                    tc::map_rank(bar_lo, (uint32_t)d));
+                        for (int s = 1; s < KS; ++s) {
+                            const int d = ((int)kpart + s) % KS;
+                            tc::bulk_copy_to_peer(
+                                tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                                send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                                tc::map_rank(bar_lo, (uint32_t)d));
+                        }
                         tc::bulk_commit();
                     }
                     const bool w2 = tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x406,
@@ -589,7 +592,9 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
         constexpr uint32_t PART_BYTES = B_PART_BYTES;  // one partner's 16 units
         constexpr int ROUND0 = B_ROUND0;
         float *stage = reinterpret_cast<float *>(ring);
-        auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
+        // partners are served in the order kpart + 1, kpart + 2, ... so each
+        // CTA receives from one sender at a time; src_slot(d): this CTA's
+        // receive slot at d
         auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
         const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
         float dc[UPT], dbacc[4][UPT];
@@ -664,12 +669,12 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                     rec::named_bar(1, B_EPI_THREADS);
                 }
 #pragma unroll
-                for (int d = 0; d < KS; ++d) {
-                    if (d == (int)kpart || dst_pos(d) < p0 || dst_pos(d) >= p1) continue;
+                for (int sp = p0; sp < p1; ++sp) {
+                    const int d = ((int)kpart + 1 + sp) % KS;  // dst_pos(d) == sp
                     uint32_t v[UPT];
                     tc::tmem_ld8(col0 + d * UPC, v);
                     tc::tmem_ld_wait();
-                    float *blk = stage + (dst_pos(d) - p0) * (PART_BYTES / 4);
+                    float *blk = stage + (sp - p0) * (PART_BYTES / 4);
 #pragma unroll
                     for (int k = 0; k < 2; ++k)  // units uo + 4k .. +3: chunk uo/4 + k
                         *reinterpret_cast<float4 *>(blk + ((uo / 4 + k) * B_MROWS + m) * 4) =
@@ -681,11 +686,11 @@ __global__ void __launch_bounds__(B_THREADS, 1) bwd2_kernel(const __grid_constan
                 if (et == 0) {
                     if (round == 0) tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
 #pragma unroll
-                    for (int d = 0; d < KS; ++d) {
-                        if (d == (int)kpart || dst_pos(d) < p0 || dst_pos(d) >= p1) continue;
+                    for (int sp = p0; sp < p1; ++sp) {
+                        const int d = ((int)kpart + 1 + sp) % KS;
                         tc::bulk_copy_to_peer(
                             tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
-                            stage + (dst_pos(d) - p0) * (PART_BYTES / 4), PART_BYTES,
+                            stage + (sp - p0) * (PART_BYTES / 4), PART_BYTES,
                             tc::map_rank(recvbar_lo, (uint32_t)d));
                     }
                     tc::bulk_commit();
