@@ -18,6 +18,7 @@
 #include "tc_host.cuh"
 #include "tc_recur.cuh"
 #include "tc_recur2.cuh"
+#include "tc_recur3.cuh"
 
 using namespace lstm;
 
@@ -523,6 +524,41 @@ bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
     return true;
 }
 
+// Backward with W_h^T in TMEM: same grid as plan_bwd2; the K slice (H/2) must
+// fit TMEM beside the accumulator (H <= 1536) and the ring must stage one
+// exchange round (at least 4 stages, H >= 512).  LSTM_BWD_TMEM_W=0 turns it
+// off (comparison runs).
+bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
+    const char *e = getenv("LSTM_BWD_TMEM_W");
+    if (e && e[0] == '0') return false;
+    if (d->dtype != LSTM_BF16 || d->H % rec3::UNITS != 0 || d->B < 1 ||
+        tcg::encode_fn() == nullptr || force_simt())
+        return false;
+    P.KS = rec3::KS;
+    P.R = d->H / rec3::UNITS;
+    P.kcc = 4 * d->H / rec3::KS / 64;
+    if (rec3::W_COL + (uint32_t)(P.kcc * 32) > rec3::TMEM_COLS) return false;
+    int stages = std::min(P.kcc, rec3::MAX_STAGES);
+    while (stages >= rec3::MIN_STAGES && rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
+    if (stages < rec3::MIN_STAGES) return false;
+    P.smem = rec3::Bwd3Smem(stages).total + 1024;
+    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel, rec3::THREADS, P.smem,
+                                         P.KS);
+    const int gmax = std::min(maxc / P.R, kMaxGroups);
+    if (gmax < 1) return false;
+    int G = std::min(gmax, (d->B + 15) / 16);
+    int NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    if (NB > rec3::NMAX) {
+        G = (d->B + rec3::NMAX - 1) / rec3::NMAX;
+        NB = ((d->B + G - 1) / G + 15) / 16 * 16;
+    }
+    P.G = (d->B + NB - 1) / NB;
+    if (P.G > gmax) return false;
+    P.stages = stages;
+    P.NB = NB;
+    return true;
+}
+
 // One cooperative launch of `grid` CTAs in clusters of KS (all CTAs co-resident
 // or the launch fails).  If this runtime refuses cooperative cluster launches,
 // the cluster launch goes ahead when the occupancy calculator says every
@@ -650,6 +686,42 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
     return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
+// a3 (+ a5) on the cluster kernel with W_h^T in TMEM (written to the
+// workspace first, then copied into each CTA's tensor memory).
+int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
+                       const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
+                       const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
+                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I, G4 = 4 * H;
+    rec3::Bwd3Params prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB)) return LSTM_ERR_UNSUPPORTED;
+    {
+        dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
+        rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)I);
+        note_launch();
+        if (cudaGetLastError() != cudaSuccess) return LSTM_ERR_CUDA;
+    }
+    prm.wt = WT;
+    prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
+    prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
+    prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
+    prm.kcc = P.kcc; prm.stages = P.stages;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_cluster(rec3::bwd3_kernel, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
+                                         rec3::THREADS);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    if (e != cudaSuccess) return LSTM_ERR_CUDA;
+    simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ forward pass
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
@@ -741,14 +813,20 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     }
 
     RecPlan plan;
-    Rec2Plan plan2;
-    const bool v2 = plan_bwd2(d, plan2);
-    if (v2 || plan_bwd_recur(d, plan)) {
+    Rec2Plan plan2, plan3;
+    const bool v3 = plan_bwd3(d, plan3);
+    const bool v2 = !v3 && plan_bwd2(d, plan2);
+    if (v3 || v2 || plan_bwd_recur(d, plan)) {
         {   // a3 + a5: persistent tcgen05 recurrence with db fused
             prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
             int rc = LSTM_ERR_NOT_CORESIDENT;
-            g_last_bwd_path = 2;
-            if (v2)
+            g_last_bwd_path = v3 ? 3 : 2;
+            if (v3)
+                rc = tc_bwd_recurrence3(d, plan3, (const bf16 *)dy, (const bf16 *)dhT, dcT,
+                                        (const bf16 *)W, c0, (const bf16 *)gates, cells,
+                                        (bf16 *)dG, (bf16 *)(ws + L.wt),
+                                        (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
+            else if (v2)
                 rc = tc_bwd_recurrence2(d, plan2, (const bf16 *)dy, (const bf16 *)dhT, dcT,
                                         (const bf16 *)W, c0, (const bf16 *)gates, cells,
                                         (bf16 *)dG, (bf16 *)(ws + L.wt),

@@ -2,8 +2,9 @@
 CTA 0 never signals its step barrier must give up after its bounded wait,
 record LSTM_ERR_TIMEOUT in the workspace status word (read by lstm_status), and
 leave the context usable -- the next normal call succeeds and matches the
-oracle.  Covered for the K-resident kernels (H = 64) and the cluster kernels
-(H = 256: forward clusters of 4, backward clusters of 8)."""
+oracle.  Covered for the K-resident kernels (H = 64), the cluster kernels
+(H = 256: forward clusters of 4, backward clusters of 8) and the backward
+cluster kernel with the weights in tensor memory (H = 512)."""
 import pytest
 import torch
 
@@ -15,7 +16,7 @@ from tests.parity_util import assert_within, compare, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H", [64, 256])
+@pytest.mark.parametrize("H", [64, 256, 512])
 def test_missing_arrival_times_out_and_recovers(H, cuda_device):
     lbuild.build()
     w = synth.custom(6, 32, 64, H, "bf16", seed=11)
@@ -34,6 +35,7 @@ def test_missing_arrival_times_out_and_recovers(H, cuda_device):
         L.lstm_bwd(st.dims, inp["dy"], inp["dhT"], inp["dcT"], inp["x"], inp["W"], inp["h0"],
                    inp["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0, wsb)
         assert L.lstm_status(wsb) == L.LSTM_ERR_TIMEOUT
+        assert L.test_last_paths()[1] == {64: 1, 256: 2, 512: 3}[H]
     finally:
         L.test_set_wait_fault(-1, 0)
     # the context is still usable and the next call is correct

@@ -25,9 +25,9 @@ SAMPLED = {"lstm_T256_B128_I1024_H1024_bf16": [0, 37, 101, 127],
 
 # recurrent kernel each workload must run on (see lstm_test_last_paths)
 EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (0, 0), "lstm_T64_B32_I256_H256_fp32": (0, 0),
-                  "lstm_T128_B64_I512_H512_bf16": (2, 2),
-                  "lstm_T256_B128_I1024_H1024_bf16": (2, 2),
-                  "lstm_T1024_B16_I256_H1024_bf16": (2, 2)}
+                  "lstm_T128_B64_I512_H512_bf16": (2, 3),
+                  "lstm_T256_B128_I1024_H1024_bf16": (2, 3),
+                  "lstm_T1024_B16_I256_H1024_bf16": (2, 3)}
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -64,7 +64,14 @@ ODD = [
     (2, 130, 64, 128, "fp32"), (7, 5, 16, 33, "fp32"),
     (5, 3, 37, 45, "bf16"), (1, 1, 1, 1, "bf16"), (3, 67, 100, 72, "bf16"),
     (4, 130, 128, 128, "bf16"), (9, 16, 64, 64, "bf16"), (3, 200, 192, 256, "bf16"),
+    # backward with the weights in tensor memory: two ragged batch groups,
+    # an odd count of unit slices, and the largest H whose K slice fits TMEM
+    (5, 200, 96, 512, "bf16"), (3, 37, 64, 640, "bf16"), (2, 16, 32, 1536, "bf16"),
 ]
+
+
+# backward recurrent kernel of the odd shapes above (see lstm_test_last_paths)
+ODD_BWD_PATH = {512: 3, 640: 3, 1536: 3}
 
 
 @pytest.mark.parametrize("T,B,I,H,dt", ODD)
@@ -72,6 +79,8 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
     w = synth.custom(T, B, I, H, dt, seed=T * 1000 + B + I + H)
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
+    if H in ODD_BWD_PATH:
+        assert L.test_last_paths()[1] == ODD_BWD_PATH[H]
     ref = run_oracle(inp)
     assert_within(compare(gpu, ref, dt), dt, w.name)
 
