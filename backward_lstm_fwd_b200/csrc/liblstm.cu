@@ -411,6 +411,7 @@ int tc_bwd_recurrence(const lstm_dims *d, const RecPlan &P, const bf16 *dy, cons
 // --------------------------------------- cluster recurrence kernels (bf16)
 struct Rec2Plan {
     int KS, G, NB, kcc, R, stages;
+    int kcx;  // fused forward: K chunks of x per CTA
     size_t smem;
 };
 
@@ -487,6 +488,54 @@ bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
     return false;
 }
 
+const void *fwd3_kernel_ptr(int NB, int KS) {
+#define LSTM_F3(nb, ks) \
+    if (NB == nb && KS == ks) return (const void *)rec3::fwd3_kernel<nb, ks>;
+    LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
+    LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
+    LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
+    LSTM_F3(128, 4) LSTM_F3(128, 8)
+#undef LSTM_F3
+    return nullptr;
+}
+
+// Forward with the input projection fused: the grid of plan_fwd2, and the
+// CTA's W_h and W_x K-slices must fit TMEM beside two accumulators.
+// LSTM_FWD_FUSED_X=0 turns it off (comparison runs).
+bool plan_fwd3(const lstm_dims *d, Rec2Plan &P) {
+    const char *e = getenv("LSTM_FWD_FUSED_X");
+    if (e && e[0] == '0') return false;
+    if (d->dtype != LSTM_BF16 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
+        d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
+        return false;
+    const int nsm = tcg::sm_count();
+    P.R = d->H / rec2::F_UNITS;
+    for (int KS : {4, 2, 8, 1}) {
+        if ((d->H / KS) % 64 != 0 || d->H % KS != 0) continue;
+        const int kcc = d->H / KS / 64;
+        const int kcx = (d->I + KS * 64 - 1) / (KS * 64);
+        if (kcc < 1 || kcc > rec3::F3_MAXC || kcx > rec3::F3_MAXC) continue;
+        const int gsm = std::min(nsm / (P.R * KS), kMaxGroups);  // SM bound first
+        if (gsm < 1) continue;
+        const int G0 = std::min(gsm, (d->B + 15) / 16);
+        int NB = 16;
+        while (NB < (d->B + G0 - 1) / G0) NB *= 2;
+        NB = std::max(NB, 4 * KS);
+        if (NB > 128 || NB / KS > 32) continue;
+        if (rec3::fwd3_tmem_cols(NB, kcc, kcx) > 512) continue;
+        const int G = (d->B + NB - 1) / NB;
+        const size_t smem = rec3::Fwd3Smem(kcc, kcx, NB, KS).total + 1024;
+        if (smem > kMaxSmem) continue;
+        const void *kern = fwd3_kernel_ptr(NB, KS);
+        if (!kern) continue;
+        const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
+        if (G * P.R > maxc) continue;
+        P.KS = KS; P.G = G; P.NB = NB; P.kcc = kcc; P.kcx = kcx; P.smem = smem;
+        return true;
+    }
+    return false;
+}
+
 // Backward: U = H/128 unit slices x 8 K-parts of 4H x G batch groups of NB rows;
 // U * G clusters of 8 must be co-resident (cudaOccupancyMaxActiveClusters).
 bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
@@ -539,7 +588,7 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     P.kcc = 4 * d->H / rec3::KS / 64;
     if (rec3::W_COL + (uint32_t)(P.kcc * 32) > rec3::TMEM_COLS) return false;
     int stages = std::min(P.kcc, rec3::MAX_STAGES);
-    while (stages >= rec3::MIN_STAGES && rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
+    while (stages >= rec3::MIN_STAGES && (size_t)rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
     if (stages < rec3::MIN_STAGES) return false;
     P.smem = rec3::Bwd3Smem(stages).total + 1024;
     const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel, rec3::THREADS, P.smem,
@@ -649,6 +698,51 @@ int tc_fwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *W, con
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
+template <int NB, int KS>
+cudaError_t launch_fwd3_t(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStream_t s) {
+    return launch_cluster(rec3::fwd3_kernel<NB, KS>, prm, P.R * KS * P.G, KS, P.smem, s,
+                          rec2::F_THREADS);
+}
+
+cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStream_t s) {
+#define LSTM_F3(nb, ks) \
+    if (P.NB == nb && P.KS == ks) return launch_fwd3_t<nb, ks>(prm, P, s);
+    LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
+    LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
+    LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
+    LSTM_F3(128, 4) LSTM_F3(128, 8)
+#undef LSTM_F3
+    return cudaErrorInvalidConfiguration;
+}
+
+// a1 + a2 in one cluster kernel (x-part contracted inside the recurrence);
+// LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
+int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, const bf16 *W,
+                       const bf16 *b, const bf16 *h0, const float *c0, bf16 *y, bf16 *hT,
+                       float *cT, bf16 *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, I = d->I;
+    rec3::Fwd3Params prm;
+    memset(&prm, 0, sizeof(prm));
+    bool ok = tcg::make_map(&prm.map_y, y, H, T * B, H * 2, 64, P.NB) &&
+              tcg::make_map(&prm.map_x, x, I, T * B, I * 2, 64, P.NB);
+    if (h0) ok = ok && tcg::make_map(&prm.map_h0, h0, H, B, H * 2, 64, P.NB);
+    else prm.map_h0 = prm.map_y;
+    if (!ok) return LSTM_ERR_UNSUPPORTED;
+    prm.W = W; prm.bias = b; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
+    prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.I = (int)I; prm.R = P.R; prm.G = P.G;
+    prm.kcc = P.kcc; prm.kcx = P.kcx;
+    prm.has_h0 = h0 != nullptr;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_fwd3(prm, P, s);
+    if (e == cudaErrorInvalidConfiguration || e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
 // a3 (+ a5) on the cluster kernel.  W_h^T is written to the workspace first;
 // db is the sum of the batch groups' partials.
 int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
@@ -732,6 +826,15 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
     const FwdLayout L = fwd_layout(d);
     float *Gx = (float *)(ws + L.gx);
     if ((long long)T_ * B > 0 && H > 0) {
+        Rec2Plan plan3;
+        if (plan_fwd3(d, plan3)) {  // a1 fused into a2
+            prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
+            const int rc = tc_fwd_recurrence3(d, plan3, (const bf16 *)x, (const bf16 *)W,
+                                              (const bf16 *)b, (const bf16 *)h0, c0, (bf16 *)y,
+                                              (bf16 *)hT, cT, (bf16 *)gates, cells, (Ctrl *)ws, s);
+            g_last_fwd_path = 3;
+            if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
+        }
         {   // a1: Gx = X W_x^T + b over all T*B rows (input concat, x-part)
             prof::Phase ph(LSTM_PHASE_INPUT_PROJ, s);
             if (tc_gemm_ok(d)) {

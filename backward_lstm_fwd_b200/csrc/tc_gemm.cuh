@@ -10,7 +10,8 @@
 //   warp 0      one thread issues TMA loads into a 4-stage shared-memory ring;
 //   warp 1      allocates TMEM and one thread issues tcgen05.mma (M=128,
 //               N=256, K=16 per instruction) into one of two accumulators;
-//   warps 2-5   epilogue: TMEM -> registers -> (+ bias) -> fp32 global stores,
+//   warps 2-5   epilogue: TMEM -> registers -> (+ bias) -> fp32 global stores
+//               (32-byte vector stores where the output is aligned for them),
 //               overlapping the next tile's MMAs through the second accumulator.
 #pragma once
 
@@ -227,6 +228,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
             const int nbase = nt * BN;
             const bool vec = ((P.ldo & 3) == 0) && ((P.out_col0 & 3) == 0) &&
                              ((((uintptr_t)P.out) & 15) == 0);
+            // 32-byte stores when rows and the base are 32-byte aligned: each
+            // store fills a whole sector instead of half of one
+            const bool vec8 = ((P.ldo & 7) == 0) && ((P.out_col0 & 7) == 0) &&
+                              ((((uintptr_t)P.out) & 31) == 0);
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 if (nbase + c0 >= P.N) break;  // warp-uniform
                 uint32_t r[32];
@@ -242,7 +247,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
                         v[j] = x;
                     }
                     float *orow = P.out + (long long)m * P.ldo + P.out_col0 + nbase + c0;
-                    if (vec && nbase + c0 + 32 <= P.N) {
+                    if (vec8 && nbase + c0 + 32 <= P.N) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) tc::st_global_v8(orow + j, v + j);
+                    } else if (vec && nbase + c0 + 32 <= P.N) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4)
                             *reinterpret_cast<float4 *>(orow + j) =

@@ -1,5 +1,18 @@
-// Backward recurrence (bf16) with the recurrent weights resident in tensor
-// memory.  "SingleLayerLstmGrad", backward pass, steps 1-6: per reverse time
+// Recurrent kernels (bf16) with their weights resident in tensor memory: the
+// tcgen05.mma A operand is read from TMEM, which leaves shared memory to the
+// streamed operands and the cluster exchange.
+//
+// Forward (fwd3_kernel, "SingleLayerLstmGrad", forward-formula table, with the
+// input concatenation of the operator page): the x-part of the gate
+// pre-activation is contracted inside the recurrence instead of by a separate
+// GEMM.  Per step the CTA accumulates W_x x_t (its K-slice of I) into the step's
+// TMEM accumulator before the step's h_{t-1} arrives -- those MMAs depend on
+// no other CTA, so they run while the tensor pipe would otherwise wait for the
+// previous step's exchange and group barrier -- and then adds W_h h_{t-1}.  The
+// work split, the DSMEM reduce-scatter and the epilogue are those of the
+// cluster kernel in tc_recur2.cuh; the bias is added in the epilogue.
+//
+// Backward recurrence: "SingleLayerLstmGrad", backward pass, steps 1-6: per reverse time
 // step, delta h = dG_{t+1} W_h (the K = 4H contraction) feeds the pointwise
 // gradient of the cell, and the step's dG_t feeds the next contraction.
 //
@@ -219,7 +232,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         float *stage_buf = reinterpret_cast<float *>(ring);
         const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
         float dc[UPT], dbacc[4][UPT];
-        float gv[4][UPT], ct[UPT], cp[UPT], dyv[UPT];
+        uint4 gpk[4], dypk;  // prefetched gates and dy of the next step, still packed bf16
+        float ct[UPT], cp[UPT];
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
             dc[u] = (valid && p.dcT) ? p.dcT[(long long)b * H + jb + u] : 0.f;
@@ -229,18 +243,16 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         auto load_step = [&](int t) {
             if (!valid) {
 #pragma unroll
-                for (int u = 0; u < UPT; ++u) {
-                    ct[u] = cp[u] = dyv[u] = 0.f;
+                for (int u = 0; u < UPT; ++u) ct[u] = cp[u] = 0.f;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) gv[g][u] = 0.f;
-                }
+                for (int g = 0; g < 4; ++g) gpk[g] = make_uint4(0, 0, 0, 0);
+                dypk = make_uint4(0, 0, 0, 0);
                 return;
             }
             const long long row = (long long)t * B + b;
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-                rec::bf16x8_to_f32(
-                    __ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + g * H + jb)), gv[g]);
+                gpk[g] = __ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + g * H + jb));
             const float4 *c4 = reinterpret_cast<const float4 *>(p.cells + row * H + jb);
             const float4 x0 = __ldg(c4), x1 = __ldg(c4 + 1);
             ct[0] = x0.x; ct[1] = x0.y; ct[2] = x0.z; ct[3] = x0.w;
@@ -256,12 +268,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
 #pragma unroll
                 for (int u = 0; u < UPT; ++u) cp[u] = 0.f;
             }
-            if (p.dy) {
-                rec::bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(p.dy + row * H + jb)), dyv);
-            } else {
-#pragma unroll
-                for (int u = 0; u < UPT; ++u) dyv[u] = 0.f;
-            }
+            dypk = p.dy ? __ldg(reinterpret_cast<const uint4 *>(p.dy + row * H + jb))
+                        : make_uint4(0, 0, 0, 0);
         };
         // delta h of row m, units uo..uo+7 from MMA iteration i: each thread
         // moves its accumulator row (one unit, 64 batch rows) to the block of
@@ -281,15 +289,15 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                                  ? recv + (int)kpart * (PART_BYTES / 4)
                                  : stage_buf + ((dst - (int)kpart - 1 + KS) % KS) * (PART_BYTES / 4);
 #pragma unroll
-                for (int s = 0; s < 2; ++s) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + D_COL +
-                                      (uint32_t)(hh * 64 + 32 * s),
+                for (int s = 0; s < 4; ++s) {
+                    uint32_t v[16];
+                    tc::tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + D_COL +
+                                      (uint32_t)(hh * 64 + 16 * s),
                                   v);
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int n = hh * 64 + 32 * s + 4 * k;
+                    for (int k = 0; k < 4; ++k) {
+                        const int n = hh * 64 + 16 * s + 4 * k;
                         *reinterpret_cast<float4 *>(blk + part_off(r, n)) =
                             make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
                                         __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
@@ -348,6 +356,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 break;
             }
             float dI[UPT], dF[UPT], dGg[UPT], dO[UPT];
+            float gv[4][UPT], dyv[UPT];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) rec::bf16x8_to_f32(gpk[g], gv[g]);
+            rec::bf16x8_to_f32(dypk, dyv);
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const float ig = gv[0][u], fg = gv[1][u], gg = gv[2][u], og = gv[3][u];
@@ -360,25 +372,29 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 dF[u] = dcv * cp[u] * fg * (1.f - fg);
                 dc[u] = dcv * fg;                                       // step 5
             }
-            if (valid) {
-                __nv_bfloat16 *o = p.dG + ((long long)t * B + b) * G4 + jb;
+            {
                 const uint4 vi = rec::f32x8_to_bf16(dI), vf = rec::f32x8_to_bf16(dF);
                 const uint4 vg = rec::f32x8_to_bf16(dGg), vo = rec::f32x8_to_bf16(dO);
-                *reinterpret_cast<uint4 *>(o) = vi;
-                *reinterpret_cast<uint4 *>(o + H) = vf;
-                *reinterpret_cast<uint4 *>(o + 2 * H) = vg;
-                *reinterpret_cast<uint4 *>(o + 3 * H) = vo;
-                float ri[UPT], rf[UPT], rg[UPT], ro[UPT];  // db sums the stored values
-                rec::bf16x8_to_f32(vi, ri);
-                rec::bf16x8_to_f32(vf, rf);
-                rec::bf16x8_to_f32(vg, rg);
-                rec::bf16x8_to_f32(vo, ro);
+                if (valid) {
+                    __nv_bfloat16 *o = p.dG + ((long long)t * B + b) * G4 + jb;
+                    *reinterpret_cast<uint4 *>(o) = vi;
+                    *reinterpret_cast<uint4 *>(o + H) = vf;
+                    *reinterpret_cast<uint4 *>(o + 2 * H) = vg;
+                    *reinterpret_cast<uint4 *>(o + 3 * H) = vo;
+                }
+                if (valid) {
+                    float ri[UPT], rf[UPT], rg[UPT], ro[UPT];  // db sums the stored values
+                    rec::bf16x8_to_f32(vi, ri);
+                    rec::bf16x8_to_f32(vf, rf);
+                    rec::bf16x8_to_f32(vg, rg);
+                    rec::bf16x8_to_f32(vo, ro);
 #pragma unroll
-                for (int u = 0; u < UPT; ++u) {
-                    dbacc[0][u] += ri[u];
-                    dbacc[1][u] += rf[u];
-                    dbacc[2][u] += rg[u];
-                    dbacc[3][u] += ro[u];
+                    for (int u = 0; u < UPT; ++u) {
+                        dbacc[0][u] += ri[u];
+                        dbacc[1][u] += rf[u];
+                        dbacc[2][u] += rg[u];
+                        dbacc[3][u] += ro[u];
+                    }
                 }
             }
             rec::named_bar(1, EPI_THREADS);
@@ -423,6 +439,447 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     tc::tc_fence_before();
     __syncthreads();
     tc::cluster_sync_all();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// =========================================================================
+// forward with the input projection fused
+// =========================================================================
+constexpr int F3_MAXC = 16;         // K chunks (of 64) per operand ring
+constexpr int F3_BAR_BYTES = 1024;
+
+struct Fwd3Params {
+    CUtensorMap map_y;                // y  [T*B][H] bf16, box {64, NB}: h_{t-1}
+    CUtensorMap map_h0;               // h0 [B][H]   bf16, box {64, NB}
+    CUtensorMap map_x;                // x  [T*B][I] bf16, box {64, NB}
+    const __nv_bfloat16 *W;           // [4H][H + I]: W_h | W_x
+    const __nv_bfloat16 *bias;        // [4H] or NULL
+    const float *c0;
+    __nv_bfloat16 *y, *gates, *hT;
+    float *cells, *cT;
+    Ctrl *ctrl;
+    int T, B, H, I, R, G, kcc, kcx, has_h0;
+    int fault_skip_cta;
+    unsigned long long wait_ns;
+};
+
+// TMEM columns: two accumulators of NB, then the W_h slice (kcc x 32), then the
+// W_x slice (kcx x 32)
+__host__ __device__ constexpr int fwd3_tmem_cols(int NB, int kcc, int kcx) {
+    return 2 * NB + 32 * (kcc + kcx);
+}
+
+// ring_h: kcc chunks of h_{t-1} (NB rows x 64 K); ring_x: kcx chunks of x_t;
+// recv / xbuf / send as in the cluster forward kernel (send aliases ring_h,
+// idle between a step's last MMA and the next step's h loads, when it is
+// large enough)
+struct Fwd3Smem {
+    int ring_h, ring_x, recv, xbuf, send, bars, total;
+    __host__ __device__ Fwd3Smem(int kcc, int kcx, int NB, int KS) {
+        const int NBc = NB / KS;
+        const int hbytes = kcc * NB * 128, xbytes = kcx * NB * 128;
+        const int part_bytes = (KS - 1) * NBc * rec2::F_ROWS * 4;
+        const int xbuf_bytes = 4 * NBc * rec2::F_UNITS * 4;
+        ring_h = 0;
+        ring_x = hbytes;
+        recv = ring_x + xbytes;
+        xbuf = recv + part_bytes;
+        send = hbytes >= part_bytes ? ring_h : xbuf + xbuf_bytes;
+        bars = send == ring_h ? xbuf + xbuf_bytes : send + part_bytes;
+        bars = (bars + 15) & ~15;
+        total = bars + F3_BAR_BYTES;
+    }
+};
+
+template <int NB, int KS>
+__global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params p) {
+    using rec2::F_ROWS;
+    using rec2::F_UNITS;
+    using rec2::F_EPI_THREADS;
+    constexpr int NBc = NB / KS;       // batch columns finalised by this CTA
+    constexpr int NBh = NBc / 2;       // columns each of the two warps of a quarter moves
+    constexpr int NP = (NBc + 7) / 8;  // (unit, batch) pairs per epilogue thread
+    constexpr int VW = NBh >= 4 ? 4 : 2;  // floats per staged vector / receive chunk
+    static_assert(NBc >= 4 && NBc % 4 == 0 && NBc <= 32, "columns per CTA");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int kcc = p.kcc, kcx = p.kcx;
+    const Fwd3Smem L(kcc, kcx, NB, KS);
+    uint8_t *ring_h = smem + L.ring_h;
+    uint8_t *ring_x = smem + L.ring_x;
+    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][NBc/VW chunks][128 rows][VW]
+    float *xbuf = (float *)(smem + L.xbuf);  // [4 gates][NBc][32 units]
+    float *send = (float *)(smem + L.send);  // [KS-1 destinations][NBc/VW][128 rows][VW]
+    uint64_t *bars = (uint64_t *)(smem + L.bars);
+    uint64_t *h_full = bars;
+    uint64_t *h_empty = bars + F3_MAXC;
+    uint64_t *x_full = bars + 2 * F3_MAXC;
+    uint64_t *x_empty = bars + 3 * F3_MAXC;
+    uint64_t *w_ready = bars + 4 * F3_MAXC;  // W_h and W_x slices written to TMEM
+    uint64_t *mma_done = w_ready + 1;        // [2]: accumulator complete
+    uint64_t *d_free = w_ready + 3;          // [2]: accumulator read out by the epilogue
+    uint64_t *recv_full = w_ready + 5;
+    uint32_t *tmem_slot = (uint32_t *)(w_ready + 6);
+    volatile int *abort_flag = (volatile int *)(w_ready + 7);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t kpart = tc::cluster_rank();
+    const int cid = blockIdx.x / KS;
+    const int rs = cid % p.R, gi = cid / p.R;
+    const int u0 = rs * F_UNITS, b0 = gi * NB;
+    const int H = p.H, B = p.B, T = p.T, I = p.I;
+    const int kbase = (int)kpart * kcc * 64;  // this CTA's K range of W_h / h
+    const int xbase = (int)kpart * kcx * 64;  // and of W_x / x
+    const uint32_t WH_COL = 2 * NB, WX_COL = 2 * NB + 32 * kcc;
+    unsigned int *ctr = &p.ctrl->bar[gi];
+    const unsigned int group_ctas = (unsigned)(p.R * KS);
+    constexpr uint32_t TMEM_COLS = 512;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kcc; ++i) {
+            tc::mbar_init(&h_full[i], 1);
+            tc::mbar_init(&h_empty[i], 1);
+        }
+        for (int i = 0; i < kcx; ++i) {
+            tc::mbar_init(&x_full[i], 1);
+            tc::mbar_init(&x_empty[i], 1);
+        }
+        tc::mbar_init(w_ready, F_EPI_THREADS);
+        tc::mbar_init(&mma_done[0], 1);
+        tc::mbar_init(&mma_done[1], 1);
+        tc::mbar_init(&d_free[0], 1);
+        tc::mbar_init(&d_free[1], 1);
+        tc::mbar_init(recv_full, 1);  // one local arrival (with the expected bytes) per step
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::cluster_sync_all();  // every CTA's barriers exist before any remote arrival
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            constexpr uint32_t CHUNK = NB * 128;
+            // loads issued per chunk, so that an aborted CTA can let them land
+            int rounds_h = 0, part_h = 0, rounds_x = 0, part_x = 0;
+            uint32_t phh = 0, phx = 0;
+            bool aborted = false;
+            auto load_x = [&](int t) -> bool {
+                for (int c = 0; c < kcx; ++c) {
+                    if (!tc::mbar_wait(&x_empty[c], phx ^ 1, p.ctrl, abort_flag, 0x702, p.wait_ns))
+                        return false;
+                    tc::mbar_arrive_expect_tx(&x_full[c], CHUNK);
+                    tc::tma_load_2d(ring_x + c * CHUNK, &p.map_x, &x_full[c], xbase + 64 * c,
+                                    t * B + b0);
+                    part_x = c + 1;
+                }
+                phx ^= 1;
+                ++rounds_x;
+                part_x = 0;
+                return true;
+            };
+            aborted = !load_x(0);
+            for (int t = 0; t < T && !aborted; ++t) {
+                if (t > 0) {
+                    if (!rec::wait_counter(ctr, group_ctas * (unsigned)t, p.ctrl, abort_flag, 0x701,
+                                           p.wait_ns)) {
+                        aborted = true;
+                        break;
+                    }
+                    // the group's generic-proxy stores were released to this
+                    // thread's acquire; order the TMA (async-proxy) reads after it
+                    tc::fence_proxy_async_global();
+                }
+                if (t > 0 || p.has_h0) {
+                    const CUtensorMap *m = t > 0 ? &p.map_y : &p.map_h0;
+                    const int row0 = t > 0 ? (t - 1) * B + b0 : b0;
+                    for (int c = 0; c < kcc && !aborted; ++c) {
+                        if (!tc::mbar_wait(&h_empty[c], phh ^ 1, p.ctrl, abort_flag, 0x703,
+                                           p.wait_ns)) {
+                            aborted = true;
+                            break;
+                        }
+                        tc::mbar_arrive_expect_tx(&h_full[c], CHUNK);
+                        tc::tma_load_2d(ring_h + c * CHUNK, m, &h_full[c], kbase + 64 * c, row0);
+                        part_h = c + 1;
+                    }
+                    if (aborted) break;
+                    phh ^= 1;
+                    ++rounds_h;
+                    part_h = 0;
+                }
+                // x_{t+1} does not depend on the group: issue it now
+                if (t + 1 < T && !load_x(t + 1)) aborted = true;
+            }
+            if (aborted) {  // let every issued copy land before the CTA can exit
+                for (int c = 0; c < kcc; ++c) {
+                    const int n = rounds_h + (c < part_h ? 1 : 0);
+                    if (n > 0) tc::mbar_wait(&h_full[c], (uint32_t)((n - 1) & 1), nullptr, nullptr, 0, 200000000ull);
+                }
+                for (int c = 0; c < kcx; ++c) {
+                    const int n = rounds_x + (c < part_x ? 1 : 0);
+                    if (n > 0) tc::mbar_wait(&x_full[c], (uint32_t)((n - 1) & 1), nullptr, nullptr, 0, 200000000ull);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // D[128 gate rows][NB] = W_x slice (TMEM) x x_t chunk^T (+)
+            //                        W_h slice (TMEM) x h_{t-1} chunk^T
+            const uint32_t idesc = tc::idesc_bf16_f32(F_ROWS, NB, 0, 0);
+            const uint64_t hi = tc::smem_desc_sw128(0, 16, 1024);
+            const uint64_t rh_lo0 = tc::smem_u32(ring_h) >> 4, rx_lo0 = tc::smem_u32(ring_x) >> 4;
+            constexpr uint32_t CSTEP = (NB * 128) >> 4;
+            uint32_t phh = 0, phx = 0;
+            bool ok = tc::mbar_wait(w_ready, 0, p.ctrl, abort_flag, 0x704, p.wait_ns);
+            tc::tc_fence_after();
+            // x-part of step s into accumulator s & 1, once the epilogue has
+            // read that accumulator's previous use (step s - 2)
+            auto x_part = [&](int s) -> bool {
+                const int acc = s & 1;
+                if (!tc::mbar_wait(&d_free[acc], (uint32_t)(((s >> 1) & 1) ^ 1), p.ctrl, abort_flag,
+                                   0x705, p.wait_ns))
+                    return false;
+                tc::tc_fence_after();
+                const uint32_t d = tmem_base + acc * NB;
+                for (int c = 0; c < kcx; ++c) {
+                    if (!tc::mbar_wait(&x_full[c], phx, p.ctrl, abort_flag, 0x706, p.wait_ns))
+                        return false;
+                    tc::tc_fence_after();
+                    const uint64_t bd = hi | (rx_lo0 + c * CSTEP);
+                    const uint32_t a = tmem_base + WX_COL + 32 * c;
+                    tc::mma_bf16_ts(d, a, bd, idesc, c != 0);
+                    tc::mma_bf16_ts(d, a + 8, bd + 2, idesc, 1);
+                    tc::mma_bf16_ts(d, a + 16, bd + 4, idesc, 1);
+                    tc::mma_bf16_ts(d, a + 24, bd + 6, idesc, 1);
+                    tc::mma_commit(&x_empty[c]);
+                }
+                phx ^= 1;
+                return true;
+            };
+            ok = ok && x_part(0);
+            for (int t = 0; ok && t < T; ++t) {
+                const int acc = t & 1;
+                const uint32_t d = tmem_base + acc * NB;
+                if (t > 0 || p.has_h0) {
+                    for (int c = 0; c < kcc; ++c) {
+                        if (!tc::mbar_wait(&h_full[c], phh, p.ctrl, abort_flag, 0x707, p.wait_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                        const uint64_t bd = hi | (rh_lo0 + c * CSTEP);
+                        const uint32_t a = tmem_base + WH_COL + 32 * c;
+                        tc::mma_bf16_ts(d, a, bd, idesc, 1);
+                        tc::mma_bf16_ts(d, a + 8, bd + 2, idesc, 1);
+                        tc::mma_bf16_ts(d, a + 16, bd + 4, idesc, 1);
+                        tc::mma_bf16_ts(d, a + 24, bd + 6, idesc, 1);
+                        tc::mma_commit(&h_empty[c]);
+                    }
+                    if (!ok) break;
+                    phh ^= 1;
+                }
+                tc::mma_commit(&mma_done[acc]);
+                if (t + 1 < T) ok = x_part(t + 1);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int et = threadIdx.x - 64;  // 0..255
+        const int q = warp & 3;           // TMEM lane quarter = gate of the row read
+        const int hh = (warp - 2) >> 2;   // which half of each column block it moves
+        const int mrow = 32 * q + lane;   // row of the partial tile: gate q, unit lane
+        {
+            // W rows q*H + u0 + lane: this warp's half of the CTA's K range of
+            // W_h and of W_x (zero past I) -> TMEM lane mrow, two bf16 per column
+            const __nv_bfloat16 *wrow = p.W + (long long)(q * H + u0 + lane) * (H + I);
+            const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16);
+            const int hn = kcc * 2;  // 16-element groups per half of the W_h range
+            for (int n = 0; n < hn; ++n) {
+                const __nv_bfloat16 *src = wrow + kbase + hh * kcc * 32 + 16 * n;
+                const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(src));
+                const uint4 x1 = __ldg(reinterpret_cast<const uint4 *>(src + 8));
+                const uint32_t r[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                tc::tmem_st8(trow + WH_COL + (uint32_t)(hh * kcc * 16 + 8 * n), r);
+            }
+            const int xn = kcx * 2;
+            for (int n = 0; n < xn; ++n) {
+                const int e = xbase + hh * kcx * 32 + 16 * n;  // first x feature of the group
+                const __nv_bfloat16 *src = wrow + H + e;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                const uint4 x0 = e < I ? __ldg(reinterpret_cast<const uint4 *>(src)) : z;
+                const uint4 x1 = e + 8 < I ? __ldg(reinterpret_cast<const uint4 *>(src + 8)) : z;
+                const uint32_t r[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                tc::tmem_st8(trow + WX_COL + (uint32_t)(hh * kcx * 16 + 8 * n), r);
+            }
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            tc::mbar_arrive(w_ready);
+        }
+        const int bc0 = b0 + (int)kpart * NBc;  // first batch row finalised here
+        constexpr uint32_t PART_BYTES = NBc * F_ROWS * 4;  // one partner's partial tile
+        // position of destination d among this CTA's partners (its send block),
+        // and of this CTA among d's sources (its receive slot at d)
+        auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
+        auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
+        // pointwise pairs of this thread: pair index et + 256 k -> unit, column
+        float c[NP], bias[4][NP];
+        auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
+        auto pair_col = [&](int k) { return (et + F_EPI_THREADS * k) >> 5; };
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+            c[k] = (p.c0 && n < NBc && b < B) ? p.c0[(long long)b * H + j] : 0.f;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                bias[g][k] = p.bias ? __bfloat162float(p.bias[g * H + j]) : 0.f;
+        }
+        uint32_t dph[2] = {0, 0}, rph = 0;
+        for (int t = 0; t < T; ++t) {
+            const int acc = t & 1;
+            const bool w = tc::mbar_wait(&mma_done[acc], dph[acc], p.ctrl, abort_flag, 0x708,
+                                         p.wait_ns);
+            if (!rec::epi_vote_all_n<F_EPI_THREADS>(w)) break;
+            dph[acc] ^= 1;
+            tc::tc_fence_after();
+            float own[NBh];
+#pragma unroll
+            for (int d = 0; d < KS; ++d) {
+                uint32_t v[NBh];
+                rec2::tmem_ld_cols<NBh>(
+                    tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + d * NBc + hh * NBh, v);
+                tc::tmem_ld_wait();
+                if (d == (int)kpart) {
+#pragma unroll
+                    for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(v[n]);
+                } else {
+                    float *blk = send + dst_pos(d) * (PART_BYTES / 4);
+#pragma unroll
+                    for (int k = 0; k < NBh / VW; ++k) {
+                        const int ch = hh * (NBh / VW) + k;
+                        float *a = blk + (ch * F_ROWS + mrow) * VW;
+                        if constexpr (VW == 4)
+                            *reinterpret_cast<float4 *>(a) =
+                                make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                            __uint_as_float(v[4 * k + 2]),
+                                            __uint_as_float(v[4 * k + 3]));
+                        else
+                            *reinterpret_cast<float2 *>(a) =
+                                make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                    }
+                }
+            }
+            tc::tc_fence_before();
+            if (KS > 1) tc::fence_proxy_async_smem();  // staged partials -> bulk copies
+            rec::named_bar(1, F_EPI_THREADS);
+            // accumulator read out: the MMA thread may start step t + 2's x-part in it
+            if (et == 0) tc::mbar_arrive(&d_free[acc]);
+            if (KS > 1) {
+                if (et == 0) {
+                    tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
+                    const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(recv_full);
+                    // rank kpart + s first: each CTA receives from one sender at a time
+#pragma unroll
+                    for (int s = 1; s < KS; ++s) {
+                        const int d = ((int)kpart + s) % KS;
+                        tc::bulk_copy_to_peer(
+                            tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                            send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                            tc::map_rank(bar_lo, (uint32_t)d));
+                    }
+                    tc::bulk_commit();
+                }
+                const bool w2 = tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x709,
+                                                      p.wait_ns);
+                if (!rec::epi_vote_all_n<F_EPI_THREADS>(w2)) break;
+                rph ^= 1;
+#pragma unroll
+                for (int sl = 0; sl < KS - 1; ++sl) {
+                    const float *src = recv + sl * F_ROWS * NBc;
+#pragma unroll
+                    for (int k = 0; k < NBh / VW; ++k) {
+                        const int ch = hh * (NBh / VW) + k;
+                        if constexpr (VW == 4) {
+                            const float4 x = *reinterpret_cast<const float4 *>(src + (ch * F_ROWS + mrow) * 4);
+                            own[4 * k] += x.x;
+                            own[4 * k + 1] += x.y;
+                            own[4 * k + 2] += x.z;
+                            own[4 * k + 3] += x.w;
+                        } else {
+                            const float2 x = *reinterpret_cast<const float2 *>(src + (ch * F_ROWS + mrow) * 2);
+                            own[2 * k] += x.x;
+                            own[2 * k + 1] += x.y;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
+            rec::named_bar(1, F_EPI_THREADS);
+            __nv_bfloat16 *yt = p.y + (long long)t * B * H;
+            __nv_bfloat16 *gt = p.gates + (long long)t * B * 4 * H;
+            float *ct = p.cells + (long long)t * B * H;
+            float gsave[4][NP];
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = pair_col(k), uu = pair_unit(k);
+                if (n >= NBc) continue;
+                const int b = bc0 + n, j = u0 + uu;
+                const float ig = rec::sigmoid_fast(xbuf[(0 * NBc + n) * F_UNITS + uu] + bias[0][k]);
+                const float fg = rec::sigmoid_fast(xbuf[(1 * NBc + n) * F_UNITS + uu] + bias[1][k]);
+                const float gg = rec::tanh_fast(xbuf[(2 * NBc + n) * F_UNITS + uu] + bias[2][k]);
+                const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
+                c[k] = fg * c[k] + ig * gg;
+                const float h = og * rec::tanh_fast(c[k]);
+                gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
+                if (b < B) {
+                    const long long o = (long long)b * H + j;
+                    yt[o] = __float2bfloat16_rn(h);  // h_t: what the other CTAs wait for
+                    if (t == T - 1) {
+                        p.hT[o] = __float2bfloat16_rn(h);
+                        p.cT[o] = c[k];
+                    }
+                }
+            }
+            rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
+            if (et == 0) {
+                // the staging block must be read out before this CTA's arrival
+                // lets the next step's TMA refill ring_h
+                if (KS > 1) tc::bulk_wait_read_all();
+                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+            }
+            // saved state for the backward pass, outside the writes the
+            // arrival's release has to cover
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = pair_col(k), uu = pair_unit(k);
+                const int b = bc0 + n, j = u0 + uu;
+                if (n >= NBc || b >= B) continue;
+                ct[(long long)b * H + j] = c[k];
+                __nv_bfloat16 *g4 = gt + (long long)b * 4 * H + j;
+                g4[0] = __float2bfloat16_rn(gsave[0][k]);
+                g4[H] = __float2bfloat16_rn(gsave[1][k]);
+                g4[2 * H] = __float2bfloat16_rn(gsave[2][k]);
+                g4[3 * H] = __float2bfloat16_rn(gsave[3][k]);
+            }
+        }
+        if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::cluster_sync_all();  // no partner may still be writing into this CTA's smem
     if (warp == 1) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem_base, TMEM_COLS);

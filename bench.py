@@ -67,12 +67,16 @@ def measured_traffic(phase: str, workload: str):
         return None
 
 
-def phase_work(w: synth.Workload):
+def phase_work(w: synth.Workload, phases=None):
     """Algorithmic work per phase: FLOPs for the contractions (2 * M * N * K of
-    the products the method defines), bytes for the db column reduction."""
+    the products the method defines), bytes for the db column reduction.  With
+    the measured `phases` ({name: (ms, launches)}), work moves to the phase
+    that ran it: the x-part of the gate pre-activations into the forward
+    recurrence when no input-projection launch ran (the fused forward kernel),
+    dx into the dW phase when both share one launch."""
     TB, H, I = w.rows, w.H, w.I
     es = 2 if w.dtype == "bf16" else 4
-    return {
+    work = {
         "input_proj": ("flop", 2.0 * TB * 4 * H * I),
         "fwd_recur": ("flop", 2.0 * TB * 4 * H * H),
         "bwd_recur": ("flop", 2.0 * TB * 4 * H * H),
@@ -81,6 +85,13 @@ def phase_work(w: synth.Workload):
         "dx": ("flop", 2.0 * TB * 4 * H * I),
         "other": ("byte", 0.0),
     }
+    if phases is not None:
+        ran = lambda k: phases.get(k, (0.0, 0))[1] > 0
+        if not ran("input_proj") and ran("fwd_recur"):
+            work["fwd_recur"] = ("flop", work["fwd_recur"][1] + work["input_proj"][1])
+        if not ran("dx") and ran("dW"):
+            work["dW"] = ("flop", work["dW"][1] + work["dx"][1])
+    return work
 
 
 class ClockSampler:
@@ -293,7 +304,7 @@ def run_ours(args, w, rank, world, local_rank):
         return 0
 
     peaks, peak_src = load_peaks()
-    work = phase_work(w)
+    work = phase_work(w, phases)
     dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
     dom_ms, dom_launches = phases[dom]
     kind, amount = work[dom]

@@ -41,9 +41,9 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
  * Which recurrent kernel the most recent lstm_fwd / lstm_bwd of this process
  * used: 0 = one CUDA-core launch per step (fp32, or shapes off the tensor-core
  * grid), 1 = persistent kernel with K resident per CTA, 2 = persistent cluster
- * kernel with K split across the CTAs of a cluster, 3 = (backward only) the
- * cluster kernel with the recurrent weights held in tensor memory; -1 = none
- * yet.
+ * kernel with K split across the CTAs of a cluster, 3 = the cluster kernel
+ * with the weights held in tensor memory (forward: with the input projection
+ * contracted inside the recurrence); -1 = none yet.
  */
 int lstm_test_last_paths(int *fwd_path, int *bwd_path);
 

@@ -25,9 +25,9 @@ SAMPLED = {"lstm_T256_B128_I1024_H1024_bf16": [0, 37, 101, 127],
 
 # recurrent kernel each workload must run on (see lstm_test_last_paths)
 EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (0, 0), "lstm_T64_B32_I256_H256_fp32": (0, 0),
-                  "lstm_T128_B64_I512_H512_bf16": (2, 3),
-                  "lstm_T256_B128_I1024_H1024_bf16": (2, 3),
-                  "lstm_T1024_B16_I256_H1024_bf16": (2, 3)}
+                  "lstm_T128_B64_I512_H512_bf16": (3, 3),
+                  "lstm_T256_B128_I1024_H1024_bf16": (3, 3),
+                  "lstm_T1024_B16_I256_H1024_bf16": (3, 3)}
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -70,7 +70,10 @@ ODD = [
 ]
 
 
-# backward recurrent kernel of the odd shapes above (see lstm_test_last_paths)
+# recurrent kernels of the odd bf16 shapes above (see lstm_test_last_paths):
+# the forward with the input projection fused wherever H is a multiple of 32
+# (clusters of 4, 2 and 1 among these), the backward with the weights in TMEM
+ODD_FWD_PATH = {64: 3, 128: 3, 256: 3, 512: 3, 640: 3, 1536: 3}
 ODD_BWD_PATH = {512: 3, 640: 3, 1536: 3}
 
 
@@ -79,7 +82,9 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
     w = synth.custom(T, B, I, H, dt, seed=T * 1000 + B + I + H)
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
-    if H in ODD_BWD_PATH:
+    if dt == "bf16" and H in ODD_FWD_PATH:
+        assert L.test_last_paths()[0] == ODD_FWD_PATH[H]
+    if dt == "bf16" and H in ODD_BWD_PATH:
         assert L.test_last_paths()[1] == ODD_BWD_PATH[H]
     ref = run_oracle(inp)
     assert_within(compare(gpu, ref, dt), dt, w.name)
@@ -132,3 +137,4 @@ def test_side_stream_and_repeat(cuda_device):
     for k in OUTS:
         np.testing.assert_array_equal(a[k], b[k])
     assert_within(compare(a, run_oracle(inp), "bf16"), "bf16", "side stream")
+
