@@ -201,29 +201,83 @@ cudaError_t tc_input_projection(const lstm_dims *d, const bf16 *x, const bf16 *W
 //   dx          = dG W_x
 // dG^T and the z-rows are MN-major operands read straight from their
 // row-major storage; the time shift of h_prev is a TMA row offset.
+// a4 + a6 over the rows of time steps [t_lo, t_hi):
+//   dW (+)= dG[rows]^T [h_prev | x][rows],   dx[rows] = dG[rows] W_x.
+// The operand maps end at the range's last row, so a partial 64-row K block
+// reads zeros rather than rows of the next range.  At most max_ctas CTAs
+// (0: one per SM).
 cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf16 *W,
                      const bf16 *h0, const bf16 *y, float *dW, float *dx, Ctrl *ctrl,
-                     cudaStream_t s) {
-    const long long T = d->T, B = d->B, TB = T * B, H = d->H, I = d->I, G4 = 4 * H;
+                     cudaStream_t s, int t_lo, int t_hi, bool accumulate, int max_ctas) {
+    const long long B = d->B, H = d->H, I = d->I, G4 = 4 * H;
+    const long long r0 = (long long)t_lo * B, r1 = (long long)t_hi * B;
     tcg::Builder bld(ctrl);
-    const int m_dg_mn = bld.add_map({dG, TB, G4, G4}, 1, 0);
-    const int m_x_mn = bld.add_map({x, TB, I, I}, 1, 0);
-    const int m_dg_k = bld.add_map({dG, TB, G4, G4}, 0, tcg::BM);
+    const int m_dg_mn = bld.add_map({dG, r1, G4, G4}, 1, 0);
+    const int m_x_mn = bld.add_map({x, r1, I, I}, 1, 0);
+    const int m_dg_k = bld.add_map({dG, r1, G4, G4}, 0, tcg::BM);
     const int m_wx_mn = bld.add_map({W + H, G4, I, H + I}, 1, 0);
-    const int m_y_mn = (T > 1) ? bld.add_map({y, (T - 1) * B, H, H}, 1, 0) : -1;
-    const int m_h0_mn = h0 ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
-    // dW, h-part (zero when T == 1 and h0 is absent: no K segment)
+    // h_prev of row r is y row r - B (r >= B) or h0 row r (r < B, only when t_lo == 0)
+    const long long ry0 = std::max(r0, B);
+    const int m_y_mn = (r1 > ry0) ? bld.add_map({y, r1 - B, H, H}, 1, 0) : -1;
+    const int m_h0_mn = (h0 && r0 < B) ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
+    // dW, h-part (no K segment, i.e. zero, when the range is t = 0 alone and h0 is absent)
     tcg::Problem &p0 = bld.add_problem((int)G4, (int)H, 1, 1, dW, H + I, 0, nullptr);
-    if (m_y_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, (int)B, m_y_mn, 0, (T - 1) * B);
+    p0.accumulate = accumulate;
+    if (m_y_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, (int)ry0, m_y_mn, (int)(ry0 - B), r1 - ry0);
     if (m_h0_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, 0, m_h0_mn, 0, B);
     // dW, x-part
     tcg::Problem &p1 = bld.add_problem((int)G4, (int)I, 1, 1, dW, H + I, (int)H, nullptr);
-    tcg::Builder::add_seg(p1, m_dg_mn, 0, m_x_mn, 0, TB);
-    // dx
-    tcg::Problem &p2 = bld.add_problem((int)TB, (int)I, 0, 1, dx, I, 0, nullptr);
+    p1.accumulate = accumulate;
+    tcg::Builder::add_seg(p1, m_dg_mn, (int)r0, m_x_mn, (int)r0, r1 - r0);
+    // dx rows r0 .. r1-1
+    tcg::Problem &p2 = bld.add_problem((int)(r1 - r0), (int)I, 0, 1, dx + r0 * I, I, 0, nullptr);
+    p2.a_mn0 = (int)r0;
     tcg::Builder::add_seg(p2, m_dg_k, 0, m_wx_mn, 0, G4);
     if (!bld.ok) return cudaErrorInvalidValue;
-    return tcg::launch(bld, s);
+    return tcg::launch(bld, s, max_ctas);
+}
+
+// Streams of a chunked backward call, per device: the recurrence on a
+// high-priority stream (its clusters are placed before pending GEMM CTAs),
+// the dW / dx GEMMs on a low-priority one, joined back into the caller's
+// stream with events.  Created on first use and kept for the process.
+constexpr int kMaxChunks = 16;
+struct AuxStreams {
+    cudaStream_t rec = nullptr, gemm = nullptr;
+    cudaEvent_t ev[kMaxChunks + 3] = {};
+    bool ready = false, tried = false;
+    std::mutex mu;  // one chunked call enqueues at a time (the events are shared)
+};
+
+AuxStreams *aux_streams() {
+    static std::mutex mu;
+    static AuxStreams per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    AuxStreams &a = per_dev[dev];
+    if (!a.tried) {
+        a.tried = true;
+        int lo = 0, hi = 0;
+        bool ok = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
+                  cudaStreamCreateWithPriority(&a.rec, cudaStreamNonBlocking, hi) == cudaSuccess &&
+                  cudaStreamCreateWithPriority(&a.gemm, cudaStreamNonBlocking, lo) == cudaSuccess;
+        for (int i = 0; ok && i < kMaxChunks + 3; ++i)
+            ok = cudaEventCreateWithFlags(&a.ev[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+        a.ready = ok;
+    }
+    return a.ready ? &a : nullptr;
+}
+
+// Number of reverse-time chunks of a backward call whose dW / dx GEMMs run
+// beside the recurrence (1: no overlap): at least 16 steps per chunk, at most
+// 8 chunks (the last chunk's GEMM is the part that cannot overlap; each chunk
+// costs one more launch of the recurrence).  LSTM_BWD_CHUNKS overrides.
+int bwd_chunks(const lstm_dims *d) {
+    const char *e = getenv("LSTM_BWD_CHUNKS");
+    int n = e ? atoi(e) : (d->T >= 32 ? std::min(8, d->T / 16) : 1);
+    return std::max(1, std::min(std::min(n, kMaxChunks), d->T));
 }
 
 // ------------------------------------------- persistent recurrence (bf16)
@@ -780,28 +834,24 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
     return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
-// a3 (+ a5) on the cluster kernel with W_h^T in TMEM (written to the
-// workspace first, then copied into each CTA's tensor memory).
-int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                       const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
-                       const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
-                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
-    const long long T = d->T, B = d->B, H = d->H, I = d->I, G4 = 4 * H;
+// One launch of the TMEM-weight backward kernel over epilogue iterations
+// [i0, i1) (time steps T-i1 .. T-i0-1); WT must already hold W_h^T.
+int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
+                   const float *dcT, const float *c0, const bf16 *gates, const float *cells,
+                   bf16 *dG, const bf16 *WT, float *dbgroup, float *dh0, float *dc0,
+                   float *dc_carry, Ctrl *ctrl, int i0, int i1, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
     rec3::Bwd3Params prm;
     memset(&prm, 0, sizeof(prm));
     if (!tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB)) return LSTM_ERR_UNSUPPORTED;
-    {
-        dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
-        rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)I);
-        note_launch();
-        if (cudaGetLastError() != cudaSuccess) return LSTM_ERR_CUDA;
-    }
     prm.wt = WT;
     prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
     prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
+    prm.dc_carry = dc_carry;
     prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
     prm.kcc = P.kcc; prm.stages = P.stages;
+    prm.i0 = i0; prm.i1 = i1;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
     const cudaError_t e = launch_cluster(rec3::bwd3_kernel, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
@@ -810,10 +860,89 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
     }
-    if (e != cudaSuccess) return LSTM_ERR_CUDA;
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cudaStream_t s) {
+    const long long H = d->H, G4 = 4 * H;
+    dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
+    rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)d->I);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// a3 (+ a5) on the cluster kernel with W_h^T in TMEM (written to the
+// workspace first, then copied into each CTA's tensor memory), one launch.
+int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
+                       const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
+                       const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
+                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+    const long long G4 = 4LL * d->H;
+    if (launch_transpose_wh(d, W, WT, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, gates, cells, dG, WT, dbgroup, dh0,
+                                  dc0, nullptr, ctrl, 0, d->T, s);
+    if (rc != LSTM_OK) return rc;
     simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
     note_launch();
     return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+// a3 + a5 in `nch` reverse-time chunks (one launch each, delta c carried
+// through the workspace) on a high-priority stream, and a4 + a6 of every
+// finished chunk on a low-priority stream, beside the next chunk: the GEMM
+// takes the SMs the recurrence leaves idle (all of them for the last chunk).
+// No kernel waits on another; the streams are ordered by events and joined
+// back into `s` on every return.
+int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int nch,
+                       const bf16 *dy, const bf16 *dhT, const float *dcT, const bf16 *x,
+                       const bf16 *W, const bf16 *h0, const float *c0, const bf16 *y,
+                       const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
+                       float *dbgroup, float *dc_carry, float *dx, float *dW, float *db,
+                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+    std::lock_guard<std::mutex> lock(A.mu);
+    const int T = d->T;
+    const long long G4 = 4LL * d->H;
+    cudaEvent_t ev_fork = A.ev[kMaxChunks], ev_rec = A.ev[kMaxChunks + 1],
+                ev_gemm = A.ev[kMaxChunks + 2];
+    if (cudaEventRecord(ev_fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(A.rec, ev_fork, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(A.gemm, ev_fork, 0) != cudaSuccess)
+        return LSTM_ERR_CUDA;
+    const int gemm_ctas = std::max(1, tcg::sm_count() - P.R * P.KS * P.G);
+    int rc = LSTM_OK;
+    {
+        prof::Phase ph(LSTM_PHASE_BWD_RECUR, A.rec);
+        if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
+        for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
+            const int i0 = (int)((long long)T * c / nch), i1 = (int)((long long)T * (c + 1) / nch);
+            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, gates, cells, dG, WT, dbgroup, dh0, dc0,
+                                dc_carry, ctrl, i0, i1, A.rec);
+            if (rc != LSTM_OK) break;
+            if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
+                cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess) {
+                rc = LSTM_ERR_CUDA;
+                break;
+            }
+            prof::Phase phg(LSTM_PHASE_DW, A.gemm);
+            // rows of time steps T-i1 .. T-i0-1; dW accumulates after the first chunk
+            if (tc_dw_dx(d, dG, x, W, h0, y, dW, dx, ctrl, A.gemm, T - i1, T - i0, c > 0,
+                         c + 1 < nch ? gemm_ctas : 0) != cudaSuccess)
+                rc = LSTM_ERR_CUDA;
+        }
+        if (rc == LSTM_OK) {
+            simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, A.rec>>>(dbgroup, P.G,
+                                                                                 (int)G4, db);
+            note_launch();
+            if (cudaGetLastError() != cudaSuccess) rc = LSTM_ERR_CUDA;
+        }
+    }
+    // join: nothing of this call stays unordered with the caller's stream
+    if (cudaEventRecord(ev_rec, A.rec) != cudaSuccess ||
+        cudaEventRecord(ev_gemm, A.gemm) != cudaSuccess ||
+        cudaStreamWaitEvent(s, ev_rec, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(s, ev_gemm, 0) != cudaSuccess)
+        return LSTM_ERR_CUDA;
+    return rc;
 }
 
 // ------------------------------------------------------------ forward pass
@@ -920,6 +1049,19 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     const bool v3 = plan_bwd3(d, plan3);
     const bool v2 = !v3 && plan_bwd2(d, plan2);
     if (v3 || v2 || plan_bwd_recur(d, plan)) {
+        if (v3 && tc_gemm_ok(d) && bwd_chunks(d) > 1) {
+            AuxStreams *A = aux_streams();
+            if (A) {  // a3 + a5 with a4 + a6 overlapped
+                g_last_bwd_path = 3;
+                const int rc = tc_bwd3_overlapped(
+                    d, plan3, *A, bwd_chunks(d), (const bf16 *)dy, (const bf16 *)dhT, dcT,
+                    (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)y,
+                    (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
+                    (float *)(ws + L.dbgroup), (float *)(ws + L.dc), dx, dW, db, dh0, dc0,
+                    (Ctrl *)ws, s);
+                if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
+            }
+        }
         {   // a3 + a5: persistent tcgen05 recurrence with db fused
             prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
             int rc = LSTM_ERR_NOT_CORESIDENT;
@@ -946,7 +1088,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         if (tc_gemm_ok(d)) {
             prof::Phase ph(LSTM_PHASE_DW, s);
             LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
-                              (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s));
+                              (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0,
+                              d->T, false, 0));
             return LSTM_OK;
         }
         // dW / dx on CUDA cores (shapes off the TMA grid)
@@ -994,7 +1137,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         // a4 + a6 together on the tensor cores (one launch, timed as dW)
         prof::Phase ph(LSTM_PHASE_DW, s);
         LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
-                          (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s));
+                          (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0, d->T,
+                          false, 0));
     } else {
         // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
         prof::Phase ph(LSTM_PHASE_DW, s);

@@ -48,6 +48,7 @@ struct Problem {
     float *out;                // out[m * ldo + out_col0 + n]
     long long ldo;
     int out_col0;
+    int accumulate;            // out += product (otherwise out = product)
     const __nv_bfloat16 *bias; // added per column n, or NULL
     int tiles_n, tile_begin, tile_end;
 };
@@ -247,10 +248,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
                         v[j] = x;
                     }
                     float *orow = P.out + (long long)m * P.ldo + P.out_col0 + nbase + c0;
-                    if (vec8 && nbase + c0 + 32 <= P.N) {
+                    const bool full = nbase + c0 + 32 <= P.N;
+                    if (P.accumulate) {
+                        if (vec && full) {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4) {
+                                const float4 o = *reinterpret_cast<const float4 *>(orow + j);
+                                v[j] += o.x; v[j + 1] += o.y; v[j + 2] += o.z; v[j + 3] += o.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (nbase + c0 + j < P.N) v[j] += orow[j];
+                        }
+                    }
+                    if (vec8 && full) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) tc::st_global_v8(orow + j, v + j);
-                    } else if (vec && nbase + c0 + 32 <= P.N) {
+                    } else if (vec && full) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4)
                             *reinterpret_cast<float4 *>(orow + j) =

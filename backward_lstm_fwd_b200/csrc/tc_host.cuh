@@ -83,7 +83,7 @@ struct Builder {
         Problem &q = P.prob[P.nprob++];
         memset(&q, 0, sizeof(q));
         q.M = M; q.N = N; q.a_mn_major = a_mn; q.b_mn_major = b_mn;
-        q.out = out; q.ldo = ldo; q.out_col0 = out_col0; q.bias = bias;
+        q.out = out; q.ldo = ldo; q.out_col0 = out_col0; q.bias = bias; q.accumulate = 0;
         return q;
     }
     static void add_seg(Problem &q, int a_map, int a_k0, int b_map, int b_k0, long long K) {

@@ -55,8 +55,10 @@ struct Bwd3Params {
     const float *dcT, *cells, *c0;
     __nv_bfloat16 *dG;
     float *dh0, *dc0, *db_part;
+    float *dc_carry;  // [B][H]: delta c between the launches of a chunked call
     Ctrl *ctrl;
     int T, B, H, U, G, NBr, kcc, stages;
+    int i0, i1;       // this launch runs epilogue iterations i0 .. i1-1 (t = T-1-i)
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -103,6 +105,12 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     const int us = cid % p.U, gi = cid / p.U;
     const int j0 = us * UNITS, b0 = gi * p.NBr;
     const int H = p.H, B = p.B, T = p.T, kcc = p.kcc, NBr = p.NBr, stages = p.stages;
+    // A call may run in several launches over consecutive ranges of reverse
+    // time.  Epilogue iteration i >= 1 consumes MMA iteration i; the launch
+    // that ends the call also runs MMA iteration T (delta h_0).
+    const int i0 = p.i0, i1 = p.i1;
+    const bool first = i0 == 0, last = i1 == T;
+    const int mma_lo = i0 > 1 ? i0 : 1, mma_hi = last ? T : i1 - 1;
     const int kslice = kcc * 64;              // this CTA's part of the 4H axis
     const int kbase = (int)kpart * kslice;
     unsigned int *ctr = &p.ctrl->bar[gi];
@@ -135,8 +143,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         if (lane == 0) {
             uint32_t stage = 0, ph = 0;
             bool aborted = false;
-            // MMA iteration i = 1..T consumes dG_{T-i}, written in iteration i-1
-            for (int i = 1; i <= T && !aborted; ++i) {
+            // MMA iteration i consumes dG_{T-i}, written in iteration i-1
+            for (int i = mma_lo; i <= mma_hi && !aborted; ++i) {
                 if (!rec::wait_counter(ctr, group_ctas * (unsigned)i, p.ctrl, abort_flag, 0x601,
                                        p.wait_ns)) {
                     aborted = true;
@@ -180,7 +188,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             // One accumulator suffices: iteration i + 1 starts after the group
             // barrier, which needs this CTA's arrival, which follows the
             // epilogue's reads of iteration i's accumulator.
-            for (int i = 1; ok && i <= T; ++i) {
+            for (int i = mma_lo; ok && i <= mma_hi; ++i) {
                 for (int c = 0; c < kcc; ++c) {
                     if (!tc::mbar_wait(&full[stage], ph, p.ctrl, abort_flag, 0x604, p.wait_ns)) {
                         ok = false;
@@ -236,7 +244,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         float ct[UPT], cp[UPT];
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
-            dc[u] = (valid && p.dcT) ? p.dcT[(long long)b * H + jb + u] : 0.f;
+            const float *dcin = first ? p.dcT : p.dc_carry;
+            dc[u] = (valid && dcin) ? dcin[(long long)b * H + jb + u] : 0.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g) dbacc[g][u] = 0.f;
         }
@@ -338,9 +347,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             return true;
         };
 
-        load_step(T - 1);
+        load_step(T - 1 - i0);
         bool ok = true;
-        for (int i = 0; i < T; ++i) {
+        for (int i = i0; i < i1; ++i) {
             const int t = T - 1 - i;
             float dhr[UPT];
             if (i == 0) {
@@ -402,17 +411,25 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 tc::bulk_wait_read_all();  // the ring is refilled after this arrival
                 if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
             }
-            if (t > 0) load_step(t - 1);
+            if (i + 1 < i1) load_step(t - 1);
         }
         float dh0v[UPT];
-        ok = ok && read_dh(dh0v);  // uniform over the epilogue threads
-        if (ok && valid) {
-            float4 *o = reinterpret_cast<float4 *>(p.dh0 + (long long)b * H + jb);
-            o[0] = make_float4(dh0v[0], dh0v[1], dh0v[2], dh0v[3]);
-            o[1] = make_float4(dh0v[4], dh0v[5], dh0v[6], dh0v[7]);
-            float4 *oc = reinterpret_cast<float4 *>(p.dc0 + (long long)b * H + jb);
-            oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
-            oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
+        if (!last) {
+            if (ok && valid) {  // delta c for the launch that continues the call
+                float4 *oc = reinterpret_cast<float4 *>(p.dc_carry + (long long)b * H + jb);
+                oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
+                oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
+            }
+        } else {
+            ok = ok && read_dh(dh0v);  // uniform over the epilogue threads
+            if (ok && valid) {
+                float4 *o = reinterpret_cast<float4 *>(p.dh0 + (long long)b * H + jb);
+                o[0] = make_float4(dh0v[0], dh0v[1], dh0v[2], dh0v[3]);
+                o[1] = make_float4(dh0v[4], dh0v[5], dh0v[6], dh0v[7]);
+                float4 *oc = reinterpret_cast<float4 *>(p.dc0 + (long long)b * H + jb);
+                oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
+                oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
+            }
         }
         if (et == 0) tc::bulk_wait_all();  // no copy of this CTA in flight from here on
         if (ok) {
@@ -431,7 +448,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 float sum = 0.f;
                 for (int r = 0; r < NMAX; ++r) sum += red[r * 64 + et];
                 const int g = et / UPC, u = et % UPC;
-                p.db_part[(long long)gi * G4 + (long long)g * H + j0 + (int)kpart * UPC + u] = sum;
+                float *dst = p.db_part + (long long)gi * G4 + (long long)g * H + j0 + (int)kpart * UPC + u;
+                *dst = first ? sum : *dst + sum;  // launches of one call run in order
             }
         }
     }

@@ -67,6 +67,9 @@ ODD = [
     # backward with the weights in tensor memory: two ragged batch groups,
     # an odd count of unit slices, and the largest H whose K slice fits TMEM
     (5, 200, 96, 512, "bf16"), (3, 37, 64, 640, "bf16"), (2, 16, 32, 1536, "bf16"),
+    # the backward in reverse-time chunks with dW / dx of each chunk beside the
+    # next one: 37 steps in 2 chunks, chunk row counts off the 64-row K blocks
+    (37, 200, 96, 512, "bf16"),
 ]
 
 
