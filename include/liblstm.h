@@ -25,8 +25,9 @@
  *   - Every pointer is a DEVICE pointer into memory the caller allocated and
  *     owns; it must be 16-byte aligned.  The library allocates no device memory
  *     and keeps no device state between calls; all scratch lives in the
- *     caller's workspace.  (Its only process state is the optional profiling
- *     record and a launch counter, see lstm_profile_begin.)
+ *     caller's workspace.  (Its process state: the optional profiling record,
+ *     a launch counter (see lstm_profile_begin), and per device two internal
+ *     streams and a few events that lstm_bwd creates on first use and keeps.)
  *   - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
  *     stream).  Argument errors are returned synchronously before anything is
  *     enqueued.  Device-side waits that give up record LSTM_ERR_TIMEOUT in the
@@ -113,6 +114,15 @@ int lstm_fwd(const lstm_dims *d, const void *x, const void *W, const void *b,
  *   dh0   [B][H]      float         dL/dinitH (the page's dh_prev at t = 0)
  *   dc0   [B][H]      float         dL/dinitC (the page's dc_prev at t = 0)
  *   ws / ws_bytes                   scratch, >= lstm_bwd_workspace_size(d)
+ *
+ * On the tensor-core path lstm_bwd may run its recurrence and its dW / dx
+ * products on two internal streams of the library (the recurrence at the
+ * device's highest stream priority), so that the products of finished time
+ * chunks run beside the rest of the recurrence.  Those streams start after
+ * the work already enqueued in `stream`, and `stream` waits for both before
+ * anything enqueued after the call: the ordering seen on `stream` is that of
+ * a single-stream call.  Calls from several host threads are serialised while
+ * they enqueue.
  *
  * Returns LSTM_OK or an LSTM_ERR_* code.
  */
