@@ -908,7 +908,10 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         cudaStreamWaitEvent(A.rec, ev_fork, 0) != cudaSuccess ||
         cudaStreamWaitEvent(A.gemm, ev_fork, 0) != cudaSuccess)
         return LSTM_ERR_CUDA;
-    const int gemm_ctas = std::max(1, tcg::sm_count() - P.R * P.KS * P.G);
+    // the GEMM beside the recurrence takes at most the SMs the recurrence
+    // leaves idle (LSTM_BWD_GEMM_CTAS caps it lower, for comparison runs)
+    int gemm_ctas = std::max(1, tcg::sm_count() - P.R * P.KS * P.G);
+    if (const char *e = getenv("LSTM_BWD_GEMM_CTAS")) gemm_ctas = std::max(1, std::min(gemm_ctas, atoi(e)));
     int rc = LSTM_OK;
     {
         prof::Phase ph(LSTM_PHASE_BWD_RECUR, A.rec);

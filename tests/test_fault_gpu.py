@@ -16,12 +16,13 @@ from tests.parity_util import assert_within, compare, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H", [64, 256, 512])
-def test_missing_arrival_times_out_and_recovers(H, cuda_device):
+@pytest.mark.parametrize("H,T", [(64, 6), (256, 6), (512, 6), (512, 40)])
+def test_missing_arrival_times_out_and_recovers(H, T, cuda_device):
+    """T = 40 runs the backward in reverse-time chunks with dW / dx beside them."""
     lbuild.build()
-    w = synth.custom(6, 32, 64, H, "bf16", seed=11)
+    w = synth.custom(T, 32, 64, H, "bf16", seed=11)
     inp = {k: v.to(cuda_device) for k, v in synth.make_inputs(w).items()}
-    T, B, I = w.T, w.B, w.I
+    B, I = w.B, w.I
     st = L.State(T, B, I, H, torch.bfloat16, cuda_device)
     gr = L.Grads(T, B, I, H, cuda_device)
     wsf = L.empty_workspace(L.fwd_workspace_size(st.dims), cuda_device)

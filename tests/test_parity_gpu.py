@@ -141,3 +141,15 @@ def test_side_stream_and_repeat(cuda_device):
         np.testing.assert_array_equal(a[k], b[k])
     assert_within(compare(a, run_oracle(inp), "bf16"), "bf16", "side stream")
 
+
+
+@pytest.mark.parametrize("chunks", ["1", "3", "5"])
+def test_backward_chunk_counts(chunks, cuda_device, monkeypatch):
+    """The backward in 1 (one launch, no overlap), 3 or 5 reverse-time chunks
+    (dW / dx of each chunk beside the next one) gives the oracle's gradients."""
+    monkeypatch.setenv("LSTM_BWD_CHUNKS", chunks)
+    w = synth.custom(41, 40, 64, 512, "bf16", seed=17)
+    inp = synth.make_inputs(w)
+    gpu = run_gpu(inp, cuda_device)
+    assert L.test_last_paths() == (3, 3)
+    assert_within(compare(gpu, run_oracle(inp), "bf16"), "bf16", f"{chunks} chunks")
