@@ -33,6 +33,17 @@
  *   dy[T][B][H], dhT[B][H], dcT[B][H], dx[T][B][I], dW[4H][H+I], db[4H],
  *   dh0[B][H], dc0[B][H].
  *
+ * Variable length ("seq_length", the parameter table's optional mask input of
+ * shape [T][B][H], read as 1 = real step, 0 = padding): at a padded element
+ * the state does not move -- c_t = m c~_t + (1 - m) c_{t-1} and
+ * h_t = m h~_t + (1 - m) h_{t-1}, with c~, h~ the unmasked update, y_t = h_t --
+ * and the backward pass is the exact gradient of that function (padding passes
+ * delta h and delta c through unchanged and has zero gate gradients).  The
+ * page gives no formula for the mask; this reading follows the Darknet LSTM
+ * page's note that padding steps must not update the state or the gradients.
+ * Mask values other than 0 and 1 are outside the reading (the backward uses
+ * tanh of the saved cell state, which equals tanh c~ only where m = 1).
+ *
  * Parity is pinned (tests/test_oracle.py) by central finite differences of the
  * surrogate loss L = sum_t <dy_t, h_t> + <dhT, h_{T-1}> + <dcT, c_{T-1}>,
  * by the T = 1 closed form, the W = 0 closed form, a hand-computed example,
@@ -77,12 +88,13 @@ static double sigm(double a)
 }
 
 /* Forward pass, forward-formula table of "SingleLayerLstmGrad".
- * b, h0, c0 may be NULL (zeros).  Returns 0, or -1 on bad sizes / no memory. */
-int oracle_lstm_fwd(int T, int B, int I, int H,
-                    const double *x, const double *W, const double *b,
-                    const double *h0, const double *c0,
-                    double *y, double *gates, double *cells,
-                    double *hT, double *cT)
+ * b, h0, c0 and mask may be NULL (zeros; no padding).  Returns 0, or -1 on bad
+ * sizes / no memory. */
+int oracle_lstm_fwd_masked(int T, int B, int I, int H,
+                           const double *x, const double *W, const double *b,
+                           const double *h0, const double *c0, const double *mask,
+                           double *y, double *gates, double *cells,
+                           double *hT, double *cT)
 {
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
@@ -106,6 +118,7 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
         for (int t = 0; t < T; ++t) {
             /* input concat: z_t = [h_{t-1}; x_t] */
             const double *xt = x + ((long)t * B + n) * I;
+            const double *mt = mask ? mask + ((long)t * B + n) * H : NULL;
             for (int k = 0; k < I; ++k)
                 z[H + k] = xt[k];
             /* a = W z_t + b for all four gates at once */
@@ -129,6 +142,10 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
                 double o_ = sigm(a[3L * H + j]);      /* output gate */
                 double c_ = f_ * cprev[j] + i_ * g_;  /* cell state */
                 double h_ = o_ * tanh(c_);            /* hidden state */
+                if (mt) {  /* padding keeps the previous state */
+                    c_ = mt[j] * c_ + (1.0 - mt[j]) * cprev[j];
+                    h_ = mt[j] * h_ + (1.0 - mt[j]) * z[j];
+                }
                 gt[j] = i_;
                 gt[H + j] = f_;
                 gt[2L * H + j] = g_;
@@ -148,19 +165,28 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
     return err ? -1 : 0;
 }
 
+int oracle_lstm_fwd(int T, int B, int I, int H,
+                    const double *x, const double *W, const double *b,
+                    const double *h0, const double *c0,
+                    double *y, double *gates, double *cells,
+                    double *hT, double *cT)
+{
+    return oracle_lstm_fwd_masked(T, B, I, H, x, W, b, h0, c0, NULL, y, gates, cells, hT, cT);
+}
+
 /* Backward pass, "backward algorithm (time step t -> t-1)" of
  * "SingleLayerLstmGrad", consuming the forward's saved y, gates and cells.
- * dy, dhT, dcT, h0, c0 may be NULL (zeros).  dG is optional scratch of
- * T*B*4H doubles (allocated here when NULL); on return it holds the
- * pre-activation gate gradients [di | df | dg | do] of every step.
+ * dy, dhT, dcT, h0, c0 and mask may be NULL (zeros; no padding).  dG is
+ * optional scratch of T*B*4H doubles (allocated here when NULL); on return it
+ * holds the pre-activation gate gradients [di | df | dg | do] of every step.
  * Returns 0, or -1 on bad sizes / no memory. */
-int oracle_lstm_bwd(int T, int B, int I, int H,
-                    const double *x, const double *W,
-                    const double *h0, const double *c0,
-                    const double *y, const double *gates, const double *cells,
-                    const double *dy, const double *dhT, const double *dcT,
-                    double *dx, double *dW, double *db,
-                    double *dh0, double *dc0, double *dG)
+int oracle_lstm_bwd_masked(int T, int B, int I, int H,
+                           const double *x, const double *W,
+                           const double *h0, const double *c0, const double *mask,
+                           const double *y, const double *gates, const double *cells,
+                           const double *dy, const double *dhT, const double *dcT,
+                           double *dx, double *dW, double *db,
+                           double *dh0, double *dc0, double *dG)
 {
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
@@ -181,9 +207,10 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
         double *dh_next = (double *)malloc(sizeof(double) * (H > 0 ? H : 1));
         double *dc_next = (double *)malloc(sizeof(double) * (H > 0 ? H : 1));
         double *dz = (double *)malloc(sizeof(double) * (K > 0 ? K : 1));
-        if (!dh_next || !dc_next || !dz) {
+        double *dh_pass = (double *)malloc(sizeof(double) * (H > 0 ? H : 1));
+        if (!dh_next || !dc_next || !dz || !dh_pass) {
             err |= 1;
-            free(dh_next); free(dc_next); free(dz);
+            free(dh_next); free(dc_next); free(dz); free(dh_pass);
             continue;
         }
         /* initialisation: the gradients arriving from time T are the dh / dc
@@ -198,17 +225,23 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
             const double *cp = (t > 0) ? cells + ((long)(t - 1) * B + n) * H
                                        : (c0 ? c0 + (long)n * H : NULL);
             const double *dyt = dy ? dy + ((long)t * B + n) * H : NULL;
+            const double *mt = mask ? mask + ((long)t * B + n) * H : NULL;
             double *dGt = dG + ((long)t * B + n) * G4;
             for (int j = 0; j < H; ++j) {
                 double i_ = gt[j], f_ = gt[H + j], g_ = gt[2L * H + j], o_ = gt[3L * H + j];
                 double c_ = ct[j];
                 double c_prev = cp ? cp[j] : 0.0;
                 double tc = tanh(c_);
-                /* step 1: delta h_t = dL_t/dh_t + delta h_next */
-                double dh = (dyt ? dyt[j] : 0.0) + dh_next[j];
+                double m = mt ? mt[j] : 1.0;
+                /* step 1: delta h_t = dL_t/dh_t + delta h_next; the update h~
+                 * receives the share m, padding passes the rest to h_{t-1} */
+                double dh_tot = (dyt ? dyt[j] : 0.0) + dh_next[j];
+                double dh = m * dh_tot;
+                dh_pass[j] = (1.0 - m) * dh_tot;
                 /* step 2: delta c_t = delta h o (1 - tanh^2 c) + delta c_next,
-                 * where delta c_next already carries the factor f_{t+1} */
-                double dc = dh * o_ * (1.0 - tc * tc) + dc_next[j];
+                 * where delta c_next already carries the factor f_{t+1} (the
+                 * update c~ receives the share m of delta c_next) */
+                double dc = dh * o_ * (1.0 - tc * tc) + m * dc_next[j];
                 /* step 3: pre-activation gate gradients */
                 double d_o = dh * tc * o_ * (1.0 - o_);
                 double d_g = dc * i_ * (1.0 - g_ * g_);
@@ -218,8 +251,8 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
                 dGt[H + j] = d_f;
                 dGt[2L * H + j] = d_g;
                 dGt[3L * H + j] = d_o;
-                /* step 5: delta c_prev = delta c_t * f_t */
-                dc_next[j] = dc * f_;
+                /* step 5: delta c_prev = delta c_t * f_t (+ what padding passes) */
+                dc_next[j] = dc * f_ + (1.0 - m) * dc_next[j];
             }
             /* step 5: delta z_t = sum over gates of W_*^T delta_* = W^T dG_t */
             for (long k = 0; k < K; ++k)
@@ -236,13 +269,13 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
                 dxt[k] = dz[H + k];
             /* step 6: carry delta h_prev into the next (earlier) step */
             for (int j = 0; j < H; ++j)
-                dh_next[j] = dz[j];
+                dh_next[j] = dz[j] + dh_pass[j];
         }
         for (int j = 0; j < H; ++j) {
             if (dh0) dh0[(long)n * H + j] = dh_next[j];  /* dh_prev at t = 0 */
             if (dc0) dc0[(long)n * H + j] = dc_next[j];  /* dc_prev at t = 0 */
         }
-        free(dh_next); free(dc_next); free(dz);
+        free(dh_next); free(dc_next); free(dz); free(dh_pass);
     }
 
     /* Step 4: dW = sum_{t,n} dG_{t,n} z_{t,n}^T and db = sum_{t,n} dG_{t,n},
@@ -275,4 +308,16 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
     if (own_dG)
         free(dG);
     return err ? -1 : 0;
+}
+
+int oracle_lstm_bwd(int T, int B, int I, int H,
+                    const double *x, const double *W,
+                    const double *h0, const double *c0,
+                    const double *y, const double *gates, const double *cells,
+                    const double *dy, const double *dhT, const double *dcT,
+                    double *dx, double *dW, double *db,
+                    double *dh0, double *dc0, double *dG)
+{
+    return oracle_lstm_bwd_masked(T, B, I, H, x, W, h0, c0, NULL, y, gates, cells, dy, dhT, dcT,
+                                  dx, dW, db, dh0, dc0, dG);
 }

@@ -39,19 +39,19 @@ def random_case(T, B, I, H, seed, wscale=1.5, dhdc=True, dy=True):
     return p, g
 
 
-def run(p, g, lib=None):
+def run(p, g, lib=None, mask=None):
     return oracle.lstm_fwd_bwd(p["x"], p["W"], p["b"], p["h0"], p["c0"],
-                               g["dy"], g["dhT"], g["dcT"], lib=lib)
+                               g["dy"], g["dhT"], g["dcT"], lib=lib, mask=mask)
 
 
-def loss(p, g, lib=None):
-    f = oracle.lstm_fwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], lib=lib)
+def loss(p, g, lib=None, mask=None):
+    f = oracle.lstm_fwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], lib=lib, mask=mask)
     return oracle.surrogate_loss(f, g["dy"], g["dhT"], g["dcT"])
 
 
-def fd_max_error(p, g, lib=None, max_entries=None, seed=0):
+def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None):
     """max over checked entries of |analytic - central FD| / max(1, |analytic|)."""
-    out = run(p, g, lib)
+    out = run(p, g, lib, mask)
     rng = np.random.default_rng(seed)
     worst = 0.0
     for name, gname in GRAD_OF.items():
@@ -65,9 +65,9 @@ def fd_max_error(p, g, lib=None, max_entries=None, seed=0):
             old = flat[k]
             h = 1e-6 * max(1.0, abs(old))
             flat[k] = old + h
-            lp = loss(p, g, lib)
+            lp = loss(p, g, lib, mask)
             flat[k] = old - h
-            lm = loss(p, g, lib)
+            lm = loss(p, g, lib, mask)
             flat[k] = old
             fd = (lp - lm) / (2 * h)
             worst = max(worst, abs(fd - an[k]) / max(1.0, abs(an[k])))
@@ -311,3 +311,69 @@ def test_empty_sequence_and_batch():
     out = run(p, g)
     assert out["y"].shape == (3, 0, 4)
     np.testing.assert_array_equal(out["dW"], 0.0)
+
+
+# ---------------------------------------------------------------- seq_length
+# The parameter table's optional "seq_length" mask [T][B][H], read as 1 = real
+# step, 0 = padding: padding keeps the state (c_t = c_{t-1}, h_t = h_{t-1}) and
+# passes delta h / delta c through (the Darknet LSTM page's note that padding
+# must not update state or gradients).
+
+def random_mask(T, B, H, seed, p_pad=0.35):
+    return (np.random.default_rng(seed).random((T, B, H)) >= p_pad).astype(np.float64)
+
+
+@pytest.mark.parametrize("T,B,I,H", [(3, 2, 3, 4), (4, 3, 2, 5), (2, 1, 3, 3)])
+def test_masked_finite_differences(T, B, I, H):
+    """The masked backward is the gradient of the masked forward (0/1 mask per
+    element, fixed while differentiating)."""
+    p, g = random_case(T, B, I, H, seed=300 + T * H)
+    mask = random_mask(T, B, H, seed=7 + T)
+    assert fd_max_error(p, g, mask=mask) < 1e-6
+
+
+def test_mask_all_ones_is_unmasked():
+    p, g = random_case(4, 3, 5, 6, seed=41)
+    a = run(p, g)
+    b = run(p, g, mask=np.ones((4, 3, 6)))
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k], err_msg=k)
+
+
+def test_length_mask_equals_truncated_sequences():
+    """With mask[t, n, :] = (t < L_n) every sequence behaves as the unmasked
+    LSTM run on its first L_n steps: outputs and gradients on those steps agree,
+    padded steps carry the final state and get no input gradient, the dy of
+    padded steps reaches h_{L_n - 1} (its value is carried there), and dW / db
+    are the sums over the truncated runs.  Lengths include 0 and T."""
+    T, B, I, H = 6, 5, 3, 4
+    p, g = random_case(T, B, I, H, seed=77)
+    lengths = [6, 0, 3, 1, 5]
+    mask = np.zeros((T, B, H))
+    for n, L in enumerate(lengths):
+        mask[:L, n, :] = 1.0
+    out = run(p, g, mask=mask)
+    dW = np.zeros_like(out["dW"])
+    db = np.zeros_like(out["db"])
+    for n, L in enumerate(lengths):
+        sl = slice(n, n + 1)
+        q = dict(x=p["x"][:L, sl], W=p["W"], b=p["b"], h0=p["h0"][sl], c0=p["c0"][sl])
+        dhT = g["dhT"][sl] + g["dy"][L:, sl].sum(axis=0)
+        ref = run(q, dict(dy=g["dy"][:L, sl], dhT=dhT, dcT=g["dcT"][sl]))
+        close = lambda a, b: np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+        close(out["y"][:L, sl], ref["y"])
+        close(out["gates"][:L, sl], ref["gates"])
+        close(out["cells"][:L, sl], ref["cells"])
+        close(out["hT"][sl], ref["hT"])
+        close(out["cT"][sl], ref["cT"])
+        for t in range(L, T):  # padding carries the final state
+            close(out["y"][t, sl], ref["hT"])
+            close(out["cells"][t, sl], ref["cT"])
+        close(out["dx"][:L, sl], ref["dx"])
+        assert not out["dx"][L:, sl].any()
+        close(out["dh0"][sl], ref["dh0"])
+        close(out["dc0"][sl], ref["dc0"])
+        dW += ref["dW"]
+        db += ref["db"]
+    np.testing.assert_allclose(out["dW"], dW, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(out["db"], db, rtol=1e-11, atol=1e-12)
