@@ -110,7 +110,7 @@ FwdLayout fwd_layout(const lstm_dims *d) {
 constexpr long long kDbMaxChunks = 2048;
 
 struct BwdLayout {
-    size_t dG, dc, dbpart, wt, dbgroup, total;
+    size_t dG, dc, dhp, dbpart, wt, dbgroup, total;
     int db_chunks, db_rows_per_chunk;
 };
 constexpr int kMaxGroups = 48;
@@ -124,7 +124,9 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     L.db_chunks = (int)(((long long)TB + rows - 1) / rows);
     L.dG = kCtrlBytes;
     L.dc = align_up(L.dG + TB * G4 * esize(d), 256);
-    L.dbpart = align_up(L.dc + 2 * BH * sizeof(float), 256);
+    // delta h that padding passes to h_{t-1} (variable-length calls), ping-pong
+    L.dhp = align_up(L.dc + 2 * BH * sizeof(float), 256);
+    L.dbpart = align_up(L.dhp + 2 * BH * sizeof(float), 256);
     L.wt = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
     L.dbgroup = L.wt;
     L.total = L.wt;
@@ -542,9 +544,11 @@ bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
     return false;
 }
 
-const void *fwd3_kernel_ptr(int NB, int KS) {
-#define LSTM_F3(nb, ks) \
-    if (NB == nb && KS == ks) return (const void *)rec3::fwd3_kernel<nb, ks>;
+const void *fwd3_kernel_ptr(int NB, int KS, bool masked) {
+#define LSTM_F3(nb, ks)                                                                    \
+    if (NB == nb && KS == ks)                                                              \
+        return masked ? (const void *)rec3::fwd3_kernel<nb, ks, true>                      \
+                      : (const void *)rec3::fwd3_kernel<nb, ks, false>;
     LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
     LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
     LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
@@ -556,7 +560,7 @@ const void *fwd3_kernel_ptr(int NB, int KS) {
 // Forward with the input projection fused: the grid of plan_fwd2, and the
 // CTA's W_h and W_x K-slices must fit TMEM beside two accumulators.
 // LSTM_FWD_FUSED_X=0 turns it off (comparison runs).
-bool plan_fwd3(const lstm_dims *d, Rec2Plan &P) {
+bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
     const char *e = getenv("LSTM_FWD_FUSED_X");
     if (e && e[0] == '0') return false;
     if (d->dtype != LSTM_BF16 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
@@ -580,7 +584,7 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P) {
         const int G = (d->B + NB - 1) / NB;
         const size_t smem = rec3::Fwd3Smem(kcc, kcx, NB, KS).total + 1024;
         if (smem > kMaxSmem) continue;
-        const void *kern = fwd3_kernel_ptr(NB, KS);
+        const void *kern = fwd3_kernel_ptr(NB, KS, masked);
         if (!kern) continue;
         const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
         if (G * P.R > maxc) continue;
@@ -645,8 +649,8 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     while (stages >= rec3::MIN_STAGES && (size_t)rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
     if (stages < rec3::MIN_STAGES) return false;
     P.smem = rec3::Bwd3Smem(stages).total + 1024;
-    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel, rec3::THREADS, P.smem,
-                                         P.KS);
+    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel<false>, rec3::THREADS,
+                                         P.smem, P.KS);
     const int gmax = std::min(maxc / P.R, kMaxGroups);
     if (gmax < 1) return false;
     int G = std::min(gmax, (d->B + 15) / 16);
@@ -754,7 +758,10 @@ int tc_fwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *W, con
 
 template <int NB, int KS>
 cudaError_t launch_fwd3_t(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStream_t s) {
-    return launch_cluster(rec3::fwd3_kernel<NB, KS>, prm, P.R * KS * P.G, KS, P.smem, s,
+    if (prm.mask)
+        return launch_cluster(rec3::fwd3_kernel<NB, KS, true>, prm, P.R * KS * P.G, KS, P.smem,
+                              s, rec2::F_THREADS);
+    return launch_cluster(rec3::fwd3_kernel<NB, KS, false>, prm, P.R * KS * P.G, KS, P.smem, s,
                           rec2::F_THREADS);
 }
 
@@ -772,8 +779,9 @@ cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStre
 // a1 + a2 in one cluster kernel (x-part contracted inside the recurrence);
 // LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
 int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, const bf16 *W,
-                       const bf16 *b, const bf16 *h0, const float *c0, bf16 *y, bf16 *hT,
-                       float *cT, bf16 *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
+                       const bf16 *b, const bf16 *h0, const float *c0, const bf16 *mask,
+                       bf16 *y, bf16 *hT, float *cT, bf16 *gates, float *cells, Ctrl *ctrl,
+                       cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, I = d->I;
     rec3::Fwd3Params prm;
     memset(&prm, 0, sizeof(prm));
@@ -783,6 +791,7 @@ int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, con
     else prm.map_h0 = prm.map_y;
     if (!ok) return LSTM_ERR_UNSUPPORTED;
     prm.W = W; prm.bias = b; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
+    prm.mask = mask; prm.h0 = h0;
     prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.I = (int)I; prm.R = P.R; prm.G = P.G;
     prm.kcc = P.kcc; prm.kcx = P.kcx;
@@ -837,9 +846,10 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 // One launch of the TMEM-weight backward kernel over epilogue iterations
 // [i0, i1) (time steps T-i1 .. T-i0-1); WT must already hold W_h^T.
 int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                   const float *dcT, const float *c0, const bf16 *gates, const float *cells,
-                   bf16 *dG, const bf16 *WT, float *dbgroup, float *dh0, float *dc0,
-                   float *dc_carry, Ctrl *ctrl, int i0, int i1, cudaStream_t s) {
+                   const float *dcT, const float *c0, const bf16 *mask, const bf16 *gates,
+                   const float *cells, bf16 *dG, const bf16 *WT, float *dbgroup, float *dh0,
+                   float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0, int i1,
+                   cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
     rec3::Bwd3Params prm;
     memset(&prm, 0, sizeof(prm));
@@ -848,14 +858,18 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const 
     prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
     prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
     prm.dc_carry = dc_carry;
+    prm.mask = mask; prm.dhp_carry = dhp_carry;
     prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
     prm.kcc = P.kcc; prm.stages = P.stages;
     prm.i0 = i0; prm.i1 = i1;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
-    const cudaError_t e = launch_cluster(rec3::bwd3_kernel, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
-                                         rec3::THREADS);
+    const cudaError_t e =
+        mask ? launch_cluster(rec3::bwd3_kernel<true>, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
+                              rec3::THREADS)
+             : launch_cluster(rec3::bwd3_kernel<false>, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
+                              rec3::THREADS);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
@@ -874,13 +888,14 @@ cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cud
 // a3 (+ a5) on the cluster kernel with W_h^T in TMEM (written to the
 // workspace first, then copied into each CTA's tensor memory), one launch.
 int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                       const float *dcT, const bf16 *W, const float *c0, const bf16 *gates,
-                       const float *cells, bf16 *dG, bf16 *WT, float *dbgroup, float *db,
-                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+                       const float *dcT, const bf16 *W, const float *c0, const bf16 *mask,
+                       const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
+                       float *dbgroup, float *db, float *dh0, float *dc0, Ctrl *ctrl,
+                       cudaStream_t s) {
     const long long G4 = 4LL * d->H;
     if (launch_transpose_wh(d, W, WT, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, gates, cells, dG, WT, dbgroup, dh0,
-                                  dc0, nullptr, ctrl, 0, d->T, s);
+    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, gates, cells, dG, WT, dbgroup,
+                                  dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
     if (rc != LSTM_OK) return rc;
     simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
     note_launch();
@@ -895,10 +910,11 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 // back into `s` on every return.
 int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int nch,
                        const bf16 *dy, const bf16 *dhT, const float *dcT, const bf16 *x,
-                       const bf16 *W, const bf16 *h0, const float *c0, const bf16 *y,
-                       const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
-                       float *dbgroup, float *dc_carry, float *dx, float *dW, float *db,
-                       float *dh0, float *dc0, Ctrl *ctrl, cudaStream_t s) {
+                       const bf16 *W, const bf16 *h0, const float *c0, const bf16 *mask,
+                       const bf16 *y, const bf16 *gates, const float *cells, bf16 *dG,
+                       bf16 *WT, float *dbgroup, float *dc_carry, float *dhp_carry, float *dx,
+                       float *dW, float *db, float *dh0, float *dc0, Ctrl *ctrl,
+                       cudaStream_t s) {
     std::lock_guard<std::mutex> lock(A.mu);
     const int T = d->T;
     const long long G4 = 4LL * d->H;
@@ -918,8 +934,8 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
         for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
             const int i0 = (int)((long long)T * c / nch), i1 = (int)((long long)T * (c + 1) / nch);
-            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, gates, cells, dG, WT, dbgroup, dh0, dc0,
-                                dc_carry, ctrl, i0, i1, A.rec);
+            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, gates, cells, dG, WT, dbgroup, dh0,
+                                dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
             if (rc != LSTM_OK) break;
             if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
                 cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess) {
@@ -949,21 +965,24 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
 }
 
 // ------------------------------------------------------------ forward pass
+// mask (variable length) or NULL; masked calls run on the TMEM-weight cluster
+// kernel or the per-step kernels only.
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
-             const float *c0, T *y, T *hT, float *cT, T *gates, float *cells, char *ws,
-             cudaStream_t s) {
+             const float *c0, const T *mask, T *y, T *hT, float *cT, T *gates, float *cells,
+             char *ws, cudaStream_t s) {
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H;
     const FwdLayout L = fwd_layout(d);
     float *Gx = (float *)(ws + L.gx);
     if ((long long)T_ * B > 0 && H > 0) {
         Rec2Plan plan3;
-        if (plan_fwd3(d, plan3)) {  // a1 fused into a2
+        if (plan_fwd3(d, plan3, mask != nullptr)) {  // a1 fused into a2
             prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
             const int rc = tc_fwd_recurrence3(d, plan3, (const bf16 *)x, (const bf16 *)W,
-                                              (const bf16 *)b, (const bf16 *)h0, c0, (bf16 *)y,
-                                              (bf16 *)hT, cT, (bf16 *)gates, cells, (Ctrl *)ws, s);
+                                              (const bf16 *)b, (const bf16 *)h0, c0,
+                                              (const bf16 *)mask, (bf16 *)y, (bf16 *)hT, cT,
+                                              (bf16 *)gates, cells, (Ctrl *)ws, s);
             g_last_fwd_path = 3;
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
         }
@@ -982,7 +1001,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         // a2: the recurrence
         prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
         Rec2Plan plan2;
-        if (plan_fwd2(d, plan2)) {
+        if (!mask && plan_fwd2(d, plan2)) {
             const int rc = tc_fwd_recurrence2(d, plan2, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
                                               (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells,
                                               (Ctrl *)ws, s);
@@ -990,7 +1009,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
         }
         RecPlan plan;
-        if (plan_fwd_recur(d, plan)) {
+        if (!mask && plan_fwd_recur(d, plan)) {
             g_last_fwd_path = 1;
             // persistent tcgen05 kernel: all T steps in one launch; it writes hT and cT
             return tc_fwd_recurrence(d, plan, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
@@ -1004,6 +1023,10 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             const float *cp = t > 0 ? cells + (long long)(t - 1) * BH : c0;
             simt::EpFwdStep<T> ep{Gx + (long long)t * B * 4 * H, cp, y + (long long)t * BH,
                                   gates + (long long)t * B * 4 * H, cells + (long long)t * BH, H};
+            if (mask) {
+                ep.mask = mask + (long long)t * BH;
+                ep.hprev = hp;
+            }
             LSTM_TRY((simt::gemm<true, true>(B, 4 * H, H, simt::Hprev<T>{hp, H},
                                               simt::WhT4<T>{W, H, I}, ep, s)));
         }
@@ -1024,17 +1047,20 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
 }
 
 // ----------------------------------------------------------- backward pass
+// mask (variable length) or NULL; masked calls run on the TMEM-weight cluster
+// kernel or the per-step kernels only.
 template <class T>
 int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, const T *x,
-             const T *W, const T *h0, const float *c0, const T *y, const T *gates,
-             const float *cells, float *dx, float *dW, float *db, float *dh0, float *dc0,
-             char *ws, cudaStream_t s) {
+             const T *W, const T *h0, const float *c0, const T *mask, const T *y,
+             const T *gates, const float *cells, float *dx, float *dW, float *db, float *dh0,
+             float *dc0, char *ws, cudaStream_t s) {
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H, TB = (long long)T_ * B;
     const int G4 = 4 * H, K = H + I;
     const BwdLayout L = bwd_layout(d);
     T *dG = (T *)(ws + L.dG);
     float *dcbuf[2] = {(float *)(ws + L.dc), (float *)(ws + L.dc) + BH};
+    float *dhpbuf[2] = {(float *)(ws + L.dhp), (float *)(ws + L.dhp) + BH};
 
     if (TB == 0 || H == 0) {
         // no step runs: the incoming gradients pass straight through
@@ -1050,18 +1076,20 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     RecPlan plan;
     Rec2Plan plan2, plan3;
     const bool v3 = plan_bwd3(d, plan3);
-    const bool v2 = !v3 && plan_bwd2(d, plan2);
-    if (v3 || v2 || plan_bwd_recur(d, plan)) {
+    const bool v2 = !v3 && !mask && plan_bwd2(d, plan2);
+    const bool v1 = !mask && plan_bwd_recur(d, plan);
+    bool per_step = false;  // a masked call whose cluster kernel cannot be placed
+    if (v3 || v2 || v1) {
         if (v3 && tc_gemm_ok(d) && bwd_chunks(d) > 1) {
             AuxStreams *A = aux_streams();
             if (A) {  // a3 + a5 with a4 + a6 overlapped
                 g_last_bwd_path = 3;
                 const int rc = tc_bwd3_overlapped(
                     d, plan3, *A, bwd_chunks(d), (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                    (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)y,
-                    (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
-                    (float *)(ws + L.dbgroup), (float *)(ws + L.dc), dx, dW, db, dh0, dc0,
-                    (Ctrl *)ws, s);
+                    (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)mask,
+                    (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
+                    (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), (float *)(ws + L.dc),
+                    (float *)(ws + L.dhp), dx, dW, db, dh0, dc0, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
             }
         }
@@ -1071,43 +1099,47 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
             g_last_bwd_path = v3 ? 3 : 2;
             if (v3)
                 rc = tc_bwd_recurrence3(d, plan3, (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                                        (const bf16 *)W, c0, (const bf16 *)gates, cells,
-                                        (bf16 *)dG, (bf16 *)(ws + L.wt),
-                                        (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
+                                        (const bf16 *)W, c0, (const bf16 *)mask,
+                                        (const bf16 *)gates, cells, (bf16 *)dG,
+                                        (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), db, dh0,
+                                        dc0, (Ctrl *)ws, s);
             else if (v2)
                 rc = tc_bwd_recurrence2(d, plan2, (const bf16 *)dy, (const bf16 *)dhT, dcT,
                                         (const bf16 *)W, c0, (const bf16 *)gates, cells,
                                         (bf16 *)dG, (bf16 *)(ws + L.wt),
                                         (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
-            if (rc == LSTM_ERR_NOT_CORESIDENT && plan_bwd_recur(d, plan)) {
+            if (rc == LSTM_ERR_NOT_CORESIDENT && v1) {
                 g_last_bwd_path = 1;
                 rc = tc_bwd_recurrence(
                 d, plan, (const bf16 *)dy, (const bf16 *)dhT, dcT, (const bf16 *)W, c0,
                 (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
                 (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
             }
-            if (rc != LSTM_OK) return rc;
+            if (rc == LSTM_ERR_NOT_CORESIDENT && mask) per_step = true;
+            else if (rc != LSTM_OK) return rc;
         }
-        if (tc_gemm_ok(d)) {
-            prof::Phase ph(LSTM_PHASE_DW, s);
-            LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
-                              (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0,
-                              d->T, false, 0));
+        if (!per_step) {
+            if (tc_gemm_ok(d)) {
+                prof::Phase ph(LSTM_PHASE_DW, s);
+                LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
+                                  (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0,
+                                  d->T, false, 0));
+                return LSTM_OK;
+            }
+            // dW / dx on CUDA cores (shapes off the TMA grid)
+            {
+                prof::Phase ph(LSTM_PHASE_DW, s);
+                LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
+                                                    simt::Zrows<T>{x, y, h0, B, I, H},
+                                                    simt::EpStore{dW, K}, s)));
+            }
+            prof::Phase ph(LSTM_PHASE_DX, s);
+            if (I > 0)
+                LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
+                                                   simt::RowMajor<T>{W + H, K},
+                                                   simt::EpStore{dx, I}, s)));
             return LSTM_OK;
         }
-        // dW / dx on CUDA cores (shapes off the TMA grid)
-        {
-            prof::Phase ph(LSTM_PHASE_DW, s);
-            LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
-                                                simt::Zrows<T>{x, y, h0, B, I, H},
-                                                simt::EpStore{dW, K}, s)));
-        }
-        prof::Phase ph(LSTM_PHASE_DX, s);
-        if (I > 0)
-            LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
-                                               simt::RowMajor<T>{W + H, K},
-                                               simt::EpStore{dx, I}, s)));
-        return LSTM_OK;
     }
 
     // a3: reverse-time recursion, steps 1-3 and 5 fused with delta h = W_h^T dG_{t+1}
@@ -1127,13 +1159,20 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         ep.dc_out = (t == 0) ? dc0 : dcbuf[t & 1];
         ep.H = H;
         ep.use_acc = !last;
+        if (mask) {
+            ep.mask = mask + (long long)t * BH;
+            ep.dhp_in = last ? nullptr : dhpbuf[(t + 1) & 1];
+            ep.dhp_out = dhpbuf[t & 1];
+        }
         const T *dGn = last ? dG : dG + (long long)(t + 1) * B * G4;
         LSTM_TRY((simt::gemm<true, false>(B, H, last ? 0 : G4, simt::RowMajor<T>{dGn, G4},
                                            simt::RowMajor<T>{W, K}, ep, s)));
     }
-    // dinitH = W_h^T dG_0 (delta h_prev at t = 0, step 5)
+    // dinitH = W_h^T dG_0 (delta h_prev at t = 0, step 5), plus what padding at
+    // t = 0 passes on
     LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG, G4},
-                                       simt::RowMajor<T>{W, K}, simt::EpStore{dh0, H}, s)));
+                                       simt::RowMajor<T>{W, K},
+                                       simt::EpStore{dh0, H, mask ? dhpbuf[0] : nullptr}, s)));
     }
     const bool tc = tc_gemm_ok(d);
     if (tc) {
@@ -1202,6 +1241,63 @@ int noalloc_scratch(void **out) {
 }  // namespace
 
 // =================================================================== C ABI
+namespace {
+int fwd_entry(const lstm_dims *d, const void *x, const void *W, const void *b, const void *h0,
+              const float *c0, const void *mask, void *y, void *hT, float *cT, void *gates,
+              float *cells, void *ws, size_t ws_bytes, void *stream) {
+    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
+    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
+    if (!ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(b, false) ||
+        !ptr_ok(h0, false) || !ptr_ok(c0, false) || !ptr_ok(mask, false) ||
+        !ptr_ok(y, TB * d->H > 0) || !ptr_ok(hT, BH > 0) || !ptr_ok(cT, BH > 0) ||
+        !ptr_ok(gates, TB * d->H > 0) || !ptr_ok(cells, TB * d->H > 0))
+        return LSTM_ERR_INVALID_ARG;
+    const int wsrc = ws_ok(ws, ws_bytes, fwd_layout(d).total);
+    if (wsrc != LSTM_OK) return wsrc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (d->dtype == LSTM_F32)
+        return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
+                               (const float *)h0, c0, (const float *)mask, (float *)y,
+                               (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
+    typedef __nv_bfloat16 bf;
+    return fwd_simt<bf>(d, (const bf *)x, (const bf *)W, (const bf *)b, (const bf *)h0, c0,
+                        (const bf *)mask, (bf *)y, (bf *)hT, cT, (bf *)gates, cells, (char *)ws,
+                        s);
+}
+
+int bwd_entry(const lstm_dims *d, const void *mask, const void *dy, const void *dhT,
+              const float *dcT, const void *x, const void *W, const void *h0, const float *c0,
+              const void *y, const void *gates, const float *cells, float *dx, float *dW,
+              float *db, float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream) {
+    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
+    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
+    const long long G4 = 4LL * d->H, K = (long long)d->H + d->I;
+    if (!ptr_ok(mask, false) || !ptr_ok(dy, false) || !ptr_ok(dhT, false) ||
+        !ptr_ok(dcT, false) || !ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) ||
+        !ptr_ok(h0, false) || !ptr_ok(c0, false) || !ptr_ok(y, TB * d->H > 0) ||
+        !ptr_ok(gates, TB * d->H > 0) || !ptr_ok(cells, TB * d->H > 0) ||
+        !ptr_ok(dx, TB * d->I > 0) || !ptr_ok(dW, G4 * K > 0) || !ptr_ok(db, G4 > 0) ||
+        !ptr_ok(dh0, BH > 0) || !ptr_ok(dc0, BH > 0))
+        return LSTM_ERR_INVALID_ARG;
+    const int wsrc = ws_ok(ws, ws_bytes, bwd_layout(d).total);
+    if (wsrc != LSTM_OK) return wsrc;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    if (d->dtype == LSTM_F32)
+        return bwd_simt<float>(d, (const float *)dy, (const float *)dhT, dcT, (const float *)x,
+                               (const float *)W, (const float *)h0, c0, (const float *)mask,
+                               (const float *)y, (const float *)gates, cells, dx, dW, db, dh0,
+                               dc0, (char *)ws, s);
+    typedef __nv_bfloat16 bf;
+    return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
+                        (const bf *)h0, c0, (const bf *)mask, (const bf *)y, (const bf *)gates,
+                        cells, dx, dW, db, dh0, dc0, (char *)ws, s);
+}
+}  // namespace
+
 extern "C" {
 
 int lstm_abi_version(void) { return 100; }
@@ -1229,58 +1325,35 @@ size_t lstm_bwd_workspace_size(const lstm_dims *d) {
     return bwd_layout(d).total;
 }
 
+
 int lstm_fwd(const lstm_dims *d, const void *x, const void *W, const void *b, const void *h0,
              const float *c0, void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
              size_t ws_bytes, void *stream) {
-    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
-    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
-    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
-    if (!ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(b, false) ||
-        !ptr_ok(h0, false) || !ptr_ok(c0, false) || !ptr_ok(y, TB * d->H > 0) ||
-        !ptr_ok(hT, BH > 0) || !ptr_ok(cT, BH > 0) || !ptr_ok(gates, TB * d->H > 0) ||
-        !ptr_ok(cells, TB * d->H > 0))
-        return LSTM_ERR_INVALID_ARG;
-    const int wsrc = ws_ok(ws, ws_bytes, fwd_layout(d).total);
-    if (wsrc != LSTM_OK) return wsrc;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    if (d->dtype == LSTM_F32)
-        return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
-                               (const float *)h0, c0, (float *)y, (float *)hT, cT,
-                               (float *)gates, cells, (char *)ws, s);
-    return fwd_simt<__nv_bfloat16>(d, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)W,
-                                   (const __nv_bfloat16 *)b, (const __nv_bfloat16 *)h0, c0,
-                                   (__nv_bfloat16 *)y, (__nv_bfloat16 *)hT, cT,
-                                   (__nv_bfloat16 *)gates, cells, (char *)ws, s);
+    return fwd_entry(d, x, W, b, h0, c0, nullptr, y, hT, cT, gates, cells, ws, ws_bytes, stream);
+}
+
+int lstm_fwd_masked(const lstm_dims *d, const void *x, const void *W, const void *b,
+                    const void *h0, const float *c0, const void *mask, void *y, void *hT,
+                    float *cT, void *gates, float *cells, void *ws, size_t ws_bytes,
+                    void *stream) {
+    return fwd_entry(d, x, W, b, h0, c0, mask, y, hT, cT, gates, cells, ws, ws_bytes, stream);
 }
 
 int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *dcT,
              const void *x, const void *W, const void *h0, const float *c0, const void *y,
              const void *gates, const float *cells, float *dx, float *dW, float *db,
              float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream) {
-    if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
-    if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
-    const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
-    const long long G4 = 4LL * d->H, K = (long long)d->H + d->I;
-    if (!ptr_ok(dy, false) || !ptr_ok(dhT, false) || !ptr_ok(dcT, false) ||
-        !ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(h0, false) ||
-        !ptr_ok(c0, false) || !ptr_ok(y, TB * d->H > 0) || !ptr_ok(gates, TB * d->H > 0) ||
-        !ptr_ok(cells, TB * d->H > 0) || !ptr_ok(dx, TB * d->I > 0) ||
-        !ptr_ok(dW, G4 * K > 0) || !ptr_ok(db, G4 > 0) || !ptr_ok(dh0, BH > 0) ||
-        !ptr_ok(dc0, BH > 0))
-        return LSTM_ERR_INVALID_ARG;
-    const int wsrc = ws_ok(ws, ws_bytes, bwd_layout(d).total);
-    if (wsrc != LSTM_OK) return wsrc;
-    cudaStream_t s = (cudaStream_t)stream;
-    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    if (d->dtype == LSTM_F32)
-        return bwd_simt<float>(d, (const float *)dy, (const float *)dhT, dcT, (const float *)x,
-                               (const float *)W, (const float *)h0, c0, (const float *)y,
-                               (const float *)gates, cells, dx, dW, db, dh0, dc0, (char *)ws, s);
-    typedef __nv_bfloat16 bf;
-    return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
-                        (const bf *)h0, c0, (const bf *)y, (const bf *)gates, cells, dx, dW, db,
-                        dh0, dc0, (char *)ws, s);
+    return bwd_entry(d, nullptr, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0,
+                     dc0, ws, ws_bytes, stream);
+}
+
+int lstm_bwd_masked(const lstm_dims *d, const void *mask, const void *dy, const void *dhT,
+                    const float *dcT, const void *x, const void *W, const void *h0,
+                    const float *c0, const void *y, const void *gates, const float *cells,
+                    float *dx, float *dW, float *db, float *dh0, float *dc0, void *ws,
+                    size_t ws_bytes, void *stream) {
+    return bwd_entry(d, mask, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0,
+                     ws, ws_bytes, stream);
 }
 
 int lstm_profile_begin(void) {

@@ -160,6 +160,10 @@ template <class T> struct EpFwdStep {
     const float *cprev;         // cells[t-1] or c0 (may be NULL), [B][H]
     T *y; T *gates; float *cells;  // step-t slices: [B][H], [B][4H], [B][H]
     int H;
+    // variable length: mask[t] [B][H] (1 = real step, 0 = padding, which keeps
+    // h_{t-1} = y[t-1] or h0, and c_{t-1}); NULL = every step real
+    const T *mask = nullptr;
+    const T *hprev = nullptr;
     __device__ void operator()(int m, int q0, const float *acc) const {
         const int j = q0 >> 2;
         if (j >= H) return;
@@ -169,8 +173,14 @@ template <class T> struct EpFwdStep {
         const float gg = tanhf_(acc[2] + gx[2 * H + j]);
         const float og = sigmoidf_(acc[3] + gx[3 * H + j]);
         const float cp = cprev ? cprev[(long long)m * H + j] : 0.f;
-        const float c = fg * cp + ig * gg;
-        const float h = og * tanhf_(c);
+        float c = fg * cp + ig * gg;
+        float h = og * tanhf_(c);
+        if (mask) {
+            const float mk = to_f(mask[(long long)m * H + j]);
+            const float hp = hprev ? to_f(hprev[(long long)m * H + j]) : 0.f;
+            c = mk * c + (1.f - mk) * cp;
+            h = mk * h + (1.f - mk) * hp;
+        }
         T *gt = gates + (long long)m * 4 * H;
         gt[j] = from_f<T>(ig);
         gt[H + j] = from_f<T>(fg);
@@ -193,6 +203,12 @@ template <class T> struct EpBwdStep {
     T *dG;              // dG[t] [B][4H]
     float *dc_out;      // delta c_prev [B][H]
     int H; bool use_acc;
+    // variable length: mask[t] [B][H] (NULL = every step real); padding passes
+    // the share (1 - m) of delta h to h_{t-1} through dhp_out (read back as
+    // dhp_in one step earlier) and of delta c_next to c_{t-1}
+    const T *mask = nullptr;
+    const float *dhp_in = nullptr;
+    float *dhp_out = nullptr;
     __device__ void operator()(int m, int n0, const float *acc) const {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -201,7 +217,18 @@ template <class T> struct EpBwdStep {
             const long long o = (long long)m * H + j;
             float dh = dy ? to_f(dy[o]) : 0.f;                       // step 1
             dh += use_acc ? acc[c] : (dh_in ? to_f(dh_in[o]) : 0.f);
-            const float dcn = dc_in ? dc_in[o] : 0.f;
+            if (dhp_in) dh += dhp_in[o];
+            float dcn = dc_in ? dc_in[o] : 0.f;
+            float mk = 1.f;
+            // (__fmul_rn: no contraction into the sums below, so that m = 1
+            // rounds exactly as an unmasked call does)
+            if (mask) {
+                mk = to_f(mask[o]);
+                dhp_out[o] = __fmul_rn(1.f - mk, dh);
+                dh = __fmul_rn(dh, mk);
+            }
+            const float dc_pass = __fmul_rn(1.f - mk, dcn);
+            dcn = __fmul_rn(dcn, mk);
             const T *g4 = gates + (long long)m * 4 * H;
             const float ig = to_f(g4[j]), fg = to_f(g4[H + j]);
             const float gg = to_f(g4[2 * H + j]), og = to_f(g4[3 * H + j]);
@@ -218,18 +245,22 @@ template <class T> struct EpBwdStep {
             d4[H + j] = from_f<T>(d_f);
             d4[2 * H + j] = from_f<T>(d_g);
             d4[3 * H + j] = from_f<T>(d_o);
-            dc_out[o] = dc * fg;                                       // step 5
+            dc_out[o] = dc * fg + dc_pass;                             // step 5
         }
     }
 };
 
-// Plain float store of the GEMM result: out[m][n], row stride N.
+// Plain float store of the GEMM result: out[m][n], row stride N (plus
+// add[m][n] when add is not NULL).
 struct EpStore {
     float *out; int N;
+    const float *add = nullptr;
     __device__ void operator()(int m, int n0, const float *acc) const {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-            if (n0 + c < N) out[(long long)m * N + n0 + c] = acc[c];
+            if (n0 + c < N)
+                out[(long long)m * N + n0 + c] =
+                    acc[c] + (add ? add[(long long)m * N + n0 + c] : 0.f);
     }
 };
 

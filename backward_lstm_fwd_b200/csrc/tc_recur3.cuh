@@ -56,6 +56,11 @@ struct Bwd3Params {
     __nv_bfloat16 *dG;
     float *dh0, *dc0, *db_part;
     float *dc_carry;  // [B][H]: delta c between the launches of a chunked call
+    // variable length (MASKED kernels): mask [T][B][H] bf16, 1 = real step,
+    // 0 = padding; dhp_carry [B][H]: the delta h that padding passes to
+    // h_{t-1}, between the launches of a chunked call
+    const __nv_bfloat16 *mask;
+    float *dhp_carry;
     Ctrl *ctrl;
     int T, B, H, U, G, NBr, kcc, stages;
     int i0, i1;       // this launch runs epilogue iterations i0 .. i1-1 (t = T-1-i)
@@ -83,6 +88,7 @@ __device__ __forceinline__ int part_off(int r, int n) {
     return r * NMAX + ((((n >> 2) ^ (r & 7)) << 2) | (n & 3));
 }
 
+template <bool MASKED>
 __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant__ Bwd3Params p) {
     constexpr int UPT = 8;  // units per epilogue thread in the pointwise part
     extern __shared__ uint8_t smem_raw[];
@@ -241,11 +247,14 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
         float dc[UPT], dbacc[4][UPT];
         uint4 gpk[4], dypk;  // prefetched gates and dy of the next step, still packed bf16
+        uint4 mpk;           // and its mask (MASKED)
         float ct[UPT], cp[UPT];
+        float dhp[UPT];      // delta h that padding passes to h_{t-1} (MASKED)
 #pragma unroll
         for (int u = 0; u < UPT; ++u) {
             const float *dcin = first ? p.dcT : p.dc_carry;
             dc[u] = (valid && dcin) ? dcin[(long long)b * H + jb + u] : 0.f;
+            dhp[u] = (MASKED && !first && valid) ? p.dhp_carry[(long long)b * H + jb + u] : 0.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g) dbacc[g][u] = 0.f;
         }
@@ -256,6 +265,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
 #pragma unroll
                 for (int g = 0; g < 4; ++g) gpk[g] = make_uint4(0, 0, 0, 0);
                 dypk = make_uint4(0, 0, 0, 0);
+                mpk = make_uint4(0, 0, 0, 0);
                 return;
             }
             const long long row = (long long)t * B + b;
@@ -279,6 +289,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             }
             dypk = p.dy ? __ldg(reinterpret_cast<const uint4 *>(p.dy + row * H + jb))
                         : make_uint4(0, 0, 0, 0);
+            if (MASKED) mpk = __ldg(reinterpret_cast<const uint4 *>(p.mask + row * H + jb));
         };
         // delta h of row m, units uo..uo+7 from MMA iteration i: each thread
         // moves its accumulator row (one unit, 64 batch rows) to the block of
@@ -369,17 +380,29 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
 #pragma unroll
             for (int g = 0; g < 4; ++g) rec::bf16x8_to_f32(gpk[g], gv[g]);
             rec::bf16x8_to_f32(dypk, dyv);
+            float mkv[UPT];
+            if (MASKED) rec::bf16x8_to_f32(mpk, mkv);
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const float ig = gv[0][u], fg = gv[1][u], gg = gv[2][u], og = gv[3][u];
-                const float dh = dyv[u] + dhr[u];                       // step 1
+                float dh = dyv[u] + dhr[u];                             // step 1
+                float dcn = dc[u], dc_pass = 0.f;
+                if (MASKED) {  // padding: the share 1 - m passes to h_{t-1}, c_{t-1}
+                    // (__fmul_rn: no contraction into the sums below, so that
+                    // m = 1 rounds exactly as the unmasked kernel does)
+                    dh += dhp[u];
+                    dhp[u] = __fmul_rn(1.f - mkv[u], dh);
+                    dh = __fmul_rn(dh, mkv[u]);
+                    dc_pass = __fmul_rn(1.f - mkv[u], dcn);
+                    dcn = __fmul_rn(dcn, mkv[u]);
+                }
                 const float tc_ = rec::tanh_fast(ct[u]);
-                const float dcv = dh * og * (1.f - tc_ * tc_) + dc[u];  // step 2
+                const float dcv = dh * og * (1.f - tc_ * tc_) + dcn;    // step 2
                 dO[u] = dh * tc_ * og * (1.f - og);                     // step 3
                 dGg[u] = dcv * ig * (1.f - gg * gg);
                 dI[u] = dcv * gg * ig * (1.f - ig);
                 dF[u] = dcv * cp[u] * fg * (1.f - fg);
-                dc[u] = dcv * fg;                                       // step 5
+                dc[u] = dcv * fg + dc_pass;                             // step 5
             }
             {
                 const uint4 vi = rec::f32x8_to_bf16(dI), vf = rec::f32x8_to_bf16(dF);
@@ -415,13 +438,22 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         }
         float dh0v[UPT];
         if (!last) {
-            if (ok && valid) {  // delta c for the launch that continues the call
+            if (ok && valid) {  // delta c (and delta h passed by padding) for the next launch
                 float4 *oc = reinterpret_cast<float4 *>(p.dc_carry + (long long)b * H + jb);
                 oc[0] = make_float4(dc[0], dc[1], dc[2], dc[3]);
                 oc[1] = make_float4(dc[4], dc[5], dc[6], dc[7]);
+                if (MASKED) {
+                    float4 *oh = reinterpret_cast<float4 *>(p.dhp_carry + (long long)b * H + jb);
+                    oh[0] = make_float4(dhp[0], dhp[1], dhp[2], dhp[3]);
+                    oh[1] = make_float4(dhp[4], dhp[5], dhp[6], dhp[7]);
+                }
             }
         } else {
             ok = ok && read_dh(dh0v);  // uniform over the epilogue threads
+            if (MASKED) {
+#pragma unroll
+                for (int u = 0; u < UPT; ++u) dh0v[u] += dhp[u];
+            }
             if (ok && valid) {
                 float4 *o = reinterpret_cast<float4 *>(p.dh0 + (long long)b * H + jb);
                 o[0] = make_float4(dh0v[0], dh0v[1], dh0v[2], dh0v[3]);
@@ -476,6 +508,9 @@ struct Fwd3Params {
     const __nv_bfloat16 *W;           // [4H][H + I]: W_h | W_x
     const __nv_bfloat16 *bias;        // [4H] or NULL
     const float *c0;
+    // variable length (MASKED kernels): mask [T][B][H], 1 = real step,
+    // 0 = padding (which keeps h_{t-1}, c_{t-1}); h0 [B][H] or NULL
+    const __nv_bfloat16 *mask, *h0;
     __nv_bfloat16 *y, *gates, *hT;
     float *cells, *cT;
     Ctrl *ctrl;
@@ -512,7 +547,7 @@ struct Fwd3Smem {
     }
 };
 
-template <int NB, int KS>
+template <int NB, int KS, bool MASKED>
 __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params p) {
     using rec2::F_ROWS;
     using rec2::F_UNITS;
@@ -753,16 +788,28 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
         // pointwise pairs of this thread: pair index et + 256 k -> unit, column
         float c[NP], bias[4][NP];
+        float hprev[NP], mk[NP];  // MASKED: h_{t-1} of each pair, and step t's mask
         auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
         auto pair_col = [&](int k) { return (et + F_EPI_THREADS * k) >> 5; };
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
             const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
-            c[k] = (p.c0 && n < NBc && b < B) ? p.c0[(long long)b * H + j] : 0.f;
+            const bool v = n < NBc && b < B;
+            c[k] = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
+            if (MASKED) hprev[k] = (p.h0 && v) ? __bfloat162float(p.h0[(long long)b * H + j]) : 0.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 bias[g][k] = p.bias ? __bfloat162float(p.bias[g * H + j]) : 0.f;
         }
+        auto load_mask = [&](int t) {
+#pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+                mk[k] = (n < NBc && b < B)
+                            ? __bfloat162float(p.mask[((long long)t * B + b) * H + j]) : 0.f;
+            }
+        };
+        if (MASKED) load_mask(0);
         uint32_t dph[2] = {0, 0}, rph = 0;
         for (int t = 0; t < T; ++t) {
             const int acc = t & 1;
@@ -858,8 +905,15 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 const float fg = rec::sigmoid_fast(xbuf[(1 * NBc + n) * F_UNITS + uu] + bias[1][k]);
                 const float gg = rec::tanh_fast(xbuf[(2 * NBc + n) * F_UNITS + uu] + bias[2][k]);
                 const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
-                c[k] = fg * c[k] + ig * gg;
-                const float h = og * rec::tanh_fast(c[k]);
+                const float cn = fg * c[k] + ig * gg;
+                float h = og * rec::tanh_fast(cn);
+                if (MASKED) {  // padding keeps the previous state
+                    c[k] = mk[k] * cn + (1.f - mk[k]) * c[k];
+                    h = mk[k] * h + (1.f - mk[k]) * hprev[k];
+                    hprev[k] = h;
+                } else {
+                    c[k] = cn;
+                }
                 gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
                 if (b < B) {
                     const long long o = (long long)b * H + j;
@@ -891,6 +945,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 g4[2 * H] = __float2bfloat16_rn(gsave[2][k]);
                 g4[3 * H] = __float2bfloat16_rn(gsave[3][k]);
             }
+            if (MASKED && t + 1 < T) load_mask(t + 1);
         }
         if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
     }

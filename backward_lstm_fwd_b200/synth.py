@@ -104,7 +104,7 @@ def select_sequences(inputs: Dict[str, torch.Tensor], idx: Sequence[int]) -> Dic
     ix = torch.as_tensor(list(idx), dtype=torch.long)
     out = {}
     for k, v in inputs.items():
-        if k in ("x", "dy"):
+        if k in ("x", "dy", "mask"):
             out[k] = v.index_select(1, ix).contiguous()
         elif k in ("h0", "c0", "dhT", "dcT"):
             out[k] = v.index_select(0, ix).contiguous()
@@ -116,3 +116,30 @@ def select_sequences(inputs: Dict[str, torch.Tensor], idx: Sequence[int]) -> Dic
 def as_float64(inputs: Dict[str, torch.Tensor]):
     """Exact widening of every input to float64 numpy arrays (what the oracle reads)."""
     return {k: v.double().numpy() for k, v in inputs.items()}
+
+
+# ------------------------------------------------------------- variable length
+def random_lengths(T: int, B: int, seed: int) -> list:
+    """Per-sequence lengths in 0..T, seeded; the first three sequences (when
+    there are that many) take the edge lengths T, 0 and 1."""
+    g = torch.Generator().manual_seed(seed)
+    lengths = torch.randint(0, T + 1, (B,), generator=g).tolist()
+    for n, L in enumerate([T, 0, 1][:B]):
+        lengths[n] = min(L, T)
+    return lengths
+
+
+def length_mask(T: int, B: int, H: int, lengths, dtype: str) -> torch.Tensor:
+    """Mask [T][B][H] with 1 on the first lengths[n] steps of sequence n and 0
+    on the padding after them (the seq_length input, in the compute type)."""
+    m = torch.zeros(T, B, H)
+    for n, L in enumerate(lengths):
+        m[:L, n, :] = 1.0
+    return m.to(torch_dtype(dtype)).contiguous()
+
+
+def random_mask(T: int, B: int, H: int, dtype: str, seed: int, p_pad: float = 0.3) -> torch.Tensor:
+    """Element-wise random 0/1 mask [T][B][H] (padding with probability p_pad)."""
+    g = torch.Generator().manual_seed(seed)
+    m = (torch.rand(T, B, H, generator=g) >= p_pad).float()
+    return m.to(torch_dtype(dtype)).contiguous()

@@ -210,9 +210,12 @@ def run_ours(args, w, rank, world, local_rank):
         import torch.distributed as dist
 
     inputs = synth.make_inputs(w)
+    T, B, I, H = w.T, w.B, w.I, w.H
+    if args.seq_mask:  # variable length: seeded per-sequence lengths in 0..T
+        inputs["mask"] = synth.length_mask(T, B, H, synth.random_lengths(T, B, seed=w.seed),
+                                           w.dtype)
     d = {k: v.to(dev) for k, v in inputs.items()}
     cd = synth.torch_dtype(w.dtype)
-    T, B, I, H = w.T, w.B, w.I, w.H
     st = L.State(T, B, I, H, cd, dev)
     gr = L.Grads(T, B, I, H, dev)
     dims = st.dims
@@ -223,10 +226,10 @@ def run_ours(args, w, rank, world, local_rank):
 
     def step(src):
         L.lstm_fwd(dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT, st.cT,
-                   st.gates, st.cells, ws_f, stream=stream)
+                   st.gates, st.cells, ws_f, stream=stream, mask=src.get("mask"))
         L.lstm_bwd(dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
                    src["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0,
-                   ws_b, stream=stream)
+                   ws_b, stream=stream, mask=src.get("mask"))
 
     def barrier():
         if dist is not None:
@@ -301,10 +304,10 @@ def run_ours(args, w, rank, world, local_rank):
             src = dev_in[i]
             g = grads[i]
             L.lstm_fwd(dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT,
-                       st.cT, st.gates, st.cells, ws_f, stream=stream)
+                       st.cT, st.gates, st.cells, ws_f, stream=stream, mask=src.get("mask"))
             L.lstm_bwd(dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
                        src["c0"], st.y, st.gates, st.cells, g.dx, g.dW, g.db, g.dh0, g.dc0,
-                       ws_b, stream=stream)
+                       ws_b, stream=stream, mask=src.get("mask"))
         in_free[i].record(stream)
         out_ready[i].record(stream)
         s_d2h.wait_event(out_ready[i])
@@ -377,6 +380,10 @@ def run_ours(args, w, rank, world, local_rank):
                 "overlap": "uploads and read-backs on their own streams, two buffer sets"},
         "clocks": clk,
     }
+    if args.seq_mask:
+        real = float(inputs["mask"][:, :, 0].float().mean())
+        line["config"]["seq_mask"] = (f"per-sequence lengths uniform in 0..T (seeded), "
+                                      f"{100 * real:.0f} % of the T*B steps real; all counted")
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, inputs)
     print(json.dumps(line), flush=True)
@@ -393,6 +400,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override T (profiling aid: same per-step shape, fewer steps)")
+    ap.add_argument("--seq-mask", action="store_true",
+                    help="variable length: a seq_length mask with seeded per-sequence "
+                         "lengths in 0..T (every step is still computed and counted)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     if args.seq_len is not None:
