@@ -57,10 +57,10 @@ def _bind(path: str):
     lib.oracle_lstm_fwd.restype = i
     lib.oracle_lstm_bwd.argtypes = [i, i, i, i] + [dp] * 9 + [dp] * 6
     lib.oracle_lstm_bwd.restype = i
-    lib.oracle_lstm_fwd_masked.argtypes = [i, i, i, i] + [dp] * 6 + [dp] * 5
-    lib.oracle_lstm_fwd_masked.restype = i
-    lib.oracle_lstm_bwd_masked.argtypes = [i, i, i, i] + [dp] * 10 + [dp] * 6
-    lib.oracle_lstm_bwd_masked.restype = i
+    lib.oracle_lstm_fwd_ex.argtypes = [i, i, i, i] + [dp] * 6 + [i] + [dp] * 5
+    lib.oracle_lstm_fwd_ex.restype = i
+    lib.oracle_lstm_bwd_ex.argtypes = [i, i, i, i] + [dp] * 5 + [i] + [dp] * 5 + [dp] * 6
+    lib.oracle_lstm_bwd_ex.restype = i
     lib.oracle_set_threads.argtypes = [i]
     lib.oracle_set_threads.restype = None
     lib.oracle_max_threads.argtypes = []
@@ -108,9 +108,10 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None):
+def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None, reverse=False):
     """Forward pass.  Returns dict(y, gates, cells, hT, cT) of float64 arrays.
-    mask [T][B][H] (1 = real step, 0 = padding) or None."""
+    mask [T][B][H] (1 = real step, 0 = padding) or None; reverse: the
+    recurrence runs over t = T-1 .. 0 (direction "REDIRECTIONAL")."""
     x = _f64(x)
     T, B, I = x.shape
     W = _f64(W)
@@ -125,17 +126,18 @@ def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None):
     hT = np.empty((B, H))
     cT = np.empty((B, H))
     mask = _f64(mask, (T, B, H))
-    rc = _load(lib).oracle_lstm_fwd_masked(T, B, I, H, _ptr(x), _ptr(W), _ptr(b), _ptr(h0),
-                                        _ptr(c0), _ptr(mask), _ptr(y), _ptr(gates),
-                                        _ptr(cells), _ptr(hT), _ptr(cT))
+    rc = _load(lib).oracle_lstm_fwd_ex(T, B, I, H, _ptr(x), _ptr(W), _ptr(b), _ptr(h0),
+                                    _ptr(c0), _ptr(mask), int(bool(reverse)), _ptr(y),
+                                    _ptr(gates), _ptr(cells), _ptr(hT), _ptr(cT))
     if rc != 0:
         raise RuntimeError("oracle_lstm_fwd failed")
     return dict(y=y, gates=gates, cells=cells, hT=hT, cT=cT)
 
 
-def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None):
+def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None,
+             reverse=False):
     """BPTT given the forward's saved state ``fwd`` (the dict lstm_fwd returns,
-    run with the same mask).
+    run with the same mask and direction).
 
     Returns dict(dx, dW, db, dh0, dc0, dG) of float64 arrays; dG holds the
     pre-activation gate gradients [di|df|dg|do] of every step."""
@@ -156,8 +158,9 @@ def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None
     dc0 = np.empty((B, H))
     dG = np.empty((T, B, 4 * H))
     mask = _f64(mask, (T, B, H))
-    rc = _load(lib).oracle_lstm_bwd_masked(T, B, I, H, _ptr(x), _ptr(W), _ptr(h0), _ptr(c0),
-                                        _ptr(mask), _ptr(y), _ptr(gates), _ptr(cells),
+    rc = _load(lib).oracle_lstm_bwd_ex(T, B, I, H, _ptr(x), _ptr(W), _ptr(h0), _ptr(c0),
+                                    _ptr(mask), int(bool(reverse)), _ptr(y), _ptr(gates),
+                                    _ptr(cells),
                                  _ptr(dy), _ptr(dhT), _ptr(dcT),
                                  _ptr(dx), _ptr(dW), _ptr(db), _ptr(dh0), _ptr(dc0), _ptr(dG))
     if rc != 0:
@@ -166,10 +169,10 @@ def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None
 
 
 def lstm_fwd_bwd(x, W, b=None, h0=None, c0=None, dy=None, dhT=None, dcT=None, lib=None,
-                 mask=None):
+                 mask=None, reverse=False):
     """Forward then backward; returns the union of both result dicts."""
-    f = lstm_fwd(x, W, b, h0, c0, lib=lib, mask=mask)
-    g = lstm_bwd(x, W, h0, c0, f, dy, dhT, dcT, lib=lib, mask=mask)
+    f = lstm_fwd(x, W, b, h0, c0, lib=lib, mask=mask, reverse=reverse)
+    g = lstm_bwd(x, W, h0, c0, f, dy, dhT, dcT, lib=lib, mask=mask, reverse=reverse)
     out = dict(f)
     out.update(g)
     return out

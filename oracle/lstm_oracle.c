@@ -44,6 +44,12 @@
  * Mask values other than 0 and 1 are outside the reading (the backward uses
  * tanh of the saved cell state, which equals tanh c~ only where m = 1).
  *
+ * Direction (the operator's "direction" attribute): "UNIDIRECTIONAL" runs the
+ * recurrence over t = 0 .. T-1, "REDIRECTIONAL" (reverse = 1) over
+ * t = T-1 .. 0: the step at time t then reads the state of time t+1 (initH /
+ * initC before the first step, t = T-1), and hT / cT are the state after the
+ * last step (t = 0).
+ *
  * Parity is pinned (tests/test_oracle.py) by central finite differences of the
  * surrogate loss L = sum_t <dy_t, h_t> + <dhT, h_{T-1}> + <dcT, c_{T-1}>,
  * by the T = 1 closed form, the W = 0 closed form, a hand-computed example,
@@ -90,11 +96,11 @@ static double sigm(double a)
 /* Forward pass, forward-formula table of "SingleLayerLstmGrad".
  * b, h0, c0 and mask may be NULL (zeros; no padding).  Returns 0, or -1 on bad
  * sizes / no memory. */
-int oracle_lstm_fwd_masked(int T, int B, int I, int H,
-                           const double *x, const double *W, const double *b,
-                           const double *h0, const double *c0, const double *mask,
-                           double *y, double *gates, double *cells,
-                           double *hT, double *cT)
+int oracle_lstm_fwd_ex(int T, int B, int I, int H,
+                       const double *x, const double *W, const double *b,
+                       const double *h0, const double *c0, const double *mask, int reverse,
+                       double *y, double *gates, double *cells,
+                       double *hT, double *cT)
 {
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
@@ -115,8 +121,9 @@ int oracle_lstm_fwd_masked(int T, int B, int I, int H,
             z[j] = h0 ? h0[(long)n * H + j] : 0.0;      /* h_{-1} = initH */
             cprev[j] = c0 ? c0[(long)n * H + j] : 0.0;  /* c_{-1} = initC */
         }
-        for (int t = 0; t < T; ++t) {
-            /* input concat: z_t = [h_{t-1}; x_t] */
+        for (int s = 0; s < T; ++s) {
+            const int t = reverse ? T - 1 - s : s;  /* time of the s-th step */
+            /* input concat: z_t = [h_prev; x_t] (h_prev: the previous step's) */
             const double *xt = x + ((long)t * B + n) * I;
             const double *mt = mask ? mask + ((long)t * B + n) * H : NULL;
             for (int k = 0; k < I; ++k)
@@ -171,7 +178,7 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
                     double *y, double *gates, double *cells,
                     double *hT, double *cT)
 {
-    return oracle_lstm_fwd_masked(T, B, I, H, x, W, b, h0, c0, NULL, y, gates, cells, hT, cT);
+    return oracle_lstm_fwd_ex(T, B, I, H, x, W, b, h0, c0, NULL, 0, y, gates, cells, hT, cT);
 }
 
 /* Backward pass, "backward algorithm (time step t -> t-1)" of
@@ -180,13 +187,13 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
  * optional scratch of T*B*4H doubles (allocated here when NULL); on return it
  * holds the pre-activation gate gradients [di | df | dg | do] of every step.
  * Returns 0, or -1 on bad sizes / no memory. */
-int oracle_lstm_bwd_masked(int T, int B, int I, int H,
-                           const double *x, const double *W,
-                           const double *h0, const double *c0, const double *mask,
-                           const double *y, const double *gates, const double *cells,
-                           const double *dy, const double *dhT, const double *dcT,
-                           double *dx, double *dW, double *db,
-                           double *dh0, double *dc0, double *dG)
+int oracle_lstm_bwd_ex(int T, int B, int I, int H,
+                       const double *x, const double *W,
+                       const double *h0, const double *c0, const double *mask, int reverse,
+                       const double *y, const double *gates, const double *cells,
+                       const double *dy, const double *dhT, const double *dcT,
+                       double *dx, double *dW, double *db,
+                       double *dh0, double *dc0, double *dG)
 {
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
@@ -219,10 +226,12 @@ int oracle_lstm_bwd_masked(int T, int B, int I, int H,
             dh_next[j] = dhT ? dhT[(long)n * H + j] : 0.0;
             dc_next[j] = dcT ? dcT[(long)n * H + j] : 0.0;
         }
-        for (int t = T - 1; t >= 0; --t) {
+        for (int s = T - 1; s >= 0; --s) {  /* steps in reverse order of the forward's */
+            const int t = reverse ? T - 1 - s : s;         /* time of step s */
+            const int tp = reverse ? t + 1 : t - 1;        /* time of step s - 1 */
             const double *gt = gates + ((long)t * B + n) * G4;
             const double *ct = cells + ((long)t * B + n) * H;
-            const double *cp = (t > 0) ? cells + ((long)(t - 1) * B + n) * H
+            const double *cp = (s > 0) ? cells + ((long)tp * B + n) * H
                                        : (c0 ? c0 + (long)n * H : NULL);
             const double *dyt = dy ? dy + ((long)t * B + n) * H : NULL;
             const double *mt = mask ? mask + ((long)t * B + n) * H : NULL;
@@ -289,11 +298,14 @@ int oracle_lstm_bwd_masked(int T, int B, int I, int H,
             for (long k = 0; k < K; ++k)
                 dWr[k] = 0.0;
             for (int t = 0; t < T; ++t) {
+                /* time of the step before time t's step (none: h_prev = initH) */
+                const int tp = reverse ? t + 1 : t - 1;
+                const int first = reverse ? (t == T - 1) : (t == 0);
                 for (int n = 0; n < B; ++n) {
                     double d = dG[((long)t * B + n) * G4 + r];
                     s_b += d;
-                    const double *hp = (t > 0) ? y + ((long)(t - 1) * B + n) * H
-                                               : (h0 ? h0 + (long)n * H : NULL);
+                    const double *hp = !first ? y + ((long)tp * B + n) * H
+                                              : (h0 ? h0 + (long)n * H : NULL);
                     const double *xt = x + ((long)t * B + n) * I;
                     if (hp)
                         for (int k = 0; k < H; ++k)
@@ -318,6 +330,6 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
                     double *dx, double *dW, double *db,
                     double *dh0, double *dc0, double *dG)
 {
-    return oracle_lstm_bwd_masked(T, B, I, H, x, W, h0, c0, NULL, y, gates, cells, dy, dhT, dcT,
-                                  dx, dW, db, dh0, dc0, dG);
+    return oracle_lstm_bwd_ex(T, B, I, H, x, W, h0, c0, NULL, 0, y, gates, cells, dy, dhT, dcT,
+                              dx, dW, db, dh0, dc0, dG);
 }

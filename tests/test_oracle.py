@@ -39,19 +39,20 @@ def random_case(T, B, I, H, seed, wscale=1.5, dhdc=True, dy=True):
     return p, g
 
 
-def run(p, g, lib=None, mask=None):
+def run(p, g, lib=None, mask=None, reverse=False):
     return oracle.lstm_fwd_bwd(p["x"], p["W"], p["b"], p["h0"], p["c0"],
-                               g["dy"], g["dhT"], g["dcT"], lib=lib, mask=mask)
+                               g["dy"], g["dhT"], g["dcT"], lib=lib, mask=mask, reverse=reverse)
 
 
-def loss(p, g, lib=None, mask=None):
-    f = oracle.lstm_fwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], lib=lib, mask=mask)
+def loss(p, g, lib=None, mask=None, reverse=False):
+    f = oracle.lstm_fwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], lib=lib, mask=mask,
+                        reverse=reverse)
     return oracle.surrogate_loss(f, g["dy"], g["dhT"], g["dcT"])
 
 
-def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None):
+def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None, reverse=False):
     """max over checked entries of |analytic - central FD| / max(1, |analytic|)."""
-    out = run(p, g, lib, mask)
+    out = run(p, g, lib, mask, reverse)
     rng = np.random.default_rng(seed)
     worst = 0.0
     for name, gname in GRAD_OF.items():
@@ -65,9 +66,9 @@ def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None):
             old = flat[k]
             h = 1e-6 * max(1.0, abs(old))
             flat[k] = old + h
-            lp = loss(p, g, lib, mask)
+            lp = loss(p, g, lib, mask, reverse)
             flat[k] = old - h
-            lm = loss(p, g, lib, mask)
+            lm = loss(p, g, lib, mask, reverse)
             flat[k] = old
             fd = (lp - lm) / (2 * h)
             worst = max(worst, abs(fd - an[k]) / max(1.0, abs(an[k])))
@@ -377,3 +378,31 @@ def test_length_mask_equals_truncated_sequences():
         db += ref["db"]
     np.testing.assert_allclose(out["dW"], dW, rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(out["db"], db, rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------- direction
+# The operator's "direction" attribute: "REDIRECTIONAL" runs the recurrence over
+# t = T-1 .. 0 (initH / initC before step t = T-1; hT / cT after step t = 0).
+
+@pytest.mark.parametrize("T,B,I,H,masked", [(3, 2, 3, 4, False), (4, 2, 2, 3, True)])
+def test_reverse_finite_differences(T, B, I, H, masked):
+    p, g = random_case(T, B, I, H, seed=500 + T * H)
+    mask = random_mask(T, B, H, seed=9 + T) if masked else None
+    assert fd_max_error(p, g, mask=mask, reverse=True) < 1e-6
+
+
+def test_reverse_is_forward_on_flipped_time():
+    """The reverse LSTM is the forward LSTM on the time-flipped sequences, its
+    per-step outputs flipped back: y, gates, cells, dx (and the mask) flip;
+    hT, cT, dW, db, dh0, dc0 are the same."""
+    T, B, I, H = 5, 3, 4, 6
+    p, g = random_case(T, B, I, H, seed=91)
+    mask = random_mask(T, B, H, seed=92)
+    rev = run(p, g, mask=mask, reverse=True)
+    pf = dict(p, x=p["x"][::-1].copy())
+    gf = dict(g, dy=g["dy"][::-1].copy())
+    fwd = run(pf, gf, mask=mask[::-1].copy())
+    for k in ("y", "gates", "cells", "dx"):
+        np.testing.assert_allclose(rev[k], fwd[k][::-1], rtol=1e-12, atol=1e-13, err_msg=k)
+    for k in ("hT", "cT", "dW", "db", "dh0", "dc0"):
+        np.testing.assert_allclose(rev[k], fwd[k], rtol=1e-11, atol=1e-12, err_msg=k)

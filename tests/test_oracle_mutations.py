@@ -44,10 +44,16 @@ MUTATIONS = {
     "mask_no_h_pass": ("dh_pass[j] = (1.0 - m) * dh_tot;", "dh_pass[j] = 0.0;"),
     # padding updates the cell state anyway (variable-length mask, forward)
     "mask_c_moves": ("c_ = mt[j] * c_ + (1.0 - mt[j]) * cprev[j];", "c_ = c_;"),
+    # reverse direction: c_{t-1} of the forget-gate gradient taken from the
+    # forward direction's neighbour
+    "reverse_cprev": ("const int tp = reverse ? t + 1 : t - 1;        /* time of step s - 1 */",
+                      "const int tp = t - 1;"),
 }
 
 # mutations that only a masked case can reveal
 MASKED = {"mask_no_h_pass", "mask_c_moves"}
+# and only a reverse-direction case
+REVERSE = {"reverse_cprev"}
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
@@ -60,6 +66,8 @@ def test_planted_mistake_is_caught(name, tmp_path):
     lib = oracle.load_variant(oracle.compile_source(str(path), str(tmp_path / "mutant.so")))
     p, g = random_case(3, 2, 3, 4, seed=99)
     mask = random_mask(3, 2, 4, seed=5) if name in MASKED else None
-    assert fd_max_error(p, g, lib=lib, mask=mask) > 1e-3, f"mutation {name} slipped through"
+    rev = name in REVERSE
+    assert fd_max_error(p, g, lib=lib, mask=mask, reverse=rev) > 1e-3, \
+        f"mutation {name} slipped through"
     # the unmutated oracle passes the same pin
-    assert fd_max_error(p, g, mask=mask) < 1e-6
+    assert fd_max_error(p, g, mask=mask, reverse=rev) < 1e-6
