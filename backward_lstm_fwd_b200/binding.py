@@ -27,7 +27,7 @@ LSTM_F32 = 0
 LSTM_BF16 = 1
 
 EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd", "lstm_bwd",
-           "lstm_fwd_masked", "lstm_bwd_masked",
+           "lstm_fwd_ex", "lstm_bwd_ex",
            "lstm_status", "lstm_profile_begin", "lstm_profile_end", "lstm_launch_count",
            "lstm_strerror", "lstm_abi_version")
 
@@ -43,6 +43,15 @@ class LstmError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int), ("B", ctypes.c_int), ("I", ctypes.c_int),
                 ("H", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+LSTM_DIR_FORWARD, LSTM_DIR_REVERSE = 0, 1
+
+
+class Options(ctypes.Structure):
+    """lstm_options: the seq_length mask (device pointer or None) and the
+    direction (LSTM_DIR_FORWARD / LSTM_DIR_REVERSE)."""
+    _fields_ = [("seq_mask", ctypes.c_void_p), ("direction", ctypes.c_int)]
 
 
 _lib = None
@@ -67,10 +76,11 @@ def load(path: str = LIB_PATH):
     lib.lstm_fwd.restype = ip
     lib.lstm_bwd.argtypes = [dp] + [vp] * 15 + [vp, sz, vp]
     lib.lstm_bwd.restype = ip
-    lib.lstm_fwd_masked.argtypes = [dp] + [vp] * 11 + [vp, sz, vp]
-    lib.lstm_fwd_masked.restype = ip
-    lib.lstm_bwd_masked.argtypes = [dp] + [vp] * 16 + [vp, sz, vp]
-    lib.lstm_bwd_masked.restype = ip
+    op = ctypes.POINTER(Options)
+    lib.lstm_fwd_ex.argtypes = [dp, op] + [vp] * 10 + [vp, sz, vp]
+    lib.lstm_fwd_ex.restype = ip
+    lib.lstm_bwd_ex.argtypes = [dp, op] + [vp] * 15 + [vp, sz, vp]
+    lib.lstm_bwd_ex.restype = ip
     lib.lstm_status.argtypes = [vp, sz, vp]
     lib.lstm_status.restype = ip
     lib.lstm_strerror.argtypes = [ip]
@@ -142,41 +152,48 @@ def bwd_workspace_size(d: Dims) -> int:
     return int(load().lstm_bwd_workspace_size(ctypes.byref(d)))
 
 
+def _options(mask, reverse):
+    return Options(_p(mask), LSTM_DIR_REVERSE if reverse else LSTM_DIR_FORWARD)
+
+
 def lstm_fwd(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes=None,
-             stream=None, check: bool = True, mask=None) -> int:
-    """Direct call of the C entry point lstm_fwd, or lstm_fwd_masked when a
-    variable-length mask [T,B,H] (1 = real step, 0 = padding) is given (device
-    tensors or raw pointers)."""
+             stream=None, check: bool = True, mask=None, reverse: bool = False) -> int:
+    """Direct call of the C entry point lstm_fwd, or lstm_fwd_ex with a
+    variable-length mask [T,B,H] (1 = real step, 0 = padding) and / or the
+    reverse direction (device tensors or raw pointers)."""
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
-    if mask is None:
+    if mask is None and not reverse:
         rc = load().lstm_fwd(ctypes.byref(d), _p(x), _p(W), _p(b), _p(h0), _p(c0), _p(y),
                              _p(hT), _p(cT), _p(gates), _p(cells), _p(ws), ws_bytes,
                              _stream(stream))
     else:
-        rc = load().lstm_fwd_masked(ctypes.byref(d), _p(x), _p(W), _p(b), _p(h0), _p(c0),
-                                    _p(mask), _p(y), _p(hT), _p(cT), _p(gates), _p(cells),
-                                    _p(ws), ws_bytes, _stream(stream))
+        opt = _options(mask, reverse)
+        rc = load().lstm_fwd_ex(ctypes.byref(d), ctypes.byref(opt), _p(x), _p(W), _p(b), _p(h0),
+                                _p(c0), _p(y), _p(hT), _p(cT), _p(gates), _p(cells), _p(ws),
+                                ws_bytes, _stream(stream))
     if check and rc != LSTM_OK:
         raise LstmError(rc, "lstm_fwd")
     return rc
 
 
 def lstm_bwd(d: Dims, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0, ws,
-             ws_bytes=None, stream=None, check: bool = True, mask=None) -> int:
-    """Direct call of the C entry point lstm_bwd, or lstm_bwd_masked when the
-    forward's variable-length mask is given (device tensors or raw pointers)."""
+             ws_bytes=None, stream=None, check: bool = True, mask=None,
+             reverse: bool = False) -> int:
+    """Direct call of the C entry point lstm_bwd, or lstm_bwd_ex with the
+    forward's mask and direction (device tensors or raw pointers)."""
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
-    if mask is None:
+    if mask is None and not reverse:
         rc = load().lstm_bwd(ctypes.byref(d), _p(dy), _p(dhT), _p(dcT), _p(x), _p(W), _p(h0),
                              _p(c0), _p(y), _p(gates), _p(cells), _p(dx), _p(dW), _p(db),
                              _p(dh0), _p(dc0), _p(ws), ws_bytes, _stream(stream))
     else:
-        rc = load().lstm_bwd_masked(ctypes.byref(d), _p(mask), _p(dy), _p(dhT), _p(dcT), _p(x),
-                                    _p(W), _p(h0), _p(c0), _p(y), _p(gates), _p(cells), _p(dx),
-                                    _p(dW), _p(db), _p(dh0), _p(dc0), _p(ws), ws_bytes,
-                                    _stream(stream))
+        opt = _options(mask, reverse)
+        rc = load().lstm_bwd_ex(ctypes.byref(d), ctypes.byref(opt), _p(dy), _p(dhT), _p(dcT),
+                                _p(x), _p(W), _p(h0), _p(c0), _p(y), _p(gates), _p(cells),
+                                _p(dx), _p(dW), _p(db), _p(dh0), _p(dc0), _p(ws), ws_bytes,
+                                _stream(stream))
     if check and rc != LSTM_OK:
         raise LstmError(rc, "lstm_bwd")
     return rc
@@ -273,29 +290,30 @@ class Grads:
         self.dc0 = torch.empty((B, H), dtype=f, device=device)
 
 
-def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None, mask=None) -> State:
-    """Allocate outputs and run lstm_fwd (lstm_fwd_masked with a mask).  x
-    [T,B,I], W [4H,H+I] and mask [T,B,H] share the compute dtype (float32 or
-    bfloat16); c0 is float32."""
+def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None, mask=None,
+            reverse: bool = False) -> State:
+    """Allocate outputs and run lstm_fwd (lstm_fwd_ex with a mask or the
+    reverse direction).  x [T,B,I], W [4H,H+I] and mask [T,B,H] share the
+    compute dtype (float32 or bfloat16); c0 is float32."""
     T, B, I = x.shape
     H = W.shape[0] // 4
     st = State(T, B, I, H, x.dtype, x.device)
     if ws is None:
         ws = empty_workspace(fwd_workspace_size(st.dims), x.device)
     lstm_fwd(st.dims, x, W, b, h0, c0, st.y, st.hT, st.cT, st.gates, st.cells, ws, stream=stream,
-             mask=mask)
+             mask=mask, reverse=reverse)
     return st
 
 
 def backward(st: State, x, W, h0=None, c0=None, dy=None, dhT=None, dcT=None, ws=None,
-             stream=None, mask=None) -> Grads:
+             stream=None, mask=None, reverse: bool = False) -> Grads:
     """Allocate gradients and run lstm_bwd on the saved state of forward()
-    (lstm_bwd_masked with the forward's mask)."""
+    (lstm_bwd_ex with the forward's mask and direction)."""
     T, B, I = x.shape
     H = W.shape[0] // 4
     g = Grads(T, B, I, H, x.device)
     if ws is None:
         ws = empty_workspace(bwd_workspace_size(st.dims), x.device)
     lstm_bwd(st.dims, dy, dhT, dcT, x, W, h0, c0, st.y, st.gates, st.cells, g.dx, g.dW, g.db,
-             g.dh0, g.dc0, ws, stream=stream, mask=mask)
+             g.dh0, g.dc0, ws, stream=stream, mask=mask, reverse=reverse)
     return g

@@ -162,7 +162,9 @@ int ws_ok(void *ws, size_t ws_bytes, size_t need) {
     } while (0)
 
 cudaError_t reset_barriers(void *ws, cudaStream_t s) {
-    return cudaMemsetAsync((char *)ws + offsetof(Ctrl, bar), 0, sizeof(((Ctrl *)0)->bar), s);
+    // the whole control block: status word, failing site and barrier counters
+    // (a workspace fresh from an allocator holds anything)
+    return cudaMemsetAsync(ws, 0, kCtrlBytes, s);
 }
 
 template <class T>
@@ -210,7 +212,8 @@ cudaError_t tc_input_projection(const lstm_dims *d, const bf16 *x, const bf16 *W
 // (0: one per SM).
 cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf16 *W,
                      const bf16 *h0, const bf16 *y, float *dW, float *dx, Ctrl *ctrl,
-                     cudaStream_t s, int t_lo, int t_hi, bool accumulate, int max_ctas) {
+                     cudaStream_t s, int t_lo, int t_hi, bool accumulate, int max_ctas,
+                     bool reverse = false) {
     const long long B = d->B, H = d->H, I = d->I, G4 = 4 * H;
     const long long r0 = (long long)t_lo * B, r1 = (long long)t_hi * B;
     tcg::Builder bld(ctrl);
@@ -218,15 +221,28 @@ cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf
     const int m_x_mn = bld.add_map({x, r1, I, I}, 1, 0);
     const int m_dg_k = bld.add_map({dG, r1, G4, G4}, 0, tcg::BM);
     const int m_wx_mn = bld.add_map({W + H, G4, I, H + I}, 1, 0);
-    // h_prev of row r is y row r - B (r >= B) or h0 row r (r < B, only when t_lo == 0)
-    const long long ry0 = std::max(r0, B);
-    const int m_y_mn = (r1 > ry0) ? bld.add_map({y, r1 - B, H, H}, 1, 0) : -1;
-    const int m_h0_mn = (h0 && r0 < B) ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
-    // dW, h-part (no K segment, i.e. zero, when the range is t = 0 alone and h0 is absent)
     tcg::Problem &p0 = bld.add_problem((int)G4, (int)H, 1, 1, dW, H + I, 0, nullptr);
     p0.accumulate = accumulate;
-    if (m_y_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, (int)ry0, m_y_mn, (int)(ry0 - B), r1 - ry0);
-    if (m_h0_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, 0, m_h0_mn, 0, B);
+    if (!reverse) {
+        // h_prev of row r is y row r - B (r >= B) or h0 row r (r < B, only when t_lo == 0)
+        const long long ry0 = std::max(r0, B);
+        const int m_y_mn = (r1 > ry0) ? bld.add_map({y, r1 - B, H, H}, 1, 0) : -1;
+        const int m_h0_mn = (h0 && r0 < B) ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
+        // dW, h-part (no K segment, i.e. zero, when the range is t = 0 alone and h0 is absent)
+        if (m_y_mn >= 0)
+            tcg::Builder::add_seg(p0, m_dg_mn, (int)ry0, m_y_mn, (int)(ry0 - B), r1 - ry0);
+        if (m_h0_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, 0, m_h0_mn, 0, B);
+    } else {
+        // reverse direction: h_prev of row r is y row r + B (r < last0 = (T-1) B) or
+        // h0 row r - last0 (the last time, only when t_hi == T)
+        const long long last0 = (long long)(d->T - 1) * B;
+        const long long ry1 = std::min(r1, last0);
+        const int m_y_mn = (ry1 > r0) ? bld.add_map({y, ry1 + B, H, H}, 1, 0) : -1;
+        const int m_h0_mn = (h0 && r1 > last0) ? bld.add_map({h0, B, H, H}, 1, 0) : -1;
+        if (m_y_mn >= 0)
+            tcg::Builder::add_seg(p0, m_dg_mn, (int)r0, m_y_mn, (int)(r0 + B), ry1 - r0);
+        if (m_h0_mn >= 0) tcg::Builder::add_seg(p0, m_dg_mn, (int)last0, m_h0_mn, 0, B);
+    }
     // dW, x-part
     tcg::Problem &p1 = bld.add_problem((int)G4, (int)I, 1, 1, dW, H + I, (int)H, nullptr);
     p1.accumulate = accumulate;
@@ -780,8 +796,8 @@ cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStre
 // LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
 int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, const bf16 *W,
                        const bf16 *b, const bf16 *h0, const float *c0, const bf16 *mask,
-                       bf16 *y, bf16 *hT, float *cT, bf16 *gates, float *cells, Ctrl *ctrl,
-                       cudaStream_t s) {
+                       bool reverse, bf16 *y, bf16 *hT, float *cT, bf16 *gates, float *cells,
+                       Ctrl *ctrl, cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, I = d->I;
     rec3::Fwd3Params prm;
     memset(&prm, 0, sizeof(prm));
@@ -791,7 +807,7 @@ int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, con
     else prm.map_h0 = prm.map_y;
     if (!ok) return LSTM_ERR_UNSUPPORTED;
     prm.W = W; prm.bias = b; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
-    prm.mask = mask; prm.h0 = h0;
+    prm.mask = mask; prm.h0 = h0; prm.reverse = reverse;
     prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.I = (int)I; prm.R = P.R; prm.G = P.G;
     prm.kcc = P.kcc; prm.kcx = P.kcx;
@@ -846,10 +862,10 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 // One launch of the TMEM-weight backward kernel over epilogue iterations
 // [i0, i1) (time steps T-i1 .. T-i0-1); WT must already hold W_h^T.
 int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                   const float *dcT, const float *c0, const bf16 *mask, const bf16 *gates,
-                   const float *cells, bf16 *dG, const bf16 *WT, float *dbgroup, float *dh0,
-                   float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0, int i1,
-                   cudaStream_t s) {
+                   const float *dcT, const float *c0, const bf16 *mask, bool reverse,
+                   const bf16 *gates, const float *cells, bf16 *dG, const bf16 *WT,
+                   float *dbgroup, float *dh0, float *dc0, float *dc_carry, float *dhp_carry,
+                   Ctrl *ctrl, int i0, int i1, cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
     rec3::Bwd3Params prm;
     memset(&prm, 0, sizeof(prm));
@@ -862,7 +878,7 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const 
     prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
     prm.kcc = P.kcc; prm.stages = P.stages;
-    prm.i0 = i0; prm.i1 = i1;
+    prm.i0 = i0; prm.i1 = i1; prm.reverse = reverse;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
     const cudaError_t e =
@@ -889,13 +905,13 @@ cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cud
 // workspace first, then copied into each CTA's tensor memory), one launch.
 int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
                        const float *dcT, const bf16 *W, const float *c0, const bf16 *mask,
-                       const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
+                       bool reverse, const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
                        float *dbgroup, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
     const long long G4 = 4LL * d->H;
     if (launch_transpose_wh(d, W, WT, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, gates, cells, dG, WT, dbgroup,
-                                  dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
+    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, gates, cells, dG, WT,
+                                  dbgroup, dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
     if (rc != LSTM_OK) return rc;
     simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
     note_launch();
@@ -911,9 +927,9 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int nch,
                        const bf16 *dy, const bf16 *dhT, const float *dcT, const bf16 *x,
                        const bf16 *W, const bf16 *h0, const float *c0, const bf16 *mask,
-                       const bf16 *y, const bf16 *gates, const float *cells, bf16 *dG,
-                       bf16 *WT, float *dbgroup, float *dc_carry, float *dhp_carry, float *dx,
-                       float *dW, float *db, float *dh0, float *dc0, Ctrl *ctrl,
+                       bool reverse, const bf16 *y, const bf16 *gates, const float *cells,
+                       bf16 *dG, bf16 *WT, float *dbgroup, float *dc_carry, float *dhp_carry,
+                       float *dx, float *dW, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
     std::lock_guard<std::mutex> lock(A.mu);
     const int T = d->T;
@@ -934,8 +950,8 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
         for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
             const int i0 = (int)((long long)T * c / nch), i1 = (int)((long long)T * (c + 1) / nch);
-            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, gates, cells, dG, WT, dbgroup, dh0,
-                                dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
+            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, gates, cells, dG, WT,
+                                dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
             if (rc != LSTM_OK) break;
             if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
                 cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess) {
@@ -943,9 +959,11 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
                 break;
             }
             prof::Phase phg(LSTM_PHASE_DW, A.gemm);
-            // rows of time steps T-i1 .. T-i0-1; dW accumulates after the first chunk
-            if (tc_dw_dx(d, dG, x, W, h0, y, dW, dx, ctrl, A.gemm, T - i1, T - i0, c > 0,
-                         c + 1 < nch ? gemm_ctas : 0) != cudaSuccess)
+            // rows of the chunk's times (steps T-i1 .. T-i0-1: times i0 .. i1-1 in
+            // the reverse direction); dW accumulates after the first chunk
+            const int t_lo = reverse ? i0 : T - i1, t_hi = reverse ? i1 : T - i0;
+            if (tc_dw_dx(d, dG, x, W, h0, y, dW, dx, ctrl, A.gemm, t_lo, t_hi, c > 0,
+                         c + 1 < nch ? gemm_ctas : 0, reverse) != cudaSuccess)
                 rc = LSTM_ERR_CUDA;
         }
         if (rc == LSTM_OK) {
@@ -969,8 +987,10 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
 // kernel or the per-step kernels only.
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
-             const float *c0, const T *mask, T *y, T *hT, float *cT, T *gates, float *cells,
-             char *ws, cudaStream_t s) {
+             const float *c0, const T *mask, bool reverse, T *y, T *hT, float *cT, T *gates,
+             float *cells, char *ws, cudaStream_t s) {
+    // masked or reverse-direction calls: TMEM-weight kernel or per-step kernels
+    const bool special = mask != nullptr || reverse;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H;
     const FwdLayout L = fwd_layout(d);
@@ -981,8 +1001,9 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
             const int rc = tc_fwd_recurrence3(d, plan3, (const bf16 *)x, (const bf16 *)W,
                                               (const bf16 *)b, (const bf16 *)h0, c0,
-                                              (const bf16 *)mask, (bf16 *)y, (bf16 *)hT, cT,
-                                              (bf16 *)gates, cells, (Ctrl *)ws, s);
+                                              (const bf16 *)mask, reverse, (bf16 *)y,
+                                              (bf16 *)hT, cT, (bf16 *)gates, cells,
+                                              (Ctrl *)ws, s);
             g_last_fwd_path = 3;
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
         }
@@ -1001,7 +1022,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         // a2: the recurrence
         prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
         Rec2Plan plan2;
-        if (!mask && plan_fwd2(d, plan2)) {
+        if (!special && plan_fwd2(d, plan2)) {
             const int rc = tc_fwd_recurrence2(d, plan2, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
                                               (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells,
                                               (Ctrl *)ws, s);
@@ -1009,7 +1030,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
         }
         RecPlan plan;
-        if (!mask && plan_fwd_recur(d, plan)) {
+        if (!special && plan_fwd_recur(d, plan)) {
             g_last_fwd_path = 1;
             // persistent tcgen05 kernel: all T steps in one launch; it writes hT and cT
             return tc_fwd_recurrence(d, plan, (const bf16 *)W, (const bf16 *)h0, c0, Gx,
@@ -1018,9 +1039,11 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         }
         // otherwise one fused GEMM + gate/cell/hidden epilogue launch per step
         g_last_fwd_path = 0;
-        for (int t = 0; t < T_; ++t) {
-            const T *hp = t > 0 ? y + (long long)(t - 1) * BH : h0;
-            const float *cp = t > 0 ? cells + (long long)(t - 1) * BH : c0;
+        for (int st = 0; st < T_; ++st) {
+            // step st is at time t; the previous step at time tp
+            const int t = reverse ? T_ - 1 - st : st, tp = reverse ? t + 1 : t - 1;
+            const T *hp = st > 0 ? y + (long long)tp * BH : h0;
+            const float *cp = st > 0 ? cells + (long long)tp * BH : c0;
             simt::EpFwdStep<T> ep{Gx + (long long)t * B * 4 * H, cp, y + (long long)t * BH,
                                   gates + (long long)t * B * 4 * H, cells + (long long)t * BH, H};
             if (mask) {
@@ -1033,10 +1056,11 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
     }
     if (BH > 0) {
         prof::Phase ph(LSTM_PHASE_OTHER, s);
-        if (T_ > 0) {
-            LSTM_TRY(cudaMemcpyAsync(hT, y + (long long)(T_ - 1) * BH, BH * sizeof(T),
-                                     cudaMemcpyDeviceToDevice, s));
-            LSTM_TRY(cudaMemcpyAsync(cT, cells + (long long)(T_ - 1) * BH, BH * sizeof(float),
+        if (T_ > 0) {  // the state after the last step (time 0 in the reverse direction)
+            const long long tl = reverse ? 0 : T_ - 1;
+            LSTM_TRY(cudaMemcpyAsync(hT, y + tl * BH, BH * sizeof(T), cudaMemcpyDeviceToDevice,
+                                     s));
+            LSTM_TRY(cudaMemcpyAsync(cT, cells + tl * BH, BH * sizeof(float),
                                      cudaMemcpyDeviceToDevice, s));
         } else {
             LSTM_TRY(launch_copy_or_zero<T>(h0, hT, BH, s));
@@ -1051,9 +1075,10 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
 // kernel or the per-step kernels only.
 template <class T>
 int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, const T *x,
-             const T *W, const T *h0, const float *c0, const T *mask, const T *y,
+             const T *W, const T *h0, const float *c0, const T *mask, bool reverse, const T *y,
              const T *gates, const float *cells, float *dx, float *dW, float *db, float *dh0,
              float *dc0, char *ws, cudaStream_t s) {
+    const bool special = mask != nullptr || reverse;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H, TB = (long long)T_ * B;
     const int G4 = 4 * H, K = H + I;
@@ -1076,8 +1101,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     RecPlan plan;
     Rec2Plan plan2, plan3;
     const bool v3 = plan_bwd3(d, plan3);
-    const bool v2 = !v3 && !mask && plan_bwd2(d, plan2);
-    const bool v1 = !mask && plan_bwd_recur(d, plan);
+    const bool v2 = !v3 && !special && plan_bwd2(d, plan2);
+    const bool v1 = !special && plan_bwd_recur(d, plan);
     bool per_step = false;  // a masked call whose cluster kernel cannot be placed
     if (v3 || v2 || v1) {
         if (v3 && tc_gemm_ok(d) && bwd_chunks(d) > 1) {
@@ -1087,7 +1112,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                 const int rc = tc_bwd3_overlapped(
                     d, plan3, *A, bwd_chunks(d), (const bf16 *)dy, (const bf16 *)dhT, dcT,
                     (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)mask,
-                    (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
+                    reverse, (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
                     (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), (float *)(ws + L.dc),
                     (float *)(ws + L.dhp), dx, dW, db, dh0, dc0, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
@@ -1099,7 +1124,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
             g_last_bwd_path = v3 ? 3 : 2;
             if (v3)
                 rc = tc_bwd_recurrence3(d, plan3, (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                                        (const bf16 *)W, c0, (const bf16 *)mask,
+                                        (const bf16 *)W, c0, (const bf16 *)mask, reverse,
                                         (const bf16 *)gates, cells, (bf16 *)dG,
                                         (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), db, dh0,
                                         dc0, (Ctrl *)ws, s);
@@ -1115,7 +1140,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                 (const bf16 *)gates, cells, (bf16 *)dG, (bf16 *)(ws + L.wt),
                 (float *)(ws + L.dbgroup), db, dh0, dc0, (Ctrl *)ws, s);
             }
-            if (rc == LSTM_ERR_NOT_CORESIDENT && mask) per_step = true;
+            if (rc == LSTM_ERR_NOT_CORESIDENT && special) per_step = true;
             else if (rc != LSTM_OK) return rc;
         }
         if (!per_step) {
@@ -1123,14 +1148,14 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                 prof::Phase ph(LSTM_PHASE_DW, s);
                 LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
                                   (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0,
-                                  d->T, false, 0));
+                                  d->T, false, 0, reverse));
                 return LSTM_OK;
             }
             // dW / dx on CUDA cores (shapes off the TMA grid)
             {
                 prof::Phase ph(LSTM_PHASE_DW, s);
                 LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
-                                                    simt::Zrows<T>{x, y, h0, B, I, H},
+                                                    simt::Zrows<T>{x, y, h0, B, I, H, reverse, (long long)(T_ - 1) * B},
                                                     simt::EpStore{dW, K}, s)));
             }
             prof::Phase ph(LSTM_PHASE_DX, s);
@@ -1146,31 +1171,34 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     g_last_bwd_path = 0;
     {
     prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
-    for (int t = T_ - 1; t >= 0; --t) {
-        const bool last = (t == T_ - 1);
+    // steps st = T-1 .. 0 of the forward recurrence; step st is at time tau(st)
+    auto tau = [&](int st) -> long long { return reverse ? T_ - 1 - st : st; };
+    for (int st = T_ - 1; st >= 0; --st) {
+        const bool last = (st == T_ - 1);
+        const long long t = tau(st);
         simt::EpBwdStep<T> ep;
-        ep.dy = dy ? dy + (long long)t * BH : nullptr;
+        ep.dy = dy ? dy + t * BH : nullptr;
         ep.dh_in = last ? dhT : nullptr;
-        ep.dc_in = last ? dcT : dcbuf[(t + 1) & 1];
-        ep.gates = gates + (long long)t * B * G4;
-        ep.cells = cells + (long long)t * BH;
-        ep.cprev = t > 0 ? cells + (long long)(t - 1) * BH : c0;
-        ep.dG = dG + (long long)t * B * G4;
-        ep.dc_out = (t == 0) ? dc0 : dcbuf[t & 1];
+        ep.dc_in = last ? dcT : dcbuf[(st + 1) & 1];
+        ep.gates = gates + t * B * G4;
+        ep.cells = cells + t * BH;
+        ep.cprev = st > 0 ? cells + tau(st - 1) * BH : c0;
+        ep.dG = dG + t * B * G4;
+        ep.dc_out = (st == 0) ? dc0 : dcbuf[st & 1];
         ep.H = H;
         ep.use_acc = !last;
         if (mask) {
-            ep.mask = mask + (long long)t * BH;
-            ep.dhp_in = last ? nullptr : dhpbuf[(t + 1) & 1];
-            ep.dhp_out = dhpbuf[t & 1];
+            ep.mask = mask + t * BH;
+            ep.dhp_in = last ? nullptr : dhpbuf[(st + 1) & 1];
+            ep.dhp_out = dhpbuf[st & 1];
         }
-        const T *dGn = last ? dG : dG + (long long)(t + 1) * B * G4;
+        const T *dGn = last ? dG : dG + tau(st + 1) * B * G4;
         LSTM_TRY((simt::gemm<true, false>(B, H, last ? 0 : G4, simt::RowMajor<T>{dGn, G4},
                                            simt::RowMajor<T>{W, K}, ep, s)));
     }
-    // dinitH = W_h^T dG_0 (delta h_prev at t = 0, step 5), plus what padding at
-    // t = 0 passes on
-    LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG, G4},
+    // dinitH = W_h^T dG of the first step (delta h_prev before it, step 5), plus
+    // what padding at that step passes on
+    LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG + tau(0) * B * G4, G4},
                                        simt::RowMajor<T>{W, K},
                                        simt::EpStore{dh0, H, mask ? dhpbuf[0] : nullptr}, s)));
     }
@@ -1180,12 +1208,12 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         prof::Phase ph(LSTM_PHASE_DW, s);
         LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
                           (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0, d->T,
-                          false, 0));
+                          false, 0, reverse));
     } else {
         // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
         prof::Phase ph(LSTM_PHASE_DW, s);
         LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
-                                            simt::Zrows<T>{x, y, h0, B, I, H},
+                                            simt::Zrows<T>{x, y, h0, B, I, H, reverse, (long long)(T_ - 1) * B},
                                             simt::EpStore{dW, K}, s)));
     }
     // a5: db = column sums of dG (step 4)
@@ -1242,10 +1270,14 @@ int noalloc_scratch(void **out) {
 
 // =================================================================== C ABI
 namespace {
-int fwd_entry(const lstm_dims *d, const void *x, const void *W, const void *b, const void *h0,
-              const float *c0, const void *mask, void *y, void *hT, float *cT, void *gates,
-              float *cells, void *ws, size_t ws_bytes, void *stream) {
+int fwd_entry(const lstm_dims *d, const lstm_options *opt, const void *x, const void *W,
+              const void *b, const void *h0, const float *c0, void *y, void *hT, float *cT,
+              void *gates, float *cells, void *ws, size_t ws_bytes, void *stream) {
     if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    const void *mask = opt ? opt->seq_mask : nullptr;
+    const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
+    if (dir != LSTM_DIR_FORWARD && dir != LSTM_DIR_REVERSE) return LSTM_ERR_INVALID_ARG;
+    const bool reverse = dir == LSTM_DIR_REVERSE;
     if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
     const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
     if (!ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(b, false) ||
@@ -1259,19 +1291,23 @@ int fwd_entry(const lstm_dims *d, const void *x, const void *W, const void *b, c
     if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
     if (d->dtype == LSTM_F32)
         return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
-                               (const float *)h0, c0, (const float *)mask, (float *)y,
+                               (const float *)h0, c0, (const float *)mask, reverse, (float *)y,
                                (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
     typedef __nv_bfloat16 bf;
     return fwd_simt<bf>(d, (const bf *)x, (const bf *)W, (const bf *)b, (const bf *)h0, c0,
-                        (const bf *)mask, (bf *)y, (bf *)hT, cT, (bf *)gates, cells, (char *)ws,
-                        s);
+                        (const bf *)mask, reverse, (bf *)y, (bf *)hT, cT, (bf *)gates, cells,
+                        (char *)ws, s);
 }
 
-int bwd_entry(const lstm_dims *d, const void *mask, const void *dy, const void *dhT,
+int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const void *dhT,
               const float *dcT, const void *x, const void *W, const void *h0, const float *c0,
               const void *y, const void *gates, const float *cells, float *dx, float *dW,
               float *db, float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream) {
     if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
+    const void *mask = opt ? opt->seq_mask : nullptr;
+    const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
+    if (dir != LSTM_DIR_FORWARD && dir != LSTM_DIR_REVERSE) return LSTM_ERR_INVALID_ARG;
+    const bool reverse = dir == LSTM_DIR_REVERSE;
     if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
     const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
     const long long G4 = 4LL * d->H, K = (long long)d->H + d->I;
@@ -1289,12 +1325,12 @@ int bwd_entry(const lstm_dims *d, const void *mask, const void *dy, const void *
     if (d->dtype == LSTM_F32)
         return bwd_simt<float>(d, (const float *)dy, (const float *)dhT, dcT, (const float *)x,
                                (const float *)W, (const float *)h0, c0, (const float *)mask,
-                               (const float *)y, (const float *)gates, cells, dx, dW, db, dh0,
-                               dc0, (char *)ws, s);
+                               reverse, (const float *)y, (const float *)gates, cells, dx, dW,
+                               db, dh0, dc0, (char *)ws, s);
     typedef __nv_bfloat16 bf;
     return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
-                        (const bf *)h0, c0, (const bf *)mask, (const bf *)y, (const bf *)gates,
-                        cells, dx, dW, db, dh0, dc0, (char *)ws, s);
+                        (const bf *)h0, c0, (const bf *)mask, reverse, (const bf *)y,
+                        (const bf *)gates, cells, dx, dW, db, dh0, dc0, (char *)ws, s);
 }
 }  // namespace
 
@@ -1329,14 +1365,13 @@ size_t lstm_bwd_workspace_size(const lstm_dims *d) {
 int lstm_fwd(const lstm_dims *d, const void *x, const void *W, const void *b, const void *h0,
              const float *c0, void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
              size_t ws_bytes, void *stream) {
-    return fwd_entry(d, x, W, b, h0, c0, nullptr, y, hT, cT, gates, cells, ws, ws_bytes, stream);
+    return fwd_entry(d, nullptr, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes, stream);
 }
 
-int lstm_fwd_masked(const lstm_dims *d, const void *x, const void *W, const void *b,
-                    const void *h0, const float *c0, const void *mask, void *y, void *hT,
-                    float *cT, void *gates, float *cells, void *ws, size_t ws_bytes,
-                    void *stream) {
-    return fwd_entry(d, x, W, b, h0, c0, mask, y, hT, cT, gates, cells, ws, ws_bytes, stream);
+int lstm_fwd_ex(const lstm_dims *d, const lstm_options *opt, const void *x, const void *W,
+                const void *b, const void *h0, const float *c0, void *y, void *hT, float *cT,
+                void *gates, float *cells, void *ws, size_t ws_bytes, void *stream) {
+    return fwd_entry(d, opt, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes, stream);
 }
 
 int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *dcT,
@@ -1347,12 +1382,12 @@ int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *d
                      dc0, ws, ws_bytes, stream);
 }
 
-int lstm_bwd_masked(const lstm_dims *d, const void *mask, const void *dy, const void *dhT,
-                    const float *dcT, const void *x, const void *W, const void *h0,
-                    const float *c0, const void *y, const void *gates, const float *cells,
-                    float *dx, float *dW, float *db, float *dh0, float *dc0, void *ws,
-                    size_t ws_bytes, void *stream) {
-    return bwd_entry(d, mask, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0,
+int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, const void *dhT,
+                const float *dcT, const void *x, const void *W, const void *h0,
+                const float *c0, const void *y, const void *gates, const float *cells,
+                float *dx, float *dW, float *db, float *dh0, float *dc0, void *ws,
+                size_t ws_bytes, void *stream) {
+    return bwd_entry(d, opt, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0,
                      ws, ws_bytes, stream);
 }
 

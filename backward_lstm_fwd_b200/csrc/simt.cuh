@@ -131,10 +131,18 @@ template <class T> struct Hprev {
 // z-rows for dW: row r = t*B + n, column c < H -> h_{t-1}[n][c], else x_t[n][c-H].
 template <class T> struct Zrows {
     const T *x, *y, *h0; int B, I, H;
+    // reverse direction: h_prev of time t is y[t+1], and h0 at the last time
+    // (whose rows start at last0 = (T-1) * B)
+    bool reverse = false;
+    long long last0 = 0;
     __device__ float operator()(int r, int c) const {
         if (c < H) {
-            if (r < B) return h0 ? to_f(h0[(long long)r * H + c]) : 0.f;
-            return to_f(y[(long long)(r - B) * H + c]);
+            if (!reverse) {
+                if (r < B) return h0 ? to_f(h0[(long long)r * H + c]) : 0.f;
+                return to_f(y[(long long)(r - B) * H + c]);
+            }
+            if (r >= last0) return h0 ? to_f(h0[(long long)(r - last0) * H + c]) : 0.f;
+            return to_f(y[(long long)(r + B) * H + c]);
         }
         return to_f(x[(long long)r * I + (c - H)]);
     }

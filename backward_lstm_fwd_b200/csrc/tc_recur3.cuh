@@ -63,7 +63,8 @@ struct Bwd3Params {
     float *dhp_carry;
     Ctrl *ctrl;
     int T, B, H, U, G, NBr, kcc, stages;
-    int i0, i1;       // this launch runs epilogue iterations i0 .. i1-1 (t = T-1-i)
+    int i0, i1;       // this launch runs epilogue iterations i0 .. i1-1 (step T-1-i)
+    int reverse;      // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -117,6 +118,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     const int i0 = p.i0, i1 = p.i1;
     const bool first = i0 == 0, last = i1 == T;
     const int mma_lo = i0 > 1 ? i0 : 1, mma_hi = last ? T : i1 - 1;
+    // time of recurrence step s of the forward pass
+    auto tau = [&](int s) { return p.reverse ? T - 1 - s : s; };
     const int kslice = kcc * 64;              // this CTA's part of the 4H axis
     const int kbase = (int)kpart * kslice;
     unsigned int *ctr = &p.ctrl->bar[gi];
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 // acquire above, then the proxy fence: the TMA reads below see
                 // every dG store the group released
                 tc::fence_proxy_async_global();
-                const int row0 = (T - i) * B + b0;
+                const int row0 = tau(T - i) * B + b0;  // dG of step T-i
                 for (int c = 0; c < kcc; ++c) {
                     if (!tc::mbar_wait(&empty[stage], ph ^ 1, p.ctrl, abort_flag, 0x602, p.wait_ns)) {
                         aborted = true;
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 mpk = make_uint4(0, 0, 0, 0);
                 return;
             }
-            const long long row = (long long)t * B + b;
+            const long long row = (long long)tau(t) * B + b;  // t: a step, not a time
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 gpk[g] = __ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + g * H + jb));
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             const float4 x0 = __ldg(c4), x1 = __ldg(c4 + 1);
             ct[0] = x0.x; ct[1] = x0.y; ct[2] = x0.z; ct[3] = x0.w;
             ct[4] = x1.x; ct[5] = x1.y; ct[6] = x1.z; ct[7] = x1.w;
-            const float *cpp = t > 0 ? p.cells + (row - B) * H + jb
+            const float *cpp = t > 0 ? p.cells + ((long long)tau(t - 1) * B + b) * H + jb
                                      : (p.c0 ? p.c0 + (long long)b * H + jb : nullptr);
             if (cpp) {
                 const float4 y0 = __ldg(reinterpret_cast<const float4 *>(cpp));
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 const uint4 vi = rec::f32x8_to_bf16(dI), vf = rec::f32x8_to_bf16(dF);
                 const uint4 vg = rec::f32x8_to_bf16(dGg), vo = rec::f32x8_to_bf16(dO);
                 if (valid) {
-                    __nv_bfloat16 *o = p.dG + ((long long)t * B + b) * G4 + jb;
+                    __nv_bfloat16 *o = p.dG + ((long long)tau(t) * B + b) * G4 + jb;
                     *reinterpret_cast<uint4 *>(o) = vi;
                     *reinterpret_cast<uint4 *>(o + H) = vf;
                     *reinterpret_cast<uint4 *>(o + 2 * H) = vg;
@@ -511,6 +514,7 @@ struct Fwd3Params {
     // variable length (MASKED kernels): mask [T][B][H], 1 = real step,
     // 0 = padding (which keeps h_{t-1}, c_{t-1}); h0 [B][H] or NULL
     const __nv_bfloat16 *mask, *h0;
+    int reverse;  // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
     __nv_bfloat16 *y, *gates, *hT;
     float *cells, *cT;
     Ctrl *ctrl;
@@ -586,6 +590,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     const int H = p.H, B = p.B, T = p.T, I = p.I;
     const int kbase = (int)kpart * kcc * 64;  // this CTA's K range of W_h / h
     const int xbase = (int)kpart * kcx * 64;  // and of W_x / x
+    // time of recurrence step s (step s reads the state step s-1 left)
+    auto tau = [&](int s) { return p.reverse ? T - 1 - s : s; };
     const uint32_t WH_COL = 2 * NB, WX_COL = 2 * NB + 32 * kcc;
     unsigned int *ctr = &p.ctrl->bar[gi];
     const unsigned int group_ctas = (unsigned)(p.R * KS);
@@ -633,7 +639,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                         return false;
                     tc::mbar_arrive_expect_tx(&x_full[c], CHUNK);
                     tc::tma_load_2d(ring_x + c * CHUNK, &p.map_x, &x_full[c], xbase + 64 * c,
-                                    t * B + b0);
+                                    tau(t) * B + b0);
                     part_x = c + 1;
                 }
                 phx ^= 1;
@@ -655,7 +661,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 }
                 if (t > 0 || p.has_h0) {
                     const CUtensorMap *m = t > 0 ? &p.map_y : &p.map_h0;
-                    const int row0 = t > 0 ? (t - 1) * B + b0 : b0;
+                    const int row0 = t > 0 ? tau(t - 1) * B + b0 : b0;
                     for (int c = 0; c < kcc && !aborted; ++c) {
                         if (!tc::mbar_wait(&h_empty[c], phh ^ 1, p.ctrl, abort_flag, 0x703,
                                            p.wait_ns)) {
@@ -801,7 +807,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             for (int g = 0; g < 4; ++g)
                 bias[g][k] = p.bias ? __bfloat162float(p.bias[g * H + j]) : 0.f;
         }
-        auto load_mask = [&](int t) {
+        auto load_mask = [&](int s) {  // mask of step s (time tau(s))
+            const int t = tau(s);
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
                 const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
@@ -892,9 +899,10 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
 #pragma unroll
             for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
             rec::named_bar(1, F_EPI_THREADS);
-            __nv_bfloat16 *yt = p.y + (long long)t * B * H;
-            __nv_bfloat16 *gt = p.gates + (long long)t * B * 4 * H;
-            float *ct = p.cells + (long long)t * B * H;
+            const int tt = tau(t);  // time of this step
+            __nv_bfloat16 *yt = p.y + (long long)tt * B * H;
+            __nv_bfloat16 *gt = p.gates + (long long)tt * B * 4 * H;
+            float *ct = p.cells + (long long)tt * B * H;
             float gsave[4][NP];
 #pragma unroll
             for (int k = 0; k < NP; ++k) {

@@ -133,42 +133,57 @@ int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *d
              void *stream);
 
 /*
- * lstm_fwd_masked / lstm_bwd_masked -- lstm_fwd / lstm_bwd with the optional
- * variable-length input of the "SingleLayerLstmGrad" parameter table
- * (seq_length: a mask per step, sequence and hidden unit).
+ * lstm_fwd_ex / lstm_bwd_ex -- lstm_fwd / lstm_bwd with the optional input and
+ * the attribute of the "SingleLayerLstmGrad" parameter table that plain calls
+ * leave at their defaults.  opt NULL (or zero-initialised) = lstm_fwd /
+ * lstm_bwd.
  *
- *   mask  [T][B][H]   compute type  1 = real step, 0 = padding (no other
- *                                   values); NULL = every step real, exactly
- *                                   lstm_fwd / lstm_bwd
+ * seq_mask  [T][B][H], compute type: the variable-length input seq_length,
+ *   1 = real step, 0 = padding (no other values); NULL = every step real.
+ *   The page gives no formula for it.  Reading: at a padded element the state
+ *   does not move -- c_t = m c~_t + (1 - m) c_prev, h_t = m h~_t +
+ *   (1 - m) h_prev with c~, h~ the unmasked update -- y_t = h_t and
+ *   cells_t = c_t (gates are stored as computed), and the backward returns the
+ *   exact gradient of that function: padding passes delta h and delta c on
+ *   unchanged and has no gate gradient.  With per-sequence lengths
+ *   (mask[t][n][:] = t < L_n) every sequence behaves as the LSTM run on its
+ *   first L_n steps, carrying its final state through the padding.
  *
- * The page gives no formula for the mask.  Reading: at a padded element the
- * state does not move -- c_t = m c~_t + (1 - m) c_{t-1},
- * h_t = m h~_t + (1 - m) h_{t-1} with c~, h~ the unmasked update, and
- * y_t = h_t, cells_t = c_t (gates are stored as computed) -- and the backward
- * returns the exact gradient of that function: padding passes delta h and
- * delta c on unchanged and has no gate gradient.  With per-sequence lengths
- * (mask[t][n][:] = t < L_n) every sequence behaves as the LSTM run on its
- * first L_n steps, carrying its final state through the padding.
+ * direction  LSTM_DIR_FORWARD ("UNIDIRECTIONAL": the recurrence runs over
+ *   t = 0 .. T-1) or LSTM_DIR_REVERSE ("REDIRECTIONAL": t = T-1 .. 0; h0 / c0
+ *   precede the step at t = T-1, hT / cT follow the step at t = 0, dh0 / dc0
+ *   are the gradients at h0 / c0).  Tensor layouts are unchanged: y[t], gates[t],
+ *   dx[t] ... belong to time t in both directions.  A bidirectional layer is
+ *   one call in each direction.  Other values: LSTM_ERR_INVALID_ARG.
  *
- * The backward must receive the mask the forward received, and the forward's
- * saved y, gates and cells.  Other arguments, ownership, workspace sizes and
- * errors are those of lstm_fwd / lstm_bwd.
+ * The backward must receive the options the forward received, and the
+ * forward's saved y, gates and cells.  Other arguments, ownership, workspace
+ * sizes and errors are those of lstm_fwd / lstm_bwd.
  */
-int lstm_fwd_masked(const lstm_dims *d, const void *x, const void *W, const void *b,
-                    const void *h0, const float *c0, const void *mask, void *y, void *hT,
-                    float *cT, void *gates, float *cells, void *ws, size_t ws_bytes,
-                    void *stream);
-int lstm_bwd_masked(const lstm_dims *d, const void *mask, const void *dy, const void *dhT,
-                    const float *dcT, const void *x, const void *W, const void *h0,
-                    const float *c0, const void *y, const void *gates, const float *cells,
-                    float *dx, float *dW, float *db, float *dh0, float *dc0, void *ws,
-                    size_t ws_bytes, void *stream);
+#define LSTM_DIR_FORWARD 0
+#define LSTM_DIR_REVERSE 1
+typedef struct {
+    const void *seq_mask;
+    int direction;
+} lstm_options;
+
+int lstm_fwd_ex(const lstm_dims *d, const lstm_options *opt, const void *x, const void *W,
+                const void *b, const void *h0, const float *c0, void *y, void *hT, float *cT,
+                void *gates, float *cells, void *ws, size_t ws_bytes, void *stream);
+int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, const void *dhT,
+                const float *dcT, const void *x, const void *W, const void *h0,
+                const float *c0, const void *y, const void *gates, const float *cells,
+                float *dx, float *dW, float *db, float *dh0, float *dc0, void *ws,
+                size_t ws_bytes, void *stream);
 
 /*
  * lstm_status -- synchronise `stream`, then read and clear the device status
  * word kept in the first bytes of a workspace used by lstm_fwd / lstm_bwd.
- * Returns LSTM_OK, LSTM_ERR_TIMEOUT (a device-side wait gave up; the results of
- * that call are invalid), LSTM_ERR_CUDA, or LSTM_ERR_INVALID_ARG.
+ * Every call zeroes the word when it starts (in stream order), so it reports
+ * the most recent call on that workspace; a fresh workspace needs no
+ * initialisation.  Returns LSTM_OK, LSTM_ERR_TIMEOUT (a device-side wait gave
+ * up; the results of that call are invalid), LSTM_ERR_CUDA, or
+ * LSTM_ERR_INVALID_ARG.
  */
 int lstm_status(void *ws, size_t ws_bytes, void *stream);
 

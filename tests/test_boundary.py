@@ -153,3 +153,28 @@ def test_status_argument_checks(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError):
         L.load(str(tmp_path / "nope.so"))
+
+
+@pytest.mark.parametrize("direction", [-1, 2, 7])
+def test_unknown_direction_rejected(lib, direction):
+    """lstm_fwd_ex / lstm_bwd_ex reject a direction other than LSTM_DIR_FORWARD /
+    LSTM_DIR_REVERSE before anything is enqueued."""
+    opt = L.Options(None, direction)
+    a = fwd_args(D)
+    rc = lib.lstm_fwd_ex(ctypes.byref(D), ctypes.byref(opt), a["x"], a["W"], a["b"], a["h0"],
+                         a["c0"], a["y"], a["hT"], a["cT"], a["gates"], a["cells"], a["ws"],
+                         a["ws_bytes"], None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
+    rc = lib.lstm_bwd_ex(ctypes.byref(D), ctypes.byref(opt), None, None, None, FAKE, FAKE, None,
+                         None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                         L.bwd_workspace_size(D), None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
+
+
+def test_misaligned_mask_rejected(lib):
+    opt = L.Options(FAKE + 2, L.LSTM_DIR_FORWARD)
+    a = fwd_args(D)
+    rc = lib.lstm_fwd_ex(ctypes.byref(D), ctypes.byref(opt), a["x"], a["W"], a["b"], a["h0"],
+                         a["c0"], a["y"], a["hT"], a["cT"], a["gates"], a["cells"], a["ws"],
+                         a["ws_bytes"], None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
