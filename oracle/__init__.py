@@ -57,9 +57,9 @@ def _bind(path: str):
     lib.oracle_lstm_fwd.restype = i
     lib.oracle_lstm_bwd.argtypes = [i, i, i, i] + [dp] * 9 + [dp] * 6
     lib.oracle_lstm_bwd.restype = i
-    lib.oracle_lstm_fwd_ex.argtypes = [i, i, i, i] + [dp] * 6 + [i] + [dp] * 5
+    lib.oracle_lstm_fwd_ex.argtypes = [i, i, i, i] + [dp] * 6 + [i, i] + [dp] * 5
     lib.oracle_lstm_fwd_ex.restype = i
-    lib.oracle_lstm_bwd_ex.argtypes = [i, i, i, i] + [dp] * 5 + [i] + [dp] * 5 + [dp] * 6
+    lib.oracle_lstm_bwd_ex.argtypes = [i, i, i, i] + [dp] * 5 + [i, i] + [dp] * 5 + [dp] * 6
     lib.oracle_lstm_bwd_ex.restype = i
     lib.oracle_set_threads.argtypes = [i]
     lib.oracle_set_threads.restype = None
@@ -108,10 +108,11 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
-def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None, reverse=False):
+def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None, reverse=False, ijfo=False):
     """Forward pass.  Returns dict(y, gates, cells, hT, cT) of float64 arrays.
     mask [T][B][H] (1 = real step, 0 = padding) or None; reverse: the
-    recurrence runs over t = T-1 .. 0 (direction "REDIRECTIONAL")."""
+    recurrence runs over t = T-1 .. 0 (direction "REDIRECTIONAL"); ijfo: gate
+    row blocks in the order i, j (= g), f, o (gate_order "ijfo")."""
     x = _f64(x)
     T, B, I = x.shape
     W = _f64(W)
@@ -127,7 +128,8 @@ def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None, reverse=False)
     cT = np.empty((B, H))
     mask = _f64(mask, (T, B, H))
     rc = _load(lib).oracle_lstm_fwd_ex(T, B, I, H, _ptr(x), _ptr(W), _ptr(b), _ptr(h0),
-                                    _ptr(c0), _ptr(mask), int(bool(reverse)), _ptr(y),
+                                    _ptr(c0), _ptr(mask), int(bool(reverse)), int(bool(ijfo)),
+                                    _ptr(y),
                                     _ptr(gates), _ptr(cells), _ptr(hT), _ptr(cT))
     if rc != 0:
         raise RuntimeError("oracle_lstm_fwd failed")
@@ -135,7 +137,7 @@ def lstm_fwd(x, W, b=None, h0=None, c0=None, lib=None, mask=None, reverse=False)
 
 
 def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None,
-             reverse=False):
+             reverse=False, ijfo=False):
     """BPTT given the forward's saved state ``fwd`` (the dict lstm_fwd returns,
     run with the same mask and direction).
 
@@ -159,7 +161,8 @@ def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None
     dG = np.empty((T, B, 4 * H))
     mask = _f64(mask, (T, B, H))
     rc = _load(lib).oracle_lstm_bwd_ex(T, B, I, H, _ptr(x), _ptr(W), _ptr(h0), _ptr(c0),
-                                    _ptr(mask), int(bool(reverse)), _ptr(y), _ptr(gates),
+                                    _ptr(mask), int(bool(reverse)), int(bool(ijfo)), _ptr(y),
+                                    _ptr(gates),
                                     _ptr(cells),
                                  _ptr(dy), _ptr(dhT), _ptr(dcT),
                                  _ptr(dx), _ptr(dW), _ptr(db), _ptr(dh0), _ptr(dc0), _ptr(dG))
@@ -169,10 +172,10 @@ def lstm_bwd(x, W, h0, c0, fwd, dy=None, dhT=None, dcT=None, lib=None, mask=None
 
 
 def lstm_fwd_bwd(x, W, b=None, h0=None, c0=None, dy=None, dhT=None, dcT=None, lib=None,
-                 mask=None, reverse=False):
+                 mask=None, reverse=False, ijfo=False):
     """Forward then backward; returns the union of both result dicts."""
-    f = lstm_fwd(x, W, b, h0, c0, lib=lib, mask=mask, reverse=reverse)
-    g = lstm_bwd(x, W, h0, c0, f, dy, dhT, dcT, lib=lib, mask=mask, reverse=reverse)
+    f = lstm_fwd(x, W, b, h0, c0, lib=lib, mask=mask, reverse=reverse, ijfo=ijfo)
+    g = lstm_bwd(x, W, h0, c0, f, dy, dhT, dcT, lib=lib, mask=mask, reverse=reverse, ijfo=ijfo)
     out = dict(f)
     out.update(g)
     return out

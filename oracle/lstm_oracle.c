@@ -50,6 +50,10 @@
  * initC before the first step, t = T-1), and hT / cT are the state after the
  * last step (t = 0).
  *
+ * Gate order (the operator's "gate_order" attribute): "ifjo" (ijfo = 0) has the
+ * row blocks of W, b, gates and dG in the order i, f, j (= g), o; "ijfo"
+ * (ijfo = 1) in the order i, j, f, o.
+ *
  * Parity is pinned (tests/test_oracle.py) by central finite differences of the
  * surrogate loss L = sum_t <dy_t, h_t> + <dhT, h_{T-1}> + <dcT, c_{T-1}>,
  * by the T = 1 closed form, the W = 0 closed form, a hand-computed example,
@@ -99,9 +103,11 @@ static double sigm(double a)
 int oracle_lstm_fwd_ex(int T, int B, int I, int H,
                        const double *x, const double *W, const double *b,
                        const double *h0, const double *c0, const double *mask, int reverse,
-                       double *y, double *gates, double *cells,
+                       int ijfo, double *y, double *gates, double *cells,
                        double *hT, double *cT)
 {
+    /* row block of each gate */
+    const long BF = ijfo ? 2L * H : (long)H, BG = ijfo ? (long)H : 2L * H;
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
     const long K = (long)H + I;  /* length of z_t */
@@ -144,8 +150,8 @@ int oracle_lstm_fwd_ex(int T, int B, int I, int H,
             double *yt = y + ((long)t * B + n) * H;
             for (int j = 0; j < H; ++j) {
                 double i_ = sigm(a[j]);               /* input gate */
-                double f_ = sigm(a[H + j]);           /* forget gate */
-                double g_ = tanh(a[2L * H + j]);      /* candidate state */
+                double f_ = sigm(a[BF + j]);          /* forget gate */
+                double g_ = tanh(a[BG + j]);          /* candidate state */
                 double o_ = sigm(a[3L * H + j]);      /* output gate */
                 double c_ = f_ * cprev[j] + i_ * g_;  /* cell state */
                 double h_ = o_ * tanh(c_);            /* hidden state */
@@ -154,8 +160,8 @@ int oracle_lstm_fwd_ex(int T, int B, int I, int H,
                     h_ = mt[j] * h_ + (1.0 - mt[j]) * z[j];
                 }
                 gt[j] = i_;
-                gt[H + j] = f_;
-                gt[2L * H + j] = g_;
+                gt[BF + j] = f_;
+                gt[BG + j] = g_;
                 gt[3L * H + j] = o_;
                 ct[j] = c_;
                 yt[j] = h_;
@@ -178,7 +184,7 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
                     double *y, double *gates, double *cells,
                     double *hT, double *cT)
 {
-    return oracle_lstm_fwd_ex(T, B, I, H, x, W, b, h0, c0, NULL, 0, y, gates, cells, hT, cT);
+    return oracle_lstm_fwd_ex(T, B, I, H, x, W, b, h0, c0, NULL, 0, 0, y, gates, cells, hT, cT);
 }
 
 /* Backward pass, "backward algorithm (time step t -> t-1)" of
@@ -190,11 +196,12 @@ int oracle_lstm_fwd(int T, int B, int I, int H,
 int oracle_lstm_bwd_ex(int T, int B, int I, int H,
                        const double *x, const double *W,
                        const double *h0, const double *c0, const double *mask, int reverse,
-                       const double *y, const double *gates, const double *cells,
+                       int ijfo, const double *y, const double *gates, const double *cells,
                        const double *dy, const double *dhT, const double *dcT,
                        double *dx, double *dW, double *db,
                        double *dh0, double *dc0, double *dG)
 {
+    const long BF = ijfo ? 2L * H : (long)H, BG = ijfo ? (long)H : 2L * H;
     if (T < 0 || B < 0 || I < 0 || H < 0)
         return -1;
     const long K = (long)H + I;
@@ -237,7 +244,7 @@ int oracle_lstm_bwd_ex(int T, int B, int I, int H,
             const double *mt = mask ? mask + ((long)t * B + n) * H : NULL;
             double *dGt = dG + ((long)t * B + n) * G4;
             for (int j = 0; j < H; ++j) {
-                double i_ = gt[j], f_ = gt[H + j], g_ = gt[2L * H + j], o_ = gt[3L * H + j];
+                double i_ = gt[j], f_ = gt[BF + j], g_ = gt[BG + j], o_ = gt[3L * H + j];
                 double c_ = ct[j];
                 double c_prev = cp ? cp[j] : 0.0;
                 double tc = tanh(c_);
@@ -257,8 +264,8 @@ int oracle_lstm_bwd_ex(int T, int B, int I, int H,
                 double d_i = dc * g_ * i_ * (1.0 - i_);
                 double d_f = dc * c_prev * f_ * (1.0 - f_);
                 dGt[j] = d_i;
-                dGt[H + j] = d_f;
-                dGt[2L * H + j] = d_g;
+                dGt[BF + j] = d_f;
+                dGt[BG + j] = d_g;
                 dGt[3L * H + j] = d_o;
                 /* step 5: delta c_prev = delta c_t * f_t (+ what padding passes) */
                 dc_next[j] = dc * f_ + (1.0 - m) * dc_next[j];
@@ -330,6 +337,6 @@ int oracle_lstm_bwd(int T, int B, int I, int H,
                     double *dx, double *dW, double *db,
                     double *dh0, double *dc0, double *dG)
 {
-    return oracle_lstm_bwd_ex(T, B, I, H, x, W, h0, c0, NULL, 0, y, gates, cells, dy, dhT, dcT,
-                              dx, dW, db, dh0, dc0, dG);
+    return oracle_lstm_bwd_ex(T, B, I, H, x, W, h0, c0, NULL, 0, 0, y, gates, cells, dy, dhT,
+                              dcT, dx, dW, db, dh0, dc0, dG);
 }

@@ -39,20 +39,22 @@ def random_case(T, B, I, H, seed, wscale=1.5, dhdc=True, dy=True):
     return p, g
 
 
-def run(p, g, lib=None, mask=None, reverse=False):
+def run(p, g, lib=None, mask=None, reverse=False, ijfo=False):
     return oracle.lstm_fwd_bwd(p["x"], p["W"], p["b"], p["h0"], p["c0"],
-                               g["dy"], g["dhT"], g["dcT"], lib=lib, mask=mask, reverse=reverse)
+                               g["dy"], g["dhT"], g["dcT"], lib=lib, mask=mask, reverse=reverse,
+                               ijfo=ijfo)
 
 
-def loss(p, g, lib=None, mask=None, reverse=False):
+def loss(p, g, lib=None, mask=None, reverse=False, ijfo=False):
     f = oracle.lstm_fwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], lib=lib, mask=mask,
-                        reverse=reverse)
+                        reverse=reverse, ijfo=ijfo)
     return oracle.surrogate_loss(f, g["dy"], g["dhT"], g["dcT"])
 
 
-def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None, reverse=False):
+def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None, reverse=False,
+                 ijfo=False):
     """max over checked entries of |analytic - central FD| / max(1, |analytic|)."""
-    out = run(p, g, lib, mask, reverse)
+    out = run(p, g, lib, mask, reverse, ijfo)
     rng = np.random.default_rng(seed)
     worst = 0.0
     for name, gname in GRAD_OF.items():
@@ -66,9 +68,9 @@ def fd_max_error(p, g, lib=None, max_entries=None, seed=0, mask=None, reverse=Fa
             old = flat[k]
             h = 1e-6 * max(1.0, abs(old))
             flat[k] = old + h
-            lp = loss(p, g, lib, mask, reverse)
+            lp = loss(p, g, lib, mask, reverse, ijfo)
             flat[k] = old - h
-            lm = loss(p, g, lib, mask, reverse)
+            lm = loss(p, g, lib, mask, reverse, ijfo)
             flat[k] = old
             fd = (lp - lm) / (2 * h)
             worst = max(worst, abs(fd - an[k]) / max(1.0, abs(an[k])))
@@ -406,3 +408,35 @@ def test_reverse_is_forward_on_flipped_time():
         np.testing.assert_allclose(rev[k], fwd[k][::-1], rtol=1e-12, atol=1e-13, err_msg=k)
     for k in ("hT", "cT", "dW", "db", "dh0", "dc0"):
         np.testing.assert_allclose(rev[k], fwd[k], rtol=1e-11, atol=1e-12, err_msg=k)
+
+
+# ---------------------------------------------------------------- gate order
+# The operator's "gate_order" attribute: "ifjo" (the default reading) or
+# "ijfo", the row blocks of W, b, the saved gates and dG in the order i, j, f, o.
+
+def _swap_fg_blocks(a, H, axis):
+    """Exchange row blocks 1 and 2 (f and j) of a [.. 4H ..] array."""
+    idx = np.r_[0:H, 2 * H:3 * H, H:2 * H, 3 * H:4 * H]
+    return np.take(a, idx, axis=axis)
+
+
+def test_ijfo_finite_differences():
+    p, g = random_case(3, 2, 3, 4, seed=611)
+    assert fd_max_error(p, g, ijfo=True) < 1e-6
+
+
+def test_ijfo_is_ifjo_with_blocks_swapped():
+    """gate_order "ijfo" on W, b equals "ifjo" on the same weights with row
+    blocks 1 and 2 exchanged; gates, dG-shaped outputs (dW rows, db) come back
+    with the blocks exchanged, everything else equal."""
+    T, B, I, H = 4, 3, 5, 6
+    p, g = random_case(T, B, I, H, seed=612)
+    a = run(p, g, ijfo=True)
+    q = dict(p, W=_swap_fg_blocks(p["W"], H, 0), b=_swap_fg_blocks(p["b"], H, 0))
+    r = run(q, g)
+    for k in ("y", "cells", "hT", "cT", "dx", "dh0", "dc0"):
+        np.testing.assert_allclose(a[k], r[k], rtol=1e-12, atol=1e-13, err_msg=k)
+    np.testing.assert_allclose(a["gates"], _swap_fg_blocks(r["gates"], H, 2), rtol=1e-12,
+                               atol=1e-13)
+    np.testing.assert_allclose(a["dW"], _swap_fg_blocks(r["dW"], H, 0), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(a["db"], _swap_fg_blocks(r["db"], H, 0), rtol=1e-11, atol=1e-12)

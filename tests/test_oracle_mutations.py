@@ -24,8 +24,8 @@ MUTATIONS = {
     "sign_df": ("double d_f = dc * c_prev * f_ * (1.0 - f_);",
                 "double d_f = dc * c_prev * f_ * (1.0 + f_);"),
     # i and f gradients stored in each other's rows
-    "swap_rows": ("dGt[j] = d_i;\n                dGt[H + j] = d_f;",
-                  "dGt[j] = d_f;\n                dGt[H + j] = d_i;"),
+    "swap_rows": ("dGt[j] = d_i;\n                dGt[BF + j] = d_f;",
+                  "dGt[j] = d_f;\n                dGt[BF + j] = d_i;"),
     # c_t used where c_{t-1} belongs in the forget-gate gradient
     "wrong_cprev": ("double d_f = dc * c_prev * f_ * (1.0 - f_);",
                     "double d_f = dc * c_ * f_ * (1.0 - f_);"),
