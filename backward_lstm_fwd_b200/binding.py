@@ -46,12 +46,16 @@ class Dims(ctypes.Structure):
 
 
 LSTM_DIR_FORWARD, LSTM_DIR_REVERSE = 0, 1
+LSTM_GATES_IFJO, LSTM_GATES_IJFO = 0, 1
+GATE_ORDERS = {"ifjo": LSTM_GATES_IFJO, "ijfo": LSTM_GATES_IJFO}
 
 
 class Options(ctypes.Structure):
-    """lstm_options: the seq_length mask (device pointer or None) and the
-    direction (LSTM_DIR_FORWARD / LSTM_DIR_REVERSE)."""
-    _fields_ = [("seq_mask", ctypes.c_void_p), ("direction", ctypes.c_int)]
+    """lstm_options: the seq_length mask (device pointer or None), the
+    direction (LSTM_DIR_FORWARD / LSTM_DIR_REVERSE) and the gate_order
+    (LSTM_GATES_IFJO / LSTM_GATES_IJFO)."""
+    _fields_ = [("seq_mask", ctypes.c_void_p), ("direction", ctypes.c_int),
+                ("gate_order", ctypes.c_int)]
 
 
 _lib = None
@@ -152,23 +156,34 @@ def bwd_workspace_size(d: Dims) -> int:
     return int(load().lstm_bwd_workspace_size(ctypes.byref(d)))
 
 
-def _options(mask, reverse):
-    return Options(_p(mask), LSTM_DIR_REVERSE if reverse else LSTM_DIR_FORWARD)
+def _gate_order(gate_order) -> int:
+    """"ifjo" / "ijfo" (the attribute's values) or the C constant itself."""
+    return GATE_ORDERS[gate_order] if isinstance(gate_order, str) else int(gate_order)
+
+
+def _options(mask, reverse, gate_order):
+    return Options(_p(mask), LSTM_DIR_REVERSE if reverse else LSTM_DIR_FORWARD,
+                   _gate_order(gate_order))
+
+
+def _plain(mask, reverse, gate_order) -> bool:
+    return mask is None and not reverse and _gate_order(gate_order) == LSTM_GATES_IFJO
 
 
 def lstm_fwd(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes=None,
-             stream=None, check: bool = True, mask=None, reverse: bool = False) -> int:
+             stream=None, check: bool = True, mask=None, reverse: bool = False,
+             gate_order="ifjo") -> int:
     """Direct call of the C entry point lstm_fwd, or lstm_fwd_ex with a
-    variable-length mask [T,B,H] (1 = real step, 0 = padding) and / or the
-    reverse direction (device tensors or raw pointers)."""
+    variable-length mask [T,B,H] (1 = real step, 0 = padding), the reverse
+    direction and / or gate_order "ijfo" (device tensors or raw pointers)."""
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
-    if mask is None and not reverse:
+    if _plain(mask, reverse, gate_order):
         rc = load().lstm_fwd(ctypes.byref(d), _p(x), _p(W), _p(b), _p(h0), _p(c0), _p(y),
                              _p(hT), _p(cT), _p(gates), _p(cells), _p(ws), ws_bytes,
                              _stream(stream))
     else:
-        opt = _options(mask, reverse)
+        opt = _options(mask, reverse, gate_order)
         rc = load().lstm_fwd_ex(ctypes.byref(d), ctypes.byref(opt), _p(x), _p(W), _p(b), _p(h0),
                                 _p(c0), _p(y), _p(hT), _p(cT), _p(gates), _p(cells), _p(ws),
                                 ws_bytes, _stream(stream))
@@ -179,17 +194,17 @@ def lstm_fwd(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes=Non
 
 def lstm_bwd(d: Dims, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0, ws,
              ws_bytes=None, stream=None, check: bool = True, mask=None,
-             reverse: bool = False) -> int:
+             reverse: bool = False, gate_order="ifjo") -> int:
     """Direct call of the C entry point lstm_bwd, or lstm_bwd_ex with the
-    forward's mask and direction (device tensors or raw pointers)."""
+    forward's mask, direction and gate_order (device tensors or raw pointers)."""
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
-    if mask is None and not reverse:
+    if _plain(mask, reverse, gate_order):
         rc = load().lstm_bwd(ctypes.byref(d), _p(dy), _p(dhT), _p(dcT), _p(x), _p(W), _p(h0),
                              _p(c0), _p(y), _p(gates), _p(cells), _p(dx), _p(dW), _p(db),
                              _p(dh0), _p(dc0), _p(ws), ws_bytes, _stream(stream))
     else:
-        opt = _options(mask, reverse)
+        opt = _options(mask, reverse, gate_order)
         rc = load().lstm_bwd_ex(ctypes.byref(d), ctypes.byref(opt), _p(dy), _p(dhT), _p(dcT),
                                 _p(x), _p(W), _p(h0), _p(c0), _p(y), _p(gates), _p(cells),
                                 _p(dx), _p(dW), _p(db), _p(dh0), _p(dc0), _p(ws), ws_bytes,
@@ -291,9 +306,9 @@ class Grads:
 
 
 def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None, mask=None,
-            reverse: bool = False) -> State:
-    """Allocate outputs and run lstm_fwd (lstm_fwd_ex with a mask or the
-    reverse direction).  x [T,B,I], W [4H,H+I] and mask [T,B,H] share the
+            reverse: bool = False, gate_order="ifjo") -> State:
+    """Allocate outputs and run lstm_fwd (lstm_fwd_ex with a mask, the
+    reverse direction or gate_order "ijfo").  x [T,B,I], W [4H,H+I] and mask [T,B,H] share the
     compute dtype (float32 or bfloat16); c0 is float32."""
     T, B, I = x.shape
     H = W.shape[0] // 4
@@ -301,19 +316,20 @@ def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None, mask=None,
     if ws is None:
         ws = empty_workspace(fwd_workspace_size(st.dims), x.device)
     lstm_fwd(st.dims, x, W, b, h0, c0, st.y, st.hT, st.cT, st.gates, st.cells, ws, stream=stream,
-             mask=mask, reverse=reverse)
+             mask=mask, reverse=reverse, gate_order=gate_order)
     return st
 
 
 def backward(st: State, x, W, h0=None, c0=None, dy=None, dhT=None, dcT=None, ws=None,
-             stream=None, mask=None, reverse: bool = False) -> Grads:
+             stream=None, mask=None, reverse: bool = False, gate_order="ifjo") -> Grads:
     """Allocate gradients and run lstm_bwd on the saved state of forward()
-    (lstm_bwd_ex with the forward's mask and direction)."""
+    (lstm_bwd_ex with the forward's mask, direction and gate_order)."""
     T, B, I = x.shape
     H = W.shape[0] // 4
     g = Grads(T, B, I, H, x.device)
     if ws is None:
         ws = empty_workspace(bwd_workspace_size(st.dims), x.device)
     lstm_bwd(st.dims, dy, dhT, dcT, x, W, h0, c0, st.y, st.gates, st.cells, g.dx, g.dW, g.db,
-             g.dh0, g.dc0, ws, stream=stream, mask=mask, reverse=reverse)
+             g.dh0, g.dc0, ws, stream=stream, mask=mask, reverse=reverse,
+             gate_order=gate_order)
     return g

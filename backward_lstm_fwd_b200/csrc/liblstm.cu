@@ -665,7 +665,7 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     while (stages >= rec3::MIN_STAGES && (size_t)rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
     if (stages < rec3::MIN_STAGES) return false;
     P.smem = rec3::Bwd3Smem(stages).total + 1024;
-    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel<false>, rec3::THREADS,
+    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel<false, false>, rec3::THREADS,
                                          P.smem, P.KS);
     const int gmax = std::min(maxc / P.R, kMaxGroups);
     if (gmax < 1) return false;
@@ -796,8 +796,8 @@ cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStre
 // LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
 int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, const bf16 *W,
                        const bf16 *b, const bf16 *h0, const float *c0, const bf16 *mask,
-                       bool reverse, bf16 *y, bf16 *hT, float *cT, bf16 *gates, float *cells,
-                       Ctrl *ctrl, cudaStream_t s) {
+                       bool reverse, bool ijfo, bf16 *y, bf16 *hT, float *cT, bf16 *gates,
+                       float *cells, Ctrl *ctrl, cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, I = d->I;
     rec3::Fwd3Params prm;
     memset(&prm, 0, sizeof(prm));
@@ -807,7 +807,7 @@ int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, con
     else prm.map_h0 = prm.map_y;
     if (!ok) return LSTM_ERR_UNSUPPORTED;
     prm.W = W; prm.bias = b; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
-    prm.mask = mask; prm.h0 = h0; prm.reverse = reverse;
+    prm.mask = mask; prm.h0 = h0; prm.reverse = reverse; prm.ijfo = ijfo;
     prm.cells = cells; prm.cT = cT; prm.ctrl = ctrl;
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.I = (int)I; prm.R = P.R; prm.G = P.G;
     prm.kcc = P.kcc; prm.kcx = P.kcx;
@@ -863,7 +863,7 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 // [i0, i1) (time steps T-i1 .. T-i0-1); WT must already hold W_h^T.
 int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
                    const float *dcT, const float *c0, const bf16 *mask, bool reverse,
-                   const bf16 *gates, const float *cells, bf16 *dG, const bf16 *WT,
+                   bool ijfo, const bf16 *gates, const float *cells, bf16 *dG, const bf16 *WT,
                    float *dbgroup, float *dh0, float *dc0, float *dc_carry, float *dhp_carry,
                    Ctrl *ctrl, int i0, int i1, cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
@@ -881,11 +881,16 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const 
     prm.i0 = i0; prm.i1 = i1; prm.reverse = reverse;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
+    const int nctas = P.R * P.KS * P.G;
     const cudaError_t e =
-        mask ? launch_cluster(rec3::bwd3_kernel<true>, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
-                              rec3::THREADS)
-             : launch_cluster(rec3::bwd3_kernel<false>, prm, P.R * P.KS * P.G, P.KS, P.smem, s,
-                              rec3::THREADS);
+        mask ? (ijfo ? launch_cluster(rec3::bwd3_kernel<true, true>, prm, nctas, P.KS, P.smem, s,
+                                      rec3::THREADS)
+                     : launch_cluster(rec3::bwd3_kernel<true, false>, prm, nctas, P.KS, P.smem, s,
+                                      rec3::THREADS))
+             : (ijfo ? launch_cluster(rec3::bwd3_kernel<false, true>, prm, nctas, P.KS, P.smem, s,
+                                      rec3::THREADS)
+                     : launch_cluster(rec3::bwd3_kernel<false, false>, prm, nctas, P.KS, P.smem,
+                                      s, rec3::THREADS));
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
@@ -905,13 +910,14 @@ cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cud
 // workspace first, then copied into each CTA's tensor memory), one launch.
 int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
                        const float *dcT, const bf16 *W, const float *c0, const bf16 *mask,
-                       bool reverse, const bf16 *gates, const float *cells, bf16 *dG, bf16 *WT,
+                       bool reverse, bool ijfo, const bf16 *gates, const float *cells, bf16 *dG,
+                       bf16 *WT,
                        float *dbgroup, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
     const long long G4 = 4LL * d->H;
     if (launch_transpose_wh(d, W, WT, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, gates, cells, dG, WT,
-                                  dbgroup, dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
+    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG,
+                                  WT, dbgroup, dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
     if (rc != LSTM_OK) return rc;
     simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
     note_launch();
@@ -927,7 +933,8 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int nch,
                        const bf16 *dy, const bf16 *dhT, const float *dcT, const bf16 *x,
                        const bf16 *W, const bf16 *h0, const float *c0, const bf16 *mask,
-                       bool reverse, const bf16 *y, const bf16 *gates, const float *cells,
+                       bool reverse, bool ijfo, const bf16 *y, const bf16 *gates,
+                       const float *cells,
                        bf16 *dG, bf16 *WT, float *dbgroup, float *dc_carry, float *dhp_carry,
                        float *dx, float *dW, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
@@ -950,7 +957,7 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
         for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
             const int i0 = (int)((long long)T * c / nch), i1 = (int)((long long)T * (c + 1) / nch);
-            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, gates, cells, dG, WT,
+            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
                                 dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
             if (rc != LSTM_OK) break;
             if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
@@ -987,10 +994,10 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
 // kernel or the per-step kernels only.
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
-             const float *c0, const T *mask, bool reverse, T *y, T *hT, float *cT, T *gates,
-             float *cells, char *ws, cudaStream_t s) {
-    // masked or reverse-direction calls: TMEM-weight kernel or per-step kernels
-    const bool special = mask != nullptr || reverse;
+             const float *c0, const T *mask, bool reverse, bool ijfo, T *y, T *hT, float *cT,
+             T *gates, float *cells, char *ws, cudaStream_t s) {
+    // masked, reverse-direction or "ijfo" calls: TMEM-weight kernel or per-step kernels
+    const bool special = mask != nullptr || reverse || ijfo;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H;
     const FwdLayout L = fwd_layout(d);
@@ -1001,7 +1008,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
             const int rc = tc_fwd_recurrence3(d, plan3, (const bf16 *)x, (const bf16 *)W,
                                               (const bf16 *)b, (const bf16 *)h0, c0,
-                                              (const bf16 *)mask, reverse, (bf16 *)y,
+                                              (const bf16 *)mask, reverse, ijfo, (bf16 *)y,
                                               (bf16 *)hT, cT, (bf16 *)gates, cells,
                                               (Ctrl *)ws, s);
             g_last_fwd_path = 3;
@@ -1050,6 +1057,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
                 ep.mask = mask + (long long)t * BH;
                 ep.hprev = hp;
             }
+            ep.fb = ijfo ? 2 : 1;
             LSTM_TRY((simt::gemm<true, true>(B, 4 * H, H, simt::Hprev<T>{hp, H},
                                               simt::WhT4<T>{W, H, I}, ep, s)));
         }
@@ -1075,10 +1083,10 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
 // kernel or the per-step kernels only.
 template <class T>
 int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, const T *x,
-             const T *W, const T *h0, const float *c0, const T *mask, bool reverse, const T *y,
-             const T *gates, const float *cells, float *dx, float *dW, float *db, float *dh0,
-             float *dc0, char *ws, cudaStream_t s) {
-    const bool special = mask != nullptr || reverse;
+             const T *W, const T *h0, const float *c0, const T *mask, bool reverse, bool ijfo,
+             const T *y, const T *gates, const float *cells, float *dx, float *dW, float *db,
+             float *dh0, float *dc0, char *ws, cudaStream_t s) {
+    const bool special = mask != nullptr || reverse || ijfo;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H, TB = (long long)T_ * B;
     const int G4 = 4 * H, K = H + I;
@@ -1112,7 +1120,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                 const int rc = tc_bwd3_overlapped(
                     d, plan3, *A, bwd_chunks(d), (const bf16 *)dy, (const bf16 *)dhT, dcT,
                     (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)mask,
-                    reverse, (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
+                    reverse, ijfo, (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
                     (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), (float *)(ws + L.dc),
                     (float *)(ws + L.dhp), dx, dW, db, dh0, dc0, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
@@ -1124,7 +1132,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
             g_last_bwd_path = v3 ? 3 : 2;
             if (v3)
                 rc = tc_bwd_recurrence3(d, plan3, (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                                        (const bf16 *)W, c0, (const bf16 *)mask, reverse,
+                                        (const bf16 *)W, c0, (const bf16 *)mask, reverse, ijfo,
                                         (const bf16 *)gates, cells, (bf16 *)dG,
                                         (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), db, dh0,
                                         dc0, (Ctrl *)ws, s);
@@ -1187,6 +1195,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         ep.dc_out = (st == 0) ? dc0 : dcbuf[st & 1];
         ep.H = H;
         ep.use_acc = !last;
+        ep.fb = ijfo ? 2 : 1;
         if (mask) {
             ep.mask = mask + t * BH;
             ep.dhp_in = last ? nullptr : dhpbuf[(st + 1) & 1];
@@ -1278,6 +1287,9 @@ int fwd_entry(const lstm_dims *d, const lstm_options *opt, const void *x, const 
     const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
     if (dir != LSTM_DIR_FORWARD && dir != LSTM_DIR_REVERSE) return LSTM_ERR_INVALID_ARG;
     const bool reverse = dir == LSTM_DIR_REVERSE;
+    const int order = opt ? opt->gate_order : LSTM_GATES_IFJO;
+    if (order != LSTM_GATES_IFJO && order != LSTM_GATES_IJFO) return LSTM_ERR_INVALID_ARG;
+    const bool ijfo = order == LSTM_GATES_IJFO;
     if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
     const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
     if (!ptr_ok(x, TB * d->I > 0) || !ptr_ok(W, d->H > 0) || !ptr_ok(b, false) ||
@@ -1291,12 +1303,12 @@ int fwd_entry(const lstm_dims *d, const lstm_options *opt, const void *x, const 
     if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
     if (d->dtype == LSTM_F32)
         return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
-                               (const float *)h0, c0, (const float *)mask, reverse, (float *)y,
-                               (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
+                               (const float *)h0, c0, (const float *)mask, reverse, ijfo,
+                               (float *)y, (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
     typedef __nv_bfloat16 bf;
     return fwd_simt<bf>(d, (const bf *)x, (const bf *)W, (const bf *)b, (const bf *)h0, c0,
-                        (const bf *)mask, reverse, (bf *)y, (bf *)hT, cT, (bf *)gates, cells,
-                        (char *)ws, s);
+                        (const bf *)mask, reverse, ijfo, (bf *)y, (bf *)hT, cT, (bf *)gates,
+                        cells, (char *)ws, s);
 }
 
 int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const void *dhT,
@@ -1308,6 +1320,9 @@ int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const
     const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
     if (dir != LSTM_DIR_FORWARD && dir != LSTM_DIR_REVERSE) return LSTM_ERR_INVALID_ARG;
     const bool reverse = dir == LSTM_DIR_REVERSE;
+    const int order = opt ? opt->gate_order : LSTM_GATES_IFJO;
+    if (order != LSTM_GATES_IFJO && order != LSTM_GATES_IJFO) return LSTM_ERR_INVALID_ARG;
+    const bool ijfo = order == LSTM_GATES_IJFO;
     if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
     const long long TB = (long long)d->T * d->B, BH = (long long)d->B * d->H;
     const long long G4 = 4LL * d->H, K = (long long)d->H + d->I;
@@ -1325,11 +1340,11 @@ int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const
     if (d->dtype == LSTM_F32)
         return bwd_simt<float>(d, (const float *)dy, (const float *)dhT, dcT, (const float *)x,
                                (const float *)W, (const float *)h0, c0, (const float *)mask,
-                               reverse, (const float *)y, (const float *)gates, cells, dx, dW,
-                               db, dh0, dc0, (char *)ws, s);
+                               reverse, ijfo, (const float *)y, (const float *)gates, cells, dx,
+                               dW, db, dh0, dc0, (char *)ws, s);
     typedef __nv_bfloat16 bf;
     return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
-                        (const bf *)h0, c0, (const bf *)mask, reverse, (const bf *)y,
+                        (const bf *)h0, c0, (const bf *)mask, reverse, ijfo, (const bf *)y,
                         (const bf *)gates, cells, dx, dW, db, dh0, dc0, (char *)ws, s);
 }
 }  // namespace

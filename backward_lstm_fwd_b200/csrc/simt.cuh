@@ -172,13 +172,17 @@ template <class T> struct EpFwdStep {
     // h_{t-1} = y[t-1] or h0, and c_{t-1}); NULL = every step real
     const T *mask = nullptr;
     const T *hprev = nullptr;
+    // row block of the forget gate: 1 for gate_order "ifjo", 2 for "ijfo"
+    // (the candidate j = g takes the other of blocks 1 and 2)
+    int fb = 1;
     __device__ void operator()(int m, int q0, const float *acc) const {
         const int j = q0 >> 2;
         if (j >= H) return;
+        const int gb = 3 - fb;
         const float *gx = Gx + (long long)m * 4 * H;
         const float ig = sigmoidf_(acc[0] + gx[j]);
-        const float fg = sigmoidf_(acc[1] + gx[H + j]);
-        const float gg = tanhf_(acc[2] + gx[2 * H + j]);
+        const float fg = sigmoidf_(acc[fb] + gx[fb * H + j]);
+        const float gg = tanhf_(acc[gb] + gx[gb * H + j]);
         const float og = sigmoidf_(acc[3] + gx[3 * H + j]);
         const float cp = cprev ? cprev[(long long)m * H + j] : 0.f;
         float c = fg * cp + ig * gg;
@@ -191,8 +195,8 @@ template <class T> struct EpFwdStep {
         }
         T *gt = gates + (long long)m * 4 * H;
         gt[j] = from_f<T>(ig);
-        gt[H + j] = from_f<T>(fg);
-        gt[2 * H + j] = from_f<T>(gg);
+        gt[fb * H + j] = from_f<T>(fg);
+        gt[gb * H + j] = from_f<T>(gg);
         gt[3 * H + j] = from_f<T>(og);
         cells[(long long)m * H + j] = c;
         y[(long long)m * H + j] = from_f<T>(h);
@@ -217,7 +221,9 @@ template <class T> struct EpBwdStep {
     const T *mask = nullptr;
     const float *dhp_in = nullptr;
     float *dhp_out = nullptr;
+    int fb = 1;  // row block of the forget gate (2 for gate_order "ijfo")
     __device__ void operator()(int m, int n0, const float *acc) const {
+        const int gb = 3 - fb;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int j = n0 + c;
@@ -238,8 +244,8 @@ template <class T> struct EpBwdStep {
             const float dc_pass = __fmul_rn(1.f - mk, dcn);
             dcn = __fmul_rn(dcn, mk);
             const T *g4 = gates + (long long)m * 4 * H;
-            const float ig = to_f(g4[j]), fg = to_f(g4[H + j]);
-            const float gg = to_f(g4[2 * H + j]), og = to_f(g4[3 * H + j]);
+            const float ig = to_f(g4[j]), fg = to_f(g4[fb * H + j]);
+            const float gg = to_f(g4[gb * H + j]), og = to_f(g4[3 * H + j]);
             const float ct = cells[o];
             const float cp = cprev ? cprev[o] : 0.f;
             const float tc = tanhf_(ct);
@@ -250,8 +256,8 @@ template <class T> struct EpBwdStep {
             const float d_f = dc * cp * fg * (1.f - fg);
             T *d4 = dG + (long long)m * 4 * H;
             d4[j] = from_f<T>(d_i);
-            d4[H + j] = from_f<T>(d_f);
-            d4[2 * H + j] = from_f<T>(d_g);
+            d4[fb * H + j] = from_f<T>(d_f);
+            d4[gb * H + j] = from_f<T>(d_g);
             d4[3 * H + j] = from_f<T>(d_o);
             dc_out[o] = dc * fg + dc_pass;                             // step 5
         }

@@ -89,7 +89,9 @@ __device__ __forceinline__ int part_off(int r, int n) {
     return r * NMAX + ((((n >> 2) ^ (r & 7)) << 2) | (n & 3));
 }
 
-template <bool MASKED>
+// MASKED: variable-length mask; IJFO: gate_order "ijfo" (a template argument,
+// not a runtime one: the epilogue is at the register limit of its launch)
+template <bool MASKED, bool IJFO>
 __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant__ Bwd3Params p) {
     constexpr int UPT = 8;  // units per epilogue thread in the pointwise part
     extern __shared__ uint8_t smem_raw[];
@@ -249,6 +251,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         float *stage_buf = reinterpret_cast<float *>(ring);
         const uint32_t recv_lo = tc::smem_u32(recv), recvbar_lo = tc::smem_u32(recv_full);
         float dc[UPT], dbacc[4][UPT];
+        // row block of each gate role i, f, g, o (gate_order); the registers
+        // below hold the gates by role
+        constexpr int kBlk[4] = {0, IJFO ? 2 : 1, IJFO ? 1 : 2, 3};
         uint4 gpk[4], dypk;  // prefetched gates and dy of the next step, still packed bf16
         uint4 mpk;           // and its mask (MASKED)
         float ct[UPT], cp[UPT];
@@ -274,7 +279,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             const long long row = (long long)tau(t) * B + b;  // t: a step, not a time
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-                gpk[g] = __ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + g * H + jb));
+                gpk[g] = __ldg(reinterpret_cast<const uint4 *>(p.gates + row * G4 + kBlk[g] * H + jb));
             const float4 *c4 = reinterpret_cast<const float4 *>(p.cells + row * H + jb);
             const float4 x0 = __ldg(c4), x1 = __ldg(c4 + 1);
             ct[0] = x0.x; ct[1] = x0.y; ct[2] = x0.z; ct[3] = x0.w;
@@ -413,8 +418,8 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 if (valid) {
                     __nv_bfloat16 *o = p.dG + ((long long)tau(t) * B + b) * G4 + jb;
                     *reinterpret_cast<uint4 *>(o) = vi;
-                    *reinterpret_cast<uint4 *>(o + H) = vf;
-                    *reinterpret_cast<uint4 *>(o + 2 * H) = vg;
+                    *reinterpret_cast<uint4 *>(o + kBlk[1] * H) = vf;
+                    *reinterpret_cast<uint4 *>(o + kBlk[2] * H) = vg;
                     *reinterpret_cast<uint4 *>(o + 3 * H) = vo;
                 }
                 if (valid) {
@@ -482,8 +487,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             if (et < 64) {
                 float sum = 0.f;
                 for (int r = 0; r < NMAX; ++r) sum += red[r * 64 + et];
-                const int g = et / UPC, u = et % UPC;
-                float *dst = p.db_part + (long long)gi * G4 + (long long)g * H + j0 + (int)kpart * UPC + u;
+                const int g = et / UPC, u = et % UPC;  // g: the role
+                const int blk = IJFO && (g == 1 || g == 2) ? 3 - g : g;
+                float *dst = p.db_part + (long long)gi * G4 + (long long)blk * H + j0 + (int)kpart * UPC + u;
                 *dst = first ? sum : *dst + sum;  // launches of one call run in order
             }
         }
@@ -515,6 +521,7 @@ struct Fwd3Params {
     // 0 = padding (which keeps h_{t-1}, c_{t-1}); h0 [B][H] or NULL
     const __nv_bfloat16 *mask, *h0;
     int reverse;  // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
+    int ijfo;     // gate_order "ijfo": row blocks i, j (= g), f, o instead of i, f, j, o
     __nv_bfloat16 *y, *gates, *hT;
     float *cells, *cT;
     Ctrl *ctrl;
@@ -900,6 +907,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
             rec::named_bar(1, F_EPI_THREADS);
             const int tt = tau(t);  // time of this step
+            // row blocks of the forget gate and the candidate (gate_order)
+            const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
             __nv_bfloat16 *yt = p.y + (long long)tt * B * H;
             __nv_bfloat16 *gt = p.gates + (long long)tt * B * 4 * H;
             float *ct = p.cells + (long long)tt * B * H;
@@ -909,9 +918,11 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 const int n = pair_col(k), uu = pair_unit(k);
                 if (n >= NBc) continue;
                 const int b = bc0 + n, j = u0 + uu;
+                const float bf_ = fb == 1 ? bias[1][k] : bias[2][k];
+                const float bg_ = fb == 1 ? bias[2][k] : bias[1][k];
                 const float ig = rec::sigmoid_fast(xbuf[(0 * NBc + n) * F_UNITS + uu] + bias[0][k]);
-                const float fg = rec::sigmoid_fast(xbuf[(1 * NBc + n) * F_UNITS + uu] + bias[1][k]);
-                const float gg = rec::tanh_fast(xbuf[(2 * NBc + n) * F_UNITS + uu] + bias[2][k]);
+                const float fg = rec::sigmoid_fast(xbuf[(fb * NBc + n) * F_UNITS + uu] + bf_);
+                const float gg = rec::tanh_fast(xbuf[(gb * NBc + n) * F_UNITS + uu] + bg_);
                 const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
                 const float cn = fg * c[k] + ig * gg;
                 float h = og * rec::tanh_fast(cn);
@@ -948,9 +959,10 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 if (n >= NBc || b >= B) continue;
                 ct[(long long)b * H + j] = c[k];
                 __nv_bfloat16 *g4 = gt + (long long)b * 4 * H + j;
+                const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
                 g4[0] = __float2bfloat16_rn(gsave[0][k]);
-                g4[H] = __float2bfloat16_rn(gsave[1][k]);
-                g4[2 * H] = __float2bfloat16_rn(gsave[2][k]);
+                g4[fb * H] = __float2bfloat16_rn(gsave[1][k]);
+                g4[gb * H] = __float2bfloat16_rn(gsave[2][k]);
                 g4[3 * H] = __float2bfloat16_rn(gsave[3][k]);
             }
             if (MASKED && t + 1 < T) load_mask(t + 1);

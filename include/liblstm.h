@@ -156,15 +156,24 @@ int lstm_bwd(const lstm_dims *d, const void *dy, const void *dhT, const float *d
  *   dx[t] ... belong to time t in both directions.  A bidirectional layer is
  *   one call in each direction.  Other values: LSTM_ERR_INVALID_ARG.
  *
+ * gate_order  LSTM_GATES_IFJO (the default, "ifjo": the 4H rows of W, b, gates
+ *   and dG are the row blocks [i | f | g | o]) or LSTM_GATES_IJFO ("ijfo":
+ *   [i | g | f | o], the candidate j = g in block 1 and the forget gate in
+ *   block 2).  The attribute only names which row block plays which role; the
+ *   arithmetic of every gate is unchanged.  Other values: LSTM_ERR_INVALID_ARG.
+ *
  * The backward must receive the options the forward received, and the
  * forward's saved y, gates and cells.  Other arguments, ownership, workspace
  * sizes and errors are those of lstm_fwd / lstm_bwd.
  */
 #define LSTM_DIR_FORWARD 0
 #define LSTM_DIR_REVERSE 1
+#define LSTM_GATES_IFJO 0
+#define LSTM_GATES_IJFO 1
 typedef struct {
     const void *seq_mask;
     int direction;
+    int gate_order;
 } lstm_options;
 
 int lstm_fwd_ex(const lstm_dims *d, const lstm_options *opt, const void *x, const void *W,

@@ -42,10 +42,12 @@ def to_dev(inputs, device, drop=()):
     return {k: (None if k in drop else v.to(device)) for k, v in inputs.items()}
 
 
-def run_gpu(inputs, device, drop=(), stream=None, mask=None, reverse=False):
+def run_gpu(inputs, device, drop=(), stream=None, mask=None, reverse=False, ijfo=False):
     """Forward + backward through the C ABI.  Inputs named in `drop` are passed
     as NULL (the library treats them as zeros); `mask` (variable length,
-    [T,B,H] in the compute type) selects the masked entry points."""
+    [T,B,H] in the compute type), `reverse` and `ijfo` (gate_order "ijfo")
+    select the _ex entry points."""
+    order = "ijfo" if ijfo else "ifjo"
     lbuild.build()
     d = to_dev(inputs, device, drop)
     mk = mask.to(device) if mask is not None else None
@@ -53,22 +55,22 @@ def run_gpu(inputs, device, drop=(), stream=None, mask=None, reverse=False):
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         st = L.forward(d["x"], d["W"], d["b"], d["h0"], d["c0"], stream=s, mask=mk,
-                       reverse=reverse)
+                       reverse=reverse, gate_order=order)
         g = L.backward(st, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"], d["dcT"],
-                       stream=s, mask=mk, reverse=reverse)
+                       stream=s, mask=mk, reverse=reverse, gate_order=order)
     torch.cuda.synchronize()
     out = dict(y=st.y, hT=st.hT, cT=st.cT, gates=st.gates, cells=st.cells, dx=g.dx, dW=g.dW,
                db=g.db, dh0=g.dh0, dc0=g.dc0)
     return {k: v.float().cpu().double().numpy() for k, v in out.items()}
 
 
-def run_oracle(inputs, drop=(), mask=None, reverse=False):
+def run_oracle(inputs, drop=(), mask=None, reverse=False, ijfo=False):
     p = synth.as_float64(inputs)
     for k in drop:
         p[k] = None
     mk = mask.double().numpy() if mask is not None else None
     return oracle.lstm_fwd_bwd(p["x"], p["W"], p["b"], p["h0"], p["c0"], p["dy"], p["dhT"],
-                               p["dcT"], mask=mk, reverse=reverse)
+                               p["dcT"], mask=mk, reverse=reverse, ijfo=ijfo)
 
 
 def compare(gpu, ref, dtype, names=OUTS, idx=None):

@@ -171,6 +171,31 @@ def test_unknown_direction_rejected(lib, direction):
     assert rc == L.LSTM_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("order", [-1, 2, 5])
+def test_unknown_gate_order_rejected(lib, order):
+    """lstm_fwd_ex / lstm_bwd_ex reject a gate_order other than LSTM_GATES_IFJO /
+    LSTM_GATES_IJFO before anything is enqueued."""
+    opt = L.Options(None, L.LSTM_DIR_FORWARD, order)
+    a = fwd_args(D)
+    rc = lib.lstm_fwd_ex(ctypes.byref(D), ctypes.byref(opt), a["x"], a["W"], a["b"], a["h0"],
+                         a["c0"], a["y"], a["hT"], a["cT"], a["gates"], a["cells"], a["ws"],
+                         a["ws_bytes"], None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
+    rc = lib.lstm_bwd_ex(ctypes.byref(D), ctypes.byref(opt), None, None, None, FAKE, FAKE, None,
+                         None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                         L.bwd_workspace_size(D), None)
+    assert rc == L.LSTM_ERR_INVALID_ARG
+
+
+def test_options_layout_matches_header():
+    """The ctypes mirror of lstm_options has the C layout: a pointer, then the
+    two ints (no padding between them)."""
+    assert L.Options.seq_mask.offset == 0
+    assert L.Options.direction.offset == ctypes.sizeof(ctypes.c_void_p)
+    assert L.Options.gate_order.offset == ctypes.sizeof(ctypes.c_void_p) + 4
+    assert ctypes.sizeof(L.Options) == ctypes.sizeof(ctypes.c_void_p) + 8
+
+
 def test_misaligned_mask_rejected(lib):
     opt = L.Options(FAKE + 2, L.LSTM_DIR_FORWARD)
     a = fwd_args(D)
