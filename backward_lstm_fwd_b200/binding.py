@@ -25,6 +25,7 @@ LSTM_ERR_NOT_CORESIDENT = 6
 
 LSTM_F32 = 0
 LSTM_BF16 = 1
+LSTM_F16 = 2
 
 EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd", "lstm_bwd",
            "lstm_fwd_ex", "lstm_bwd_ex",
@@ -124,6 +125,8 @@ def dtype_code(dt: torch.dtype) -> int:
         return LSTM_F32
     if dt == torch.bfloat16:
         return LSTM_BF16
+    if dt == torch.float16:
+        return LSTM_F16
     raise ValueError(f"unsupported compute dtype {dt}")
 
 

@@ -70,7 +70,7 @@ struct Phase {
 bool dims_ok(const lstm_dims *d) {
     if (!d) return false;
     if (d->T < 0 || d->B < 0 || d->I < 0 || d->H < 0) return false;
-    if (d->dtype != LSTM_F32 && d->dtype != LSTM_BF16) return false;
+    if (d->dtype != LSTM_F32 && d->dtype != LSTM_BF16 && d->dtype != LSTM_F16) return false;
     const long long TB = (long long)d->T * d->B;
     const long long G4 = 4LL * d->H;
     const long long K = (long long)d->H + d->I;
@@ -85,7 +85,7 @@ bool dims_supported(const lstm_dims *d) {
     return 4LL * d->H <= maxcols && (long long)d->H + d->I <= maxcols;
 }
 
-size_t esize(const lstm_dims *d) { return d->dtype == LSTM_BF16 ? 2 : 4; }
+size_t esize(const lstm_dims *d) { return d->dtype == LSTM_F32 ? 4 : 2; }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -130,7 +130,7 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     L.wt = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
     L.dbgroup = L.wt;
     L.total = L.wt;
-    if (d->dtype == LSTM_BF16) {
+    if (d->dtype != LSTM_F32) {
         // W_h^T [H][4H] and per-batch-group db partials of the persistent kernel
         L.dbgroup = align_up(L.wt + (size_t)d->H * G4 * 2, 256);
         L.total = align_up(L.dbgroup + (size_t)kMaxGroups * G4 * sizeof(float), 256);
@@ -138,15 +138,16 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     return L;
 }
 
-// The tcgen05 GEMM core serves bf16 problems whose rows are whole 16-byte
-// groups (TMA strides and the W_x base offset are then 16-byte aligned).
+// The tcgen05 GEMM core serves 16-bit (bf16 or fp16) problems whose rows are
+// whole 16-byte groups (TMA strides and the W_x base offset are then 16-byte
+// aligned).
 bool tc_gemm_ok(const lstm_dims *d) {
     static int force_simt = -1;
     if (force_simt < 0) {
         const char *e = getenv("LSTM_FORCE_SIMT");
         force_simt = (e && e[0] == '1') ? 1 : 0;
     }
-    return !force_simt && d->dtype == LSTM_BF16 && d->H >= 8 && d->I >= 8 && d->H % 8 == 0 &&
+    return !force_simt && d->dtype != LSTM_F32 && d->H >= 8 && d->I >= 8 && d->H % 8 == 0 &&
            d->I % 8 == 0 && tcg::encode_fn() != nullptr;
 }
 
@@ -186,11 +187,17 @@ cudaError_t launch_to_float(const T *in, float *out, long long n, cudaStream_t s
 // ------------------------------------------- tensor-core GEMM problems
 typedef __nv_bfloat16 bf16;
 
+// The 16-bit type the tensor-core paths of fwd_simt<T> / bwd_simt<T> use: T
+// itself for bf16 and fp16 (float never reaches them).
+template <class T> struct Tc16 { typedef T type; };
+template <> struct Tc16<float> { typedef bf16 type; };
+
 // a1 on tcgen05: Gx[TB][4H] = X[TB][I] W_x^T + b, both operands K-major.
-cudaError_t tc_input_projection(const lstm_dims *d, const bf16 *x, const bf16 *W, const bf16 *b,
+template <class E>
+cudaError_t tc_input_projection(const lstm_dims *d, const E *x, const E *W, const E *b,
                                 float *Gx, Ctrl *ctrl, cudaStream_t s) {
     const long long TB = (long long)d->T * d->B, H = d->H, I = d->I;
-    tcg::Builder bld(ctrl);
+    tcg::Builder bld(ctrl, Elem<E>::kFmt);
     const int mx = bld.add_map({x, TB, I, I}, 0, tcg::BM);
     const int mw = bld.add_map({W + H, 4 * H, I, H + I}, 0, tcg::BN);
     tcg::Problem &q = bld.add_problem((int)TB, (int)(4 * H), 0, 0, Gx, 4 * H, 0, b);
@@ -210,13 +217,13 @@ cudaError_t tc_input_projection(const lstm_dims *d, const bf16 *x, const bf16 *W
 // The operand maps end at the range's last row, so a partial 64-row K block
 // reads zeros rather than rows of the next range.  At most max_ctas CTAs
 // (0: one per SM).
-cudaError_t tc_dw_dx(const lstm_dims *d, const bf16 *dG, const bf16 *x, const bf16 *W,
-                     const bf16 *h0, const bf16 *y, float *dW, float *dx, Ctrl *ctrl,
-                     cudaStream_t s, int t_lo, int t_hi, bool accumulate, int max_ctas,
-                     bool reverse = false) {
+template <class E>
+cudaError_t tc_dw_dx(const lstm_dims *d, const E *dG, const E *x, const E *W, const E *h0,
+                     const E *y, float *dW, float *dx, Ctrl *ctrl, cudaStream_t s, int t_lo,
+                     int t_hi, bool accumulate, int max_ctas, bool reverse = false) {
     const long long B = d->B, H = d->H, I = d->I, G4 = 4 * H;
     const long long r0 = (long long)t_lo * B, r1 = (long long)t_hi * B;
-    tcg::Builder bld(ctrl);
+    tcg::Builder bld(ctrl, Elem<E>::kFmt);
     const int m_dg_mn = bld.add_map({dG, r1, G4, G4}, 1, 0);
     const int m_x_mn = bld.add_map({x, r1, I, I}, 1, 0);
     const int m_dg_k = bld.add_map({dG, r1, G4, G4}, 0, tcg::BM);
@@ -560,11 +567,12 @@ bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
     return false;
 }
 
+template <class E>
 const void *fwd3_kernel_ptr(int NB, int KS, bool masked) {
 #define LSTM_F3(nb, ks)                                                                    \
     if (NB == nb && KS == ks)                                                              \
-        return masked ? (const void *)rec3::fwd3_kernel<nb, ks, true>                      \
-                      : (const void *)rec3::fwd3_kernel<nb, ks, false>;
+        return masked ? (const void *)rec3::fwd3_kernel<E, nb, ks, true>                   \
+                      : (const void *)rec3::fwd3_kernel<E, nb, ks, false>;
     LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
     LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
     LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
@@ -579,7 +587,7 @@ const void *fwd3_kernel_ptr(int NB, int KS, bool masked) {
 bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
     const char *e = getenv("LSTM_FWD_FUSED_X");
     if (e && e[0] == '0') return false;
-    if (d->dtype != LSTM_BF16 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
+    if (d->dtype == LSTM_F32 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
         d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
     const int nsm = tcg::sm_count();
@@ -600,7 +608,8 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
         const int G = (d->B + NB - 1) / NB;
         const size_t smem = rec3::Fwd3Smem(kcc, kcx, NB, KS).total + 1024;
         if (smem > kMaxSmem) continue;
-        const void *kern = fwd3_kernel_ptr(NB, KS, masked);
+        const void *kern = d->dtype == LSTM_F16 ? fwd3_kernel_ptr<__half>(NB, KS, masked)
+                                                : fwd3_kernel_ptr<bf16>(NB, KS, masked);
         if (!kern) continue;
         const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
         if (G * P.R > maxc) continue;
@@ -654,7 +663,7 @@ bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
 bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     const char *e = getenv("LSTM_BWD_TMEM_W");
     if (e && e[0] == '0') return false;
-    if (d->dtype != LSTM_BF16 || d->H % rec3::UNITS != 0 || d->B < 1 ||
+    if (d->dtype == LSTM_F32 || d->H % rec3::UNITS != 0 || d->B < 1 ||
         tcg::encode_fn() == nullptr || force_simt())
         return false;
     P.KS = rec3::KS;
@@ -665,8 +674,9 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     while (stages >= rec3::MIN_STAGES && (size_t)rec3::Bwd3Smem(stages).total + 1024 > kMaxSmem) --stages;
     if (stages < rec3::MIN_STAGES) return false;
     P.smem = rec3::Bwd3Smem(stages).total + 1024;
-    const int maxc = max_active_clusters((const void *)rec3::bwd3_kernel<false, false>, rec3::THREADS,
-                                         P.smem, P.KS);
+    const void *kern = d->dtype == LSTM_F16 ? (const void *)rec3::bwd3_kernel<__half, false, false>
+                                            : (const void *)rec3::bwd3_kernel<bf16, false, false>;
+    const int maxc = max_active_clusters(kern, rec3::THREADS, P.smem, P.KS);
     const int gmax = std::min(maxc / P.R, kMaxGroups);
     if (gmax < 1) return false;
     int G = std::min(gmax, (d->B + 15) / 16);
@@ -772,18 +782,19 @@ int tc_fwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *W, con
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
-template <int NB, int KS>
-cudaError_t launch_fwd3_t(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStream_t s) {
+template <class E, int NB, int KS>
+cudaError_t launch_fwd3_t(const rec3::Fwd3Params<E> &prm, const Rec2Plan &P, cudaStream_t s) {
     if (prm.mask)
-        return launch_cluster(rec3::fwd3_kernel<NB, KS, true>, prm, P.R * KS * P.G, KS, P.smem,
-                              s, rec2::F_THREADS);
-    return launch_cluster(rec3::fwd3_kernel<NB, KS, false>, prm, P.R * KS * P.G, KS, P.smem, s,
-                          rec2::F_THREADS);
+        return launch_cluster(rec3::fwd3_kernel<E, NB, KS, true>, prm, P.R * KS * P.G, KS,
+                              P.smem, s, rec2::F_THREADS);
+    return launch_cluster(rec3::fwd3_kernel<E, NB, KS, false>, prm, P.R * KS * P.G, KS, P.smem,
+                          s, rec2::F_THREADS);
 }
 
-cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStream_t s) {
+template <class E>
+cudaError_t launch_fwd3(const rec3::Fwd3Params<E> &prm, const Rec2Plan &P, cudaStream_t s) {
 #define LSTM_F3(nb, ks) \
-    if (P.NB == nb && P.KS == ks) return launch_fwd3_t<nb, ks>(prm, P, s);
+    if (P.NB == nb && P.KS == ks) return launch_fwd3_t<E, nb, ks>(prm, P, s);
     LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
     LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
     LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
@@ -794,16 +805,18 @@ cudaError_t launch_fwd3(const rec3::Fwd3Params &prm, const Rec2Plan &P, cudaStre
 
 // a1 + a2 in one cluster kernel (x-part contracted inside the recurrence);
 // LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
-int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *x, const bf16 *W,
-                       const bf16 *b, const bf16 *h0, const float *c0, const bf16 *mask,
-                       bool reverse, bool ijfo, bf16 *y, bf16 *hT, float *cT, bf16 *gates,
-                       float *cells, Ctrl *ctrl, cudaStream_t s) {
+template <class E>
+int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *x, const E *W,
+                       const E *b, const E *h0, const float *c0, const E *mask, bool reverse,
+                       bool ijfo, E *y, E *hT, float *cT, E *gates, float *cells, Ctrl *ctrl,
+                       cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, I = d->I;
-    rec3::Fwd3Params prm;
+    const CUtensorMapDataType dt = tcg::map_type(Elem<E>::kFmt);
+    rec3::Fwd3Params<E> prm;
     memset(&prm, 0, sizeof(prm));
-    bool ok = tcg::make_map(&prm.map_y, y, H, T * B, H * 2, 64, P.NB) &&
-              tcg::make_map(&prm.map_x, x, I, T * B, I * 2, 64, P.NB);
-    if (h0) ok = ok && tcg::make_map(&prm.map_h0, h0, H, B, H * 2, 64, P.NB);
+    bool ok = tcg::make_map(&prm.map_y, y, H, T * B, H * 2, 64, P.NB, dt) &&
+              tcg::make_map(&prm.map_x, x, I, T * B, I * 2, 64, P.NB, dt);
+    if (h0) ok = ok && tcg::make_map(&prm.map_h0, h0, H, B, H * 2, 64, P.NB, dt);
     else prm.map_h0 = prm.map_y;
     if (!ok) return LSTM_ERR_UNSUPPORTED;
     prm.W = W; prm.bias = b; prm.c0 = c0; prm.y = y; prm.gates = gates; prm.hT = hT;
@@ -861,15 +874,18 @@ int tc_bwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 
 // One launch of the TMEM-weight backward kernel over epilogue iterations
 // [i0, i1) (time steps T-i1 .. T-i0-1); WT must already hold W_h^T.
-int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                   const float *dcT, const float *c0, const bf16 *mask, bool reverse,
-                   bool ijfo, const bf16 *gates, const float *cells, bf16 *dG, const bf16 *WT,
-                   float *dbgroup, float *dh0, float *dc0, float *dc_carry, float *dhp_carry,
-                   Ctrl *ctrl, int i0, int i1, cudaStream_t s) {
+template <class E>
+int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *dhT,
+                   const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
+                   const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
+                   float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0,
+                   int i1, cudaStream_t s) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
-    rec3::Bwd3Params prm;
+    rec3::Bwd3Params<E> prm;
     memset(&prm, 0, sizeof(prm));
-    if (!tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB)) return LSTM_ERR_UNSUPPORTED;
+    if (!tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, P.NB,
+                       tcg::map_type(Elem<E>::kFmt)))
+        return LSTM_ERR_UNSUPPORTED;
     prm.wt = WT;
     prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
     prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
@@ -883,14 +899,14 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const 
     prm.wait_ns = g_wait_ns;
     const int nctas = P.R * P.KS * P.G;
     const cudaError_t e =
-        mask ? (ijfo ? launch_cluster(rec3::bwd3_kernel<true, true>, prm, nctas, P.KS, P.smem, s,
-                                      rec3::THREADS)
-                     : launch_cluster(rec3::bwd3_kernel<true, false>, prm, nctas, P.KS, P.smem, s,
-                                      rec3::THREADS))
-             : (ijfo ? launch_cluster(rec3::bwd3_kernel<false, true>, prm, nctas, P.KS, P.smem, s,
-                                      rec3::THREADS)
-                     : launch_cluster(rec3::bwd3_kernel<false, false>, prm, nctas, P.KS, P.smem,
-                                      s, rec3::THREADS));
+        mask ? (ijfo ? launch_cluster(rec3::bwd3_kernel<E, true, true>, prm, nctas, P.KS, P.smem,
+                                      s, rec3::THREADS)
+                     : launch_cluster(rec3::bwd3_kernel<E, true, false>, prm, nctas, P.KS, P.smem,
+                                      s, rec3::THREADS))
+             : (ijfo ? launch_cluster(rec3::bwd3_kernel<E, false, true>, prm, nctas, P.KS, P.smem,
+                                      s, rec3::THREADS)
+                     : launch_cluster(rec3::bwd3_kernel<E, false, false>, prm, nctas, P.KS,
+                                      P.smem, s, rec3::THREADS));
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
@@ -898,7 +914,10 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const 
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
-cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cudaStream_t s) {
+// W_h^T of a 16-bit W (bf16 or fp16: the kernel only moves 16-bit values)
+cudaError_t launch_transpose_wh(const lstm_dims *d, const void *W_, void *WT_, cudaStream_t s) {
+    const bf16 *W = static_cast<const bf16 *>(W_);
+    bf16 *WT = static_cast<bf16 *>(WT_);
     const long long H = d->H, G4 = 4 * H;
     dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
     rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)d->I);
@@ -908,10 +927,11 @@ cudaError_t launch_transpose_wh(const lstm_dims *d, const bf16 *W, bf16 *WT, cud
 
 // a3 (+ a5) on the cluster kernel with W_h^T in TMEM (written to the
 // workspace first, then copied into each CTA's tensor memory), one launch.
-int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, const bf16 *dhT,
-                       const float *dcT, const bf16 *W, const float *c0, const bf16 *mask,
-                       bool reverse, bool ijfo, const bf16 *gates, const float *cells, bf16 *dG,
-                       bf16 *WT,
+template <class E>
+int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *dhT,
+                       const float *dcT, const E *W, const float *c0, const E *mask,
+                       bool reverse, bool ijfo, const E *gates, const float *cells, E *dG,
+                       E *WT,
                        float *dbgroup, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
     const long long G4 = 4LL * d->H;
@@ -930,12 +950,13 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const bf16 *dy, co
 // takes the SMs the recurrence leaves idle (all of them for the last chunk).
 // No kernel waits on another; the streams are ordered by events and joined
 // back into `s` on every return.
+template <class E>
 int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int nch,
-                       const bf16 *dy, const bf16 *dhT, const float *dcT, const bf16 *x,
-                       const bf16 *W, const bf16 *h0, const float *c0, const bf16 *mask,
-                       bool reverse, bool ijfo, const bf16 *y, const bf16 *gates,
+                       const E *dy, const E *dhT, const float *dcT, const E *x,
+                       const E *W, const E *h0, const float *c0, const E *mask,
+                       bool reverse, bool ijfo, const E *y, const E *gates,
                        const float *cells,
-                       bf16 *dG, bf16 *WT, float *dbgroup, float *dc_carry, float *dhp_carry,
+                       E *dG, E *WT, float *dbgroup, float *dc_carry, float *dhp_carry,
                        float *dx, float *dW, float *db, float *dh0, float *dc0, Ctrl *ctrl,
                        cudaStream_t s) {
     std::lock_guard<std::mutex> lock(A.mu);
@@ -996,8 +1017,10 @@ template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
              const float *c0, const T *mask, bool reverse, bool ijfo, T *y, T *hT, float *cT,
              T *gates, float *cells, char *ws, cudaStream_t s) {
-    // masked, reverse-direction or "ijfo" calls: TMEM-weight kernel or per-step kernels
-    const bool special = mask != nullptr || reverse || ijfo;
+    typedef typename Tc16<T>::type E;  // the 16-bit type of the tensor-core paths
+    // masked, reverse-direction, "ijfo" or fp16 calls: TMEM-weight kernel or
+    // per-step kernels (the other kernels are bf16 / default-order only)
+    const bool special = mask != nullptr || reverse || ijfo || d->dtype == LSTM_F16;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H;
     const FwdLayout L = fwd_layout(d);
@@ -1006,10 +1029,10 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         Rec2Plan plan3;
         if (plan_fwd3(d, plan3, mask != nullptr)) {  // a1 fused into a2
             prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
-            const int rc = tc_fwd_recurrence3(d, plan3, (const bf16 *)x, (const bf16 *)W,
-                                              (const bf16 *)b, (const bf16 *)h0, c0,
-                                              (const bf16 *)mask, reverse, ijfo, (bf16 *)y,
-                                              (bf16 *)hT, cT, (bf16 *)gates, cells,
+            const int rc = tc_fwd_recurrence3(d, plan3, (const E *)x, (const E *)W,
+                                              (const E *)b, (const E *)h0, c0,
+                                              (const E *)mask, reverse, ijfo, (E *)y,
+                                              (E *)hT, cT, (E *)gates, cells,
                                               (Ctrl *)ws, s);
             g_last_fwd_path = 3;
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
@@ -1017,9 +1040,9 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         {   // a1: Gx = X W_x^T + b over all T*B rows (input concat, x-part)
             prof::Phase ph(LSTM_PHASE_INPUT_PROJ, s);
             if (tc_gemm_ok(d)) {
-                LSTM_TRY(tc_input_projection(d, (const __nv_bfloat16 *)x,
-                                             (const __nv_bfloat16 *)W,
-                                             (const __nv_bfloat16 *)b, Gx, (Ctrl *)ws, s));
+                LSTM_TRY(tc_input_projection(d, (const E *)x,
+                                             (const E *)W,
+                                             (const E *)b, Gx, (Ctrl *)ws, s));
             } else {
                 LSTM_TRY((simt::gemm<true, true>(T_ * B, 4 * H, I, simt::RowMajor<T>{x, I},
                                                   simt::WxT<T>{W, H, I},
@@ -1086,7 +1109,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
              const T *W, const T *h0, const float *c0, const T *mask, bool reverse, bool ijfo,
              const T *y, const T *gates, const float *cells, float *dx, float *dW, float *db,
              float *dh0, float *dc0, char *ws, cudaStream_t s) {
-    const bool special = mask != nullptr || reverse || ijfo;
+    typedef typename Tc16<T>::type E;  // the 16-bit type of the tensor-core paths
+    const bool special = mask != nullptr || reverse || ijfo || d->dtype == LSTM_F16;
     const int T_ = d->T, B = d->B, I = d->I, H = d->H;
     const long long BH = (long long)B * H, TB = (long long)T_ * B;
     const int G4 = 4 * H, K = H + I;
@@ -1111,17 +1135,17 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     const bool v3 = plan_bwd3(d, plan3);
     const bool v2 = !v3 && !special && plan_bwd2(d, plan2);
     const bool v1 = !special && plan_bwd_recur(d, plan);
-    bool per_step = false;  // a masked call whose cluster kernel cannot be placed
+    bool per_step = false;  // a special call whose cluster kernel cannot be placed
     if (v3 || v2 || v1) {
         if (v3 && tc_gemm_ok(d) && bwd_chunks(d) > 1) {
             AuxStreams *A = aux_streams();
             if (A) {  // a3 + a5 with a4 + a6 overlapped
                 g_last_bwd_path = 3;
                 const int rc = tc_bwd3_overlapped(
-                    d, plan3, *A, bwd_chunks(d), (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                    (const bf16 *)x, (const bf16 *)W, (const bf16 *)h0, c0, (const bf16 *)mask,
-                    reverse, ijfo, (const bf16 *)y, (const bf16 *)gates, cells, (bf16 *)dG,
-                    (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), (float *)(ws + L.dc),
+                    d, plan3, *A, bwd_chunks(d), (const E *)dy, (const E *)dhT, dcT,
+                    (const E *)x, (const E *)W, (const E *)h0, c0, (const E *)mask,
+                    reverse, ijfo, (const E *)y, (const E *)gates, cells, (E *)dG,
+                    (E *)(ws + L.wt), (float *)(ws + L.dbgroup), (float *)(ws + L.dc),
                     (float *)(ws + L.dhp), dx, dW, db, dh0, dc0, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
             }
@@ -1131,10 +1155,10 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
             int rc = LSTM_ERR_NOT_CORESIDENT;
             g_last_bwd_path = v3 ? 3 : 2;
             if (v3)
-                rc = tc_bwd_recurrence3(d, plan3, (const bf16 *)dy, (const bf16 *)dhT, dcT,
-                                        (const bf16 *)W, c0, (const bf16 *)mask, reverse, ijfo,
-                                        (const bf16 *)gates, cells, (bf16 *)dG,
-                                        (bf16 *)(ws + L.wt), (float *)(ws + L.dbgroup), db, dh0,
+                rc = tc_bwd_recurrence3(d, plan3, (const E *)dy, (const E *)dhT, dcT,
+                                        (const E *)W, c0, (const E *)mask, reverse, ijfo,
+                                        (const E *)gates, cells, (E *)dG,
+                                        (E *)(ws + L.wt), (float *)(ws + L.dbgroup), db, dh0,
                                         dc0, (Ctrl *)ws, s);
             else if (v2)
                 rc = tc_bwd_recurrence2(d, plan2, (const bf16 *)dy, (const bf16 *)dhT, dcT,
@@ -1154,8 +1178,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         if (!per_step) {
             if (tc_gemm_ok(d)) {
                 prof::Phase ph(LSTM_PHASE_DW, s);
-                LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
-                                  (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0,
+                LSTM_TRY(tc_dw_dx(d, (const E *)dG, (const E *)x, (const E *)W,
+                                  (const E *)h0, (const E *)y, dW, dx, (Ctrl *)ws, s, 0,
                                   d->T, false, 0, reverse));
                 return LSTM_OK;
             }
@@ -1215,8 +1239,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     if (tc) {
         // a4 + a6 together on the tensor cores (one launch, timed as dW)
         prof::Phase ph(LSTM_PHASE_DW, s);
-        LSTM_TRY(tc_dw_dx(d, (const bf16 *)dG, (const bf16 *)x, (const bf16 *)W,
-                          (const bf16 *)h0, (const bf16 *)y, dW, dx, (Ctrl *)ws, s, 0, d->T,
+        LSTM_TRY(tc_dw_dx(d, (const E *)dG, (const E *)x, (const E *)W,
+                          (const E *)h0, (const E *)y, dW, dx, (Ctrl *)ws, s, 0, d->T,
                           false, 0, reverse));
     } else {
         // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
@@ -1305,6 +1329,12 @@ int fwd_entry(const lstm_dims *d, const lstm_options *opt, const void *x, const 
         return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
                                (const float *)h0, c0, (const float *)mask, reverse, ijfo,
                                (float *)y, (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
+    if (d->dtype == LSTM_F16) {
+        typedef __half hf;
+        return fwd_simt<hf>(d, (const hf *)x, (const hf *)W, (const hf *)b, (const hf *)h0, c0,
+                            (const hf *)mask, reverse, ijfo, (hf *)y, (hf *)hT, cT, (hf *)gates,
+                            cells, (char *)ws, s);
+    }
     typedef __nv_bfloat16 bf;
     return fwd_simt<bf>(d, (const bf *)x, (const bf *)W, (const bf *)b, (const bf *)h0, c0,
                         (const bf *)mask, reverse, ijfo, (bf *)y, (bf *)hT, cT, (bf *)gates,
@@ -1342,6 +1372,13 @@ int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const
                                (const float *)W, (const float *)h0, c0, (const float *)mask,
                                reverse, ijfo, (const float *)y, (const float *)gates, cells, dx,
                                dW, db, dh0, dc0, (char *)ws, s);
+    if (d->dtype == LSTM_F16) {
+        typedef __half hf;
+        return bwd_simt<hf>(d, (const hf *)dy, (const hf *)dhT, dcT, (const hf *)x,
+                            (const hf *)W, (const hf *)h0, c0, (const hf *)mask, reverse, ijfo,
+                            (const hf *)y, (const hf *)gates, cells, dx, dW, db, dh0, dc0,
+                            (char *)ws, s);
+    }
     typedef __nv_bfloat16 bf;
     return bwd_simt<bf>(d, (const bf *)dy, (const bf *)dhT, dcT, (const bf *)x, (const bf *)W,
                         (const bf *)h0, c0, (const bf *)mask, reverse, ijfo, (const bf *)y,

@@ -1,5 +1,5 @@
-// tc_gemm.cuh -- persistent tcgen05 / TMA GEMM core for bf16 operands with fp32
-// accumulation in TMEM, used for the time-parallel contractions of the path:
+// tc_gemm.cuh -- persistent tcgen05 / TMA GEMM core for 16-bit operands (bf16
+// or fp16, one type per launch) with fp32 accumulation in TMEM, used for the time-parallel contractions of the path:
 //   input projection   Gx = X W_x^T + b        (A = X K-major, B = W_x K-major)
 //   dW                 dG^T [h_prev | x]        (A = dG MN-major, B = y / x MN-major)
 //   dx                 dG W_x                  (A = dG K-major, B = W_x MN-major)
@@ -49,7 +49,7 @@ struct Problem {
     long long ldo;
     int out_col0;
     int accumulate;            // out += product (otherwise out = product)
-    const __nv_bfloat16 *bias; // added per column n, or NULL
+    const void *bias;          // added per column n (operand type), or NULL
     int tiles_n, tile_begin, tile_end;
 };
 
@@ -57,6 +57,7 @@ struct Params {
     CUtensorMap maps[MAX_MAPS];
     Problem prob[MAX_PROB];
     int nprob, total_tiles;
+    uint32_t fmt;              // operand format of every problem: 0 = fp16, 1 = bf16
     Ctrl *ctrl;
 };
 
@@ -181,7 +182,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
                 if (!tc::mbar_wait(&tempty[acc], aphase ^ 1, p.ctrl, abort_flag, 0x102)) break;
                 tc::tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
-                const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, P.a_mn_major, P.b_mn_major);
+                const uint32_t idesc =
+                    tc::idesc_f16kind_f32(p.fmt, BM, BN, P.a_mn_major, P.b_mn_major);
                 const uint64_t a_hi = operand_desc(0, P.a_mn_major, 0);  // address field 0
                 const uint64_t b_hi = operand_desc(0, P.b_mn_major, 0);
                 const uint32_t a_k = P.a_mn_major ? 2048 >> 4 : 32 >> 4;  // per K=16 step
@@ -244,7 +246,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
                     for (int j = 0; j < 32; ++j) {
                         const int n = nbase + c0 + j;
                         float x = nk ? __uint_as_float(r[j]) : 0.f;
-                        if (P.bias && n < P.N) x += __bfloat162float(P.bias[n]);
+                        if (P.bias && n < P.N) {
+                            const unsigned short bb = static_cast<const unsigned short *>(P.bias)[n];
+                            x += p.fmt ? __bfloat162float(__ushort_as_bfloat16(bb))
+                                       : __half2float(__ushort_as_half(bb));
+                        }
                         v[j] = x;
                     }
                     float *orow = P.out + (long long)m * P.ldo + P.out_col0 + nbase + c0;

@@ -34,51 +34,60 @@ inline EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map with 128-byte swizzle: `inner` contiguous elements per
-// row, `outer` rows `row_bytes` apart, boxes of box_inner x box_outer.  Reads
-// outside the extents return zeros.
+// 2-D tensor map of 16-bit elements (bf16 by default, or fp16) with 128-byte
+// swizzle: `inner` contiguous elements per row, `outer` rows `row_bytes`
+// apart, boxes of box_inner x box_outer.  Reads outside the extents return
+// zeros.
 inline bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || inner == 0 || outer == 0) return false;
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
 
-// Operand view for a problem: a row-major bf16 matrix of `rows` x `cols`
-// (row stride ld elements).  As a K-major operand the rows are M (or N) and
-// the columns K; as an MN-major operand the rows are K and the columns M / N.
+// Operand view for a problem: a row-major matrix of 16-bit elements, `rows` x
+// `cols` (row stride ld elements).  As a K-major operand the rows are M (or N)
+// and the columns K; as an MN-major operand the rows are K and the columns M / N.
 struct View {
-    const __nv_bfloat16 *p;
+    const void *p;
     long long rows, cols, ld;
 };
 
-inline bool map_for(CUtensorMap *m, const View &v, int mn_major, int mn_tile) {
-    return mn_major ? make_map(m, v.p, v.cols, v.rows, v.ld * 2, 64, BK)
-                    : make_map(m, v.p, v.cols, v.rows, v.ld * 2, BK, mn_tile);
+// the tensor-map element type of operand format fmt (0 = fp16, 1 = bf16)
+inline CUtensorMapDataType map_type(uint32_t fmt) {
+    return fmt ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
+inline bool map_for(CUtensorMap *m, const View &v, int mn_major, int mn_tile, uint32_t fmt) {
+    return mn_major ? make_map(m, v.p, v.cols, v.rows, v.ld * 2, 64, BK, map_type(fmt))
+                    : make_map(m, v.p, v.cols, v.rows, v.ld * 2, BK, mn_tile, map_type(fmt));
 }
 
 struct Builder {
     Params P;
     int nmaps = 0;
     bool ok = true;
-    Builder(Ctrl *ctrl) {
+    // fmt: operand format of the launch, 0 = fp16, 1 = bf16
+    Builder(Ctrl *ctrl, uint32_t fmt = 1) {
         memset(&P, 0, sizeof(P));
         P.ctrl = ctrl;
+        P.fmt = fmt;
     }
     int add_map(const View &v, int mn_major, int mn_tile) {
         if (nmaps >= MAX_MAPS) { ok = false; return 0; }
-        if (!map_for(&P.maps[nmaps], v, mn_major, mn_tile)) ok = false;
+        if (!map_for(&P.maps[nmaps], v, mn_major, mn_tile, P.fmt)) ok = false;
         return nmaps++;
     }
     Problem &add_problem(int M, int N, int a_mn, int b_mn, float *out, long long ldo,
-                         int out_col0, const __nv_bfloat16 *bias) {
+                         int out_col0, const void *bias) {
         if (P.nprob >= MAX_PROB) { ok = false; return P.prob[0]; }
         Problem &q = P.prob[P.nprob++];
         memset(&q, 0, sizeof(q));

@@ -322,15 +322,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 operands and an
-// fp32 accumulator: [4,6) D format (1 = f32), [7,10) A format (1 = bf16),
-// [10,13) B format (1 = bf16), bit 15 A major, bit 16 B major (0 = K-major,
-// 1 = MN-major), [17,23) N >> 3, [24,29) M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
-                                                     int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
+// Instruction descriptor of tcgen05.mma kind::f16 with 16-bit operands of
+// format `fmt` (0 = f16, 1 = bf16; A and B always the same) and an fp32
+// accumulator: [4,6) D format (1 = f32), [7,10) A format, [10,13) B format,
+// bit 15 A major, bit 16 B major (0 = K-major, 1 = MN-major), [17,23) N >> 3,
+// [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(uint32_t fmt, int M, int N,
+                                                        int a_mn_major, int b_mn_major) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)a_mn_major << 15) |
            ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major,
+                                                     int b_mn_major) {
+    return idesc_f16kind_f32(1u, M, N, a_mn_major, b_mn_major);
 }
 
 }  // namespace tc

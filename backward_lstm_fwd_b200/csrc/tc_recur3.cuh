@@ -1,4 +1,5 @@
-// Recurrent kernels (bf16) with their weights resident in tensor memory: the
+// Recurrent kernels (16-bit operands: bf16, or fp16 for the page's FLOAT16
+// data type; fp32 accumulation) with their weights resident in tensor memory: the
 // tcgen05.mma A operand is read from TMEM, which leaves shared memory to the
 // streamed operands and the cluster exchange.
 //
@@ -22,7 +23,7 @@
 // finalises 16 of the 128 units after a reduce-scatter over DSMEM.
 //
 // What differs from that kernel: the CTA's slice of W_h^T (128 units x H/2 of
-// K, 128 KB of bf16) is the MMA's A operand in TMEM (tcgen05.mma with A from
+// K, 128 KB of 16-bit values) is the MMA's A operand in TMEM (tcgen05.mma with A from
 // tensor memory), so the accumulator is [128 units (lanes)][batch (columns)]
 // and shared memory is free for a ring that holds the whole dG K-slice of a
 // step (every chunk load of a step in flight at once) and for one exchange
@@ -48,18 +49,19 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_STAGES = 12;
 constexpr int MIN_STAGES = (KS - 1) * PART_BYTES / ACHUNK + 1;  // the ring stages one exchange: 4
 
+template <class E>  // E: the 16-bit compute type, __nv_bfloat16 or __half
 struct Bwd3Params {
-    CUtensorMap map_dg;               // dG [T*B][4H] bf16, box {64, NBr}
-    const __nv_bfloat16 *wt;          // W_h^T [H][4H] bf16
-    const __nv_bfloat16 *dy, *dhT, *gates;
+    CUtensorMap map_dg;               // dG [T*B][4H], box {64, NBr}
+    const E *wt;                      // W_h^T [H][4H]
+    const E *dy, *dhT, *gates;
     const float *dcT, *cells, *c0;
-    __nv_bfloat16 *dG;
+    E *dG;
     float *dh0, *dc0, *db_part;
     float *dc_carry;  // [B][H]: delta c between the launches of a chunked call
-    // variable length (MASKED kernels): mask [T][B][H] bf16, 1 = real step,
+    // variable length (MASKED kernels): mask [T][B][H], 1 = real step,
     // 0 = padding; dhp_carry [B][H]: the delta h that padding passes to
     // h_{t-1}, between the launches of a chunked call
-    const __nv_bfloat16 *mask;
+    const E *mask;
     float *dhp_carry;
     Ctrl *ctrl;
     int T, B, H, U, G, NBr, kcc, stages;
@@ -91,8 +93,8 @@ __device__ __forceinline__ int part_off(int r, int n) {
 
 // MASKED: variable-length mask; IJFO: gate_order "ijfo" (a template argument,
 // not a runtime one: the epilogue is at the register limit of its launch)
-template <bool MASKED, bool IJFO>
-__global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant__ Bwd3Params p) {
+template <class E, bool MASKED, bool IJFO>
+__global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant__ Bwd3Params<E> p) {
     constexpr int UPT = 8;  // units per epilogue thread in the pointwise part
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             // D[128 units][NBr] (+)= W_h^T slice (TMEM) x dG chunk^T (smem, K-major)
-            const uint32_t idesc = tc::idesc_bf16_f32(UNITS, NBr, 0, 0);
+            const uint32_t idesc = tc::idesc_f16kind_f32(Elem<E>::kFmt, UNITS, NBr, 0, 0);
             const uint64_t hi = tc::smem_desc_sw128(0, 16, 1024);
             const uint64_t r_lo0 = tc::smem_u32(ring) >> 4;
             constexpr uint32_t RSTEP = ACHUNK >> 4;
@@ -225,9 +227,9 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         const int hh = (warp - 2) >> 2;   // which half of the columns this warp moves
         {
             // W_h^T rows j0 + 32q + lane, this warp's half of the K slice ->
-            // TMEM lanes 32q + lane, two bf16 per column (lower K in the low half)
+            // TMEM lanes 32q + lane, two elements per column (lower K in the low half)
             const int u = 32 * q + lane;
-            const __nv_bfloat16 *src =
+            const E *src =
                 p.wt + (long long)(j0 + u) * (4LL * H) + kbase + hh * (kslice / 2);
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(32 * q) << 16) + W_COL + (uint32_t)(hh * (kslice / 4));
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             float dhr[UPT];
             if (i == 0) {
                 if (valid && p.dhT) {
-                    rec::bf16x8_to_f32(
+                    x8_to_f32<E>(
                         __ldg(reinterpret_cast<const uint4 *>(p.dhT + (long long)b * H + jb)), dhr);
                 } else {
 #pragma unroll
@@ -386,10 +388,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
             float dI[UPT], dF[UPT], dGg[UPT], dO[UPT];
             float gv[4][UPT], dyv[UPT];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) rec::bf16x8_to_f32(gpk[g], gv[g]);
-            rec::bf16x8_to_f32(dypk, dyv);
+            for (int g = 0; g < 4; ++g) x8_to_f32<E>(gpk[g], gv[g]);
+            x8_to_f32<E>(dypk, dyv);
             float mkv[UPT];
-            if (MASKED) rec::bf16x8_to_f32(mpk, mkv);
+            if (MASKED) x8_to_f32<E>(mpk, mkv);
 #pragma unroll
             for (int u = 0; u < UPT; ++u) {
                 const float ig = gv[0][u], fg = gv[1][u], gg = gv[2][u], og = gv[3][u];
@@ -413,10 +415,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 dc[u] = dcv * fg + dc_pass;                             // step 5
             }
             {
-                const uint4 vi = rec::f32x8_to_bf16(dI), vf = rec::f32x8_to_bf16(dF);
-                const uint4 vg = rec::f32x8_to_bf16(dGg), vo = rec::f32x8_to_bf16(dO);
+                const uint4 vi = f32x8_to<E>(dI), vf = f32x8_to<E>(dF);
+                const uint4 vg = f32x8_to<E>(dGg), vo = f32x8_to<E>(dO);
                 if (valid) {
-                    __nv_bfloat16 *o = p.dG + ((long long)tau(t) * B + b) * G4 + jb;
+                    E *o = p.dG + ((long long)tau(t) * B + b) * G4 + jb;
                     *reinterpret_cast<uint4 *>(o) = vi;
                     *reinterpret_cast<uint4 *>(o + kBlk[1] * H) = vf;
                     *reinterpret_cast<uint4 *>(o + kBlk[2] * H) = vg;
@@ -424,10 +426,10 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
                 }
                 if (valid) {
                     float ri[UPT], rf[UPT], rg[UPT], ro[UPT];  // db sums the stored values
-                    rec::bf16x8_to_f32(vi, ri);
-                    rec::bf16x8_to_f32(vf, rf);
-                    rec::bf16x8_to_f32(vg, rg);
-                    rec::bf16x8_to_f32(vo, ro);
+                    x8_to_f32<E>(vi, ri);
+                    x8_to_f32<E>(vf, rf);
+                    x8_to_f32<E>(vg, rg);
+                    x8_to_f32<E>(vo, ro);
 #pragma unroll
                     for (int u = 0; u < UPT; ++u) {
                         dbacc[0][u] += ri[u];
@@ -510,19 +512,20 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
 constexpr int F3_MAXC = 16;         // K chunks (of 64) per operand ring
 constexpr int F3_BAR_BYTES = 1024;
 
+template <class E>  // E: the 16-bit compute type, __nv_bfloat16 or __half
 struct Fwd3Params {
-    CUtensorMap map_y;                // y  [T*B][H] bf16, box {64, NB}: h_{t-1}
-    CUtensorMap map_h0;               // h0 [B][H]   bf16, box {64, NB}
-    CUtensorMap map_x;                // x  [T*B][I] bf16, box {64, NB}
-    const __nv_bfloat16 *W;           // [4H][H + I]: W_h | W_x
-    const __nv_bfloat16 *bias;        // [4H] or NULL
+    CUtensorMap map_y;                // y  [T*B][H], box {64, NB}: h_{t-1}
+    CUtensorMap map_h0;               // h0 [B][H],   box {64, NB}
+    CUtensorMap map_x;                // x  [T*B][I], box {64, NB}
+    const E *W;                       // [4H][H + I]: W_h | W_x
+    const E *bias;                    // [4H] or NULL
     const float *c0;
     // variable length (MASKED kernels): mask [T][B][H], 1 = real step,
     // 0 = padding (which keeps h_{t-1}, c_{t-1}); h0 [B][H] or NULL
-    const __nv_bfloat16 *mask, *h0;
+    const E *mask, *h0;
     int reverse;  // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
     int ijfo;     // gate_order "ijfo": row blocks i, j (= g), f, o instead of i, f, j, o
-    __nv_bfloat16 *y, *gates, *hT;
+    E *y, *gates, *hT;
     float *cells, *cT;
     Ctrl *ctrl;
     int T, B, H, I, R, G, kcc, kcx, has_h0;
@@ -558,8 +561,8 @@ struct Fwd3Smem {
     }
 };
 
-template <int NB, int KS, bool MASKED>
-__global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params p) {
+template <class E, int NB, int KS, bool MASKED>
+__global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params<E> p) {
     using rec2::F_ROWS;
     using rec2::F_UNITS;
     using rec2::F_EPI_THREADS;
@@ -703,7 +706,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         if (lane == 0) {
             // D[128 gate rows][NB] = W_x slice (TMEM) x x_t chunk^T (+)
             //                        W_h slice (TMEM) x h_{t-1} chunk^T
-            const uint32_t idesc = tc::idesc_bf16_f32(F_ROWS, NB, 0, 0);
+            const uint32_t idesc = tc::idesc_f16kind_f32(Elem<E>::kFmt, F_ROWS, NB, 0, 0);
             const uint64_t hi = tc::smem_desc_sw128(0, 16, 1024);
             const uint64_t rh_lo0 = tc::smem_u32(ring_h) >> 4, rx_lo0 = tc::smem_u32(ring_x) >> 4;
             constexpr uint32_t CSTEP = (NB * 128) >> 4;
@@ -768,12 +771,12 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         const int mrow = 32 * q + lane;   // row of the partial tile: gate q, unit lane
         {
             // W rows q*H + u0 + lane: this warp's half of the CTA's K range of
-            // W_h and of W_x (zero past I) -> TMEM lane mrow, two bf16 per column
-            const __nv_bfloat16 *wrow = p.W + (long long)(q * H + u0 + lane) * (H + I);
+            // W_h and of W_x (zero past I) -> TMEM lane mrow, two elements per column
+            const E *wrow = p.W + (long long)(q * H + u0 + lane) * (H + I);
             const uint32_t trow = tmem_base + ((uint32_t)(32 * q) << 16);
             const int hn = kcc * 2;  // 16-element groups per half of the W_h range
             for (int n = 0; n < hn; ++n) {
-                const __nv_bfloat16 *src = wrow + kbase + hh * kcc * 32 + 16 * n;
+                const E *src = wrow + kbase + hh * kcc * 32 + 16 * n;
                 const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(src));
                 const uint4 x1 = __ldg(reinterpret_cast<const uint4 *>(src + 8));
                 const uint32_t r[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
@@ -782,7 +785,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             const int xn = kcx * 2;
             for (int n = 0; n < xn; ++n) {
                 const int e = xbase + hh * kcx * 32 + 16 * n;  // first x feature of the group
-                const __nv_bfloat16 *src = wrow + H + e;
+                const E *src = wrow + H + e;
                 const uint4 z = make_uint4(0, 0, 0, 0);
                 const uint4 x0 = e < I ? __ldg(reinterpret_cast<const uint4 *>(src)) : z;
                 const uint4 x1 = e + 8 < I ? __ldg(reinterpret_cast<const uint4 *>(src + 8)) : z;
@@ -809,10 +812,10 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
             const bool v = n < NBc && b < B;
             c[k] = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
-            if (MASKED) hprev[k] = (p.h0 && v) ? __bfloat162float(p.h0[(long long)b * H + j]) : 0.f;
+            if (MASKED) hprev[k] = (p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-                bias[g][k] = p.bias ? __bfloat162float(p.bias[g * H + j]) : 0.f;
+                bias[g][k] = p.bias ? to_f(p.bias[g * H + j]) : 0.f;
         }
         auto load_mask = [&](int s) {  // mask of step s (time tau(s))
             const int t = tau(s);
@@ -820,7 +823,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             for (int k = 0; k < NP; ++k) {
                 const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
                 mk[k] = (n < NBc && b < B)
-                            ? __bfloat162float(p.mask[((long long)t * B + b) * H + j]) : 0.f;
+                            ? to_f(p.mask[((long long)t * B + b) * H + j]) : 0.f;
             }
         };
         if (MASKED) load_mask(0);
@@ -909,8 +912,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             const int tt = tau(t);  // time of this step
             // row blocks of the forget gate and the candidate (gate_order)
             const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
-            __nv_bfloat16 *yt = p.y + (long long)tt * B * H;
-            __nv_bfloat16 *gt = p.gates + (long long)tt * B * 4 * H;
+            E *yt = p.y + (long long)tt * B * H;
+            E *gt = p.gates + (long long)tt * B * 4 * H;
             float *ct = p.cells + (long long)tt * B * H;
             float gsave[4][NP];
 #pragma unroll
@@ -936,9 +939,9 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
                 if (b < B) {
                     const long long o = (long long)b * H + j;
-                    yt[o] = __float2bfloat16_rn(h);  // h_t: what the other CTAs wait for
+                    yt[o] = from_f<E>(h);  // h_t: what the other CTAs wait for
                     if (t == T - 1) {
-                        p.hT[o] = __float2bfloat16_rn(h);
+                        p.hT[o] = from_f<E>(h);
                         p.cT[o] = c[k];
                     }
                 }
@@ -958,12 +961,12 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 const int b = bc0 + n, j = u0 + uu;
                 if (n >= NBc || b >= B) continue;
                 ct[(long long)b * H + j] = c[k];
-                __nv_bfloat16 *g4 = gt + (long long)b * 4 * H + j;
+                E *g4 = gt + (long long)b * 4 * H + j;
                 const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
-                g4[0] = __float2bfloat16_rn(gsave[0][k]);
-                g4[fb * H] = __float2bfloat16_rn(gsave[1][k]);
-                g4[gb * H] = __float2bfloat16_rn(gsave[2][k]);
-                g4[3 * H] = __float2bfloat16_rn(gsave[3][k]);
+                g4[0] = from_f<E>(gsave[0][k]);
+                g4[fb * H] = from_f<E>(gsave[1][k]);
+                g4[gb * H] = from_f<E>(gsave[2][k]);
+                g4[3 * H] = from_f<E>(gsave[3][k]);
             }
             if (MASKED && t + 1 < T) load_mask(t + 1);
         }

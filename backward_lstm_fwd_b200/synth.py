@@ -13,8 +13,8 @@ Draw order (one torch CPU generator seeded per workload, all in fp32):
   W[4H, H+I], b[4H], x[T, B, I], h0[B, H], c0[B, H], dy[T, B, H],
   then dhT[B, H] and dcT[B, H] only for workloads that carry them
   (otherwise both are zero and nothing is drawn).
-For bf16 workloads x, W, b, h0, dy and dhT are rounded to bf16 after the
-draw; c0 and dcT stay fp32 (the cell state is fp32 throughout).
+For bf16 (fp16) workloads x, W, b, h0, dy and dhT are rounded to bf16 (fp16)
+after the draw; c0 and dcT stay fp32 (the cell state is fp32 throughout).
 """
 from __future__ import annotations
 
@@ -32,7 +32,7 @@ class Workload:
     B: int
     I: int
     H: int
-    dtype: str            # "fp32" or "bf16": the type x, W, b, h0, dy, y, gates are stored in
+    dtype: str            # "fp32", "bf16" or "fp16": the type x, W, b, h0, dy, y, gates are stored in
     seed: int
     dhdc: bool            # draw dhT / dcT (else zeros)
     dy_last: Optional[int] = None  # keep dy only on the last dy_last steps
@@ -67,7 +67,7 @@ def custom(T: int, B: int, I: int, H: int, dtype: str, seed: int = 123,
 
 
 def torch_dtype(dtype: str) -> torch.dtype:
-    return {"fp32": torch.float32, "bf16": torch.bfloat16}[dtype]
+    return {"fp32": torch.float32, "bf16": torch.bfloat16, "fp16": torch.float16}[dtype]
 
 
 def make_inputs(w: Workload) -> Dict[str, torch.Tensor]:

@@ -75,7 +75,7 @@ def phase_work(w: synth.Workload, phases=None):
     recurrence when no input-projection launch ran (the fused forward kernel),
     dx into the dW phase when both share one launch."""
     TB, H, I = w.rows, w.H, w.I
-    es = 2 if w.dtype == "bf16" else 4
+    es = 4 if w.dtype == "fp32" else 2
     work = {
         "input_proj": ("flop", 2.0 * TB * 4 * H * I),
         "fwd_recur": ("flop", 2.0 * TB * 4 * H * H),
@@ -400,11 +400,20 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override T (profiling aid: same per-step shape, fewer steps)")
+    ap.add_argument("--dtype", choices=("bf16", "fp16"), default=None,
+                    help="16-bit compute type override (fp16: the page's FLOAT16) on the "
+                         "workload's shape")
     ap.add_argument("--seq-mask", action="store_true",
                     help="variable length: a seq_length mask with seeded per-sequence "
                          "lengths in 0..T (every step is still computed and counted)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.dtype is not None and args.dtype != w.dtype:
+        import dataclasses
+        if w.dtype == "fp32":
+            ap.error("--dtype applies to the 16-bit workloads")
+        w = dataclasses.replace(w, name=w.name.replace("_" + w.dtype, "_" + args.dtype),
+                                dtype=args.dtype)
     if args.seq_len is not None:
         import dataclasses
         w = dataclasses.replace(w, name=f"{w.name}_T{args.seq_len}", T=args.seq_len,

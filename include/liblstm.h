@@ -19,9 +19,13 @@
  *   - Sequences are time-major and row-major: x[T][B][I], y[T][B][H], ...
  *     Row r = t*B + n of a [T*B][.] view is time step t of sequence n.
  *   - "compute type" (lstm_dims.dtype) is the element type of x, W, b, h0, y,
- *     hT, gates, dy and dhT: LSTM_F32 (float) or LSTM_BF16 (bfloat16).  The cell
+ *     hT, gates, dy and dhT: LSTM_F32 (float, the page's FLOAT), LSTM_BF16
+ *     (bfloat16) or LSTM_F16 (IEEE binary16, the page's FLOAT16).  The cell
  *     state (c0, cT, cells, dcT) and every gradient output (dx, dW, db, dh0,
- *     dc0) are float.  Products accumulate in float.
+ *     dc0) are float.  Products accumulate in float.  In LSTM_F16 the saved
+ *     gates and the gate gradients dG are stored in binary16: gradients below
+ *     its range (about 6e-8) flush to zero, as in any fp16 backward without
+ *     loss scaling.
  *   - Every pointer is a DEVICE pointer into memory the caller allocated and
  *     owns; it must be 16-byte aligned.  The library allocates no device memory
  *     and keeps no device state between calls; all scratch lives in the
@@ -55,6 +59,7 @@ extern "C" {
 /* Compute types. */
 #define LSTM_F32 0
 #define LSTM_BF16 1
+#define LSTM_F16 2
 
 /* Problem sizes: T time steps, B sequences, I input features, H hidden units
  * (parameter table: x [T, batch, input_size], w [4*hidden, input+hidden]).
@@ -64,7 +69,7 @@ typedef struct lstm_dims {
     int B;
     int I;
     int H;
-    int dtype; /* LSTM_F32 or LSTM_BF16 */
+    int dtype; /* LSTM_F32, LSTM_BF16 or LSTM_F16 */
 } lstm_dims;
 
 /* Workspace bytes lstm_fwd / lstm_bwd need for these dims (0 on invalid dims).

@@ -83,7 +83,8 @@ D = L.dims(4, 3, 5, 8, L.LSTM_F32)
 
 @pytest.mark.parametrize("bad", [
     L.dims(-1, 3, 5, 8, 0), L.dims(4, -3, 5, 8, 0), L.dims(4, 3, -5, 8, 0),
-    L.dims(4, 3, 5, -8, 0), L.dims(4, 3, 5, 8, 2), L.dims(1 << 20, 1 << 12, 5, 8, 0),
+    L.dims(4, 3, 5, -8, 0), L.dims(4, 3, 5, 8, 3), L.dims(4, 3, 5, 8, -1),
+    L.dims(1 << 20, 1 << 12, 5, 8, 0),
     L.dims(1, 1, 5, 1 << 29, 0),
 ])
 def test_bad_dims(lib, bad):

@@ -3,7 +3,7 @@
 Full-size runs of the five workloads (the launch configuration bench.py times),
 odd shapes that leave ragged tiles, and the degenerate cases (empty sequence or
 batch, no input features, absent optional inputs).  Tolerance per output
-tensor: max|gpu - ref| / max|ref| <= 1e-4 (fp32) or 2e-2 (bf16)."""
+tensor: max|gpu - ref| / max|ref| <= 1e-4 (fp32), 2e-2 (bf16) or 2.5e-3 (fp16)."""
 import numpy as np
 import pytest
 import torch
@@ -93,7 +93,7 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
     assert_within(compare(gpu, ref, dt), dt, w.name)
 
 
-@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+@pytest.mark.parametrize("dt", ["fp32", "bf16", "fp16"])
 def test_optional_inputs_absent(dt, cuda_device):
     w = synth.custom(6, 4, 24, 40, dt, seed=5)
     inp = synth.make_inputs(w)
@@ -107,7 +107,7 @@ def test_optional_inputs_absent(dt, cuda_device):
     assert_within(compare(gpu, ref, dt), dt, "dy NULL")
 
 
-@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+@pytest.mark.parametrize("dt", ["fp32", "bf16", "fp16"])
 def test_empty_sequence(dt, cuda_device):
     w = synth.custom(0, 3, 8, 16, dt, seed=2)
     inp = synth.make_inputs(w)
@@ -119,7 +119,7 @@ def test_empty_sequence(dt, cuda_device):
     assert not gpu["dW"].any() and not gpu["db"].any()
 
 
-@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+@pytest.mark.parametrize("dt", ["fp32", "bf16", "fp16"])
 def test_empty_batch_and_no_inputs(dt, cuda_device):
     gpu = run_gpu(synth.make_inputs(synth.custom(4, 0, 8, 16, dt)), cuda_device)
     assert gpu["y"].shape == (4, 0, 16)
