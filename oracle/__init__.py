@@ -9,7 +9,8 @@ The arithmetic lives in ``lstm_oracle.c`` (plain C, fp64, OpenMP over the batch
 of independent sequences), which states the forward-formula table and the
 "backward algorithm (time step t -> t-1)" of the "SingleLayerLstmGrad" operator
 page.  This module only builds that file, marshals numpy arrays into it and
-hands the results back.
+hands the results back.  The stacked (multi-layer) LSTM is the composition of
+single-layer calls, written out in ``lstm_stack_fwd`` / ``lstm_stack_bwd``.
 
 Layouts: x[T,B,I], W[4H,H+I] (columns [h | x], rows [i|f|g|o]), b[4H],
 h0/c0/hT/cT/dhT/dcT/dh0/dc0 [B,H], y/cells/dy [T,B,H], gates/dG [T,B,4H],
@@ -179,6 +180,48 @@ def lstm_fwd_bwd(x, W, b=None, h0=None, c0=None, dy=None, dhT=None, dcT=None, li
     out = dict(f)
     out.update(g)
     return out
+
+
+def lstm_stack_fwd(x, Ws, bs=None, h0s=None, c0s=None, lib=None, mask=None, reverse=False,
+                   ijfo=False):
+    """Stacked LSTM forward ("cmu 10-414 HW4" page, the multi-layer LSTM
+    module's forward; "mxnet-lstm" page, "Stack Multiple RNN Cells"): layer 0
+    runs the single-layer cell on x; layer l > 0 runs it on the outputs y of
+    layer l-1.  Layer l has its own W_l [4H, H + I_l] (I_0 = I, I_l = H after),
+    b_l and initial state h0s[l], c0s[l] [B, H]; its final state is kept apart
+    (hT / cT per layer) and only y passes upward.  mask / reverse / ijfo apply
+    to every layer.  Returns the list of per-layer forward dicts; the stack's
+    output is the last one's "y"."""
+    L = len(Ws)
+    out, inp = [], x
+    for l in range(L):
+        f = lstm_fwd(inp, Ws[l], None if bs is None else bs[l],
+                     None if h0s is None else h0s[l], None if c0s is None else c0s[l],
+                     lib=lib, mask=mask, reverse=reverse, ijfo=ijfo)
+        out.append(f)
+        inp = f["y"]
+    return out
+
+
+def lstm_stack_bwd(x, Ws, h0s, c0s, fwds, dy=None, dhTs=None, dcTs=None, lib=None, mask=None,
+                   reverse=False, ijfo=False):
+    """Stacked LSTM backward: the chain rule through the composition of
+    lstm_stack_fwd.  The top layer takes dy; layer l-1 takes the gradient at
+    its outputs y, which is the dx of layer l; dhTs[l] / dcTs[l] enter at layer
+    l's final state.  Returns the list of per-layer gradient dicts (layer 0's
+    "dx" is the gradient at x)."""
+    L = len(Ws)
+    grads = [None] * L
+    up = dy
+    for l in reversed(range(L)):
+        xin = x if l == 0 else fwds[l - 1]["y"]
+        g = lstm_bwd(xin, Ws[l], None if h0s is None else h0s[l],
+                     None if c0s is None else c0s[l], fwds[l], up,
+                     None if dhTs is None else dhTs[l], None if dcTs is None else dcTs[l],
+                     lib=lib, mask=mask, reverse=reverse, ijfo=ijfo)
+        grads[l] = g
+        up = g["dx"]
+    return grads
 
 
 def surrogate_loss(fwd, dy=None, dhT=None, dcT=None) -> float:
