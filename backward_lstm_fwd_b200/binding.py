@@ -28,7 +28,8 @@ LSTM_BF16 = 1
 LSTM_F16 = 2
 
 EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd", "lstm_bwd",
-           "lstm_fwd_ex", "lstm_bwd_ex",
+           "lstm_fwd_ex", "lstm_bwd_ex", "lstm_stack_fwd_workspace_size",
+           "lstm_stack_bwd_workspace_size", "lstm_stack_fwd", "lstm_stack_bwd",
            "lstm_status", "lstm_profile_begin", "lstm_profile_end", "lstm_launch_count",
            "lstm_strerror", "lstm_abi_version")
 
@@ -86,6 +87,16 @@ def load(path: str = LIB_PATH):
     lib.lstm_fwd_ex.restype = ip
     lib.lstm_bwd_ex.argtypes = [dp, op] + [vp] * 15 + [vp, sz, vp]
     lib.lstm_bwd_ex.restype = ip
+    pp = ctypes.POINTER(ctypes.c_void_p)  # host array of device pointers
+    lib.lstm_stack_fwd_workspace_size.argtypes = [dp, ip]
+    lib.lstm_stack_fwd_workspace_size.restype = sz
+    lib.lstm_stack_bwd_workspace_size.argtypes = [dp, ip]
+    lib.lstm_stack_bwd_workspace_size.restype = sz
+    lib.lstm_stack_fwd.argtypes = [dp, ip, op, vp, pp, pp] + [vp] * 7 + [vp, sz, vp]
+    lib.lstm_stack_fwd.restype = ip
+    lib.lstm_stack_bwd.argtypes = [dp, ip, op] + [vp] * 4 + [pp] + [vp] * 6 + [pp, pp] + \
+        [vp] * 2 + [vp, sz, vp]
+    lib.lstm_stack_bwd.restype = ip
     lib.lstm_status.argtypes = [vp, sz, vp]
     lib.lstm_status.restype = ip
     lib.lstm_strerror.argtypes = [ip]
@@ -220,6 +231,57 @@ def lstm_bwd(d: Dims, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, d
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
+def _ptr_array(ts):
+    """A host array of device pointers (None, a tensor or an int per entry);
+    None for no array at all."""
+    if ts is None:
+        return None
+    return (ctypes.c_void_p * len(ts))(*[_p(t) for t in ts])
+
+
+def stack_fwd_workspace_size(d: Dims, L: int) -> int:
+    return int(load().lstm_stack_fwd_workspace_size(ctypes.byref(d), int(L)))
+
+
+def stack_bwd_workspace_size(d: Dims, L: int) -> int:
+    return int(load().lstm_stack_bwd_workspace_size(ctypes.byref(d), int(L)))
+
+
+def lstm_stack_fwd(d: Dims, L: int, x, Ws, bs, h0, c0, y, hT, cT, gates, cells, ws,
+                   ws_bytes=None, stream=None, check: bool = True, mask=None,
+                   reverse: bool = False, gate_order="ifjo") -> int:
+    """Direct call of lstm_stack_fwd: Ws / bs are lists of L device tensors
+    (bs may be None); the [L][...] arrays are single tensors."""
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    opt = _options(mask, reverse, gate_order)
+    Wa, ba = _ptr_array(Ws), _ptr_array(bs)
+    rc = load().lstm_stack_fwd(ctypes.byref(d), int(L), ctypes.byref(opt), _p(x), Wa, ba, _p(h0),
+                               _p(c0), _p(y), _p(hT), _p(cT), _p(gates), _p(cells), _p(ws),
+                               ws_bytes, _stream(stream))
+    if check and rc != LSTM_OK:
+        raise LstmError(rc, "lstm_stack_fwd")
+    return rc
+
+
+def lstm_stack_bwd(d: Dims, L: int, dy, dhT, dcT, x, Ws, h0, c0, y, gates, cells, dx, dWs, dbs,
+                   dh0, dc0, ws, ws_bytes=None, stream=None, check: bool = True, mask=None,
+                   reverse: bool = False, gate_order="ifjo") -> int:
+    """Direct call of lstm_stack_bwd: Ws, dWs and dbs are lists of L device
+    tensors."""
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    opt = _options(mask, reverse, gate_order)
+    Wa, dWa, dba = _ptr_array(Ws), _ptr_array(dWs), _ptr_array(dbs)
+    rc = load().lstm_stack_bwd(ctypes.byref(d), int(L), ctypes.byref(opt), _p(dy), _p(dhT),
+                               _p(dcT), _p(x), Wa, _p(h0), _p(c0), _p(y), _p(gates), _p(cells),
+                               _p(dx), dWa, dba, _p(dh0), _p(dc0), _p(ws), ws_bytes,
+                               _stream(stream))
+    if check and rc != LSTM_OK:
+        raise LstmError(rc, "lstm_stack_bwd")
+    return rc
+
+
 def lstm_fwd_noalloc(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, stream=None,
                      check: bool = True) -> int:
     """Direct call of lstm_fwd_noalloc: lstm_fwd with the library's static
@@ -335,4 +397,58 @@ def backward(st: State, x, W, h0=None, c0=None, dy=None, dhT=None, dcT=None, ws=
     lstm_bwd(st.dims, dy, dhT, dcT, x, W, h0, c0, st.y, st.gates, st.cells, g.dx, g.dW, g.db,
              g.dh0, g.dc0, ws, stream=stream, mask=mask, reverse=reverse,
              gate_order=gate_order)
+    return g
+
+
+class StackState:
+    """Outputs of one lstm_stack_fwd call: every layer's saved state."""
+
+    def __init__(self, L, T, B, I, H, cd, device):
+        self.L = L
+        self.dims = dims(T, B, I, H, cd)
+        self.y = torch.empty((L, T, B, H), dtype=cd, device=device)
+        self.hT = torch.empty((L, B, H), dtype=cd, device=device)
+        self.cT = torch.empty((L, B, H), dtype=torch.float32, device=device)
+        self.gates = torch.empty((L, T, B, 4 * H), dtype=cd, device=device)
+        self.cells = torch.empty((L, T, B, H), dtype=torch.float32, device=device)
+
+
+class StackGrads:
+    def __init__(self, L, T, B, I, H, device):
+        f = torch.float32
+        self.dx = torch.empty((T, B, I), dtype=f, device=device)
+        self.dW = [torch.empty((4 * H, H + (I if l == 0 else H)), dtype=f, device=device)
+                   for l in range(L)]
+        self.db = [torch.empty((4 * H,), dtype=f, device=device) for _ in range(L)]
+        self.dh0 = torch.empty((L, B, H), dtype=f, device=device)
+        self.dc0 = torch.empty((L, B, H), dtype=f, device=device)
+
+
+def forward_stack(x, Ws, bs=None, h0=None, c0=None, ws=None, stream=None, mask=None,
+                  reverse: bool = False, gate_order="ifjo") -> StackState:
+    """Allocate outputs and run lstm_stack_fwd.  x [T,B,I]; Ws[l] [4H, H+I_l];
+    h0 [L,B,H] (compute dtype), c0 [L,B,H] float32."""
+    T, B, I = x.shape
+    L, H = len(Ws), Ws[0].shape[0] // 4
+    st = StackState(L, T, B, I, H, x.dtype, x.device)
+    if ws is None:
+        ws = empty_workspace(stack_fwd_workspace_size(st.dims, L), x.device)
+    lstm_stack_fwd(st.dims, L, x, Ws, bs, h0, c0, st.y, st.hT, st.cT, st.gates, st.cells, ws,
+                   stream=stream, mask=mask, reverse=reverse, gate_order=gate_order)
+    return st
+
+
+def backward_stack(st: StackState, x, Ws, h0=None, c0=None, dy=None, dhT=None, dcT=None,
+                   ws=None, stream=None, mask=None, reverse: bool = False,
+                   gate_order="ifjo") -> StackGrads:
+    """Allocate gradients and run lstm_stack_bwd on the saved state of
+    forward_stack()."""
+    T, B, I = x.shape
+    L, H = len(Ws), Ws[0].shape[0] // 4
+    g = StackGrads(L, T, B, I, H, x.device)
+    if ws is None:
+        ws = empty_workspace(stack_bwd_workspace_size(st.dims, L), x.device)
+    lstm_stack_bwd(st.dims, L, dy, dhT, dcT, x, Ws, h0, c0, st.y, st.gates, st.cells, g.dx, g.dW,
+                   g.db, g.dh0, g.dc0, ws, stream=stream, mask=mask, reverse=reverse,
+                   gate_order=gate_order)
     return g

@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdlib>
 #include <mutex>
@@ -324,8 +325,10 @@ constexpr size_t kMaxSmem = 227 * 1024;
 // Grid of the persistent forward recurrence: S = H/16 unit slices times G
 // batch groups of NB rows (NB a power of two in 16..128), S*G <= SM count.
 bool plan_fwd_recur(const lstm_dims *d, RecPlan &P) {
+    // (the kernel reads W through a tensor map: rows of H + I elements must be
+    // whole 16-byte groups)
     if (d->dtype != LSTM_BF16 || d->H % rec::UNITS != 0 || d->H > 1024 || d->B < 1 ||
-        tcg::encode_fn() == nullptr)
+        (d->H + d->I) % 8 != 0 || tcg::encode_fn() == nullptr)
         return false;
     const char *e = getenv("LSTM_FORCE_SIMT");
     if (e && e[0] == '1') return false;
@@ -538,8 +541,9 @@ const void *fwd2_kernel_ptr(int NB, int KS) {
 // Forward: R = H/32 row slices x KS K-parts x G batch groups of NB rows;
 // R * G clusters of KS must be co-resident.
 bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
+    // (W through a tensor map: rows of H + I elements in whole 16-byte groups)
     if (d->dtype != LSTM_BF16 || d->H % rec2::F_UNITS != 0 || d->B < 1 ||
-        tcg::encode_fn() == nullptr || force_simt())
+        (d->H + d->I) % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
     const int nsm = tcg::sm_count();
     P.R = d->H / rec2::F_UNITS;
@@ -1384,6 +1388,129 @@ int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const
                         (const bf *)h0, c0, (const bf *)mask, reverse, ijfo, (const bf *)y,
                         (const bf *)gates, cells, dx, dW, db, dh0, dc0, (char *)ws, s);
 }
+// ------------------------------------------------------- stacked layers
+// Layer l of a stack: layer 0 has the caller's sizes, every later layer reads
+// the H-wide outputs of the one below it.
+lstm_dims layer_dims(const lstm_dims *d, int l) {
+    lstm_dims e = *d;
+    if (l > 0) e.I = d->H;
+    return e;
+}
+
+// Per-layer slices of the [L][...] arrays start 16-byte aligned when B*H
+// elements of every stored type are whole 16-byte groups.
+bool stack_slices_aligned(const lstm_dims *d) {
+    const long long BH = (long long)d->B * d->H;
+    return (BH * (long long)esize(d)) % 16 == 0 && (BH * 4) % 16 == 0;
+}
+
+struct StackBwdLayout {
+    size_t layer, dxbuf, dybuf, total;
+};
+StackBwdLayout stack_bwd_layout(const lstm_dims *d, int L) {
+    StackBwdLayout S;
+    S.layer = bwd_layout(d).total;
+    if (L > 1) {
+        const lstm_dims d1 = layer_dims(d, 1);
+        S.layer = std::max(S.layer, bwd_layout(&d1).total);
+    }
+    S.dxbuf = S.dybuf = S.total = S.layer;
+    if (L > 1) {  // dx of the layer above (float) and its compute-type copy
+        const size_t TBH = (size_t)d->T * d->B * d->H;
+        S.dybuf = align_up(S.dxbuf + TBH * sizeof(float), 256);
+        S.total = align_up(S.dybuf + TBH * esize(d), 256);
+    }
+    return S;
+}
+
+size_t stack_fwd_ws(const lstm_dims *d, int L) {
+    size_t n = fwd_layout(d).total;
+    if (L > 1) {
+        const lstm_dims d1 = layer_dims(d, 1);
+        n = std::max(n, fwd_layout(&d1).total);
+    }
+    return n;
+}
+
+// Layers 0 .. L-1 in order, each one lstm_fwd_ex call on the same stream.
+int stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
+              const void *const *W, const void *const *b, const void *h0, const float *c0,
+              void *y, void *hT, float *cT, void *gates, float *cells, void *ws, size_t ws_bytes,
+              void *stream) {
+    if (!dims_ok(d) || L < 1 || !W) return LSTM_ERR_INVALID_ARG;
+    for (int l = 0; l < L; ++l)  // every layer's parameters, before any layer runs
+        if (!ptr_ok(W[l], d->H > 0) || (b && !ptr_ok(b[l], false))) return LSTM_ERR_INVALID_ARG;
+    if (L > 1 && !stack_slices_aligned(d)) return LSTM_ERR_UNSUPPORTED;
+    const size_t es = esize(d);
+    const long long BH = (long long)d->B * d->H, TBH = (long long)d->T * BH;
+    const char *yb = static_cast<const char *>(y);
+    for (int l = 0; l < L; ++l) {
+        const lstm_dims dl = layer_dims(d, l);
+        const void *xl = l == 0 ? x : yb + (size_t)(l - 1) * TBH * es;
+        const int rc = fwd_entry(
+            &dl, opt, xl, W[l], b ? b[l] : nullptr,
+            h0 ? static_cast<const char *>(h0) + (size_t)l * BH * es : nullptr,
+            c0 ? c0 + (size_t)l * BH : nullptr, static_cast<char *>(y) + (size_t)l * TBH * es,
+            static_cast<char *>(hT) + (size_t)l * BH * es, cT + (size_t)l * BH,
+            static_cast<char *>(gates) + (size_t)l * TBH * 4 * es, cells + (size_t)l * TBH, ws,
+            ws_bytes, stream);
+        if (rc != LSTM_OK) return rc;
+    }
+    return LSTM_OK;
+}
+
+// Layers L-1 .. 0, each one lstm_bwd_ex call; between two calls the float dx
+// of the upper layer becomes the lower layer's dy in the compute type.
+int stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy,
+              const void *dhT, const float *dcT, const void *x, const void *const *W,
+              const void *h0, const float *c0, const void *y, const void *gates,
+              const float *cells, float *dx, float *const *dW, float *const *db, float *dh0,
+              float *dc0, void *ws, size_t ws_bytes, void *stream) {
+    if (!dims_ok(d) || L < 1 || !W || !dW || !db) return LSTM_ERR_INVALID_ARG;
+    for (int l = 0; l < L; ++l) {  // every layer's parameters, before any layer runs
+        const long long K = (long long)d->H + (l == 0 ? d->I : d->H);
+        if (!ptr_ok(W[l], d->H > 0) || !ptr_ok(dW[l], 4LL * d->H * K > 0) ||
+            !ptr_ok(db[l], d->H > 0))
+            return LSTM_ERR_INVALID_ARG;
+    }
+    if (L > 1 && !stack_slices_aligned(d)) return LSTM_ERR_UNSUPPORTED;
+    const StackBwdLayout S = stack_bwd_layout(d, L);
+    const int wsrc = ws_ok(ws, ws_bytes, S.total);
+    if (wsrc != LSTM_OK) return wsrc;
+    const size_t es = esize(d);
+    const long long BH = (long long)d->B * d->H, TBH = (long long)d->T * BH;
+    char *wsb = static_cast<char *>(ws);
+    float *dxbuf = reinterpret_cast<float *>(wsb + S.dxbuf);
+    void *dybuf = wsb + S.dybuf;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int l = L - 1; l >= 0; --l) {
+        const lstm_dims dl = layer_dims(d, l);
+        const void *xl = l == 0 ? x : static_cast<const char *>(y) + (size_t)(l - 1) * TBH * es;
+        const int rc = bwd_entry(
+            &dl, opt, l == L - 1 ? dy : dybuf,
+            dhT ? static_cast<const char *>(dhT) + (size_t)l * BH * es : nullptr,
+            dcT ? dcT + (size_t)l * BH : nullptr, xl, W[l],
+            h0 ? static_cast<const char *>(h0) + (size_t)l * BH * es : nullptr,
+            c0 ? c0 + (size_t)l * BH : nullptr,
+            static_cast<const char *>(y) + (size_t)l * TBH * es,
+            static_cast<const char *>(gates) + (size_t)l * TBH * 4 * es, cells + (size_t)l * TBH,
+            l == 0 ? dx : dxbuf, dW[l], db[l], dh0 + (size_t)l * BH, dc0 + (size_t)l * BH, ws,
+            S.layer, stream);
+        if (rc != LSTM_OK) return rc;
+        if (l > 0 && TBH > 0) {
+            const unsigned grid = (unsigned)((TBH + 255) / 256);
+            if (d->dtype == LSTM_F32)
+                simt::from_float_copy<float><<<grid, 256, 0, s>>>(dxbuf, (float *)dybuf, TBH);
+            else if (d->dtype == LSTM_F16)
+                simt::from_float_copy<__half><<<grid, 256, 0, s>>>(dxbuf, (__half *)dybuf, TBH);
+            else
+                simt::from_float_copy<bf16><<<grid, 256, 0, s>>>(dxbuf, (bf16 *)dybuf, TBH);
+            note_launch();
+            if (cudaGetLastError() != cudaSuccess) return LSTM_ERR_CUDA;
+        }
+    }
+    return LSTM_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -1441,6 +1568,32 @@ int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, con
                 size_t ws_bytes, void *stream) {
     return bwd_entry(d, opt, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0, dc0,
                      ws, ws_bytes, stream);
+}
+
+size_t lstm_stack_fwd_workspace_size(const lstm_dims *d, int L) {
+    if (!dims_ok(d) || L < 1) return 0;
+    return stack_fwd_ws(d, L);
+}
+
+size_t lstm_stack_bwd_workspace_size(const lstm_dims *d, int L) {
+    if (!dims_ok(d) || L < 1) return 0;
+    return stack_bwd_layout(d, L).total;
+}
+
+int lstm_stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
+                   const void *const *W, const void *const *b, const void *h0, const float *c0,
+                   void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
+                   size_t ws_bytes, void *stream) {
+    return stack_fwd(d, L, opt, x, W, b, h0, c0, y, hT, cT, gates, cells, ws, ws_bytes, stream);
+}
+
+int lstm_stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy,
+                   const void *dhT, const float *dcT, const void *x, const void *const *W,
+                   const void *h0, const float *c0, const void *y, const void *gates,
+                   const float *cells, float *dx, float *const *dW, float *const *db,
+                   float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream) {
+    return stack_bwd(d, L, opt, dy, dhT, dcT, x, W, h0, c0, y, gates, cells, dx, dW, db, dh0,
+                     dc0, ws, ws_bytes, stream);
 }
 
 int lstm_profile_begin(void) {

@@ -308,6 +308,14 @@ __global__ void to_float_copy(const T *in, float *out, long long n) {
     if (i < n) out[i] = in ? to_f(in[i]) : 0.f;
 }
 
+// float -> compute type (the gradient at a layer's outputs, handed to the
+// layer below it as its dy)
+template <class T>
+__global__ void from_float_copy(const float *in, T *out, long long n) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) out[i] = from_f<T>(in[i]);
+}
+
 template <class T>
 __global__ void copy_or_zero(const T *in, T *out, long long n) {
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;

@@ -390,6 +390,155 @@ def run_ours(args, w, rank, world, local_rank):
     return 0
 
 
+def run_stack(args, w, rank, world, local_rank):
+    """--layers L > 1: one step = lstm_stack_fwd + lstm_stack_bwd over L layers
+    (layer 0 on the workload's x, layers above on H-wide inputs), inputs
+    resident in HBM.  `value` counts the T*B timesteps of the stack per step;
+    the roofline's FLOPs sum every layer's share of the dominant phase."""
+    import dataclasses
+
+    from backward_lstm_fwd_b200 import binding as L
+    from backward_lstm_fwd_b200 import build as lbuild
+    lbuild.build()
+    L.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    Lc, T, B, I, H = args.layers, w.T, w.B, w.I, w.H
+    layers = [synth.make_inputs(w if l == 0 else dataclasses.replace(
+        w, name=f"{w.name}_layer{l}", I=H, seed=w.seed + 7 * l)) for l in range(Lc)]
+    inputs = dict(x=layers[0]["x"], dy=layers[-1]["dy"])
+    for k in ("h0", "c0", "dhT", "dcT"):
+        inputs[k] = torch.stack([p[k] for p in layers]).contiguous()
+    Ws = [p["W"].to(dev) for p in layers]
+    bs = [p["b"].to(dev) for p in layers]
+    d = {k: v.to(dev) for k, v in inputs.items()}
+    cd = synth.torch_dtype(w.dtype)
+    st = L.StackState(Lc, T, B, I, H, cd, dev)
+    gr = L.StackGrads(Lc, T, B, I, H, dev)
+    ws_f = L.empty_workspace(L.stack_fwd_workspace_size(st.dims, Lc), dev)
+    ws_b = L.empty_workspace(L.stack_bwd_workspace_size(st.dims, Lc), dev)
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+
+    def step(src):
+        L.lstm_stack_fwd(st.dims, Lc, src["x"], Ws, bs, src["h0"], src["c0"], st.y, st.hT,
+                         st.cT, st.gates, st.cells, ws_f, stream=stream)
+        L.lstm_stack_bwd(st.dims, Lc, src["dy"], src["dhT"], src["dcT"], src["x"], Ws,
+                         src["h0"], src["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db,
+                         gr.dh0, gr.dc0, ws_b, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(d)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    n0 = L.launch_count()
+    L.profile_begin()
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step(d)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    phases = L.profile_end()
+    launches = L.launch_count() - n0
+    barrier()
+    clk = clocks.stop() if clocks else None
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    for ws in (ws_f, ws_b):
+        if L.lstm_status(ws, stream=stream) != L.LSTM_OK:
+            raise RuntimeError("device-side status set during the timed region")
+
+    # end to end: every step uploads its inputs from pinned host memory and
+    # reads every gradient back (no overlap with the compute)
+    pin_in = {k: v.pin_memory() for k, v in inputs.items()}
+    outs = [gr.dx, gr.dh0, gr.dc0] + gr.dW + gr.db
+    pin_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    f0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            for k in pin_in:
+                d[k].copy_(pin_in[k], non_blocking=True)
+            step(d)
+            for t, p in zip(outs, pin_out):
+                p.copy_(t, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1))
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    layer_w = [w] + [dataclasses.replace(w, I=H)] * (Lc - 1)
+    works = [phase_work(lw, phases) for lw in layer_w]
+    dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
+    dom_ms, dom_launches = phases[dom]
+    kind = works[0][dom][0]
+    amount = sum(wk[dom][1] for wk in works) * args.steps
+    if kind == "flop":
+        achieved = amount / (dom_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None}
+    else:
+        achieved = amount / (dom_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None}
+    roof.update({"kernel": dom, "launches_per_step": dom_launches / args.steps,
+                 "ms_per_step": dom_ms / args.steps,
+                 "peak_source": f"{peak_src} ({'sustained bf16' if kind == 'flop' else 'HBM copy'})"})
+    step_s = ms / args.steps * 1e-3
+    tflops = sum(lw.flops for lw in layer_w) / step_s / 1e12
+    line = {
+        "metric": METRIC, "value": world * w.rows / step_s, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded, distributions of the workload definition)",
+        "config": {"workload": f"{w.name}_stack{Lc}", "T": T, "B": B, "I": I, "H": H,
+                   "layers": Lc,
+                   "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+                   "l2": "working set > 126 MB L2 per step (no flush needed)"},
+        "tflops": tflops,
+        "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+        "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
+        "roofline": roof,
+        "phases_ms_per_step": {p: v[0] / args.steps for p, v in phases.items()},
+        "gpu_launches": launches,
+        "e2e": {"value": world * w.rows * args.steps / (ms_e2e * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e / args.steps, "overlap": "none"},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,6 +552,8 @@ def main():
     ap.add_argument("--dtype", choices=("bf16", "fp16"), default=None,
                     help="16-bit compute type override (fp16: the page's FLOAT16) on the "
                          "workload's shape")
+    ap.add_argument("--layers", type=int, default=1,
+                    help="a stack of this many LSTM layers (lstm_stack_fwd / lstm_stack_bwd)")
     ap.add_argument("--seq-mask", action="store_true",
                     help="variable length: a seq_length mask with seeded per-sequence "
                          "lengths in 0..T (every step is still computed and counted)")
@@ -431,6 +582,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.layers > 1:
+            return run_stack(args, w, rank, world, local_rank)
         return run_ours(args, w, rank, world, local_rank)
     finally:
         if world > 1:

@@ -191,6 +191,50 @@ int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, con
                 size_t ws_bytes, void *stream);
 
 /*
+ * lstm_stack_fwd / lstm_stack_bwd -- a stack of L >= 1 LSTM layers (the
+ * multi-layer LSTM module of the "cmu 10-414 HW4" page; "Stack Multiple RNN
+ * Cells" of the "mxnet-lstm" page).  Layer 0 reads x [T][B][I]; layer l > 0
+ * reads the outputs y of layer l-1.  Every layer has its own weights, bias
+ * and initial state, and its final state is an output of its own; only y
+ * passes upward.  Each layer is one lstm_fwd_ex / lstm_bwd_ex call (in that
+ * order on `stream`), so options, precision and errors are those calls'.
+ *
+ * d       sizes and compute type of layer 0; layer l > 0 has I = H.
+ * L       number of layers (< 1: LSTM_ERR_INVALID_ARG).
+ * W, b    HOST arrays of L DEVICE pointers: W[l] [4H][H + I_l] (I_0 = d->I,
+ *         I_l = d->H), b[l] [4H].  b may be NULL (no bias), as may any b[l].
+ * h0 [L][B][H] (compute type), c0 [L][B][H] (float): initial states, layer
+ *         after layer; either may be NULL (zeros).
+ * y [L][T][B][H], gates [L][T][B][4H], cells [L][T][B][H]: every layer's
+ *         saved state (the backward reads them); the stack's output is the
+ *         slice y[L-1].  hT [L][B][H], cT [L][B][H] (float): final states.
+ * opt     as for lstm_fwd_ex, applied to every layer (NULL = defaults).
+ * ws      at least lstm_stack_fwd_workspace_size(d, L) bytes.
+ * With L > 1 every [L][...] slice must start 16-byte aligned: B*H a
+ * multiple of 8 for the 16-bit types, of 4 for float (else
+ * LSTM_ERR_UNSUPPORTED).
+ *
+ * lstm_stack_bwd: dy [T][B][H] (compute type, or NULL) is the gradient at the
+ * top layer's outputs; dhT [L][B][H] (compute type) and dcT [L][B][H]
+ * (float), either NULL, the gradients at every layer's final state.  Outputs
+ * (float): dx [T][B][I]; dW and db, HOST arrays of L DEVICE pointers to
+ * dW[l] [4H][H + I_l] and db[l] [4H]; dh0, dc0 [L][B][H].  Layer l-1's dy is
+ * layer l's dx rounded to the compute type.  ws at least
+ * lstm_stack_bwd_workspace_size(d, L) bytes.  The layers run L-1 .. 0.
+ */
+size_t lstm_stack_fwd_workspace_size(const lstm_dims *d, int L);
+size_t lstm_stack_bwd_workspace_size(const lstm_dims *d, int L);
+int lstm_stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
+                   const void *const *W, const void *const *b, const void *h0, const float *c0,
+                   void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
+                   size_t ws_bytes, void *stream);
+int lstm_stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy,
+                   const void *dhT, const float *dcT, const void *x, const void *const *W,
+                   const void *h0, const float *c0, const void *y, const void *gates,
+                   const float *cells, float *dx, float *const *dW, float *const *db,
+                   float *dh0, float *dc0, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * lstm_status -- synchronise `stream`, then read and clear the device status
  * word kept in the first bytes of a workspace used by lstm_fwd / lstm_bwd.
  * Every call zeroes the word when it starts (in stream order), so it reports

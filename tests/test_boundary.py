@@ -204,3 +204,66 @@ def test_misaligned_mask_rejected(lib):
                          a["c0"], a["y"], a["hT"], a["cT"], a["gates"], a["cells"], a["ws"],
                          a["ws_bytes"], None)
     assert rc == L.LSTM_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------- stacked layers
+DS = L.dims(4, 8, 16, 32, L.LSTM_BF16)
+
+
+def call_stack_fwd(d, Lc, Ws=(FAKE, FAKE), bs=None, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.stack_fwd_workspace_size(d, max(Lc, 1))
+    return L.lstm_stack_fwd(d, Lc, FAKE, None if Ws is None else list(Ws), bs, None, None, FAKE,
+                            FAKE, FAKE, FAKE, FAKE, FAKE, ws_bytes=ws_bytes, stream=0,
+                            check=False)
+
+
+def call_stack_bwd(d, Lc, Ws=(FAKE, FAKE), dWs=(FAKE, FAKE), dbs=(FAKE, FAKE), ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.stack_bwd_workspace_size(d, max(Lc, 1))
+    return L.lstm_stack_bwd(d, Lc, FAKE, None, None, FAKE, None if Ws is None else list(Ws),
+                            None, None, FAKE, FAKE, FAKE, FAKE,
+                            None if dWs is None else list(dWs),
+                            None if dbs is None else list(dbs), FAKE, FAKE, FAKE,
+                            ws_bytes=ws_bytes, stream=0, check=False)
+
+
+def test_stack_workspace_sizes(lib):
+    one = L.bwd_workspace_size(DS)
+    upper = L.bwd_workspace_size(L.dims(4, 8, 32, 32, L.LSTM_BF16))
+    assert L.stack_fwd_workspace_size(DS, 1) == L.fwd_workspace_size(DS)
+    assert L.stack_bwd_workspace_size(DS, 1) == one
+    # two layers: the larger layer's workspace plus dx (float) and dy (bf16)
+    # of the upper layer, [T][B][H] each
+    need = max(one, upper) + 4 * 8 * 32 * (4 + 2)
+    assert L.stack_bwd_workspace_size(DS, 2) >= need
+    assert L.stack_bwd_workspace_size(DS, 0) == 0 and L.stack_fwd_workspace_size(DS, -1) == 0
+
+
+@pytest.mark.parametrize("Lc", [0, -2])
+def test_stack_layer_count_rejected(lib, Lc):
+    assert call_stack_fwd(DS, Lc, ws_bytes=1 << 20) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_bwd(DS, Lc, ws_bytes=1 << 20) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_stack_parameter_arrays_checked_before_any_layer(lib):
+    """A missing or misaligned W / dW / db of any layer is reported before the
+    first layer is enqueued."""
+    assert call_stack_fwd(DS, 2, Ws=None) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_fwd(DS, 2, Ws=(FAKE, None)) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_fwd(DS, 2, Ws=(FAKE, FAKE + 2)) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_fwd(DS, 2, bs=[None, FAKE + 4]) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_bwd(DS, 2, dWs=(FAKE, None)) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_bwd(DS, 2, dbs=None) == L.LSTM_ERR_INVALID_ARG
+    assert call_stack_bwd(DS, 2, Ws=(None, FAKE)) == L.LSTM_ERR_INVALID_ARG
+
+
+def test_stack_slices_must_align(lib):
+    d = L.dims(4, 3, 16, 12, L.LSTM_BF16)  # B*H = 36: per-layer slices off 16 bytes
+    assert call_stack_fwd(d, 2) == L.LSTM_ERR_UNSUPPORTED
+    assert call_stack_bwd(d, 2) == L.LSTM_ERR_UNSUPPORTED
+
+
+def test_stack_workspace_too_small(lib):
+    need = L.stack_bwd_workspace_size(DS, 2)
+    assert call_stack_bwd(DS, 2, ws_bytes=need - 1) == L.LSTM_ERR_WORKSPACE

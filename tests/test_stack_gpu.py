@@ -1,0 +1,145 @@
+"""Stacked LSTM layers (lstm_stack_fwd / lstm_stack_bwd: the multi-layer LSTM
+module of the "cmu 10-414 HW4" page, "Stack Multiple RNN Cells" of the
+"mxnet-lstm" page) through the C ABI against the fp64 stacked oracle, element
+by element, on the kernel paths of the layers (per-step kernels, the fused
+forward and the TMEM-weight backward in one launch and in chunks, with the
+layer-0 input width differing from H), in every compute type, and with the
+options; plus two identities: one layer is the single-layer call, and L layers
+are L single-layer calls with dx rounded to the compute type in between, bit
+for bit.  Tolerance as in the other parity tests."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from backward_lstm_fwd_b200 import binding as L
+from backward_lstm_fwd_b200 import synth
+from tests.parity_util import assert_within, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+def stack_inputs(T, B, I, H, Lc, dt, seed):
+    """Layer 0 from the workload generator; the upper layers' W, b, h0, c0,
+    dhT, dcT from the generator of a workload with I = H (another seed each)."""
+    layers = [synth.make_inputs(synth.custom(T, B, I if l == 0 else H, H, dt, seed=seed + 7 * l))
+              for l in range(Lc)]
+    inp = dict(x=layers[0]["x"], dy=layers[-1]["dy"])
+    inp["W"] = [p["W"] for p in layers]
+    inp["b"] = [p["b"] for p in layers]
+    for k in ("h0", "c0", "dhT", "dcT"):
+        inp[k] = torch.stack([p[k] for p in layers]).contiguous()
+    return inp
+
+
+def run_gpu_stack(inp, dev, **opt):
+    Lc = len(inp["W"])
+    d = {k: ([t.to(dev) for t in v] if isinstance(v, list) else v.to(dev))
+         for k, v in inp.items()}
+    mk = opt.pop("mask", None)
+    if mk is not None:
+        mk = mk.to(dev)
+    st = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"], mask=mk, **opt)
+    g = L.backward_stack(st, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"], d["dcT"],
+                         mask=mk, **opt)
+    torch.cuda.synchronize()
+    n = lambda t: t.float().cpu().double().numpy()
+    return dict(y=n(st.y), hT=n(st.hT), cT=n(st.cT), dx=n(g.dx), dh0=n(g.dh0), dc0=n(g.dc0),
+                dW=[n(t) for t in g.dW], db=[n(t) for t in g.db], L=Lc)
+
+
+def run_oracle_stack(inp, mask=None, reverse=False, gate_order="ifjo"):
+    f64 = lambda t: t.double().numpy()
+    Lc = len(inp["W"])
+    Ws, bs = [f64(w) for w in inp["W"]], [f64(b) for b in inp["b"]]
+    h0s, c0s = [f64(inp["h0"][l]) for l in range(Lc)], [f64(inp["c0"][l]) for l in range(Lc)]
+    dhTs, dcTs = [f64(inp["dhT"][l]) for l in range(Lc)], [f64(inp["dcT"][l]) for l in range(Lc)]
+    opt = dict(mask=None if mask is None else f64(mask), reverse=reverse,
+               ijfo=gate_order == "ijfo")
+    f = oracle.lstm_stack_fwd(f64(inp["x"]), Ws, bs, h0s, c0s, **opt)
+    g = oracle.lstm_stack_bwd(f64(inp["x"]), Ws, h0s, c0s, f, f64(inp["dy"]), dhTs, dcTs, **opt)
+    return dict(y=np.stack([fl["y"] for fl in f]), hT=np.stack([fl["hT"] for fl in f]),
+                cT=np.stack([fl["cT"] for fl in f]), dx=g[0]["dx"],
+                dh0=np.stack([gl["dh0"] for gl in g]), dc0=np.stack([gl["dc0"] for gl in g]),
+                dW=[gl["dW"] for gl in g], db=[gl["db"] for gl in g])
+
+
+def check(gpu, ref, dt, label):
+    errs = {k: rel_err(gpu[k], ref[k]) for k in ("y", "hT", "cT", "dx", "dh0", "dc0")}
+    for l in range(gpu["L"]):
+        errs[f"dW{l}"] = rel_err(gpu["dW"][l], ref["dW"][l])
+        errs[f"db{l}"] = rel_err(gpu["db"][l], ref["db"][l])
+    assert_within(errs, dt, label)
+
+
+CASES = [
+    (6, 4, 24, 40, 3, "fp32"),      # per-step kernels, three layers
+    (7, 5, 37, 48, 2, "bf16"),      # per-step kernels, bf16
+    (12, 48, 64, 512, 2, "bf16"),   # TMEM-weight kernels, layer 0 narrower than H
+    (40, 64, 1024, 512, 2, "bf16"), # chunked backward, layer 0 wider than H
+    (12, 48, 64, 512, 3, "fp16"),   # fp16
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_stack(case, cuda_device):
+    T, B, I, H, Lc, dt = case
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=T + B + H)
+    gpu = run_gpu_stack(inp, cuda_device)
+    ref = run_oracle_stack(inp)
+    check(gpu, ref, dt, f"stack {case}")
+
+
+def test_stack_with_options(cuda_device):
+    T, B, I, H, Lc, dt = 40, 64, 96, 512, 2, "bf16"
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=5)
+    mask = synth.length_mask(T, B, H, synth.random_lengths(T, B, seed=3), dt)
+    gpu = run_gpu_stack(inp, cuda_device, mask=mask, reverse=True, gate_order="ijfo")
+    ref = run_oracle_stack(inp, mask=mask, reverse=True, gate_order="ijfo")
+    check(gpu, ref, dt, "stack, mask, reverse, ijfo")
+
+
+def test_one_layer_stack_is_the_single_layer_call(cuda_device):
+    T, B, I, H = 12, 48, 64, 512
+    inp = stack_inputs(T, B, I, H, 1, "bf16", seed=1)
+    d = {k: ([t.to(cuda_device) for t in v] if isinstance(v, list) else v.to(cuda_device))
+         for k, v in inp.items()}
+    st = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"])
+    g = L.backward_stack(st, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"], d["dcT"])
+    s1 = L.forward(d["x"], d["W"][0], d["b"][0], d["h0"][0], d["c0"][0])
+    g1 = L.backward(s1, d["x"], d["W"][0], d["h0"][0], d["c0"][0], d["dy"], d["dhT"][0],
+                    d["dcT"][0])
+    torch.cuda.synchronize()
+    assert torch.equal(st.y[0], s1.y) and torch.equal(st.cT[0], s1.cT)
+    assert torch.equal(g.dx, g1.dx) and torch.equal(g.dW[0], g1.dW)
+    assert torch.equal(g.db[0], g1.db) and torch.equal(g.dh0[0], g1.dh0)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp32"])
+def test_stack_is_composed_single_layer_calls(dt, cuda_device):
+    """The host loop adds nothing: the same layers run as separate calls, with
+    the upper layer's dx rounded to the compute type by torch, give the same
+    bits."""
+    T, B, I, H, Lc = 9, 32, 48, 256, 3
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=8)
+    d = {k: ([t.to(cuda_device) for t in v] if isinstance(v, list) else v.to(cuda_device))
+         for k, v in inp.items()}
+    st = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"])
+    g = L.backward_stack(st, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"], d["dcT"])
+    xs, states = [d["x"]], []
+    for l in range(Lc):
+        s = L.forward(xs[-1], d["W"][l], d["b"][l], d["h0"][l], d["c0"][l])
+        states.append(s)
+        xs.append(s.y)
+    up, grads = d["dy"], [None] * Lc
+    for l in reversed(range(Lc)):
+        grads[l] = L.backward(states[l], xs[l], d["W"][l], d["h0"][l], d["c0"][l], up,
+                              d["dhT"][l], d["dcT"][l])
+        up = grads[l].dx.to(synth.torch_dtype(dt))
+    torch.cuda.synchronize()
+    for l in range(Lc):
+        assert torch.equal(st.y[l], states[l].y), l
+        assert torch.equal(st.hT[l], states[l].hT) and torch.equal(st.cT[l], states[l].cT), l
+        assert torch.equal(g.dW[l], grads[l].dW) and torch.equal(g.db[l], grads[l].db), l
+        assert torch.equal(g.dh0[l], grads[l].dh0) and torch.equal(g.dc0[l], grads[l].dc0), l
+    assert torch.equal(g.dx, grads[0].dx)
