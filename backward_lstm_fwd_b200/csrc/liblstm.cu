@@ -495,6 +495,7 @@ struct Rec2Plan {
     int KS, G, NB, kcc, R, stages;
     int kcx;  // fused forward: K chunks of x per CTA
     size_t smem;
+    int split = 1;  // fused forward: batch streams per cluster (NB rows each)
 };
 
 bool force_simt() {
@@ -571,16 +572,25 @@ bool plan_fwd2(const lstm_dims *d, Rec2Plan &P) {
     return false;
 }
 
+// Instantiations of the fused forward: (NB, KS) with one batch stream, and
+// (NB, KS) per stream with two.
+#define LSTM_F3_SPLIT1(X) X(16, 1) X(16, 2) X(16, 4) X(32, 1) X(32, 2) X(32, 4) X(32, 8) \
+    X(64, 2) X(64, 4) X(64, 8) X(128, 4) X(128, 8)
+#define LSTM_F3_SPLIT2(X) X(32, 2) X(32, 4) X(32, 8) X(64, 4) X(64, 8)
+
 template <class E>
-const void *fwd3_kernel_ptr(int NB, int KS, bool masked) {
+const void *fwd3_kernel_ptr(int NB, int KS, bool masked, int split) {
 #define LSTM_F3(nb, ks)                                                                    \
     if (NB == nb && KS == ks)                                                              \
-        return masked ? (const void *)rec3::fwd3_kernel<E, nb, ks, true>                   \
-                      : (const void *)rec3::fwd3_kernel<E, nb, ks, false>;
-    LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
-    LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
-    LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
-    LSTM_F3(128, 4) LSTM_F3(128, 8)
+        return masked ? (const void *)rec3::fwd3_kernel<E, nb, ks, true, SPLIT_>           \
+                      : (const void *)rec3::fwd3_kernel<E, nb, ks, false, SPLIT_>;
+    if (split == 1) {
+        constexpr int SPLIT_ = 1;
+        LSTM_F3_SPLIT1(LSTM_F3)
+    } else if (split == 2) {
+        constexpr int SPLIT_ = 2;
+        LSTM_F3_SPLIT2(LSTM_F3)
+    }
 #undef LSTM_F3
     return nullptr;
 }
@@ -591,6 +601,8 @@ const void *fwd3_kernel_ptr(int NB, int KS, bool masked) {
 bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
     const char *e = getenv("LSTM_FWD_FUSED_X");
     if (e && e[0] == '0') return false;
+    const char *es = getenv("LSTM_FWD_SPLIT");  // "1": one batch stream per cluster
+    const bool split_ok = !(es && es[0] == '1');
     if (d->dtype == LSTM_F32 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
         d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
@@ -608,17 +620,26 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
         while (NB < (d->B + G0 - 1) / G0) NB *= 2;
         NB = std::max(NB, 4 * KS);
         if (NB > 128 || NB / KS > 32) continue;
-        if (rec3::fwd3_tmem_cols(NB, kcc, kcx) > 512) continue;
         const int G = (d->B + NB - 1) / NB;
-        const size_t smem = rec3::Fwd3Smem(kcc, kcx, NB, KS).total + 1024;
-        if (smem > kMaxSmem) continue;
-        const void *kern = d->dtype == LSTM_F16 ? fwd3_kernel_ptr<__half>(NB, KS, masked)
-                                                : fwd3_kernel_ptr<bf16>(NB, KS, masked);
-        if (!kern) continue;
-        const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
-        if (G * P.R > maxc) continue;
-        P.KS = KS; P.G = G; P.NB = NB; P.kcc = kcc; P.kcx = kcx; P.smem = smem;
-        return true;
+        // two interleaved batch streams of NB / 2 rows per cluster where that
+        // instantiation exists and fits, else one
+        for (int split : {2, 1}) {
+            if (split == 2 && (!split_ok || NB < 64 || G * 2 > kMaxGroups)) continue;
+            const int NBv = NB / split;
+            if (NBv / KS < 4) continue;
+            if (rec3::fwd3_tmem_cols(NBv, kcc, kcx) > 512) continue;
+            const size_t smem = rec3::Fwd3Smem(kcc, kcx, NBv, KS, split).total + 1024;
+            if (smem > kMaxSmem) continue;
+            const void *kern = d->dtype == LSTM_F16
+                                   ? fwd3_kernel_ptr<__half>(NBv, KS, masked, split)
+                                   : fwd3_kernel_ptr<bf16>(NBv, KS, masked, split);
+            if (!kern) continue;
+            const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
+            if (G * P.R > maxc) continue;
+            P.KS = KS; P.G = G; P.NB = NBv; P.kcc = kcc; P.kcx = kcx; P.smem = smem;
+            P.split = split;
+            return true;
+        }
     }
     return false;
 }
@@ -786,23 +807,26 @@ int tc_fwd_recurrence2(const lstm_dims *d, const Rec2Plan &P, const bf16 *W, con
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
-template <class E, int NB, int KS>
+template <class E, int NB, int KS, int SPLIT>
 cudaError_t launch_fwd3_t(const rec3::Fwd3Params<E> &prm, const Rec2Plan &P, cudaStream_t s) {
     if (prm.mask)
-        return launch_cluster(rec3::fwd3_kernel<E, NB, KS, true>, prm, P.R * KS * P.G, KS,
+        return launch_cluster(rec3::fwd3_kernel<E, NB, KS, true, SPLIT>, prm, P.R * KS * P.G, KS,
                               P.smem, s, rec2::F_THREADS);
-    return launch_cluster(rec3::fwd3_kernel<E, NB, KS, false>, prm, P.R * KS * P.G, KS, P.smem,
-                          s, rec2::F_THREADS);
+    return launch_cluster(rec3::fwd3_kernel<E, NB, KS, false, SPLIT>, prm, P.R * KS * P.G, KS,
+                          P.smem, s, rec2::F_THREADS);
 }
 
 template <class E>
 cudaError_t launch_fwd3(const rec3::Fwd3Params<E> &prm, const Rec2Plan &P, cudaStream_t s) {
 #define LSTM_F3(nb, ks) \
-    if (P.NB == nb && P.KS == ks) return launch_fwd3_t<E, nb, ks>(prm, P, s);
-    LSTM_F3(16, 1) LSTM_F3(16, 2) LSTM_F3(16, 4)
-    LSTM_F3(32, 1) LSTM_F3(32, 2) LSTM_F3(32, 4) LSTM_F3(32, 8)
-    LSTM_F3(64, 2) LSTM_F3(64, 4) LSTM_F3(64, 8)
-    LSTM_F3(128, 4) LSTM_F3(128, 8)
+    if (P.NB == nb && P.KS == ks) return launch_fwd3_t<E, nb, ks, SPLIT_>(prm, P, s);
+    if (P.split == 1) {
+        constexpr int SPLIT_ = 1;
+        LSTM_F3_SPLIT1(LSTM_F3)
+    } else if (P.split == 2) {
+        constexpr int SPLIT_ = 2;
+        LSTM_F3_SPLIT2(LSTM_F3)
+    }
 #undef LSTM_F3
     return cudaErrorInvalidConfiguration;
 }

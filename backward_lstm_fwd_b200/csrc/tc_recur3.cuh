@@ -540,12 +540,15 @@ __host__ __device__ constexpr int fwd3_tmem_cols(int NB, int kcc, int kcx) {
 }
 
 // ring_h: kcc chunks of h_{t-1} (NB rows x 64 K); ring_x: kcx chunks of x_t;
-// recv / xbuf / send as in the cluster forward kernel (send aliases ring_h,
-// idle between a step's last MMA and the next step's h loads, when it is
-// large enough)
+// recv / xbuf / send as in the cluster forward kernel.  One batch stream
+// (SPLIT = 1): send aliases ring_h, idle between a step's last MMA and the
+// next step's h loads, when it is large enough.  Two interleaved streams
+// (SPLIT = 2): the next virtual step's h loads and MMAs overlap this one's
+// exchange, so send has a place of its own, and recv and send are
+// double-buffered by virtual step.
 struct Fwd3Smem {
     int ring_h, ring_x, recv, xbuf, send, bars, total;
-    __host__ __device__ Fwd3Smem(int kcc, int kcx, int NB, int KS) {
+    __host__ __device__ Fwd3Smem(int kcc, int kcx, int NB, int KS, int SPLIT = 1) {
         const int NBc = NB / KS;
         const int hbytes = kcc * NB * 128, xbytes = kcx * NB * 128;
         const int part_bytes = (KS - 1) * NBc * rec2::F_ROWS * 4;
@@ -553,15 +556,26 @@ struct Fwd3Smem {
         ring_h = 0;
         ring_x = hbytes;
         recv = ring_x + xbytes;
-        xbuf = recv + part_bytes;
-        send = hbytes >= part_bytes ? ring_h : xbuf + xbuf_bytes;
-        bars = send == ring_h ? xbuf + xbuf_bytes : send + part_bytes;
+        if (SPLIT == 1) {
+            xbuf = recv + part_bytes;
+            send = hbytes >= part_bytes ? ring_h : xbuf + xbuf_bytes;
+            bars = send == ring_h ? xbuf + xbuf_bytes : send + part_bytes;
+        } else {
+            xbuf = recv + 2 * part_bytes;
+            send = xbuf + xbuf_bytes;
+            bars = send + 2 * part_bytes;
+        }
         bars = (bars + 15) & ~15;
         total = bars + F3_BAR_BYTES;
     }
 };
 
-template <class E, int NB, int KS, bool MASKED>
+// SPLIT = 2: the cluster's batch group of 2 NB rows is two independent
+// streams of NB rows, processed in alternating virtual steps v = 2t + half
+// (each with its own group barrier), so that one stream's h-part MMAs run
+// while the other's partial sums cross DSMEM.  NB is the batch width of one
+// virtual step.
+template <class E, int NB, int KS, bool MASKED, int SPLIT = 1>
 __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params<E> p) {
     using rec2::F_ROWS;
     using rec2::F_UNITS;
@@ -571,15 +585,17 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     constexpr int NP = (NBc + 7) / 8;  // (unit, batch) pairs per epilogue thread
     constexpr int VW = NBh >= 4 ? 4 : 2;  // floats per staged vector / receive chunk
     static_assert(NBc >= 4 && NBc % 4 == 0 && NBc <= 32, "columns per CTA");
+    static_assert(SPLIT == 1 || SPLIT == 2, "one or two batch streams");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int kcc = p.kcc, kcx = p.kcx;
-    const Fwd3Smem L(kcc, kcx, NB, KS);
+    const Fwd3Smem L(kcc, kcx, NB, KS, SPLIT);
     uint8_t *ring_h = smem + L.ring_h;
     uint8_t *ring_x = smem + L.ring_x;
-    float *recv = (float *)(smem + L.recv);  // [KS-1 sources][NBc/VW chunks][128 rows][VW]
+    // recv / send: [SPLIT buffers][KS-1 partners][NBc/VW chunks][128 rows][VW]
+    float *recv = (float *)(smem + L.recv);
     float *xbuf = (float *)(smem + L.xbuf);  // [4 gates][NBc][32 units]
-    float *send = (float *)(smem + L.send);  // [KS-1 destinations][NBc/VW][128 rows][VW]
+    float *send = (float *)(smem + L.send);
     uint64_t *bars = (uint64_t *)(smem + L.bars);
     uint64_t *h_full = bars;
     uint64_t *h_empty = bars + F3_MAXC;
@@ -588,22 +604,23 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     uint64_t *w_ready = bars + 4 * F3_MAXC;  // W_h and W_x slices written to TMEM
     uint64_t *mma_done = w_ready + 1;        // [2]: accumulator complete
     uint64_t *d_free = w_ready + 3;          // [2]: accumulator read out by the epilogue
-    uint64_t *recv_full = w_ready + 5;
-    uint32_t *tmem_slot = (uint32_t *)(w_ready + 6);
-    volatile int *abort_flag = (volatile int *)(w_ready + 7);
+    uint64_t *recv_full = w_ready + 5;       // [SPLIT]
+    uint32_t *tmem_slot = (uint32_t *)(w_ready + 7);
+    volatile int *abort_flag = (volatile int *)(w_ready + 8);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t kpart = tc::cluster_rank();
     const int cid = blockIdx.x / KS;
     const int rs = cid % p.R, gi = cid / p.R;
-    const int u0 = rs * F_UNITS, b0 = gi * NB;
+    const int u0 = rs * F_UNITS, b0 = gi * NB * SPLIT;  // the group's first batch row
     const int H = p.H, B = p.B, T = p.T, I = p.I;
     const int kbase = (int)kpart * kcc * 64;  // this CTA's K range of W_h / h
     const int xbase = (int)kpart * kcx * 64;  // and of W_x / x
     // time of recurrence step s (step s reads the state step s-1 left)
     auto tau = [&](int s) { return p.reverse ? T - 1 - s : s; };
     const uint32_t WH_COL = 2 * NB, WX_COL = 2 * NB + 32 * kcc;
-    unsigned int *ctr = &p.ctrl->bar[gi];
+    unsigned int *ctr = &p.ctrl->bar[gi * SPLIT];  // + stream: one counter per stream
+    const int V = T * SPLIT;                        // virtual steps
     const unsigned int group_ctas = (unsigned)(p.R * KS);
     constexpr uint32_t TMEM_COLS = 512;
 
@@ -621,7 +638,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         tc::mbar_init(&mma_done[1], 1);
         tc::mbar_init(&d_free[0], 1);
         tc::mbar_init(&d_free[1], 1);
-        tc::mbar_init(recv_full, 1);  // one local arrival (with the expected bytes) per step
+        // one local arrival (with the expected bytes) per (virtual) step
+        for (int i = 0; i < SPLIT; ++i) tc::mbar_init(&recv_full[i], 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -643,13 +661,13 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             int rounds_h = 0, part_h = 0, rounds_x = 0, part_x = 0;
             uint32_t phh = 0, phx = 0;
             bool aborted = false;
-            auto load_x = [&](int t) -> bool {
+            auto load_x = [&](int v) -> bool {  // x rows of virtual step v
+                const int row = tau(v / SPLIT) * B + b0 + (v % SPLIT) * NB;
                 for (int c = 0; c < kcx; ++c) {
                     if (!tc::mbar_wait(&x_empty[c], phx ^ 1, p.ctrl, abort_flag, 0x702, p.wait_ns))
                         return false;
                     tc::mbar_arrive_expect_tx(&x_full[c], CHUNK);
-                    tc::tma_load_2d(ring_x + c * CHUNK, &p.map_x, &x_full[c], xbase + 64 * c,
-                                    tau(t) * B + b0);
+                    tc::tma_load_2d(ring_x + c * CHUNK, &p.map_x, &x_full[c], xbase + 64 * c, row);
                     part_x = c + 1;
                 }
                 phx ^= 1;
@@ -658,10 +676,11 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 return true;
             };
             aborted = !load_x(0);
-            for (int t = 0; t < T && !aborted; ++t) {
+            for (int v = 0; v < V && !aborted; ++v) {
+                const int t = v / SPLIT, bh = b0 + (v % SPLIT) * NB;  // step, first row
                 if (t > 0) {
-                    if (!rec::wait_counter(ctr, group_ctas * (unsigned)t, p.ctrl, abort_flag, 0x701,
-                                           p.wait_ns)) {
+                    if (!rec::wait_counter(ctr + v % SPLIT, group_ctas * (unsigned)t, p.ctrl,
+                                           abort_flag, 0x701, p.wait_ns)) {
                         aborted = true;
                         break;
                     }
@@ -671,7 +690,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 }
                 if (t > 0 || p.has_h0) {
                     const CUtensorMap *m = t > 0 ? &p.map_y : &p.map_h0;
-                    const int row0 = t > 0 ? tau(t - 1) * B + b0 : b0;
+                    const int row0 = t > 0 ? tau(t - 1) * B + bh : bh;
                     for (int c = 0; c < kcc && !aborted; ++c) {
                         if (!tc::mbar_wait(&h_empty[c], phh ^ 1, p.ctrl, abort_flag, 0x703,
                                            p.wait_ns)) {
@@ -687,8 +706,8 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                     ++rounds_h;
                     part_h = 0;
                 }
-                // x_{t+1} does not depend on the group: issue it now
-                if (t + 1 < T && !load_x(t + 1)) aborted = true;
+                // the next virtual step's x does not depend on the group: issue it now
+                if (v + 1 < V && !load_x(v + 1)) aborted = true;
             }
             if (aborted) {  // let every issued copy land before the CTA can exit
                 for (int c = 0; c < kcc; ++c) {
@@ -738,10 +757,10 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 return true;
             };
             ok = ok && x_part(0);
-            for (int t = 0; ok && t < T; ++t) {
-                const int acc = t & 1;
+            for (int v = 0; ok && v < V; ++v) {
+                const int acc = v & 1;
                 const uint32_t d = tmem_base + acc * NB;
-                if (t > 0 || p.has_h0) {
+                if (v >= SPLIT || p.has_h0) {  // h_{t-1} is zero at t = 0 without h0
                     for (int c = 0; c < kcc; ++c) {
                         if (!tc::mbar_wait(&h_full[c], phh, p.ctrl, abort_flag, 0x707, p.wait_ns)) {
                             ok = false;
@@ -760,7 +779,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                     phh ^= 1;
                 }
                 tc::mma_commit(&mma_done[acc]);
-                if (t + 1 < T) ok = x_part(t + 1);
+                if (v + 1 < V) ok = x_part(v + 1);
             }
         }
     } else {
@@ -796,40 +815,54 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             tc::tc_fence_before();
             tc::mbar_arrive(w_ready);
         }
-        const int bc0 = b0 + (int)kpart * NBc;  // first batch row finalised here
+        // first batch row finalised here in virtual steps of stream `half`
+        auto col0 = [&](int half) { return b0 + half * NB + (int)kpart * NBc; };
         constexpr uint32_t PART_BYTES = NBc * F_ROWS * 4;  // one partner's partial tile
+        constexpr int BUF_FLOATS = (KS - 1) * (int)PART_BYTES / 4;  // one recv / send buffer
         // position of destination d among this CTA's partners (its send block),
         // and of this CTA among d's sources (its receive slot at d)
         auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
         auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
-        // pointwise pairs of this thread: pair index et + 256 k -> unit, column
-        float c[NP], bias[4][NP];
-        float hprev[NP], mk[NP];  // MASKED: h_{t-1} of each pair, and step t's mask
+        // pointwise pairs of this thread: pair index et + 256 k -> unit, column.
+        // c / hprev: the state of the stream of the current virtual step; with
+        // two streams, c2 / hprev2 hold the other one's, swapped every step.
+        float c[NP], c2[NP], bias[4][NP];
+        float hprev[NP], hprev2[NP], mk[NP];  // MASKED: h_{t-1} of each pair, the step's mask
         auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
         auto pair_col = [&](int k) { return (et + F_EPI_THREADS * k) >> 5; };
 #pragma unroll
         for (int k = 0; k < NP; ++k) {
-            const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
-            const bool v = n < NBc && b < B;
-            c[k] = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
-            if (MASKED) hprev[k] = (p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
+            const int n = pair_col(k), j = u0 + pair_unit(k);
+#pragma unroll
+            for (int half = 0; half < SPLIT; ++half) {
+                const int b = col0(half) + n;
+                const bool v = n < NBc && b < B;
+                const float cv = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
+                const float hv = (MASKED && p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
+                if (half == 0) { c[k] = cv; hprev[k] = hv; }
+                else { c2[k] = cv; hprev2[k] = hv; }
+            }
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 bias[g][k] = p.bias ? to_f(p.bias[g * H + j]) : 0.f;
         }
-        auto load_mask = [&](int s) {  // mask of step s (time tau(s))
-            const int t = tau(s);
+        auto load_mask = [&](int v) {  // mask of virtual step v (time tau(v / SPLIT))
+            const int t = tau(v / SPLIT), bc = col0(v % SPLIT);
 #pragma unroll
             for (int k = 0; k < NP; ++k) {
-                const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+                const int n = pair_col(k), b = bc + n, j = u0 + pair_unit(k);
                 mk[k] = (n < NBc && b < B)
                             ? to_f(p.mask[((long long)t * B + b) * H + j]) : 0.f;
             }
         };
         if (MASKED) load_mask(0);
-        uint32_t dph[2] = {0, 0}, rph = 0;
-        for (int t = 0; t < T; ++t) {
-            const int acc = t & 1;
+        uint32_t dph[2] = {0, 0}, rph[2] = {0, 0};
+        for (int v = 0; v < V; ++v) {
+            const int acc = v & 1, t = v / SPLIT, half = v % SPLIT;
+            const int bc0 = col0(half);
+            const int buf = SPLIT == 2 ? (v & 1) : 0;
+            float *rv = recv + buf * BUF_FLOATS;  // this virtual step's receive block
+            float *sd = send + buf * BUF_FLOATS;  // and staging block
             const bool w = tc::mbar_wait(&mma_done[acc], dph[acc], p.ctrl, abort_flag, 0x708,
                                          p.wait_ns);
             if (!rec::epi_vote_all_n<F_EPI_THREADS>(w)) break;
@@ -838,57 +871,57 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
             float own[NBh];
 #pragma unroll
             for (int d = 0; d < KS; ++d) {
-                uint32_t v[NBh];
+                uint32_t tv[NBh];
                 rec2::tmem_ld_cols<NBh>(
-                    tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + d * NBc + hh * NBh, v);
+                    tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + d * NBc + hh * NBh, tv);
                 tc::tmem_ld_wait();
                 if (d == (int)kpart) {
 #pragma unroll
-                    for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(v[n]);
+                    for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(tv[n]);
                 } else {
-                    float *blk = send + dst_pos(d) * (PART_BYTES / 4);
+                    float *blk = sd + dst_pos(d) * (PART_BYTES / 4);
 #pragma unroll
                     for (int k = 0; k < NBh / VW; ++k) {
                         const int ch = hh * (NBh / VW) + k;
                         float *a = blk + (ch * F_ROWS + mrow) * VW;
                         if constexpr (VW == 4)
                             *reinterpret_cast<float4 *>(a) =
-                                make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                            __uint_as_float(v[4 * k + 2]),
-                                            __uint_as_float(v[4 * k + 3]));
+                                make_float4(__uint_as_float(tv[4 * k]), __uint_as_float(tv[4 * k + 1]),
+                                            __uint_as_float(tv[4 * k + 2]),
+                                            __uint_as_float(tv[4 * k + 3]));
                         else
                             *reinterpret_cast<float2 *>(a) =
-                                make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                                make_float2(__uint_as_float(tv[2 * k]), __uint_as_float(tv[2 * k + 1]));
                     }
                 }
             }
             tc::tc_fence_before();
             if (KS > 1) tc::fence_proxy_async_smem();  // staged partials -> bulk copies
             rec::named_bar(1, F_EPI_THREADS);
-            // accumulator read out: the MMA thread may start step t + 2's x-part in it
+            // accumulator read out: the MMA thread may start virtual step v + 2's x-part in it
             if (et == 0) tc::mbar_arrive(&d_free[acc]);
             if (KS > 1) {
                 if (et == 0) {
-                    tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
-                    const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(recv_full);
+                    tc::mbar_arrive_expect_tx(&recv_full[buf], (KS - 1) * PART_BYTES);
+                    const uint32_t recv_lo = tc::smem_u32(rv), bar_lo = tc::smem_u32(&recv_full[buf]);
                     // rank kpart + s first: each CTA receives from one sender at a time
 #pragma unroll
                     for (int s = 1; s < KS; ++s) {
                         const int d = ((int)kpart + s) % KS;
                         tc::bulk_copy_to_peer(
                             tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
-                            send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                            sd + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
                             tc::map_rank(bar_lo, (uint32_t)d));
                     }
                     tc::bulk_commit();
                 }
-                const bool w2 = tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x709,
-                                                      p.wait_ns);
+                const bool w2 = tc::mbar_wait_cluster(&recv_full[buf], rph[buf], p.ctrl, abort_flag,
+                                                      0x709, p.wait_ns);
                 if (!rec::epi_vote_all_n<F_EPI_THREADS>(w2)) break;
-                rph ^= 1;
+                rph[buf] ^= 1;
 #pragma unroll
                 for (int sl = 0; sl < KS - 1; ++sl) {
-                    const float *src = recv + sl * F_ROWS * NBc;
+                    const float *src = rv + sl * F_ROWS * NBc;
 #pragma unroll
                     for (int k = 0; k < NBh / VW; ++k) {
                         const int ch = hh * (NBh / VW) + k;
@@ -946,12 +979,15 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                     }
                 }
             }
+            // two streams: the other staging block (virtual step v - 1) must be
+            // read out before any thread stages step v + 1 into it
+            if (SPLIT == 2 && KS > 1 && et == 0) tc::bulk_wait_read_but_one();
             rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
             if (et == 0) {
-                // the staging block must be read out before this CTA's arrival
-                // lets the next step's TMA refill ring_h
-                if (KS > 1) tc::bulk_wait_read_all();
-                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+                // one stream: the staging block must be read out before this
+                // CTA's arrival lets the next step's TMA refill ring_h
+                if (SPLIT == 1 && KS > 1) tc::bulk_wait_read_all();
+                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr + half, 1u);
             }
             // saved state for the backward pass, outside the writes the
             // arrival's release has to cover
@@ -968,7 +1004,15 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
                 g4[gb * H] = from_f<E>(gsave[2][k]);
                 g4[3 * H] = from_f<E>(gsave[3][k]);
             }
-            if (MASKED && t + 1 < T) load_mask(t + 1);
+            if (MASKED && v + 1 < V) load_mask(v + 1);
+            if (SPLIT == 2) {  // the next virtual step belongs to the other stream
+#pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    const float tc_ = c[k], th = hprev[k];
+                    c[k] = c2[k]; c2[k] = tc_;
+                    hprev[k] = hprev2[k]; hprev2[k] = th;
+                }
+            }
         }
         if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
     }

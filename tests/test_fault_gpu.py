@@ -3,8 +3,9 @@ CTA 0 never signals its step barrier must give up after its bounded wait,
 record LSTM_ERR_TIMEOUT in the workspace status word (read by lstm_status), and
 leave the context usable -- the next normal call succeeds and matches the
 oracle.  Covered for the K-resident kernels (H = 64), the cluster kernels
-(H = 256: forward clusters of 4, backward clusters of 8) and the backward
-cluster kernel with the weights in tensor memory (H = 512)."""
+(H = 256: forward clusters of 4, backward clusters of 8), the backward
+cluster kernel with the weights in tensor memory (H = 512), and the fused
+forward with one and with two batch streams per cluster."""
 import pytest
 import torch
 
@@ -16,13 +17,15 @@ from tests.parity_util import assert_within, compare, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H,T", [(64, 6), (256, 6), (512, 6), (512, 40)])
-def test_missing_arrival_times_out_and_recovers(H, T, cuda_device):
-    """T = 40 runs the backward in reverse-time chunks with dW / dx beside them."""
+@pytest.mark.parametrize("H,T,B", [(64, 6, 32), (256, 6, 32), (512, 6, 32), (512, 40, 32),
+                                   (512, 6, 128)])
+def test_missing_arrival_times_out_and_recovers(H, T, B, cuda_device):
+    """T = 40 runs the backward in reverse-time chunks with dW / dx beside them;
+    B = 128 runs the forward with two interleaved batch streams per cluster."""
     lbuild.build()
-    w = synth.custom(T, 32, 64, H, "bf16", seed=11)
+    w = synth.custom(T, B, 64, H, "bf16", seed=11)
     inp = {k: v.to(cuda_device) for k, v in synth.make_inputs(w).items()}
-    B, I = w.B, w.I
+    I = w.I
     st = L.State(T, B, I, H, torch.bfloat16, cuda_device)
     gr = L.Grads(T, B, I, H, cuda_device)
     wsf = L.empty_workspace(L.fwd_workspace_size(st.dims), cuda_device)
