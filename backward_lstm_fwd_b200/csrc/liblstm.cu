@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstdlib>
 #include <mutex>
 #include <vector>
@@ -304,6 +305,26 @@ int bwd_chunks(const lstm_dims *d) {
     const char *e = getenv("LSTM_BWD_CHUNKS");
     int n = e ? atoi(e) : (d->T >= 32 ? std::min(8, d->T / 16) : 1);
     return std::max(1, std::min(std::min(n, kMaxChunks), d->T));
+}
+
+// First epilogue iteration of chunk c of nch over T steps (c = nch gives T).
+// Chunk sizes shrink geometrically (ratio r = 0.8; LSTM_BWD_CHUNK_RATIO
+// overrides it, 1 = equal chunks): the dW / dx GEMM of a chunk runs beside the
+// next, smaller one, and the GEMM of the last chunk, which runs alone, is the
+// smallest.  Every chunk keeps at least one step.
+int chunk_bound(int T, int nch, int c) {
+    static double r = -1.0;
+    if (r < 0.0) {
+        const char *e = getenv("LSTM_BWD_CHUNK_RATIO");
+        r = e ? atof(e) : 0.8;
+        if (!(r > 0.0 && r <= 1.0)) r = 0.8;
+    }
+    if (c <= 0) return 0;
+    if (c >= nch) return T;
+    const double f = r == 1.0 ? (double)c / nch : (1.0 - pow(r, c)) / (1.0 - pow(r, nch));
+    int b = (int)(T * f + 0.5);
+    b = std::max(b, c);               // at least one step per earlier chunk
+    return std::min(b, T - (nch - c));  // and per later one
 }
 
 // ------------------------------------------- persistent recurrence (bf16)
@@ -1005,7 +1026,7 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         prof::Phase ph(LSTM_PHASE_BWD_RECUR, A.rec);
         if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
         for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
-            const int i0 = (int)((long long)T * c / nch), i1 = (int)((long long)T * (c + 1) / nch);
+            const int i0 = chunk_bound(T, nch, c), i1 = chunk_bound(T, nch, c + 1);
             rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
                                 dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
             if (rc != LSTM_OK) break;
