@@ -543,9 +543,8 @@ __host__ __device__ constexpr int fwd3_tmem_cols(int NB, int kcc, int kcx) {
 // recv / xbuf / send as in the cluster forward kernel.  One batch stream
 // (SPLIT = 1): send aliases ring_h, idle between a step's last MMA and the
 // next step's h loads, when it is large enough.  Two interleaved streams
-// (SPLIT = 2): the next virtual step's h loads and MMAs overlap this one's
-// exchange, so send has a place of its own, and recv and send are
-// double-buffered by virtual step.
+// (SPLIT = 2): one stream's h loads and MMAs overlap the other's exchange, so
+// send has a place of its own, and recv, xbuf and send are one per stream.
 struct Fwd3Smem {
     int ring_h, ring_x, recv, xbuf, send, bars, total;
     __host__ __device__ Fwd3Smem(int kcc, int kcx, int NB, int KS, int SPLIT = 1) {
@@ -561,8 +560,8 @@ struct Fwd3Smem {
             send = hbytes >= part_bytes ? ring_h : xbuf + xbuf_bytes;
             bars = send == ring_h ? xbuf + xbuf_bytes : send + part_bytes;
         } else {
-            xbuf = recv + 2 * part_bytes;
-            send = xbuf + xbuf_bytes;
+            xbuf = recv + 2 * part_bytes;  // one gate-exchange block per stream
+            send = xbuf + 2 * xbuf_bytes;
             bars = send + 2 * part_bytes;
         }
         bars = (bars + 15) & ~15;
@@ -570,11 +569,26 @@ struct Fwd3Smem {
     }
 };
 
+// AND of `v` over the `n` threads that use named barrier `id`
+__device__ __forceinline__ bool vote_all(bool v, int id, int n) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
 // SPLIT = 2: the cluster's batch group of 2 NB rows is two independent
 // streams of NB rows, processed in alternating virtual steps v = 2t + half
 // (each with its own group barrier), so that one stream's h-part MMAs run
 // while the other's partial sums cross DSMEM.  NB is the batch width of one
-// virtual step.
+// virtual step, and each stream has an epilogue warpgroup of its own, so that
+// the two streams' epilogues also overlap each other.
 template <class E, int NB, int KS, bool MASKED, int SPLIT = 1>
 __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_constant__ Fwd3Params<E> p) {
     using rec2::F_ROWS;
@@ -823,198 +837,355 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         // and of this CTA among d's sources (its receive slot at d)
         auto dst_pos = [&](int d) { return d < (int)kpart ? d : d - 1; };
         auto src_slot = [&](int d) { return (int)kpart < d ? (int)kpart : (int)kpart - 1; };
-        // pointwise pairs of this thread: pair index et + 256 k -> unit, column.
-        // c / hprev: the state of the stream of the current virtual step; with
-        // two streams, c2 / hprev2 hold the other one's, swapped every step.
-        float c[NP], c2[NP], bias[4][NP];
-        float hprev[NP], hprev2[NP], mk[NP];  // MASKED: h_{t-1} of each pair, the step's mask
-        auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
-        auto pair_col = [&](int k) { return (et + F_EPI_THREADS * k) >> 5; };
+        if constexpr (SPLIT == 2) {
+            // One epilogue warpgroup per stream (warps 2-5: stream 0, 6-9:
+            // stream 1), each with one warp per TMEM lane quarter, its own
+            // named barriers, receive / staging / gate-exchange blocks and
+            // state: while one stream waits for its partials or its group
+            // barrier, the other's read-out and pointwise work proceed.
+            constexpr int WG = F_EPI_THREADS / 2;
+            constexpr int NP2 = NBc * F_UNITS / WG;  // (unit, column) pairs per thread
+            static_assert(NBc * F_UNITS % WG == 0, "pairs per warpgroup thread");
+            const int sw = hh, wt = et - sw * WG;  // stream, thread within the warpgroup
+            const int bar_sync = 1 + 2 * sw, bar_vote = 2 + 2 * sw;
+            const int bc0 = col0(sw);
+            float *rv = recv + sw * BUF_FLOATS, *sd = send + sw * BUF_FLOATS;
+            float *xb = xbuf + sw * (4 * NBc * F_UNITS);  // [4 gates][NBc][32 units]
+            uint64_t *rf = &recv_full[sw];
+            float c[NP2], hprev[NP2], mk[NP2], bias[4][NP2];
+            auto pair_unit = [&](int k) { return (wt + WG * k) & 31; };
+            auto pair_col = [&](int k) { return (wt + WG * k) >> 5; };
 #pragma unroll
-        for (int k = 0; k < NP; ++k) {
-            const int n = pair_col(k), j = u0 + pair_unit(k);
+            for (int k = 0; k < NP2; ++k) {
+                const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+                const bool v = b < B;
+                c[k] = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
+                hprev[k] = (MASKED && p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
 #pragma unroll
-            for (int half = 0; half < SPLIT; ++half) {
-                const int b = col0(half) + n;
-                const bool v = n < NBc && b < B;
-                const float cv = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
-                const float hv = (MASKED && p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
-                if (half == 0) { c[k] = cv; hprev[k] = hv; }
-                else { c2[k] = cv; hprev2[k] = hv; }
+                for (int g = 0; g < 4; ++g)
+                    bias[g][k] = p.bias ? to_f(p.bias[g * H + j]) : 0.f;
             }
+            auto load_mask = [&](int t) {  // this stream's mask of step t (time tau(t))
+                const int tt = tau(t);
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-                bias[g][k] = p.bias ? to_f(p.bias[g * H + j]) : 0.f;
-        }
-        auto load_mask = [&](int v) {  // mask of virtual step v (time tau(v / SPLIT))
-            const int t = tau(v / SPLIT), bc = col0(v % SPLIT);
-#pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const int n = pair_col(k), b = bc + n, j = u0 + pair_unit(k);
-                mk[k] = (n < NBc && b < B)
-                            ? to_f(p.mask[((long long)t * B + b) * H + j]) : 0.f;
-            }
-        };
-        if (MASKED) load_mask(0);
-        uint32_t dph[2] = {0, 0}, rph[2] = {0, 0};
-        for (int v = 0; v < V; ++v) {
-            const int acc = v & 1, t = v / SPLIT, half = v % SPLIT;
-            const int bc0 = col0(half);
-            const int buf = SPLIT == 2 ? (v & 1) : 0;
-            float *rv = recv + buf * BUF_FLOATS;  // this virtual step's receive block
-            float *sd = send + buf * BUF_FLOATS;  // and staging block
-            const bool w = tc::mbar_wait(&mma_done[acc], dph[acc], p.ctrl, abort_flag, 0x708,
-                                         p.wait_ns);
-            if (!rec::epi_vote_all_n<F_EPI_THREADS>(w)) break;
-            dph[acc] ^= 1;
-            tc::tc_fence_after();
-            float own[NBh];
-#pragma unroll
-            for (int d = 0; d < KS; ++d) {
-                uint32_t tv[NBh];
-                rec2::tmem_ld_cols<NBh>(
-                    tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + d * NBc + hh * NBh, tv);
-                tc::tmem_ld_wait();
-                if (d == (int)kpart) {
-#pragma unroll
-                    for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(tv[n]);
-                } else {
-                    float *blk = sd + dst_pos(d) * (PART_BYTES / 4);
-#pragma unroll
-                    for (int k = 0; k < NBh / VW; ++k) {
-                        const int ch = hh * (NBh / VW) + k;
-                        float *a = blk + (ch * F_ROWS + mrow) * VW;
-                        if constexpr (VW == 4)
-                            *reinterpret_cast<float4 *>(a) =
-                                make_float4(__uint_as_float(tv[4 * k]), __uint_as_float(tv[4 * k + 1]),
-                                            __uint_as_float(tv[4 * k + 2]),
-                                            __uint_as_float(tv[4 * k + 3]));
-                        else
-                            *reinterpret_cast<float2 *>(a) =
-                                make_float2(__uint_as_float(tv[2 * k]), __uint_as_float(tv[2 * k + 1]));
-                    }
+                for (int k = 0; k < NP2; ++k) {
+                    const int b = bc0 + pair_col(k), j = u0 + pair_unit(k);
+                    mk[k] = b < B ? to_f(p.mask[((long long)tt * B + b) * H + j]) : 0.f;
                 }
-            }
-            tc::tc_fence_before();
-            if (KS > 1) tc::fence_proxy_async_smem();  // staged partials -> bulk copies
-            rec::named_bar(1, F_EPI_THREADS);
-            // accumulator read out: the MMA thread may start virtual step v + 2's x-part in it
-            if (et == 0) tc::mbar_arrive(&d_free[acc]);
-            if (KS > 1) {
-                if (et == 0) {
-                    tc::mbar_arrive_expect_tx(&recv_full[buf], (KS - 1) * PART_BYTES);
-                    const uint32_t recv_lo = tc::smem_u32(rv), bar_lo = tc::smem_u32(&recv_full[buf]);
-                    // rank kpart + s first: each CTA receives from one sender at a time
+            };
+            if (MASKED) load_mask(0);
+            uint32_t dph = 0, rph = 0;
+            for (int t = 0; t < T; ++t) {
+                const bool w = tc::mbar_wait(&mma_done[sw], dph, p.ctrl, abort_flag, 0x708,
+                                             p.wait_ns);
+                if (!vote_all(w, bar_vote, WG)) break;
+                dph ^= 1;
+                tc::tc_fence_after();
+                float own[NBc];
 #pragma unroll
-                    for (int s = 1; s < KS; ++s) {
-                        const int d = ((int)kpart + s) % KS;
-                        tc::bulk_copy_to_peer(
-                            tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
-                            sd + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
-                            tc::map_rank(bar_lo, (uint32_t)d));
-                    }
-                    tc::bulk_commit();
-                }
-                const bool w2 = tc::mbar_wait_cluster(&recv_full[buf], rph[buf], p.ctrl, abort_flag,
-                                                      0x709, p.wait_ns);
-                if (!rec::epi_vote_all_n<F_EPI_THREADS>(w2)) break;
-                rph[buf] ^= 1;
+                for (int d = 0; d < KS; ++d) {
 #pragma unroll
-                for (int sl = 0; sl < KS - 1; ++sl) {
-                    const float *src = rv + sl * F_ROWS * NBc;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t tv[NBh];
+                        rec2::tmem_ld_cols<NBh>(tmem_base + ((uint32_t)(32 * q) << 16) + sw * NB +
+                                                    d * NBc + h2 * NBh,
+                                                tv);
+                        tc::tmem_ld_wait();
+                        if (d == (int)kpart) {
 #pragma unroll
-                    for (int k = 0; k < NBh / VW; ++k) {
-                        const int ch = hh * (NBh / VW) + k;
-                        if constexpr (VW == 4) {
-                            const float4 x = *reinterpret_cast<const float4 *>(src + (ch * F_ROWS + mrow) * 4);
-                            own[4 * k] += x.x;
-                            own[4 * k + 1] += x.y;
-                            own[4 * k + 2] += x.z;
-                            own[4 * k + 3] += x.w;
+                            for (int n = 0; n < NBh; ++n) own[h2 * NBh + n] = __uint_as_float(tv[n]);
                         } else {
-                            const float2 x = *reinterpret_cast<const float2 *>(src + (ch * F_ROWS + mrow) * 2);
-                            own[2 * k] += x.x;
-                            own[2 * k + 1] += x.y;
+                            float *blk = sd + dst_pos(d) * (PART_BYTES / 4);
+#pragma unroll
+                            for (int k = 0; k < NBh / VW; ++k) {
+                                const int ch = h2 * (NBh / VW) + k;
+                                float *a = blk + (ch * F_ROWS + mrow) * VW;
+                                if constexpr (VW == 4)
+                                    *reinterpret_cast<float4 *>(a) = make_float4(
+                                        __uint_as_float(tv[4 * k]), __uint_as_float(tv[4 * k + 1]),
+                                        __uint_as_float(tv[4 * k + 2]), __uint_as_float(tv[4 * k + 3]));
+                                else
+                                    *reinterpret_cast<float2 *>(a) = make_float2(
+                                        __uint_as_float(tv[2 * k]), __uint_as_float(tv[2 * k + 1]));
+                            }
                         }
                     }
                 }
-            }
+                tc::tc_fence_before();
+                if (KS > 1) tc::fence_proxy_async_smem();  // staged partials -> bulk copies
+                rec::named_bar(bar_sync, WG);
+                // accumulator read out: the MMA thread may start this stream's next x-part in it
+                if (wt == 0) tc::mbar_arrive(&d_free[sw]);
+                if (KS > 1) {
+                    if (wt == 0) {
+                        tc::mbar_arrive_expect_tx(rf, (KS - 1) * PART_BYTES);
+                        const uint32_t recv_lo = tc::smem_u32(rv), bar_lo = tc::smem_u32(rf);
 #pragma unroll
-            for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
-            rec::named_bar(1, F_EPI_THREADS);
-            const int tt = tau(t);  // time of this step
-            // row blocks of the forget gate and the candidate (gate_order)
-            const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
-            E *yt = p.y + (long long)tt * B * H;
-            E *gt = p.gates + (long long)tt * B * 4 * H;
-            float *ct = p.cells + (long long)tt * B * H;
-            float gsave[4][NP];
+                        for (int s = 1; s < KS; ++s) {
+                            const int d = ((int)kpart + s) % KS;
+                            tc::bulk_copy_to_peer(
+                                tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                                sd + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                                tc::map_rank(bar_lo, (uint32_t)d));
+                        }
+                        tc::bulk_commit();
+                    }
+                    const bool w2 = tc::mbar_wait_cluster(rf, rph, p.ctrl, abort_flag, 0x709,
+                                                          p.wait_ns);
+                    if (!vote_all(w2, bar_vote, WG)) break;
+                    rph ^= 1;
 #pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const int n = pair_col(k), uu = pair_unit(k);
-                if (n >= NBc) continue;
-                const int b = bc0 + n, j = u0 + uu;
-                const float bf_ = fb == 1 ? bias[1][k] : bias[2][k];
-                const float bg_ = fb == 1 ? bias[2][k] : bias[1][k];
-                const float ig = rec::sigmoid_fast(xbuf[(0 * NBc + n) * F_UNITS + uu] + bias[0][k]);
-                const float fg = rec::sigmoid_fast(xbuf[(fb * NBc + n) * F_UNITS + uu] + bf_);
-                const float gg = rec::tanh_fast(xbuf[(gb * NBc + n) * F_UNITS + uu] + bg_);
-                const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
-                const float cn = fg * c[k] + ig * gg;
-                float h = og * rec::tanh_fast(cn);
-                if (MASKED) {  // padding keeps the previous state
-                    c[k] = mk[k] * cn + (1.f - mk[k]) * c[k];
-                    h = mk[k] * h + (1.f - mk[k]) * hprev[k];
-                    hprev[k] = h;
-                } else {
-                    c[k] = cn;
-                }
-                gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
-                if (b < B) {
-                    const long long o = (long long)b * H + j;
-                    yt[o] = from_f<E>(h);  // h_t: what the other CTAs wait for
-                    if (t == T - 1) {
-                        p.hT[o] = from_f<E>(h);
-                        p.cT[o] = c[k];
+                    for (int sl = 0; sl < KS - 1; ++sl) {
+                        const float *src = rv + sl * F_ROWS * NBc;
+#pragma unroll
+                        for (int ch = 0; ch < NBc / VW; ++ch) {
+                            const float *a = src + (ch * F_ROWS + mrow) * VW;
+                            if constexpr (VW == 4) {
+                                const float4 x = *reinterpret_cast<const float4 *>(a);
+                                own[4 * ch] += x.x;
+                                own[4 * ch + 1] += x.y;
+                                own[4 * ch + 2] += x.z;
+                                own[4 * ch + 3] += x.w;
+                            } else {
+                                const float2 x = *reinterpret_cast<const float2 *>(a);
+                                own[2 * ch] += x.x;
+                                own[2 * ch + 1] += x.y;
+                            }
+                        }
                     }
                 }
-            }
-            // two streams: the other staging block (virtual step v - 1) must be
-            // read out before any thread stages step v + 1 into it
-            if (SPLIT == 2 && KS > 1 && et == 0) tc::bulk_wait_read_but_one();
-            rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
-            if (et == 0) {
-                // one stream: the staging block must be read out before this
-                // CTA's arrival lets the next step's TMA refill ring_h
-                if (SPLIT == 1 && KS > 1) tc::bulk_wait_read_all();
-                if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr + half, 1u);
-            }
-            // saved state for the backward pass, outside the writes the
-            // arrival's release has to cover
 #pragma unroll
-            for (int k = 0; k < NP; ++k) {
-                const int n = pair_col(k), uu = pair_unit(k);
-                const int b = bc0 + n, j = u0 + uu;
-                if (n >= NBc || b >= B) continue;
-                ct[(long long)b * H + j] = c[k];
-                E *g4 = gt + (long long)b * 4 * H + j;
-                const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
-                g4[0] = from_f<E>(gsave[0][k]);
-                g4[fb * H] = from_f<E>(gsave[1][k]);
-                g4[gb * H] = from_f<E>(gsave[2][k]);
-                g4[3 * H] = from_f<E>(gsave[3][k]);
-            }
-            if (MASKED && v + 1 < V) load_mask(v + 1);
-            if (SPLIT == 2) {  // the next virtual step belongs to the other stream
+                for (int n = 0; n < NBc; ++n) xb[(q * NBc + n) * F_UNITS + lane] = own[n];
+                rec::named_bar(bar_sync, WG);
+                const int tt = tau(t);  // time of this step
+                const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;  // forget / candidate row blocks
+                E *yt = p.y + (long long)tt * B * H;
+                E *gt = p.gates + (long long)tt * B * 4 * H;
+                float *ct = p.cells + (long long)tt * B * H;
+                float gsave[4][NP2];
 #pragma unroll
-                for (int k = 0; k < NP; ++k) {
-                    const float tc_ = c[k], th = hprev[k];
-                    c[k] = c2[k]; c2[k] = tc_;
-                    hprev[k] = hprev2[k]; hprev2[k] = th;
+                for (int k = 0; k < NP2; ++k) {
+                    const int n = pair_col(k), uu = pair_unit(k);
+                    const int b = bc0 + n, j = u0 + uu;
+                    const float bf_ = fb == 1 ? bias[1][k] : bias[2][k];
+                    const float bg_ = fb == 1 ? bias[2][k] : bias[1][k];
+                    const float ig = rec::sigmoid_fast(xb[(0 * NBc + n) * F_UNITS + uu] + bias[0][k]);
+                    const float fg = rec::sigmoid_fast(xb[(fb * NBc + n) * F_UNITS + uu] + bf_);
+                    const float gg = rec::tanh_fast(xb[(gb * NBc + n) * F_UNITS + uu] + bg_);
+                    const float og = rec::sigmoid_fast(xb[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
+                    const float cn = fg * c[k] + ig * gg;
+                    float h = og * rec::tanh_fast(cn);
+                    if (MASKED) {  // padding keeps the previous state
+                        c[k] = mk[k] * cn + (1.f - mk[k]) * c[k];
+                        h = mk[k] * h + (1.f - mk[k]) * hprev[k];
+                        hprev[k] = h;
+                    } else {
+                        c[k] = cn;
+                    }
+                    gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
+                    if (b < B) {
+                        const long long o = (long long)b * H + j;
+                        yt[o] = from_f<E>(h);  // h_t: what the other CTAs wait for
+                        if (t == T - 1) {
+                            p.hT[o] = from_f<E>(h);
+                            p.cT[o] = c[k];
+                        }
+                    }
                 }
+                // this step's copies must have read the staging block before
+                // the next step stages into it
+                if (KS > 1 && wt == 0) tc::bulk_wait_read_all();
+                rec::named_bar(bar_sync, WG);  // y[t] stored; xb and rv free again
+                if (wt == 0 && (int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr + sw, 1u);
+                // saved state for the backward pass, outside the writes the
+                // arrival's release has to cover
+#pragma unroll
+                for (int k = 0; k < NP2; ++k) {
+                    const int n = pair_col(k), uu = pair_unit(k);
+                    const int b = bc0 + n, j = u0 + uu;
+                    if (b >= B) continue;
+                    ct[(long long)b * H + j] = c[k];
+                    E *g4 = gt + (long long)b * 4 * H + j;
+                    g4[0] = from_f<E>(gsave[0][k]);
+                    g4[fb * H] = from_f<E>(gsave[1][k]);
+                    g4[gb * H] = from_f<E>(gsave[2][k]);
+                    g4[3 * H] = from_f<E>(gsave[3][k]);
+                }
+                if (MASKED && t + 1 < T) load_mask(t + 1);
             }
+            if (wt == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
+        } else {
+            const int bc0 = col0(0);  // first batch row finalised here
+            // pointwise pairs of this thread: pair index et + 256 k -> unit, column
+            float c[NP], bias[4][NP];
+            float hprev[NP], mk[NP];  // MASKED: h_{t-1} of each pair, and step t's mask
+            auto pair_unit = [&](int k) { return (et + F_EPI_THREADS * k) & 31; };
+            auto pair_col = [&](int k) { return (et + F_EPI_THREADS * k) >> 5; };
+    #pragma unroll
+            for (int k = 0; k < NP; ++k) {
+                const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+                const bool v = n < NBc && b < B;
+                c[k] = (p.c0 && v) ? p.c0[(long long)b * H + j] : 0.f;
+                if (MASKED) hprev[k] = (p.h0 && v) ? to_f(p.h0[(long long)b * H + j]) : 0.f;
+    #pragma unroll
+                for (int g = 0; g < 4; ++g)
+                    bias[g][k] = p.bias ? to_f(p.bias[g * H + j]) : 0.f;
+            }
+            auto load_mask = [&](int s) {  // mask of step s (time tau(s))
+                const int t = tau(s);
+    #pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    const int n = pair_col(k), b = bc0 + n, j = u0 + pair_unit(k);
+                    mk[k] = (n < NBc && b < B)
+                                ? to_f(p.mask[((long long)t * B + b) * H + j]) : 0.f;
+                }
+            };
+            if (MASKED) load_mask(0);
+            uint32_t dph[2] = {0, 0}, rph = 0;
+            for (int t = 0; t < T; ++t) {
+                const int acc = t & 1;
+                const bool w = tc::mbar_wait(&mma_done[acc], dph[acc], p.ctrl, abort_flag, 0x708,
+                                             p.wait_ns);
+                if (!rec::epi_vote_all_n<F_EPI_THREADS>(w)) break;
+                dph[acc] ^= 1;
+                tc::tc_fence_after();
+                float own[NBh];
+    #pragma unroll
+                for (int d = 0; d < KS; ++d) {
+                    uint32_t v[NBh];
+                    rec2::tmem_ld_cols<NBh>(
+                        tmem_base + ((uint32_t)(32 * q) << 16) + acc * NB + d * NBc + hh * NBh, v);
+                    tc::tmem_ld_wait();
+                    if (d == (int)kpart) {
+    #pragma unroll
+                        for (int n = 0; n < NBh; ++n) own[n] = __uint_as_float(v[n]);
+                    } else {
+                        float *blk = send + dst_pos(d) * (PART_BYTES / 4);
+    #pragma unroll
+                        for (int k = 0; k < NBh / VW; ++k) {
+                            const int ch = hh * (NBh / VW) + k;
+                            float *a = blk + (ch * F_ROWS + mrow) * VW;
+                            if constexpr (VW == 4)
+                                *reinterpret_cast<float4 *>(a) =
+                                    make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                                __uint_as_float(v[4 * k + 2]),
+                                                __uint_as_float(v[4 * k + 3]));
+                            else
+                                *reinterpret_cast<float2 *>(a) =
+                                    make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+                        }
+                    }
+                }
+                tc::tc_fence_before();
+                if (KS > 1) tc::fence_proxy_async_smem();  // staged partials -> bulk copies
+                rec::named_bar(1, F_EPI_THREADS);
+                // accumulator read out: the MMA thread may start step t + 2's x-part in it
+                if (et == 0) tc::mbar_arrive(&d_free[acc]);
+                if (KS > 1) {
+                    if (et == 0) {
+                        tc::mbar_arrive_expect_tx(recv_full, (KS - 1) * PART_BYTES);
+                        const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(recv_full);
+                        // rank kpart + s first: each CTA receives from one sender at a time
+    #pragma unroll
+                        for (int s = 1; s < KS; ++s) {
+                            const int d = ((int)kpart + s) % KS;
+                            tc::bulk_copy_to_peer(
+                                tc::map_rank(recv_lo + (uint32_t)src_slot(d) * PART_BYTES, (uint32_t)d),
+                                send + dst_pos(d) * (PART_BYTES / 4), PART_BYTES,
+                                tc::map_rank(bar_lo, (uint32_t)d));
+                        }
+                        tc::bulk_commit();
+                    }
+                    const bool w2 = tc::mbar_wait_cluster(recv_full, rph, p.ctrl, abort_flag, 0x709,
+                                                          p.wait_ns);
+                    if (!rec::epi_vote_all_n<F_EPI_THREADS>(w2)) break;
+                    rph ^= 1;
+    #pragma unroll
+                    for (int sl = 0; sl < KS - 1; ++sl) {
+                        const float *src = recv + sl * F_ROWS * NBc;
+    #pragma unroll
+                        for (int k = 0; k < NBh / VW; ++k) {
+                            const int ch = hh * (NBh / VW) + k;
+                            if constexpr (VW == 4) {
+                                const float4 x = *reinterpret_cast<const float4 *>(src + (ch * F_ROWS + mrow) * 4);
+                                own[4 * k] += x.x;
+                                own[4 * k + 1] += x.y;
+                                own[4 * k + 2] += x.z;
+                                own[4 * k + 3] += x.w;
+                            } else {
+                                const float2 x = *reinterpret_cast<const float2 *>(src + (ch * F_ROWS + mrow) * 2);
+                                own[2 * k] += x.x;
+                                own[2 * k + 1] += x.y;
+                            }
+                        }
+                    }
+                }
+    #pragma unroll
+                for (int n = 0; n < NBh; ++n) xbuf[(q * NBc + hh * NBh + n) * F_UNITS + lane] = own[n];
+                rec::named_bar(1, F_EPI_THREADS);
+                const int tt = tau(t);  // time of this step
+                // row blocks of the forget gate and the candidate (gate_order)
+                const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
+                E *yt = p.y + (long long)tt * B * H;
+                E *gt = p.gates + (long long)tt * B * 4 * H;
+                float *ct = p.cells + (long long)tt * B * H;
+                float gsave[4][NP];
+    #pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    const int n = pair_col(k), uu = pair_unit(k);
+                    if (n >= NBc) continue;
+                    const int b = bc0 + n, j = u0 + uu;
+                    const float bf_ = fb == 1 ? bias[1][k] : bias[2][k];
+                    const float bg_ = fb == 1 ? bias[2][k] : bias[1][k];
+                    const float ig = rec::sigmoid_fast(xbuf[(0 * NBc + n) * F_UNITS + uu] + bias[0][k]);
+                    const float fg = rec::sigmoid_fast(xbuf[(fb * NBc + n) * F_UNITS + uu] + bf_);
+                    const float gg = rec::tanh_fast(xbuf[(gb * NBc + n) * F_UNITS + uu] + bg_);
+                    const float og = rec::sigmoid_fast(xbuf[(3 * NBc + n) * F_UNITS + uu] + bias[3][k]);
+                    const float cn = fg * c[k] + ig * gg;
+                    float h = og * rec::tanh_fast(cn);
+                    if (MASKED) {  // padding keeps the previous state
+                        c[k] = mk[k] * cn + (1.f - mk[k]) * c[k];
+                        h = mk[k] * h + (1.f - mk[k]) * hprev[k];
+                        hprev[k] = h;
+                    } else {
+                        c[k] = cn;
+                    }
+                    gsave[0][k] = ig; gsave[1][k] = fg; gsave[2][k] = gg; gsave[3][k] = og;
+                    if (b < B) {
+                        const long long o = (long long)b * H + j;
+                        yt[o] = from_f<E>(h);  // h_t: what the other CTAs wait for
+                        if (t == T - 1) {
+                            p.hT[o] = from_f<E>(h);
+                            p.cT[o] = c[k];
+                        }
+                    }
+                }
+                rec::named_bar(1, F_EPI_THREADS);  // y[t] stored; xbuf and recv free again
+                if (et == 0) {
+                    // the staging block must be read out before this CTA's arrival
+                    // lets the next step's TMA refill ring_h
+                    if (KS > 1) tc::bulk_wait_read_all();
+                    if ((int)blockIdx.x != p.fault_skip_cta) rec::red_release_add(ctr, 1u);
+                }
+                // saved state for the backward pass, outside the writes the
+                // arrival's release has to cover
+    #pragma unroll
+                for (int k = 0; k < NP; ++k) {
+                    const int n = pair_col(k), uu = pair_unit(k);
+                    const int b = bc0 + n, j = u0 + uu;
+                    if (n >= NBc || b >= B) continue;
+                    ct[(long long)b * H + j] = c[k];
+                    E *g4 = gt + (long long)b * 4 * H + j;
+                    const int fb = p.ijfo ? 2 : 1, gb = 3 - fb;
+                    g4[0] = from_f<E>(gsave[0][k]);
+                    g4[fb * H] = from_f<E>(gsave[1][k]);
+                    g4[gb * H] = from_f<E>(gsave[2][k]);
+                    g4[3 * H] = from_f<E>(gsave[3][k]);
+                }
+                if (MASKED && t + 1 < T) load_mask(t + 1);
+            }
+            if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
         }
-        if (et == 0) tc::bulk_wait_all();  // no copy of this CTA still in flight at exit
     }
 
     tc::tc_fence_before();
