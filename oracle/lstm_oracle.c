@@ -15,10 +15,10 @@
  *   - "gradient derivation" (cell-state chain rule, dL/dW = sum_t delta z_t^T);
  *   - parameter table (tensor shapes, layouts, optional inputs).
  *
- * Readings taken where the page is ambiguous (each is listed in the design doc):
+ * Readings taken where the page is ambiguous:
  *   - W columns are [h | x], i.e. W = [W_h | W_x] with z_t = [h_{t-1}; x_t]
  *     (forward table "input concat" and step 5 "delta h_prev = delta z[1:dim h]");
- *   - gate rows are [i | f | g | o] (gate_order "ifjo", j = g);
+ *   - gate rows are [i | f | g | o] (gate_order "ifjo", j = g) by default;
  *   - one bias b[4H];
  *   - the cell-gradient carry applies the forget gate ONCE: step 5 already sets
  *     delta c_prev = delta c_t * f_t, so step 2 adds delta c_next without a
