@@ -67,6 +67,22 @@ def measured_traffic(phase: str, workload: str):
         return None
 
 
+def reduce_max(v: float, dist=None, device="cpu") -> float:
+    """The max of `v` over the ranks of the default process group (`v` itself
+    without one): a multi-GPU time is the slowest rank's."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, rows: int, steps: int, ms: float) -> float:
+    """Whole-job timesteps/s: every rank processes `rows` timesteps per step
+    (weak scaling), and `ms` is the max over ranks of the timed region."""
+    return world * rows * steps / (ms * 1e-3)
+
+
 def phase_work(w: synth.Workload, phases=None):
     """Algorithmic work per phase: FLOPs for the contractions (2 * M * N * K of
     the products the method defines), bytes for the db column reduction.  With
@@ -236,11 +252,7 @@ def run_ours(args, w, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist, dev)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -358,7 +370,7 @@ def run_ours(args, w, rank, world, local_rank):
                  "ms_per_step": dom_ms / args.steps,
                  "peak_source": f"{peak_src} ({'sustained bf16' if kind == 'flop' else 'HBM copy'})"})
     step_s = ms / args.steps * 1e-3
-    value = world * w.rows / step_s
+    value = job_throughput(world, w.rows, args.steps, ms)
     tflops = w.flops / step_s / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -374,7 +386,7 @@ def run_ours(args, w, rank, world, local_rank):
         "roofline": roof,
         "phases_ms_per_step": {p: v[0] / args.steps for p, v in phases.items()},
         "gpu_launches": launches,
-        "e2e": {"value": world * w.rows * args.steps / (ms_e2e * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_throughput(world, w.rows, args.steps, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e / args.steps,
                 "overlap": "uploads and read-backs on their own streams, two buffer sets"},
@@ -435,11 +447,7 @@ def run_stack(args, w, rank, world, local_rank):
             dist.barrier()
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist, dev)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -516,7 +524,8 @@ def run_stack(args, w, rank, world, local_rank):
     step_s = ms / args.steps * 1e-3
     tflops = sum(lw.flops for lw in layer_w) / step_s / 1e12
     line = {
-        "metric": METRIC, "value": world * w.rows / step_s, "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": job_throughput(world, w.rows, args.steps, ms), "unit": UNIT,
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic (seeded, distributions of the workload definition)",
@@ -530,7 +539,7 @@ def run_stack(args, w, rank, world, local_rank):
         "roofline": roof,
         "phases_ms_per_step": {p: v[0] / args.steps for p, v in phases.items()},
         "gpu_launches": launches,
-        "e2e": {"value": world * w.rows * args.steps / (ms_e2e * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_throughput(world, w.rows, args.steps, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e / args.steps, "overlap": "none"},
         "clocks": clk,

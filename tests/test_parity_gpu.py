@@ -73,13 +73,15 @@ ODD = [
     # W rows of H + I elements off the 16-byte grid, with H on the unit grids
     # of the tensor-map recurrences: those must step aside for the per-step kernels
     (4, 6, 37, 48, "bf16"), (4, 6, 37, 64, "bf16"),
+    # the forward with two batch streams per cluster at its shortest sequences
+    (1, 200, 96, 512, "bf16"), (2, 100, 64, 1024, "bf16"),
 ]
 
 
 # recurrent kernels of the odd bf16 shapes above (see lstm_test_last_paths):
 # the forward with the input projection fused wherever H is a multiple of 32
 # (clusters of 4, 2 and 1 among these), the backward with the weights in TMEM
-ODD_FWD_PATH = {64: 3, 128: 3, 256: 3, 512: 3, 640: 3, 1536: 3}
+ODD_FWD_PATH = {64: 3, 128: 3, 256: 3, 512: 3, 640: 3, 1024: 3, 1536: 3}
 ODD_BWD_PATH = {512: 3, 640: 3, 1536: 3}
 
 
