@@ -143,3 +143,18 @@ def test_stack_is_composed_single_layer_calls(dt, cuda_device):
         assert torch.equal(g.dW[l], grads[l].dW) and torch.equal(g.db[l], grads[l].db), l
         assert torch.equal(g.dh0[l], grads[l].dh0) and torch.equal(g.dc0[l], grads[l].dc0), l
     assert torch.equal(g.dx, grads[0].dx)
+
+
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_stack_empty_sequence(dt, cuda_device):
+    """T = 0: no layer steps; every layer's final state is its initial state and
+    the gradients at the initial states are the ones given at the final states."""
+    T, B, I, H, Lc = 0, 8, 16, 32, 2
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=4)
+    gpu = run_gpu_stack(inp, cuda_device)
+    for l in range(Lc):
+        np.testing.assert_array_equal(gpu["hT"][l], inp["h0"][l].double().numpy())
+        np.testing.assert_array_equal(gpu["cT"][l], inp["c0"][l].double().numpy())
+        np.testing.assert_array_equal(gpu["dh0"][l], inp["dhT"][l].double().numpy())
+        np.testing.assert_array_equal(gpu["dc0"][l], inp["dcT"][l].double().numpy())
+        assert not gpu["dW"][l].any() and not gpu["db"][l].any()
