@@ -23,6 +23,7 @@ LSTM_ERR_CUDA = 4
 LSTM_ERR_TIMEOUT = 5
 LSTM_ERR_NOT_CORESIDENT = 6
 
+ABI_VERSION = 101  # the liblstm.h this binding mirrors (100 * major + minor)
 LSTM_F32 = 0
 LSTM_BF16 = 1
 LSTM_F16 = 2
@@ -119,6 +120,10 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_set_wait_fault.restype = ip
     lib.lstm_test_last_paths.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_paths.restype = ip
+    v = lib.lstm_abi_version()
+    if v // 100 != ABI_VERSION // 100 or v < ABI_VERSION:
+        raise RuntimeError(f"{path}: ABI version {v}, this binding needs {ABI_VERSION} "
+                           "(rebuild with `python -m backward_lstm_fwd_b200.build`)")
     if path == LIB_PATH:
         _lib = lib
     return lib

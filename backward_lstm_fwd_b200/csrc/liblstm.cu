@@ -1560,7 +1560,7 @@ int stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy
 
 extern "C" {
 
-int lstm_abi_version(void) { return 100; }
+int lstm_abi_version(void) { return LSTM_ABI_VERSION; }
 
 const char *lstm_strerror(int code) {
     switch (code) {

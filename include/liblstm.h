@@ -303,7 +303,9 @@ int lstm_fwd_noalloc(const lstm_dims *d, const void *x, const void *W, const voi
 /* Static description of a status code. */
 const char *lstm_strerror(int code);
 
-/* ABI version: 100 * major + minor. */
+/* ABI version: 100 * major + minor (1.1: lstm_options with gate_order, the
+ * LSTM_F16 compute type and the stack entry points). */
+#define LSTM_ABI_VERSION 101
 int lstm_abi_version(void);
 
 #ifdef __cplusplus

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) >= set(L.EXPORTS)
     for n in names:
         assert hasattr(lib, n), f"{n} declared in liblstm.h but not exported"
-    assert lib.lstm_abi_version() == 100
+    assert lib.lstm_abi_version() == L.ABI_VERSION == 101
 
 
 def test_strerror(lib):
