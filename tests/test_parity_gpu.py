@@ -100,9 +100,12 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
     assert_within(compare(gpu, ref, dt), dt, w.name)
 
 
-@pytest.mark.parametrize("dt", ["fp32", "bf16", "fp16"])
-def test_optional_inputs_absent(dt, cuda_device):
-    w = synth.custom(6, 4, 24, 40, dt, seed=5)
+@pytest.mark.parametrize("dt,B,I,H", [("fp32", 4, 24, 40), ("bf16", 4, 24, 40), ("fp16", 4, 24, 40),
+                                      ("bf16", 128, 64, 512)])
+def test_optional_inputs_absent(dt, B, I, H, cuda_device):
+    """Also at B = 128, H = 512: the fused forward with two batch streams
+    starts from h0 = 0 without loading it."""
+    w = synth.custom(6, B, I, H, dt, seed=5)
     inp = synth.make_inputs(w)
     drop = ("b", "h0", "c0", "dhT", "dcT")
     gpu = run_gpu(inp, cuda_device, drop=drop)

@@ -78,6 +78,7 @@ CASES = [
     (12, 48, 64, 512, 2, "bf16"),   # TMEM-weight kernels, layer 0 narrower than H
     (40, 64, 1024, 512, 2, "bf16"), # chunked backward, layer 0 wider than H
     (12, 48, 64, 512, 3, "fp16"),   # fp16
+    (6, 128, 64, 512, 2, "bf16"),   # the forward with two batch streams per cluster
 ]
 
 
