@@ -35,7 +35,7 @@ def _outputs(st):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("T,B,I,H,dt", [(16, 32, 64, 128, "bf16"), (9, 5, 24, 40, "fp32"),
-                                        (12, 64, 256, 256, "bf16")])
+                                        (12, 64, 256, 256, "bf16"), (4, 128, 64, 512, "bf16")])
 def test_noalloc_matches_lstm_fwd_twice(T, B, I, H, dt, cuda_device):
     lbuild.build()
     w = synth.custom(T, B, I, H, dt, seed=T + B + I + H)
