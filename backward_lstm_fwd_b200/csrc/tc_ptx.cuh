@@ -234,18 +234,6 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
-}
-__device__ __forceinline__ void st_cluster_v2(uint32_t caddr, float a, float b) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(caddr), "f"(a), "f"(b)
-                 : "memory");
-}
 // Bulk copy (TMA engine) of `bytes` from this CTA's shared memory to shared
 // memory of another CTA of the cluster; completes `bytes` transactions on the
 // destination CTA's mbarrier.  Addresses 16-byte aligned, bytes % 16 == 0.
@@ -257,11 +245,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_caddr, const void
         : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until every committed bulk-copy group of this thread but the most
-// recent one has finished reading its source.
-__device__ __forceinline__ void bulk_wait_read_but_one() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 // Wait until every committed bulk copy of this thread has finished reading its source.
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -269,12 +252,6 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 // Wait until every committed bulk copy of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's earlier writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
-                 : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
