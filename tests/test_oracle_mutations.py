@@ -44,10 +44,11 @@ MUTATIONS = {
     "mask_no_h_pass": ("dh_pass[j] = (1.0 - m) * dh_tot;", "dh_pass[j] = 0.0;"),
     # padding updates the cell state anyway (variable-length mask, forward)
     "mask_c_moves": ("c_ = mt[j] * c_ + (1.0 - mt[j]) * cprev[j];", "c_ = c_;"),
-    # reverse direction: c_{t-1} of the forget-gate gradient taken from the
-    # forward direction's neighbour
+    # reverse direction: the previous cell state of the forget-gate gradient
+    # taken at the step's own time instead of time t + 1 (stays in bounds, unlike
+    # the forward direction's neighbour t - 1, which runs off the array at t = 0)
     "reverse_cprev": ("const int tp = reverse ? t + 1 : t - 1;        /* time of step s - 1 */",
-                      "const int tp = t - 1;"),
+                      "const int tp = reverse ? t : t - 1;"),
 }
 
 # mutations that only a masked case can reveal
