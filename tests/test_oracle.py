@@ -239,6 +239,37 @@ def test_zero_weights_closed_form():
     np.testing.assert_allclose(out["dc0"], 0.5 * dc[0], rtol=1e-12, atol=1e-14)
 
 
+def test_one_step_closed_form():
+    """T = 1 in closed form: with z = W [h0; x_0] + b, i, f, o = sigma(z_i, z_f,
+    z_o), g = tanh(z_g), the forward table gives c = f c0 + i g and y_0 = hT =
+    o tanh(c).  That expression, written out in torch (fp64) and differentiated
+    by autograd, gives every gradient of L = <dy_0 + dhT, h> + <dcT, c>."""
+    B, I, H = 3, 4, 5
+    p, g = random_case(1, B, I, H, seed=21)
+    out = run(p, g)
+    t = {k: torch.from_numpy(np.array(v)).requires_grad_() for k, v in p.items()}
+    z = torch.cat([t["h0"], t["x"][0]], dim=1) @ t["W"].T + t["b"]
+    i, f = torch.sigmoid(z[:, :H]), torch.sigmoid(z[:, H:2 * H])
+    gg, o = torch.tanh(z[:, 2 * H:3 * H]), torch.sigmoid(z[:, 3 * H:])
+    c = f * t["c0"] + i * gg
+    h = o * torch.tanh(c)
+    L = ((torch.from_numpy(g["dy"][0]) + torch.from_numpy(g["dhT"])) * h).sum() + \
+        (torch.from_numpy(g["dcT"]) * c).sum()
+    L.backward()
+
+    def close(a, b):
+        np.testing.assert_allclose(a, b.detach().numpy(), rtol=1e-12, atol=1e-14)
+
+    close(out["y"][0], h)
+    close(out["hT"], h)
+    close(out["cT"], c)
+    close(out["dx"], t["x"].grad)
+    close(out["dW"], t["W"].grad)
+    close(out["db"], t["b"].grad)
+    close(out["dh0"], t["h0"].grad)
+    close(out["dc0"], t["c0"].grad)
+
+
 def test_invariants():
     """db = sum over t and batch of dG; dW = sum dG z^T; dx_t and dh_prev are the
     x- and h-parts of W^T dG_t; delta c_prev = delta c_t * f_t (steps 4-5)."""
