@@ -1,6 +1,9 @@
 /*
- * liblstm.h -- C ABI of liblstm: single-layer, unidirectional LSTM forward pass
- * and backpropagation through time on one NVIDIA B200 (sm_100a).
+ * liblstm.h -- C ABI of liblstm: the LSTM forward pass and backpropagation
+ * through time on one NVIDIA B200 (sm_100a).  lstm_fwd / lstm_bwd run the
+ * single-layer, unidirectional operation; lstm_fwd_ex / lstm_bwd_ex add the
+ * operator's options (variable length, reverse direction, gate order);
+ * lstm_stack_fwd / lstm_stack_bwd run a stack of layers.
  *
  * The operation is the one defined on the "SingleLayerLstmGrad" operator page
  * (CANN ops-nn):
