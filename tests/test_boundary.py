@@ -52,6 +52,12 @@ def test_workspace_sizes(lib):
     assert L.fwd_workspace_size(L.dims(-1, 2, 3, 4, 0)) == 0
     assert L.bwd_workspace_size(L.dims(1, 2, 3, 4, 7)) == 0
     assert L.fwd_workspace_size(L.dims(0, 0, 0, 0, 0)) >= 256
+    # fp16 has bf16's layout (two-byte dG, W_h^T, per-group db partials)
+    h = L.dims(256, 128, 1024, 1024, L.LSTM_F16)
+    assert L.fwd_workspace_size(h) == fw and L.bwd_workspace_size(h) == bw
+    # fp32 keeps dG in fp32 and needs no W_h^T copy
+    f = L.dims(256, 128, 1024, 1024, L.LSTM_F32)
+    assert L.bwd_workspace_size(f) >= 256 + TB * G4 * 4
 
 
 def fwd_args(d, **over):
