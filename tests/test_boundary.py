@@ -273,3 +273,27 @@ def test_stack_slices_must_align(lib):
 def test_stack_workspace_too_small(lib):
     need = L.stack_bwd_workspace_size(DS, 2)
     assert call_stack_bwd(DS, 2, ws_bytes=need - 1) == L.LSTM_ERR_WORKSPACE
+
+
+def test_option_marshalling():
+    """The binding's option struct: direction and gate_order constants, the
+    attribute spellings, and when the plain entry points are used."""
+    assert L._gate_order("ifjo") == L.LSTM_GATES_IFJO and L._gate_order("ijfo") == L.LSTM_GATES_IJFO
+    assert L._gate_order(7) == 7  # raw values pass through (the library rejects them)
+    with pytest.raises(KeyError):
+        L._gate_order("iofj")
+    o = L._options(None, True, "ijfo")
+    assert o.seq_mask is None and o.direction == L.LSTM_DIR_REVERSE
+    assert o.gate_order == L.LSTM_GATES_IJFO
+    assert L._plain(None, False, "ifjo")
+    assert not L._plain(None, True, "ifjo") and not L._plain(None, False, "ijfo")
+    assert not L._plain(FAKE, False, "ifjo")
+
+
+def test_dtype_codes():
+    import torch
+    assert L.dtype_code(torch.float32) == L.LSTM_F32
+    assert L.dtype_code(torch.bfloat16) == L.LSTM_BF16
+    assert L.dtype_code(torch.float16) == L.LSTM_F16
+    with pytest.raises(ValueError):
+        L.dtype_code(torch.float64)
