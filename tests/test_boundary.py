@@ -37,6 +37,29 @@ def test_exports_every_declared_symbol(lib):
     assert lib.lstm_abi_version() == L.ABI_VERSION == 101
 
 
+def declared_arities():
+    """{function: number of parameters} of every prototype in liblstm.h (the
+    testing header's too)."""
+    out = {}
+    for h in (HEADER, HEADER.replace("liblstm.h", "liblstm_testing.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for name, args in re.findall(r"\b(lstm_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+            args = args.strip()
+            out[name] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_headers(lib):
+    """Every prototype the binding types has as many ctypes argtypes as the
+    header has parameters (drift between the two would pass garbage)."""
+    arity = declared_arities()
+    assert "lstm_stack_bwd" in arity and "lstm_test_tc_gemm" in arity
+    for name, n in arity.items():
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, name
+        assert len(argtypes) == n, (name, len(argtypes), n)
+
+
 def test_strerror(lib):
     for code in range(7):
         assert L.strerror(code)
