@@ -120,6 +120,10 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_set_wait_fault.restype = ip
     lib.lstm_test_last_paths.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_paths.restype = ip
+    lib.lstm_test_bwd_chunks.argtypes = [ip]
+    lib.lstm_test_bwd_chunks.restype = ip
+    lib.lstm_test_chunk_bound.argtypes = [ip, ip, ip]
+    lib.lstm_test_chunk_bound.restype = ip
     v = lib.lstm_abi_version()
     if v // 100 != ABI_VERSION // 100 or v < ABI_VERSION:
         raise RuntimeError(f"{path}: ABI version {v}, this binding needs {ABI_VERSION} "

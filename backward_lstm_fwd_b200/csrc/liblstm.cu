@@ -1718,6 +1718,16 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns) {
     return LSTM_OK;
 }
 
+int lstm_test_bwd_chunks(int T) {
+    lstm_dims d = {T, 1, 1, 1, LSTM_BF16};
+    return T < 0 ? -1 : bwd_chunks(&d);
+}
+
+int lstm_test_chunk_bound(int T, int nch, int c) {
+    if (T < 0 || nch < 1 || c < 0 || c > nch) return -1;
+    return chunk_bound(T, nch, c);
+}
+
 int lstm_test_last_paths(int *fwd_path, int *bwd_path) {
     if (fwd_path) *fwd_path = g_last_fwd_path;
     if (bwd_path) *bwd_path = g_last_bwd_path;

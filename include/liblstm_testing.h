@@ -47,6 +47,15 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
  */
 int lstm_test_last_paths(int *fwd_path, int *bwd_path);
 
+/*
+ * Reverse-time chunking of the tensor-core backward: the number of chunk
+ * launches a call over `T` steps uses (after LSTM_BWD_CHUNKS), and the first
+ * epilogue iteration of chunk `c` (c = nch gives T).  Host logic only; no GPU
+ * needed.
+ */
+int lstm_test_bwd_chunks(int T);
+int lstm_test_chunk_bound(int T, int nch, int c);
+
 #ifdef __cplusplus
 }
 #endif

@@ -320,3 +320,25 @@ def test_dtype_codes():
     assert L.dtype_code(torch.float16) == L.LSTM_F16
     with pytest.raises(ValueError):
         L.dtype_code(torch.float64)
+
+
+def test_backward_chunking_host_logic(lib, monkeypatch):
+    """The reverse-time chunks of the tensor-core backward (host logic, no
+    GPU): min(8, T/16) chunks from T = 32 on, one below; boundaries strictly
+    increasing from 0 to T; sizes shrinking geometrically, so that the last
+    chunk (whose dW / dx GEMM runs alone) is the smallest."""
+    monkeypatch.delenv("LSTM_BWD_CHUNKS", raising=False)
+    assert lib.lstm_test_bwd_chunks(-1) == -1
+    for T in list(range(0, 300)) + [1024, 4096]:
+        n = lib.lstm_test_bwd_chunks(T)
+        assert n == (min(8, T // 16) if T >= 32 else 1), T
+        b = [lib.lstm_test_chunk_bound(T, n, c) for c in range(n + 1)]
+        assert b[0] == 0 and b[-1] == T, (T, b)
+        if T >= n:
+            assert all(b[i + 1] > b[i] for i in range(n)), (T, b)
+        sizes = [b[i + 1] - b[i] for i in range(n)]
+        if n > 1 and T >= 64:
+            assert sizes[-1] == min(sizes) and sizes[0] == max(sizes), (T, sizes)
+    assert [lib.lstm_test_chunk_bound(256, 8, c) for c in range(9)] == \
+        [0, 62, 111, 150, 182, 207, 227, 243, 256]
+    assert lib.lstm_test_chunk_bound(10, 2, 3) == -1  # c > nch
