@@ -23,12 +23,13 @@ LSTM_ERR_CUDA = 4
 LSTM_ERR_TIMEOUT = 5
 LSTM_ERR_NOT_CORESIDENT = 6
 
-ABI_VERSION = 101  # the liblstm.h this binding mirrors (100 * major + minor)
+ABI_VERSION = 102  # the liblstm.h this binding mirrors (100 * major + minor)
 LSTM_F32 = 0
 LSTM_BF16 = 1
 LSTM_F16 = 2
 
-EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd", "lstm_bwd",
+EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd_workspace_size_ex",
+           "lstm_fwd_workspace_size_max", "lstm_fwd", "lstm_bwd",
            "lstm_fwd_ex", "lstm_bwd_ex", "lstm_stack_fwd_workspace_size",
            "lstm_stack_bwd_workspace_size", "lstm_stack_fwd", "lstm_stack_bwd",
            "lstm_status", "lstm_profile_begin", "lstm_profile_end", "lstm_launch_count",
@@ -79,11 +80,15 @@ def load(path: str = LIB_PATH):
     lib.lstm_fwd_workspace_size.restype = sz
     lib.lstm_bwd_workspace_size.argtypes = [dp]
     lib.lstm_bwd_workspace_size.restype = sz
+    lib.lstm_fwd_workspace_size_max.argtypes = [dp]
+    lib.lstm_fwd_workspace_size_max.restype = sz
     lib.lstm_fwd.argtypes = [dp] + [vp] * 10 + [vp, sz, vp]
     lib.lstm_fwd.restype = ip
     lib.lstm_bwd.argtypes = [dp] + [vp] * 15 + [vp, sz, vp]
     lib.lstm_bwd.restype = ip
     op = ctypes.POINTER(Options)
+    lib.lstm_fwd_workspace_size_ex.argtypes = [dp, op]
+    lib.lstm_fwd_workspace_size_ex.restype = sz
     lib.lstm_fwd_ex.argtypes = [dp, op] + [vp] * 10 + [vp, sz, vp]
     lib.lstm_fwd_ex.restype = ip
     lib.lstm_bwd_ex.argtypes = [dp, op] + [vp] * 15 + [vp, sz, vp]
@@ -113,6 +118,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_launch_count.restype = ctypes.c_longlong
     lib.lstm_fwd_noalloc.argtypes = [dp] + [vp] * 10 + [vp]
     lib.lstm_fwd_noalloc.restype = ip
+    lib.lstm_fwd_noalloc_status.argtypes = [vp]
+    lib.lstm_fwd_noalloc_status.restype = ip
     ll = ctypes.c_longlong
     lib.lstm_test_tc_gemm.argtypes = [ip, ip, ip, vp, ll, ip, vp, ll, ip, vp, vp, ll, vp, sz, vp]
     lib.lstm_test_tc_gemm.restype = ip
@@ -171,8 +178,18 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def fwd_workspace_size(d: Dims) -> int:
-    return int(load().lstm_fwd_workspace_size(ctypes.byref(d)))
+def fwd_workspace_size(d: Dims, mask=None, reverse: bool = False, gate_order="ifjo") -> int:
+    """Forward workspace bytes for the plan this call takes on the current
+    device (lstm_fwd_workspace_size, or _ex with the call's options)."""
+    if _plain(mask, reverse, gate_order):
+        return int(load().lstm_fwd_workspace_size(ctypes.byref(d)))
+    opt = _options(mask, reverse, gate_order)
+    return int(load().lstm_fwd_workspace_size_ex(ctypes.byref(d), ctypes.byref(opt)))
+
+
+def fwd_workspace_size_max(d: Dims) -> int:
+    """Forward workspace bytes that cover every plan on every device."""
+    return int(load().lstm_fwd_workspace_size_max(ctypes.byref(d)))
 
 
 def bwd_workspace_size(d: Dims) -> int:
@@ -303,6 +320,12 @@ def lstm_fwd_noalloc(d: Dims, x, W, b, h0, c0, y, hT, cT, gates, cells, stream=N
     return rc
 
 
+def lstm_fwd_noalloc_status(stream=None) -> int:
+    """Synchronise `stream`, then read and clear the status word of the static
+    scratch lstm_fwd_noalloc uses on the current device."""
+    return int(load().lstm_fwd_noalloc_status(_stream(stream)))
+
+
 def lstm_status(ws, ws_bytes=None, stream=None) -> int:
     if ws_bytes is None:
         ws_bytes = ws.numel() * ws.element_size()
@@ -388,7 +411,7 @@ def forward(x, W, b=None, h0=None, c0=None, ws=None, stream=None, mask=None,
     H = W.shape[0] // 4
     st = State(T, B, I, H, x.dtype, x.device)
     if ws is None:
-        ws = empty_workspace(fwd_workspace_size(st.dims), x.device)
+        ws = empty_workspace(fwd_workspace_size(st.dims, mask, reverse, gate_order), x.device)
     lstm_fwd(st.dims, x, W, b, h0, c0, st.y, st.hT, st.cT, st.gates, st.cells, ws, stream=stream,
              mask=mask, reverse=reverse, gate_order=gate_order)
     return st

@@ -68,6 +68,22 @@ struct Phase {
 };
 }  // namespace prof
 
+// ----------------------------------------------------- environment switches
+// The library reads exactly these variables, at every call (no caching); the
+// list, with defaults, is in include/liblstm_testing.h:
+//   LSTM_FORCE_SIMT=1      CUDA-core kernels only
+//   LSTM_FWD_FUSED_X=0     no fused forward kernel (the Gx plans)
+//   LSTM_BWD_TMEM_W=0      no backward kernel with the weights in tensor memory
+//   LSTM_BWD_CHUNKS=n      reverse-time chunks of the overlapped backward
+//   LSTM_LAUNCH_NONCOOP=1  cluster launches without the cooperative attribute
+//                          (also taken when a CUDA injection library -- a
+//                          profiler or sanitizer -- is attached)
+bool env_is(const char *name, char value) {
+    const char *e = getenv(name);
+    return e && e[0] == value && e[1] == '\0';
+}
+bool force_simt() { return env_is("LSTM_FORCE_SIMT", '1'); }
+
 // ------------------------------------------------------------ validation
 bool dims_ok(const lstm_dims *d) {
     if (!d) return false;
@@ -144,12 +160,7 @@ BwdLayout bwd_layout(const lstm_dims *d) {
 // whole 16-byte groups (TMA strides and the W_x base offset are then 16-byte
 // aligned).
 bool tc_gemm_ok(const lstm_dims *d) {
-    static int force_simt = -1;
-    if (force_simt < 0) {
-        const char *e = getenv("LSTM_FORCE_SIMT");
-        force_simt = (e && e[0] == '1') ? 1 : 0;
-    }
-    return !force_simt && d->dtype != LSTM_F32 && d->H >= 8 && d->I >= 8 && d->H % 8 == 0 &&
+    return !force_simt() && d->dtype != LSTM_F32 && d->H >= 8 && d->I >= 8 && d->H % 8 == 0 &&
            d->I % 8 == 0 && tcg::encode_fn() != nullptr;
 }
 
@@ -308,20 +319,14 @@ int bwd_chunks(const lstm_dims *d) {
 }
 
 // First epilogue iteration of chunk c of nch over T steps (c = nch gives T).
-// Chunk sizes shrink geometrically (ratio r = 0.8; LSTM_BWD_CHUNK_RATIO
-// overrides it, 1 = equal chunks): the dW / dx GEMM of a chunk runs beside the
-// next, smaller one, and the GEMM of the last chunk, which runs alone, is the
-// smallest.  Every chunk keeps at least one step.
+// Chunk sizes shrink geometrically (ratio 0.8): the dW / dx GEMM of a chunk
+// runs beside the next, smaller one, and the GEMM of the last chunk, which
+// runs alone, is the smallest.  Every chunk keeps at least one step.
 int chunk_bound(int T, int nch, int c) {
-    static double r = -1.0;
-    if (r < 0.0) {
-        const char *e = getenv("LSTM_BWD_CHUNK_RATIO");
-        r = e ? atof(e) : 0.8;
-        if (!(r > 0.0 && r <= 1.0)) r = 0.8;
-    }
+    constexpr double r = 0.8;
     if (c <= 0) return 0;
     if (c >= nch) return T;
-    const double f = r == 1.0 ? (double)c / nch : (1.0 - pow(r, c)) / (1.0 - pow(r, nch));
+    const double f = (1.0 - pow(r, c)) / (1.0 - pow(r, nch));
     int b = (int)(T * f + 0.5);
     b = std::max(b, c);               // at least one step per earlier chunk
     return std::min(b, T - (nch - c));  // and per later one
@@ -351,8 +356,7 @@ bool plan_fwd_recur(const lstm_dims *d, RecPlan &P) {
     if (d->dtype != LSTM_BF16 || d->H % rec::UNITS != 0 || d->H > 1024 || d->B < 1 ||
         (d->H + d->I) % 8 != 0 || tcg::encode_fn() == nullptr)
         return false;
-    const char *e = getenv("LSTM_FORCE_SIMT");
-    if (e && e[0] == '1') return false;
+    if (force_simt()) return false;
     P.S = d->H / rec::UNITS;
     const int gmax = tcg::sm_count() / P.S;
     if (gmax < 1) return false;
@@ -435,8 +439,7 @@ bool plan_bwd_recur(const lstm_dims *d, RecPlan &P) {
     if (d->dtype != LSTM_BF16 || d->H % rec::UNITS != 0 || d->H > 1024 || d->B < 1 ||
         tcg::encode_fn() == nullptr)
         return false;
-    const char *e = getenv("LSTM_FORCE_SIMT");
-    if (e && e[0] == '1') return false;
+    if (force_simt()) return false;
     P.S = d->H / rec::UNITS;
     const int gmax = std::min(tcg::sm_count() / P.S, kMaxGroups);
     if (gmax < 1) return false;
@@ -518,11 +521,6 @@ struct Rec2Plan {
     size_t smem;
     int split = 1;  // fused forward: batch streams per cluster (NB rows each)
 };
-
-bool force_simt() {
-    const char *e = getenv("LSTM_FORCE_SIMT");
-    return e && e[0] == '1';
-}
 
 int max_active_clusters(const void *kern, int threads, size_t smem, int KS) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -620,10 +618,7 @@ const void *fwd3_kernel_ptr(int NB, int KS, bool masked, int split) {
 // CTA's W_h and W_x K-slices must fit TMEM beside two accumulators.
 // LSTM_FWD_FUSED_X=0 turns it off (comparison runs).
 bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
-    const char *e = getenv("LSTM_FWD_FUSED_X");
-    if (e && e[0] == '0') return false;
-    const char *es = getenv("LSTM_FWD_SPLIT");  // "1": one batch stream per cluster
-    const bool split_ok = !(es && es[0] == '1');
+    if (env_is("LSTM_FWD_FUSED_X", '0')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
         d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
@@ -645,7 +640,7 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
         // two interleaved batch streams of NB / 2 rows per cluster where that
         // instantiation exists and fits, else one
         for (int split : {2, 1}) {
-            if (split == 2 && (!split_ok || NB < 64 || G * 2 > kMaxGroups)) continue;
+            if (split == 2 && (NB < 64 || G * 2 > kMaxGroups)) continue;
             const int NBv = NB / split;
             if (NBv / KS < 4) continue;
             if (rec3::fwd3_tmem_cols(NBv, kcc, kcx) > 512) continue;
@@ -707,8 +702,7 @@ bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
 // exchange round (at least 4 stages, H >= 512).  LSTM_BWD_TMEM_W=0 turns it
 // off (comparison runs).
 bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
-    const char *e = getenv("LSTM_BWD_TMEM_W");
-    if (e && e[0] == '0') return false;
+    if (env_is("LSTM_BWD_TMEM_W", '0')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec3::UNITS != 0 || d->B < 1 ||
         tcg::encode_fn() == nullptr || force_simt())
         return false;
@@ -761,11 +755,13 @@ cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t s
     at[1].val.cooperative = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    // LSTM_LAUNCH_NONCOOP=1 (profiling aid: some profilers cannot replay a
-    // cooperative cluster launch) skips straight to the occupancy-checked
-    // cluster launch below.
-    const char *nc = getenv("LSTM_LAUNCH_NONCOOP");
-    if (!(nc && nc[0] == '1')) {
+    // Profilers cannot replay a cooperative cluster launch: with
+    // LSTM_LAUNCH_NONCOOP=1, or when a CUDA injection library (a profiler or
+    // a sanitizer) is attached, go straight to the occupancy-checked cluster
+    // launch below.
+    const char *inj = getenv("CUDA_INJECTION64_PATH");
+    const bool noncoop = env_is("LSTM_LAUNCH_NONCOOP", '1') || (inj && inj[0]);
+    if (!noncoop) {
         e = cudaLaunchKernelEx(&cfg, kern, prm);
         if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) {
             note_launch();
@@ -1018,9 +1014,8 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         cudaStreamWaitEvent(A.gemm, ev_fork, 0) != cudaSuccess)
         return LSTM_ERR_CUDA;
     // the GEMM beside the recurrence takes at most the SMs the recurrence
-    // leaves idle (LSTM_BWD_GEMM_CTAS caps it lower, for comparison runs)
-    int gemm_ctas = std::max(1, tcg::sm_count() - P.R * P.KS * P.G);
-    if (const char *e = getenv("LSTM_BWD_GEMM_CTAS")) gemm_ctas = std::max(1, std::min(gemm_ctas, atoi(e)));
+    // leaves idle
+    const int gemm_ctas = std::max(1, tcg::sm_count() - P.R * P.KS * P.G);
     int rc = LSTM_OK;
     {
         prof::Phase ph(LSTM_PHASE_BWD_RECUR, A.rec);
@@ -1062,10 +1057,13 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
 // ------------------------------------------------------------ forward pass
 // mask (variable length) or NULL; masked calls run on the TMEM-weight cluster
 // kernel or the per-step kernels only.
+// plan3: the fused forward's plan when it applies (NULL otherwise); every
+// other path needs the Gx buffer, i.e. ws_bytes >= fwd_layout(d).total.
 template <class T>
 int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0,
              const float *c0, const T *mask, bool reverse, bool ijfo, T *y, T *hT, float *cT,
-             T *gates, float *cells, char *ws, cudaStream_t s) {
+             T *gates, float *cells, char *ws, size_t ws_bytes, const Rec2Plan *plan3,
+             cudaStream_t s) {
     typedef typename Tc16<T>::type E;  // the 16-bit type of the tensor-core paths
     // masked, reverse-direction, "ijfo" or fp16 calls: TMEM-weight kernel or
     // per-step kernels (the other kernels are bf16 / default-order only)
@@ -1075,10 +1073,9 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
     const FwdLayout L = fwd_layout(d);
     float *Gx = (float *)(ws + L.gx);
     if ((long long)T_ * B > 0 && H > 0) {
-        Rec2Plan plan3;
-        if (plan_fwd3(d, plan3, mask != nullptr)) {  // a1 fused into a2
+        if (plan3) {  // a1 fused into a2
             prof::Phase ph(LSTM_PHASE_FWD_RECUR, s);
-            const int rc = tc_fwd_recurrence3(d, plan3, (const E *)x, (const E *)W,
+            const int rc = tc_fwd_recurrence3(d, *plan3, (const E *)x, (const E *)W,
                                               (const E *)b, (const E *)h0, c0,
                                               (const E *)mask, reverse, ijfo, (E *)y,
                                               (E *)hT, cT, (E *)gates, cells,
@@ -1086,6 +1083,8 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
             g_last_fwd_path = 3;
             if (rc != LSTM_ERR_NOT_CORESIDENT) return rc;
         }
+        // every path below reads the input projection from Gx
+        if (ws_bytes < L.total) return LSTM_ERR_WORKSPACE;
         {   // a1: Gx = X W_x^T + b over all T*B rows (input concat, x-part)
             prof::Phase ph(LSTM_PHASE_INPUT_PROJ, s);
             if (tc_gemm_ok(d)) {
@@ -1321,6 +1320,21 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
 
 }  // namespace
 
+namespace {
+// The forward's plan on the current device: the fused kernel (input projection
+// inside the recurrence) when it applies to these dims and options.
+bool fwd_fused_plan(const lstm_dims *d, bool masked, Rec2Plan &P) {
+    return (long long)d->T * d->B > 0 && d->H > 0 && plan_fwd3(d, P, masked);
+}
+
+// Bytes the forward needs: the 256-byte control block alone when the fused
+// kernel runs, else the control block and the fp32 Gx buffer.
+size_t fwd_ws_need(const lstm_dims *d, bool masked) {
+    Rec2Plan P;
+    return fwd_fused_plan(d, masked, P) ? kCtrlBytes : fwd_layout(d).total;
+}
+}  // namespace
+
 // ------------------------------------------ scratch for lstm_fwd_noalloc
 // A file-scope device array: every GPU that loads this library holds
 // LSTM_NOALLOC_SCRATCH_BYTES of it until the process exits.  In host code the
@@ -1370,24 +1384,28 @@ int fwd_entry(const lstm_dims *d, const lstm_options *opt, const void *x, const 
         !ptr_ok(y, TB * d->H > 0) || !ptr_ok(hT, BH > 0) || !ptr_ok(cT, BH > 0) ||
         !ptr_ok(gates, TB * d->H > 0) || !ptr_ok(cells, TB * d->H > 0))
         return LSTM_ERR_INVALID_ARG;
-    const int wsrc = ws_ok(ws, ws_bytes, fwd_layout(d).total);
+    Rec2Plan plan3;
+    const bool fused = fwd_fused_plan(d, mask != nullptr, plan3);
+    const int wsrc = ws_ok(ws, ws_bytes, fused ? kCtrlBytes : fwd_layout(d).total);
     if (wsrc != LSTM_OK) return wsrc;
     cudaStream_t s = (cudaStream_t)stream;
     if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    const Rec2Plan *p3 = fused ? &plan3 : nullptr;
     if (d->dtype == LSTM_F32)
         return fwd_simt<float>(d, (const float *)x, (const float *)W, (const float *)b,
                                (const float *)h0, c0, (const float *)mask, reverse, ijfo,
-                               (float *)y, (float *)hT, cT, (float *)gates, cells, (char *)ws, s);
+                               (float *)y, (float *)hT, cT, (float *)gates, cells, (char *)ws,
+                               ws_bytes, p3, s);
     if (d->dtype == LSTM_F16) {
         typedef __half hf;
         return fwd_simt<hf>(d, (const hf *)x, (const hf *)W, (const hf *)b, (const hf *)h0, c0,
                             (const hf *)mask, reverse, ijfo, (hf *)y, (hf *)hT, cT, (hf *)gates,
-                            cells, (char *)ws, s);
+                            cells, (char *)ws, ws_bytes, p3, s);
     }
     typedef __nv_bfloat16 bf;
     return fwd_simt<bf>(d, (const bf *)x, (const bf *)W, (const bf *)b, (const bf *)h0, c0,
                         (const bf *)mask, reverse, ijfo, (bf *)y, (bf *)hT, cT, (bf *)gates,
-                        cells, (char *)ws, s);
+                        cells, (char *)ws, ws_bytes, p3, s);
 }
 
 int bwd_entry(const lstm_dims *d, const lstm_options *opt, const void *dy, const void *dhT,
@@ -1577,6 +1595,16 @@ const char *lstm_strerror(int code) {
 
 size_t lstm_fwd_workspace_size(const lstm_dims *d) {
     if (!dims_ok(d)) return 0;
+    return fwd_ws_need(d, false);
+}
+
+size_t lstm_fwd_workspace_size_ex(const lstm_dims *d, const lstm_options *opt) {
+    if (!dims_ok(d)) return 0;
+    return fwd_ws_need(d, opt && opt->seq_mask);
+}
+
+size_t lstm_fwd_workspace_size_max(const lstm_dims *d) {
+    if (!dims_ok(d)) return 0;
     return fwd_layout(d).total;
 }
 
@@ -1679,17 +1707,22 @@ int lstm_fwd_noalloc(const lstm_dims *d, const void *x, const void *W, const voi
                      void *gates, float *cells, void *stream) {
     if (!dims_ok(d)) return LSTM_ERR_INVALID_ARG;
     if (!dims_supported(d)) return LSTM_ERR_UNSUPPORTED;
-    const size_t need = fwd_layout(d).total;
-    if (need > (size_t)LSTM_NOALLOC_SCRATCH_BYTES) return LSTM_ERR_UNSUPPORTED;
+    if (fwd_ws_need(d, false) > (size_t)LSTM_NOALLOC_SCRATCH_BYTES) return LSTM_ERR_UNSUPPORTED;
     void *ws = nullptr;
     const int rc = noalloc_scratch(&ws);
     if (rc != LSTM_OK) return rc;
-    // the shared buffer keeps the last call's bytes: zero the control block
-    // (status word and barrier counters) that the kernels expect at zero
-    if (cudaMemsetAsync(ws, 0, kCtrlBytes, (cudaStream_t)stream) != cudaSuccess)
-        return LSTM_ERR_CUDA;
+    // lstm_fwd checks every argument before it enqueues anything, then zeroes
+    // the scratch's control block (status word, barrier counters) in stream
+    // order: the previous call's bytes are never read
     return lstm_fwd(d, x, W, b, h0, c0, y, hT, cT, gates, cells, ws,
                     (size_t)LSTM_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int lstm_fwd_noalloc_status(void *stream) {
+    void *ws = nullptr;
+    const int rc = noalloc_scratch(&ws);
+    if (rc != LSTM_OK) return rc;
+    return lstm_status(ws, kCtrlBytes, stream);
 }
 
 int lstm_test_tc_gemm(int M, int N, int K, const void *A, long long lda, int a_mn_major,

@@ -37,6 +37,7 @@ from backward_lstm_fwd_b200 import synth  # noqa: E402
 METRIC = "LSTM fwd+bwd (T·B) timesteps/sec and % of bf16 tensor peak, 1×B200"
 UNIT = "timesteps/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # dense bf16, B200 data sheet (context only)
 
 
 def load_peaks():
@@ -47,6 +48,18 @@ def load_peaks():
         return d, "measured"
     except (OSError, ValueError):
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def tensor_peak(peaks, clk):
+    """The bf16 peak a kernel timed inside this run is held to: the burst
+    figure when the sampled SM clock stayed at its maximum with no throttle
+    reason active (the conditions the burst figure was measured under), else
+    the sustained one."""
+    at_max = (clk is not None and clk.get("sm_mhz") and clk.get("sm_max_mhz")
+              and clk["sm_mhz"] >= 0.98 * clk["sm_max_mhz"] and not clk.get("reasons"))
+    if at_max:
+        return peaks["bf16_tflops"], "burst bf16 (clocks at max, no throttle reason)"
+    return peaks["bf16_tflops_sustained"], "sustained bf16 (clocks below max or throttled)"
 
 
 def measured_traffic(phase: str, workload: str):
@@ -214,6 +227,82 @@ def run_reference(args, w, rank, world):
     return 0
 
 
+class Problem:
+    """One workload resident on the device: inputs, outputs, workspaces and a
+    stream, and the step (lstm_fwd + lstm_bwd) that bench times."""
+
+    def __init__(self, L, w, dev, seq_mask=False):
+        self.L, self.w, self.dev = L, w, dev
+        self.inputs = synth.make_inputs(w)
+        T, B, I, H = w.T, w.B, w.I, w.H
+        if seq_mask:  # variable length: seeded per-sequence lengths in 0..T
+            self.inputs["mask"] = synth.length_mask(
+                T, B, H, synth.random_lengths(T, B, seed=w.seed), w.dtype)
+        self.d = {k: v.to(dev) for k, v in self.inputs.items()}
+        cd = synth.torch_dtype(w.dtype)
+        self.st = L.State(T, B, I, H, cd, dev)
+        self.gr = L.Grads(T, B, I, H, dev)
+        self.dims = self.st.dims
+        self.ws_f = L.empty_workspace(L.fwd_workspace_size(self.dims, self.d.get("mask")), dev)
+        self.ws_b = L.empty_workspace(L.bwd_workspace_size(self.dims), dev)
+        self.stream = torch.cuda.Stream(dev)
+        self.stream.wait_stream(torch.cuda.current_stream(dev))
+
+    def step(self, src=None, st=None, gr=None):
+        L, src = self.L, src if src is not None else self.d
+        st, gr = st or self.st, gr or self.gr
+        L.lstm_fwd(self.dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT,
+                   st.cT, st.gates, st.cells, self.ws_f, stream=self.stream, mask=src.get("mask"))
+        L.lstm_bwd(self.dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
+                   src["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0,
+                   self.ws_b, stream=self.stream, mask=src.get("mask"))
+
+    def check_status(self, where):
+        for ws in (self.ws_f, self.ws_b):
+            if self.L.lstm_status(ws, stream=self.stream) != self.L.LSTM_OK:
+                raise RuntimeError(f"device-side status set during {where}")
+
+    def timed(self, steps, warmup, barrier=lambda: None):
+        """Device time of `steps` steps after `warmup` untimed ones: (ms,
+        per-phase {name: (ms, launches)}, kernel launches)."""
+        L = self.L
+        with torch.cuda.stream(self.stream):
+            for _ in range(warmup):
+                self.step()
+        torch.cuda.synchronize(self.dev)
+        self.check_status("warm-up")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(self.dev)
+        n0 = L.launch_count()
+        L.profile_begin()
+        e0.record(self.stream)
+        with torch.cuda.stream(self.stream):
+            for _ in range(steps):
+                self.step()
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        phases = L.profile_end()
+        launches = L.launch_count() - n0
+        barrier()
+        self.check_status("the timed region")
+        return e0.elapsed_time(e1), phases, launches
+
+
+def config_line(w, ms, phases, steps, peak):
+    """Per-workload figures of one timed run: ms and timesteps/s per step,
+    TFLOP/s and its fraction of `peak`, and the device microseconds per
+    recurrent step of the forward and backward recurrences."""
+    step_s = ms / steps * 1e-3
+    tfl = w.flops / step_s / 1e12
+    us = lambda k: 1e3 * phases.get(k, (0.0, 0))[0] / steps / max(w.T, 1)
+    return {"T": w.T, "B": w.B, "I": w.I, "H": w.H, "dtype": w.dtype, "steps": steps,
+            "ms_per_step": ms / steps, "timesteps_per_s": w.rows / step_s, "tflops": tfl,
+            "frac_bf16_peak": tfl / peak,
+            "us_per_recurrent_step": {"fwd": us("fwd_recur"), "bwd": us("bwd_recur")},
+            "phases_ms_per_step": {p: v[0] / steps for p, v in phases.items() if v[1] > 0}}
+
+
 def run_ours(args, w, rank, world, local_rank):
     from backward_lstm_fwd_b200 import binding as L
     from backward_lstm_fwd_b200 import build as lbuild
@@ -225,28 +314,6 @@ def run_ours(args, w, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
 
-    inputs = synth.make_inputs(w)
-    T, B, I, H = w.T, w.B, w.I, w.H
-    if args.seq_mask:  # variable length: seeded per-sequence lengths in 0..T
-        inputs["mask"] = synth.length_mask(T, B, H, synth.random_lengths(T, B, seed=w.seed),
-                                           w.dtype)
-    d = {k: v.to(dev) for k, v in inputs.items()}
-    cd = synth.torch_dtype(w.dtype)
-    st = L.State(T, B, I, H, cd, dev)
-    gr = L.Grads(T, B, I, H, dev)
-    dims = st.dims
-    ws_f = L.empty_workspace(L.fwd_workspace_size(dims), dev)
-    ws_b = L.empty_workspace(L.bwd_workspace_size(dims), dev)
-    stream = torch.cuda.Stream(dev)
-    stream.wait_stream(torch.cuda.current_stream(dev))
-
-    def step(src):
-        L.lstm_fwd(dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT, st.cT,
-                   st.gates, st.cells, ws_f, stream=stream, mask=src.get("mask"))
-        L.lstm_bwd(dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
-                   src["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0,
-                   ws_b, stream=stream, mask=src.get("mask"))
-
     def barrier():
         if dist is not None:
             dist.barrier()
@@ -254,50 +321,34 @@ def run_ours(args, w, rank, world, local_rank):
     def max_over_ranks(v):
         return reduce_max(v, dist, dev)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step(d)
-    torch.cuda.synchronize(dev)
-    for ws in (ws_f, ws_b):
-        if L.lstm_status(ws, stream=stream) != L.LSTM_OK:
-            raise RuntimeError("device-side status set during warm-up")
+    pb = Problem(L, w, dev, seq_mask=args.seq_mask)
+    T, B, I, H = w.T, w.B, w.I, w.H
+    inputs, stream = pb.inputs, pb.stream
 
     # ---------------------------------------------------------- timed region
     clocks = ClockSampler(dev) if rank == 0 else None
     if clocks:
         clocks.start()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    n0 = L.launch_count()
-    L.profile_begin()
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            step(d)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    phases = L.profile_end()
-    launches = L.launch_count() - n0
-    barrier()
+    ms, phases, launches = pb.timed(args.steps, args.warmup, barrier)
     clk = clocks.stop() if clocks else None
-    ms = max_over_ranks(e0.elapsed_time(e1))
-    for ws in (ws_f, ws_b):
-        if L.lstm_status(ws, stream=stream) != L.LSTM_OK:
-            raise RuntimeError("device-side status set during the timed region")
+    ms = max_over_ranks(ms)
 
     # -------------------------------------------------- end to end (host I/O)
-    # Every step copies all of its inputs from pinned host memory and reads all
-    # of its gradients back.  Two device buffer sets and separate copy streams
-    # let step k+1's upload and step k-1's download run under step k's compute.
+    # Every step copies all of its inputs from pinned host memory and reads its
+    # results back: the forward's outputs (y, hT, cT) and every gradient.  Two
+    # device buffer sets and separate copy streams let step k+1's upload and
+    # step k-1's download run under step k's compute.
+    cd = synth.torch_dtype(w.dtype)
     pin_in = {k: v.pin_memory() for k, v in inputs.items()}
     dev_in = [{k: torch.empty_like(v, device=dev) for k, v in inputs.items()} for _ in range(2)]
-    grads = [gr, L.Grads(T, B, I, H, dev)]
-    out_names = ("dx", "dW", "db", "dh0", "dc0")
-    pin_out = [[torch.empty(getattr(g, n).shape, dtype=getattr(g, n).dtype, pin_memory=True)
-                for n in out_names] for g in grads]
+    states = [pb.st, L.State(T, B, I, H, cd, dev)]
+    grads = [pb.gr, L.Grads(T, B, I, H, dev)]
+    fwd_names, grad_names = ("y", "hT", "cT"), ("dx", "dW", "db", "dh0", "dc0")
+    results = [[getattr(states[i], n) for n in fwd_names] +
+               [getattr(grads[i], n) for n in grad_names] for i in range(2)]
+    pin_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in r] for r in results]
     h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
-    d2h = sum(getattr(gr, n).numel() * getattr(gr, n).element_size() for n in out_names)
+    d2h = sum(t.numel() * t.element_size() for t in results[0])
     s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()
     in_ready, in_free = [ev(), ev()], [ev(), ev()]
@@ -311,21 +362,15 @@ def run_ours(args, w, rank, world, local_rank):
                 dev_in[i][n].copy_(pin_in[n], non_blocking=True)
         in_ready[i].record(s_h2d)
         stream.wait_event(in_ready[i])
-        stream.wait_event(out_free[i])     # step k-2's gradients have been read back
+        stream.wait_event(out_free[i])     # step k-2's results have been read back
         with torch.cuda.stream(stream):
-            src = dev_in[i]
-            g = grads[i]
-            L.lstm_fwd(dims, src["x"], src["W"], src["b"], src["h0"], src["c0"], st.y, st.hT,
-                       st.cT, st.gates, st.cells, ws_f, stream=stream, mask=src.get("mask"))
-            L.lstm_bwd(dims, src["dy"], src["dhT"], src["dcT"], src["x"], src["W"], src["h0"],
-                       src["c0"], st.y, st.gates, st.cells, g.dx, g.dW, g.db, g.dh0, g.dc0,
-                       ws_b, stream=stream, mask=src.get("mask"))
+            pb.step(dev_in[i], states[i], grads[i])
         in_free[i].record(stream)
         out_ready[i].record(stream)
         s_d2h.wait_event(out_ready[i])
         with torch.cuda.stream(s_d2h):
-            for n, p in zip(out_names, pin_out[i]):
-                p.copy_(getattr(g, n), non_blocking=True)
+            for t, p in zip(results[i], pin_out[i]):
+                p.copy_(t, non_blocking=True)
         out_free[i].record(s_d2h)
 
     def e2e_run(nsteps):
@@ -347,10 +392,23 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     ms_e2e = max_over_ranks(f0.elapsed_time(f1))
 
+    # ------------------------------------- the other workloads (figures only)
+    per_config = {}
+    if not args.no_per_config and args.seq_len is None and not args.seq_mask:
+        for name, ow in synth.WORKLOADS.items():
+            if name == w.name:
+                continue
+            op = Problem(L, ow, dev)
+            osteps = max(3, min(args.steps, int(2000 // max(ow.T, 1))))
+            oms, oph, _ = op.timed(osteps, max(3, args.warmup), barrier)
+            per_config[name] = (ow, max_over_ranks(oms), oph, osteps)
+            del op
+
     if rank != 0:
         return 0
 
     peaks, peak_src = load_peaks()
+    tpeak, tpeak_kind = tensor_peak(peaks, clk)
     work = phase_work(w, phases)
     dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
     dom_ms, dom_launches = phases[dom]
@@ -358,9 +416,10 @@ def run_ours(args, w, rank, world, local_rank):
     amount *= args.steps  # work of the timed region
     if kind == "flop":
         achieved = amount / (dom_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": measured_traffic(dom, w.name)}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
+                "frac": achieved / tpeak, "traffic": measured_traffic(dom, w.name),
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS}
     else:
         achieved = amount / (dom_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
@@ -368,7 +427,9 @@ def run_ours(args, w, rank, world, local_rank):
                 "frac": achieved / peak, "traffic": None}
     roof.update({"kernel": dom, "launches_per_step": dom_launches / args.steps,
                  "ms_per_step": dom_ms / args.steps,
-                 "peak_source": f"{peak_src} ({'sustained bf16' if kind == 'flop' else 'HBM copy'})"})
+                 "us_per_recurrent_step": 1e3 * dom_ms / args.steps / max(T, 1)
+                 if dom in ("fwd_recur", "bwd_recur") else None,
+                 "peak_source": f"{peak_src} ({tpeak_kind if kind == 'flop' else 'HBM copy'})"})
     step_s = ms / args.steps * 1e-3
     value = job_throughput(world, w.rows, args.steps, ms)
     tflops = w.flops / step_s / 1e12
@@ -383,15 +444,22 @@ def run_ours(args, w, rank, world, local_rank):
         "tflops": tflops,
         "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
         "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
+        "pct_bf16_peak_nominal": 100.0 * tflops / NOMINAL_BF16_TFLOPS,
         "roofline": roof,
         "phases_ms_per_step": {p: v[0] / args.steps for p, v in phases.items()},
+        "us_per_recurrent_step": config_line(w, ms, phases, args.steps, tpeak)[
+            "us_per_recurrent_step"],
         "gpu_launches": launches,
         "e2e": {"value": job_throughput(world, w.rows, args.steps, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e / args.steps,
+                "read_back": list(fwd_names + grad_names),
                 "overlap": "uploads and read-backs on their own streams, two buffer sets"},
         "clocks": clk,
     }
+    if per_config:
+        line["per_config"] = {n: config_line(ow, oms, oph, ost, tpeak)
+                              for n, (ow, oms, oph, ost) in per_config.items()}
     if args.seq_mask:
         real = float(inputs["mask"][:, :, 0].float().mean())
         line["config"]["seq_mask"] = (f"per-sequence lengths uniform in 0..T (seeded), "
@@ -502,6 +570,7 @@ def run_stack(args, w, rank, world, local_rank):
         return 0
 
     peaks, peak_src = load_peaks()
+    tpeak, tpeak_kind = tensor_peak(peaks, clk)
     layer_w = [w] + [dataclasses.replace(w, I=H)] * (Lc - 1)
     works = [phase_work(lw, phases) for lw in layer_w]
     dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
@@ -510,9 +579,8 @@ def run_stack(args, w, rank, world, local_rank):
     amount = sum(wk[dom][1] for wk in works) * args.steps
     if kind == "flop":
         achieved = amount / (dom_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tpeak, "unit": "TFLOP/s",
+                "frac": achieved / tpeak, "traffic": None}
     else:
         achieved = amount / (dom_ms * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
@@ -520,7 +588,7 @@ def run_stack(args, w, rank, world, local_rank):
                 "frac": achieved / peak, "traffic": None}
     roof.update({"kernel": dom, "launches_per_step": dom_launches / args.steps,
                  "ms_per_step": dom_ms / args.steps,
-                 "peak_source": f"{peak_src} ({'sustained bf16' if kind == 'flop' else 'HBM copy'})"})
+                 "peak_source": f"{peak_src} ({tpeak_kind if kind == 'flop' else 'HBM copy'})"})
     step_s = ms / args.steps * 1e-3
     tflops = sum(lw.flops for lw in layer_w) / step_s / 1e12
     line = {
@@ -556,6 +624,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=synth.BENCH_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other four workloads (the per_config key)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override T (profiling aid: same per-step shape, fewer steps)")
     ap.add_argument("--dtype", choices=("bf16", "fp16"), default=None,

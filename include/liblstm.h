@@ -76,9 +76,26 @@ typedef struct lstm_dims {
 } lstm_dims;
 
 /* Workspace bytes lstm_fwd / lstm_bwd need for these dims (0 on invalid dims).
- * The workspace must be 256-byte aligned. */
+ * The workspace must be 256-byte aligned.
+ *
+ * The forward's size depends on the plan the call takes on the CURRENT device:
+ * when the fused forward kernel runs (the input projection contracted inside
+ * the recurrence: 16-bit compute types with H a multiple of 32, I a multiple
+ * of 8, and a grid that fits the device) it needs the 256-byte control block
+ * only; every other plan also needs the fp32 input projection Gx [T*B][4H].
+ *   lstm_fwd_workspace_size     the plan of a call with default options
+ *   lstm_fwd_workspace_size_ex  the plan of a call with these options (a
+ *                               seq_mask selects other kernel instantiations)
+ *   lstm_fwd_workspace_size_max enough for every plan on every device
+ * Without a usable device the first two return the _max size.  A forward call
+ * whose plan needs more than ws_bytes returns LSTM_ERR_WORKSPACE; if the fused
+ * kernel is planned but cannot be launched (LSTM_ERR_NOT_CORESIDENT inside the
+ * library), the call falls back to a Gx plan and returns LSTM_ERR_WORKSPACE
+ * when ws_bytes is below the _max size.  lstm_bwd_workspace_size does not
+ * depend on the device. */
 size_t lstm_fwd_workspace_size(const lstm_dims *d);
 size_t lstm_bwd_workspace_size(const lstm_dims *d);
+size_t lstm_fwd_workspace_size_max(const lstm_dims *d);
 
 /*
  * lstm_fwd -- forward pass ("SingleLayerLstmGrad", forward-formula table).
@@ -95,7 +112,7 @@ size_t lstm_bwd_workspace_size(const lstm_dims *d);
  *   gates [T][B][4H]  compute type  post-activation i,f,g,o of every step, kept
  *                                    for lstm_bwd (the page's i, j, f, o inputs)
  *   cells [T][B][H]   float         c_t of every step, kept for lstm_bwd
- *   ws / ws_bytes                   scratch, >= lstm_fwd_workspace_size(d)
+ *   ws / ws_bytes                   scratch, >= lstm_fwd_workspace_size(d) (see there)
  *
  * y, gates and cells must stay unchanged until the matching lstm_bwd has run.
  * Returns LSTM_OK or an LSTM_ERR_* code.
@@ -184,6 +201,7 @@ typedef struct {
     int gate_order;
 } lstm_options;
 
+size_t lstm_fwd_workspace_size_ex(const lstm_dims *d, const lstm_options *opt);
 int lstm_fwd_ex(const lstm_dims *d, const lstm_options *opt, const void *x, const void *W,
                 const void *b, const void *h0, const float *c0, void *y, void *hT, float *cT,
                 void *gates, float *cells, void *ws, size_t ws_bytes, void *stream);
@@ -225,6 +243,8 @@ int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, con
  * layer l's dx rounded to the compute type.  ws at least
  * lstm_stack_bwd_workspace_size(d, L) bytes.  The layers run L-1 .. 0.
  */
+/* (The stack's forward workspace covers every plan of every layer, like
+ * lstm_fwd_workspace_size_max.) */
 size_t lstm_stack_fwd_workspace_size(const lstm_dims *d, int L);
 size_t lstm_stack_bwd_workspace_size(const lstm_dims *d, int L);
 int lstm_stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
@@ -283,32 +303,40 @@ long long lstm_launch_count(void);
  * every GPU on which the library is loaded holds that buffer until the
  * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
  *
- *   - Problems whose lstm_fwd_workspace_size() exceeds
+ *   - Problems whose lstm_fwd_workspace_size() on the current device exceeds
  *     LSTM_NOALLOC_SCRATCH_BYTES are rejected with LSTM_ERR_UNSUPPORTED
- *     before anything is enqueued.
+ *     before anything is enqueued.  (Where the fused forward kernel runs the
+ *     call needs only the 256-byte control block, at any T and B; other plans
+ *     need T*B*4H floats of Gx as well.)
  *   - The first call on a device (the current device) looks up that device's
- *     address of the buffer; make that first call before any stream capture.
+ *     address of the buffer and keeps it for the life of the process; make
+ *     that first call before any stream capture, and do not use this entry
+ *     point across a cudaDeviceReset of that device (the kept address would
+ *     then be stale).
  *   - All calls share the one buffer per device, which keeps the previous
  *     call's contents; each call clears the parts that must start at zero (the
- *     status word and barrier counters).  Calls whose executions overlap on the
- *     GPU (different streams, or different host threads) race on the buffer:
- *     serialise them.
- *   - The status word lives in the shared buffer, so lstm_status cannot be
- *     used with this entry point; callers that need device-side status use
- *     lstm_fwd with their own workspace.
+ *     status word and barrier counters), after its arguments are checked and
+ *     in stream order.  Calls whose executions overlap on the GPU (different
+ *     streams, or different host threads) race on the buffer: serialise them.
+ *   - lstm_fwd_noalloc_status(stream) synchronises `stream` and reads and
+ *     clears the buffer's status word on the current device, like lstm_status
+ *     does for a caller workspace: it reports a device-side wait that gave up
+ *     (LSTM_ERR_TIMEOUT) in the most recent call.
  * Returns LSTM_OK or an LSTM_ERR_* code, like lstm_fwd.
  */
 #define LSTM_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int lstm_fwd_noalloc(const lstm_dims *d, const void *x, const void *W, const void *b,
                      const void *h0, const float *c0, void *y, void *hT, float *cT,
                      void *gates, float *cells, void *stream);
+int lstm_fwd_noalloc_status(void *stream);
 
 /* Static description of a status code. */
 const char *lstm_strerror(int code);
 
 /* ABI version: 100 * major + minor (1.1: lstm_options with gate_order, the
- * LSTM_F16 compute type and the stack entry points). */
-#define LSTM_ABI_VERSION 101
+ * LSTM_F16 compute type and the stack entry points; 1.2: the plan-aware
+ * forward workspace sizes and lstm_fwd_noalloc_status). */
+#define LSTM_ABI_VERSION 102
 int lstm_abi_version(void);
 
 #ifdef __cplusplus

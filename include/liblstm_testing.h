@@ -8,6 +8,32 @@
 
 #include <stddef.h>
 
+/*
+ * Environment variables.  The library reads exactly these, at every call
+ * (nothing is cached); each is unset by default, and any other value than
+ * the one shown means "unset".  They exist for tests, comparison runs and
+ * profiling, never for results: every setting gives results within the same
+ * tolerance.
+ *
+ *   LSTM_FORCE_SIMT=1      run every step on the CUDA-core kernels (no tensor
+ *                          cores, no persistent kernels).
+ *   LSTM_FWD_FUSED_X=0     do not run the forward kernel with the input
+ *                          projection fused into the recurrence; the forward
+ *                          then needs the Gx workspace
+ *                          (lstm_fwd_workspace_size_max).
+ *   LSTM_BWD_TMEM_W=0      do not run the backward kernel with W_h^T in tensor
+ *                          memory (the older cluster kernels run instead).
+ *   LSTM_BWD_CHUNKS=n      run the tensor-core backward recurrence in n
+ *                          reverse-time chunks (1..16; 1 = one launch, dW / dx
+ *                          after it).  Default: min(8, T / 16), 1 below T = 32.
+ *   LSTM_LAUNCH_NONCOOP=1  launch the persistent cluster kernels without the
+ *                          cooperative attribute, after the same co-residency
+ *                          check (profilers cannot replay cooperative cluster
+ *                          launches).  Taken automatically when a CUDA
+ *                          injection library is attached
+ *                          (CUDA_INJECTION64_PATH set: a profiler or sanitizer).
+ */
+
 #ifdef __cplusplus
 extern "C" {
 #endif

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from backward_lstm_fwd_b200 import build as lbuild
 from backward_lstm_fwd_b200 import binding as L
@@ -34,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) >= set(L.EXPORTS)
     for n in names:
         assert hasattr(lib, n), f"{n} declared in liblstm.h but not exported"
-    assert lib.lstm_abi_version() == L.ABI_VERSION == 101
+    assert lib.lstm_abi_version() == L.ABI_VERSION == 102
 
 
 def declared_arities():
@@ -68,16 +69,26 @@ def test_strerror(lib):
 
 def test_workspace_sizes(lib):
     d = L.dims(256, 128, 1024, 1024, L.LSTM_BF16)
-    fw, bw = L.fwd_workspace_size(d), L.bwd_workspace_size(d)
+    fmax, bw = L.fwd_workspace_size_max(d), L.bwd_workspace_size(d)
     TB, G4 = 256 * 128, 4 * 1024
-    assert fw >= 256 + TB * G4 * 4 and fw % 256 == 0
+    assert fmax >= 256 + TB * G4 * 4 and fmax % 256 == 0
     assert bw >= 256 + TB * G4 * 2 and bw % 256 == 0
-    assert L.fwd_workspace_size(L.dims(-1, 2, 3, 4, 0)) == 0
+    # the plan-aware size: the control block alone (fused forward on a device
+    # where it fits) or the whole layout; without a device, the whole layout
+    fw = L.fwd_workspace_size(d)
+    assert fw in (256, fmax)
+    if not torch.cuda.is_available():
+        assert fw == fmax
+    mask_opt = L.Options(FAKE, L.LSTM_DIR_FORWARD, L.LSTM_GATES_IFJO)
+    assert lib.lstm_fwd_workspace_size_ex(ctypes.byref(d), ctypes.byref(mask_opt)) in (256, fmax)
+    assert lib.lstm_fwd_workspace_size_ex(ctypes.byref(d), None) == fw
+    for q in (L.fwd_workspace_size, L.fwd_workspace_size_max):
+        assert q(L.dims(-1, 2, 3, 4, 0)) == 0
+        assert q(L.dims(0, 0, 0, 0, 0)) >= 256
     assert L.bwd_workspace_size(L.dims(1, 2, 3, 4, 7)) == 0
-    assert L.fwd_workspace_size(L.dims(0, 0, 0, 0, 0)) >= 256
     # fp16 has bf16's layout (two-byte dG, W_h^T, per-group db partials)
     h = L.dims(256, 128, 1024, 1024, L.LSTM_F16)
-    assert L.fwd_workspace_size(h) == fw and L.bwd_workspace_size(h) == bw
+    assert L.fwd_workspace_size_max(h) == fmax and L.bwd_workspace_size(h) == bw
     # fp32 keeps dG in fp32 and needs no W_h^T copy
     f = L.dims(256, 128, 1024, 1024, L.LSTM_F32)
     assert L.bwd_workspace_size(f) >= 256 + TB * G4 * 4
@@ -260,7 +271,7 @@ def call_stack_bwd(d, Lc, Ws=(FAKE, FAKE), dWs=(FAKE, FAKE), dbs=(FAKE, FAKE), w
 def test_stack_workspace_sizes(lib):
     one = L.bwd_workspace_size(DS)
     upper = L.bwd_workspace_size(L.dims(4, 8, 32, 32, L.LSTM_BF16))
-    assert L.stack_fwd_workspace_size(DS, 1) == L.fwd_workspace_size(DS)
+    assert L.stack_fwd_workspace_size(DS, 1) == L.fwd_workspace_size_max(DS)
     assert L.stack_bwd_workspace_size(DS, 1) == one
     # two layers: the larger layer's workspace plus dx (float) and dy (bf16)
     # of the upper layer, [T][B][H] each
@@ -342,3 +353,14 @@ def test_backward_chunking_host_logic(lib, monkeypatch):
     assert [lib.lstm_test_chunk_bound(256, 8, c) for c in range(9)] == \
         [0, 62, 111, 150, 182, 207, 227, 243, 256]
     assert lib.lstm_test_chunk_bound(10, 2, 3) == -1  # c > nch
+
+
+def test_environment_switches_are_the_documented_ones():
+    """Every environment variable the library reads is listed in
+    liblstm_testing.h, and every listed one is read."""
+    src = open(os.path.join(ROOT, "backward_lstm_fwd_b200", "csrc", "liblstm.cu")).read()
+    read = set(re.findall(r'(?:getenv|env_is)\("([A-Z0-9_]+)"', src))
+    hdr = open(HEADER.replace("liblstm.h", "liblstm_testing.h")).read()
+    listed = set(re.findall(r"^ \*   (LSTM_[A-Z0-9_]+)=", hdr, flags=re.M))
+    listed.add("CUDA_INJECTION64_PATH")
+    assert read == listed, (sorted(read), sorted(listed))

@@ -1,6 +1,7 @@
 """CUDA path vs the fp64 oracle, element by element, through the C ABI.
 
-Full-size runs of the five workloads (the launch configuration bench.py times),
+Full-size runs of the five workloads on the whole batch (the launch
+configuration bench.py times), a long sequence with upstream gradient on every step,
 odd shapes that leave ragged tiles, and the degenerate cases (empty sequence or
 batch, no input features, absent optional inputs).  Tolerance per output
 tensor: max|gpu - ref| / max|ref| <= 1e-4 (fp32), 2e-2 (bf16) or 2.5e-3 (fp16)."""
@@ -10,17 +11,14 @@ import torch
 
 from backward_lstm_fwd_b200 import binding as L
 from backward_lstm_fwd_b200 import synth
-from tests.parity_util import (OUTS, TOL, assert_within, compare, mask_upstream, rel_err,
-                               run_gpu, run_oracle)
+from tests.parity_util import OUTS, assert_within, compare, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
-# Workloads small enough for the full oracle; the other two are checked on
-# sampled sequences (all per-sequence outputs) plus a masked-gradient run that
-# makes dW and db checkable on the same sample.
-FULL = ["lstm_T8_B2_I16_H32_fp32", "lstm_T64_B32_I256_H256_fp32", "lstm_T128_B64_I512_H512_bf16"]
-SAMPLED = {"lstm_T256_B128_I1024_H1024_bf16": [0, 37, 101, 127],
-           "lstm_T1024_B16_I256_H1024_bf16": [0, 11]}
+# The five workloads, full size, every output tensor against the oracle on the
+# whole batch (the two largest take the oracle about 20-40 s on 16 host cores).
+FULL = ["lstm_T8_B2_I16_H32_fp32", "lstm_T64_B32_I256_H256_fp32", "lstm_T128_B64_I512_H512_bf16",
+        "lstm_T256_B128_I1024_H1024_bf16", "lstm_T1024_B16_I256_H1024_bf16"]
 
 
 # recurrent kernel each workload must run on (see lstm_test_last_paths)
@@ -41,22 +39,19 @@ def test_workload_full(name, cuda_device):
     assert_within(errs, w.dtype, name)
 
 
-@pytest.mark.parametrize("name", sorted(SAMPLED))
-def test_workload_sampled(name, cuda_device):
-    w = synth.WORKLOADS[name]
-    idx = SAMPLED[name]
+def test_long_sequence_dense_upstream(cuda_device):
+    """The T = 1024, B = 16, I = 256, H = 1024 shape with dy drawn on every
+    step: dh0 and dc0 are then O(1), so the whole 1024-step delta h / delta c
+    carry down to t = 0 is checked at the bf16 tolerance (the workload itself
+    has dy only on its last 64 steps, which leaves dh0 / dc0 near 1e-189)."""
+    w = synth.custom(1024, 16, 256, 1024, "bf16", seed=41)
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
-    assert L.test_last_paths() == EXPECTED_PATHS[name]
-    ref = run_oracle(synth.select_sequences(inp, idx))
-    errs = compare(gpu, ref, w.dtype, ("y", "hT", "cT", "dx", "dh0", "dc0"), idx=idx)
-    assert_within(errs, w.dtype, name + " per-sequence")
-    # dW, db: only the sampled sequences carry upstream gradient
-    masked = mask_upstream(inp, idx)
-    gpu_m = run_gpu(masked, cuda_device)
-    ref_m = run_oracle(synth.select_sequences(masked, idx))
-    errs = compare(gpu_m, ref_m, w.dtype, ("dW", "db"))
-    assert_within(errs, w.dtype, name + " dW/db")
+    assert L.test_last_paths() == (3, 3)
+    ref = run_oracle(inp)
+    for k in ("dh0", "dc0"):
+        assert float(np.max(np.abs(ref[k]))) > 1e-3, (k, float(np.max(np.abs(ref[k]))))
+    assert_within(compare(gpu, ref, "bf16", OUTS + ("gates", "cells")), "bf16", w.name)
 
 
 ODD = [
