@@ -21,6 +21,7 @@
 #include "tc_recur.cuh"
 #include "tc_recur2.cuh"
 #include "tc_recur3.cuh"
+#include "tc_recur4.cuh"
 
 using namespace lstm;
 
@@ -74,10 +75,12 @@ struct Phase {
 //   LSTM_FORCE_SIMT=1      CUDA-core kernels only
 //   LSTM_FWD_FUSED_X=0     no fused forward kernel (the Gx plans)
 //   LSTM_BWD_TMEM_W=0      no backward kernel with the weights in tensor memory
+//   LSTM_BWD_STREAMS=1     that backward with one batch stream per group
 //   LSTM_BWD_CHUNKS=n      reverse-time chunks of the overlapped backward
 //   LSTM_LAUNCH_NONCOOP=1  cluster launches without the cooperative attribute
-//                          (also taken when a CUDA injection library -- a
-//                          profiler or sanitizer -- is attached)
+//                          (also taken when a profiler or sanitizer is attached:
+//                          NV_COMPUTE_PROFILER_PERFWORKS_DIR or
+//                          CUDA_INJECTION64_PATH set)
 bool env_is(const char *name, char value) {
     const char *e = getenv(name);
     return e && e[0] == value && e[1] == '\0';
@@ -520,6 +523,7 @@ struct Rec2Plan {
     int kcx;  // fused forward: K chunks of x per CTA
     size_t smem;
     int split = 1;  // fused forward: batch streams per cluster (NB rows each)
+    int family = 3; // backward with the weights in TMEM: 3, or 4 with two stream agents each
 };
 
 int max_active_clusters(const void *kern, int threads, size_t smem, int KS) {
@@ -654,6 +658,7 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
             if (G * P.R > maxc) continue;
             P.KS = KS; P.G = G; P.NB = NBv; P.kcc = kcc; P.kcx = kcx; P.smem = smem;
             P.split = split;
+            P.family = 3;
             return true;
         }
     }
@@ -729,6 +734,46 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     if (P.G > gmax) return false;
     P.stages = stages;
     P.NB = NB;
+    P.family = 3;
+    return true;
+}
+
+// Backward with two decoupled batch streams per group (rec4): the grid of
+// plan_bwd3 with groups of a multiple of 32 rows (two streams of a multiple of
+// 16), 384 threads, and each stream's ring staging its send blocks.
+bool plan_bwd4(const lstm_dims *d, Rec2Plan &P) {
+    if (env_is("LSTM_BWD_TMEM_W", '0') || env_is("LSTM_BWD_STREAMS", '1')) return false;
+    if (d->dtype == LSTM_F32 || d->H % rec4::UNITS != 0 || d->B < 1 ||
+        tcg::encode_fn() == nullptr || force_simt())
+        return false;
+    P.KS = rec4::KS;
+    P.R = d->H / rec4::UNITS;
+    P.kcc = 4 * d->H / rec4::KS / 64;
+    if (rec4::W_COL + (uint32_t)(P.kcc * 32) > rec4::TMEM_COLS) return false;
+    int stages = std::min(P.kcc, rec4::MAX_STAGES);
+    while (stages >= rec4::MIN_STAGES && (size_t)rec4::Bwd4Smem(stages).total + 1024 > kMaxSmem)
+        --stages;
+    if (stages < rec4::MIN_STAGES) return false;
+    P.smem = rec4::Bwd4Smem(stages).total + 1024;
+    const void *kern = d->dtype == LSTM_F16 ? (const void *)rec4::bwd4_kernel<__half, false, false>
+                                            : (const void *)rec4::bwd4_kernel<bf16, false, false>;
+    const int maxc = max_active_clusters(kern, rec4::THREADS, P.smem, P.KS);
+    const int gmax = std::min(maxc / P.R, kMaxGroups / rec4::NSTREAM);
+    if (gmax < 1) return false;
+    const int rows_max = rec4::NSTREAM * rec4::NBS_MAX;
+    int G = std::min(gmax, (d->B + 31) / 32);
+    int NB = ((d->B + G - 1) / G + 31) / 32 * 32;
+    if (NB > rows_max) {
+        G = (d->B + rows_max - 1) / rows_max;
+        NB = ((d->B + G - 1) / G + 31) / 32 * 32;
+    }
+    P.G = (d->B + NB - 1) / NB;
+    if (P.G > gmax) return false;
+    // both streams of every group hold rows (else the one-stream kernel serves)
+    if (d->B <= (NB / 2) * (2 * P.G - 1)) return false;
+    P.stages = stages;
+    P.NB = NB;
+    P.family = 4;
     return true;
 }
 
@@ -756,11 +801,13 @@ cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t s
     cfg.attrs = at;
     cfg.numAttrs = 2;
     // Profilers cannot replay a cooperative cluster launch: with
-    // LSTM_LAUNCH_NONCOOP=1, or when a CUDA injection library (a profiler or
-    // a sanitizer) is attached, go straight to the occupancy-checked cluster
-    // launch below.
+    // LSTM_LAUNCH_NONCOOP=1, or when a profiler or sanitizer is attached
+    // (Nsight Compute sets NV_COMPUTE_PROFILER_PERFWORKS_DIR in the profiled
+    // process; tools that inject through CUDA_INJECTION64_PATH set that),
+    // go straight to the occupancy-checked cluster launch below.
     const char *inj = getenv("CUDA_INJECTION64_PATH");
-    const bool noncoop = env_is("LSTM_LAUNCH_NONCOOP", '1') || (inj && inj[0]);
+    const char *ncu = getenv("NV_COMPUTE_PROFILER_PERFWORKS_DIR");
+    const bool noncoop = env_is("LSTM_LAUNCH_NONCOOP", '1') || (inj && inj[0]) || (ncu && ncu[0]);
     if (!noncoop) {
         e = cudaLaunchKernelEx(&cfg, kern, prm);
         if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) {
@@ -959,6 +1006,63 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *
     return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
+// One launch of the two-stream backward kernel over epilogue iterations
+// [i0, i1); WT must already hold W_h^T.
+template <class E>
+int tc_bwd4_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *dhT,
+                   const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
+                   const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
+                   float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0,
+                   int i1, cudaStream_t s) {
+    const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
+    rec4::Bwd4Params<E> prm;
+    memset(&prm, 0, sizeof(prm));
+    const int NBS = P.NB / rec4::NSTREAM;
+    if (!tcg::make_map(&prm.map_dg, dG, G4, T * B, G4 * 2, 64, NBS,
+                       tcg::map_type(Elem<E>::kFmt)))
+        return LSTM_ERR_UNSUPPORTED;
+    prm.wt = WT;
+    prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.dcT = dcT; prm.cells = cells;
+    prm.c0 = c0; prm.dG = dG; prm.dh0 = dh0; prm.dc0 = dc0; prm.db_part = dbgroup;
+    prm.dc_carry = dc_carry;
+    prm.mask = mask; prm.dhp_carry = dhp_carry;
+    prm.ctrl = ctrl;
+    prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
+    prm.NBS = NBS; prm.kcc = P.kcc; prm.stages = P.stages;
+    prm.i0 = i0; prm.i1 = i1; prm.reverse = reverse;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const int nctas = P.R * P.KS * P.G;
+    const cudaError_t e =
+        mask ? (ijfo ? launch_cluster(rec4::bwd4_kernel<E, true, true>, prm, nctas, P.KS, P.smem,
+                                      s, rec4::THREADS)
+                     : launch_cluster(rec4::bwd4_kernel<E, true, false>, prm, nctas, P.KS, P.smem,
+                                      s, rec4::THREADS))
+             : (ijfo ? launch_cluster(rec4::bwd4_kernel<E, false, true>, prm, nctas, P.KS, P.smem,
+                                      s, rec4::THREADS)
+                     : launch_cluster(rec4::bwd4_kernel<E, false, false>, prm, nctas, P.KS,
+                                      P.smem, s, rec4::THREADS));
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+// One launch of the TMEM-weight backward family the plan names.
+template <class E>
+int tc_bwd_tmem_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *dhT,
+                       const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
+                       const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
+                       float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl,
+                       int i0, int i1, cudaStream_t s) {
+    if (P.family == 4)
+        return tc_bwd4_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
+                              dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s);
+    return tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
+                          dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s);
+}
+
 // W_h^T of a 16-bit W (bf16 or fp16: the kernel only moves 16-bit values)
 cudaError_t launch_transpose_wh(const lstm_dims *d, const void *W_, void *WT_, cudaStream_t s) {
     const bf16 *W = static_cast<const bf16 *>(W_);
@@ -981,8 +1085,9 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *dy, const
                        cudaStream_t s) {
     const long long G4 = 4LL * d->H;
     if (launch_transpose_wh(d, W, WT, s) != cudaSuccess) return LSTM_ERR_CUDA;
-    const int rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG,
-                                  WT, dbgroup, dh0, dc0, nullptr, nullptr, ctrl, 0, d->T, s);
+    const int rc = tc_bwd_tmem_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells,
+                                      dG, WT, dbgroup, dh0, dc0, nullptr, nullptr, ctrl, 0, d->T,
+                                      s);
     if (rc != LSTM_OK) return rc;
     simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, s>>>(dbgroup, P.G, (int)G4, db);
     note_launch();
@@ -1022,8 +1127,9 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
         if (launch_transpose_wh(d, W, WT, A.rec) != cudaSuccess) rc = LSTM_ERR_CUDA;
         for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
             const int i0 = chunk_bound(T, nch, c), i1 = chunk_bound(T, nch, c + 1);
-            rc = tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
-                                dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, A.rec);
+            rc = tc_bwd_tmem_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG,
+                                    WT, dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1,
+                                    A.rec);
             if (rc != LSTM_OK) break;
             if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
                 cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess) {
@@ -1180,7 +1286,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
 
     RecPlan plan;
     Rec2Plan plan2, plan3;
-    const bool v3 = plan_bwd3(d, plan3);
+    const bool v3 = plan_bwd4(d, plan3) || plan_bwd3(d, plan3);
     const bool v2 = !v3 && !special && plan_bwd2(d, plan2);
     const bool v1 = !special && plan_bwd_recur(d, plan);
     bool per_step = false;  // a special call whose cluster kernel cannot be placed
@@ -1188,7 +1294,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         if (v3 && tc_gemm_ok(d) && bwd_chunks(d) > 1) {
             AuxStreams *A = aux_streams();
             if (A) {  // a3 + a5 with a4 + a6 overlapped
-                g_last_bwd_path = 3;
+                g_last_bwd_path = plan3.family;
                 const int rc = tc_bwd3_overlapped(
                     d, plan3, *A, bwd_chunks(d), (const E *)dy, (const E *)dhT, dcT,
                     (const E *)x, (const E *)W, (const E *)h0, c0, (const E *)mask,
@@ -1201,7 +1307,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         {   // a3 + a5: persistent tcgen05 recurrence with db fused
             prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
             int rc = LSTM_ERR_NOT_CORESIDENT;
-            g_last_bwd_path = v3 ? 3 : 2;
+            g_last_bwd_path = v3 ? plan3.family : 2;
             if (v3)
                 rc = tc_bwd_recurrence3(d, plan3, (const E *)dy, (const E *)dhT, dcT,
                                         (const E *)W, c0, (const E *)mask, reverse, ijfo,

@@ -23,15 +23,19 @@
  *                          (lstm_fwd_workspace_size_max).
  *   LSTM_BWD_TMEM_W=0      do not run the backward kernel with W_h^T in tensor
  *                          memory (the older cluster kernels run instead).
+ *   LSTM_BWD_STREAMS=1     run that backward kernel with one batch stream per
+ *                          group instead of two decoupled streams.
  *   LSTM_BWD_CHUNKS=n      run the tensor-core backward recurrence in n
  *                          reverse-time chunks (1..16; 1 = one launch, dW / dx
  *                          after it).  Default: min(8, T / 16), 1 below T = 32.
  *   LSTM_LAUNCH_NONCOOP=1  launch the persistent cluster kernels without the
  *                          cooperative attribute, after the same co-residency
  *                          check (profilers cannot replay cooperative cluster
- *                          launches).  Taken automatically when a CUDA
- *                          injection library is attached
- *                          (CUDA_INJECTION64_PATH set: a profiler or sanitizer).
+ *                          launches).  Taken automatically when a profiler
+ *                          or sanitizer is attached: Nsight Compute sets
+ *                          NV_COMPUTE_PROFILER_PERFWORKS_DIR in the profiled
+ *                          process, injection-based tools set
+ *                          CUDA_INJECTION64_PATH.
  */
 
 #ifdef __cplusplus
@@ -69,7 +73,9 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
  * grid), 1 = persistent kernel with K resident per CTA, 2 = persistent cluster
  * kernel with K split across the CTAs of a cluster, 3 = the cluster kernel
  * with the weights held in tensor memory (forward: with the input projection
- * contracted inside the recurrence); -1 = none yet.
+ * contracted inside the recurrence), 4 = (backward) that kernel with two
+ * batch streams per group, each with its own TMA producer, MMA issuer and
+ * epilogue warpgroup; -1 = none yet.
  */
 int lstm_test_last_paths(int *fwd_path, int *bwd_path);
 

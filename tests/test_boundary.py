@@ -362,5 +362,5 @@ def test_environment_switches_are_the_documented_ones():
     read = set(re.findall(r'(?:getenv|env_is)\("([A-Z0-9_]+)"', src))
     hdr = open(HEADER.replace("liblstm.h", "liblstm_testing.h")).read()
     listed = set(re.findall(r"^ \*   (LSTM_[A-Z0-9_]+)=", hdr, flags=re.M))
-    listed.add("CUDA_INJECTION64_PATH")
+    listed |= {"CUDA_INJECTION64_PATH", "NV_COMPUTE_PROFILER_PERFWORKS_DIR"}
     assert read == listed, (sorted(read), sorted(listed))

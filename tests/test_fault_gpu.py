@@ -4,8 +4,9 @@ record LSTM_ERR_TIMEOUT in the workspace status word (read by lstm_status), and
 leave the context usable -- the next normal call succeeds and matches the
 oracle.  Covered for the K-resident kernels (H = 64), the cluster kernels
 (H = 256: forward clusters of 4, backward clusters of 8), the backward
-cluster kernel with the weights in tensor memory (H = 512, 1024), and the
-fused forward with one and with two batch streams per cluster."""
+cluster kernel with the weights in tensor memory with two decoupled batch
+streams per group (H = 512, 1024) and with one (forced), and the fused
+forward with one and with two batch streams per cluster."""
 import pytest
 import torch
 
@@ -17,13 +18,16 @@ from tests.parity_util import assert_within, compare, run_gpu, run_oracle
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("H,T,B", [(64, 6, 32), (256, 6, 32), (512, 6, 32), (512, 40, 32),
-                                   (512, 6, 128), (1024, 6, 128)])
-def test_missing_arrival_times_out_and_recovers(H, T, B, cuda_device):
+@pytest.mark.parametrize("H,T,B,streams", [(64, 6, 32, 2), (256, 6, 32, 2), (512, 6, 32, 2),
+                                           (512, 40, 32, 2), (512, 6, 128, 2), (1024, 6, 128, 2),
+                                           (1024, 40, 128, 1)])
+def test_missing_arrival_times_out_and_recovers(H, T, B, streams, cuda_device, monkeypatch):
     """T = 40 runs the backward in reverse-time chunks with dW / dx beside them;
     B = 128 runs the forward with two interleaved batch streams per cluster (at
     H = 1024 with the bench workload's cluster grid)."""
     lbuild.build()
+    if streams == 1:
+        monkeypatch.setenv("LSTM_BWD_STREAMS", "1")
     w = synth.custom(T, B, 64, H, "bf16", seed=11)
     inp = {k: v.to(cuda_device) for k, v in synth.make_inputs(w).items()}
     I = w.I
@@ -40,7 +44,7 @@ def test_missing_arrival_times_out_and_recovers(H, T, B, cuda_device):
         L.lstm_bwd(st.dims, inp["dy"], inp["dhT"], inp["dcT"], inp["x"], inp["W"], inp["h0"],
                    inp["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0, wsb)
         assert L.lstm_status(wsb) == L.LSTM_ERR_TIMEOUT
-        assert L.test_last_paths()[1] == {64: 1, 256: 2, 512: 3, 1024: 3}[H]
+        assert L.test_last_paths()[1] == {64: 1, 256: 2, 512: 4, 1024: 4 if streams == 2 else 3}[H]
     finally:
         L.test_set_wait_fault(-1, 0)
     # the context is still usable and the next call is correct

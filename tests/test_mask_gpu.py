@@ -21,7 +21,7 @@ CASES = {
     (7, 5, 37, 45, "bf16"): (0, 0),       # per-step kernels, bf16 off the tensor-core grid
     (10, 24, 64, 256, "bf16"): (3, 0),    # fused forward; per-step backward
     (12, 48, 64, 512, "bf16"): (3, 3),    # TMEM-weight kernels, one launch each
-    (40, 64, 96, 512, "bf16"): (3, 3),    # backward in 2 chunks, dW / dx beside
+    (40, 64, 96, 512, "bf16"): (3, 4),    # backward in 2 chunks, two batch streams
     (64, 200, 96, 512, "bf16"): (3, 3),   # ragged batch groups, backward in 4 chunks
 }
 

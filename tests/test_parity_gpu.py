@@ -23,8 +23,8 @@ FULL = ["lstm_T8_B2_I16_H32_fp32", "lstm_T64_B32_I256_H256_fp32", "lstm_T128_B64
 
 # recurrent kernel each workload must run on (see lstm_test_last_paths)
 EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (0, 0), "lstm_T64_B32_I256_H256_fp32": (0, 0),
-                  "lstm_T128_B64_I512_H512_bf16": (3, 3),
-                  "lstm_T256_B128_I1024_H1024_bf16": (3, 3),
+                  "lstm_T128_B64_I512_H512_bf16": (3, 4),
+                  "lstm_T256_B128_I1024_H1024_bf16": (3, 4),
                   "lstm_T1024_B16_I256_H1024_bf16": (3, 3)}
 
 
@@ -47,7 +47,7 @@ def test_long_sequence_dense_upstream(cuda_device):
     w = synth.custom(1024, 16, 256, 1024, "bf16", seed=41)
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
-    assert L.test_last_paths() == (3, 3)
+    assert L.test_last_paths() == (3, 3)  # 16 rows: one batch stream
     ref = run_oracle(inp)
     for k in ("dh0", "dc0"):
         assert float(np.max(np.abs(ref[k]))) > 1e-3, (k, float(np.max(np.abs(ref[k]))))
@@ -70,14 +70,21 @@ ODD = [
     (4, 6, 37, 48, "bf16"), (4, 6, 37, 64, "bf16"),
     # the forward with two batch streams per cluster at its shortest sequences
     (1, 200, 96, 512, "bf16"), (2, 100, 64, 1024, "bf16"),
+    # the backward with two batch streams per group: a ragged last stream
+    # (rows 112..119 of 4 groups of 32), a ragged second stream of one group
+    # of 128, and H = 1536, whose 12 K chunks per step wrap around an
+    # 8-stage ring per stream
+    (5, 120, 96, 512, "bf16"), (3, 100, 64, 1024, "bf16"), (3, 64, 64, 1536, "bf16"),
 ]
 
 
 # recurrent kernels of the odd bf16 shapes above (see lstm_test_last_paths):
 # the forward with the input projection fused wherever H is a multiple of 32
-# (clusters of 4, 2 and 1 among these), the backward with the weights in TMEM
+# (clusters of 4, 2 and 1 among these), the backward with the weights in TMEM,
+# keyed by (B, H)
 ODD_FWD_PATH = {64: 3, 128: 3, 256: 3, 512: 3, 640: 3, 1024: 3, 1536: 3}
-ODD_BWD_PATH = {512: 3, 640: 3, 1536: 3}
+ODD_BWD_PATH = {(200, 512): 3, (37, 640): 3, (16, 1536): 3, (120, 512): 4, (100, 1024): 4,
+                (64, 1536): 4}
 
 
 @pytest.mark.parametrize("T,B,I,H,dt", ODD)
@@ -89,8 +96,8 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
         assert L.test_last_paths()[0] == 0
     elif dt == "bf16" and H in ODD_FWD_PATH:
         assert L.test_last_paths()[0] == ODD_FWD_PATH[H]
-    if dt == "bf16" and H in ODD_BWD_PATH:
-        assert L.test_last_paths()[1] == ODD_BWD_PATH[H]
+    if dt == "bf16" and (B, H) in ODD_BWD_PATH:
+        assert L.test_last_paths()[1] == ODD_BWD_PATH[(B, H)]
     ref = run_oracle(inp)
     assert_within(compare(gpu, ref, dt), dt, w.name)
 
@@ -149,12 +156,32 @@ def test_side_stream_and_repeat(cuda_device):
 
 
 @pytest.mark.parametrize("chunks", ["1", "3", "5"])
-def test_backward_chunk_counts(chunks, cuda_device, monkeypatch):
+@pytest.mark.parametrize("B,path", [(40, 3), (64, 4)])
+def test_backward_chunk_counts(chunks, B, path, cuda_device, monkeypatch):
     """The backward in 1 (one launch, no overlap), 3 or 5 reverse-time chunks
-    (dW / dx of each chunk beside the next one) gives the oracle's gradients."""
+    (dW / dx of each chunk beside the next one) gives the oracle's gradients,
+    with one batch stream per group (B = 40) and with two (B = 64)."""
     monkeypatch.setenv("LSTM_BWD_CHUNKS", chunks)
-    w = synth.custom(41, 40, 64, 512, "bf16", seed=17)
+    w = synth.custom(41, B, 64, 512, "bf16", seed=17)
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
-    assert L.test_last_paths() == (3, 3)
+    assert L.test_last_paths() == (3, path)
     assert_within(compare(gpu, run_oracle(inp), "bf16"), "bf16", f"{chunks} chunks")
+
+
+@pytest.mark.parametrize("shape", [(20, 128, 64, 1024), (33, 64, 96, 512)])
+def test_two_stream_backward_equals_one_stream(shape, cuda_device, monkeypatch):
+    """The backward with two decoupled batch streams per group computes every
+    element in the same order as the one-stream kernel: the same bits."""
+    T, B, I, H = shape
+    w = synth.custom(T, B, I, H, "bf16", seed=T + B)
+    inp = synth.make_inputs(w)
+    two = run_gpu(inp, cuda_device)
+    fwd_path = L.test_last_paths()[0]
+    assert L.test_last_paths()[1] == 4
+    monkeypatch.setenv("LSTM_BWD_STREAMS", "1")
+    one = run_gpu(inp, cuda_device)
+    assert L.test_last_paths() == (fwd_path, 3)
+    for k in ("dx", "dW", "db", "dh0", "dc0"):
+        np.testing.assert_array_equal(two[k], one[k], err_msg=k)
+
