@@ -22,6 +22,7 @@
 #include "tc_recur2.cuh"
 #include "tc_recur3.cuh"
 #include "tc_recur4.cuh"
+#include "persist.cuh"
 
 using namespace lstm;
 
@@ -77,6 +78,7 @@ struct Phase {
 //   LSTM_BWD_TMEM_W=0      no backward kernel with the weights in tensor memory
 //   LSTM_BWD_STREAMS=1     that backward with one batch stream per group
 //   LSTM_BWD_CHUNKS=n      reverse-time chunks of the overlapped backward
+//   LSTM_PERSIST=0         no persistent CUDA-core recurrences (one launch per step)
 //   LSTM_LAUNCH_NONCOOP=1  cluster launches without the cooperative attribute
 //                          (also taken when a profiler or sanitizer is attached:
 //                          NV_COMPUTE_PROFILER_PERFWORKS_DIR or
@@ -86,6 +88,15 @@ bool env_is(const char *name, char value) {
     return e && e[0] == value && e[1] == '\0';
 }
 bool force_simt() { return env_is("LSTM_FORCE_SIMT", '1'); }
+// Persistent grids are launched without the cooperative attribute (after an
+// occupancy check) when LSTM_LAUNCH_NONCOOP=1 or a profiler or sanitizer is
+// attached: Nsight Compute sets NV_COMPUTE_PROFILER_PERFWORKS_DIR in the
+// process it profiles, tools that inject through CUDA_INJECTION64_PATH set that.
+bool profiler_attached() {
+    const char *inj = getenv("CUDA_INJECTION64_PATH");
+    const char *ncu = getenv("NV_COMPUTE_PROFILER_PERFWORKS_DIR");
+    return env_is("LSTM_LAUNCH_NONCOOP", '1') || (inj && inj[0]) || (ncu && ncu[0]);
+}
 
 // ------------------------------------------------------------ validation
 bool dims_ok(const lstm_dims *d) {
@@ -801,14 +812,9 @@ cudaError_t launch_cluster(Kern kern, const Prm &prm, int grid, int KS, size_t s
     cfg.attrs = at;
     cfg.numAttrs = 2;
     // Profilers cannot replay a cooperative cluster launch: with
-    // LSTM_LAUNCH_NONCOOP=1, or when a profiler or sanitizer is attached
-    // (Nsight Compute sets NV_COMPUTE_PROFILER_PERFWORKS_DIR in the profiled
-    // process; tools that inject through CUDA_INJECTION64_PATH set that),
-    // go straight to the occupancy-checked cluster launch below.
-    const char *inj = getenv("CUDA_INJECTION64_PATH");
-    const char *ncu = getenv("NV_COMPUTE_PROFILER_PERFWORKS_DIR");
-    const bool noncoop = env_is("LSTM_LAUNCH_NONCOOP", '1') || (inj && inj[0]) || (ncu && ncu[0]);
-    if (!noncoop) {
+    // LSTM_LAUNCH_NONCOOP=1, or when a profiler or sanitizer is attached, go
+    // straight to the occupancy-checked cluster launch below.
+    if (!profiler_attached()) {
         e = cudaLaunchKernelEx(&cfg, kern, prm);
         if (e == cudaSuccess || e == cudaErrorCooperativeLaunchTooLarge) {
             note_launch();
@@ -1160,6 +1166,99 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
     return rc;
 }
 
+// --------------------------------- persistent CUDA-core recurrences (pst)
+// One cooperative launch of `grid` CTAs of pst::NTHR threads (all co-resident
+// or nothing runs); with a profiler attached, an occupancy-checked plain launch.
+template <class Kern, class Prm>
+cudaError_t launch_persistent(Kern kern, const Prm &prm, int grid, size_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, pst::NTHR, smem) != cudaSuccess ||
+        per_sm * tcg::sm_count() < grid) {
+        cudaGetLastError();
+        return cudaErrorCooperativeLaunchTooLarge;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(pst::NTHR);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = profiler_attached() ? 0 : 1;
+    note_launch();
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+// Units per CTA of the persistent recurrences: every SM holds a slice (the
+// backward in quads of units, the grain of its epilogue), within the shared
+// memory budget and the kernels' per-thread item limit.
+bool plan_persist(const lstm_dims *d, bool backward, int &UN, int &P, int &KC, size_t &smem) {
+    if (env_is("LSTM_PERSIST", '0') || d->H < 1 || d->B < 1 || d->T < 1) return false;
+    const int nsm = tcg::sm_count();
+    const int q = backward ? 4 : 1;
+    UN = q * ((d->H + q * nsm - 1) / (q * nsm));
+    P = (d->H + UN - 1) / UN;
+    const long long items = (long long)d->B * (backward ? UN / 4 : UN);
+    if (items > (long long)pst::MAXP * pst::NTHR || P > nsm) return false;
+    // K chunks of 64 (staging the whole K in one chunk measured slower: fewer
+    // loads in flight per thread than chunk rounds overlapped with the FMAs)
+    KC = 64;
+    smem = backward ? pst::bwd_smem(d->B, d->H, UN, KC) : pst::fwd_smem(d->B, d->H, UN, KC);
+    return smem <= kMaxSmem;
+}
+
+// a2 over all T steps in one launch; Gx holds the input projection.
+// LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
+template <class T>
+int persist_fwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T *W, const float *Gx,
+                const T *h0, const float *c0, const T *mask, bool reverse, bool ijfo, T *y,
+                T *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
+    pst::FwdParams<T> prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.W = W; prm.Gx = Gx; prm.h0 = h0; prm.c0 = c0; prm.mask = mask;
+    prm.y = y; prm.gates = gates; prm.cells = cells; prm.ctrl = ctrl;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = UN; prm.KC = KC;
+    prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_persistent(pst::fwd_kernel<T>, prm, P, smem, s);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
+// a3 over all T steps in one launch (dinitH follows as one more product).
+template <class T>
+int persist_bwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T *W, const T *dy,
+                const T *dhT, const float *dcT, const T *gates, const float *cells,
+                const float *c0, const T *mask, bool reverse, bool ijfo, T *dG,
+                float *const dcbuf[2], float *const dhpbuf[2], float *dc0, Ctrl *ctrl,
+                cudaStream_t s) {
+    pst::BwdParams<T> prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.W = W; prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.mask = mask;
+    prm.dcT = dcT; prm.cells = cells; prm.c0 = c0; prm.dG = dG;
+    prm.dcbuf[0] = dcbuf[0]; prm.dcbuf[1] = dcbuf[1];
+    prm.dhpbuf[0] = dhpbuf[0]; prm.dhpbuf[1] = dhpbuf[1];
+    prm.dc0 = dc0; prm.ctrl = ctrl;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = UN; prm.KC = KC;
+    prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
+    prm.fault_skip_cta = g_fault_skip_cta;
+    prm.wait_ns = g_wait_ns;
+    const cudaError_t e = launch_persistent(pst::bwd_kernel<T>, prm, P, smem, s);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ forward pass
 // mask (variable length) or NULL; masked calls run on the TMEM-weight cluster
 // kernel or the per-step kernels only.
@@ -1221,9 +1320,21 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
                                      (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells, (Ctrl *)ws,
                                      s);
         }
-        // otherwise one fused GEMM + gate/cell/hidden epilogue launch per step
-        g_last_fwd_path = 0;
-        for (int st = 0; st < T_; ++st) {
+        // otherwise the persistent CUDA-core recurrence (all steps, one launch)
+        bool persisted = false;
+        {
+            int UN = 0, P = 0, KC = 0;
+            size_t psmem = 0;
+            if (plan_persist(d, false, UN, P, KC, psmem)) {
+                const int rc = persist_fwd<T>(d, UN, P, KC, psmem, W, Gx, h0, c0, mask, reverse, ijfo,
+                                              y, gates, cells, (Ctrl *)ws, s);
+                if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
+                persisted = rc == LSTM_OK;
+            }
+        }
+        // or one fused GEMM + gate/cell/hidden epilogue launch per step
+        g_last_fwd_path = persisted ? 5 : 0;
+        for (int st = 0; !persisted && st < T_; ++st) {
             // step st is at time t; the previous step at time tp
             const int t = reverse ? T_ - 1 - st : st, tp = reverse ? t + 1 : t - 1;
             const T *hp = st > 0 ? y + (long long)tp * BH : h0;
@@ -1353,13 +1464,25 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         }
     }
 
-    // a3: reverse-time recursion, steps 1-3 and 5 fused with delta h = W_h^T dG_{t+1}
-    g_last_bwd_path = 0;
+    // a3: reverse-time recursion, steps 1-3 and 5 fused with delta h = W_h^T dG_{t+1}:
+    // the persistent CUDA-core recurrence (all steps, one launch), or one launch per step
     {
     prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
+    bool persisted = false;
+    {
+        int UN = 0, P = 0, KC = 0;
+        size_t psmem = 0;
+        if (plan_persist(d, true, UN, P, KC, psmem)) {
+            const int rc = persist_bwd<T>(d, UN, P, KC, psmem, W, dy, dhT, dcT, gates, cells, c0, mask,
+                                          reverse, ijfo, dG, dcbuf, dhpbuf, dc0, (Ctrl *)ws, s);
+            if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
+            persisted = rc == LSTM_OK;
+        }
+    }
+    g_last_bwd_path = persisted ? 5 : 0;
     // steps st = T-1 .. 0 of the forward recurrence; step st is at time tau(st)
     auto tau = [&](int st) -> long long { return reverse ? T_ - 1 - st : st; };
-    for (int st = T_ - 1; st >= 0; --st) {
+    for (int st = T_ - 1; !persisted && st >= 0; --st) {
         const bool last = (st == T_ - 1);
         const long long t = tau(st);
         simt::EpBwdStep<T> ep;

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     uint64_t *recv_full = w_ready + 2;
     uint32_t *tmem_slot = (uint32_t *)(w_ready + 3);
     volatile int *abort_flag = (volatile int *)(w_ready + 4);
+    volatile int *cluster_bad = abort_flag + 1;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t kpart = tc::cluster_rank();
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(recv_full, 1);  // one local arrival (with the expected bytes) per step
         *abort_flag = 0;
+        *cluster_bad = tc::cluster_nctarank() != (uint32_t)KS;
         tc::fence_mbar_init();
     }
     if (warp == 1) {
@@ -146,6 +148,14 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     }
     tc::tc_fence_before();
     __syncthreads();
+    if (*cluster_bad) {  // a launch without the cluster shape: report, touch no peer
+        if (threadIdx.x == 0) atomicCAS(&p.ctrl->status, 0u, 2u);  // LSTM_ERR_UNSUPPORTED
+        if (warp == 1) {
+            tc::tc_fence_after();
+            tc::tmem_dealloc(*tmem_slot, TMEM_COLS);
+        }
+        return;
+    }
     tc::cluster_sync_all();
     tc::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
@@ -621,6 +631,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     uint64_t *recv_full = w_ready + 5;       // [SPLIT]
     uint32_t *tmem_slot = (uint32_t *)(w_ready + 7);
     volatile int *abort_flag = (volatile int *)(w_ready + 8);
+    volatile int *cluster_bad = abort_flag + 1;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t kpart = tc::cluster_rank();
@@ -655,6 +666,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
         // one local arrival (with the expected bytes) per (virtual) step
         for (int i = 0; i < SPLIT; ++i) tc::mbar_init(&recv_full[i], 1);
         *abort_flag = 0;
+        *cluster_bad = tc::cluster_nctarank() != (uint32_t)KS;
         tc::fence_mbar_init();
     }
     if (warp == 1) {
@@ -663,6 +675,14 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     }
     tc::tc_fence_before();
     __syncthreads();
+    if (*cluster_bad) {  // a launch without the cluster shape: report, touch no peer
+        if (threadIdx.x == 0) atomicCAS(&p.ctrl->status, 0u, 2u);  // LSTM_ERR_UNSUPPORTED
+        if (warp == 1) {
+            tc::tc_fence_after();
+            tc::tmem_dealloc(*tmem_slot, TMEM_COLS);
+        }
+        return;
+    }
     tc::cluster_sync_all();  // every CTA's barriers exist before any remote arrival
     tc::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;

@@ -130,9 +130,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
         tc::mbar_init(w_ready, NSTREAM * EPI_WG);
         *abort_flag = 0;
         // the kernel is written for clusters of exactly KS CTAs
-        uint32_t nrank;
-        asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(nrank));
-        *cluster_bad = nrank != (uint32_t)KS;
+        *cluster_bad = tc::cluster_nctarank() != (uint32_t)KS;
         tc::fence_mbar_init();
     }
     if (warp == 2) {

@@ -25,6 +25,9 @@
  *                          memory (the older cluster kernels run instead).
  *   LSTM_BWD_STREAMS=1     run that backward kernel with one batch stream per
  *                          group instead of two decoupled streams.
+ *   LSTM_PERSIST=0         run the CUDA-core recurrences (fp32, and 16-bit
+ *                          shapes off the tensor-core grids) as one launch
+ *                          per step instead of one persistent launch.
  *   LSTM_BWD_CHUNKS=n      run the tensor-core backward recurrence in n
  *                          reverse-time chunks (1..16; 1 = one launch, dW / dx
  *                          after it).  Default: min(8, T / 16), 1 below T = 32.
@@ -70,7 +73,8 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
 /*
  * Which recurrent kernel the most recent lstm_fwd / lstm_bwd of this process
  * used: 0 = one CUDA-core launch per step (fp32, or shapes off the tensor-core
- * grid), 1 = persistent kernel with K resident per CTA, 2 = persistent cluster
+ * grid), 5 = the persistent CUDA-core kernel for those (all steps in one
+ * launch), 1 = persistent tensor-core kernel with K resident per CTA, 2 = persistent cluster
  * kernel with K split across the CTAs of a cluster, 3 = the cluster kernel
  * with the weights held in tensor memory (forward: with the input projection
  * contracted inside the recurrence), 4 = (backward) that kernel with two

@@ -13,9 +13,9 @@ pytestmark = pytest.mark.gpu
 
 # (T, B, I, H, dtype) -> (forward path, backward path) of lstm_test_last_paths
 CASES = {
-    (9, 6, 24, 40, "fp32"): (0, 0),       # per-step kernels, fp32
-    (7, 5, 37, 45, "bf16"): (0, 0),       # per-step kernels, bf16
-    (10, 24, 64, 256, "bf16"): (3, 0),    # fused forward; per-step backward
+    (9, 6, 24, 40, "fp32"): (5, 5),       # persistent CUDA-core kernels, fp32
+    (7, 5, 37, 45, "bf16"): (5, 5),       # persistent CUDA-core kernels, bf16 off the tensor-core grid
+    (10, 24, 64, 256, "bf16"): (3, 5),    # fused forward; persistent CUDA-core backward
     (12, 48, 64, 512, "bf16"): (3, 3),    # TMEM-weight kernels, one launch each
     (40, 64, 96, 512, "bf16"): (3, 4),    # backward in 2 chunks, two batch streams
     (64, 200, 96, 512, "bf16"): (3, 3),   # ragged batch groups, 4 chunks

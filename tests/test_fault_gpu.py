@@ -50,3 +50,32 @@ def test_missing_arrival_times_out_and_recovers(H, T, B, streams, cuda_device, m
     # the context is still usable and the next call is correct
     out = run_gpu(synth.make_inputs(w), cuda_device)
     assert_within(compare(out, run_oracle(synth.make_inputs(w)), "bf16"), "bf16", "after fault")
+
+
+@pytest.mark.parametrize("dt,H", [("fp32", 256), ("bf16", 45)])
+def test_persistent_cuda_core_time_out_and_recover(dt, H, cuda_device):
+    """The persistent CUDA-core recurrences (fp32, and 16-bit shapes off the
+    tensor-core grids) meet at a grid-wide step counter: with CTA 0 never
+    arriving, both give up, report LSTM_ERR_TIMEOUT, and the next call runs."""
+    lbuild.build()
+    T, B, I = 6, 32, 37
+    w = synth.custom(T, B, I, H, dt, seed=13)
+    inp = {k: v.to(cuda_device) for k, v in synth.make_inputs(w).items()}
+    cd = synth.torch_dtype(dt)
+    st = L.State(T, B, I, H, cd, cuda_device)
+    gr = L.Grads(T, B, I, H, cuda_device)
+    wsf = L.empty_workspace(L.fwd_workspace_size(st.dims), cuda_device)
+    wsb = L.empty_workspace(L.bwd_workspace_size(st.dims), cuda_device)
+    try:
+        L.test_set_wait_fault(0, 50_000_000)
+        L.lstm_fwd(st.dims, inp["x"], inp["W"], inp["b"], inp["h0"], inp["c0"], st.y, st.hT,
+                   st.cT, st.gates, st.cells, wsf)
+        assert L.lstm_status(wsf) == L.LSTM_ERR_TIMEOUT
+        L.lstm_bwd(st.dims, inp["dy"], inp["dhT"], inp["dcT"], inp["x"], inp["W"], inp["h0"],
+                   inp["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0, wsb)
+        assert L.lstm_status(wsb) == L.LSTM_ERR_TIMEOUT
+        assert L.test_last_paths() == (5, 5)
+    finally:
+        L.test_set_wait_fault(-1, 0)
+    out = run_gpu(synth.make_inputs(w), cuda_device)
+    assert_within(compare(out, run_oracle(synth.make_inputs(w)), dt), dt, "after fault")

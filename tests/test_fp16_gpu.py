@@ -17,9 +17,9 @@ pytestmark = pytest.mark.gpu
 
 # (T, B, I, H) -> (forward path, backward path) of lstm_test_last_paths
 CASES = {
-    (7, 5, 37, 45): (0, 0),        # per-step kernels (H off the 32-unit grid)
-    (4, 130, 128, 128): (3, 0),    # fused forward; per-step backward (H < 512)
-    (10, 24, 64, 256): (3, 0),
+    (7, 5, 37, 45): (5, 5),        # persistent CUDA-core kernels (H off the 32-unit grid)
+    (4, 130, 128, 128): (3, 5),    # fused forward; persistent CUDA-core backward (H < 512)
+    (10, 24, 64, 256): (3, 5),
     (12, 48, 64, 512): (3, 3),     # TMEM-weight kernels, one launch each
     (40, 64, 96, 512): (3, 4),     # backward in 2 chunks, two batch streams
     (64, 200, 96, 512): (3, 3),    # ragged batch groups, 4 chunks

@@ -22,7 +22,7 @@ FULL = ["lstm_T8_B2_I16_H32_fp32", "lstm_T64_B32_I256_H256_fp32", "lstm_T128_B64
 
 
 # recurrent kernel each workload must run on (see lstm_test_last_paths)
-EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (0, 0), "lstm_T64_B32_I256_H256_fp32": (0, 0),
+EXPECTED_PATHS = {"lstm_T8_B2_I16_H32_fp32": (5, 5), "lstm_T64_B32_I256_H256_fp32": (5, 5),
                   "lstm_T128_B64_I512_H512_bf16": (3, 4),
                   "lstm_T256_B128_I1024_H1024_bf16": (3, 4),
                   "lstm_T1024_B16_I256_H1024_bf16": (3, 3)}
@@ -93,7 +93,7 @@ def test_odd_shapes(T, B, I, H, dt, cuda_device):
     inp = synth.make_inputs(w)
     gpu = run_gpu(inp, cuda_device)
     if dt == "bf16" and I % 8 != 0:  # no tensor-map forward recurrence
-        assert L.test_last_paths()[0] == 0
+        assert L.test_last_paths()[0] == 5
     elif dt == "bf16" and H in ODD_FWD_PATH:
         assert L.test_last_paths()[0] == ODD_FWD_PATH[H]
     if dt == "bf16" and (B, H) in ODD_BWD_PATH:
@@ -185,3 +185,26 @@ def test_two_stream_backward_equals_one_stream(shape, cuda_device, monkeypatch):
     for k in ("dx", "dW", "db", "dh0", "dc0"):
         np.testing.assert_array_equal(two[k], one[k], err_msg=k)
 
+
+
+@pytest.mark.parametrize("shape", [(64, 32, 256, 256, "fp32"), (9, 6, 24, 40, "fp32"),
+                                   (7, 5, 37, 45, "bf16"), (5, 130, 96, 1024, "fp32")])
+@pytest.mark.parametrize("opts", [{}, {"reverse": True, "ijfo": True}, {"mask": True}])
+def test_persistent_cuda_core_recurrences(shape, opts, cuda_device, monkeypatch):
+    """The persistent CUDA-core recurrences (all steps in one launch) against
+    the oracle and against the per-step kernels (LSTM_PERSIST=0): the same
+    epilogues, the products summed in another order."""
+    T, B, I, H, dt = shape
+    w = synth.custom(T, B, I, H, dt, seed=T * 7 + H)
+    inp = synth.make_inputs(w)
+    kw = dict(opts)
+    if kw.pop("mask", False):
+        kw["mask"] = synth.length_mask(T, B, H, synth.random_lengths(T, B, seed=B + H), dt)
+    per = run_gpu(inp, cuda_device, **kw)
+    assert L.test_last_paths() == (5, 5)
+    ref = run_oracle(inp, **kw)
+    assert_within(compare(per, ref, dt, OUTS + ("gates", "cells")), dt, w.name + " persistent")
+    monkeypatch.setenv("LSTM_PERSIST", "0")
+    stp = run_gpu(inp, cuda_device, **kw)
+    assert L.test_last_paths() == (0, 0)
+    assert_within(compare(stp, ref, dt, OUTS + ("gates", "cells")), dt, w.name + " per step")
