@@ -1195,37 +1195,47 @@ cudaError_t launch_persistent(Kern kern, const Prm &prm, int grid, size_t smem, 
 
 // Units per CTA of the persistent recurrences: every SM holds a slice (the
 // backward in quads of units, the grain of its epilogue), within the shared
-// memory budget and the kernels' per-thread item limit.
-bool plan_persist(const lstm_dims *d, bool backward, int &UN, int &P, int &KC, size_t &smem) {
+// memory budget and the kernels' per-thread item limit.  K is staged in
+// chunks of at most 8192 floats over all B rows (fewer syncs than small
+// chunks, and every thread has several loads in flight), and each item's dot
+// product is split over the lanes the CTA would otherwise leave idle.
+struct PstPlan {
+    int UN = 0, P = 0, KC = 0, KSPLIT = 1;
+    size_t smem = 0;
+};
+
+bool plan_persist(const lstm_dims *d, bool backward, PstPlan &Q) {
     if (env_is("LSTM_PERSIST", '0') || d->H < 1 || d->B < 1 || d->T < 1) return false;
     const int nsm = tcg::sm_count();
     const int q = backward ? 4 : 1;
-    UN = q * ((d->H + q * nsm - 1) / (q * nsm));
-    P = (d->H + UN - 1) / UN;
-    const long long items = (long long)d->B * (backward ? UN / 4 : UN);
-    if (items > (long long)pst::MAXP * pst::NTHR || P > nsm) return false;
-    // K chunks of 64 (staging the whole K in one chunk measured slower: fewer
-    // loads in flight per thread than chunk rounds overlapped with the FMAs)
-    KC = 64;
-    smem = backward ? pst::bwd_smem(d->B, d->H, UN, KC) : pst::fwd_smem(d->B, d->H, UN, KC);
-    return smem <= kMaxSmem;
+    Q.UN = q * ((d->H + q * nsm - 1) / (q * nsm));
+    Q.P = (d->H + Q.UN - 1) / Q.UN;
+    const long long items = (long long)d->B * (backward ? Q.UN / 4 : Q.UN);
+    if (items > (long long)pst::MAXP * pst::NTHR || Q.P > nsm) return false;
+    const int K = backward ? 4 * d->H : d->H;
+    Q.KC = std::min(std::max(32, 8192 / d->B / 32 * 32), (K + 31) / 32 * 32);
+    Q.KSPLIT = 1;
+    while (Q.KSPLIT < 32 && items * Q.KSPLIT * 2 <= pst::NTHR) Q.KSPLIT *= 2;
+    Q.smem = backward ? pst::bwd_smem(d->B, d->H, Q.UN, Q.KC) : pst::fwd_smem(d->B, d->H, Q.UN, Q.KC);
+    return Q.smem <= kMaxSmem;
 }
 
 // a2 over all T steps in one launch; Gx holds the input projection.
 // LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
 template <class T>
-int persist_fwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T *W, const float *Gx,
+int persist_fwd(const lstm_dims *d, const PstPlan &Q, const T *W, const float *Gx,
                 const T *h0, const float *c0, const T *mask, bool reverse, bool ijfo, T *y,
                 T *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
     pst::FwdParams<T> prm;
     memset(&prm, 0, sizeof(prm));
     prm.W = W; prm.Gx = Gx; prm.h0 = h0; prm.c0 = c0; prm.mask = mask;
     prm.y = y; prm.gates = gates; prm.cells = cells; prm.ctrl = ctrl;
-    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = UN; prm.KC = KC;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = Q.UN; prm.KC = Q.KC;
+    prm.KSPLIT = Q.KSPLIT;
     prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
-    const cudaError_t e = launch_persistent(pst::fwd_kernel<T>, prm, P, smem, s);
+    const cudaError_t e = launch_persistent(pst::fwd_kernel<T>, prm, Q.P, Q.smem, s);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
@@ -1235,7 +1245,7 @@ int persist_fwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T 
 
 // a3 over all T steps in one launch (dinitH follows as one more product).
 template <class T>
-int persist_bwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T *W, const T *dy,
+int persist_bwd(const lstm_dims *d, const PstPlan &Q, const T *W, const T *dy,
                 const T *dhT, const float *dcT, const T *gates, const float *cells,
                 const float *c0, const T *mask, bool reverse, bool ijfo, T *dG,
                 float *const dcbuf[2], float *const dhpbuf[2], float *dc0, Ctrl *ctrl,
@@ -1247,11 +1257,12 @@ int persist_bwd(const lstm_dims *d, int UN, int P, int KC, size_t smem, const T 
     prm.dcbuf[0] = dcbuf[0]; prm.dcbuf[1] = dcbuf[1];
     prm.dhpbuf[0] = dhpbuf[0]; prm.dhpbuf[1] = dhpbuf[1];
     prm.dc0 = dc0; prm.ctrl = ctrl;
-    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = UN; prm.KC = KC;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = Q.UN; prm.KC = Q.KC;
+    prm.KSPLIT = Q.KSPLIT;
     prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
-    const cudaError_t e = launch_persistent(pst::bwd_kernel<T>, prm, P, smem, s);
+    const cudaError_t e = launch_persistent(pst::bwd_kernel<T>, prm, Q.P, Q.smem, s);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
         cudaGetLastError();
         return LSTM_ERR_NOT_CORESIDENT;
@@ -1323,10 +1334,9 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         // otherwise the persistent CUDA-core recurrence (all steps, one launch)
         bool persisted = false;
         {
-            int UN = 0, P = 0, KC = 0;
-            size_t psmem = 0;
-            if (plan_persist(d, false, UN, P, KC, psmem)) {
-                const int rc = persist_fwd<T>(d, UN, P, KC, psmem, W, Gx, h0, c0, mask, reverse, ijfo,
+            PstPlan Q;
+            if (plan_persist(d, false, Q)) {
+                const int rc = persist_fwd<T>(d, Q, W, Gx, h0, c0, mask, reverse, ijfo,
                                               y, gates, cells, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
                 persisted = rc == LSTM_OK;
@@ -1470,10 +1480,9 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     prof::Phase ph(LSTM_PHASE_BWD_RECUR, s);
     bool persisted = false;
     {
-        int UN = 0, P = 0, KC = 0;
-        size_t psmem = 0;
-        if (plan_persist(d, true, UN, P, KC, psmem)) {
-            const int rc = persist_bwd<T>(d, UN, P, KC, psmem, W, dy, dhT, dcT, gates, cells, c0, mask,
+        PstPlan Q;
+        if (plan_persist(d, true, Q)) {
+            const int rc = persist_bwd<T>(d, Q, W, dy, dhT, dcT, gates, cells, c0, mask,
                                           reverse, ijfo, dG, dcbuf, dhpbuf, dc0, (Ctrl *)ws, s);
             if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
             persisted = rc == LSTM_OK;

@@ -25,9 +25,15 @@ namespace pst {
 
 constexpr int NTHR = 256;
 constexpr int MAXP = 4;         // (row, unit) pairs / (row, unit quad) items per thread
+constexpr int STAGE_UNR = 8;    // operand loads in flight per thread while staging
 
-// The step's operand is staged in K chunks of KC (the host picks 64), rows
-// padded to KC + 1 floats so that rows m, m+1, ... start in different banks.
+// The step's operand is staged in K chunks of KC (a multiple of 32 the host
+// picks so that a chunk of all B rows holds at most 8192 floats), rows padded
+// to KC + 1 floats so that rows m, m+1, ... start in different banks.  Each
+// output item's dot product is split over KSPLIT lanes of one warp (a power of
+// two <= 32 the host picks so that items x KSPLIT fill the CTA): lane `ks`
+// of the group takes k = ks, ks + KSPLIT, ... of every chunk and the group's
+// partial sums meet in a butterfly of shuffles.
 // Forward: CTA c owns hidden units [c*UN, c*UN + UN) (all four gates).
 // Shared memory: Ws [4][UN][H] fp32 (W_h rows g*H + j), hs [B][KC + 1] fp32.
 __host__ __device__ inline size_t fwd_smem(int B, int H, int UN, int KC) {
@@ -49,7 +55,7 @@ struct FwdParams {
     E *y, *gates;
     float *cells;
     Ctrl *ctrl;
-    int T, B, H, I, UN, KC, reverse, fb;
+    int T, B, H, I, UN, KC, KSPLIT, reverse, fb;
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -64,7 +70,7 @@ struct BwdParams {
     float *dc0;            // [B][H]: delta c after the first step (dinitC)
     float *dhpbuf[2];      // delta h passed on by padding, ping-pong [B][H]
     Ctrl *ctrl;
-    int T, B, H, I, UN, KC, reverse, fb;
+    int T, B, H, I, UN, KC, KSPLIT, reverse, fb;
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -85,11 +91,50 @@ __device__ __forceinline__ bool grid_step(unsigned int *ctr, unsigned int target
     return ok_s != 0;
 }
 
+// Rows [0, B) x columns [k0, k0 + kn) of a row-major operand with row pitch
+// `ld` into dst[B][KC + 1] as fp32 (zeros past kn), by all threads, with
+// STAGE_UNR independent loads in flight per thread.
+template <class T>
+__device__ __forceinline__ void stage_chunk(float *dst, const T *src, long long ld, int B, int k0,
+                                            int kn, int KC) {
+    const int n = B * KC, KCP = KC + 1;
+    for (int base = threadIdx.x; base < n; base += NTHR * STAGE_UNR) {
+        float v[STAGE_UNR];
+#pragma unroll
+        for (int u = 0; u < STAGE_UNR; ++u) {
+            const int e = base + u * NTHR;
+            const int m = e / KC, kk = e - m * KC;
+            v[u] = (e < n && kk < kn) ? to_f(src[(long long)m * ld + k0 + kk]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < STAGE_UNR; ++u) {
+            const int e = base + u * NTHR;
+            if (e < n) {
+                const int m = e / KC;
+                dst[m * KCP + (e - m * KC)] = v[u];
+            }
+        }
+    }
+}
+
+// Sum of the four accumulators of each item over the KSPLIT lanes of its
+// group (every lane of the warp takes part; each ends with the group's sums).
+__device__ __forceinline__ void group_sum(float (&acc)[MAXP][4], int ksplit) {
+    for (int off = ksplit / 2; off > 0; off /= 2)
+#pragma unroll
+        for (int i = 0; i < MAXP; ++i)
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                acc[i][g] += __shfl_xor_sync(0xffffffffu, acc[i][g], off);
+}
+
 template <class T>
 __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
     extern __shared__ float4 smem_f4[];
     float *Ws = reinterpret_cast<float *>(smem_f4);
     const int H = p.H, B = p.B, T_ = p.T, UN = p.UN, KC = p.KC, KCP = KC + 1;
+    const int KSPLIT = p.KSPLIT, slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT;
+    const int nslots = NTHR / KSPLIT;
     float *hs = Ws + (size_t)4 * UN * H;
     __shared__ int abort_s;
     if (threadIdx.x == 0) abort_s = 0;
@@ -118,13 +163,11 @@ __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
             for (int k0 = 0; k0 < H; k0 += KC) {
                 const int kn = min(KC, H - k0);
                 __syncthreads();  // the previous chunk has been read
-                for (int m = 0; m < B; ++m)
-                    for (int kk = threadIdx.x; kk < KC; kk += NTHR)
-                        hs[m * KCP + kk] = kk < kn ? to_f(hp[(long long)m * H + k0 + kk]) : 0.f;
+                stage_chunk(hs, hp, H, B, k0, kn, KC);
                 __syncthreads();
 #pragma unroll
                 for (int i = 0; i < MAXP; ++i) {
-                    const int q = threadIdx.x + i * NTHR;
+                    const int q = slot + i * nslots;
                     if (q >= npairs) break;
                     const int m = q % B, jj = q / B;
                     const float *hrow = hs + m * KCP;
@@ -132,7 +175,7 @@ __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
                     const float *w1 = Ws + ((size_t)1 * UN + jj) * H + k0;
                     const float *w2 = Ws + ((size_t)2 * UN + jj) * H + k0;
                     const float *w3 = Ws + ((size_t)3 * UN + jj) * H + k0;
-                    for (int kk = 0; kk < kn; ++kk) {
+                    for (int kk = ks; kk < kn; kk += KSPLIT) {
                         const float h = hrow[kk];
                         acc[i][0] = fmaf(h, w0[kk], acc[i][0]);
                         acc[i][1] = fmaf(h, w1[kk], acc[i][1]);
@@ -151,12 +194,13 @@ __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
             ep.hprev = hp;
         }
         ep.fb = p.fb;
+        group_sum(acc, KSPLIT);
 #pragma unroll
         for (int i = 0; i < MAXP; ++i) {
-            const int q = threadIdx.x + i * NTHR;
+            const int q = slot + i * nslots;
             if (q >= npairs) break;
             const int m = q % B, jj = q / B;
-            ep(m, 4 * (j0 + jj), acc[i]);
+            if (ks == 0) ep(m, 4 * (j0 + jj), acc[i]);
         }
         // h_t of every unit is the next step's operand: grid barrier
         if (st + 1 < T_) {
@@ -172,6 +216,8 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
     extern __shared__ float4 smem_f4[];
     float *Wt = reinterpret_cast<float *>(smem_f4);
     const int H = p.H, B = p.B, T_ = p.T, UN = p.UN, KC = p.KC, KCP = KC + 1;
+    const int KSPLIT = p.KSPLIT, slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT;
+    const int nslots = NTHR / KSPLIT;
     const int G4 = 4 * H;
     float *gs = Wt + (size_t)UN * G4;
     __shared__ int abort_s;
@@ -203,13 +249,11 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
             for (int k0 = 0; k0 < G4; k0 += KC) {
                 const int kn = min(KC, G4 - k0);
                 __syncthreads();
-                for (int m = 0; m < B; ++m)
-                    for (int kk = threadIdx.x; kk < KC; kk += NTHR)
-                        gs[m * KCP + kk] = kk < kn ? to_f(dGn[(long long)m * G4 + k0 + kk]) : 0.f;
+                stage_chunk(gs, dGn, G4, B, k0, kn, KC);
                 __syncthreads();
 #pragma unroll
                 for (int i = 0; i < MAXP; ++i) {
-                    const int q = threadIdx.x + i * NTHR;
+                    const int q = slot + i * nslots;
                     if (q >= nitems) break;
                     const int m = q % B, jq = q / B;
                     const float *grow = gs + m * KCP;
@@ -217,7 +261,7 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
                     const float *w1 = Wt + (size_t)(4 * jq + 1) * G4 + k0;
                     const float *w2 = Wt + (size_t)(4 * jq + 2) * G4 + k0;
                     const float *w3 = Wt + (size_t)(4 * jq + 3) * G4 + k0;
-                    for (int kk = 0; kk < kn; ++kk) {
+                    for (int kk = ks; kk < kn; kk += KSPLIT) {
                         const float g = grow[kk];
                         acc[i][0] = fmaf(g, w0[kk], acc[i][0]);
                         acc[i][1] = fmaf(g, w1[kk], acc[i][1]);
@@ -244,12 +288,13 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
             ep.dhp_in = last ? nullptr : p.dhpbuf[(st + 1) & 1];
             ep.dhp_out = p.dhpbuf[st & 1];
         }
+        group_sum(acc, KSPLIT);
 #pragma unroll
         for (int i = 0; i < MAXP; ++i) {
-            const int q = threadIdx.x + i * NTHR;
+            const int q = slot + i * nslots;
             if (q >= nitems) break;
             const int m = q % B, jq = q / B;
-            ep(m, j0 + 4 * jq, acc[i]);
+            if (ks == 0) ep(m, j0 + 4 * jq, acc[i]);
         }
         // dG_t of every unit is the next step's operand: grid barrier
         if (st > 0) {

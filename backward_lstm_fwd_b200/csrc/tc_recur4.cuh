@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
     uint64_t *w_ready = bars + NSTREAM * 2 * MAX_STAGES;  // W_h^T slice written to TMEM
     uint64_t *mma_done = w_ready + 1;                     // [NSTREAM]
     uint64_t *recv_full = w_ready + 1 + NSTREAM;          // [NSTREAM]
-    uint64_t *xtok = w_ready + 1 + 2 * NSTREAM;           // [0]: stream 0's first exchange done
+    uint64_t *xtok = w_ready + 1 + 2 * NSTREAM;           // [NSTREAM]: a stream's exchange is done
     uint32_t *tmem_slot = (uint32_t *)(w_ready + 1 + 3 * NSTREAM);
     volatile int *abort_flag = (volatile int *)(w_ready + 2 + 3 * NSTREAM);
     volatile int *cluster_bad = abort_flag + 1;
@@ -314,14 +314,15 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
         // to the block of the CTA that finalises the unit (its own recv slot,
         // or the send staging), one bulk copy per partner, then the 8 slots
         // are summed in source order.
-        // Stream 1's first DSMEM exchange of a launch waits for stream 0's
-        // first exchange; after that the streams run free.  Started together,
-        // the two symmetric chains run in lockstep and contend for the SM's
-        // DSMEM, TMA and memory bandwidth at the same moments (and settle into
-        // one of two step periods, the slower one 45 % longer); started a
-        // DSMEM exchange apart, they stay offset, one stream's exchange beside
-        // the other stream's hand-off, loads and pointwise work.  (Holding
-        // them to strict alternation at every step measured 1 % slower.)
+        // The two streams' DSMEM exchanges alternate: exchange k of stream 1
+        // follows exchange k of stream 0, which follows exchange k - 1 of
+        // stream 1.  Left free, the two symmetric chains fall into lockstep
+        // and contend for the SM's DSMEM, TMA and memory bandwidth at the same
+        // moments, settling into one of two step periods (the slower one 45 %
+        // longer); offset only at the start of a launch they mostly stay
+        // apart (2 % faster than strict alternation) but drifted into the slow
+        // period in one run of 17.  Alternating, one stream's exchange runs
+        // beside the other's hand-off, loads and pointwise work at every step.
         uint32_t dph = 0, rph = 0;
         int xk = 0;  // exchanges of this stream so far in this launch
         auto read_dh = [&](float (&dh)[UPT]) -> bool {
@@ -355,8 +356,13 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
             tc::fence_proxy_async_smem();
             rec::named_bar(bar_sync, EPI_WG);
             if (wt == 0) {
-                const bool go = !(sw == 1 && xk == 0) ||
-                                tc::mbar_wait(&xtok[0], 0, p.ctrl, abort_flag, 0x807, p.wait_ns);
+                bool go = true;
+                if (sw == 1)
+                    go = tc::mbar_wait(&xtok[0], (uint32_t)(xk & 1), p.ctrl, abort_flag, 0x807,
+                                       p.wait_ns);
+                else if (xk > 0)
+                    go = tc::mbar_wait(&xtok[1], (uint32_t)((xk - 1) & 1), p.ctrl, abort_flag,
+                                       0x807, p.wait_ns);
                 if (go) {
                     tc::mbar_arrive_expect_tx(rf, (KS - 1) * PART_BYTES);
                     // partners kpart + 1, kpart + 2, ...: each CTA receives from
@@ -374,7 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
             }
             const bool w2 = tc::mbar_wait_cluster(rf, rph, p.ctrl, abort_flag, 0x806, p.wait_ns);
             if (!rec3::vote_all(w2, bar_vote, EPI_WG)) return false;
-            if (wt == 0 && sw == 0 && xk == 0) tc::mbar_arrive(&xtok[0]);
+            if (wt == 0) tc::mbar_arrive(&xtok[sw]);
             ++xk;
             rph ^= 1;
 #pragma unroll
