@@ -127,6 +127,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_set_wait_fault.restype = ip
     lib.lstm_test_last_paths.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_paths.restype = ip
+    lib.lstm_test_last_stack_chunks.argtypes = []
+    lib.lstm_test_last_stack_chunks.restype = ip
     lib.lstm_test_bwd_chunks.argtypes = [ip]
     lib.lstm_test_bwd_chunks.restype = ip
     lib.lstm_test_chunk_bound.argtypes = [ip, ip, ip]
@@ -371,6 +373,12 @@ def test_last_paths():
     f, b = ctypes.c_int(), ctypes.c_int()
     load().lstm_test_last_paths(ctypes.byref(f), ctypes.byref(b))
     return f.value, b.value
+
+
+def test_last_stack_chunks() -> int:
+    """Test hook: chunks per layer of the last stack forward's layer wavefront
+    (0: layer after layer; -1: no stack forward yet)."""
+    return int(load().lstm_test_last_stack_chunks())
 
 
 # ------------------------------------------------------------------ helpers

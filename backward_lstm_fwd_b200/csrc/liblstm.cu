@@ -322,6 +322,40 @@ AuxStreams *aux_streams() {
     return a.ready ? &a : nullptr;
 }
 
+// Streams and events of the stacked forward's layer wavefront: one stream per
+// layer (layers past kMaxWave share them in turn), an event per (layer stream,
+// chunk), and the fork / join events.
+constexpr int kMaxWave = 8, kMaxWaveChunks = 8;
+struct WaveStreams {
+    cudaStream_t st[kMaxWave] = {};
+    cudaEvent_t ev[kMaxWave][kMaxWaveChunks] = {};
+    cudaEvent_t fork = nullptr, join[kMaxWave] = {};
+    bool ready = false, tried = false;
+    std::mutex mu;  // one wavefront call enqueues at a time (the events are shared)
+};
+
+WaveStreams *wave_streams() {
+    static std::mutex mu;
+    static WaveStreams per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    WaveStreams &w = per_dev[dev];
+    if (!w.tried) {
+        w.tried = true;
+        bool ok = cudaEventCreateWithFlags(&w.fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int l = 0; ok && l < kMaxWave; ++l) {
+            ok = cudaStreamCreateWithFlags(&w.st[l], cudaStreamNonBlocking) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&w.join[l], cudaEventDisableTiming) == cudaSuccess;
+            for (int c = 0; ok && c < kMaxWaveChunks; ++c)
+                ok = cudaEventCreateWithFlags(&w.ev[l][c], cudaEventDisableTiming) == cudaSuccess;
+        }
+        if (!ok) cudaGetLastError();
+        w.ready = ok;
+    }
+    return w.ready ? &w : nullptr;
+}
+
 // Number of reverse-time chunks of a backward call whose dW / dx GEMMs run
 // beside the recurrence (1: no overlap): at least 16 steps per chunk, at most
 // 8 chunks (the last chunk's GEMM is the part that cannot overlap; each chunk
@@ -353,6 +387,7 @@ int g_fault_skip_cta = -1;
 // Which recurrent kernel the last lstm_fwd / lstm_bwd used (test hook):
 // 0 per-step CUDA-core kernels, 1 persistent K-resident kernel, 2 cluster kernel.
 int g_last_fwd_path = -1, g_last_bwd_path = -1;
+int g_last_stack_chunks = -1;  // chunks per layer of the last stack forward's wavefront
 unsigned long long g_wait_ns = 2000000000ull;
 
 struct RecPlan {
@@ -632,12 +667,14 @@ const void *fwd3_kernel_ptr(int NB, int KS, bool masked, int split) {
 // Forward with the input projection fused: the grid of plan_fwd2, and the
 // CTA's W_h and W_x K-slices must fit TMEM beside two accumulators.
 // LSTM_FWD_FUSED_X=0 turns it off (comparison runs).
-bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked) {
+// max_ctas > 0 caps the grid (a layer of a stacked wavefront shares the SMs
+// with the layer beside it).
+bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked, int max_ctas = 0) {
     if (env_is("LSTM_FWD_FUSED_X", '0')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
         d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
-    const int nsm = tcg::sm_count();
+    const int nsm = max_ctas > 0 ? std::min(max_ctas, tcg::sm_count()) : tcg::sm_count();
     P.R = d->H / rec2::F_UNITS;
     for (int KS : {4, 2, 8, 1}) {
         if ((d->H / KS) % 64 != 0 || d->H % KS != 0) continue;
@@ -907,7 +944,7 @@ template <class E>
 int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *x, const E *W,
                        const E *b, const E *h0, const float *c0, const E *mask, bool reverse,
                        bool ijfo, E *y, E *hT, float *cT, E *gates, float *cells, Ctrl *ctrl,
-                       cudaStream_t s) {
+                       cudaStream_t s, int bar_base = 0) {
     const long long T = d->T, B = d->B, H = d->H, I = d->I;
     const CUtensorMapDataType dt = tcg::map_type(Elem<E>::kFmt);
     rec3::Fwd3Params<E> prm;
@@ -923,6 +960,7 @@ int tc_fwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *x, const 
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.I = (int)I; prm.R = P.R; prm.G = P.G;
     prm.kcc = P.kcc; prm.kcx = P.kcx;
     prm.has_h0 = h0 != nullptr;
+    prm.bar_base = bar_base;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
     const cudaError_t e = launch_fwd3(prm, P, s);
@@ -1733,6 +1771,92 @@ size_t stack_fwd_ws(const lstm_dims *d, int L) {
     return n;
 }
 
+// Layer wavefront of the stacked forward.  Layer l's step t reads layer
+// l-1's output at step t and its own state after step t-1, so layer l can run
+// one block of steps behind layer l-1 instead of after all of it.  Each
+// layer's recurrence is the fused forward kernel on a grid of at most half
+// the SMs, launched once per chunk of consecutive steps on a stream of its
+// own; chunk c of layer l is ordered after chunk c of layer l-1 by an event
+// (no kernel waits on another kernel).  Both recurrences are latency bound,
+// so two layers' chunks side by side each run at nearly their own speed.  A
+// chunk continues its layer from the saved h and c of the step before it, and
+// every launch has step counters of its own in the one control block.
+// LSTM_ERR_UNSUPPORTED / LSTM_ERR_NOT_CORESIDENT: the caller runs the layers
+// one after another instead (outputs are rewritten from scratch).
+template <class E>
+int stack_fwd_wave(const lstm_dims *d, int L, bool reverse, bool ijfo, const E *x,
+                   const void *const *W, const void *const *b, const E *h0, const float *c0,
+                   E *y, E *hT, float *cT, E *gates, float *cells, Ctrl *ctrl, cudaStream_t s) {
+    if (L < 2 || env_is("LSTM_STACK_WAVE", '0')) return LSTM_ERR_UNSUPPORTED;
+    const int T = d->T;
+    const long long B = d->B, H = d->H, BH = B * H, TBH = (long long)T * BH;
+    // layer 0 and the layers above it (whose input width is H)
+    Rec2Plan P[2];
+    for (int k = 0; k < 2; ++k) {
+        const lstm_dims dk = layer_dims(d, k);
+        if (!plan_fwd3(&dk, P[k], false, tcg::sm_count() / 2)) return LSTM_ERR_UNSUPPORTED;
+    }
+    auto counters = [&](int l) { return P[l > 0].G * P[l > 0].split; };
+    int per_chunk = 0;  // step counters of one chunk of every layer
+    for (int l = 0; l < L; ++l) per_chunk += counters(l);
+    // chunks of at least 8 steps, at most kMaxWaveChunks, and every launch's
+    // counters within the control block; LSTM_STACK_CHUNKS overrides (1: each
+    // layer in one launch, the layers still ordered by events)
+    const int nbar = (int)(sizeof(ctrl->bar) / sizeof(ctrl->bar[0]));
+    const char *ov = getenv("LSTM_STACK_CHUNKS");
+    int nch = ov ? atoi(ov) : std::min(kMaxWaveChunks, T / 8);
+    nch = std::min(std::min(std::min(nch, kMaxWaveChunks), T), nbar / per_chunk);
+    if (nch < (ov ? 1 : 2)) return LSTM_ERR_UNSUPPORTED;
+    WaveStreams *Wv = wave_streams();
+    if (!Wv) return LSTM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(Wv->mu);
+    const int ns = std::min(L, kMaxWave);
+    if (cudaEventRecord(Wv->fork, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    for (int l = 0; l < ns; ++l)
+        if (cudaStreamWaitEvent(Wv->st[l], Wv->fork, 0) != cudaSuccess) return LSTM_ERR_CUDA;
+    g_last_fwd_path = 3;
+    g_last_stack_chunks = nch;
+    int rc = LSTM_OK;
+    for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
+        // steps [s0, s1): times [s0, s1), or [T - s1, T - s0) in reverse
+        const int s0 = (int)((long long)c * T / nch), s1 = (int)((long long)(c + 1) * T / nch);
+        const long long tlo = reverse ? T - s1 : s0;        // first time of the chunk
+        const long long tprev = reverse ? T - s0 : s0 - 1;  // time of the step before it
+        int bar = c * per_chunk;
+        for (int l = 0; l < L && rc == LSTM_OK; ++l) {
+            cudaStream_t sl = Wv->st[l % kMaxWave];
+            if (l > 0 && cudaStreamWaitEvent(sl, Wv->ev[(l - 1) % kMaxWave][c], 0) != cudaSuccess) {
+                rc = LSTM_ERR_CUDA;
+                break;
+            }
+            lstm_dims dc = layer_dims(d, l);
+            dc.T = s1 - s0;
+            E *yl = y + l * TBH;
+            float *cl = cells + l * TBH;
+            const E *xc = l == 0 ? x + tlo * B * d->I : y + (l - 1) * TBH + tlo * BH;
+            const E *h0c = c > 0 ? yl + tprev * BH : (h0 ? h0 + l * BH : nullptr);
+            const float *c0c = c > 0 ? cl + tprev * BH : (c0 ? c0 + l * BH : nullptr);
+            {
+                prof::Phase ph(LSTM_PHASE_FWD_RECUR, sl);
+                rc = tc_fwd_recurrence3(&dc, P[l > 0], xc, (const E *)W[l],
+                                        b ? (const E *)b[l] : nullptr, h0c, c0c, (const E *)nullptr,
+                                        reverse, ijfo, yl + tlo * BH, hT + l * BH, cT + l * BH,
+                                        gates + 4 * (l * TBH + tlo * BH), cl + tlo * BH, ctrl, sl,
+                                        bar);
+            }
+            bar += counters(l);
+            if (rc == LSTM_OK && cudaEventRecord(Wv->ev[l % kMaxWave][c], sl) != cudaSuccess)
+                rc = LSTM_ERR_CUDA;
+        }
+    }
+    // join: nothing of this call stays unordered with the caller's stream
+    for (int l = 0; l < ns; ++l)
+        if (cudaEventRecord(Wv->join[l], Wv->st[l]) != cudaSuccess ||
+            cudaStreamWaitEvent(s, Wv->join[l], 0) != cudaSuccess)
+            return LSTM_ERR_CUDA;
+    return rc;
+}
+
 // Layers 0 .. L-1 in order, each one lstm_fwd_ex call on the same stream.
 int stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
               const void *const *W, const void *const *b, const void *h0, const float *c0,
@@ -1744,6 +1868,31 @@ int stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
     if (L > 1 && !stack_slices_aligned(d)) return LSTM_ERR_UNSUPPORTED;
     const size_t es = esize(d);
     const long long BH = (long long)d->B * d->H, TBH = (long long)d->T * BH;
+    g_last_stack_chunks = 0;
+    // the layer wavefront where it applies (16-bit types, no length mask)
+    const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
+    const int order = opt ? opt->gate_order : LSTM_GATES_IFJO;
+    if (L > 1 && d->dtype != LSTM_F32 && !(opt && opt->seq_mask) && dims_supported(d) &&
+        (dir == LSTM_DIR_FORWARD || dir == LSTM_DIR_REVERSE) &&
+        (order == LSTM_GATES_IFJO || order == LSTM_GATES_IJFO) && (long long)d->T * BH > 0 &&
+        ptr_ok(x, (long long)d->T * d->B * d->I > 0) && ptr_ok(h0, false) && ptr_ok(c0, false) &&
+        ptr_ok(y, true) && ptr_ok(hT, true) && ptr_ok(cT, true) && ptr_ok(gates, true) &&
+        ptr_ok(cells, true) && ws_ok(ws, ws_bytes, kCtrlBytes) == LSTM_OK) {
+        cudaStream_t s = (cudaStream_t)stream;
+        if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+        const bool rev = dir == LSTM_DIR_REVERSE, ijfo = order == LSTM_GATES_IJFO;
+        int rc;
+        if (d->dtype == LSTM_F16)
+            rc = stack_fwd_wave<__half>(d, L, rev, ijfo, (const __half *)x, W, b,
+                                        (const __half *)h0, c0, (__half *)y, (__half *)hT, cT,
+                                        (__half *)gates, cells, (Ctrl *)ws, s);
+        else
+            rc = stack_fwd_wave<bf16>(d, L, rev, ijfo, (const bf16 *)x, W, b, (const bf16 *)h0,
+                                      c0, (bf16 *)y, (bf16 *)hT, cT, (bf16 *)gates, cells,
+                                      (Ctrl *)ws, s);
+        if (rc != LSTM_ERR_UNSUPPORTED && rc != LSTM_ERR_NOT_CORESIDENT) return rc;
+        g_last_stack_chunks = 0;
+    }
     const char *yb = static_cast<const char *>(y);
     for (int l = 0; l < L; ++l) {
         const lstm_dims dl = layer_dims(d, l);
@@ -1998,6 +2147,8 @@ int lstm_test_chunk_bound(int T, int nch, int c) {
     if (T < 0 || nch < 1 || c < 0 || c > nch) return -1;
     return chunk_bound(T, nch, c);
 }
+
+int lstm_test_last_stack_chunks(void) { return g_last_stack_chunks; }
 
 int lstm_test_last_paths(int *fwd_path, int *bwd_path) {
     if (fwd_path) *fwd_path = g_last_fwd_path;

@@ -539,6 +539,7 @@ struct Fwd3Params {
     float *cells, *cT;
     Ctrl *ctrl;
     int T, B, H, I, R, G, kcc, kcx, has_h0;
+    int bar_base;  // first of this launch's G * SPLIT step counters in ctrl->bar
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -644,7 +645,7 @@ __global__ void __launch_bounds__(rec2::F_THREADS, 1) fwd3_kernel(const __grid_c
     // time of recurrence step s (step s reads the state step s-1 left)
     auto tau = [&](int s) { return p.reverse ? T - 1 - s : s; };
     const uint32_t WH_COL = 2 * NB, WX_COL = 2 * NB + 32 * kcc;
-    unsigned int *ctr = &p.ctrl->bar[gi * SPLIT];  // + stream: one counter per stream
+    unsigned int *ctr = &p.ctrl->bar[p.bar_base + gi * SPLIT];  // + stream: one per stream
     const int V = T * SPLIT;                        // virtual steps
     const unsigned int group_ctas = (unsigned)(p.R * KS);
     constexpr uint32_t TMEM_COLS = 512;

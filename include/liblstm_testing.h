@@ -28,6 +28,12 @@
  *   LSTM_PERSIST=0         run the CUDA-core recurrences (fp32, and 16-bit
  *                          shapes off the tensor-core grids) as one launch
  *                          per step instead of one persistent launch.
+ *   LSTM_STACK_WAVE=0      run the layers of lstm_stack_fwd one after another
+ *                          instead of as a layer wavefront (two layers' time
+ *                          chunks side by side on half the SMs each).
+ *   LSTM_STACK_CHUNKS=n    chunks per layer of that wavefront (1..8; 1 = each
+ *                          layer in one launch, after the layer below it).
+ *                          Default: min(8, T / 8), and no wavefront below 2.
  *   LSTM_BWD_CHUNKS=n      run the tensor-core backward recurrence in n
  *                          reverse-time chunks (1..16; 1 = one launch, dW / dx
  *                          after it).  Default: min(8, T / 16), 1 below T = 32.
@@ -82,6 +88,13 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
  * epilogue warpgroup; -1 = none yet.
  */
 int lstm_test_last_paths(int *fwd_path, int *bwd_path);
+
+/*
+ * Chunks per layer of the layer wavefront that the most recent
+ * lstm_stack_fwd of this process ran (0: its layers ran one after another;
+ * -1: none yet).
+ */
+int lstm_test_last_stack_chunks(void);
 
 /*
  * Reverse-time chunking of the tensor-core backward: the number of chunk

@@ -3,10 +3,11 @@ module of the "cmu 10-414 HW4" page, "Stack Multiple RNN Cells" of the
 "mxnet-lstm" page) through the C ABI against the fp64 stacked oracle, element
 by element, on the kernel paths of the layers (per-step kernels, the fused
 forward and the TMEM-weight backward in one launch and in chunks, with the
-layer-0 input width differing from H), in every compute type, and with the
-options; plus two identities: one layer is the single-layer call, and L layers
-are L single-layer calls with dx rounded to the compute type in between, bit
-for bit.  Tolerance as in the other parity tests."""
+layer-0 input width differing from H, and the forward as a layer wavefront),
+in every compute type, and with the options; plus three identities: one layer
+is the single-layer call, L layers are L single-layer calls with dx rounded
+to the compute type in between, and the layer wavefront in time chunks is the
+same wavefront with each layer in one launch, bit for bit.  Tolerance as in the other parity tests."""
 import numpy as np
 import pytest
 import torch
@@ -79,6 +80,7 @@ CASES = [
     (40, 64, 1024, 512, 2, "bf16"), # chunked backward, layer 0 wider than H
     (12, 48, 64, 512, 3, "fp16"),   # fp16
     (6, 128, 64, 512, 2, "bf16"),   # the forward with two batch streams per cluster
+    (64, 64, 256, 512, 2, "bf16"),  # the forward as a layer wavefront (8 chunks of 8 steps)
 ]
 
 
@@ -89,6 +91,58 @@ def test_stack(case, cuda_device):
     gpu = run_gpu_stack(inp, cuda_device)
     ref = run_oracle_stack(inp)
     check(gpu, ref, dt, f"stack {case}")
+
+
+# (T, B, I, H, L, dtype, reverse, gate order, chunks per layer)
+WAVE_CASES = [
+    (64, 64, 512, 512, 2, "bf16", False, "ifjo", 8),
+    (43, 64, 1024, 512, 3, "fp16", False, "ifjo", 5),  # chunks of 8 or 9 steps
+    (40, 128, 256, 512, 2, "bf16", True, "ijfo", 5),   # reverse direction
+]
+
+
+@pytest.mark.parametrize("case", WAVE_CASES)
+def test_stack_wavefront_chunks_are_seamless(case, cuda_device, monkeypatch):
+    """The layer wavefront runs each layer in time chunks on its own stream, a
+    layer's chunk after the same chunk of the layer below.  A chunk continues
+    its layer from the saved h (the compute type, as the kernel reads h_{t-1}
+    every step) and c (fp32, the value the kernel keeps in registers) of the
+    step before it, so the chunked run gives the bits of each layer in one
+    launch (LSTM_STACK_CHUNKS=1, the same grids); with the wavefront off, the
+    layers run one after another on the full-device plan, whose summation
+    order differs, and the stack matches the oracle either way."""
+    T, B, I, H, Lc, dt, reverse, order, nch = case
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=T + Lc)
+    d = {k: ([t.to(cuda_device) for t in v] if isinstance(v, list) else v.to(cuda_device))
+         for k, v in inp.items()}
+    outs = {}
+    for label, env, want in (("chunked", {}, nch), ("one launch", {"LSTM_STACK_CHUNKS": "1"}, 1),
+                             ("layer by layer", {"LSTM_STACK_WAVE": "0"}, 0)):
+        monkeypatch.delenv("LSTM_STACK_CHUNKS", raising=False)
+        monkeypatch.delenv("LSTM_STACK_WAVE", raising=False)
+        for k, v in env.items():
+            monkeypatch.setenv(k, v)
+        outs[label] = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"], reverse=reverse,
+                                      gate_order=order)
+        torch.cuda.synchronize()
+        assert L.test_last_stack_chunks() == want, label
+    a, b = outs["chunked"], outs["one launch"]
+    for k in ("y", "hT", "cT", "gates", "cells"):
+        assert torch.equal(getattr(a, k), getattr(b, k)), k
+    # the chunked wavefront, and the backward on its saved state, against the oracle
+    g = L.backward_stack(a, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"], d["dcT"],
+                         reverse=reverse, gate_order=order)
+    torch.cuda.synchronize()
+    n = lambda t: t.float().cpu().double().numpy()
+    gpu = dict(y=n(a.y), hT=n(a.hT), cT=n(a.cT), dx=n(g.dx), dh0=n(g.dh0), dc0=n(g.dc0),
+               dW=[n(t) for t in g.dW], db=[n(t) for t in g.db], L=Lc)
+    check(gpu, run_oracle_stack(inp, reverse=reverse, gate_order=order), dt,
+          f"stack wavefront {case}")
+    seq = outs["layer by layer"]
+    errs = {k: rel_err(getattr(a, k).float().cpu().double().numpy(),
+                       getattr(seq, k).float().cpu().double().numpy())
+            for k in ("y", "hT", "cT")}
+    assert_within(errs, dt, f"wavefront vs layer by layer {case}")
 
 
 def test_stack_with_options(cuda_device):
