@@ -23,7 +23,7 @@ LSTM_ERR_CUDA = 4
 LSTM_ERR_TIMEOUT = 5
 LSTM_ERR_NOT_CORESIDENT = 6
 
-ABI_VERSION = 102  # the liblstm.h this binding mirrors (100 * major + minor)
+ABI_VERSION = 103  # the liblstm.h this binding mirrors (100 * major + minor)
 LSTM_F32 = 0
 LSTM_BF16 = 1
 LSTM_F16 = 2
@@ -31,7 +31,8 @@ LSTM_F16 = 2
 EXPORTS = ("lstm_fwd_workspace_size", "lstm_bwd_workspace_size", "lstm_fwd_workspace_size_ex",
            "lstm_fwd_workspace_size_max", "lstm_fwd", "lstm_bwd",
            "lstm_fwd_ex", "lstm_bwd_ex", "lstm_stack_fwd_workspace_size",
-           "lstm_stack_bwd_workspace_size", "lstm_stack_fwd", "lstm_stack_bwd",
+           "lstm_stack_bwd_workspace_size", "lstm_stack_bwd_workspace_size_min",
+           "lstm_stack_fwd", "lstm_stack_bwd",
            "lstm_status", "lstm_profile_begin", "lstm_profile_end", "lstm_launch_count",
            "lstm_strerror", "lstm_abi_version")
 
@@ -98,6 +99,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_stack_fwd_workspace_size.restype = sz
     lib.lstm_stack_bwd_workspace_size.argtypes = [dp, ip]
     lib.lstm_stack_bwd_workspace_size.restype = sz
+    lib.lstm_stack_bwd_workspace_size_min.argtypes = [dp, ip]
+    lib.lstm_stack_bwd_workspace_size_min.restype = sz
     lib.lstm_stack_fwd.argtypes = [dp, ip, op, vp, pp, pp] + [vp] * 7 + [vp, sz, vp]
     lib.lstm_stack_fwd.restype = ip
     lib.lstm_stack_bwd.argtypes = [dp, ip, op] + [vp] * 4 + [pp] + [vp] * 6 + [pp, pp] + \
@@ -127,7 +130,7 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_set_wait_fault.restype = ip
     lib.lstm_test_last_paths.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_paths.restype = ip
-    lib.lstm_test_last_stack_chunks.argtypes = []
+    lib.lstm_test_last_stack_chunks.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_stack_chunks.restype = ip
     lib.lstm_test_bwd_chunks.argtypes = [ip]
     lib.lstm_test_bwd_chunks.restype = ip
@@ -275,6 +278,11 @@ def stack_bwd_workspace_size(d: Dims, L: int) -> int:
     return int(load().lstm_stack_bwd_workspace_size(ctypes.byref(d), int(L)))
 
 
+def stack_bwd_workspace_size_min(d: Dims, L: int) -> int:
+    """The smallest workspace lstm_stack_bwd accepts (layers one after another)."""
+    return int(load().lstm_stack_bwd_workspace_size_min(ctypes.byref(d), int(L)))
+
+
 def lstm_stack_fwd(d: Dims, L: int, x, Ws, bs, h0, c0, y, hT, cT, gates, cells, ws,
                    ws_bytes=None, stream=None, check: bool = True, mask=None,
                    reverse: bool = False, gate_order="ifjo") -> int:
@@ -375,10 +383,12 @@ def test_last_paths():
     return f.value, b.value
 
 
-def test_last_stack_chunks() -> int:
-    """Test hook: chunks per layer of the last stack forward's layer wavefront
-    (0: layer after layer; -1: no stack forward yet)."""
-    return int(load().lstm_test_last_stack_chunks())
+def test_last_stack_chunks():
+    """Test hook: (forward, backward) chunks per layer of the last stack calls'
+    layer wavefronts (0: layer after layer; -1: no such call yet)."""
+    f, b = ctypes.c_int(), ctypes.c_int()
+    load().lstm_test_last_stack_chunks(ctypes.byref(f), ctypes.byref(b))
+    return f.value, b.value
 
 
 # ------------------------------------------------------------------ helpers

@@ -243,18 +243,30 @@ cudaError_t tc_input_projection(const lstm_dims *d, const E *x, const E *W, cons
 //   dW (+)= dG[rows]^T [h_prev | x][rows],   dx[rows] = dG[rows] W_x.
 // The operand maps end at the range's last row, so a partial 64-row K block
 // reads zeros rather than rows of the next range.  At most max_ctas CTAs
-// (0: one per SM).
+// (0: one per SM).  parts: DW_PART and / or DX_PART.
+constexpr int DW_PART = 1, DX_PART = 2;
 template <class E>
 cudaError_t tc_dw_dx(const lstm_dims *d, const E *dG, const E *x, const E *W, const E *h0,
                      const E *y, float *dW, float *dx, Ctrl *ctrl, cudaStream_t s, int t_lo,
-                     int t_hi, bool accumulate, int max_ctas, bool reverse = false) {
+                     int t_hi, bool accumulate, int max_ctas, bool reverse = false,
+                     int parts = DW_PART | DX_PART) {
     const long long B = d->B, H = d->H, I = d->I, G4 = 4 * H;
     const long long r0 = (long long)t_lo * B, r1 = (long long)t_hi * B;
     tcg::Builder bld(ctrl, Elem<E>::kFmt);
+    if (parts & DX_PART) {  // dx rows r0 .. r1-1 first in the tile queue
+        const int m_dg_k = bld.add_map({dG, r1, G4, G4}, 0, tcg::BM);
+        const int m_wx_mn = bld.add_map({W + H, G4, I, H + I}, 1, 0);
+        tcg::Problem &p2 = bld.add_problem((int)(r1 - r0), (int)I, 0, 1, dx + r0 * I, I, 0,
+                                           nullptr);
+        p2.a_mn0 = (int)r0;
+        tcg::Builder::add_seg(p2, m_dg_k, 0, m_wx_mn, 0, G4);
+    }
+    if (!(parts & DW_PART)) {
+        if (!bld.ok) return cudaErrorInvalidValue;
+        return tcg::launch(bld, s, max_ctas);
+    }
     const int m_dg_mn = bld.add_map({dG, r1, G4, G4}, 1, 0);
     const int m_x_mn = bld.add_map({x, r1, I, I}, 1, 0);
-    const int m_dg_k = bld.add_map({dG, r1, G4, G4}, 0, tcg::BM);
-    const int m_wx_mn = bld.add_map({W + H, G4, I, H + I}, 1, 0);
     tcg::Problem &p0 = bld.add_problem((int)G4, (int)H, 1, 1, dW, H + I, 0, nullptr);
     p0.accumulate = accumulate;
     if (!reverse) {
@@ -281,10 +293,6 @@ cudaError_t tc_dw_dx(const lstm_dims *d, const E *dG, const E *x, const E *W, co
     tcg::Problem &p1 = bld.add_problem((int)G4, (int)I, 1, 1, dW, H + I, (int)H, nullptr);
     p1.accumulate = accumulate;
     tcg::Builder::add_seg(p1, m_dg_mn, (int)r0, m_x_mn, (int)r0, r1 - r0);
-    // dx rows r0 .. r1-1
-    tcg::Problem &p2 = bld.add_problem((int)(r1 - r0), (int)I, 0, 1, dx + r0 * I, I, 0, nullptr);
-    p2.a_mn0 = (int)r0;
-    tcg::Builder::add_seg(p2, m_dg_k, 0, m_wx_mn, 0, G4);
     if (!bld.ok) return cudaErrorInvalidValue;
     return tcg::launch(bld, s, max_ctas);
 }
@@ -356,6 +364,47 @@ WaveStreams *wave_streams() {
     return w.ready ? &w : nullptr;
 }
 
+// Streams and events of the stacked backward's layer wavefront, per layer:
+// the recurrence (highest priority), the dx GEMM that feeds the layer below
+// (highest priority), and the dW GEMM (lowest), with an event per (layer,
+// chunk) for a finished recurrence chunk and for the next lower layer's dy
+// rows of that chunk.
+struct WaveBwdStreams {
+    cudaStream_t rec[kMaxWave] = {}, dxs[kMaxWave] = {}, gemm[kMaxWave] = {};
+    cudaEvent_t ev_rec[kMaxWave][kMaxChunks] = {}, ev_dy[kMaxWave][kMaxChunks] = {};
+    cudaEvent_t fork = nullptr, join[3 * kMaxWave] = {};
+    bool ready = false, tried = false;
+    std::mutex mu;
+};
+
+WaveBwdStreams *wave_bwd_streams() {
+    static std::mutex mu;
+    static WaveBwdStreams per_dev[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    WaveBwdStreams &w = per_dev[dev];
+    if (!w.tried) {
+        w.tried = true;
+        int lo = 0, hi = 0;
+        bool ok = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&w.fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int l = 0; ok && l < kMaxWave; ++l) {
+            ok = cudaStreamCreateWithPriority(&w.rec[l], cudaStreamNonBlocking, hi) == cudaSuccess &&
+                 cudaStreamCreateWithPriority(&w.dxs[l], cudaStreamNonBlocking, hi) == cudaSuccess &&
+                 cudaStreamCreateWithPriority(&w.gemm[l], cudaStreamNonBlocking, lo) == cudaSuccess;
+            for (int c = 0; ok && c < kMaxChunks; ++c)
+                ok = cudaEventCreateWithFlags(&w.ev_rec[l][c], cudaEventDisableTiming) == cudaSuccess &&
+                     cudaEventCreateWithFlags(&w.ev_dy[l][c], cudaEventDisableTiming) == cudaSuccess;
+        }
+        for (int i = 0; ok && i < 3 * kMaxWave; ++i)
+            ok = cudaEventCreateWithFlags(&w.join[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+        w.ready = ok;
+    }
+    return w.ready ? &w : nullptr;
+}
+
 // Number of reverse-time chunks of a backward call whose dW / dx GEMMs run
 // beside the recurrence (1: no overlap): at least 16 steps per chunk, at most
 // 8 chunks (the last chunk's GEMM is the part that cannot overlap; each chunk
@@ -387,7 +436,8 @@ int g_fault_skip_cta = -1;
 // Which recurrent kernel the last lstm_fwd / lstm_bwd used (test hook):
 // 0 per-step CUDA-core kernels, 1 persistent K-resident kernel, 2 cluster kernel.
 int g_last_fwd_path = -1, g_last_bwd_path = -1;
-int g_last_stack_chunks = -1;  // chunks per layer of the last stack forward's wavefront
+int g_last_stack_chunks = -1;      // chunks per layer of the last stack forward's wavefront
+int g_last_stack_bwd_chunks = -1;  // and of the last stack backward's
 unsigned long long g_wait_ns = 2000000000ull;
 
 struct RecPlan {
@@ -667,14 +717,15 @@ const void *fwd3_kernel_ptr(int NB, int KS, bool masked, int split) {
 // Forward with the input projection fused: the grid of plan_fwd2, and the
 // CTA's W_h and W_x K-slices must fit TMEM beside two accumulators.
 // LSTM_FWD_FUSED_X=0 turns it off (comparison runs).
-// max_ctas > 0 caps the grid (a layer of a stacked wavefront shares the SMs
-// with the layer beside it).
-bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked, int max_ctas = 0) {
+// share > 1: the plan takes at most 1/share of the SMs and of the clusters
+// that can be co-resident (a layer of a stacked wavefront runs beside
+// another layer's launch).
+bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked, int share = 1) {
     if (env_is("LSTM_FWD_FUSED_X", '0')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec2::F_UNITS != 0 || d->B < 1 || d->I < 1 ||
         d->I % 8 != 0 || tcg::encode_fn() == nullptr || force_simt())
         return false;
-    const int nsm = max_ctas > 0 ? std::min(max_ctas, tcg::sm_count()) : tcg::sm_count();
+    const int nsm = tcg::sm_count() / share;
     P.R = d->H / rec2::F_UNITS;
     for (int KS : {4, 2, 8, 1}) {
         if ((d->H / KS) % 64 != 0 || d->H % KS != 0) continue;
@@ -703,7 +754,7 @@ bool plan_fwd3(const lstm_dims *d, Rec2Plan &P, bool masked, int max_ctas = 0) {
                                    : fwd3_kernel_ptr<bf16>(NBv, KS, masked, split);
             if (!kern) continue;
             const int maxc = max_active_clusters(kern, rec2::F_THREADS, smem, KS);
-            if (G * P.R > maxc) continue;
+            if (G * P.R > maxc / share) continue;
             P.KS = KS; P.G = G; P.NB = NBv; P.kcc = kcc; P.kcx = kcx; P.smem = smem;
             P.split = split;
             P.family = 3;
@@ -754,7 +805,7 @@ bool plan_bwd2(const lstm_dims *d, Rec2Plan &P) {
 // fit TMEM beside the accumulator (H <= 1536) and the ring must stage one
 // exchange round (at least 4 stages, H >= 512).  LSTM_BWD_TMEM_W=0 turns it
 // off (comparison runs).
-bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
+bool plan_bwd3(const lstm_dims *d, Rec2Plan &P, int share = 1) {
     if (env_is("LSTM_BWD_TMEM_W", '0')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec3::UNITS != 0 || d->B < 1 ||
         tcg::encode_fn() == nullptr || force_simt())
@@ -770,7 +821,8 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
     const void *kern = d->dtype == LSTM_F16 ? (const void *)rec3::bwd3_kernel<__half, false, false>
                                             : (const void *)rec3::bwd3_kernel<bf16, false, false>;
     const int maxc = max_active_clusters(kern, rec3::THREADS, P.smem, P.KS);
-    const int gmax = std::min(maxc / P.R, kMaxGroups);
+    const int gmax = std::min(std::min(maxc / share / P.R, kMaxGroups),
+                              tcg::sm_count() / share / (P.R * P.KS));
     if (gmax < 1) return false;
     int G = std::min(gmax, (d->B + 15) / 16);
     int NB = ((d->B + G - 1) / G + 15) / 16 * 16;
@@ -789,7 +841,7 @@ bool plan_bwd3(const lstm_dims *d, Rec2Plan &P) {
 // Backward with two decoupled batch streams per group (rec4): the grid of
 // plan_bwd3 with groups of a multiple of 32 rows (two streams of a multiple of
 // 16), 384 threads, and each stream's ring staging its send blocks.
-bool plan_bwd4(const lstm_dims *d, Rec2Plan &P) {
+bool plan_bwd4(const lstm_dims *d, Rec2Plan &P, int share = 1) {
     if (env_is("LSTM_BWD_TMEM_W", '0') || env_is("LSTM_BWD_STREAMS", '1')) return false;
     if (d->dtype == LSTM_F32 || d->H % rec4::UNITS != 0 || d->B < 1 ||
         tcg::encode_fn() == nullptr || force_simt())
@@ -806,7 +858,8 @@ bool plan_bwd4(const lstm_dims *d, Rec2Plan &P) {
     const void *kern = d->dtype == LSTM_F16 ? (const void *)rec4::bwd4_kernel<__half, false, false>
                                             : (const void *)rec4::bwd4_kernel<bf16, false, false>;
     const int maxc = max_active_clusters(kern, rec4::THREADS, P.smem, P.KS);
-    const int gmax = std::min(maxc / P.R, kMaxGroups / rec4::NSTREAM);
+    const int gmax = std::min(std::min(maxc / share / P.R, kMaxGroups / rec4::NSTREAM),
+                              tcg::sm_count() / share / (P.R * P.KS));
     if (gmax < 1) return false;
     const int rows_max = rec4::NSTREAM * rec4::NBS_MAX;
     int G = std::min(gmax, (d->B + 31) / 32);
@@ -1015,7 +1068,7 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *
                    const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
                    const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
                    float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0,
-                   int i1, cudaStream_t s) {
+                   int i1, cudaStream_t s, int bar_base = 0) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
     rec3::Bwd3Params<E> prm;
     memset(&prm, 0, sizeof(prm));
@@ -1031,6 +1084,7 @@ int tc_bwd3_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
     prm.kcc = P.kcc; prm.stages = P.stages;
     prm.i0 = i0; prm.i1 = i1; prm.reverse = reverse;
+    prm.bar_base = bar_base;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
     const int nctas = P.R * P.KS * P.G;
@@ -1057,7 +1111,7 @@ int tc_bwd4_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *
                    const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
                    const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
                    float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl, int i0,
-                   int i1, cudaStream_t s) {
+                   int i1, cudaStream_t s, int bar_base = 0) {
     const long long T = d->T, B = d->B, H = d->H, G4 = 4 * H;
     rec4::Bwd4Params<E> prm;
     memset(&prm, 0, sizeof(prm));
@@ -1074,6 +1128,7 @@ int tc_bwd4_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const E *
     prm.T = (int)T; prm.B = (int)B; prm.H = (int)H; prm.U = P.R; prm.G = P.G; prm.NBr = P.NB;
     prm.NBS = NBS; prm.kcc = P.kcc; prm.stages = P.stages;
     prm.i0 = i0; prm.i1 = i1; prm.reverse = reverse;
+    prm.bar_base = bar_base;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
     const int nctas = P.R * P.KS * P.G;
@@ -1099,12 +1154,12 @@ int tc_bwd_tmem_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const
                        const float *dcT, const float *c0, const E *mask, bool reverse, bool ijfo,
                        const E *gates, const float *cells, E *dG, const E *WT, float *dbgroup,
                        float *dh0, float *dc0, float *dc_carry, float *dhp_carry, Ctrl *ctrl,
-                       int i0, int i1, cudaStream_t s) {
+                       int i0, int i1, cudaStream_t s, int bar_base = 0) {
     if (P.family == 4)
         return tc_bwd4_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
-                              dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s);
+                              dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s, bar_base);
     return tc_bwd3_launch(d, P, dy, dhT, dcT, c0, mask, reverse, ijfo, gates, cells, dG, WT,
-                          dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s);
+                          dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s, bar_base);
 }
 
 // W_h^T of a 16-bit W (bf16 or fp16: the kernel only moves 16-bit values)
@@ -1743,22 +1798,42 @@ bool stack_slices_aligned(const lstm_dims *d) {
     return (BH * (long long)esize(d)) % 16 == 0 && (BH * 4) % 16 == 0;
 }
 
+// Layer after layer: one layer's workspace, then the upper layer's dx (float)
+// and its compute-type copy, the next lower layer's dy (seq_total bytes).
+// Layer wavefront (16-bit stacks of 2 .. kMaxWave layers): the shared control
+// block, one layer workspace per layer (their recurrences run at once), then
+// per layer l >= 1 its dx (float) and the compute-type dy of layer l - 1
+// (wave_total bytes).  total, the size query's answer, covers both; a smaller
+// workspace of at least seq_total runs the layers one after another.
 struct StackBwdLayout {
-    size_t layer, dxbuf, dybuf, total;
+    size_t layer, dxbuf, dybuf, seq_total, wave_total, total;
+    size_t xb, yb;  // one T*B*H float / compute-type buffer, 256-aligned
+    size_t wave_region(int l) const { return kCtrlBytes + (size_t)l * layer; }
+    size_t wave_dx(int l) const { return wave_bufs + (size_t)(l - 1) * (xb + yb); }
+    size_t wave_dy(int l) const { return wave_dx(l + 1) + xb; }
+    size_t wave_bufs = 0;
 };
 StackBwdLayout stack_bwd_layout(const lstm_dims *d, int L) {
     StackBwdLayout S;
-    S.layer = bwd_layout(d).total;
+    S.layer = align_up(bwd_layout(d).total, 256);
     if (L > 1) {
         const lstm_dims d1 = layer_dims(d, 1);
-        S.layer = std::max(S.layer, bwd_layout(&d1).total);
+        S.layer = std::max(S.layer, align_up(bwd_layout(&d1).total, 256));
     }
-    S.dxbuf = S.dybuf = S.total = S.layer;
+    const size_t TBH = (size_t)d->T * d->B * d->H;
+    S.xb = align_up(TBH * sizeof(float), 256);
+    S.yb = align_up(TBH * esize(d), 256);
+    S.dxbuf = S.dybuf = S.seq_total = S.layer;
     if (L > 1) {  // dx of the layer above (float) and its compute-type copy
-        const size_t TBH = (size_t)d->T * d->B * d->H;
-        S.dybuf = align_up(S.dxbuf + TBH * sizeof(float), 256);
-        S.total = align_up(S.dybuf + TBH * esize(d), 256);
+        S.dybuf = S.dxbuf + S.xb;
+        S.seq_total = S.dybuf + S.yb;
     }
+    S.wave_total = 0;
+    if (L > 1 && L <= kMaxWave && d->dtype != LSTM_F32) {
+        S.wave_bufs = kCtrlBytes + (size_t)L * S.layer;
+        S.wave_total = S.wave_bufs + (size_t)(L - 1) * (S.xb + S.yb);
+    }
+    S.total = std::max(S.seq_total, S.wave_total);
     return S;
 }
 
@@ -1777,7 +1852,9 @@ size_t stack_fwd_ws(const lstm_dims *d, int L) {
 // layer's recurrence is the fused forward kernel on a grid of at most half
 // the SMs, launched once per chunk of consecutive steps on a stream of its
 // own; chunk c of layer l is ordered after chunk c of layer l-1 by an event
-// (no kernel waits on another kernel).  Both recurrences are latency bound,
+// (no kernel waits on another kernel).  Each layer's plan takes at most half
+// of the SMs and of the clusters that can be co-resident, so that two
+// layers' launches run at once.  Both recurrences are latency bound,
 // so two layers' chunks side by side each run at nearly their own speed.  A
 // chunk continues its layer from the saved h and c of the step before it, and
 // every launch has step counters of its own in the one control block.
@@ -1794,7 +1871,7 @@ int stack_fwd_wave(const lstm_dims *d, int L, bool reverse, bool ijfo, const E *
     Rec2Plan P[2];
     for (int k = 0; k < 2; ++k) {
         const lstm_dims dk = layer_dims(d, k);
-        if (!plan_fwd3(&dk, P[k], false, tcg::sm_count() / 2)) return LSTM_ERR_UNSUPPORTED;
+        if (!plan_fwd3(&dk, P[k], false, 2)) return LSTM_ERR_UNSUPPORTED;
     }
     auto counters = [&](int l) { return P[l > 0].G * P[l > 0].split; };
     int per_chunk = 0;  // step counters of one chunk of every layer
@@ -1909,6 +1986,156 @@ int stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
     return LSTM_OK;
 }
 
+// Layer wavefront of the stacked backward.  Layer l's reverse-time chunk c
+// needs layer l+1's dx over the same times (its dy) and its own delta h,
+// delta c after the chunk before, so it runs one chunk behind layer l+1
+// instead of after all of it.  Per layer: the TMEM-weight backward recurrence
+// on at most half the SMs and half the co-resident clusters (else two layers'
+// launches would run one after the other), in the reverse-time chunks of the
+// single-layer call, on a stream of its own; after each chunk, on a second stream, the dx
+// GEMM over the chunk's rows and its rounding to the compute type into the
+// lower layer's dy, which the lower layer's same chunk waits for (an event);
+// on a third, low-priority stream the chunk's dW GEMM (with the stack's dx for
+// layer 0).  No kernel waits on another kernel.  Every layer has its own
+// workspace region and step counters in the one control block.
+// LSTM_ERR_UNSUPPORTED / LSTM_ERR_NOT_CORESIDENT: the caller runs the layers
+// one after another instead (every output is rewritten from scratch).
+template <class E>
+int stack_bwd_wave(const lstm_dims *d, int L, bool reverse, bool ijfo, const E *dy,
+                   const E *dhT, const float *dcT, const E *x, const void *const *W, const E *h0,
+                   const float *c0, const E *y, const E *gates, const float *cells, float *dx,
+                   float *const *dW, float *const *db, float *dh0, float *dc0, char *ws,
+                   size_t ws_bytes, cudaStream_t s) {
+    if (L < 2 || L > kMaxWave || env_is("LSTM_STACK_WAVE", '0')) return LSTM_ERR_UNSUPPORTED;
+    const StackBwdLayout S = stack_bwd_layout(d, L);
+    if (S.wave_total == 0 || ws_bytes < S.wave_total) return LSTM_ERR_UNSUPPORTED;
+    const int T = d->T, nsm = tcg::sm_count();
+    const long long B = d->B, H = d->H, BH = B * H, TBH = (long long)T * BH, G4 = 4 * H;
+    const int nch = bwd_chunks(d);
+    if (nch < 2) return LSTM_ERR_UNSUPPORTED;
+    Rec2Plan P[2];  // layer 0, the layers above it
+    for (int k = 0; k < 2; ++k) {
+        const lstm_dims dk = layer_dims(d, k);
+        if (!tc_gemm_ok(&dk) ||
+            !(plan_bwd4(&dk, P[k], 2) || plan_bwd3(&dk, P[k], 2)))
+            return LSTM_ERR_UNSUPPORTED;
+    }
+    auto counters = [&](int l) { return P[l > 0].G * (P[l > 0].family == 4 ? 2 : 1); };
+    auto rec_ctas = [&](int l) { return P[l > 0].R * P[l > 0].KS * P[l > 0].G; };
+    int nbar = 0;
+    for (int l = 0; l < L; ++l) nbar += counters(l);
+    if (nbar > (int)(sizeof(((Ctrl *)nullptr)->bar) / sizeof(unsigned int)))
+        return LSTM_ERR_UNSUPPORTED;
+    WaveBwdStreams *Wv = wave_bwd_streams();
+    if (!Wv) return LSTM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(Wv->mu);
+    Ctrl *ctrl = (Ctrl *)ws;
+    if (reset_barriers(ws, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    // the GEMMs beside two layers' recurrences take at most the SMs those leave
+    const int gemm_ctas = std::max(8, nsm - rec_ctas(0) - rec_ctas(std::min(1, L - 1)));
+    if (cudaEventRecord(Wv->fork, s) != cudaSuccess) return LSTM_ERR_CUDA;
+    for (int l = 0; l < L; ++l)
+        if (cudaStreamWaitEvent(Wv->rec[l], Wv->fork, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(Wv->dxs[l], Wv->fork, 0) != cudaSuccess ||
+            cudaStreamWaitEvent(Wv->gemm[l], Wv->fork, 0) != cudaSuccess)
+            return LSTM_ERR_CUDA;
+    g_last_bwd_path = P[L > 1].family;
+    g_last_stack_bwd_chunks = nch;
+    const BwdLayout Lb0 = bwd_layout(d);
+    const lstm_dims d1 = layer_dims(d, 1);
+    const BwdLayout Lb1 = bwd_layout(&d1);
+    int rc = LSTM_OK;
+    for (int c = 0; c < nch && rc == LSTM_OK; ++c) {
+        const int i0 = chunk_bound(T, nch, c), i1 = chunk_bound(T, nch, c + 1);
+        // times of the chunk's steps T-i1 .. T-i0-1 (i0 .. i1-1 in reverse)
+        const long long t_lo = reverse ? i0 : T - i1, t_hi = reverse ? i1 : T - i0;
+        int bar = nbar;
+        for (int l = L - 1; l >= 0 && rc == LSTM_OK; --l) {
+            bar -= counters(l);
+            const lstm_dims dl = layer_dims(d, l);
+            const BwdLayout &Lb = l == 0 ? Lb0 : Lb1;
+            const Rec2Plan &Pl = P[l > 0];
+            char *reg = ws + S.wave_region(l);
+            E *dG = (E *)(reg + Lb.dG);
+            E *WT = (E *)(reg + Lb.wt);
+            float *dbgroup = (float *)(reg + Lb.dbgroup);
+            const E *dyl = l == L - 1 ? dy : (const E *)(ws + S.wave_dy(l));
+            const E *xl = l == 0 ? x : y + (l - 1) * TBH;
+            const E *Wl = (const E *)W[l];
+            const E *h0l = h0 ? h0 + l * BH : nullptr;
+            const float *c0l = c0 ? c0 + l * BH : nullptr;
+            cudaStream_t sr = Wv->rec[l], sx = Wv->dxs[l], sg = Wv->gemm[l];
+            {
+                prof::Phase ph(LSTM_PHASE_BWD_RECUR, sr);
+                if (c == 0 && launch_transpose_wh(&dl, Wl, WT, sr) != cudaSuccess) {
+                    rc = LSTM_ERR_CUDA;
+                    break;
+                }
+                if (l < L - 1 && cudaStreamWaitEvent(sr, Wv->ev_dy[l][c], 0) != cudaSuccess) {
+                    rc = LSTM_ERR_CUDA;
+                    break;
+                }
+                rc = tc_bwd_tmem_launch(&dl, Pl, dyl, dhT ? dhT + l * BH : nullptr,
+                                        dcT ? dcT + l * BH : nullptr, c0l, (const E *)nullptr,
+                                        reverse, ijfo, gates + 4 * l * TBH, cells + l * TBH, dG, WT,
+                                        dbgroup, dh0 + l * BH, dc0 + l * BH,
+                                        (float *)(reg + Lb.dc), (float *)(reg + Lb.dhp), ctrl, i0,
+                                        i1, sr, bar);
+                if (rc != LSTM_OK) break;
+                if (c + 1 == nch) {
+                    simt::colsum_final<<<(unsigned)((G4 + 255) / 256), 256, 0, sr>>>(
+                        dbgroup, Pl.G, (int)G4, db[l]);
+                    note_launch();
+                    if (cudaGetLastError() != cudaSuccess) rc = LSTM_ERR_CUDA;
+                }
+                if (rc == LSTM_OK && cudaEventRecord(Wv->ev_rec[l][c], sr) != cudaSuccess)
+                    rc = LSTM_ERR_CUDA;
+            }
+            if (rc != LSTM_OK) break;
+            if (l > 0) {  // this chunk's dx rows, rounded, are the lower layer's dy
+                prof::Phase ph(LSTM_PHASE_DX, sx);
+                float *dxl = (float *)(ws + S.wave_dx(l));
+                E *dyb = (E *)(ws + S.wave_dy(l - 1));
+                const long long n = (t_hi - t_lo) * BH;
+                if (cudaStreamWaitEvent(sx, Wv->ev_rec[l][c], 0) != cudaSuccess ||
+                    tc_dw_dx(&dl, (const E *)dG, xl, Wl, h0l, y + l * TBH, dW[l], dxl, ctrl, sx,
+                             (int)t_lo, (int)t_hi, false, gemm_ctas, reverse, DX_PART) !=
+                        cudaSuccess) {
+                    rc = LSTM_ERR_CUDA;
+                    break;
+                }
+                simt::from_float_copy<E><<<(unsigned)((n + 255) / 256), 256, 0, sx>>>(
+                    dxl + t_lo * BH, dyb + t_lo * BH, n);
+                note_launch();
+                if (cudaGetLastError() != cudaSuccess ||
+                    cudaEventRecord(Wv->ev_dy[l - 1][c], sx) != cudaSuccess) {
+                    rc = LSTM_ERR_CUDA;
+                    break;
+                }
+            }
+            {   // the chunk's dW (accumulated from the second chunk on); layer 0 also dx
+                prof::Phase ph(LSTM_PHASE_DW, sg);
+                const bool alone = l == 0 && c + 1 == nch;  // nothing else left to run
+                if (cudaStreamWaitEvent(sg, Wv->ev_rec[l][c], 0) != cudaSuccess ||
+                    tc_dw_dx(&dl, (const E *)dG, xl, Wl, h0l, y + l * TBH, dW[l],
+                             l == 0 ? dx : nullptr, ctrl, sg, (int)t_lo, (int)t_hi, c > 0,
+                             alone ? 0 : gemm_ctas, reverse,
+                             l == 0 ? (DW_PART | DX_PART) : DW_PART) != cudaSuccess)
+                    rc = LSTM_ERR_CUDA;
+            }
+        }
+    }
+    // join: nothing of this call stays unordered with the caller's stream
+    for (int l = 0; l < L; ++l) {
+        cudaStream_t st[3] = {Wv->rec[l], Wv->dxs[l], Wv->gemm[l]};
+        for (int k = 0; k < 3; ++k)
+            if (cudaEventRecord(Wv->join[3 * l + k], st[k]) != cudaSuccess ||
+                cudaStreamWaitEvent(s, Wv->join[3 * l + k], 0) != cudaSuccess)
+                return LSTM_ERR_CUDA;
+    }
+    return rc;
+}
+
 // Layers L-1 .. 0, each one lstm_bwd_ex call; between two calls the float dx
 // of the upper layer becomes the lower layer's dy in the compute type.
 int stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy,
@@ -1925,7 +2152,7 @@ int stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy
     }
     if (L > 1 && !stack_slices_aligned(d)) return LSTM_ERR_UNSUPPORTED;
     const StackBwdLayout S = stack_bwd_layout(d, L);
-    const int wsrc = ws_ok(ws, ws_bytes, S.total);
+    const int wsrc = ws_ok(ws, ws_bytes, S.seq_total);
     if (wsrc != LSTM_OK) return wsrc;
     const size_t es = esize(d);
     const long long BH = (long long)d->B * d->H, TBH = (long long)d->T * BH;
@@ -1933,6 +2160,35 @@ int stack_bwd(const lstm_dims *d, int L, const lstm_options *opt, const void *dy
     float *dxbuf = reinterpret_cast<float *>(wsb + S.dxbuf);
     void *dybuf = wsb + S.dybuf;
     cudaStream_t s = (cudaStream_t)stream;
+    g_last_stack_bwd_chunks = 0;
+    // the layer wavefront where it applies (16-bit types, no length mask, the
+    // wavefront's workspace)
+    const int dir = opt ? opt->direction : LSTM_DIR_FORWARD;
+    const int order = opt ? opt->gate_order : LSTM_GATES_IFJO;
+    if (L > 1 && d->dtype != LSTM_F32 && !(opt && opt->seq_mask) && dims_supported(d) &&
+        (dir == LSTM_DIR_FORWARD || dir == LSTM_DIR_REVERSE) &&
+        (order == LSTM_GATES_IFJO || order == LSTM_GATES_IJFO) && TBH > 0 &&
+        ws_bytes >= S.wave_total && S.wave_total > 0 &&
+        ptr_ok(dy, false) && ptr_ok(dhT, false) && ptr_ok(dcT, false) &&
+        ptr_ok(x, (long long)d->T * d->B * d->I > 0) && ptr_ok(h0, false) && ptr_ok(c0, false) &&
+        ptr_ok(y, true) && ptr_ok(gates, true) && ptr_ok(cells, true) &&
+        ptr_ok(dx, (long long)d->T * d->B * d->I > 0) && ptr_ok(dh0, true) &&
+        ptr_ok(dc0, true)) {
+        const bool rev = dir == LSTM_DIR_REVERSE, ijfo = order == LSTM_GATES_IJFO;
+        int rc;
+        if (d->dtype == LSTM_F16)
+            rc = stack_bwd_wave<__half>(d, L, rev, ijfo, (const __half *)dy, (const __half *)dhT,
+                                        dcT, (const __half *)x, W, (const __half *)h0, c0,
+                                        (const __half *)y, (const __half *)gates, cells, dx, dW,
+                                        db, dh0, dc0, wsb, ws_bytes, s);
+        else
+            rc = stack_bwd_wave<bf16>(d, L, rev, ijfo, (const bf16 *)dy, (const bf16 *)dhT, dcT,
+                                      (const bf16 *)x, W, (const bf16 *)h0, c0, (const bf16 *)y,
+                                      (const bf16 *)gates, cells, dx, dW, db, dh0, dc0, wsb,
+                                      ws_bytes, s);
+        if (rc != LSTM_ERR_UNSUPPORTED && rc != LSTM_ERR_NOT_CORESIDENT) return rc;
+        g_last_stack_bwd_chunks = 0;
+    }
     for (int l = L - 1; l >= 0; --l) {
         const lstm_dims dl = layer_dims(d, l);
         const void *xl = l == 0 ? x : static_cast<const char *>(y) + (size_t)(l - 1) * TBH * es;
@@ -2038,6 +2294,11 @@ size_t lstm_stack_fwd_workspace_size(const lstm_dims *d, int L) {
 size_t lstm_stack_bwd_workspace_size(const lstm_dims *d, int L) {
     if (!dims_ok(d) || L < 1) return 0;
     return stack_bwd_layout(d, L).total;
+}
+
+size_t lstm_stack_bwd_workspace_size_min(const lstm_dims *d, int L) {
+    if (!dims_ok(d) || L < 1) return 0;
+    return stack_bwd_layout(d, L).seq_total;
 }
 
 int lstm_stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
@@ -2148,7 +2409,11 @@ int lstm_test_chunk_bound(int T, int nch, int c) {
     return chunk_bound(T, nch, c);
 }
 
-int lstm_test_last_stack_chunks(void) { return g_last_stack_chunks; }
+int lstm_test_last_stack_chunks(int *fwd_chunks, int *bwd_chunks) {
+    if (fwd_chunks) *fwd_chunks = g_last_stack_chunks;
+    if (bwd_chunks) *bwd_chunks = g_last_stack_bwd_chunks;
+    return LSTM_OK;
+}
 
 int lstm_test_last_paths(int *fwd_path, int *bwd_path) {
     if (fwd_path) *fwd_path = g_last_fwd_path;

@@ -67,6 +67,7 @@ struct Bwd3Params {
     int T, B, H, U, G, NBr, kcc, stages;
     int i0, i1;       // this launch runs epilogue iterations i0 .. i1-1 (step T-1-i)
     int reverse;      // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
+    int bar_base;     // first of the call's G step counters in ctrl->bar
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd3_kernel(const __grid_constant_
     auto tau = [&](int s) { return p.reverse ? T - 1 - s : s; };
     const int kslice = kcc * 64;              // this CTA's part of the 4H axis
     const int kbase = (int)kpart * kslice;
-    unsigned int *ctr = &p.ctrl->bar[gi];
+    unsigned int *ctr = &p.ctrl->bar[p.bar_base + gi];
     const unsigned int group_ctas = (unsigned)(p.U * KS);
 
     if (threadIdx.x == 0) {

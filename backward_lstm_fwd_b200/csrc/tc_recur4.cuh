@@ -55,6 +55,7 @@ struct Bwd4Params {
     int T, B, H, U, G, NBr, NBS, kcc, stages;
     int i0, i1;        // this launch runs epilogue iterations i0 .. i1-1 (step T-1-i)
     int reverse;       // direction "REDIRECTIONAL": recurrence step s is at time T-1-s
+    int bar_base;      // first of the call's G * NSTREAM step counters in ctrl->bar
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
         const int s = warp;
         if (lane == 0) {
             uint8_t *ring = smem + L.ring[s];
-            unsigned int *ctr = &p.ctrl->bar[gi * NSTREAM + s];
+            unsigned int *ctr = &p.ctrl->bar[p.bar_base + gi * NSTREAM + s];
             const uint32_t bytes = (uint32_t)NBS * 128;
             uint32_t stage = 0, ph = 0;
             bool aborted = false;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(THREADS, 1) bwd4_kernel(const __grid_constant_
         float *recv = reinterpret_cast<float *>(smem + L.recv[sw]);
         float *stage_buf = reinterpret_cast<float *>(smem + L.ring[sw]);
         uint64_t *rf = &recv_full[sw];
-        unsigned int *ctr = &p.ctrl->bar[gi * NSTREAM + sw];
+        unsigned int *ctr = &p.ctrl->bar[p.bar_base + gi * NSTREAM + sw];
         // pointwise part: batch row m of the stream, 8 of the CTA's 16 units
         const int m = wt & (NBS_MAX - 1);
         const int uo = 8 * (wt / NBS_MAX);

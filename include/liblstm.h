@@ -217,8 +217,17 @@ int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, con
  * Cells" of the "mxnet-lstm" page).  Layer 0 reads x [T][B][I]; layer l > 0
  * reads the outputs y of layer l-1.  Every layer has its own weights, bias
  * and initial state, and its final state is an output of its own; only y
- * passes upward.  Each layer is one lstm_fwd_ex / lstm_bwd_ex call (in that
- * order on `stream`), so options, precision and errors are those calls'.
+ * passes upward.  The stack computes what one lstm_fwd_ex / lstm_bwd_ex call
+ * per layer (in that order) computes, with those calls' options, precision
+ * and errors.  For 16-bit stacks without a length mask whose layers each fit
+ * on half the device, the layers run as a layer wavefront: each layer in
+ * chunks of consecutive steps on an internal stream of its own, a layer's
+ * chunk after the same chunk of the layer below (forward) or above
+ * (backward), all ordered after earlier work on `stream` and before later
+ * work on it.  The wavefront's forward plans each layer on half the SMs,
+ * whose summation order may differ from the whole-device plan (results
+ * within the compute type's tolerance); its backward gives the bits of the
+ * layer-by-layer backward.
  *
  * d       sizes and compute type of layer 0; layer l > 0 has I = H.
  * L       number of layers (< 1: LSTM_ERR_INVALID_ARG).
@@ -240,13 +249,18 @@ int lstm_bwd_ex(const lstm_dims *d, const lstm_options *opt, const void *dy, con
  * (float), either NULL, the gradients at every layer's final state.  Outputs
  * (float): dx [T][B][I]; dW and db, HOST arrays of L DEVICE pointers to
  * dW[l] [4H][H + I_l] and db[l] [4H]; dh0, dc0 [L][B][H].  Layer l-1's dy is
- * layer l's dx rounded to the compute type.  ws at least
- * lstm_stack_bwd_workspace_size(d, L) bytes.  The layers run L-1 .. 0.
+ * layer l's dx rounded to the compute type.  ws:
+ * lstm_stack_bwd_workspace_size(d, L) bytes (with the layer wavefront, one
+ * layer workspace per layer); a workspace of at least
+ * lstm_stack_bwd_workspace_size_min(d, L) bytes (one layer workspace and the
+ * dx / dy buffers between two layers) runs the layers one after another,
+ * L-1 .. 0; a smaller one is LSTM_ERR_WORKSPACE.
  */
 /* (The stack's forward workspace covers every plan of every layer, like
  * lstm_fwd_workspace_size_max.) */
 size_t lstm_stack_fwd_workspace_size(const lstm_dims *d, int L);
 size_t lstm_stack_bwd_workspace_size(const lstm_dims *d, int L);
+size_t lstm_stack_bwd_workspace_size_min(const lstm_dims *d, int L);
 int lstm_stack_fwd(const lstm_dims *d, int L, const lstm_options *opt, const void *x,
                    const void *const *W, const void *const *b, const void *h0, const float *c0,
                    void *y, void *hT, float *cT, void *gates, float *cells, void *ws,
@@ -335,8 +349,9 @@ const char *lstm_strerror(int code);
 
 /* ABI version: 100 * major + minor (1.1: lstm_options with gate_order, the
  * LSTM_F16 compute type and the stack entry points; 1.2: the plan-aware
- * forward workspace sizes and lstm_fwd_noalloc_status). */
-#define LSTM_ABI_VERSION 102
+ * forward workspace sizes and lstm_fwd_noalloc_status; 1.3: the stacked
+ * layer wavefront and lstm_stack_bwd_workspace_size_min). */
+#define LSTM_ABI_VERSION 103
 int lstm_abi_version(void);
 
 #ifdef __cplusplus

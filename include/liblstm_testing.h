@@ -28,9 +28,10 @@
  *   LSTM_PERSIST=0         run the CUDA-core recurrences (fp32, and 16-bit
  *                          shapes off the tensor-core grids) as one launch
  *                          per step instead of one persistent launch.
- *   LSTM_STACK_WAVE=0      run the layers of lstm_stack_fwd one after another
- *                          instead of as a layer wavefront (two layers' time
- *                          chunks side by side on half the SMs each).
+ *   LSTM_STACK_WAVE=0      run the layers of lstm_stack_fwd / lstm_stack_bwd
+ *                          one after another instead of as a layer wavefront
+ *                          (two layers' time chunks side by side on half the
+ *                          SMs each).
  *   LSTM_STACK_CHUNKS=n    chunks per layer of that wavefront (1..8; 1 = each
  *                          layer in one launch, after the layer below it).
  *                          Default: min(8, T / 8), and no wavefront below 2.
@@ -90,11 +91,11 @@ int lstm_test_set_wait_fault(int skip_cta, long long wait_ns);
 int lstm_test_last_paths(int *fwd_path, int *bwd_path);
 
 /*
- * Chunks per layer of the layer wavefront that the most recent
- * lstm_stack_fwd of this process ran (0: its layers ran one after another;
- * -1: none yet).
+ * Chunks per layer of the layer wavefronts that the most recent
+ * lstm_stack_fwd and lstm_stack_bwd of this process ran (0: its layers ran
+ * one after another; -1: none yet).
  */
-int lstm_test_last_stack_chunks(void);
+int lstm_test_last_stack_chunks(int *fwd_chunks, int *bwd_chunks);
 
 /*
  * Reverse-time chunking of the tensor-core backward: the number of chunk

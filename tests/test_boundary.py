@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
     assert set(names) >= set(L.EXPORTS)
     for n in names:
         assert hasattr(lib, n), f"{n} declared in liblstm.h but not exported"
-    assert lib.lstm_abi_version() == L.ABI_VERSION == 102
+    assert lib.lstm_abi_version() == L.ABI_VERSION == 103
 
 
 def declared_arities():
@@ -273,11 +273,22 @@ def test_stack_workspace_sizes(lib):
     upper = L.bwd_workspace_size(L.dims(4, 8, 32, 32, L.LSTM_BF16))
     assert L.stack_fwd_workspace_size(DS, 1) == L.fwd_workspace_size_max(DS)
     assert L.stack_bwd_workspace_size(DS, 1) == one
-    # two layers: the larger layer's workspace plus dx (float) and dy (bf16)
-    # of the upper layer, [T][B][H] each
+    assert L.stack_bwd_workspace_size_min(DS, 1) == one
+    # two layers, one after another: the larger layer's workspace plus dx
+    # (float) and dy (bf16) of the upper layer, [T][B][H] each
     need = max(one, upper) + 4 * 8 * 32 * (4 + 2)
-    assert L.stack_bwd_workspace_size(DS, 2) >= need
+    assert L.stack_bwd_workspace_size_min(DS, 2) >= need
+    # the layer wavefront: the control block and a workspace per layer, plus
+    # those two buffers between each pair of layers
+    for Lc in (2, 3):
+        wave = 256 + Lc * max(one, upper) + (Lc - 1) * 4 * 8 * 32 * (4 + 2)
+        assert L.stack_bwd_workspace_size(DS, Lc) >= wave
+        assert L.stack_bwd_workspace_size(DS, Lc) > L.stack_bwd_workspace_size_min(DS, Lc)
+    # float stacks run layer after layer only
+    DF = L.dims(4, 8, 16, 32, L.LSTM_F32)
+    assert L.stack_bwd_workspace_size(DF, 2) == L.stack_bwd_workspace_size_min(DF, 2)
     assert L.stack_bwd_workspace_size(DS, 0) == 0 and L.stack_fwd_workspace_size(DS, -1) == 0
+    assert L.stack_bwd_workspace_size_min(DS, 0) == 0
 
 
 @pytest.mark.parametrize("Lc", [0, -2])
@@ -305,7 +316,7 @@ def test_stack_slices_must_align(lib):
 
 
 def test_stack_workspace_too_small(lib):
-    need = L.stack_bwd_workspace_size(DS, 2)
+    need = L.stack_bwd_workspace_size_min(DS, 2)
     assert call_stack_bwd(DS, 2, ws_bytes=need - 1) == L.LSTM_ERR_WORKSPACE
 
 

@@ -125,7 +125,7 @@ def test_stack_wavefront_chunks_are_seamless(case, cuda_device, monkeypatch):
         outs[label] = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"], reverse=reverse,
                                       gate_order=order)
         torch.cuda.synchronize()
-        assert L.test_last_stack_chunks() == want, label
+        assert L.test_last_stack_chunks()[0] == want, label
     a, b = outs["chunked"], outs["one launch"]
     for k in ("y", "hT", "cT", "gates", "cells"):
         assert torch.equal(getattr(a, k), getattr(b, k)), k
@@ -143,6 +143,61 @@ def test_stack_wavefront_chunks_are_seamless(case, cuda_device, monkeypatch):
                        getattr(seq, k).float().cpu().double().numpy())
             for k in ("y", "hT", "cT")}
     assert_within(errs, dt, f"wavefront vs layer by layer {case}")
+
+
+# (T, B, I, H, L, dtype, reverse, gate order, backward chunks per layer)
+WAVE_BWD_CASES = [
+    (64, 64, 512, 512, 2, "bf16", False, "ifjo", 4),
+    (48, 64, 1024, 512, 3, "fp16", False, "ifjo", 3),
+    (40, 128, 256, 512, 2, "bf16", True, "ijfo", 2),   # reverse direction
+]
+
+
+@pytest.mark.parametrize("case", WAVE_BWD_CASES)
+def test_stack_backward_wavefront_equals_layer_by_layer(case, cuda_device):
+    """The backward layer wavefront runs each layer's reverse-time chunks on a
+    stream of its own; after a chunk, the dx GEMM over its rows and the
+    rounding to the compute type give the lower layer the dy of the same
+    chunk, which its chunk waits for.  The chunks, kernels, GEMM tiles and
+    accumulation order are those of the layer-by-layer backward, so dx, dW,
+    dh0 and dc0 are the same bits; db, whose batch sum runs per batch group,
+    follows the wavefront's grid (half the co-resident clusters per layer)
+    in its order of additions.  The layer-by-layer run here is the fallback a
+    caller gets from a workspace smaller than the wavefront's (but at least the
+    layer-by-layer size); both match the oracle (the first case through the
+    oracle cases of CASES, the others here)."""
+    T, B, I, H, Lc, dt, reverse, order, nch = case
+    inp = stack_inputs(T, B, I, H, Lc, dt, seed=3 * T + Lc)
+    d = {k: ([t.to(cuda_device) for t in v] if isinstance(v, list) else v.to(cuda_device))
+         for k, v in inp.items()}
+    st = L.forward_stack(d["x"], d["W"], d["b"], d["h0"], d["c0"], reverse=reverse,
+                         gate_order=order)
+    full = L.stack_bwd_workspace_size(st.dims, Lc)
+    least = L.stack_bwd_workspace_size_min(st.dims, Lc)
+    assert least < full
+    grads = {}
+    for label, nbytes, want in (("wavefront", full, nch), ("layer by layer", full - 1, 0),
+                                ("smallest", least, 0)):
+        ws = L.empty_workspace(nbytes, cuda_device)[:nbytes]
+        grads[label] = L.backward_stack(st, d["x"], d["W"], d["h0"], d["c0"], d["dy"], d["dhT"],
+                                        d["dcT"], ws=ws, reverse=reverse, gate_order=order)
+        torch.cuda.synchronize()
+        assert L.test_last_stack_chunks()[1] == want, label
+    a = grads["wavefront"]
+    for b in (grads["layer by layer"], grads["smallest"]):
+        for k in ("dx", "dh0", "dc0"):
+            assert torch.equal(getattr(a, k), getattr(b, k)), k
+        for l in range(Lc):
+            assert torch.equal(a.dW[l], b.dW[l]), l
+            # db adds its batch rows per batch group of the plan, then the
+            # groups: the order (not the terms) follows the grid
+            torch.testing.assert_close(a.db[l], b.db[l], rtol=1e-5, atol=1e-5)
+    if case != WAVE_BWD_CASES[0]:
+        n = lambda t: t.float().cpu().double().numpy()
+        gpu = dict(y=n(st.y), hT=n(st.hT), cT=n(st.cT), dx=n(a.dx), dh0=n(a.dh0), dc0=n(a.dc0),
+                   dW=[n(t) for t in a.dW], db=[n(t) for t in a.db], L=Lc)
+        check(gpu, run_oracle_stack(inp, reverse=reverse, gate_order=order), dt,
+              f"stack backward wavefront {case}")
 
 
 def test_stack_with_options(cuda_device):
