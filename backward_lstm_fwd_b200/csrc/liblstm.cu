@@ -1193,6 +1193,30 @@ int tc_bwd_recurrence3(const lstm_dims *d, const Rec2Plan &P, const E *dy, const
     return cudaGetLastError() == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
+// One warp that returns `ns` nanoseconds after it starts (at most 2^20 naps
+// of 256 ns).  In a stream before a GEMM that becomes ready at the moment the
+// next launch of a persistent cluster kernel does, it lets that launch take
+// its SMs first: a GEMM placed CTA by CTA on the SMs just freed can break up
+// the cluster slots the launch needs, which then waits for the GEMM to end.
+// It touches no memory and needs so few resources that it fits beside any
+// resident kernel, so it never holds an SM that launch needs.
+__global__ void __launch_bounds__(32, 1) hold_ns(unsigned long long ns) {
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (int i = 0; i < (1 << 20); ++i) {
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 >= ns) break;
+        __nanosleep(256);
+    }
+}
+constexpr unsigned long long kGemmHoldNs = 8000;
+
+cudaError_t launch_hold(cudaStream_t s) {
+    hold_ns<<<1, 32, 0, s>>>(kGemmHoldNs);
+    note_launch();
+    return cudaGetLastError();
+}
+
 // a3 + a5 in `nch` reverse-time chunks (one launch each, delta c carried
 // through the workspace) on a high-priority stream, and a4 + a6 of every
 // finished chunk on a low-priority stream, beside the next chunk: the GEMM
@@ -1231,7 +1255,8 @@ int tc_bwd3_overlapped(const lstm_dims *d, const Rec2Plan &P, AuxStreams &A, int
                                     A.rec);
             if (rc != LSTM_OK) break;
             if (cudaEventRecord(A.ev[c], A.rec) != cudaSuccess ||
-                cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess) {
+                cudaStreamWaitEvent(A.gemm, A.ev[c], 0) != cudaSuccess ||
+                (c + 1 < nch && launch_hold(A.gemm) != cudaSuccess)) {
                 rc = LSTM_ERR_CUDA;
                 break;
             }
@@ -2098,6 +2123,7 @@ int stack_bwd_wave(const lstm_dims *d, int L, bool reverse, bool ijfo, const E *
                 E *dyb = (E *)(ws + S.wave_dy(l - 1));
                 const long long n = (t_hi - t_lo) * BH;
                 if (cudaStreamWaitEvent(sx, Wv->ev_rec[l][c], 0) != cudaSuccess ||
+                    launch_hold(sx) != cudaSuccess ||
                     tc_dw_dx(&dl, (const E *)dG, xl, Wl, h0l, y + l * TBH, dW[l], dxl, ctrl, sx,
                              (int)t_lo, (int)t_hi, false, gemm_ctas, reverse, DX_PART) !=
                         cudaSuccess) {
@@ -2117,6 +2143,7 @@ int stack_bwd_wave(const lstm_dims *d, int L, bool reverse, bool ijfo, const E *
                 prof::Phase ph(LSTM_PHASE_DW, sg);
                 const bool alone = l == 0 && c + 1 == nch;  // nothing else left to run
                 if (cudaStreamWaitEvent(sg, Wv->ev_rec[l][c], 0) != cudaSuccess ||
+                    (!alone && launch_hold(sg) != cudaSuccess) ||
                     tc_dw_dx(&dl, (const E *)dG, xl, Wl, h0l, y + l * TBH, dW[l],
                              l == 0 ? dx : nullptr, ctrl, sg, (int)t_lo, (int)t_hi, c > 0,
                              alone ? 0 : gemm_ctas, reverse,
