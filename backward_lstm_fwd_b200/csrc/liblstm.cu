@@ -1314,9 +1314,10 @@ cudaError_t launch_persistent(Kern kern, const Prm &prm, int grid, size_t smem, 
 // Units per CTA of the persistent recurrences: every SM holds a slice (the
 // backward in quads of units, the grain of its epilogue), within the shared
 // memory budget and the kernels' per-thread item limit.  K is staged in
-// chunks of at most 8192 floats over all B rows (fewer syncs than small
-// chunks, and every thread has several loads in flight), and each item's dot
-// product is split over the lanes the CTA would otherwise leave idle.
+// chunks of at most 16384 floats over all B rows, halved until they fit
+// beside the weights (fewer syncs than small chunks, and every thread has
+// several loads in flight), and each item's dot product is split over the
+// lanes the CTA would otherwise leave idle.
 struct PstPlan {
     int UN = 0, P = 0, KC = 0, KSPLIT = 1;
     size_t smem = 0;
@@ -1331,10 +1332,14 @@ bool plan_persist(const lstm_dims *d, bool backward, PstPlan &Q) {
     const long long items = (long long)d->B * (backward ? Q.UN / 4 : Q.UN);
     if (items > (long long)pst::MAXP * pst::NTHR || Q.P > nsm) return false;
     const int K = backward ? 4 * d->H : d->H;
-    Q.KC = std::min(std::max(32, 8192 / d->B / 32 * 32), (K + 31) / 32 * 32);
     Q.KSPLIT = 1;
     while (Q.KSPLIT < 32 && items * Q.KSPLIT * 2 <= pst::NTHR) Q.KSPLIT *= 2;
-    Q.smem = backward ? pst::bwd_smem(d->B, d->H, Q.UN, Q.KC) : pst::fwd_smem(d->B, d->H, Q.UN, Q.KC);
+    auto smem = [&](int kc) {
+        return backward ? pst::bwd_smem(d->B, d->H, Q.UN, kc) : pst::fwd_smem(d->B, d->H, Q.UN, kc);
+    };
+    Q.KC = std::min(std::max(32, 16384 / d->B / 32 * 32), (K + 31) / 32 * 32);
+    while (Q.KC > 32 && smem(Q.KC) > kMaxSmem) Q.KC = std::max(32, Q.KC / 2 / 32 * 32);
+    Q.smem = smem(Q.KC);
     return Q.smem <= kMaxSmem;
 }
 

@@ -17,6 +17,8 @@
 // slice of the units.
 #pragma once
 
+#include <type_traits>
+
 #include "simt.cuh"
 #include "tc_recur.cuh"  // rec::ld_acquire_u32 / red_release_add / wait_counter
 
@@ -28,8 +30,9 @@ constexpr int MAXP = 4;         // (row, unit) pairs / (row, unit quad) items pe
 constexpr int STAGE_UNR = 8;    // operand loads in flight per thread while staging
 
 // The step's operand is staged in K chunks of KC (a multiple of 32 the host
-// picks so that a chunk of all B rows holds at most 8192 floats), rows padded
-// to KC + 1 floats so that rows m, m+1, ... start in different banks.  Each
+// picks so that a chunk of all B rows holds at most 16384 floats, within the
+// shared memory left beside the weights), rows padded to KC + 1 floats so that
+// rows m, m+1, ... start in different banks.  Each
 // output item's dot product is split over KSPLIT lanes of one warp (a power of
 // two <= 32 the host picks so that items x KSPLIT fill the CTA): lane `ks`
 // of the group takes k = ks, ks + KSPLIT, ... of every chunk and the group's
@@ -91,13 +94,58 @@ __device__ __forceinline__ bool grid_step(unsigned int *ctr, unsigned int target
     return ok_s != 0;
 }
 
+// 16 bytes of T as floats: the element type of one vector load
+__device__ __forceinline__ void to_f4(const float4 &v, float *o) {
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+template <class T>
+__device__ __forceinline__ void to_f8(const uint4 &v, float *o) {
+    const T *e = reinterpret_cast<const T *>(&v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = to_f(e[i]);
+}
+
 // Rows [0, B) x columns [k0, k0 + kn) of a row-major operand with row pitch
 // `ld` into dst[B][KC + 1] as fp32 (zeros past kn), by all threads, with
-// STAGE_UNR independent loads in flight per thread.
+// STAGE_UNR independent loads in flight per thread: 16-byte loads when every
+// row's slice starts on a 16-byte boundary and holds whole vectors, else
+// element loads.
 template <class T>
 __device__ __forceinline__ void stage_chunk(float *dst, const T *src, long long ld, int B, int k0,
                                             int kn, int KC) {
-    const int n = B * KC, KCP = KC + 1;
+    const int KCP = KC + 1;
+    constexpr int V = 16 / (int)sizeof(T);  // elements per 16-byte load
+    if (KC % V == 0 && kn % V == 0 && k0 % V == 0 && ld % V == 0 &&
+        ((uintptr_t)src & 15u) == 0) {
+        const int vpr = KC / V, nv = B * vpr;  // vectors per row, per chunk
+        for (int base = threadIdx.x; base < nv; base += NTHR * STAGE_UNR) {
+            typedef typename std::conditional<sizeof(T) == 4, float4, uint4>::type Vt;
+            Vt v[STAGE_UNR];
+#pragma unroll
+            for (int u = 0; u < STAGE_UNR; ++u) {
+                const int e = base + u * NTHR;
+                const int m = e / vpr, kk = (e - m * vpr) * V;
+                if (e < nv && kk < kn)
+                    v[u] = *reinterpret_cast<const Vt *>(src + (long long)m * ld + k0 + kk);
+                else
+                    memset(&v[u], 0, sizeof(Vt));
+            }
+#pragma unroll
+            for (int u = 0; u < STAGE_UNR; ++u) {
+                const int e = base + u * NTHR;
+                if (e < nv) {
+                    const int m = e / vpr, kk = (e - m * vpr) * V;
+                    float f[V];
+                    if constexpr (sizeof(T) == 4) to_f4(v[u], f);
+                    else to_f8<T>(v[u], f);
+#pragma unroll
+                    for (int i = 0; i < V; ++i) dst[m * KCP + kk + i] = f[i];
+                }
+            }
+        }
+        return;
+    }
+    const int n = B * KC;
     for (int base = threadIdx.x; base < n; base += NTHR * STAGE_UNR) {
         float v[STAGE_UNR];
 #pragma unroll
