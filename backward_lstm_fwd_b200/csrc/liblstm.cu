@@ -407,11 +407,12 @@ WaveBwdStreams *wave_bwd_streams() {
 
 // Number of reverse-time chunks of a backward call whose dW / dx GEMMs run
 // beside the recurrence (1: no overlap): at least 16 steps per chunk, at most
-// 8 chunks (the last chunk's GEMM is the part that cannot overlap; each chunk
-// costs one more launch of the recurrence).  LSTM_BWD_CHUNKS overrides.
+// 6 chunks (the last chunk's GEMM is the part that cannot overlap; each chunk
+// costs one more launch of the recurrence, with its weights loaded again).
+// LSTM_BWD_CHUNKS overrides.
 int bwd_chunks(const lstm_dims *d) {
     const char *e = getenv("LSTM_BWD_CHUNKS");
-    int n = e ? atoi(e) : (d->T >= 32 ? std::min(8, d->T / 16) : 1);
+    int n = e ? atoi(e) : (d->T >= 32 ? std::min(6, d->T / 16) : 1);
     return std::max(1, std::min(std::min(n, kMaxChunks), d->T));
 }
 

@@ -37,7 +37,7 @@
  *                          Default: min(8, T / 8), and no wavefront below 2.
  *   LSTM_BWD_CHUNKS=n      run the tensor-core backward recurrence in n
  *                          reverse-time chunks (1..16; 1 = one launch, dW / dx
- *                          after it).  Default: min(8, T / 16), 1 below T = 32.
+ *                          after it).  Default: min(6, T / 16), 1 below T = 32.
  *   LSTM_LAUNCH_NONCOOP=1  launch the persistent cluster kernels without the
  *                          cooperative attribute, after the same co-residency
  *                          check (profilers cannot replay cooperative cluster

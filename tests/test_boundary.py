@@ -346,14 +346,14 @@ def test_dtype_codes():
 
 def test_backward_chunking_host_logic(lib, monkeypatch):
     """The reverse-time chunks of the tensor-core backward (host logic, no
-    GPU): min(8, T/16) chunks from T = 32 on, one below; boundaries strictly
+    GPU): min(6, T/16) chunks from T = 32 on, one below; boundaries strictly
     increasing from 0 to T; sizes shrinking geometrically, so that the last
     chunk (whose dW / dx GEMM runs alone) is the smallest."""
     monkeypatch.delenv("LSTM_BWD_CHUNKS", raising=False)
     assert lib.lstm_test_bwd_chunks(-1) == -1
     for T in list(range(0, 300)) + [1024, 4096]:
         n = lib.lstm_test_bwd_chunks(T)
-        assert n == (min(8, T // 16) if T >= 32 else 1), T
+        assert n == (min(6, T // 16) if T >= 32 else 1), T
         b = [lib.lstm_test_chunk_bound(T, n, c) for c in range(n + 1)]
         assert b[0] == 0 and b[-1] == T, (T, b)
         if T >= n:
