@@ -114,7 +114,11 @@ __device__ __forceinline__ bool wait_counter(const unsigned int *ctr, unsigned i
     if (ld_acquire_u32(ctr) >= target) return true;
     const uint64_t t0 = tc::globaltimer_ns();
     while (true) {
-        if (ld_acquire_u32(ctr) >= target) return true;
+        // 32 polls per look at the clock and the abort flag: reading
+        // %globaltimer on every poll made the step barrier's detection slower
+        // (the recurrences 1.8 % slower per step on the bench workload)
+        for (int k = 0; k < 32; ++k)
+            if (ld_acquire_u32(ctr) >= target) return true;
         if (*abort_flag) return false;
         if (tc::globaltimer_ns() - t0 > limit_ns) {
             atomicCAS(&ctrl->status, 0u, 5u);
