@@ -24,3 +24,16 @@ def test_config_line():
     assert abs(c["us_per_recurrent_step"]["fwd"] - 5.0) < 1e-9
     assert abs(c["us_per_recurrent_step"]["bwd"] - 6.0) < 1e-9
     assert "dW" not in c["phases_ms_per_step"]
+
+
+def test_split_by_size_balances_copy_streams():
+    """The end-to-end leg's copies go to two streams per direction, largest
+    first onto the lighter stream: every tensor once, loads within the largest
+    item of each other."""
+    items = [(134, "dx"), (67, "y"), (33, "dW"), (1, "hT"), (1, "cT"), (0.5, "db")]
+    lanes = bench.split_by_size(items, 2)
+    assert sorted(k for lane in lanes for k in lane) == sorted(k for _, k in items)
+    size = dict((k, v) for v, k in items)
+    loads = [sum(size[k] for k in lane) for lane in lanes]
+    assert abs(loads[0] - loads[1]) <= max(size.values())
+    assert bench.split_by_size([(5, "a")], 2) == [["a"]]  # an empty stream is dropped
