@@ -132,6 +132,8 @@ def load(path: str = LIB_PATH):
     lib.lstm_test_last_paths.restype = ip
     lib.lstm_test_last_stack_chunks.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.lstm_test_last_stack_chunks.restype = ip
+    lib.lstm_test_last_persist_split.argtypes = [ctypes.POINTER(ip), ctypes.POINTER(ip)]
+    lib.lstm_test_last_persist_split.restype = ip
     lib.lstm_test_bwd_chunks.argtypes = [ip]
     lib.lstm_test_bwd_chunks.restype = ip
     lib.lstm_test_chunk_bound.argtypes = [ip, ip, ip]
@@ -388,6 +390,14 @@ def test_last_stack_chunks():
     layer wavefronts (0: layer after layer; -1: no such call yet)."""
     f, b = ctypes.c_int(), ctypes.c_int()
     load().lstm_test_last_stack_chunks(ctypes.byref(f), ctypes.byref(b))
+    return f.value, b.value
+
+
+def test_last_persist_split():
+    """Test hook: (forward, backward) cluster size of the last persistent
+    CUDA-core recurrences (0: none yet)."""
+    f, b = ctypes.c_int(), ctypes.c_int()
+    load().lstm_test_last_persist_split(ctypes.byref(f), ctypes.byref(b))
     return f.value, b.value
 
 

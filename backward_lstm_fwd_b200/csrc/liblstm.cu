@@ -79,6 +79,9 @@ struct Phase {
 //   LSTM_BWD_STREAMS=1     that backward with one batch stream per group
 //   LSTM_BWD_CHUNKS=n      reverse-time chunks of the overlapped backward
 //   LSTM_PERSIST=0         no persistent CUDA-core recurrences (one launch per step)
+//   LSTM_PERSIST_KS=n      their K split over clusters of n CTAs only (1, 2, 4, 8)
+//   LSTM_STACK_WAVE=0      stacked layers one after another (no layer wavefront)
+//   LSTM_STACK_CHUNKS=n    chunks per layer of the layer wavefront
 //   LSTM_LAUNCH_NONCOOP=1  cluster launches without the cooperative attribute
 //                          (also taken when a profiler or sanitizer is attached:
 //                          NV_COMPUTE_PROFILER_PERFWORKS_DIR or
@@ -1312,40 +1315,127 @@ cudaError_t launch_persistent(Kern kern, const Prm &prm, int grid, size_t smem, 
     return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
-// Units per CTA of the persistent recurrences: every SM holds a slice (the
-// backward in quads of units, the grain of its epilogue), within the shared
-// memory budget and the kernels' per-thread item limit.  K is staged in
-// chunks of at most 16384 floats over all B rows, halved until they fit
-// beside the weights (fewer syncs than small chunks, and every thread has
-// several loads in flight), and each item's dot product is split over the
-// lanes the CTA would otherwise leave idle.
+// Whether `grid` CTAs of `kern` in clusters of KS (1: no clusters) can all be
+// resident at once with `smem` bytes of dynamic shared memory each.
+template <class Kern>
+bool pst_coresident(Kern kern, int KS, int grid, size_t smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (KS == 1) {
+        int per_sm = 0;
+        const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, pst::NTHR,
+                                                                      smem) == cudaSuccess &&
+                        per_sm * tcg::sm_count() >= grid;
+        cudaGetLastError();
+        return ok;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(pst::NTHR);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = KS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    const bool ok = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) == cudaSuccess &&
+                    nclusters * KS >= grid;
+    cudaGetLastError();
+    return ok;
+}
+
+// Work split of the persistent recurrences (pst::Split): for each cluster
+// size KS in 8, 4, 2, 1 the fewest units per CTA (quads in the backward, the
+// grain of its epilogue) that keep the grid within one CTA per SM, the
+// staging chunk (at most 16384 floats over all B rows, halved until the
+// shared memory fits) and the lanes per dot product (those the CTA would
+// otherwise leave idle); of the splits that fit and are co-resident, the one
+// with the lowest estimated step time in SM cycles: the K slice's operand
+// bytes at 16 B per cycle (an SM's share of L2 in the burst after a step
+// barrier), the exchange (≈ 1200 cycles plus its bytes at the same rate), the
+// contraction (≈ 42 cycles per float4 column step of a thread's items: two
+// warps per scheduler, ≈ 21 instructions each) and 300 cycles per extra chunk.
+// LSTM_PERSIST_KS=n keeps only cluster size n.
 struct PstPlan {
-    int UN = 0, P = 0, KC = 0, KSPLIT = 1;
+    pst::Split s = {};
+    int P = 0;
     size_t smem = 0;
 };
+int g_last_pst_ks[2] = {0, 0};  // cluster size of the last persistent fwd / bwd (test hook)
 
+template <class T>
 bool plan_persist(const lstm_dims *d, bool backward, PstPlan &Q) {
     if (env_is("LSTM_PERSIST", '0') || d->H < 1 || d->B < 1 || d->T < 1) return false;
-    const int nsm = tcg::sm_count();
+    const char *ov = getenv("LSTM_PERSIST_KS");
+    const int only = ov ? atoi(ov) : 0;
+    const int nsm = tcg::sm_count(), B = d->B, H = d->H;
     const int q = backward ? 4 : 1;
-    Q.UN = q * ((d->H + q * nsm - 1) / (q * nsm));
-    Q.P = (d->H + Q.UN - 1) / Q.UN;
-    const long long items = (long long)d->B * (backward ? Q.UN / 4 : Q.UN);
-    if (items > (long long)pst::MAXP * pst::NTHR || Q.P > nsm) return false;
-    const int K = backward ? 4 * d->H : d->H;
-    Q.KSPLIT = 1;
-    while (Q.KSPLIT < 32 && items * Q.KSPLIT * 2 <= pst::NTHR) Q.KSPLIT *= 2;
-    auto smem = [&](int kc) {
-        return backward ? pst::bwd_smem(d->B, d->H, Q.UN, kc) : pst::fwd_smem(d->B, d->H, Q.UN, kc);
-    };
-    Q.KC = std::min(std::max(32, 16384 / d->B / 32 * 32), (K + 31) / 32 * 32);
-    while (Q.KC > 32 && smem(Q.KC) > kMaxSmem) Q.KC = std::max(32, Q.KC / 2 / 32 * 32);
-    Q.smem = smem(Q.KC);
-    return Q.smem <= kMaxSmem;
+    const int K = backward ? 4 * H : H;
+    double best = 1e30;
+    for (int KS : {8, 4, 2, 1}) {
+        if (only && only != KS) continue;
+        pst::Split s = {};
+        s.KS = KS;
+        s.KSL = ((K + KS - 1) / KS + 7) / 8 * 8;
+        if (KS > 1 && (long long)s.KSL * (KS - 1) >= K) continue;  // a rank without columns
+        s.UN = q;
+        while ((long long)(H + KS * s.UN - 1) / (KS * s.UN) * KS > nsm) s.UN += q;
+        const int UC = KS * s.UN, P = (H + UC - 1) / UC * KS;
+        const long long items = (long long)B * (backward ? UC / 4 : UC);
+        if (items > (long long)pst::MAXP * pst::NTHR) continue;
+        s.KSPLIT = 1;
+        while (s.KSPLIT < 32 && items * s.KSPLIT * 2 <= pst::NTHR) s.KSPLIT *= 2;
+        const int pad = 4 * std::min(s.KSPLIT, 8);
+        s.KC = std::min(std::max(32, 16384 / B / 32 * 32), (s.KSL + 31) / 32 * 32);
+        s.KCP = s.KC + pad;
+        while (s.KC > 32 && pst::layout(backward, B, s).bytes > kMaxSmem) {
+            s.KC = std::max(32, s.KC / 2 / 32 * 32);
+            s.KCP = s.KC + pad;
+        }
+        const size_t smem = pst::layout(backward, B, s).bytes;
+        if (smem > kMaxSmem) continue;
+        const bool cores = backward ? pst_coresident(pst::bwd_kernel<T>, KS, P, smem)
+                                    : pst_coresident(pst::fwd_kernel<T>, KS, P, smem);
+        if (!cores) continue;
+        const int nslots = pst::NTHR / s.KSPLIT;
+        const double cost =
+            (double)B * s.KSL * sizeof(T) / 16.0 +
+            (KS > 1 ? 1200.0 + (KS - 1) * pst::part_floats(backward, B, s.UN) * 4 / 16.0 : 0.0) +
+            42.0 * (double)((items + nslots - 1) / nslots) *
+                (double)((s.KSL / 4 + s.KSPLIT - 1) / s.KSPLIT) +
+            300.0 * (double)((s.KSL + s.KC - 1) / s.KC - 1);
+        if (cost < best) {
+            best = cost;
+            Q.s = s;
+            Q.P = P;
+            Q.smem = smem;
+        }
+    }
+    return best < 1e30;
+}
+
+// One launch of a persistent recurrence: a cooperative cluster launch when the
+// split has KS > 1.  LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the
+// caller fall back.
+template <class Kern, class Prm>
+int launch_pst(Kern kern, const Prm &prm, const PstPlan &Q, cudaStream_t s) {
+    const cudaError_t e = Q.s.KS > 1
+                              ? launch_cluster(kern, prm, Q.P, Q.s.KS, Q.smem, s, pst::NTHR)
+                              : launch_persistent(kern, prm, Q.P, Q.smem, s);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+        cudaGetLastError();
+        return LSTM_ERR_NOT_CORESIDENT;
+    }
+    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
 }
 
 // a2 over all T steps in one launch; Gx holds the input projection.
-// LSTM_ERR_NOT_CORESIDENT (nothing launched) lets the caller fall back.
 template <class T>
 int persist_fwd(const lstm_dims *d, const PstPlan &Q, const T *W, const float *Gx,
                 const T *h0, const float *c0, const T *mask, bool reverse, bool ijfo, T *y,
@@ -1354,17 +1444,13 @@ int persist_fwd(const lstm_dims *d, const PstPlan &Q, const T *W, const float *G
     memset(&prm, 0, sizeof(prm));
     prm.W = W; prm.Gx = Gx; prm.h0 = h0; prm.c0 = c0; prm.mask = mask;
     prm.y = y; prm.gates = gates; prm.cells = cells; prm.ctrl = ctrl;
-    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = Q.UN; prm.KC = Q.KC;
-    prm.KSPLIT = Q.KSPLIT;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I;
     prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
+    prm.s = Q.s;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
-    const cudaError_t e = launch_persistent(pst::fwd_kernel<T>, prm, Q.P, Q.smem, s);
-    if (e == cudaErrorCooperativeLaunchTooLarge) {
-        cudaGetLastError();
-        return LSTM_ERR_NOT_CORESIDENT;
-    }
-    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+    g_last_pst_ks[0] = Q.s.KS;
+    return launch_pst(pst::fwd_kernel<T>, prm, Q, s);
 }
 
 // a3 over all T steps in one launch (dinitH follows as one more product).
@@ -1381,17 +1467,13 @@ int persist_bwd(const lstm_dims *d, const PstPlan &Q, const T *W, const T *dy,
     prm.dcbuf[0] = dcbuf[0]; prm.dcbuf[1] = dcbuf[1];
     prm.dhpbuf[0] = dhpbuf[0]; prm.dhpbuf[1] = dhpbuf[1];
     prm.dc0 = dc0; prm.ctrl = ctrl;
-    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I; prm.UN = Q.UN; prm.KC = Q.KC;
-    prm.KSPLIT = Q.KSPLIT;
+    prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I;
     prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
+    prm.s = Q.s;
     prm.fault_skip_cta = g_fault_skip_cta;
     prm.wait_ns = g_wait_ns;
-    const cudaError_t e = launch_persistent(pst::bwd_kernel<T>, prm, Q.P, Q.smem, s);
-    if (e == cudaErrorCooperativeLaunchTooLarge) {
-        cudaGetLastError();
-        return LSTM_ERR_NOT_CORESIDENT;
-    }
-    return e == cudaSuccess ? LSTM_OK : LSTM_ERR_CUDA;
+    g_last_pst_ks[1] = Q.s.KS;
+    return launch_pst(pst::bwd_kernel<T>, prm, Q, s);
 }
 
 // ------------------------------------------------------------ forward pass
@@ -1459,7 +1541,7 @@ int fwd_simt(const lstm_dims *d, const T *x, const T *W, const T *b, const T *h0
         bool persisted = false;
         {
             PstPlan Q;
-            if (plan_persist(d, false, Q)) {
+            if (plan_persist<T>(d, false, Q)) {
                 const int rc = persist_fwd<T>(d, Q, W, Gx, h0, c0, mask, reverse, ijfo,
                                               y, gates, cells, (Ctrl *)ws, s);
                 if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
@@ -1605,7 +1687,7 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
     bool persisted = false;
     {
         PstPlan Q;
-        if (plan_persist(d, true, Q)) {
+        if (plan_persist<T>(d, true, Q)) {
             const int rc = persist_bwd<T>(d, Q, W, dy, dhT, dcT, gates, cells, c0, mask,
                                           reverse, ijfo, dG, dcbuf, dhpbuf, dc0, (Ctrl *)ws, s);
             if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
@@ -2445,6 +2527,12 @@ int lstm_test_chunk_bound(int T, int nch, int c) {
 int lstm_test_last_stack_chunks(int *fwd_chunks, int *bwd_chunks) {
     if (fwd_chunks) *fwd_chunks = g_last_stack_chunks;
     if (bwd_chunks) *bwd_chunks = g_last_stack_bwd_chunks;
+    return LSTM_OK;
+}
+
+int lstm_test_last_persist_split(int *fwd_ks, int *bwd_ks) {
+    if (fwd_ks) *fwd_ks = g_last_pst_ks[0];
+    if (bwd_ks) *bwd_ks = g_last_pst_ks[1];
     return LSTM_OK;
 }
 

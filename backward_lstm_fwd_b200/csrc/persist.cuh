@@ -7,14 +7,18 @@
 // per-step kernel's work -- the contraction with W_h and the fused epilogue of
 // simt.cuh (EpFwdStep: the forward-formula table; EpBwdStep: backward steps 1,
 // 2, 3 and 5) -- so the epilogue arithmetic is shared, element for element.
-// What differs is the schedule: the CTA that owns a slice of hidden units
-// keeps that slice of W_h in shared memory (converted to fp32 once) for the
-// whole call, every step streams the step's operand (h_{t-1} or dG_{t+1}, all
-// batch rows, K in chunks) from L2, and the CTAs meet at a grid-wide
-// step counter instead of a kernel boundary.  The per-step kernels put a
-// B x 4H (or B x H) output on a few 64 x 64 tiles -- 4 CTAs for the backward
-// step at B = 32, H = 256 -- and pay a launch per step; here every SM holds a
-// slice of the units.
+// What differs is the schedule.  A cluster of KS CTAs owns UC = KS * UN hidden
+// units and splits the contraction's K axis (H for h_{t-1} W_h^T, 4H for
+// dG_{t+1} W_h) into KS slices: CTA r keeps slice r of the cluster's weights
+// in shared memory (converted to fp32 once) for the whole call, and every step
+// streams only slice r of the step's operand (all batch rows) from L2.  Its
+// partial sums for the units CTA o finishes go to o by one bulk DSMEM copy
+// (slot r of o's receive block, one mbarrier with expected bytes), each CTA
+// adds the KS slots of its own UN units in rank order and runs the epilogue,
+// and all CTAs meet at a grid-wide step counter.  With KS = 1 there is no
+// exchange: the CTA streams the whole operand.  The per-step kernels instead
+// put a B x 4H (or B x H) output on a few 64 x 64 tiles and pay a launch per
+// step.
 #pragma once
 
 #include <type_traits>
@@ -26,26 +30,52 @@ namespace lstm {
 namespace pst {
 
 constexpr int NTHR = 256;
-constexpr int MAXP = 4;         // (row, unit) pairs / (row, unit quad) items per thread
+constexpr int MAXP = 8;         // contraction items per thread
 constexpr int STAGE_UNR = 8;    // operand loads in flight per thread while staging
 
-// The step's operand is staged in K chunks of KC (a multiple of 32 the host
-// picks so that a chunk of all B rows holds at most 16384 floats, within the
-// shared memory left beside the weights), rows padded to KC + 1 floats so that
-// rows m, m+1, ... start in different banks.  Each
-// output item's dot product is split over KSPLIT lanes of one warp (a power of
-// two <= 32 the host picks so that items x KSPLIT fill the CTA): lane `ks`
-// of the group takes k = ks, ks + KSPLIT, ... of every chunk and the group's
-// partial sums meet in a butterfly of shuffles.
-// Forward: CTA c owns hidden units [c*UN, c*UN + UN) (all four gates).
-// Shared memory: Ws [4][UN][H] fp32 (W_h rows g*H + j), hs [B][KC + 1] fp32.
-__host__ __device__ inline size_t fwd_smem(int B, int H, int UN, int KC) {
-    return (size_t)4 * UN * H * 4 + (size_t)B * (KC + 1) * 4;
+// Work split of one launch (host and device).
+//   KS      CTAs per cluster, each taking one K slice (1: no split)
+//   UN      units whose epilogue a CTA runs (a multiple of 4 in the backward,
+//           whose epilogue works on quads of units)
+//   KSL     K-slice length, a multiple of 8 (the last slice may hold fewer
+//           real columns; weights past K are zero)
+//   KC      staging chunk: columns of the slice staged at once for all B rows,
+//           a multiple of 32
+//   KCP     row pitch of the staged chunk in floats: KC + 4 * min(KSPLIT, 8),
+//           so that the rows a quarter warp reads start in different banks
+//   KSPLIT  lanes of a warp that share one item's dot product (a power of two;
+//           lane ks takes float4 columns ks, ks + KSPLIT, ...), their partial
+//           sums meeting in a butterfly of shuffles
+// Contraction items: forward (row m, unit u of the cluster) with the four gate
+// rows of u; backward (row m, quad of units) with one dot product per unit.
+struct Split {
+    int KS, UN, KSL, KC, KCP, KSPLIT;
+};
+
+// Floats of one CTA's partial block for one owner: forward B x UN x 4 gates,
+// backward B x UN units.
+__host__ __device__ inline int part_floats(bool bwd, int B, int UN) {
+    return bwd ? B * UN : 4 * B * UN;
 }
-// Backward: CTA c owns units [c*UN, c*UN + UN), UN a multiple of 4.
-// Shared memory: Wt [UN][4H] fp32 (column j of W_h, all 4H rows), gs [B][KC + 1].
-__host__ __device__ inline size_t bwd_smem(int B, int H, int UN, int KC) {
-    return (size_t)UN * 4 * H * 4 + (size_t)B * (KC + 1) * 4;
+
+// Shared-memory plan in floats from the (16-byte aligned) dynamic base:
+// weights, staged operand chunk, KS - 1 send blocks, KS receive slots, the
+// receive mbarrier.  Every region starts on a 16-byte boundary.
+struct Layout {
+    int w, opnd, stage, recv, bar;
+    size_t bytes;
+};
+__host__ __device__ inline Layout layout(bool bwd, int B, const Split &s) {
+    const int UC = s.KS * s.UN;
+    const int part = part_floats(bwd, B, s.UN);
+    Layout L;
+    L.w = 0;
+    L.opnd = (bwd ? 1 : 4) * UC * s.KSL;
+    L.stage = L.opnd + B * s.KCP;
+    L.recv = L.stage + (s.KS - 1) * part;
+    L.bar = L.recv + s.KS * part;
+    L.bytes = (size_t)(L.bar + 4) * 4;
+    return L;
 }
 
 template <class E>
@@ -58,7 +88,8 @@ struct FwdParams {
     E *y, *gates;
     float *cells;
     Ctrl *ctrl;
-    int T, B, H, I, UN, KC, KSPLIT, reverse, fb;
+    int T, B, H, I, reverse, fb;
+    Split s;
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -73,7 +104,8 @@ struct BwdParams {
     float *dc0;            // [B][H]: delta c after the first step (dinitC)
     float *dhpbuf[2];      // delta h passed on by padding, ping-pong [B][H]
     Ctrl *ctrl;
-    int T, B, H, I, UN, KC, KSPLIT, reverse, fb;
+    int T, B, H, I, reverse, fb;
+    Split s;
     int fault_skip_cta;
     unsigned long long wait_ns;
 };
@@ -94,6 +126,40 @@ __device__ __forceinline__ bool grid_step(unsigned int *ctr, unsigned int target
     return ok_s != 0;
 }
 
+// Partial sums to their owners: every thread calls this after the writers
+// have put this CTA's partials for itself in receive slot r and those for the
+// other CTAs in the send blocks (send block sp goes to rank r + 1 + sp, so
+// that each CTA receives from one sender at a time).  Thread 0 posts the
+// expected bytes and issues the copies; every thread waits (bounded) for the
+// other ranks' copies into this CTA, and thread 0 for its own copies to have
+// read their sources, so the send blocks may be refilled afterwards.
+__device__ __forceinline__ bool exchange(float *stage, float *recv, uint64_t *bar, uint32_t &rph,
+                                         int KS, int r, int part_bytes, Ctrl *ctrl,
+                                         volatile int *abort_flag, uint32_t site,
+                                         unsigned long long wait_ns) {
+    if (KS == 1) {
+        __syncthreads();
+        return true;
+    }
+    tc::fence_proxy_async_smem();  // these generic stores, then the copies' async reads
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)((KS - 1) * part_bytes));
+        const uint32_t recv_lo = tc::smem_u32(recv), bar_lo = tc::smem_u32(bar);
+        for (int sp = 0; sp < KS - 1; ++sp) {
+            const uint32_t d = (uint32_t)((r + 1 + sp) % KS);
+            tc::bulk_copy_to_peer(tc::map_rank(recv_lo + (uint32_t)(r * part_bytes), d),
+                                  stage + sp * (part_bytes / 4), (uint32_t)part_bytes,
+                                  tc::map_rank(bar_lo, d));
+        }
+        tc::bulk_commit();
+    }
+    const bool ok = tc::mbar_wait_cluster(bar, rph, ctrl, abort_flag, site, wait_ns);
+    rph ^= 1;
+    if (threadIdx.x == 0) tc::bulk_wait_read_all();
+    return __syncthreads_and(ok) != 0;
+}
+
 // 16 bytes of T as floats: the element type of one vector load
 __device__ __forceinline__ void to_f4(const float4 &v, float *o) {
     o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
@@ -106,14 +172,13 @@ __device__ __forceinline__ void to_f8(const uint4 &v, float *o) {
 }
 
 // Rows [0, B) x columns [k0, k0 + kn) of a row-major operand with row pitch
-// `ld` into dst[B][KC + 1] as fp32 (zeros past kn), by all threads, with
-// STAGE_UNR independent loads in flight per thread: 16-byte loads when every
-// row's slice starts on a 16-byte boundary and holds whole vectors, else
-// element loads.
+// `ld` into dst[B][KCP] as fp32 (zeros in columns kn .. KC - 1), by all
+// threads, with STAGE_UNR independent loads in flight per thread: 16-byte
+// loads when every row's slice starts on a 16-byte boundary and holds whole
+// vectors, else element loads.
 template <class T>
 __device__ __forceinline__ void stage_chunk(float *dst, const T *src, long long ld, int B, int k0,
-                                            int kn, int KC) {
-    const int KCP = KC + 1;
+                                            int kn, int KC, int KCP) {
     constexpr int V = 16 / (int)sizeof(T);  // elements per 16-byte load
     if (KC % V == 0 && kn % V == 0 && k0 % V == 0 && ld % V == 0 &&
         ((uintptr_t)src & 15u) == 0) {
@@ -139,7 +204,9 @@ __device__ __forceinline__ void stage_chunk(float *dst, const T *src, long long 
                     if constexpr (sizeof(T) == 4) to_f4(v[u], f);
                     else to_f8<T>(v[u], f);
 #pragma unroll
-                    for (int i = 0; i < V; ++i) dst[m * KCP + kk + i] = f[i];
+                    for (int i = 0; i < V; i += 4)
+                        *reinterpret_cast<float4 *>(dst + m * KCP + kk + i) =
+                            make_float4(f[i], f[i + 1], f[i + 2], f[i + 3]);
                 }
             }
         }
@@ -176,62 +243,126 @@ __device__ __forceinline__ void group_sum(float (&acc)[MAXP][4], int ksplit) {
                 acc[i][g] += __shfl_xor_sync(0xffffffffu, acc[i][g], off);
 }
 
+__device__ __forceinline__ float dot4(const float4 &a, const float4 &b, float acc) {
+    acc = fmaf(a.x, b.x, acc);
+    acc = fmaf(a.y, b.y, acc);
+    acc = fmaf(a.z, b.z, acc);
+    return fmaf(a.w, b.w, acc);
+}
+
+// acc[i][c] += sum over the chunk of opnd row m(i) times weight row wrow(i, c):
+// items q = slot + i * nslots < nitems; lane ks of the item's group takes the
+// float4 columns ks, ks + KSPLIT, ... < nv (columns past the chunk are zero in
+// both operands).
+template <class RowFn>
+__device__ __forceinline__ void contract(float (&acc)[MAXP][4], const float *opnd, int KCP,
+                                         int nitems, int B, int slot, int nslots, int ks,
+                                         int KSPLIT, int nv, RowFn wrow) {
+#pragma unroll
+    for (int i = 0; i < MAXP; ++i) {
+        const int q = slot + i * nslots;
+        if (q >= nitems) break;
+        const int m = q % B, it = q / B;
+        const float4 *o4 = reinterpret_cast<const float4 *>(opnd + m * KCP);
+        const float4 *w0 = reinterpret_cast<const float4 *>(wrow(it, 0));
+        const float4 *w1 = reinterpret_cast<const float4 *>(wrow(it, 1));
+        const float4 *w2 = reinterpret_cast<const float4 *>(wrow(it, 2));
+        const float4 *w3 = reinterpret_cast<const float4 *>(wrow(it, 3));
+        for (int v = ks; v < nv; v += KSPLIT) {
+            const float4 h = o4[v];
+            acc[i][0] = dot4(h, w0[v], acc[i][0]);
+            acc[i][1] = dot4(h, w1[v], acc[i][1]);
+            acc[i][2] = dot4(h, w2[v], acc[i][2]);
+            acc[i][3] = dot4(h, w3[v], acc[i][3]);
+        }
+    }
+}
+
+// Shared prologue of both kernels: the CTA's abort flag and, with KS > 1, the
+// receive mbarrier, initialised before any peer may complete bytes on it.
+__device__ __forceinline__ void init_exchange(uint64_t *rbar, int KS, volatile int *abort_s) {
+    if (threadIdx.x == 0) {
+        *abort_s = 0;
+        if (KS > 1) {
+            tc::mbar_init(rbar, 1);
+            tc::fence_mbar_init();
+        }
+    }
+}
+
+// Last act of both kernels, on every path: no copy of this CTA in flight, and
+// with KS > 1 no CTA of the cluster leaves while a peer may still copy into it.
+__device__ __forceinline__ void finish_exchange(int KS) {
+    if (KS > 1 && threadIdx.x == 0) tc::bulk_wait_all();
+    __syncthreads();
+    if (KS > 1) tc::cluster_sync_all();
+}
+
 template <class T>
 __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
     extern __shared__ float4 smem_f4[];
-    float *Ws = reinterpret_cast<float *>(smem_f4);
-    const int H = p.H, B = p.B, T_ = p.T, UN = p.UN, KC = p.KC, KCP = KC + 1;
-    const int KSPLIT = p.KSPLIT, slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT;
-    const int nslots = NTHR / KSPLIT;
-    float *hs = Ws + (size_t)4 * UN * H;
+    float *sm = reinterpret_cast<float *>(smem_f4);
+    const Split &sp = p.s;
+    const int H = p.H, B = p.B, T_ = p.T, KS = sp.KS, UN = sp.UN, UC = KS * UN;
+    const int KSL = sp.KSL, KC = sp.KC, KCP = sp.KCP, KSPLIT = sp.KSPLIT;
+    const int slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT, nslots = NTHR / KSPLIT;
+    const Layout L = layout(false, B, sp);
+    float *Ws = sm + L.w, *hs = sm + L.opnd, *stage = sm + L.stage, *recv = sm + L.recv;
+    uint64_t *rbar = reinterpret_cast<uint64_t *>(sm + L.bar);
     __shared__ int abort_s;
-    if (threadIdx.x == 0) abort_s = 0;
-    const int j0 = blockIdx.x * UN;
-    const int un = min(UN, H - j0);  // units this CTA owns (the last CTA may own fewer)
+    const int r = KS > 1 ? (int)tc::cluster_rank() : 0;
+    const int u0 = (int)(blockIdx.x / KS) * UC;    // first unit of the cluster
+    const int k_lo = r * KSL, kl = min(KSL, H - k_lo);  // this CTA's columns of h (<= 0: none)
     const long long K = (long long)H + p.I;
-    // W_h rows g*H + j0 + jj, all H columns, converted to fp32
-    for (int e = threadIdx.x; e < 4 * UN * H; e += NTHR) {
-        const int k = e % H, r = e / H, jj = r % UN, g = r / UN;
-        Ws[e] = jj < un ? to_f(p.W[((long long)g * H + j0 + jj) * K + k]) : 0.f;
+    init_exchange(rbar, KS, &abort_s);
+    // Ws[g][u][kk] = W_h[g*H + u0 + u][k_lo + kk] in fp32, zero past H
+    for (int e = threadIdx.x; e < 4 * UC * KSL; e += NTHR) {
+        const int kk = e % KSL, row = e / KSL, u = row % UC, g = row / UC;
+        Ws[e] = (u0 + u < H && kk < kl)
+                    ? to_f(p.W[((long long)g * H + u0 + u) * K + k_lo + kk]) : 0.f;
     }
+    if (KS > 1) tc::cluster_sync_all();
+    else __syncthreads();
     unsigned int *ctr = &p.ctrl->bar[0];
     const unsigned int P = gridDim.x;
-    const int npairs = B * un;  // pair q -> row m = q % B, unit jj = q / B
+    const int nitems = B * UC, part = part_floats(false, B, UN);
     auto tau = [&](int st) { return p.reverse ? T_ - 1 - st : st; };
+    auto wrow = [&](int u, int g) { return Ws + (size_t)(g * UC + u) * KSL; };
     const long long BH = (long long)B * H;
+    uint32_t rph = 0;
     for (int st = 0; st < T_; ++st) {
         const int t = tau(st), tp = p.reverse ? t + 1 : t - 1;
         const T *hp = st > 0 ? p.y + (long long)tp * BH : p.h0;
-        float acc[MAXP][4];
+        const bool contracted = hp != nullptr;  // h_{-1} = 0 otherwise: no product
+        if (contracted) {
+            float acc[MAXP][4];
 #pragma unroll
-        for (int i = 0; i < MAXP; ++i)
+            for (int i = 0; i < MAXP; ++i)
 #pragma unroll
-            for (int g = 0; g < 4; ++g) acc[i][g] = 0.f;
-        if (hp) {
-            for (int k0 = 0; k0 < H; k0 += KC) {
-                const int kn = min(KC, H - k0);
+                for (int g = 0; g < 4; ++g) acc[i][g] = 0.f;
+            for (int c0 = 0; c0 < kl; c0 += KC) {
+                const int kn = min(KC, kl - c0);
                 __syncthreads();  // the previous chunk has been read
-                stage_chunk(hs, hp, H, B, k0, kn, KC);
+                stage_chunk(hs, hp, H, B, k_lo + c0, kn, KC, KCP);
                 __syncthreads();
+                contract(acc, hs, KCP, nitems, B, slot, nslots, ks, KSPLIT, (kn + 3) >> 2,
+                         [&](int u, int g) { return wrow(u, g) + c0; });
+            }
+            group_sum(acc, KSPLIT);
+            if (ks == 0) {
 #pragma unroll
                 for (int i = 0; i < MAXP; ++i) {
                     const int q = slot + i * nslots;
-                    if (q >= npairs) break;
-                    const int m = q % B, jj = q / B;
-                    const float *hrow = hs + m * KCP;
-                    const float *w0 = Ws + ((size_t)0 * UN + jj) * H + k0;
-                    const float *w1 = Ws + ((size_t)1 * UN + jj) * H + k0;
-                    const float *w2 = Ws + ((size_t)2 * UN + jj) * H + k0;
-                    const float *w3 = Ws + ((size_t)3 * UN + jj) * H + k0;
-                    for (int kk = ks; kk < kn; kk += KSPLIT) {
-                        const float h = hrow[kk];
-                        acc[i][0] = fmaf(h, w0[kk], acc[i][0]);
-                        acc[i][1] = fmaf(h, w1[kk], acc[i][1]);
-                        acc[i][2] = fmaf(h, w2[kk], acc[i][2]);
-                        acc[i][3] = fmaf(h, w3[kk], acc[i][3]);
-                    }
+                    if (q >= nitems) break;
+                    const int m = q % B, u = q / B, o = u / UN, ul = u - o * UN;
+                    float *dst = o == r ? recv + r * part : stage + ((o - r - 1 + KS) % KS) * part;
+                    *reinterpret_cast<float4 *>(dst + (m * UN + ul) * 4) =
+                        make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
                 }
             }
+            if (!exchange(stage, recv, rbar, rph, KS, r, part * 4, p.ctrl, &abort_s, 0xA03,
+                          p.wait_ns))
+                break;
         }
         simt::EpFwdStep<T> ep{p.Gx + (long long)t * B * 4 * H,
                               st > 0 ? p.cells + (long long)tp * BH : p.c0,
@@ -242,82 +373,93 @@ __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
             ep.hprev = hp;
         }
         ep.fb = p.fb;
-        group_sum(acc, KSPLIT);
-#pragma unroll
-        for (int i = 0; i < MAXP; ++i) {
-            const int q = slot + i * nslots;
-            if (q >= npairs) break;
-            const int m = q % B, jj = q / B;
-            if (ks == 0) ep(m, 4 * (j0 + jj), acc[i]);
+        // the epilogue of this CTA's own units: the KS slots summed in rank order
+        for (int e = threadIdx.x; e < B * UN; e += NTHR) {
+            const int m = e % B, ul = e / B;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            if (contracted)
+                for (int sl = 0; sl < KS; ++sl) {
+                    const float4 v = *reinterpret_cast<const float4 *>(recv + sl * part +
+                                                                       (m * UN + ul) * 4);
+                    a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+                }
+            ep(m, 4 * (u0 + r * UN + ul), a);
         }
         // h_t of every unit is the next step's operand: grid barrier
         if (st + 1 < T_) {
             const bool arrive = (int)blockIdx.x != p.fault_skip_cta;
             if (!grid_step(ctr, P * (unsigned)(st + 1), arrive, p.ctrl, &abort_s, 0xA01, p.wait_ns))
-                return;
+                break;
         }
     }
+    finish_exchange(KS);
 }
 
 template <class T>
 __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
     extern __shared__ float4 smem_f4[];
-    float *Wt = reinterpret_cast<float *>(smem_f4);
-    const int H = p.H, B = p.B, T_ = p.T, UN = p.UN, KC = p.KC, KCP = KC + 1;
-    const int KSPLIT = p.KSPLIT, slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT;
-    const int nslots = NTHR / KSPLIT;
-    const int G4 = 4 * H;
-    float *gs = Wt + (size_t)UN * G4;
+    float *sm = reinterpret_cast<float *>(smem_f4);
+    const Split &sp = p.s;
+    const int H = p.H, B = p.B, T_ = p.T, KS = sp.KS, UN = sp.UN, UC = KS * UN;
+    const int KSL = sp.KSL, KC = sp.KC, KCP = sp.KCP, KSPLIT = sp.KSPLIT;
+    const int slot = threadIdx.x / KSPLIT, ks = threadIdx.x % KSPLIT, nslots = NTHR / KSPLIT;
+    const int G4 = 4 * H, QN = UN / 4;  // quads of units a CTA finishes
+    const Layout L = layout(true, B, sp);
+    float *Wt = sm + L.w, *gs = sm + L.opnd, *stage = sm + L.stage, *recv = sm + L.recv;
+    uint64_t *rbar = reinterpret_cast<uint64_t *>(sm + L.bar);
     __shared__ int abort_s;
-    if (threadIdx.x == 0) abort_s = 0;
-    const int j0 = blockIdx.x * UN;
+    const int r = KS > 1 ? (int)tc::cluster_rank() : 0;
+    const int u0 = (int)(blockIdx.x / KS) * UC;     // first unit of the cluster
+    const int k_lo = r * KSL, kl = min(KSL, G4 - k_lo);  // this CTA's columns of dG
     const long long K = (long long)H + p.I;
-    // column j0 + jj of W_h, all 4H rows, converted to fp32 (zero past H)
-    for (int e = threadIdx.x; e < UN * G4; e += NTHR) {
-        const int k = e % G4, jj = e / G4;
-        Wt[e] = j0 + jj < H ? to_f(p.W[(long long)k * K + j0 + jj]) : 0.f;
+    init_exchange(rbar, KS, &abort_s);
+    // Wt[u][kk] = W_h[k_lo + kk][u0 + u] (column u0 + u of W_h) in fp32, zero past 4H / H
+    for (int e = threadIdx.x; e < UC * KSL; e += NTHR) {
+        const int kk = e % KSL, u = e / KSL;
+        Wt[e] = (u0 + u < H && kk < kl) ? to_f(p.W[(long long)(k_lo + kk) * K + u0 + u]) : 0.f;
     }
+    if (KS > 1) tc::cluster_sync_all();
+    else __syncthreads();
     unsigned int *ctr = &p.ctrl->bar[0];
     const unsigned int P = gridDim.x;
-    const int nq = UN / 4;          // unit quads of this CTA
-    const int nitems = B * nq;      // item q -> row m = q % B, quad jq = q / B
+    const int nitems = B * (UC / 4), part = part_floats(true, B, UN);
     auto tau = [&](int st) { return p.reverse ? T_ - 1 - (long long)st : (long long)st; };
     const long long BH = (long long)B * H;
+    uint32_t rph = 0;
     for (int st = T_ - 1; st >= 0; --st) {
-        const bool last = st == T_ - 1;
+        const bool last = st == T_ - 1;  // no dG_{t+1}: delta h comes from dhT
         const long long t = tau(st);
-        float acc[MAXP][4];
-#pragma unroll
-        for (int i = 0; i < MAXP; ++i)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
         if (!last) {
-            // delta h = dG_{t_next} W_h for this CTA's units
+            // delta h = dG_{t_next} W_h, this CTA's K slice, for the cluster's units
+            float acc[MAXP][4];
+#pragma unroll
+            for (int i = 0; i < MAXP; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
             const T *dGn = p.dG + tau(st + 1) * B * G4;
-            for (int k0 = 0; k0 < G4; k0 += KC) {
-                const int kn = min(KC, G4 - k0);
+            for (int c0 = 0; c0 < kl; c0 += KC) {
+                const int kn = min(KC, kl - c0);
                 __syncthreads();
-                stage_chunk(gs, dGn, G4, B, k0, kn, KC);
+                stage_chunk(gs, dGn, G4, B, k_lo + c0, kn, KC, KCP);
                 __syncthreads();
+                contract(acc, gs, KCP, nitems, B, slot, nslots, ks, KSPLIT, (kn + 3) >> 2,
+                         [&](int jq, int c) { return Wt + (size_t)(4 * jq + c) * KSL + c0; });
+            }
+            group_sum(acc, KSPLIT);
+            if (ks == 0) {
 #pragma unroll
                 for (int i = 0; i < MAXP; ++i) {
                     const int q = slot + i * nslots;
                     if (q >= nitems) break;
-                    const int m = q % B, jq = q / B;
-                    const float *grow = gs + m * KCP;
-                    const float *w0 = Wt + (size_t)(4 * jq + 0) * G4 + k0;
-                    const float *w1 = Wt + (size_t)(4 * jq + 1) * G4 + k0;
-                    const float *w2 = Wt + (size_t)(4 * jq + 2) * G4 + k0;
-                    const float *w3 = Wt + (size_t)(4 * jq + 3) * G4 + k0;
-                    for (int kk = ks; kk < kn; kk += KSPLIT) {
-                        const float g = grow[kk];
-                        acc[i][0] = fmaf(g, w0[kk], acc[i][0]);
-                        acc[i][1] = fmaf(g, w1[kk], acc[i][1]);
-                        acc[i][2] = fmaf(g, w2[kk], acc[i][2]);
-                        acc[i][3] = fmaf(g, w3[kk], acc[i][3]);
-                    }
+                    const int m = q % B, jq = q / B, o = jq / QN, lq = jq - o * QN;
+                    float *dst = o == r ? recv + r * part : stage + ((o - r - 1 + KS) % KS) * part;
+                    *reinterpret_cast<float4 *>(dst + (m * QN + lq) * 4) =
+                        make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
                 }
             }
+            if (!exchange(stage, recv, rbar, rph, KS, r, part * 4, p.ctrl, &abort_s, 0xA04,
+                          p.wait_ns))
+                break;
         }
         simt::EpBwdStep<T> ep;
         ep.dy = p.dy ? p.dy + t * BH : nullptr;
@@ -336,22 +478,27 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
             ep.dhp_in = last ? nullptr : p.dhpbuf[(st + 1) & 1];
             ep.dhp_out = p.dhpbuf[st & 1];
         }
-        group_sum(acc, KSPLIT);
-#pragma unroll
-        for (int i = 0; i < MAXP; ++i) {
-            const int q = slot + i * nslots;
-            if (q >= nitems) break;
-            const int m = q % B, jq = q / B;
-            if (ks == 0) ep(m, j0 + 4 * jq, acc[i]);
+        // the epilogue of this CTA's own quads: the KS slots summed in rank order
+        for (int e = threadIdx.x; e < B * QN; e += NTHR) {
+            const int m = e % B, lq = e / B;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+            if (!last)
+                for (int sl = 0; sl < KS; ++sl) {
+                    const float4 v = *reinterpret_cast<const float4 *>(recv + sl * part +
+                                                                       (m * QN + lq) * 4);
+                    a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+                }
+            ep(m, u0 + r * UN + 4 * lq, a);
         }
         // dG_t of every unit is the next step's operand: grid barrier
         if (st > 0) {
             const bool arrive = (int)blockIdx.x != p.fault_skip_cta;
             if (!grid_step(ctr, P * (unsigned)(T_ - st), arrive, p.ctrl, &abort_s, 0xA02,
                            p.wait_ns))
-                return;
+                break;
         }
     }
+    finish_exchange(KS);
 }
 
 }  // namespace pst

@@ -28,6 +28,11 @@
  *   LSTM_PERSIST=0         run the CUDA-core recurrences (fp32, and 16-bit
  *                          shapes off the tensor-core grids) as one launch
  *                          per step instead of one persistent launch.
+ *   LSTM_PERSIST_KS=n      split those persistent recurrences' K axis over
+ *                          clusters of n CTAs only (1, 2, 4 or 8; 1 = no
+ *                          split).  Default: the split with the lowest
+ *                          estimated step time that fits and is co-resident;
+ *                          when n does not fit, the per-step kernels run.
  *   LSTM_STACK_WAVE=0      run the layers of lstm_stack_fwd / lstm_stack_bwd
  *                          one after another instead of as a layer wavefront
  *                          (two layers' time chunks side by side on half the
@@ -96,6 +101,13 @@ int lstm_test_last_paths(int *fwd_path, int *bwd_path);
  * one after another; -1: none yet).
  */
 int lstm_test_last_stack_chunks(int *fwd_chunks, int *bwd_chunks);
+
+/*
+ * Cluster size (the number of CTAs that split the contraction's K axis) of
+ * the persistent CUDA-core forward and backward recurrences that this process
+ * launched last (0: none yet).
+ */
+int lstm_test_last_persist_split(int *fwd_ks, int *bwd_ks);
 
 /*
  * Reverse-time chunking of the tensor-core backward: the number of chunk

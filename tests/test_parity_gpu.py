@@ -187,6 +187,36 @@ def test_two_stream_backward_equals_one_stream(shape, cuda_device, monkeypatch):
 
 
 
+@pytest.mark.parametrize("ks", [1, 2, 4, 8])
+@pytest.mark.parametrize("shape", [(12, 32, 256, 256, "fp32"), (6, 130, 64, 128, "fp32"),
+                                   (7, 5, 37, 45, "bf16"), (5, 17, 40, 100, "fp16")])
+def test_persistent_k_split_cluster_sizes(shape, ks, cuda_device, monkeypatch):
+    """Each cluster size of the persistent CUDA-core recurrences' K split (KS
+    CTAs per cluster, each contracting one K slice, the partial sums sent to
+    the CTA that finishes their units by DSMEM copies) against the oracle,
+    forward and backward; a size that does not fit the shape leaves the
+    per-step kernels to run."""
+    T, B, I, H, dt = shape
+    w = synth.custom(T, B, I, H, dt, seed=T * 11 + ks)
+    inp = synth.make_inputs(w)
+    monkeypatch.setenv("LSTM_PERSIST_KS", str(ks))
+    out = run_gpu(inp, cuda_device, reverse=ks == 4)
+    fp, bp = L.test_last_paths()
+    fk, bk = L.test_last_persist_split()
+    assert fp in (0, 5) and bp in (0, 5)
+    if fp == 5:
+        assert fk == ks
+    if bp == 5:
+        assert bk == ks
+    if ks == 1:
+        assert (fp, bp) == (5, 5)
+    if ks == 8 and H == 256:
+        assert bp == 5  # 8 clusters of 8 (the forward's 16 need not be co-resident)
+    ref = run_oracle(inp, reverse=ks == 4)
+    assert_within(compare(out, ref, dt, OUTS + ("gates", "cells")), dt,
+                  f"{w.name} persistent KS={ks}")
+
+
 @pytest.mark.parametrize("shape", [(64, 32, 256, 256, "fp32"), (9, 6, 24, 40, "fp32"),
                                    (7, 5, 37, 45, "bf16"), (5, 130, 96, 1024, "fp32")])
 @pytest.mark.parametrize("opts", [{}, {"reverse": True, "ijfo": True}, {"mask": True}])
