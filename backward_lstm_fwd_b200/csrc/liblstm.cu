@@ -141,8 +141,9 @@ FwdLayout fwd_layout(const lstm_dims *d) {
     return L;
 }
 
-// db partial sums: at most kDbMaxChunks row chunks of >= 256 rows each.
-constexpr long long kDbMaxChunks = 2048;
+// db partial sums: at most kDbMaxChunks row chunks of >= 32 rows each (enough
+// CTAs to cover the SMs at small T * B; one thread sums one column of a chunk).
+constexpr long long kDbMaxChunks = 256;
 
 struct BwdLayout {
     size_t dG, dc, dhp, dbpart, wt, dbgroup, total;
@@ -153,7 +154,7 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     BwdLayout L;
     const size_t TB = (size_t)d->T * d->B, G4 = 4 * (size_t)d->H;
     const size_t BH = (size_t)d->B * d->H;
-    long long rows = 256;
+    long long rows = 32;
     if ((long long)TB > rows * kDbMaxChunks) rows = ((long long)TB + kDbMaxChunks - 1) / kDbMaxChunks;
     L.db_rows_per_chunk = (int)rows;
     L.db_chunks = (int)(((long long)TB + rows - 1) / rows);

@@ -111,17 +111,18 @@ struct BwdParams {
 };
 
 // Grid-wide step barrier: this CTA's arrival for `step` (release, after a
-// CTA barrier that orders every thread's stores before it), and the wait for
+// CTA barrier that orders every thread's stores before it), then `meanwhile`
+// by every thread (work that must not delay the arrival), then the wait for
 // all CTAs' arrivals for `step` (acquire).  Bounded; false on time-out.
+template <class Fn>
 __device__ __forceinline__ bool grid_step(unsigned int *ctr, unsigned int target, bool arrive,
                                           Ctrl *ctrl, volatile int *abort_flag, uint32_t site,
-                                          unsigned long long wait_ns) {
+                                          unsigned long long wait_ns, Fn meanwhile) {
     __syncthreads();
     __shared__ int ok_s;
-    if (threadIdx.x == 0) {
-        if (arrive) rec::red_release_add(ctr, 1u);
-        ok_s = rec::wait_counter(ctr, target, ctrl, abort_flag, site, wait_ns);
-    }
+    if (threadIdx.x == 0 && arrive) rec::red_release_add(ctr, 1u);
+    meanwhile();
+    if (threadIdx.x == 0) ok_s = rec::wait_counter(ctr, target, ctrl, abort_flag, site, wait_ns);
     __syncthreads();
     return ok_s != 0;
 }
@@ -241,6 +242,11 @@ __device__ __forceinline__ void group_sum(float (&acc)[MAXP][4], int ksplit) {
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 acc[i][g] += __shfl_xor_sync(0xffffffffu, acc[i][g], off);
+}
+
+// Pull one line of read-only input into this SM's L1 ahead of its use.
+__device__ __forceinline__ void prefetch_l1(const void *ptr) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
 }
 
 __device__ __forceinline__ float dot4(const float4 &a, const float4 &b, float acc) {
@@ -385,10 +391,24 @@ __global__ void __launch_bounds__(NTHR, 1) fwd_kernel(const FwdParams<T> p) {
                 }
             ep(m, 4 * (u0 + r * UN + ul), a);
         }
-        // h_t of every unit is the next step's operand: grid barrier
+        // h_t of every unit is the next step's operand: grid barrier; after
+        // this CTA's arrival, the next step's read-only epilogue inputs of its
+        // units (Gx, mask) go into L1 while it waits
         if (st + 1 < T_) {
             const bool arrive = (int)blockIdx.x != p.fault_skip_cta;
-            if (!grid_step(ctr, P * (unsigned)(st + 1), arrive, p.ctrl, &abort_s, 0xA01, p.wait_ns))
+            const long long tn = tau(st + 1);
+            auto prefetch = [&]() {
+                for (int e = threadIdx.x; e < B * UN; e += NTHR) {
+                    const int m = e % B, j = u0 + r * UN + e / B;
+                    if (j >= H) continue;
+                    const float *gx = p.Gx + (tn * B + m) * 4 * H + j;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) prefetch_l1(gx + g * H);
+                    if (p.mask) prefetch_l1(p.mask + tn * BH + (long long)m * H + j);
+                }
+            };
+            if (!grid_step(ctr, P * (unsigned)(st + 1), arrive, p.ctrl, &abort_s, 0xA01, p.wait_ns,
+                           prefetch))
                 break;
         }
     }
@@ -490,11 +510,29 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
                 }
             ep(m, u0 + r * UN + 4 * lq, a);
         }
-        // dG_t of every unit is the next step's operand: grid barrier
+        // dG_t of every unit is the next step's operand: grid barrier; after
+        // this CTA's arrival, the next step's read-only epilogue inputs of its
+        // units (gates, cells, c_{t-1}, dy, mask) go into L1 while it waits
         if (st > 0) {
             const bool arrive = (int)blockIdx.x != p.fault_skip_cta;
+            const long long tn = tau(st - 1);
+            auto prefetch = [&]() {
+                for (int e = threadIdx.x; e < B * QN; e += NTHR) {
+                    const int m = e % B, j = u0 + r * UN + 4 * (e / B);
+                    if (j >= H) continue;
+                    const long long o = (long long)m * H + j;
+                    const T *g4 = p.gates + (tn * B + m) * G4 + j;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) prefetch_l1(g4 + g * H);
+                    prefetch_l1(p.cells + tn * BH + o);
+                    if (st - 1 > 0) prefetch_l1(p.cells + tau(st - 2) * BH + o);
+                    else if (p.c0) prefetch_l1(p.c0 + o);
+                    if (p.dy) prefetch_l1(p.dy + tn * BH + o);
+                    if (p.mask) prefetch_l1(p.mask + tn * BH + o);
+                }
+            };
             if (!grid_step(ctr, P * (unsigned)(T_ - st), arrive, p.ctrl, &abort_s, 0xA02,
-                           p.wait_ns))
+                           p.wait_ns, prefetch))
                 break;
         }
     }

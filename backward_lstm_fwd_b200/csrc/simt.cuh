@@ -38,26 +38,51 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-    for (int k0 = 0; k0 < K; k0 += TK) {
+    // Software pipeline: the next K slab's operands are loaded from global
+    // memory into registers while the current slab is multiplied out of
+    // shared memory, so each slab's load latency overlaps the previous
+    // slab's FMAs instead of following them.
+    constexpr int EA = (TM * TK) / NTHR, EB = (TN * TK) / NTHR;
+    float ra[EA], rb[EB];
+    auto load = [&](int k0) {
 #pragma unroll
-        for (int e = 0; e < (TM * TK) / NTHR; ++e) {
+        for (int e = 0; e < EA; ++e) {
             const int idx = tid + e * NTHR;
             int mm, kk;
             if (A_KC) { kk = idx % TK; mm = idx / TK; }
             else      { mm = idx % TM; kk = idx / TM; }
             const int m = m0 + mm, k = k0 + kk;
-            As[kk][mm] = (m < M && k < K) ? A(m, k) : 0.f;
+            ra[e] = (m < M && k < K) ? A(m, k) : 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < (TN * TK) / NTHR; ++e) {
+        for (int e = 0; e < EB; ++e) {
             const int idx = tid + e * NTHR;
             int nn, kk;
             if (B_KC) { kk = idx % TK; nn = idx / TK; }
             else      { nn = idx % TN; kk = idx / TN; }
             const int n = n0 + nn, k = k0 + kk;
-            Bs[kk][nn] = (n < N && k < K) ? Bm(k, n) : 0.f;
+            rb[e] = (n < N && k < K) ? Bm(k, n) : 0.f;
         }
+    };
+    auto store = [&]() {
+#pragma unroll
+        for (int e = 0; e < EA; ++e) {
+            const int idx = tid + e * NTHR;
+            if (A_KC) As[idx % TK][idx / TK] = ra[e];
+            else      As[idx / TM][idx % TM] = ra[e];
+        }
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+            const int idx = tid + e * NTHR;
+            if (B_KC) Bs[idx % TK][idx / TK] = rb[e];
+            else      Bs[idx / TN][idx % TN] = rb[e];
+        }
+    };
+    if (K > 0) load(0);
+    for (int k0 = 0; k0 < K; k0 += TK) {
+        store();
         __syncthreads();
+        if (k0 + TK < K) load(k0 + TK);
 #pragma unroll
         for (int kk = 0; kk < TK; ++kk) {
             float a[4];
