@@ -1454,20 +1454,21 @@ int persist_fwd(const lstm_dims *d, const PstPlan &Q, const T *W, const float *G
     return launch_pst(pst::fwd_kernel<T>, prm, Q, s);
 }
 
-// a3 over all T steps in one launch (dinitH follows as one more product).
+// a3 over all T steps in one launch, and dinitH = W_h^T dG of the first step
+// as one more contraction at its end.
 template <class T>
 int persist_bwd(const lstm_dims *d, const PstPlan &Q, const T *W, const T *dy,
                 const T *dhT, const float *dcT, const T *gates, const float *cells,
                 const float *c0, const T *mask, bool reverse, bool ijfo, T *dG,
-                float *const dcbuf[2], float *const dhpbuf[2], float *dc0, Ctrl *ctrl,
-                cudaStream_t s) {
+                float *const dcbuf[2], float *const dhpbuf[2], float *dc0, float *dh0,
+                Ctrl *ctrl, cudaStream_t s) {
     pst::BwdParams<T> prm;
     memset(&prm, 0, sizeof(prm));
     prm.W = W; prm.dy = dy; prm.dhT = dhT; prm.gates = gates; prm.mask = mask;
     prm.dcT = dcT; prm.cells = cells; prm.c0 = c0; prm.dG = dG;
     prm.dcbuf[0] = dcbuf[0]; prm.dcbuf[1] = dcbuf[1];
     prm.dhpbuf[0] = dhpbuf[0]; prm.dhpbuf[1] = dhpbuf[1];
-    prm.dc0 = dc0; prm.ctrl = ctrl;
+    prm.dc0 = dc0; prm.dh0 = dh0; prm.ctrl = ctrl;
     prm.T = d->T; prm.B = d->B; prm.H = d->H; prm.I = d->I;
     prm.reverse = reverse; prm.fb = ijfo ? 2 : 1;
     prm.s = Q.s;
@@ -1690,7 +1691,8 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         PstPlan Q;
         if (plan_persist<T>(d, true, Q)) {
             const int rc = persist_bwd<T>(d, Q, W, dy, dhT, dcT, gates, cells, c0, mask,
-                                          reverse, ijfo, dG, dcbuf, dhpbuf, dc0, (Ctrl *)ws, s);
+                                          reverse, ijfo, dG, dcbuf, dhpbuf, dc0, dh0,
+                                          (Ctrl *)ws, s);
             if (rc != LSTM_ERR_NOT_CORESIDENT && rc != LSTM_OK) return rc;
             persisted = rc == LSTM_OK;
         }
@@ -1723,10 +1725,11 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                                            simt::RowMajor<T>{W, K}, ep, s)));
     }
     // dinitH = W_h^T dG of the first step (delta h_prev before it, step 5), plus
-    // what padding at that step passes on
-    LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG + tau(0) * B * G4, G4},
-                                       simt::RowMajor<T>{W, K},
-                                       simt::EpStore{dh0, H, mask ? dhpbuf[0] : nullptr}, s)));
+    // what padding at that step passes on (inside the persistent kernel when it ran)
+    if (!persisted)
+        LSTM_TRY((simt::gemm<true, false>(B, H, G4, simt::RowMajor<T>{dG + tau(0) * B * G4, G4},
+                                           simt::RowMajor<T>{W, K},
+                                           simt::EpStore{dh0, H, mask ? dhpbuf[0] : nullptr}, s)));
     }
     const bool tc = tc_gemm_ok(d);
     if (tc) {

@@ -103,6 +103,7 @@ struct BwdParams {
     float *dcbuf[2];       // delta c ping-pong [B][H]
     float *dc0;            // [B][H]: delta c after the first step (dinitC)
     float *dhpbuf[2];      // delta h passed on by padding, ping-pong [B][H]
+    float *dh0;            // [B][H]: dinitH = W_h^T dG of the first step (+ padding's share)
     Ctrl *ctrl;
     int T, B, H, I, reverse, fb;
     Split s;
@@ -446,9 +447,11 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
     auto tau = [&](int st) { return p.reverse ? T_ - 1 - (long long)st : (long long)st; };
     const long long BH = (long long)B * H;
     uint32_t rph = 0;
-    for (int st = T_ - 1; st >= 0; --st) {
+    // steps T-1 .. 0, then st = -1: dinitH = W_h^T dG of step 0, the same
+    // contraction and exchange with only a store after it
+    for (int st = T_ - 1; st >= -1; --st) {
         const bool last = st == T_ - 1;  // no dG_{t+1}: delta h comes from dhT
-        const long long t = tau(st);
+        const long long t = st >= 0 ? tau(st) : 0;
         if (!last) {
             // delta h = dG_{t_next} W_h, this CTA's K slice, for the cluster's units
             float acc[MAXP][4];
@@ -480,6 +483,26 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
             if (!exchange(stage, recv, rbar, rph, KS, r, part * 4, p.ctrl, &abort_s, 0xA04,
                           p.wait_ns))
                 break;
+        }
+        if (st < 0) {
+            for (int e = threadIdx.x; e < B * QN; e += NTHR) {
+                const int m = e % B, lq = e / B;
+                const float4 v0 = *reinterpret_cast<const float4 *>(recv + (m * QN + lq) * 4);
+                float a[4] = {v0.x, v0.y, v0.z, v0.w};
+                for (int sl = 1; sl < KS; ++sl) {
+                    const float4 v = *reinterpret_cast<const float4 *>(recv + sl * part +
+                                                                       (m * QN + lq) * 4);
+                    a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int j = u0 + r * UN + 4 * lq + c;
+                    if (j >= H) continue;
+                    const long long o = (long long)m * H + j;
+                    p.dh0[o] = a[c] + (p.mask ? p.dhpbuf[0][o] : 0.f);
+                }
+            }
+            break;
         }
         simt::EpBwdStep<T> ep;
         ep.dy = p.dy ? p.dy + t * BH : nullptr;
@@ -513,11 +536,11 @@ __global__ void __launch_bounds__(NTHR, 1) bwd_kernel(const BwdParams<T> p) {
         // dG_t of every unit is the next step's operand: grid barrier; after
         // this CTA's arrival, the next step's read-only epilogue inputs of its
         // units (gates, cells, c_{t-1}, dy, mask) go into L1 while it waits
-        if (st > 0) {
+        {
             const bool arrive = (int)blockIdx.x != p.fault_skip_cta;
-            const long long tn = tau(st - 1);
+            const long long tn = st > 0 ? tau(st - 1) : 0;
             auto prefetch = [&]() {
-                for (int e = threadIdx.x; e < B * QN; e += NTHR) {
+                for (int e = threadIdx.x; st > 0 && e < B * QN; e += NTHR) {
                     const int m = e % B, j = u0 + r * UN + 4 * (e / B);
                     if (j >= H) continue;
                     const long long o = (long long)m * H + j;

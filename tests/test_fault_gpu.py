@@ -56,7 +56,8 @@ def test_missing_arrival_times_out_and_recovers(H, T, B, streams, cuda_device, m
 def test_persistent_cuda_core_time_out_and_recover(dt, H, cuda_device):
     """The persistent CUDA-core recurrences (fp32, and 16-bit shapes off the
     tensor-core grids) meet at a grid-wide step counter: with CTA 0 never
-    arriving, both give up, report LSTM_ERR_TIMEOUT, and the next call runs."""
+    arriving, both give up, report LSTM_ERR_TIMEOUT, and the next call runs
+    (fp32 at H = 256 with the K axis split over clusters, bf16 at H = 45 without)."""
     lbuild.build()
     T, B, I = 6, 32, 37
     w = synth.custom(T, B, I, H, dt, seed=13)
@@ -75,6 +76,11 @@ def test_persistent_cuda_core_time_out_and_recover(dt, H, cuda_device):
                    inp["c0"], st.y, st.gates, st.cells, gr.dx, gr.dW, gr.db, gr.dh0, gr.dc0, wsb)
         assert L.lstm_status(wsb) == L.LSTM_ERR_TIMEOUT
         assert L.test_last_paths() == (5, 5)
+        if dt == "fp32":
+            # K split over clusters in both directions: the time-out also
+            # exercises the exit path in which every CTA of a cluster waits for
+            # its peers before leaving
+            assert min(L.test_last_persist_split()) > 1
     finally:
         L.test_set_wait_fault(-1, 0)
     out = run_gpu(synth.make_inputs(w), cuda_device)
