@@ -1732,6 +1732,37 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                                            simt::EpStore{dh0, H, mask ? dhpbuf[0] : nullptr}, s)));
     }
     const bool tc = tc_gemm_ok(d);
+    // a4, a5 and a6 only read the finished dG: dW (with dx on the tensor cores)
+    // on the caller's stream, db and the CUDA-core dx beside it on the two
+    // auxiliary streams when they exist, joined back with events
+    AuxStreams *A = aux_streams();
+    std::unique_lock<std::mutex> lk;
+    if (A) lk = std::unique_lock<std::mutex>(A->mu);
+    cudaStream_t s_db = A ? A->rec : s, s_dx = A ? A->gemm : s;
+    if (A) {
+        LSTM_TRY(cudaEventRecord(A->ev[0], s));
+        LSTM_TRY(cudaStreamWaitEvent(s_db, A->ev[0], 0));
+        LSTM_TRY(cudaStreamWaitEvent(s_dx, A->ev[0], 0));
+    }
+    // a5: db = column sums of dG (step 4)
+    {
+        prof::Phase ph(LSTM_PHASE_DB, s_db);
+        float *part = (float *)(ws + L.dbpart);
+        dim3 g1((G4 + 255) / 256, L.db_chunks);
+        simt::colsum_partial<T><<<g1, 256, 0, s_db>>>(dG, (int)TB, G4, L.db_rows_per_chunk, part);
+        note_launch();
+        LSTM_TRY(cudaGetLastError());
+        simt::colsum_final<<<(G4 + 255) / 256, 256, 0, s_db>>>(part, L.db_chunks, G4, db);
+        note_launch();
+        LSTM_TRY(cudaGetLastError());
+    }
+    // a6: dx = dG W_x (x-part of delta z, step 5)
+    if (I > 0 && !tc) {
+        prof::Phase ph(LSTM_PHASE_DX, s_dx);
+        LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
+                                           simt::RowMajor<T>{W + H, K},
+                                           simt::EpStore{dx, I}, s_dx)));
+    }
     if (tc) {
         // a4 + a6 together on the tensor cores (one launch, timed as dW)
         prof::Phase ph(LSTM_PHASE_DW, s);
@@ -1745,24 +1776,12 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
                                             simt::Zrows<T>{x, y, h0, B, I, H, reverse, (long long)(T_ - 1) * B},
                                             simt::EpStore{dW, K}, s)));
     }
-    // a5: db = column sums of dG (step 4)
-    {
-        prof::Phase ph(LSTM_PHASE_DB, s);
-        float *part = (float *)(ws + L.dbpart);
-        dim3 g1((G4 + 255) / 256, L.db_chunks);
-        simt::colsum_partial<T><<<g1, 256, 0, s>>>(dG, (int)TB, G4, L.db_rows_per_chunk, part);
-        note_launch();
-        LSTM_TRY(cudaGetLastError());
-        simt::colsum_final<<<(G4 + 255) / 256, 256, 0, s>>>(part, L.db_chunks, G4, db);
-        note_launch();
-        LSTM_TRY(cudaGetLastError());
+    if (A) {
+        LSTM_TRY(cudaEventRecord(A->ev[1], s_db));
+        LSTM_TRY(cudaEventRecord(A->ev[2], s_dx));
+        LSTM_TRY(cudaStreamWaitEvent(s, A->ev[1], 0));
+        LSTM_TRY(cudaStreamWaitEvent(s, A->ev[2], 0));
     }
-    // a6: dx = dG W_x (x-part of delta z, step 5)
-    prof::Phase ph(LSTM_PHASE_DX, s);
-    if (I > 0 && !tc)
-        LSTM_TRY((simt::gemm<true, false>((int)TB, I, G4, simt::RowMajor<T>{dG, G4},
-                                           simt::RowMajor<T>{W + H, K},
-                                           simt::EpStore{dx, I}, s)));
     return LSTM_OK;
 }
 
