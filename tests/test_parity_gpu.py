@@ -189,7 +189,8 @@ def test_two_stream_backward_equals_one_stream(shape, cuda_device, monkeypatch):
 
 @pytest.mark.parametrize("ks", [1, 2, 4, 8])
 @pytest.mark.parametrize("shape", [(12, 32, 256, 256, "fp32"), (6, 130, 64, 128, "fp32"),
-                                   (7, 5, 37, 45, "bf16"), (5, 17, 40, 100, "fp16")])
+                                   (7, 5, 37, 45, "bf16"), (5, 17, 40, 100, "fp16"),
+                                   (1, 32, 64, 256, "fp32")])
 def test_persistent_k_split_cluster_sizes(shape, ks, cuda_device, monkeypatch):
     """Each cluster size of the persistent CUDA-core recurrences' K split (KS
     CTAs per cluster, each contracting one K slice, the partial sums sent to
