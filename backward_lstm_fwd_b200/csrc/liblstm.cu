@@ -145,9 +145,23 @@ FwdLayout fwd_layout(const lstm_dims *d) {
 // CTAs to cover the SMs at small T * B; one thread sums one column of a chunk).
 constexpr long long kDbMaxChunks = 256;
 
+// K splits of the CUDA-core dW GEMM (K = T*B rows): enough 64 x 64 output tiles
+// times splits for about two CTAs per SM of a 148-SM part (a fixed target, so
+// that the workspace size does not depend on the device), at most 8 splits of
+// at least 256 rows each; 1 when the tiles alone fill the part.
+constexpr long long kDwSplitTarget = 296;
+int dw_splits(const lstm_dims *d) {
+    const long long tiles = (4LL * d->H + 63) / 64 * ((long long)(d->H + d->I) + 63) / 64;
+    const long long rows = (long long)d->T * d->B;
+    if (tiles <= 0) return 1;
+    long long S = std::min<long long>(8, (kDwSplitTarget + tiles - 1) / tiles);
+    S = std::min<long long>(S, rows / 256);
+    return (int)std::max<long long>(1, S);
+}
+
 struct BwdLayout {
-    size_t dG, dc, dhp, dbpart, wt, dbgroup, total;
-    int db_chunks, db_rows_per_chunk;
+    size_t dG, dc, dhp, dbpart, dwsplit, wt, dbgroup, total;
+    int db_chunks, db_rows_per_chunk, dw_splits;
 };
 constexpr int kMaxGroups = 48;
 BwdLayout bwd_layout(const lstm_dims *d) {
@@ -163,7 +177,13 @@ BwdLayout bwd_layout(const lstm_dims *d) {
     // delta h that padding passes to h_{t-1} (variable-length calls), ping-pong
     L.dhp = align_up(L.dc + 2 * BH * sizeof(float), 256);
     L.dbpart = align_up(L.dhp + 2 * BH * sizeof(float), 256);
-    L.wt = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
+    // partial products of the split-K CUDA-core dW GEMM
+    L.dw_splits = dw_splits(d);
+    L.dwsplit = align_up(L.dbpart + (size_t)L.db_chunks * G4 * sizeof(float), 256);
+    const size_t dwpart = L.dw_splits > 1
+                              ? (size_t)L.dw_splits * G4 * ((size_t)d->H + d->I) * sizeof(float)
+                              : 0;
+    L.wt = align_up(L.dwsplit + dwpart, 256);
     L.dbgroup = L.wt;
     L.total = L.wt;
     if (d->dtype != LSTM_F32) {
@@ -1769,6 +1789,18 @@ int bwd_simt(const lstm_dims *d, const T *dy, const T *dhT, const float *dcT, co
         LSTM_TRY(tc_dw_dx(d, (const E *)dG, (const E *)x, (const E *)W,
                           (const E *)h0, (const E *)y, dW, dx, (Ctrl *)ws, s, 0, d->T,
                           false, 0, reverse));
+    } else if (L.dw_splits > 1) {
+        // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4), the rows split
+        // into dw_splits slabs whose partial products are summed in order
+        prof::Phase ph(LSTM_PHASE_DW, s);
+        float *part = (float *)(ws + L.dwsplit);
+        const long long MN = G4 * K;
+        LSTM_TRY((simt::gemm<false, false>(G4, K, (int)TB, simt::ColMajor<T>{dG, G4},
+                                            simt::Zrows<T>{x, y, h0, B, I, H, reverse, (long long)(T_ - 1) * B},
+                                            simt::EpPart{part, (int)K, MN}, s, L.dw_splits)));
+        simt::sum_splits<<<(unsigned)((MN + 255) / 256), 256, 0, s>>>(part, L.dw_splits, MN, dW);
+        note_launch();
+        LSTM_TRY(cudaGetLastError());
     } else {
         // a4: dW = dG^T [h_prev | x] over all T*B rows (step 4)
         prof::Phase ph(LSTM_PHASE_DW, s);

@@ -25,9 +25,10 @@ constexpr int TM = 64, TN = 64, TK = 16, NTHR = 256;
 // C[m, n] = sum_k A(m, k) B(k, n) for a 64x64 tile, handed to ep(m, n0, acc[4])
 // for the four consecutive columns n0..n0+3 a thread owns.  A_KC / B_KC say
 // whether the operand is contiguous along k (picks the coalesced load order).
+// Split K (gridDim.z > 1): block z sums k in [z * Kc, min(K, (z + 1) * Kc)).
 template <bool A_KC, bool B_KC, class AL, class BL, class EP>
 __global__ void __launch_bounds__(NTHR)
-gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
+gemm_kernel(int M, int N, int K, int Kc, AL A, BL Bm, EP ep) {
     __shared__ float As[TK][TM + 4];
     __shared__ __align__(16) float Bs[TK][TN + 4];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
@@ -43,6 +44,7 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
     // shared memory, so each slab's load latency overlaps the previous
     // slab's FMAs instead of following them.
     constexpr int EA = (TM * TK) / NTHR, EB = (TN * TK) / NTHR;
+    const int kbeg = (int)blockIdx.z * Kc, kend = min(K, kbeg + Kc);
     float ra[EA], rb[EB];
     auto load = [&](int k0) {
 #pragma unroll
@@ -52,7 +54,7 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
             if (A_KC) { kk = idx % TK; mm = idx / TK; }
             else      { mm = idx % TM; kk = idx / TM; }
             const int m = m0 + mm, k = k0 + kk;
-            ra[e] = (m < M && k < K) ? A(m, k) : 0.f;
+            ra[e] = (m < M && k < kend) ? A(m, k) : 0.f;
         }
 #pragma unroll
         for (int e = 0; e < EB; ++e) {
@@ -61,7 +63,7 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
             if (B_KC) { kk = idx % TK; nn = idx / TK; }
             else      { nn = idx % TN; kk = idx / TN; }
             const int n = n0 + nn, k = k0 + kk;
-            rb[e] = (n < N && k < K) ? Bm(k, n) : 0.f;
+            rb[e] = (n < N && k < kend) ? Bm(k, n) : 0.f;
         }
     };
     auto store = [&]() {
@@ -78,11 +80,11 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
             else      Bs[idx / TN][idx % TN] = rb[e];
         }
     };
-    if (K > 0) load(0);
-    for (int k0 = 0; k0 < K; k0 += TK) {
+    if (kbeg < kend) load(kbeg);
+    for (int k0 = kbeg; k0 < kend; k0 += TK) {
         store();
         __syncthreads();
-        if (k0 + TK < K) load(k0 + TK);
+        if (k0 + TK < kend) load(k0 + TK);
 #pragma unroll
         for (int kk = 0; kk < TK; ++kk) {
             float a[4];
@@ -104,12 +106,16 @@ gemm_kernel(int M, int N, int K, AL A, BL Bm, EP ep) {
     }
 }
 
+// splits > 1: K split into that many slabs of whole TK blocks, one grid layer
+// each (the epilogue sees blockIdx.z; see EpPart).
 template <bool A_KC, bool B_KC, class AL, class BL, class EP>
-inline cudaError_t gemm(int M, int N, int K, AL A, BL Bm, EP ep, cudaStream_t s) {
+inline cudaError_t gemm(int M, int N, int K, AL A, BL Bm, EP ep, cudaStream_t s,
+                        int splits = 1) {
     if (M <= 0 || N <= 0) return cudaSuccess;
-    dim3 grid((M + TM - 1) / TM, (N + TN - 1) / TN);
-    if (grid.y > 65535u) return cudaErrorInvalidConfiguration;
-    gemm_kernel<A_KC, B_KC><<<grid, NTHR, 0, s>>>(M, N, K, A, Bm, ep);
+    const int Kc = splits > 1 ? ((K + splits - 1) / splits + TK - 1) / TK * TK : K;
+    dim3 grid((M + TM - 1) / TM, (N + TN - 1) / TN, splits > 1 ? splits : 1);
+    if (grid.y > 65535u || grid.z > 64u) return cudaErrorInvalidConfiguration;
+    gemm_kernel<A_KC, B_KC><<<grid, NTHR, 0, s>>>(M, N, K, Kc, A, Bm, ep);
     note_launch();
     return cudaGetLastError();
 }
@@ -302,6 +308,27 @@ struct EpStore {
                     acc[c] + (add ? add[(long long)m * N + n0 + c] : 0.f);
     }
 };
+
+// Partial product of K split z (blockIdx.z) of a split-K GEMM:
+// part[z][m][n], row stride N, MN floats per split.
+struct EpPart {
+    float *part; int N; long long MN;
+    __device__ void operator()(int m, int n0, const float *acc) const {
+        float *o = part + (long long)blockIdx.z * MN + (long long)m * N;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            if (n0 + c < N) o[n0 + c] = acc[c];
+    }
+};
+
+// out[i] = sum over the S splits of part[z][i], in split order.
+__global__ void sum_splits(const float *part, int S, long long MN, float *out) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= MN) return;
+    float v = 0.f;
+    for (int z = 0; z < S; ++z) v += part[(long long)z * MN + i];
+    out[i] = v;
+}
 
 // ----------------------------------------------------------- db (step 4)
 // Column sums of dG [R][N] in two deterministic passes: per-chunk partials,
