@@ -375,3 +375,20 @@ def test_environment_switches_are_the_documented_ones():
     listed = set(re.findall(r"^ \*   (LSTM_[A-Z0-9_]+)=", hdr, flags=re.M))
     listed |= {"CUDA_INJECTION64_PATH", "NV_COMPUTE_PROFILER_PERFWORKS_DIR"}
     assert read == listed, (sorted(read), sorted(listed))
+
+
+def test_backward_workspace_holds_the_split_k_partials(lib):
+    """The CUDA-core dW splits its T*B rows into slabs when its 64 x 64 output
+    tiles are too few to fill the device (the fp32 workload T=64, B=32, I=H=256:
+    128 tiles, 3 slabs); the slabs' fp32 partial products live in the backward
+    workspace, whose size does not depend on the device.  At the bench size
+    the tiles fill the device and no such region is reserved."""
+    small = L.dims(64, 32, 256, 256, L.LSTM_F32)
+    TB, G4, K = 64 * 32, 4 * 256, 256 + 256
+    need = 256 + TB * G4 * 4 + 3 * G4 * K * 4
+    assert L.bwd_workspace_size(small) >= need
+    # and not much more: the other regions (db chunks, delta c / h buffers) are small
+    assert L.bwd_workspace_size(small) < need + 2 * G4 * K * 4
+    big = L.dims(256, 128, 1024, 1024, L.LSTM_BF16)
+    TB, G4, K = 256 * 128, 4096, 2048
+    assert L.bwd_workspace_size(big) < 256 + TB * G4 * 2 + G4 * K * 4
