@@ -1187,11 +1187,20 @@ int tc_bwd_tmem_launch(const lstm_dims *d, const Rec2Plan &P, const E *dy, const
                           dbgroup, dh0, dc0, dc_carry, dhp_carry, ctrl, i0, i1, s, bar_base);
 }
 
-// W_h^T of a 16-bit W (bf16 or fp16: the kernel only moves 16-bit values)
+// W_h^T of a 16-bit W (bf16 or fp16: the kernels only move 16-bit values):
+// 64 x 64 tiles with 16-byte accesses when the rows allow, else 32 x 32 tiles
+// of single elements.
 cudaError_t launch_transpose_wh(const lstm_dims *d, const void *W_, void *WT_, cudaStream_t s) {
+    const long long H = d->H, I = d->I, G4 = 4 * H;
+    if (H % 8 == 0 && I % 8 == 0 && aligned16(W_) && aligned16(WT_)) {
+        dim3 grid((unsigned)((H + 63) / 64), (unsigned)((G4 + 63) / 64));
+        rec::transpose_wh_v8<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(W_),
+                                                   static_cast<uint16_t *>(WT_), (int)H, (int)I);
+        note_launch();
+        return cudaGetLastError();
+    }
     const bf16 *W = static_cast<const bf16 *>(W_);
     bf16 *WT = static_cast<bf16 *>(WT_);
-    const long long H = d->H, G4 = 4 * H;
     dim3 grid((unsigned)((H + 31) / 32), (unsigned)((G4 + 31) / 32));
     rec::transpose_wh<<<grid, dim3(32, 8), 0, s>>>(W, WT, (int)H, (int)d->I);
     note_launch();

@@ -743,5 +743,37 @@ __global__ void transpose_wh(const __nv_bfloat16 *__restrict__ W, __nv_bfloat16 
     }
 }
 
+// The same transpose with 64 x 64 tiles and 16-byte accesses (8 elements):
+// W [4H][H + I] -> WT [H][4H].  Needs H and I multiples of 8 and 16-byte
+// aligned W and WT; the elements are moved as raw 16-bit values.  Loads: a
+// quarter warp reads one 128-byte row segment of W; stores: a warp writes
+// 16 bytes (8 consecutive 4H-indices) of 32 consecutive WT rows, reading 32
+// consecutive elements of one tile row per element of its vector.
+__global__ void __launch_bounds__(256) transpose_wh_v8(const uint16_t *__restrict__ W,
+                                                     uint16_t *__restrict__ WT, int H, int I) {
+    __shared__ __align__(16) uint16_t tile[64][72];  // 144-byte rows: 16-byte aligned
+    const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;  // rows of W (4H), columns (H)
+    const int G4 = 4 * H;
+    const long long ld = (long long)H + I;
+    for (int v = threadIdx.x; v < 64 * 8; v += 256) {
+        const int rr = v / 8, cv = (v % 8) * 8;
+        const int r = r0 + rr, c = c0 + cv;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (r < G4 && c < H) val = *reinterpret_cast<const uint4 *>(W + (long long)r * ld + c);
+        *reinterpret_cast<uint4 *>(&tile[rr][cv]) = val;
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < 64 * 8; v += 256) {
+        const int cc = v % 64, rv = (v / 64) * 8;
+        const int c = c0 + cc, r = r0 + rv;
+        if (c >= H || r >= G4) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            w[i] = (uint32_t)tile[rv + 2 * i][cc] | ((uint32_t)tile[rv + 2 * i + 1][cc] << 16);
+        *reinterpret_cast<uint4 *>(WT + (long long)c * G4 + r) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 }  // namespace rec
 }  // namespace lstm
