@@ -6,7 +6,7 @@
 //
 // One launch walks a table of up to four problems (each with up to two K
 // segments drawn from different tensor maps), one 128 x 256 output tile per
-// step of a static persistent schedule.  Warp roles:
+// step of a static persistent schedule (sched_tile).  Warp roles:
 //   warp 0      one thread issues TMA loads into a 4-stage shared-memory ring;
 //   warp 1      allocates TMEM and one thread issues tcgen05.mma (M=128,
 //               N=256, K=16 per instruction) into one of two accumulators;
@@ -70,6 +70,17 @@ __device__ __forceinline__ int locate(const Params &p, int tile, int &mt, int &n
     return pi;
 }
 
+// The tile of this CTA's k-th step of the static schedule: rounds of
+// gridDim.x consecutive tiles, the first in CTA order and every later one in
+// reverse CTA order.  The queue holds its largest tiles first, so the CTAs
+// that drew the larger first-round tiles draw the last, partial round's
+// tiles last, if at all (the last dW / dx chunk of the bench backward: 138
+// instead of 156 K blocks on the busiest CTA against 119 on average).  Every
+// round but the last is full, so a CTA's first tile past the queue ends it.
+__device__ __forceinline__ int sched_tile(int k) {
+    return k * (int)gridDim.x + (k == 0 ? (int)blockIdx.x : (int)gridDim.x - 1 - (int)blockIdx.x);
+}
+
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int k16) {
     // K-major: rows of 128 B (64 bf16 of K), 8-row groups 1024 B apart; a
     //          K=16 step moves 32 B inside the 128-byte swizzle row.
@@ -123,7 +134,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
             bool issued[STAGES];
             for (int s = 0; s < STAGES; ++s) issued[s] = false, issued_parity[s] = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+            for (int k = 0, tile; ok && (tile = sched_tile(k)) < p.total_tiles; ++k) {
                 int mt, nt;
                 const Problem &P = p.prob[locate(p, tile, mt, nt)];
                 const int m0 = P.a_mn0 + mt * BM, n0 = P.b_mn0 + nt * BN;
@@ -176,7 +187,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
             uint32_t stage = 0, phase = 0, acc = 0, aphase = 0;
             bool ok = true;
             const uint64_t a_lo0 = tc::smem_u32(sA) >> 4, b_lo0 = tc::smem_u32(sB) >> 4;
-            for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+            for (int k = 0, tile; ok && (tile = sched_tile(k)) < p.total_tiles; ++k) {
                 int mt, nt;
                 const Problem &P = p.prob[locate(p, tile, mt, nt)];
                 if (!tc::mbar_wait(&tempty[acc], aphase ^ 1, p.ctrl, abort_flag, 0x102)) break;
@@ -219,7 +230,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
         // ---------------------------------------------------------- epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may read
         uint32_t acc = 0, aphase = 0;
-        for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+        for (int k = 0, tile; (tile = sched_tile(k)) < p.total_tiles; ++k) {
             int mt, nt;
             const Problem &P = p.prob[locate(p, tile, mt, nt)];
             const bool w = tc::mbar_wait(&tfull[acc], aphase, p.ctrl, abort_flag, 0x104);
