@@ -1382,7 +1382,8 @@ bool pst_coresident(Kern kern, int KS, int grid, size_t smem) {
 
 // Work split of the persistent recurrences (pst::Split): for each cluster
 // size KS in 8, 4, 2, 1 the fewest units per CTA (quads in the backward, the
-// grain of its epilogue) that keep the grid within one CTA per SM, the
+// grain of its epilogue) that keep the grid within one CTA per SM and
+// co-resident (more units per CTA, fewer clusters, while it is not), the
 // staging chunk (at most 16384 floats over all B rows, halved until the
 // shared memory fits) and the lanes per dot product (those the CTA would
 // otherwise leave idle); of the splits that fit and are co-resident, the one
@@ -1416,23 +1417,32 @@ bool plan_persist(const lstm_dims *d, bool backward, PstPlan &Q) {
         if (KS > 1 && (long long)s.KSL * (KS - 1) >= K) continue;  // a rank without columns
         s.UN = q;
         while ((long long)(H + KS * s.UN - 1) / (KS * s.UN) * KS > nsm) s.UN += q;
-        const int UC = KS * s.UN, P = (H + UC - 1) / UC * KS;
-        const long long items = (long long)B * (backward ? UC / 4 : UC);
-        if (items > (long long)pst::MAXP * pst::NTHR) continue;
-        s.KSPLIT = 1;
-        while (s.KSPLIT < 32 && items * s.KSPLIT * 2 <= pst::NTHR) s.KSPLIT *= 2;
-        const int pad = 4 * std::min(s.KSPLIT, 8);
-        s.KC = std::min(std::max(32, 16384 / B / 32 * 32), (s.KSL + 31) / 32 * 32);
-        s.KCP = s.KC + pad;
-        while (s.KC > 32 && pst::layout(backward, B, s).bytes > kMaxSmem) {
-            s.KC = std::max(32, s.KC / 2 / 32 * 32);
+        // more units per CTA (fewer clusters) until the grid is co-resident
+        int UC = 0, P = 0;
+        long long items = 0;
+        size_t smem = 0;
+        bool fits = false;
+        for (; !fits; s.UN += q) {
+            UC = KS * s.UN;
+            P = (H + UC - 1) / UC * KS;
+            items = (long long)B * (backward ? UC / 4 : UC);
+            if (items > (long long)pst::MAXP * pst::NTHR) break;
+            s.KSPLIT = 1;
+            while (s.KSPLIT < 32 && items * s.KSPLIT * 2 <= pst::NTHR) s.KSPLIT *= 2;
+            const int pad = 4 * std::min(s.KSPLIT, 8);
+            s.KC = std::min(std::max(32, 16384 / B / 32 * 32), (s.KSL + 31) / 32 * 32);
             s.KCP = s.KC + pad;
+            while (s.KC > 32 && pst::layout(backward, B, s).bytes > kMaxSmem) {
+                s.KC = std::max(32, s.KC / 2 / 32 * 32);
+                s.KCP = s.KC + pad;
+            }
+            smem = pst::layout(backward, B, s).bytes;
+            if (smem > kMaxSmem) break;
+            fits = backward ? pst_coresident(pst::bwd_kernel<T>, KS, P, smem)
+                            : pst_coresident(pst::fwd_kernel<T>, KS, P, smem);
+            if (fits) break;
         }
-        const size_t smem = pst::layout(backward, B, s).bytes;
-        if (smem > kMaxSmem) continue;
-        const bool cores = backward ? pst_coresident(pst::bwd_kernel<T>, KS, P, smem)
-                                    : pst_coresident(pst::fwd_kernel<T>, KS, P, smem);
-        if (!cores) continue;
+        if (!fits) continue;
         const int nslots = pst::NTHR / s.KSPLIT;
         const double cost =
             (double)B * s.KSL * sizeof(T) / 16.0 +
