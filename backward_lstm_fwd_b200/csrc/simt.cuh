@@ -29,7 +29,7 @@ constexpr int TM = 64, TN = 64, TK = 16, NTHR = 256;
 template <bool A_KC, bool B_KC, class AL, class BL, class EP>
 __global__ void __launch_bounds__(NTHR)
 gemm_kernel(int M, int N, int K, int Kc, AL A, BL Bm, EP ep) {
-    __shared__ float As[TK][TM + 4];
+    __shared__ __align__(16) float As[TK][TM + 4];
     __shared__ __align__(16) float Bs[TK][TN + 4];
     const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
     const int m0 = blockIdx.x * TM, n0 = blockIdx.y * TN;
@@ -87,9 +87,10 @@ gemm_kernel(int M, int N, int K, int Kc, AL A, BL Bm, EP ep) {
         if (k0 + TK < kend) load(k0 + TK);
 #pragma unroll
         for (int kk = 0; kk < TK; ++kk) {
-            float a[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+            // this thread's rows 4 ty .. 4 ty + 3 and columns 4 tx .. 4 tx + 3:
+            // one 16-byte shared load for each operand per k
+            const float4 av = *reinterpret_cast<const float4 *>(&As[kk][4 * ty]);
+            const float a[4] = {av.x, av.y, av.z, av.w};
             const float4 bv = *reinterpret_cast<const float4 *>(&Bs[kk][4 * tx]);
             const float b[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
@@ -101,7 +102,7 @@ gemm_kernel(int M, int N, int K, int Kc, AL A, BL Bm, EP ep) {
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int m = m0 + ty + 16 * i;
+        const int m = m0 + 4 * ty + i;
         if (m < M) ep(m, n0 + 4 * tx, acc[i]);
     }
 }
